@@ -1,0 +1,493 @@
+"""CPU oracle of the block-diffusion decode step -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
+``bench.py`` may import this module.  The product path (the C-ABI library and
+its Python binding) never calls it and shares no code with it.
+
+Everything is plain numpy in float64.  Matrix products use numpy's matmul as
+a library primitive; nothing is blocked, fused or reordered beyond the
+definitions below.  Where the GPU stores an activation in bf16, the oracle
+rounds the exact fp64 value to bf16 at the same point (``bf16_round``), so
+that "bf16 model" means the same thing on both sides; all other arithmetic
+(norm factors, RoPE angles, softmax, accumulations) stays in fp64.
+
+Sources (page titles as they appear on the pages):
+  [FDV]  Fast-dVLM technical overview (ocdem.com news article)
+  [FDVW] Fast-dVLM walkthrough (itsolotime.com archive 34466)
+  [LOWN] Look Only When Needed: Certificate-Guided Visual Routing for
+         Efficient Diffusion VLMs
+  [DAVET] DAVET PaperDaily article (generic dVLM commit rule only)
+
+Readings taken where the pages are silent or garbled (each is listed with
+its reason in the repository's design notes):
+  shift=1   masked position j is scored by the hidden row of position j-1
+            (row -1 = the last committed row); shift=0 is kept as an option.
+  ar_seed   the block's first token is the AR prediction, committed outright.
+  N2C       noisy tokens see the clean tokens of PRECEDING blocks only (the
+            prose); the printed lower-triangular N2C matrix is not used.
+  commit    p1 >= threshold; if none passes, the masked position with the
+            highest p1 (lowest position on ties) is committed.
+  argmax    lowest vocabulary id among equal maxima.
+  norms     RMSNorm gain 1, eps 1e-6, no biases; RoPE rotate-half, base 1e4.
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+against brute force, closed forms, library routines or the pages' printed
+mask example.  Parity unpinned: none.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+# ----------------------------------------------------------------------------
+# Storage rounding
+# ----------------------------------------------------------------------------
+def bf16_round(x) -> np.ndarray:
+    """Round real values to the nearest bfloat16 (8 significant bits, ties to
+    even), returned as float64.  Direct from the exact value: no detour
+    through fp32 (which could double-round)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                    # x = m * 2**e, 0.5 <= |m| < 1
+    r = np.round(m * 256.0)               # numpy rounds half to even
+    return np.ldexp(r, e - 8)
+
+
+# ----------------------------------------------------------------------------
+# Decoder-layer pieces (plain definitions)
+# ----------------------------------------------------------------------------
+def rms_factor(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """1 / sqrt(mean(x^2) + eps) per row (RMSNorm with unit gain)."""
+    x = np.asarray(x, dtype=np.float64)
+    return 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
+def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm with unit gain: x / sqrt(mean(x^2) + eps)."""
+    return np.asarray(x, dtype=np.float64) * rms_factor(x, eps)
+
+
+def rope(x: np.ndarray, pos: Sequence[int], base: float = 10000.0) -> np.ndarray:
+    """Rotate-half rotary embedding.
+
+    x: [n, heads, D]; pos: [n] absolute positions.  For i < D/2 the pair
+    (x_i, x_{i+D/2}) is rotated by theta_i = pos * base**(-2i/D)."""
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    half = D // 2
+    inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / D)
+    theta = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]   # [n, half]
+    c = np.cos(theta)[:, None, :]
+    s = np.sin(theta)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def silu(a: np.ndarray) -> np.ndarray:
+    return a / (1.0 + np.exp(-a))
+
+
+# ----------------------------------------------------------------------------
+# Attention masks and attention  [FDV §2.2.1 masks; FDVW §4.1]
+# ----------------------------------------------------------------------------
+def mask_from_roles(q_noisy: Sequence[bool], q_block: Sequence[int], q_pos: Sequence[int],
+                    k_noisy: Sequence[bool], k_block: Sequence[int], k_pos: Sequence[int]) -> np.ndarray:
+    """Dense 0/1 visibility matrix from token roles (the three rules).
+
+    N2N: a noisy query sees the noisy keys of its own block (bidirectional).
+    N2C: a noisy query sees the clean keys of strictly preceding blocks.
+    C2C: a clean query sees clean keys at positions <= its own (causal).
+    A clean query never sees a noisy key."""
+    nq, nk = len(q_noisy), len(k_noisy)
+    m = np.zeros((nq, nk), dtype=np.int64)
+    for i in range(nq):
+        for j in range(nk):
+            if q_noisy[i] and k_noisy[j]:
+                m[i, j] = int(q_block[i] == k_block[j])
+            elif q_noisy[i] and not k_noisy[j]:
+                m[i, j] = int(k_block[j] < q_block[i])
+            elif not q_noisy[i] and not k_noisy[j]:
+                m[i, j] = int(k_pos[j] <= q_pos[i])
+    return m
+
+
+def dense_masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray,
+                           scale: float) -> np.ndarray:
+    """Brute force: q [nq, Hq, D], k/v [nk, Hkv, D], mask [nq, nk]; GQA group
+    Hq/Hkv.  Explicit masked softmax per (query, head)."""
+    nq, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((nq, Hq, D))
+    for i in range(nq):
+        vis = np.nonzero(mask[i])[0]
+        for h in range(Hq):
+            g = h // G
+            s = np.array([scale * float(np.dot(q[i, h], k[j, g])) for j in vis])
+            p = np.exp(s - s.max())
+            p = p / p.sum()
+            out[i, h] = sum(p[t] * v[vis[t], g] for t in range(len(vis)))
+    return out
+
+
+def block_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, L: int, n_clean: int,
+                    scale: float) -> np.ndarray:
+    """Attention of one step's rows against the KV cache.
+
+    q: [n, Hq, D] for rows at cache slots L .. L+n-1 (their K/V already in the
+    cache).  K, V: [Hkv, >= L+n, D].  Rows 0..n_clean-1 are clean (causal:
+    row t sees slots 0..L+t); the remaining rows form the noisy block and see
+    every slot 0..L+n-1 (the whole cache through N2C plus the whole block
+    through N2N)."""
+    q = np.asarray(q, dtype=np.float64)
+    n, Hq, D = q.shape
+    Hkv = K.shape[0]
+    G = Hq // Hkv
+    out = np.zeros((n, Hq, D))
+    for t in range(n):
+        vis = (L + t + 1) if t < n_clean else (L + n)
+        for h in range(Hq):
+            g = h // G
+            s = scale * (K[g, :vis] @ q[t, h])
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            out[t, h] = p @ V[g, :vis]
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Confidence, commit, certificate, accept
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class Conf:
+    p1: np.ndarray     # top-1 probability per row
+    top1: np.ndarray   # lowest id attaining the max logit
+    p2: np.ndarray     # second-largest probability (margin checks)
+
+
+def confidence_from_logits(logits: np.ndarray) -> Conf:
+    """Top-1 confidence = max softmax probability over the vocabulary
+    [LOWN method step (1): s = max_w p(y_i = w | ...)], argmax = lowest id."""
+    lg = np.asarray(logits, dtype=np.float64)
+    m = lg.max(axis=-1, keepdims=True)
+    e = np.exp(lg - m)
+    s = e.sum(axis=-1)
+    p1 = 1.0 / s
+    top1 = np.argmax(lg, axis=-1).astype(np.int64)      # first maximum
+    part = np.partition(lg, -2, axis=-1)[..., -2]
+    p2 = np.exp(part - m[..., 0]) / s
+    return Conf(p1=p1, top1=top1, p2=p2)
+
+
+def lm_head_conf(hidden: np.ndarray, W: np.ndarray, row_scale: Optional[np.ndarray] = None) -> Conf:
+    """logits = row_scale * (hidden @ W^T) (row_scale = final RMSNorm factor or 1)."""
+    lg = np.asarray(hidden, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+    if row_scale is not None:
+        lg = lg * np.asarray(row_scale, dtype=np.float64).reshape(-1, 1)
+    return confidence_from_logits(lg)
+
+
+def threshold_commit(p1: Sequence[float], masked: Sequence[bool], tau: float) -> List[int]:
+    """Commit every masked row with p1 >= tau; when none passes, commit the
+    masked row with the highest p1 (lowest index on ties).
+    [FDV §4.1 threshold 0.9; DAVET generic commit rule]"""
+    R = len(p1)
+    C = [r for r in range(R) if masked[r] and p1[r] >= tau]
+    if not C:
+        best = None
+        for r in range(R):
+            if masked[r] and (best is None or p1[r] > p1[best]):
+                best = r
+        if best is not None:
+            C = [best]
+    return C
+
+
+def certificate_scan(anchor_id: Sequence[int], anchor_conf: Sequence[float],
+                     top1: Sequence[int], participants: Optional[Sequence[bool]] = None) -> int:
+    """Longest certified prefix [LOWN method step (2)]: visit positions in
+    descending anchor confidence (lower index first on ties) and stop at the
+    first whose new top-1 differs from its anchor; return the count before it."""
+    R = len(anchor_id)
+    idx = [i for i in range(R) if participants is None or participants[i]]
+    idx.sort(key=lambda i: (-float(anchor_conf[i]), i))
+    n = 0
+    for i in idx:
+        if int(top1[i]) != int(anchor_id[i]):
+            break
+        n += 1
+    return n
+
+
+def prefix_accept(verify_ids: Sequence[int], draft_ids: Sequence[int]) -> int:
+    """Longest prefix on which the causal pass's argmax equals the draft
+    [FDV §2.3.1 longest-prefix acceptance]."""
+    k = 0
+    for a, b in zip(verify_ids, draft_ids):
+        if int(a) != int(b):
+            break
+        k += 1
+    return k
+
+
+# ----------------------------------------------------------------------------
+# Model
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class Dims:
+    n_layers: int
+    hidden: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    inter: int
+    vocab: int
+    rope_base: float = 10000.0
+    eps: float = 1e-6
+
+    @property
+    def mask_id(self) -> int:
+        return self.vocab - 1
+
+
+class OracleModel:
+    """The decoder as plain definitions.
+
+    weights: dict with "embed" [V,H], "lm_head" [V,H] and per layer l the
+    matrices "l.wq", "l.wk", "l.wv", "l.wo", "l.wg", "l.wu", "l.wd" ([out,in]).
+    A callable ``weights_fn(name)`` may be given instead, to regenerate big
+    matrices on demand.  ``bf16``: round activations at the GPU's storage
+    points (q/k/v after RoPE, attention output, residual stream, SwiGLU
+    activation)."""
+
+    def __init__(self, dims: Dims, weights=None, weights_fn=None, bf16: bool = True,
+                 Lmax: int = 4096):
+        self.d = dims
+        self._w = weights
+        self._wfn = weights_fn
+        self.bf16 = bf16
+        self.Lmax = Lmax
+        self.K = [np.zeros((dims.n_kv_heads, Lmax, dims.head_dim)) for _ in range(dims.n_layers)]
+        self.V = [np.zeros((dims.n_kv_heads, Lmax, dims.head_dim)) for _ in range(dims.n_layers)]
+        self.L = 0
+
+    def w(self, name: str) -> np.ndarray:
+        if self._w is not None and name in self._w:
+            return self._w[name]
+        return np.asarray(self._wfn(name), dtype=np.float64)
+
+    def rnd(self, x: np.ndarray) -> np.ndarray:
+        return bf16_round(x) if self.bf16 else x
+
+    # -- one decoder layer ---------------------------------------------------
+    def layer(self, l: int, x: np.ndarray, L: int, n_clean: int, write_kv: bool = True) -> np.ndarray:
+        d = self.d
+        n = x.shape[0]
+        D, Hq, Hkv = d.head_dim, d.n_q_heads, d.n_kv_heads
+        pos = np.arange(L, L + n)
+        h = x * rms_factor(x, d.eps)
+        q = (h @ self.w(f"{l}.wq").T).reshape(n, Hq, D)
+        k = (h @ self.w(f"{l}.wk").T).reshape(n, Hkv, D)
+        v = (h @ self.w(f"{l}.wv").T).reshape(n, Hkv, D)
+        q = self.rnd(rope(q, pos, d.rope_base))
+        k = self.rnd(rope(k, pos, d.rope_base))
+        v = self.rnd(v)
+        if write_kv:
+            self.K[l][:, L:L + n] = k.transpose(1, 0, 2)
+            self.V[l][:, L:L + n] = v.transpose(1, 0, 2)
+        a = block_attention(q, self.K[l], self.V[l], L, n_clean, 1.0 / math.sqrt(D))
+        a = self.rnd(a).reshape(n, Hq * D)
+        x = self.rnd(x + a @ self.w(f"{l}.wo").T)
+        h2 = x * rms_factor(x, d.eps)
+        g = h2 @ self.w(f"{l}.wg").T
+        u = h2 @ self.w(f"{l}.wu").T
+        act = self.rnd(silu(g) * u)
+        x = self.rnd(x + act @ self.w(f"{l}.wd").T)
+        return x
+
+    def embed(self, ids: Sequence[int]) -> np.ndarray:
+        E = self.w("embed")
+        return np.asarray(E[np.asarray(ids, dtype=np.int64)], dtype=np.float64)
+
+    def forward(self, x: np.ndarray, L: int, n_clean: int) -> np.ndarray:
+        """Run all layers over rows at slots L..L+n-1; returns the final
+        residual stream (before the final norm).  K/V of these rows are
+        written to the cache; the cache length is NOT advanced here."""
+        for l in range(self.d.n_layers):
+            x = self.layer(l, x, L, n_clean)
+        return x
+
+    def logits_conf(self, x: np.ndarray) -> Conf:
+        """Final RMSNorm + LM head + confidence."""
+        return lm_head_conf(x, self.w("lm_head"), rms_factor(x, self.d.eps)[:, 0])
+
+
+# ----------------------------------------------------------------------------
+# Decode drivers
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class DecodeTrace:
+    tokens: List[int]
+    nfe: int = 0
+    commits_per_iter: List[int] = dataclasses.field(default_factory=list)
+    accept_lens: List[int] = dataclasses.field(default_factory=list)
+    # smallest decision margin met along the trajectory (for parity exclusion)
+    min_margin: float = math.inf
+    margins: List[float] = dataclasses.field(default_factory=list)
+
+
+def prefill(model: OracleModel, vision: Optional[np.ndarray], ids: Sequence[int]) -> int:
+    """Causal pass over [vision rows | text ids]; returns the AR seed token
+    (argmax of the LM head at the last context row) and sets model.L."""
+    rows = []
+    if vision is not None and len(vision):
+        rows.append(np.asarray(vision, dtype=np.float64))
+    if len(ids):
+        rows.append(model.embed(ids))
+    x = np.concatenate(rows, axis=0)
+    n = x.shape[0]
+    xo = model.forward(x, 0, n_clean=n)
+    model.L = n
+    c = model.logits_conf(xo[-1:])
+    model.last_conf = c
+    return int(c.top1[0])
+
+
+def _note_argmax_margin(tr: DecodeTrace, c: Conf, rows) -> None:
+    for r in rows:
+        m = float(c.p1[r] - c.p2[r])
+        tr.margins.append(m)
+        tr.min_margin = min(tr.min_margin, m)
+
+
+def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, max_new: int,
+                     shift: int = 1, ar_seed: int = 1) -> DecodeTrace:
+    """Threshold (MDM-style) block decoding [FDV §2.2.1, §2.2.2, §4.1].
+
+    Per block: the first token is the AR seed (ar_seed=1); the remaining
+    positions start as [MASK].  Each iteration runs the whole block as noisy
+    rows over the cache (its K/V go to slots L..L+B-1 without advancing L),
+    scores the still-masked positions (position j from row j-shift; row -1 is
+    the previous pass's last row) and commits per ``threshold_commit``.  When
+    the block is complete a causal pass over it makes its K/V final, advances
+    L by B and yields the next block's seed from its last row."""
+    d = model.d
+    tr = DecodeTrace(tokens=[])
+    seed = seed_token
+    prev_conf = model.last_conf
+    while len(tr.tokens) < max_new:
+        L = model.L
+        toks = [d.mask_id] * B
+        masked = [True] * B
+        if ar_seed:
+            toks[0] = seed
+            masked[0] = False
+        while any(masked):
+            x = model.forward(model.embed(toks), L, n_clean=0)
+            c = model.logits_conf(x)
+            p1 = np.zeros(B)
+            top = np.zeros(B, dtype=np.int64)
+            p2 = np.zeros(B)
+            for j in range(B):
+                r = j - shift
+                cc, rr = (prev_conf, 0) if r < 0 else (c, r)
+                p1[j], top[j], p2[j] = cc.p1[rr], cc.top1[rr], cc.p2[rr]
+            C = threshold_commit(p1, masked, tau)
+            for j in range(B):
+                if masked[j]:
+                    mg = min(abs(p1[j] - tau), p1[j] - p2[j])
+                    tr.margins.append(mg)
+                    tr.min_margin = min(tr.min_margin, mg)
+            if len(C) == 1 and not (p1[C[0]] >= tau):
+                others = [p1[j] for j in range(B) if masked[j] and j != C[0]]
+                if others:
+                    mg = float(p1[C[0]] - max(others))
+                    tr.margins.append(mg)
+                    tr.min_margin = min(tr.min_margin, mg)
+            for j in C:
+                toks[j] = int(top[j])
+                masked[j] = False
+            tr.commits_per_iter.append(len(C))
+            tr.nfe += 1
+        x = model.forward(model.embed(toks), L, n_clean=B)
+        model.L = L + B
+        c = model.logits_conf(x)
+        tr.nfe += 1
+        _note_argmax_margin(tr, c, [B - 1])
+        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:])
+        seed = int(c.top1[B - 1])
+        tr.tokens.extend(toks)
+    tr.tokens = tr.tokens[:max_new]
+    return tr
+
+
+def decode_spec_linear(model: OracleModel, seed_token: int, B: int, max_new: int) -> DecodeTrace:
+    """Linear self-speculative decoding [FDV §2.3.1]: a diffusion draft pass
+    (every position takes its argmax), then a causal verify pass over the
+    draft; the longest prefix on which the verifier agrees is kept (position
+    0, the AR seed, always), L advances by its length and the verifier's
+    prediction right after it seeds the next round (shift=1)."""
+    d = model.d
+    tr = DecodeTrace(tokens=[])
+    seed = seed_token
+    while len(tr.tokens) < max_new:
+        L = model.L
+        toks = [seed] + [d.mask_id] * (B - 1)
+        x = model.forward(model.embed(toks), L, n_clean=0)
+        c = model.logits_conf(x)
+        _note_argmax_margin(tr, c, range(B - 1))
+        draft = [seed] + [int(c.top1[j - 1]) for j in range(1, B)]
+        tr.nfe += 1
+        x = model.forward(model.embed(draft), L, n_clean=B)
+        g = model.logits_conf(x)
+        _note_argmax_margin(tr, g, range(B))
+        tr.nfe += 1
+        verify = [seed] + [int(g.top1[j - 1]) for j in range(1, B)]
+        k = prefix_accept(verify, draft)
+        tr.accept_lens.append(k)
+        tr.tokens.extend(draft[:k])
+        model.L = L + k
+        seed = int(g.top1[k - 1])
+    tr.tokens = tr.tokens[:max_new]
+    return tr
+
+
+def decode_ar(model: OracleModel, seed_token: int, max_new: int) -> DecodeTrace:
+    """Greedy autoregressive decoding, one token per forward (comparator)."""
+    tr = DecodeTrace(tokens=[])
+    seed = seed_token
+    while len(tr.tokens) < max_new:
+        L = model.L
+        x = model.forward(model.embed([seed]), L, n_clean=1)
+        model.L = L + 1
+        c = model.logits_conf(x)
+        _note_argmax_margin(tr, c, [0])
+        tr.nfe += 1
+        tr.tokens.append(seed)
+        seed = int(c.top1[0])
+    return tr
+
+
+# ----------------------------------------------------------------------------
+# Weight helpers for tests and the CPU baseline (the generator draws values;
+# here they are only arranged under the names the oracle uses)
+# ----------------------------------------------------------------------------
+def weights_from_generator(gen, dims, seed: int) -> Dict[str, np.ndarray]:
+    """Materialise every matrix of a (small) model as float64."""
+    out = {"embed": np.asarray(gen.embedding_weight(dims, seed)[1], dtype=np.float64),
+           "lm_head": np.asarray(gen.lm_head_weight(dims, seed)[1], dtype=np.float64)}
+    for l in range(dims.n_layers):
+        for nm in gen.layer_weight_names():
+            out[f"{l}.{nm}"] = np.asarray(gen.layer_weight(dims, seed, l, nm)[1], dtype=np.float64)
+    return out
+
+
+def dims_from(gdims) -> Dims:
+    return Dims(n_layers=gdims.n_layers, hidden=gdims.hidden, n_q_heads=gdims.n_q_heads,
+                n_kv_heads=gdims.n_kv_heads, head_dim=gdims.head_dim, inter=gdims.inter,
+                vocab=gdims.vocab, rope_base=gdims.rope_base, eps=gdims.eps)

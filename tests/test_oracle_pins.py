@@ -1,0 +1,420 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself:
+the pages' printed mask example, closed forms, library routines (torch's
+bf16 cast, scipy's softmax/expit, numpy's sort), brute force on tiny inputs,
+and invariants of the decoding method.  Each pin is chosen so that a plausible
+slip (dropped term, wrong sign or index, transposed operand, > for >=) fails.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special as sps
+import torch
+
+import dvlm_gen as gen
+import oracle as O
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding
+# ----------------------------------------------------------------------------
+def test_bf16_round_matches_torch_cast():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(200000).astype(np.float32) * 3,
+                        rng.standard_normal(1000).astype(np.float32) * 1e-30,
+                        rng.standard_normal(1000).astype(np.float32) * 1e30])
+    # exact halfway points between neighbouring bf16 values
+    base = torch.from_numpy(rng.standard_normal(5000).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    bits = base.view(np.uint32) | np.uint32(0x8000)
+    x = np.concatenate([x, bits.view(np.float32)])
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy().astype(np.float64)
+    np.testing.assert_array_equal(O.bf16_round(x.astype(np.float64)), ref)
+
+
+def test_bf16_round_ties_to_even():
+    assert O.bf16_round(1.0 + 2.0 ** -8) == 1.0              # halfway, even is 1.0
+    assert O.bf16_round(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.bf16_round(-(1.0 + 2.0 ** -8 + 2.0 ** -20)) == -(1.0 + 2.0 ** -7)
+    assert O.bf16_round(0.0) == 0.0
+
+
+# ----------------------------------------------------------------------------
+# RMSNorm, RoPE, SiLU
+# ----------------------------------------------------------------------------
+def test_rmsnorm_closed_form():
+    for c in (0.5, -3.0, 1e-3):
+        x = np.full((2, 64), c)
+        np.testing.assert_allclose(O.rmsnorm(x, 1e-6), c / math.sqrt(c * c + 1e-6), rtol=1e-14)
+    x = np.random.default_rng(1).standard_normal((3, 128)) * 7
+    y = O.rmsnorm(x, 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-12)
+    np.testing.assert_array_equal(O.rmsnorm(np.zeros((1, 8))), 0.0)
+
+
+def test_rope_complex_form_and_invariants():
+    rng = np.random.default_rng(2)
+    D, base = 16, 10000.0
+    x = rng.standard_normal((5, 3, D))
+    pos = np.array([0, 1, 7, 100, 1523])
+    y = O.rope(x, pos, base)
+    half = D // 2
+    z = x[..., :half] + 1j * x[..., half:]
+    for t, p in enumerate(pos):
+        th = p * base ** (-2.0 * np.arange(half) / D)
+        w = z[t] * np.exp(1j * th)[None, :]
+        np.testing.assert_allclose(y[t, :, :half], w.real, atol=1e-12)
+        np.testing.assert_allclose(y[t, :, half:], w.imag, atol=1e-12)
+    np.testing.assert_allclose(y[0], x[0], atol=0)                     # position 0
+    q, k = rng.standard_normal((1, 1, D)), rng.standard_normal((1, 1, D))
+    d1 = np.sum(O.rope(q, [37], base) * O.rope(k, [12], base))
+    d2 = np.sum(O.rope(q, [1037], base) * O.rope(k, [1012], base))
+    assert abs(d1 - d2) < 1e-9                                          # relative position only
+
+
+def test_silu_matches_library():
+    a = np.linspace(-30, 30, 1001)
+    np.testing.assert_allclose(O.silu(a), a * sps.expit(a), rtol=1e-13, atol=1e-300)
+
+
+# ----------------------------------------------------------------------------
+# Masks and attention
+# ----------------------------------------------------------------------------
+def _load_matrix(name):
+    rows = []
+    with open(os.path.join(HERE, "golden", name)) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([int(v) for v in line.split()])
+    return np.array(rows)
+
+
+def test_n2n_mask_reproduces_printed_example():
+    want = _load_matrix("mask_n2n_block2.txt")
+    blocks = [0, 0, 1, 1]
+    m = O.mask_from_roles([True] * 4, blocks, [0, 1, 2, 3], [True] * 4, blocks, [0, 1, 2, 3])
+    np.testing.assert_array_equal(m, want)
+
+
+def test_n2c_and_c2c_rules():
+    blocks = [0, 0, 1, 1]
+    pos = [0, 1, 2, 3]
+    n2c = O.mask_from_roles([True] * 4, blocks, pos, [False] * 4, blocks, pos)
+    # noisy tokens see clean tokens of preceding blocks only, never the clean
+    # copy of their own block (that would leak the answer)
+    np.testing.assert_array_equal(n2c, [[0, 0, 0, 0], [0, 0, 0, 0], [1, 1, 0, 0], [1, 1, 0, 0]])
+    c2c = O.mask_from_roles([False] * 4, blocks, pos, [False] * 4, blocks, pos)
+    np.testing.assert_array_equal(c2c, np.tril(np.ones((4, 4), dtype=int)))
+    c2n = O.mask_from_roles([False] * 4, blocks, pos, [True] * 4, blocks, pos)
+    assert c2n.sum() == 0
+
+
+def _roles_case(rng, L, n, n_clean, Hq=4, Hkv=2, D=8):
+    """A cache of L clean tokens (blocks of 4) plus n rows at slots L..L+n-1."""
+    q = rng.standard_normal((n, Hq, D))
+    K = rng.standard_normal((Hkv, L + n, D))
+    V = rng.standard_normal((Hkv, L + n, D))
+    return q, K, V
+
+
+@pytest.mark.parametrize("L,n,n_clean", [(12, 4, 0), (9, 5, 0), (8, 4, 4), (0, 3, 3), (7, 1, 1), (5, 6, 2)])
+def test_block_attention_equals_dense_masked_bruteforce(L, n, n_clean):
+    rng = np.random.default_rng(L * 31 + n * 7 + n_clean)
+    q, K, V = _roles_case(rng, L, n, n_clean)
+    scale = 1 / math.sqrt(q.shape[-1])
+    got = O.block_attention(q, K, V, L, n_clean, scale)
+    # dense formulation: keys = cache (clean, blocks < current) then step rows;
+    # step rows 0..n_clean-1 are clean (causal), the rest one noisy block
+    cur = 10 ** 6
+    k_noisy = [False] * (L + n_clean) + [True] * (n - n_clean)
+    k_block = [j // 4 for j in range(L)] + [cur - 1] * n_clean + [cur] * (n - n_clean)
+    k_pos = list(range(L + n))
+    q_noisy, q_block, q_pos = k_noisy[L:], k_block[L:], k_pos[L:]
+    m = O.mask_from_roles(q_noisy, q_block, q_pos, k_noisy, k_block, k_pos)
+    want = O.dense_masked_attention(q, K.transpose(1, 0, 2), V.transpose(1, 0, 2), m, scale)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(3)
+    L, n, D = 10, 4, 8
+    q = rng.standard_normal((n, 2, D))
+    K = np.tile(rng.standard_normal((1, 1, D)), (1, L + n, 1))     # all keys equal
+    V = rng.standard_normal((1, L + n, D))
+    out = O.block_attention(q, K, V, L, 0, 0.3)
+    np.testing.assert_allclose(out[2, 1], V[0].mean(axis=0), rtol=1e-12)
+    out = O.block_attention(q, K, V, L, 2, 0.3)                       # clean row 1 sees L+2 slots
+    np.testing.assert_allclose(out[1, 0], V[0, :L + 2].mean(axis=0), rtol=1e-12)
+    K2 = rng.standard_normal((1, L + n, D)) * 0.01
+    K2[0, 5] = q[3, 0] * 1e4                                           # one dominant key
+    out = O.block_attention(q, K2, V, L, 0, 1.0)
+    np.testing.assert_allclose(out[3, 0], V[0, 5], rtol=1e-9)
+    # single causal row at the end of a cache == textbook softmax attention
+    q1 = rng.standard_normal((1, 2, D))
+    Kc, Vc = rng.standard_normal((1, 9, D)), rng.standard_normal((1, 9, D))
+    out = O.block_attention(q1, Kc, Vc, 8, 1, 0.5)
+    for h in range(2):
+        p = sps.softmax(0.5 * Kc[0] @ q1[0, h])
+        np.testing.assert_allclose(out[0, h], p @ Vc[0], rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Confidence / argmax
+# ----------------------------------------------------------------------------
+def test_confidence_matches_full_softmax_and_sort():
+    rng = np.random.default_rng(4)
+    lg = rng.standard_normal((6, 3000)) * 20
+    c = O.confidence_from_logits(lg)
+    p = sps.softmax(lg, axis=-1)
+    order = np.argsort(-lg, axis=-1, kind="stable")
+    ps = np.sort(p, axis=-1)
+    np.testing.assert_allclose(c.p1, ps[:, -1], rtol=1e-12)
+    np.testing.assert_allclose(c.p2, ps[:, -2], rtol=1e-12)
+    np.testing.assert_array_equal(c.top1, order[:, 0])
+
+
+def test_confidence_closed_forms():
+    # one-hot LM-head rows: logits are the hidden entries themselves
+    H = 16
+    W = np.eye(H)
+    h = np.arange(H, dtype=float)[None, :] * 0.1
+    c = O.lm_head_conf(h, W)
+    assert c.top1[0] == H - 1
+    want = 1.0 / np.sum(np.exp(h[0] - h[0].max()))
+    assert abs(c.p1[0] - want) < 1e-15
+    # two equal maxima: p1 <= 1/2 and the lower id wins
+    lg = np.array([[1.0, 5.0, 0.0, 5.0, 2.0]])
+    c = O.confidence_from_logits(lg)
+    assert c.top1[0] == 1 and c.p1[0] <= 0.5 and abs(c.p1[0] - c.p2[0]) < 1e-15
+    # uniform logits: p1 = 1/V
+    c = O.confidence_from_logits(np.zeros((1, 256)))
+    assert abs(c.p1[0] - 1 / 256) < 1e-15 and c.top1[0] == 0
+
+
+# ----------------------------------------------------------------------------
+# Commit, certificate, accept (hand-worked cases)
+# ----------------------------------------------------------------------------
+def test_threshold_commit_hand_cases():
+    assert O.threshold_commit([.95, .5, .91, .2], [1, 1, 1, 1], 0.9) == [0, 2]
+    assert O.threshold_commit([.5, .6, .3], [1, 1, 1], 0.9) == [1]           # force one
+    assert O.threshold_commit([.9, .1], [1, 1], 0.9) == [0]                  # >= threshold
+    assert O.threshold_commit([.9, .95, .2], [1, 1, 1], 0.9) == [0, 1]
+    assert O.threshold_commit([.6, .6, .2], [1, 1, 1], 0.9) == [0]           # tie -> lowest
+    assert O.threshold_commit([.99, .6, .2], [0, 1, 1], 0.9) == [1]          # unmasked ignored
+    assert O.threshold_commit([.99, .6], [0, 0], 0.9) == []                  # nothing masked
+    assert O.threshold_commit([.2, .3, .1], [1, 1, 1], -1.0) == [0, 1, 2]    # draft: commit all
+
+
+def test_certificate_hand_cases():
+    ids, conf = [3, 7, 9, 1], [.2, .9, .5, .8]          # order: 1, 3, 2, 0
+    assert O.certificate_scan(ids, conf, [3, 7, 4, 1]) == 2      # disagrees at position 2
+    assert O.certificate_scan(ids, conf, ids) == 4               # all agree
+    assert O.certificate_scan(ids, conf, [3, 0, 9, 1]) == 0      # first in order disagrees
+    assert O.certificate_scan(ids, conf, [0, 7, 9, 1]) == 3      # lowest-confidence one last
+    assert O.certificate_scan([1, 2, 3], [.5, .5, .5], [1, 9, 3]) == 1   # ties: lower index first
+    assert O.certificate_scan([1, 2, 3], [.5, .5, .5], [1, 2, 9]) == 2
+    assert O.certificate_scan(ids, conf, [3, 7, 4, 1], [1, 1, 0, 1]) == 3  # non-participant skipped
+
+
+def test_prefix_accept_hand_cases():
+    assert O.prefix_accept([5, 7, 1, 2], [5, 7, 9, 2]) == 2
+    assert O.prefix_accept([5, 7, 9, 2], [5, 7, 9, 2]) == 4
+    assert O.prefix_accept([4, 7, 9, 2], [5, 7, 9, 2]) == 0
+
+
+# ----------------------------------------------------------------------------
+# Decode-level invariants on tiny models
+# ----------------------------------------------------------------------------
+def _tiny(bf16=False, seed=0, layers=1, lm_scale=40.0):
+    if bf16:
+        gd = gen.ModelDims(n_layers=layers, hidden=64, n_q_heads=4, n_kv_heads=2, head_dim=16,
+                           inter=96, vocab=512, lm_scale=lm_scale, dtype="bf16")
+    else:
+        gd = gen.TINY
+    d = O.dims_from(gd)
+    w = O.weights_from_generator(gen, gd, seed)
+    vis_t, vis, ids = gen.decode_context(gd, seed, 32, 16, 16)
+    return gd, d, w, vis.astype(np.float64), ids
+
+
+def _fresh(d, w, bf16, vis, ids):
+    m = O.OracleModel(d, weights=w, bf16=bf16, Lmax=512)
+    seed_tok = O.prefill(m, vis, ids)
+    return m, seed_tok
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_spec_linear_equals_greedy_ar(bf16):
+    gd, d, w, vis, ids = _tiny(bf16)
+    m1, s1 = _fresh(d, w, bf16, vis, ids)
+    ar = O.decode_ar(m1, s1, 40)
+    m2, s2 = _fresh(d, w, bf16, vis, ids)
+    sp = O.decode_spec_linear(m2, s2, 8, 40)
+    assert sp.tokens == ar.tokens
+    assert all(1 <= k <= 8 for k in sp.accept_lens)
+    assert m2.L == m1.L + (sum(sp.accept_lens) - 40)  # spec may run past max_new
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_threshold_block1_equals_ar(bf16):
+    gd, d, w, vis, ids = _tiny(bf16)
+    m1, s1 = _fresh(d, w, bf16, vis, ids)
+    ar = O.decode_ar(m1, s1, 12)
+    m2, s2 = _fresh(d, w, bf16, vis, ids)
+    th = O.decode_threshold(m2, s2, 1, 0.9, 12)
+    assert th.tokens == ar.tokens and th.nfe == ar.nfe
+
+
+def test_threshold_extreme_thresholds():
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s = _fresh(d, w, False, vis, ids)
+    tr = O.decode_threshold(m, s, B, 1.5, 2 * B)       # nothing passes: one commit per iteration
+    assert tr.commits_per_iter == [1] * (2 * (B - 1))
+    assert tr.nfe == 2 * (B - 1) + 2
+    m, s = _fresh(d, w, False, vis, ids)
+    tr = O.decode_threshold(m, s, B, 0.0, 2 * B)       # everything passes: one iteration
+    assert tr.commits_per_iter == [B - 1, B - 1] and tr.nfe == 4
+
+
+def test_block_first_token_is_ar_token_and_append_kv_equals_prefill():
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s = _fresh(d, w, False, vis, ids)
+    m_ar, s_ar = _fresh(d, w, False, vis, ids)
+    tr = O.decode_threshold(m, s, B, 0.9, B)
+    ar = O.decode_ar(m_ar, s_ar, 1)
+    assert tr.tokens[0] == ar.tokens[0]
+    # KV of the causal append pass == KV of a prefill over the same prefix
+    m2 = O.OracleModel(d, weights=w, bf16=False, Lmax=512)
+    O.prefill(m2, vis, list(ids) + tr.tokens)
+    L = m.L
+    assert L == len(vis) + len(ids) + B == m2.L
+    np.testing.assert_allclose(m.K[0][:, :L], m2.K[0][:, :L], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(m.V[0][:, :L], m2.V[0][:, :L], rtol=1e-12, atol=1e-12)
+
+
+def test_tiny_threshold_run_completes_block():
+    """First configuration: 64-token context, one B=4 block, threshold 0.9."""
+    gd, d, w, vis, ids = _tiny()
+    m, s = _fresh(d, w, False, vis, ids)
+    tr = O.decode_threshold(m, s, 4, 0.9, 4)
+    assert len(tr.tokens) == 4 and sum(tr.commits_per_iter) == 3
+    assert all(0 <= t < d.vocab for t in tr.tokens)
+    # the tiny LM head (x40) spreads top-1 probabilities widely
+    c = O.lm_head_conf(np.random.default_rng(0).standard_normal((64, 32)), w["lm_head"])
+    assert c.p1.min() < 0.6 and c.p1.max() > 0.95
+
+
+# ----------------------------------------------------------------------------
+# Planted mistakes: each mutant of an oracle function must fail its pin
+# ----------------------------------------------------------------------------
+def _check_rope(fn):
+    x = np.random.default_rng(9).standard_normal((2, 1, 8))
+    y = fn(x, [3, 11], 10000.0)
+    z = x[..., :4] + 1j * x[..., 4:]
+    for t, p in enumerate([3, 11]):
+        w = z[t] * np.exp(1j * p * 10000.0 ** (-2.0 * np.arange(4) / 8))[None, :]
+        np.testing.assert_allclose(y[t, :, :4], w.real, atol=1e-12)
+        np.testing.assert_allclose(y[t, :, 4:], w.imag, atol=1e-12)
+
+
+def _check_commit(fn):
+    assert fn([.95, .5, .91, .2], [1, 1, 1, 1], 0.9) == [0, 2]
+    assert fn([.5, .6, .3], [1, 1, 1], 0.9) == [1]
+    assert fn([.9, .1], [1, 1], 0.9) == [0]
+    assert fn([.9, .95, .2], [1, 1, 1], 0.9) == [0, 1]
+    assert fn([.6, .6, .2], [1, 1, 1], 0.9) == [0]
+
+
+def _check_cert(fn):
+    ids, conf = [3, 7, 9, 1], [.2, .9, .5, .8]
+    assert fn(ids, conf, [3, 7, 4, 1]) == 2
+    assert fn([1, 2, 3], [.5, .5, .5], [1, 9, 3]) == 1
+    assert fn([1, 2, 3], [.5, .5, .5], [1, 2, 9]) == 2
+
+
+def _check_n2c(fn):
+    b, p = [0, 0, 1, 1], [0, 1, 2, 3]
+    np.testing.assert_array_equal(fn([True] * 4, b, p, [False] * 4, b, p),
+                                  [[0, 0, 0, 0], [0, 0, 0, 0], [1, 1, 0, 0], [1, 1, 0, 0]])
+
+
+def _check_attention(fn):
+    rng = np.random.default_rng(5)
+    q, K, V = rng.standard_normal((3, 2, 4)), rng.standard_normal((1, 8, 4)), rng.standard_normal((1, 8, 4))
+    got = fn(q, K, V, 5, 1, 0.5)
+    for t, vis in enumerate([6, 8, 8]):
+        for h in range(2):
+            np.testing.assert_allclose(got[t, h], sps.softmax(0.5 * K[0, :vis] @ q[t, h]) @ V[0, :vis], rtol=1e-12)
+
+
+def _check_argmax(fn):
+    assert fn(np.array([[1.0, 5.0, 0.0, 5.0, 2.0]])).top1[0] == 1
+
+
+def test_pins_accept_the_oracle():
+    _check_rope(O.rope)
+    _check_commit(O.threshold_commit)
+    _check_cert(O.certificate_scan)
+    _check_n2c(O.mask_from_roles)
+    _check_attention(O.block_attention)
+    _check_argmax(O.confidence_from_logits)
+
+
+def test_planted_mistakes_are_caught():
+    def rope_wrong_sign(x, pos, base=10000.0):
+        return O.rope(x, -np.asarray(pos), base)
+
+    def rope_wrong_pairing(x, pos, base=10000.0):      # interleaved pairs instead of halves
+        y = O.rope(x.reshape(*x.shape[:-1], -1, 2).swapaxes(-1, -2).reshape(x.shape), pos, base)
+        return y.reshape(*x.shape[:-1], 2, -1).swapaxes(-1, -2).reshape(x.shape)
+
+    def commit_strict(p1, masked, tau):
+        C = [r for r in range(len(p1)) if masked[r] and p1[r] > tau]
+        return C or O.threshold_commit(p1, masked, 2.0)
+
+    def commit_no_force(p1, masked, tau):
+        return [r for r in range(len(p1)) if masked[r] and p1[r] >= tau]
+
+    def cert_ascending(a, c, t, part=None):
+        return O.certificate_scan(a, [-v for v in c], t, part)
+
+    def cert_tie_high_first(a, c, t, part=None):
+        R = len(a)
+        idx = sorted(range(R), key=lambda i: (-c[i], -i))
+        n = 0
+        for i in idx:
+            if t[i] != a[i]:
+                break
+            n += 1
+        return n
+
+    def n2c_own_block(qn, qb, qp, kn, kb, kp):
+        m = O.mask_from_roles(qn, qb, qp, kn, kb, kp)
+        for i in range(len(qn)):
+            for j in range(len(kn)):
+                if qn[i] and not kn[j] and kb[j] == qb[i]:
+                    m[i, j] = 1
+        return m
+
+    def attn_clean_sees_block(q, K, V, L, n_clean, scale):
+        return O.block_attention(q, K, V, L, 0, scale)
+
+    def attn_no_scale(q, K, V, L, n_clean, scale):
+        return O.block_attention(q, K, V, L, n_clean, 1.0)
+
+    def argmax_last(lg):
+        c = O.confidence_from_logits(lg)
+        c.top1 = lg.shape[-1] - 1 - np.argmax(lg[..., ::-1], axis=-1)
+        return c
+
+    for check, mutant in [(_check_rope, rope_wrong_sign), (_check_rope, rope_wrong_pairing),
+                          (_check_commit, commit_strict), (_check_commit, commit_no_force),
+                          (_check_cert, cert_ascending), (_check_cert, cert_tie_high_first),
+                          (_check_n2c, n2c_own_block), (_check_attention, attn_clean_sees_block),
+                          (_check_attention, attn_no_scale), (_check_argmax, argmax_last)]:
+        with pytest.raises(AssertionError):
+            check(mutant)
