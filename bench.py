@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Block-decode tokens/s at batch 1 (B=16) on the Qwen2.5-3B-shaped synthetic
+decoder (36 layers, hidden 2048, 16/2 heads of 128, SwiGLU 11008, vocab
+151936, random init, LM head x25), context 1280 vision + 64 prompt, 256 new
+tokens, threshold 0.9; plus the fused LM-head's HBM GB/s against the measured
+peak.
+
+One step = one generation of 256 tokens from the prefilled context (the KV
+prefix and weights are resident in HBM; the cache length is rewound before
+each step).  Weights (6.2 GB) exceed the 126 MB L2, so no flush is needed
+between steps.  Multi-GPU runs are independent replicas (one request per GPU;
+the decode step has no data-path collective): value = all ranks' tokens / the
+slowest rank's time.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-decode tokens/sec at batch 1 (B=16); fused LM-head+commit HBM GB/s vs peak"
+N_VIS, N_PROMPT, N_NEW, BLOCK, TAU, SEED = 1280, 64, 256, 16, 0.9, 4
+WORKLOAD = "qwen2.5-3b-shaped block-diffusion decode: 36L h2048 16/2x128 ffn11008 V151936, ctx 1280 vision + 64 prompt, 256 new, B=16, tau 0.9"
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- ranks
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, value: float) -> float:
+    """Max of a per-rank float over all ranks (the job's time is the slowest rank's)."""
+    if pg is None:
+        return value
+    import torch
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank: int, world: int, max_seconds: float) -> float:
+    return tokens_per_rank * world / max_seconds
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sms, maxs, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxs.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sms if s > 0.5 * max(sms)] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "power_w_max": max(power), "samples": len(sms)}
+
+
+def gpu_uuid():
+    try:
+        import torch
+        u = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+        return f"GPU-{u}"
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- algorithmic bytes
+def algorithmic_bytes(kind: str, dims, L: int, rows: int = 16) -> float:
+    """Bytes a kernel must move per launch: its weights once, its inputs and
+    outputs once (bf16)."""
+    H, I, D, Hq, Hkv, V = dims.hidden, dims.inter, dims.head_dim, dims.n_q_heads, dims.n_kv_heads, dims.vocab
+    qkv = (Hq + 2 * Hkv) * D
+    if kind == "qkv_gemm":
+        return 2 * (qkv * H + rows * H + rows * qkv)
+    if kind == "oproj_gemm":
+        return 2 * (H * Hq * D + rows * Hq * D + 2 * rows * H)
+    if kind == "gateup_gemm":
+        return 2 * (2 * I * H + rows * H + rows * I)
+    if kind == "down_gemm":
+        return 2 * (H * I + rows * I + 2 * rows * H)
+    if kind == "lm_head":
+        return 2 * (V * H + rows * H)
+    if kind == "attention":
+        return 2 * (2 * Hkv * (L + rows) * D + 2 * rows * Hq * D)
+    return 0.0
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, when it was taken
+    on the current kernel source; else None."""
+    p = os.path.join(PROFILE_DIR, "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel)
+    if not ent:
+        return None
+    if ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_diffusion_vlm_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------- oracle CPU baseline
+def cpu_baseline(nfe_per_step: float, layers_timed: int = 4) -> dict:
+    """The oracle (fp64 numpy, as it stands) on a bounded sample of the
+    workload: one 16-row noisy-block forward at L=1344 through `layers_timed`
+    of the 36 decoder layers plus the LM head, with a generator-drawn KV
+    prefix; scaled to 36 layers and to the run's NFE per 256 tokens."""
+    import numpy as np
+    import dvlm_gen as gen
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    dims = gen.QWEN3B
+    od = O.dims_from(dims)
+    L, n = N_VIS + N_PROMPT, BLOCK
+    x = gen.normal(SEED, "cpu.x", (n, dims.hidden), 0.02).astype(np.float64)
+    t_layers = []
+    for l in range(layers_timed):
+        w = {f"{l}.{k}": gen.layer_weight(dims, SEED, l, k)[1].astype(np.float64) for k in gen.layer_weight_names()}
+        m = O.OracleModel(od, weights=w, bf16=True, Lmax=L + n)
+        m.K[l][:, :L] = gen.normal(SEED, f"cpu.k{l}", (dims.n_kv_heads, L, dims.head_dim))
+        m.V[l][:, :L] = gen.normal(SEED, f"cpu.v{l}", (dims.n_kv_heads, L, dims.head_dim))
+        t0 = time.perf_counter()
+        x = m.layer(l, x, L, 0)
+        t_layers.append(time.perf_counter() - t0)
+        del w, m
+    W = gen.lm_head_weight(dims, SEED)[1].astype(np.float64)
+    t0 = time.perf_counter()
+    O.lm_head_conf(x, W, O.rms_factor(x)[:, 0])
+    t_lm = time.perf_counter() - t0
+    del W
+    t_fwd = statistics.mean(t_layers) * dims.n_layers + t_lm
+    t_step = t_fwd * nfe_per_step
+    return {"value": N_NEW / t_step, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{layers_timed} of 36 decoder layers + LM head of one 16-row noisy forward at L=1344 "
+                      f"(fp64 numpy), scaled to 36 layers x {nfe_per_step:.1f} forwards per 256 tokens",
+            "forward_s": t_fwd}
+
+
+def workload_nfe() -> float | None:
+    p = os.path.join(PROFILE_DIR, "decode_workload.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f).get("nfe_per_256_threshold")
+    return None
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    nfe = workload_nfe() or float(N_NEW)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are not timed work
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(nfe, layers_timed=1))
+    elapsed = time.perf_counter() - t0
+    v = statistics.mean(c["value"] for c in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * elapsed / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": N_VIS + N_PROMPT + N_NEW,
+                                            "parallelism": "replicas", "l2": "weights 6.2 GB > L2"},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local, pg):
+    import torch
+    import block_diffusion_vlm_b200 as dv
+    import dvlm_gen as gen
+    from dvlm_gen.device import DeviceModel, kv_buffers
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dims = gen.QWEN3B
+    dm = DeviceModel(dims, SEED, device=dev)
+    Lmax = N_VIS + N_PROMPT + N_NEW + 32
+    kc, vc = kv_buffers(dims, Lmax, device=dev)
+    cm = dm.c_model()
+    ws = torch.zeros((dv.engine_workspace_size(cm, Lmax, BLOCK, N_VIS + N_PROMPT) + 3) // 4, dtype=torch.int32,
+                     device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    eng = dv.Engine(cm, kc, vc, Lmax, BLOCK, N_VIS + N_PROMPT, ws, stream=stream)
+    vis_t, vis, ids = gen.decode_context(dims, SEED, N_VIS, N_PROMPT)
+    vis_d, ids_d = vis_t.to(dev), torch.from_numpy(ids).to(dev)
+    eng.prefill(vis_d, N_VIS, ids_d, N_PROMPT, stream=stream)
+    eng.check(stream=stream)
+    L0, seed0 = eng.position(stream=stream)
+    mode = {"threshold": dv.MODE_THRESHOLD, "spec": dv.MODE_SPEC_LINEAR, "ar": dv.MODE_AR}[args.mode]
+    cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1)
+    out = torch.zeros(N_NEW, dtype=torch.int32, device=dev)
+
+    def step(c=cfg):
+        eng.set_position(L0, seed0, stream=stream)
+        st = dv.Stats()
+        eng.generate(c, out, st, stream=stream)
+        return st
+
+    for _ in range(args.warmup):
+        step()
+    eng.check(stream=stream)
+    clocks = ClockSampler(gpu_uuid()) if rank == 0 else None
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    stats = [step() for _ in range(args.steps)]
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(pg)
+    clk = clocks.stop() if clocks else None
+    eng.check(stream=stream)
+    secs = max_over_ranks(pg, ev0.elapsed_time(ev1) / 1000.0)
+    value = aggregate_throughput(N_NEW * args.steps, world, secs)
+    nfe = statistics.mean(s.nfe for s in stats)
+    launches = sum(s.n_launches for s in stats)
+    hist = [sum(s.commit_hist[i] for s in stats) for i in range(dv.binding.HIST)]
+
+    # end to end through the C ABI from pinned host buffers (prefill included)
+    vis_h, ids_h = vis_t.pin_memory(), torch.from_numpy(ids).pin_memory()
+    out_h = torch.zeros(N_NEW, dtype=torch.int32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    eng.generate_host(cfg, vis_h, N_VIS, ids_h, N_PROMPT, out_h, stream=stream)
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        eng.generate_host(cfg, vis_h, N_VIS, ids_h, N_PROMPT, out_h, stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_secs = max_over_ranks(pg, ev0.elapsed_time(ev1) / 1000.0)
+    e2e = {"value": aggregate_throughput(N_NEW * e2e_steps, world, e2e_secs), "unit": "tokens/s",
+           "h2d_bytes_per_step": N_VIS * dims.hidden * 2 + N_PROMPT * 4, "d2h_bytes_per_step": N_NEW * 4,
+           "includes": "H2D of vision+prompt, prefill of 1344 slots, 256-token decode, D2H of tokens"}
+
+    # live per-kernel timing (CUDA events around each launch of one eager forward)
+    eng.set_position(L0, seed0, stream=stream)
+    toks = torch.full((BLOCK,), dims.mask_id, dtype=torch.int32, device=dev)
+    prof = None
+    for _ in range(3):
+        prof = eng.profile_forward(toks, BLOCK, 0, stream=stream)
+    hbm_peak, peak_kind = peaks()
+    per = {}
+    for k, (ms, cnt) in prof.items():
+        if cnt:
+            b = algorithmic_bytes(k, dims, L0)
+            per[k] = {"ms_per_launch": ms / cnt, "launches": cnt, "gbs": b / (ms / cnt * 1e-3) / 1e9,
+                      "bytes_per_launch": b}
+    dom = max((k for k in per if k != "embed"), key=lambda k: per[k]["ms_per_launch"] * per[k]["launches"])
+
+    def roof(k):
+        return {"bound": "hbm", "achieved": per[k]["gbs"], "peak": hbm_peak, "unit": "GB/s",
+                "frac": per[k]["gbs"] / hbm_peak, "traffic": load_traffic(k), "kernel": k,
+                "peak_source": f"{peak_kind} copy bandwidth", "bytes_per_launch": per[k]["bytes_per_launch"],
+                "ms_per_launch": per[k]["ms_per_launch"]}
+
+    fwd_ms = sum(v["ms_per_launch"] * v["launches"] for v in per.values())
+    fwd_bytes = dims.n_params() * 2
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": N_VIS + N_PROMPT + N_NEW,
+                       "parallelism": f"replicas x{world}", "mode": args.mode,
+                       "l2": "inputs larger than L2 (6.2 GB of weights streamed per forward)"},
+            "roofline": roof(dom), "lmhead": roof("lm_head") if "lm_head" in per else None,
+            "gpu_launches": launches, "clocks": clk, "e2e": e2e,
+            "decode": {"nfe_per_step": nfe, "tokens_per_nfe": N_NEW / nfe, "commit_hist": hist,
+                       "ms_per_forward": 1000 * secs / args.steps / nfe,
+                       "forward_gbs": fwd_bytes / (secs / args.steps / nfe) / 1e9},
+            "kernels": per, "eager_forward_ms": fwd_ms}
+
+    # a short run of the linear self-speculative mode for context
+    if args.mode == "threshold" and not args.quick:
+        sc = dv.DecodeCfg(BLOCK, TAU, dv.MODE_SPEC_LINEAR, 1, N_NEW, 1)
+        step(sc)
+        ev0.record(stream)
+        st = step(sc)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        line["spec_linear"] = {"tokens_per_s": N_NEW / (ev0.elapsed_time(ev1) / 1000.0), "nfe": st.nfe,
+                               "accept_hist": list(st.accept_hist)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(nfe)
+    eng.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", choices=["threshold", "spec", "ar"], default="threshold")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the extra speculative-mode run")
+    args = ap.parse_args()
+    rank, world, local, pg = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

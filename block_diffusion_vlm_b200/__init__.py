@@ -1,0 +1,16 @@
+"""B200-native (sm_100a) block-diffusion decode step for Fast-dVLM-style
+block-diffusion VLM decoders.
+
+The work runs in ``libdvlm.so`` (hand-written CUDA kernels behind the C ABI of
+include/dvlm.h); this package is its ctypes binding.  Build the library with
+``python -m block_diffusion_vlm_b200.build``.
+"""
+from .binding import (DVLM_BF16, DVLM_FP32, MODE_AR, MODE_SPEC_LINEAR, MODE_THRESHOLD, DecodeCfg, DvlmError,
+                      Engine, Model, Stats, block_attn, declared_symbols, engine_workspace_size, lib,
+                      lmhead_conf_commit, lmhead_workspace_size, make_model, spec_verify_accept,
+                      spec_workspace_size, status_string)
+
+__all__ = ["DVLM_BF16", "DVLM_FP32", "MODE_AR", "MODE_SPEC_LINEAR", "MODE_THRESHOLD", "DecodeCfg", "DvlmError",
+           "Engine", "Model", "Stats", "block_attn", "declared_symbols", "engine_workspace_size", "lib",
+           "lmhead_conf_commit", "lmhead_workspace_size", "make_model", "spec_verify_accept",
+           "spec_workspace_size", "status_string"]

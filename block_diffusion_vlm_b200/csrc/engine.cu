@@ -1,0 +1,495 @@
+// Decode engine: forward orchestration (PDL-chained kernels, CUDA graphs),
+// prefill and the three decoding drivers.
+//
+//   threshold [Fast-dVLM technical overview (ocdem.com), sections 2.2.1,
+//     2.2.2, 4.1]: per block, position 0 is the AR seed; noisy passes over
+//     the whole block score the still-masked positions (position j from row
+//     j-1) and commit those with top-1 probability >= threshold (at least
+//     one); a causal pass over the finished block then makes its K/V final,
+//     advances L by B and seeds the next block from its last row;
+//   linear self-speculative [same page, section 2.3.1]: one noisy draft pass
+//     commits every position, one causal verify pass scores the draft, the
+//     longest agreeing prefix is kept and L is truncated to it;
+//   AR: one causal row per pass (the comparator).
+#include <cmath>
+#include <cstring>
+
+#include "engine.h"
+#include "ptx.cuh"
+
+using namespace dvlm;
+
+namespace dvlm {
+
+__global__ void advance_kernel(int32_t* d_len, int n) {
+  griddep_launch_dependents();
+  griddep_wait();
+  if (threadIdx.x == 0) *d_len += n;
+}
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  bool dry;
+  template <class T>
+  T* take(size_t bytes) {
+    off = align_up(off, 256);
+    T* p = dry ? nullptr : reinterpret_cast<T*>(base + off);
+    off += bytes;
+    return p;
+  }
+};
+
+static int num_tiles_max(const dvlm_model& m) {
+  const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
+  int t = std::max(qkv_rows / 128, m.hidden / 128);
+  t = std::max(t, m.inter / 64);
+  t = std::max(t, (m.vocab + 127) / 128);
+  return t;
+}
+
+// Lays the workspace out (or measures it when dry).
+static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
+  const dvlm_model& m = e->m;
+  const size_t es = e->bf16 ? 2 : 4;
+  const int H = m.hidden, I = m.inter, HD = m.n_q_heads * m.head_dim;
+  const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
+  Carver c{base, 0, dry};
+  e->x = c.take<void>(kNT * H * es);
+  e->q = c.take<void>(kNT * HD * es);
+  e->attn_o = c.take<void>(kNT * HD * es);
+  e->act = c.take<void>(static_cast<size_t>(kNT) * I * es);
+  e->ssq = c.take<float>((H / 128 + 1) * kNT * 4);
+  e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, P));
+  e->gcnt = c.take<int>(num_tiles_max(m) * 4);
+  e->lpart = c.take<float>(static_cast<size_t>(P) * 2 * kNT * 128 * 4);
+  e->lcnt = c.take<int>(((m.vocab + 127) / 128) * 4);
+  e->lrec = c.take<float>(static_cast<size_t>(2) * P * kNT * 16);
+  e->lvalid = c.take<int>(P * 4);
+  e->ldone = c.take<int>(4);
+  e->d_len = c.take<int32_t>(4);
+  e->d_seed = c.take<int32_t>(4);
+  e->d_status = c.take<int>(4);
+  e->n_remaining = c.take<int32_t>(4);
+  e->n_out = c.take<int32_t>(4);
+  e->tokens = c.take<int32_t>((kNT + 1) * 4);
+  e->vids = c.take<int32_t>((kNT + 1) * 4);
+  e->masked = c.take<uint8_t>(kNT + 1);
+  e->hist = c.take<int64_t>(DVLM_HIST * 8);
+  e->ahist = c.take<int64_t>(DVLM_HIST * 8);
+  e->stage_vis = c.take<void>(static_cast<size_t>(std::max(e->max_ctx, 1)) * H * es);
+  e->stage_ids = c.take<int32_t>(std::max(e->max_ctx, 1) * 4);
+  e->stage_out = c.take<int32_t>(static_cast<size_t>(e->Lmax) * 4);
+  if (!e->bf16) {
+    e->f_y = c.take<float>(static_cast<size_t>(kNT) * std::max(qkv_rows, H) * 4);
+    e->f_r = c.take<float>(kNT * 4);
+    e->f_g = c.take<float>(static_cast<size_t>(kNT) * I * 4);
+    e->f_u = c.take<float>(static_cast<size_t>(kNT) * I * 4);
+    e->f_p1 = c.take<float>(kNT * 4);
+    e->f_id = c.take<int32_t>(kNT * 4);
+  }
+  return align_up(c.off, 256);
+}
+
+static bool build_maps(dvlm_engine* e) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads, L = m.n_layers;
+  const int qkv_rows = (Hq + 2 * Hkv) * D;
+  bool ok = true;
+  ok &= make_tmap_2d(&e->tm_wqkv, m.wqkv, H, static_cast<uint64_t>(L) * qkv_rows, H * 2, 64, 128);
+  ok &= make_tmap_2d(&e->tm_wo, m.wo, Hq * D, static_cast<uint64_t>(L) * H, Hq * D * 2, 64, 128);
+  ok &= make_tmap_2d(&e->tm_wg, m.wgate, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
+  ok &= make_tmap_2d(&e->tm_wu, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
+  ok &= make_tmap_2d(&e->tm_wd, m.wdown, I, static_cast<uint64_t>(L) * H, static_cast<uint64_t>(I) * 2, 64, 128);
+  ok &= make_tmap_2d(&e->tm_lm, m.lm_head, H, m.vocab, H * 2, 64, 128);
+  ok &= make_tmap_2d(&e->tm_x, e->x, H, kNT, H * 2, 64, kNT);
+  ok &= make_tmap_2d(&e->tm_ao, e->attn_o, Hq * D, kNT, Hq * D * 2, 64, kNT);
+  ok &= make_tmap_2d(&e->tm_act, e->act, I, kNT, static_cast<uint64_t>(I) * 2, 64, kNT);
+  ok &= make_tmap_3d(&e->tm_q, e->q, D, Hq, kNT, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
+  ok &= make_tmap_2d(&e->tm_k, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 64);
+  ok &= make_tmap_2d(&e->tm_v, e->vc, e->Lmax, static_cast<uint64_t>(L) * Hkv * D,
+                     static_cast<uint64_t>(e->Lmax) * 2, 64, 128);
+  return ok;
+}
+
+static int ws_ctas(dvlm_engine* e, long long units) {
+  return static_cast<int>(std::min<long long>(e->sm, units));
+}
+
+static void fill_lm_scratch(dvlm_engine* e, LmArgs& a) {
+  a.part = e->lpart;
+  a.cnt = e->lcnt;
+  a.rec = e->lrec;
+  a.split_valid = e->lvalid;
+  a.done = e->ldone;
+  a.status = e->d_status;
+  a.V = e->m.vocab;
+}
+
+#define DVLM_CK(x)                            \
+  do {                                        \
+    cudaError_t err__ = (x);                  \
+    if (err__ != cudaSuccess) return err__;   \
+  } while (0)
+
+static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
+  const int qkv_rows = (Hq + 2 * Hkv) * D;
+  const bool pdl = true;
+  bf16* x = static_cast<bf16*>(e->x);
+  KernelTimer* tm = f.timer;
+  auto T0 = [&](int k) { if (tm) tm->begin(k); };
+  auto T1 = [&](int k) { if (tm) tm->end(k); };
+  T0(K_EMBED);
+  DVLM_CK(launch_embed_bf16(static_cast<const bf16*>(m.embed), static_cast<const bf16*>(f.rows_in), f.n_src,
+                            f.tokens, f.masked, m.mask_id, f.n_rows, H, m.vocab, x, e->ssq, kNT, e->d_status, pdl,
+                            s));
+  T1(K_EMBED);
+  const int l1 = f.n_layers < 0 ? m.n_layers : f.layer0 + f.n_layers;
+  GemmEpi ea{};
+  ea.n_rows = f.n_rows;
+  ea.ssq_in = e->ssq;
+  ea.n_ssq = H / 128;
+  ea.inv_h = 1.0f / H;
+  ea.eps = m.eps;
+  ea.Lmax = e->Lmax;
+  ea.n_q_heads = Hq;
+  ea.n_kv_heads = Hkv;
+  ea.d_len = e->d_len;
+  ea.log2_rope_base = std::log2(static_cast<double>(m.rope_base));
+  ea.part = e->gpart;
+  ea.cnt = e->gcnt;
+  ea.status = e->d_status;
+  const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
+  for (int l = f.layer0; l < l1; ++l) {
+    ea.epi = EPI_QKV;
+    ea.out = static_cast<bf16*>(e->q);
+    ea.out_ld = Hq * D;
+    ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
+    ea.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
+    T0(K_QKV);
+    DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
+                           ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s));
+    T1(K_QKV);
+    AttnArgs aa{};
+    aa.n_rows = f.n_rows;
+    aa.n_clean = f.n_clean;
+    aa.n_batch = 1;
+    aa.d_len = e->d_len;
+    aa.Lmax = e->Lmax;
+    aa.Hq = Hq;
+    aa.Hkv = Hkv;
+    aa.kv_base = l;
+    aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    aa.out = static_cast<bf16*>(e->attn_o);
+    aa.status = e->d_status;
+    T0(K_ATTN);
+    DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s));
+    T1(K_ATTN);
+    ea.epi = EPI_RESID;
+    ea.resid = x;
+    ea.resid_ld = H;
+    ea.ssq_out = e->ssq;
+    T0(K_OPROJ);
+    DVLM_CK(launch_gemm_ws(kNT, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64,
+                           ws_ctas(e, (H / 128) * (Hq * D / 64)), l * H, ea, pdl, s));
+    T1(K_OPROJ);
+    ea.epi = EPI_SWIGLU;
+    ea.out = static_cast<bf16*>(e->act);
+    ea.out_ld = I;
+    T0(K_GATEUP);
+    DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, ws_ctas(e, (I / 64) * (H / 64)),
+                           l * I, ea, pdl, s));
+    T1(K_GATEUP);
+    ea.epi = EPI_RESID;
+    T0(K_DOWN);
+    DVLM_CK(launch_gemm_ws(kNT, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, ws_ctas(e, (H / 128) * (I / 64)),
+                           l * H, ea, pdl, s));
+    T1(K_DOWN);
+  }
+  if (f.x_out) DVLM_CK(cudaMemcpyAsync(f.x_out, x, static_cast<size_t>(f.n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
+  if (f.lm) {
+    LmArgs a = f.lma;
+    fill_lm_scratch(e, a);
+    a.ssq_in = e->ssq;
+    a.n_ssq = H / 128;
+    a.inv_h = 1.0f / H;
+    a.eps = m.eps;
+    const int nt = (m.vocab + 127) / 128;
+    T0(K_LMHEAD);
+    DVLM_CK(launch_lmhead(kNT, e->tm_lm, e->tm_x, nt, H / 64, ws_ctas(e, static_cast<long long>(nt) * (H / 64)), a,
+                          pdl, s));
+    T1(K_LMHEAD);
+  } else if (f.advance) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    DVLM_CK(cudaLaunchKernelEx(&cfg, advance_kernel, e->d_len, f.n_rows));
+  }
+  return cudaSuccess;
+}
+
+static cudaError_t fwd_f32(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
+  const int qkv_rows = (Hq + 2 * Hkv) * D;
+  const int n = f.n_rows;
+  float* x = static_cast<float*>(e->x);
+  float* q = static_cast<float*>(e->q);
+  float* ao = static_cast<float*>(e->attn_o);
+  float* act = static_cast<float*>(e->act);
+  const float* wqkv = static_cast<const float*>(m.wqkv);
+  const float* wo = static_cast<const float*>(m.wo);
+  const float* wg = static_cast<const float*>(m.wgate);
+  const float* wu = static_cast<const float*>(m.wup);
+  const float* wd = static_cast<const float*>(m.wdown);
+  DVLM_CK(f32_embed(static_cast<const float*>(m.embed), static_cast<const float*>(f.rows_in), f.n_src, f.tokens,
+                    f.masked, m.mask_id, n, H, m.vocab, x, e->d_status, s));
+  const int l1 = f.n_layers < 0 ? m.n_layers : f.layer0 + f.n_layers;
+  const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
+  const double lb = std::log2(static_cast<double>(m.rope_base));
+  for (int l = f.layer0; l < l1; ++l) {
+    float* kc = static_cast<float*>(e->kc) + l * kv_layer;
+    float* vc = static_cast<float*>(e->vc) + l * kv_layer;
+    DVLM_CK(f32_rowscale(x, H, n, H, m.eps, e->f_r, s));
+    DVLM_CK(f32_gemm(x, H, wqkv + static_cast<size_t>(l) * qkv_rows * H, qkv_rows, H, n, e->f_r, e->f_y, qkv_rows, s));
+    DVLM_CK(f32_rope_scatter(e->f_y, n, Hq, Hkv, D, e->d_len, 0, lb, q, kc, vc, e->Lmax, s));
+    DVLM_CK(f32_attention(q, ao, kc, vc, 1, n, f.n_clean, 0, e->d_len, e->Lmax, Hq, Hkv, D,
+                          static_cast<float>(1.0 / std::sqrt(static_cast<double>(D))), s));
+    DVLM_CK(f32_gemm(ao, Hq * D, wo + static_cast<size_t>(l) * H * Hq * D, H, Hq * D, n, nullptr, e->f_y, H, s));
+    DVLM_CK(f32_add(x, H, e->f_y, H, n, H, s));
+    DVLM_CK(f32_rowscale(x, H, n, H, m.eps, e->f_r, s));
+    DVLM_CK(f32_gemm(x, H, wg + static_cast<size_t>(l) * I * H, I, H, n, e->f_r, e->f_g, I, s));
+    DVLM_CK(f32_gemm(x, H, wu + static_cast<size_t>(l) * I * H, I, H, n, e->f_r, e->f_u, I, s));
+    DVLM_CK(f32_swiglu(e->f_g, e->f_u, act, n * I, s));
+    DVLM_CK(f32_gemm(act, I, wd + static_cast<size_t>(l) * H * I, H, I, n, nullptr, e->f_y, H, s));
+    DVLM_CK(f32_add(x, H, e->f_y, H, n, H, s));
+  }
+  if (f.x_out) DVLM_CK(cudaMemcpyAsync(f.x_out, x, static_cast<size_t>(n) * H * 4, cudaMemcpyDeviceToDevice, s));
+  if (f.lm) {
+    LmArgs a = f.lma;
+    fill_lm_scratch(e, a);
+    DVLM_CK(f32_rowscale(x, H, n, H, m.eps, e->f_r, s));
+    DVLM_CK(f32_lmhead(x, static_cast<const float*>(m.lm_head), a.R, H, m.vocab, e->f_r, e->f_p1, e->f_id, a, s));
+  } else if (f.advance) {
+    advance_kernel<<<1, 32, 0, s>>>(e->d_len, n);
+    DVLM_CK(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+cudaError_t engine_forward(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
+  return e->bf16 ? fwd_bf16(e, f, s) : fwd_f32(e, f, s);
+}
+
+// Replays the captured graph for `key`, capturing `body` on first use.
+template <class F>
+static cudaError_t run_graph(dvlm_engine* e, const std::vector<long long>& key, bool use_graphs, cudaStream_t s,
+                             F&& body) {
+  if (!use_graphs || s == nullptr) return body();
+  auto it = e->graphs.find(key);
+  if (it == e->graphs.end()) {
+    DVLM_CK(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+    const cudaError_t berr = body();
+    cudaGraph_t g = nullptr;
+    const cudaError_t cerr = cudaStreamEndCapture(s, &g);
+    if (berr != cudaSuccess || cerr != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      return berr != cudaSuccess ? berr : cerr;
+    }
+    cudaGraphExec_t ex = nullptr;
+    const cudaError_t ierr = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    DVLM_CK(ierr);
+    it = e->graphs.emplace(key, ex).first;
+  }
+  return cudaGraphLaunch(it->second, s);
+}
+
+static long long fbits(float v) {
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  return u;
+}
+
+enum { G_NOISY = 1, G_APPEND, G_DRAFT, G_VERIFY, G_AR };
+
+// One block (threshold / AR) or one round (spec).  Tokens are emitted into
+// stage_out at n_out (capped at max_new).  Returns the number of tokens this
+// step emitted, via *emitted (host).
+cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new, int n_out_host, int* emitted,
+                        dvlm_stats* st, cudaStream_t s) {
+  const int B = cfg.block_size;
+  const bool ug = cfg.use_graphs != 0;
+  if (cfg.mode == DVLM_MODE_AR) {
+    DVLM_CK(run_graph(e, {G_AR, max_new}, ug, s, [&]() -> cudaError_t {
+      FwdSpec f;
+      f.tokens = e->d_seed;
+      f.n_rows = 1;
+      f.n_clean = 1;
+      f.lm = true;
+      f.lma.R = 1;
+      f.lma.threshold = -1.0f;
+      f.lma.seed_out = e->d_seed;
+      f.lma.seed_row = 0;
+      f.lma.len_ptr = e->d_len;
+      f.lma.len_advance = 1;
+      // emit the token being fed before the LM head overwrites the seed
+      DVLM_CK(launch_emit(e->d_seed, 1, e->stage_out, e->n_out, max_new, false, s));
+      return engine_forward(e, f, s);
+    }));
+    if (st) {
+      st->nfe += 1;
+      st->n_rounds += 1;
+      st->n_launches += launches_per_forward(e->m.n_layers) + 1;
+    }
+    *emitted = std::min(1, max_new - n_out_host);
+    return cudaSuccess;
+  }
+  DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, e->m.mask_id, 1, e->n_remaining, s));
+  if (cfg.mode == DVLM_MODE_THRESHOLD) {
+    int rem = B - 1;
+    while (rem > 0) {
+      DVLM_CK(run_graph(e, {G_NOISY, B, fbits(cfg.threshold)}, ug, s, [&]() -> cudaError_t {
+        FwdSpec f;
+        f.tokens = e->tokens;
+        f.masked = e->masked;
+        f.n_rows = B;
+        f.n_clean = 0;
+        f.lm = true;
+        // position j is scored by row j-1: rows 0..B-2 commit into positions 1..B-1
+        f.lma.R = B - 1;
+        f.lma.masked = e->masked + 1;
+        f.lma.tokens = e->tokens + 1;
+        f.lma.threshold = cfg.threshold;
+        f.lma.n_remaining = e->n_remaining;
+        f.lma.hist = e->hist;
+        return engine_forward(e, f, s);
+      }));
+      int32_t h = 0;
+      DVLM_CK(cudaMemcpyAsync(&h, e->n_remaining, 4, cudaMemcpyDeviceToHost, s));
+      DVLM_CK(cudaStreamSynchronize(s));
+      rem = h;
+      if (st) {
+        st->nfe += 1;
+        st->n_iters += 1;
+        st->n_launches += launches_per_forward(e->m.n_layers);
+      }
+    }
+    DVLM_CK(run_graph(e, {G_APPEND, B, max_new}, ug, s, [&]() -> cudaError_t {
+      FwdSpec f;
+      f.tokens = e->tokens;
+      f.n_rows = B;
+      f.n_clean = B;
+      f.lm = true;
+      f.lma.R = B;
+      f.lma.threshold = -1.0f;
+      f.lma.seed_out = e->d_seed;
+      f.lma.seed_row = B - 1;
+      f.lma.len_ptr = e->d_len;
+      f.lma.len_advance = B;
+      DVLM_CK(engine_forward(e, f, s));
+      return launch_emit(e->tokens, B, e->stage_out, e->n_out, max_new, true, s);
+    }));
+    if (st) {
+      st->nfe += 1;
+      st->n_rounds += 1;
+      st->n_launches += launches_per_forward(e->m.n_layers) + 2;  // + block init + emit
+    }
+    *emitted = std::min(B, max_new - n_out_host);
+    return cudaSuccess;
+  }
+  // linear self-speculative round
+  DVLM_CK(run_graph(e, {G_DRAFT, B}, ug, s, [&]() -> cudaError_t {
+    FwdSpec f;
+    f.tokens = e->tokens;
+    f.masked = e->masked;
+    f.n_rows = B;
+    f.n_clean = 0;
+    f.lm = B > 1;
+    f.lma.R = B - 1;
+    f.lma.masked = e->masked + 1;
+    f.lma.tokens = e->tokens + 1;
+    f.lma.threshold = -1.0f;  // the draft takes every position's argmax
+    return engine_forward(e, f, s);
+  }));
+  DVLM_CK(run_graph(e, {G_VERIFY, B, max_new}, ug, s, [&]() -> cudaError_t {
+    FwdSpec f;
+    f.tokens = e->tokens;
+    f.n_rows = B;
+    f.n_clean = B;
+    f.lm = true;
+    f.lma.R = B;
+    f.lma.threshold = -1.0f;
+    f.lma.id_out = e->vids + 1;  // row j predicts position j+1
+    f.lma.len_ptr = e->d_len;
+    f.lma.len_advance = B;
+    DVLM_CK(engine_forward(e, f, s));
+    return launch_decode_accept(e->vids, e->tokens, B, e->d_len, e->d_seed, e->stage_out, e->n_out, max_new,
+                                e->ahist, e->d_status, true, s);
+  }));
+  int32_t h = 0;
+  DVLM_CK(cudaMemcpyAsync(&h, e->n_out, 4, cudaMemcpyDeviceToHost, s));
+  DVLM_CK(cudaStreamSynchronize(s));
+  if (st) {
+    st->nfe += 2;
+    st->n_rounds += 1;
+    st->n_launches += 2 + (B > 1 ? 2 : 1) * launches_per_forward(e->m.n_layers);  // + block init + accept
+  }
+  *emitted = h - n_out_host;
+  return cudaSuccess;
+}
+
+cudaError_t engine_collect_stats(dvlm_engine* e, dvlm_stats* st, cudaStream_t s) {
+  int64_t h[2 * DVLM_HIST];
+  DVLM_CK(cudaMemcpyAsync(h, e->hist, DVLM_HIST * 8, cudaMemcpyDeviceToHost, s));
+  DVLM_CK(cudaMemcpyAsync(h + DVLM_HIST, e->ahist, DVLM_HIST * 8, cudaMemcpyDeviceToHost, s));
+  DVLM_CK(cudaStreamSynchronize(s));
+  if (st) {
+    for (int i = 0; i < DVLM_HIST; ++i) {
+      st->commit_hist[i] += h[i];
+      st->accept_hist[i] += h[DVLM_HIST + i];
+    }
+  }
+  DVLM_CK(cudaMemsetAsync(e->hist, 0, DVLM_HIST * 8, s));
+  return cudaMemsetAsync(e->ahist, 0, DVLM_HIST * 8, s);
+}
+
+// One eager forward with CUDA events around every kernel: per-kind device
+// time (ms, summed over layers) and launch counts.
+cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* counts, cudaStream_t s) {
+  KernelTimer tm;
+  tm.s = s;
+  FwdSpec f = f0;
+  f.timer = &tm;
+  cudaError_t err = engine_forward(e, f, s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  for (int k = 0; k < K_KINDS; ++k) {
+    ms[k] = 0.f;
+    counts[k] = 0;
+  }
+  for (auto& mk : tm.marks) {
+    float t = 0.f;
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&t, mk.second.first, mk.second.second);
+    ms[mk.first] += t;
+    counts[mk.first] += 1;
+    cudaEventDestroy(mk.second.first);
+    cudaEventDestroy(mk.second.second);
+  }
+  return err;
+}
+
+size_t engine_workspace_bytes(dvlm_engine* e, int P) { return carve(e, nullptr, true, P); }
+size_t engine_carve(dvlm_engine* e, void* ws, int P) { return carve(e, static_cast<uint8_t*>(ws), false, P); }
+bool engine_build_maps(dvlm_engine* e) { return build_maps(e); }
+
+}  // namespace dvlm

@@ -1,0 +1,152 @@
+// Internal launch interface between the C-ABI/engine layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dvlm.h"
+
+namespace dvlm {
+
+using bf16 = __nv_bfloat16;
+
+enum EpiKind { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
+
+// Fused-epilogue operands of the decoder GEMMs.
+struct GemmEpi {
+  int epi;
+  int n_rows;                 // valid token rows (<= NT)
+  // RMSNorm factor of the input rows, from per-128-feature sums of squares
+  const float* ssq_in;        // [n_ssq][NT]
+  int n_ssq;
+  float inv_h, eps;
+  // EPI_QKV: q [rows][Hq*D]; EPI_SWIGLU: act [rows][I]
+  bf16* out;
+  int out_ld;
+  // EPI_RESID: residual stream [rows][H] updated in place, ssq_out [n_tiles][NT]
+  bf16* resid;
+  int resid_ld;
+  float* ssq_out;
+  // EPI_QKV: KV cache of this layer; K [Hkv][Lmax][D], V^T [Hkv][D][Lmax]
+  bf16* kcache;
+  bf16* vcache;
+  int Lmax, n_q_heads, n_kv_heads;
+  const int* d_len;           // slot of row 0 (device); NULL -> L_static
+  int L_static;
+  double log2_rope_base;
+  // split-tile scratch: part [P][2][NT][128] fp32, cnt [n_tiles] int (zero)
+  float* part;
+  int* cnt;
+  int* status;
+};
+
+// Fused LM head operands.
+struct LmArgs {
+  int R;                     // rows to report/commit (<= NT)
+  int V;
+  const float* ssq_in;       // final RMSNorm sums of squares [n_ssq][NT] or NULL
+  int n_ssq;
+  float inv_h, eps;
+  // scratch
+  float* part;               // [P][2][NT][128]
+  int* cnt;                  // [n_tiles]
+  float* rec;                // [2][P][NT][4]: per-CTA and per-split-tile (m, s, idx)
+  int* split_valid;          // [P]
+  int* done;                 // [1]
+  // commit / outputs
+  uint8_t* masked;
+  int32_t* tokens;
+  float threshold;
+  int32_t* top1_id;
+  float* top1_prob;
+  uint8_t* commit;
+  int32_t* n_commit;
+  const int32_t* anchor_id;
+  const float* anchor_conf;
+  int32_t* cert_len;
+  int32_t* n_remaining;      // masked rows left after the commit
+  int32_t* len_ptr;          // *len_ptr += len_advance at the end (may be NULL)
+  int len_advance;
+  int32_t* seed_out;         // *seed_out = top1_id[seed_row] (may be NULL)
+  int seed_row;
+  int32_t* id_out;           // id_out[r] = top1_id[r] for r < R (may be NULL)
+  int64_t* hist;             // commit histogram (may be NULL)
+  int64_t* nfe;              // +1 per call (may be NULL)
+  int* status;
+};
+
+struct Launch {
+  int sm_count;
+  bool pdl;
+};
+
+int device_sm_count();
+cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
+                           int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s);
+size_t gemm_ws_part_bytes(int NT, int P);
+cudaError_t launch_lmhead(int NT, const CUtensorMap& mapW, const CUtensorMap& mapH, int n_tiles, int kb, int P,
+                          const LmArgs& a, bool pdl, cudaStream_t s);
+size_t lmhead_scratch_bytes(int NT, int P, int n_tiles);
+
+// Attention over the KV cache (bf16 tcgen05 path).
+struct AttnArgs {
+  int n_rows, n_clean, n_batch;
+  int L_static;
+  const int* d_len;
+  int Lmax, Hq, Hkv;
+  int kv_base;               // cache entry of batch 0 (the layer, in the engine)
+  float scale_log2;          // scale * log2(e)
+  bf16* out;                 // [n_batch][n_rows][Hq][128]
+  int* status;
+};
+cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                             const AttnArgs& a, bool pdl, cudaStream_t s);
+
+// Embedding gather / row copy + per-128-feature sums of squares.
+cudaError_t launch_embed_bf16(const bf16* E, const bf16* rows_in, int n_src, const int32_t* tokens,
+                              const uint8_t* masked, int mask_id, int n_rows, int H, int V, bf16* x,
+                              float* ssq_out, int NT, int* status, bool pdl, cudaStream_t s);
+
+// Speculative accept.
+cudaError_t launch_spec_logits(const bf16* logits, const int32_t* draft, int b, int B, int V, int32_t* accept_len,
+                               int32_t* cache_len, int poison, bf16* kc, bf16* vc, int n_layers, int Hkv, int D,
+                               int Lmax, float* ws_part, int* ws_cnt, int splits, int* status, cudaStream_t s);
+cudaError_t launch_spec_ids(const int32_t* vids, const int32_t* draft, int b, int B, int32_t* accept_len,
+                            int32_t* cache_len, int poison, bf16* kc, bf16* vc, int n_layers, int Hkv, int D,
+                            int Lmax, int* status, cudaStream_t s);
+// Decode-driver accept: k over (verify ids, draft), L = L - B + k, seed, emit.
+cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len,
+                                 int32_t* seed, int32_t* out, int32_t* n_out, int max_new, int64_t* accept_hist,
+                                 int* status, bool pdl, cudaStream_t s);
+// Block bookkeeping for the decode driver.
+cudaError_t launch_block_init(int32_t* tokens, uint8_t* masked, const int32_t* seed, int B, int mask_id,
+                              int ar_seed, int32_t* n_remaining, cudaStream_t s);
+cudaError_t launch_emit(const int32_t* tokens, int n, int32_t* out, int32_t* n_out, int max_new,
+                        bool pdl, cudaStream_t s);
+
+// fp32 CUDA-core path (tiny fp32 model).
+cudaError_t f32_embed(const float* E, const float* rows_in, int n_src, const int32_t* tokens,
+                      const uint8_t* masked, int mask_id, int n_rows, int H, int V, float* x, int* status,
+                      cudaStream_t s);
+cudaError_t f32_rowscale(const float* x, int ld, int n_rows, int H, float eps, float* r, cudaStream_t s);
+cudaError_t f32_gemm(const float* x, int ld_x, const float* W, int n_out, int K, int n_rows, const float* r,
+                     float* y, int ld_y, cudaStream_t s);
+cudaError_t f32_rope_scatter(const float* y, int n_rows, int nq, int nkv, int D, const int* d_len, int L_static,
+                             double log2_base, float* q_out, float* kc, float* vc, int Lmax, cudaStream_t s);
+cudaError_t f32_add(float* resid, int ld_r, const float* y, int ld_y, int n_rows, int H, cudaStream_t s);
+cudaError_t f32_swiglu(const float* g, const float* u, float* act, int n, cudaStream_t s);
+cudaError_t f32_attention(const float* q, float* out, const float* kc, const float* vc, int n_batch, int n_rows,
+                          int n_clean, int L, const int* d_len, int Lmax, int Hq, int Hkv, int D, float scale,
+                          cudaStream_t s);
+cudaError_t f32_lmhead(const float* hidden, const float* w, int R, int H, int V, const float* r, float* p1_buf,
+                       int32_t* id_buf, const LmArgs& a, cudaStream_t s);
+
+// Tensor maps (host).
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+                  uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+
+}  // namespace dvlm

@@ -1,0 +1,309 @@
+// Fused LM head + top-1 confidence + argmax + threshold commit (+ certificate).
+//
+// logits[v, t] = s_t * sum_k W[v, k] h[t, k] are produced 128 vocabulary rows
+// at a time in TMEM by tcgen05 UMMAs (W streamed once from HBM through TMA)
+// and folded straight into a running (max m, sum of exp(l - m), argmax) per
+// token; logits never reach memory.  p1 = 1 / sum exp(l - max) is the top-1
+// softmax probability [Look Only When Needed, method step (1)]; the argmax is
+// the lowest id among equal maxima.  The last CTA to finish merges all
+// per-CTA records in CTA order (deterministic) and applies the commit rule.
+#include "finalize.cuh"
+#include "mainloop.cuh"
+
+namespace dvlm {
+
+template <int NT>
+struct LmCfg {
+  static constexpr int STAGES = NT <= 32 ? (NT <= 16 ? 5 : 4) : (NT <= 64 ? 4 : 4);
+  static constexpr int TPT = 128 / NT;     // scan threads per token
+  static constexpr int SROW = 128 + TPT;   // padded row of the transposed tile (bank-conflict free)
+  static constexpr int kA = 0;
+  static constexpr int kB = kA + STAGES * kATileBytes;
+  static constexpr int kT = kB + STAGES * NT * 128;
+  static constexpr int kRec = kT + NT * SROW * 4;
+  static constexpr int kFin = kRec + 128 * 16;
+  static constexpr int kBar = kFin + ((static_cast<int>(sizeof(FinalizeSmem)) + 15) / 16) * 16;
+  static constexpr int kMisc = kBar + (2 * STAGES + 4) * 8;
+  static constexpr int kTotal = kMisc + 64 + 1024;
+};
+
+struct Stat {
+  float m, s;
+  int idx;
+};
+
+__device__ __forceinline__ void stat_push(Stat& st, float l, int v) {
+  if (l > st.m) {
+    st.s = st.s * expf(st.m - l) + 1.0f;
+    st.m = l;
+    st.idx = v;
+  } else {
+    st.s += expf(l - st.m);
+  }
+}
+// (m1,s1,i1) <- (m1,s1,i1) (+) (m2,s2,i2); empty records have s == 0.
+__device__ __forceinline__ void stat_merge(Stat& a, const Stat& b) {
+  if (b.s == 0.0f) return;
+  if (a.s == 0.0f) {
+    a = b;
+    return;
+  }
+  if (b.m > a.m) {
+    a.s = a.s * expf(a.m - b.m) + b.s;
+    a.m = b.m;
+    a.idx = b.idx;
+  } else if (b.m == a.m) {
+    a.s += b.s;
+    a.idx = b.idx < a.idx ? b.idx : a.idx;
+  } else {
+    a.s += b.s * expf(b.m - a.m);
+  }
+}
+
+template <int NT, int STAGES>
+__global__ void __launch_bounds__(kWsThreads, 1)
+    lmhead_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapH,
+                  const SkSched sc, const LmArgs a) {
+  using C = LmCfg<NT>;
+  constexpr int TMC = tmem_cols_for<NT>();
+  constexpr int TPT = C::TPT, SROW = C::SROW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem + C::kA;
+  uint8_t* sB = smem + C::kB;
+  float* sT = reinterpret_cast<float*>(smem + C::kT);  // [NT][SROW] logits, token-major
+  float4* sRec = reinterpret_cast<float4*>(smem + C::kRec);
+  FinalizeSmem& fs = *reinterpret_cast<FinalizeSmem*>(smem + C::kFin);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  int* sflag = reinterpret_cast<int*>(smem + C::kMisc + 4);
+  volatile int* sabort = reinterpret_cast<volatile int*>(smem + C::kMisc + 8);
+  int* slast = reinterpret_cast<int*>(smem + C::kMisc + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = sc.P;
+  const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    *sabort = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mapW);
+    tma_prefetch_map(&mapH);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMC);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0 && u1 > u0)
+      ws_producer<NT, STAGES, false>(&mapW, &mapW, &mapH, sA, sB, full, empty, sc, u0, u1, 0, 0, a.status, sabort);
+  } else if (warp == 1) {
+    if (lane == 0 && u1 > u0) ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, a.status, sabort);
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;
+    const int tok = et / TPT, sub = et % TPT;
+    auto bar = [] { named_bar_sync(1, 128); };
+    griddep_wait();
+    float rt = 1.0f;  // final RMSNorm factor of this thread's token
+    if (a.ssq_in) {
+      float s = 0.f;
+      for (int p = 0; p < a.n_ssq; ++p) s += a.ssq_in[p * NT + tok];
+      rt = 1.0f / sqrtf(s * a.inv_h + a.eps);
+    }
+    Stat run{-INFINITY, 0.0f, 0x7fffffff};
+    auto scan = [&](int T, Stat& st) {
+#pragma unroll 4
+      for (int i = 0; i < NT; ++i) {
+        const int r = sub + TPT * i;
+        const int v = T * 128 + r;
+        if (v < a.V) stat_push(st, sT[tok * SROW + r] * rt, v);
+      }
+    };
+    // Combine the TPT per-thread records of each token in sub order.
+    auto combine = [&](Stat st) -> Stat {
+      sRec[et] = make_float4(st.m, st.s, __int_as_float(st.idx), 0.f);
+      bar();
+      Stat out{-INFINITY, 0.0f, 0x7fffffff};
+      if (sub == 0) {
+        for (int k = 0; k < TPT; ++k) {
+          const float4 f = sRec[tok * TPT + k];
+          stat_merge(out, Stat{f.x, f.y, __float_as_int(f.z)});
+        }
+      }
+      bar();
+      return out;
+    };
+    const int first_tile = sc.first_tile(blockIdx.x);
+    int seg = 0;
+    bool ok = true;
+    for (long long u = u0; u < u1; ++seg) {
+      const int T = static_cast<int>(u / sc.kb);
+      const long long t_begin = static_cast<long long>(T) * sc.kb, t_end = t_begin + sc.kb;
+      const long long seg_end = t_end < u1 ? t_end : u1;
+      const int b = seg & 1;
+      mbar_wait(&accf[b], (seg >> 1) & 1, a.status, sabort);
+      bar();
+      if (*sabort) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < NT; c += 16) {
+        float tmp[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * NT + c), tmp);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) sT[(c + k) * SROW + row] = tmp[k];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
+      bar();
+      const bool whole = (u == t_begin) && (seg_end == t_end);
+      if (whole) {
+        scan(T, run);
+      } else {
+        const int slot = (T == first_tile) ? 0 : 1;
+        float* mine = a.part + (static_cast<size_t>(blockIdx.x) * 2 + slot) * NT * 128;
+        for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + et], sT[t * SROW + et]);
+        __threadfence();
+        bar();
+        const int pf = sc.cta_of(t_begin), pl = sc.cta_of(t_end - 1);
+        if (et == 0) {
+          const int old = atomicAdd(&a.cnt[T], 1);
+          *sflag = (old == pl - pf) ? 1 : 0;
+        }
+        bar();
+        if (*sflag) {
+          __threadfence();
+          for (int t = 0; t < NT; ++t) {
+            float acc = 0.f;
+            for (int p = pf; p <= pl; ++p) {
+              const int sp = (T == sc.first_tile(p)) ? 0 : 1;
+              acc += __ldcg(&a.part[((static_cast<size_t>(p) * 2 + sp) * NT + t) * 128 + et]);
+            }
+            sT[t * SROW + et] = acc;
+          }
+          if (et == 0) a.cnt[T] = 0;
+          bar();
+          Stat st{-INFINITY, 0.0f, 0x7fffffff};
+          scan(T, st);
+          const Stat tile_rec = combine(st);
+          if (sub == 0) {
+            float4* dst = reinterpret_cast<float4*>(a.rec) + (static_cast<size_t>(P) + pf) * NT + tok;
+            __stcg(dst, make_float4(tile_rec.m, tile_rec.s, __int_as_float(tile_rec.idx), 0.f));
+          }
+          if (et == 0) a.split_valid[pf] = 1;
+        }
+      }
+      bar();  // sT is rewritten by the next segment
+      u = seg_end;
+    }
+    if (ok) {
+      const Stat mine = combine(run);
+      if (sub == 0) {
+        float4* dst = reinterpret_cast<float4*>(a.rec) + static_cast<size_t>(blockIdx.x) * NT + tok;
+        __stcg(dst, make_float4(mine.m, mine.s, __int_as_float(mine.idx), 0.f));
+      }
+      __threadfence();
+      bar();
+      if (et == 0) {
+        const int old = atomicAdd(a.done, 1);
+        *slast = (old == P - 1) ? 1 : 0;
+      }
+      bar();
+      if (*slast) {
+        __threadfence();
+        Stat st{-INFINITY, 0.0f, 0x7fffffff};
+        const float4* rec = reinterpret_cast<const float4*>(a.rec);
+        for (int p = sub; p < P; p += TPT) {
+          float4 f = __ldcg(&rec[static_cast<size_t>(p) * NT + tok]);
+          stat_merge(st, Stat{f.x, f.y, __float_as_int(f.z)});
+          if (__ldcg(&a.split_valid[p])) {
+            f = __ldcg(&rec[(static_cast<size_t>(P) + p) * NT + tok]);
+            stat_merge(st, Stat{f.x, f.y, __float_as_int(f.z)});
+          }
+        }
+        const Stat fin = combine(st);
+        if (sub == 0 && tok < 128) {
+          fs.p1[tok] = fin.s > 0.f ? 1.0f / fin.s : 0.0f;
+          fs.id[tok] = fin.idx;
+        }
+        bar();
+        for (int p = et; p < P; p += 128) a.split_valid[p] = 0;
+        if (et == 0) *a.done = 0;
+        finalize_rows(et, a, fs, bar);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMC);
+  }
+}
+
+size_t lmhead_scratch_bytes(int NT, int P, int n_tiles) {
+  size_t part = static_cast<size_t>(P) * 2 * NT * 128 * 4;
+  size_t rec = static_cast<size_t>(2) * P * NT * 16;
+  size_t ints = (static_cast<size_t>(n_tiles) + P + 1) * 4;
+  return part + rec + ints + 256;
+}
+
+template <int NT>
+static cudaError_t lm_launch(const CUtensorMap& mapW, const CUtensorMap& mapH, const SkSched& sc, const LmArgs& a,
+                             bool pdl, cudaStream_t s) {
+  using C = LmCfg<NT>;
+  auto kern = lmhead_kernel<NT, C::STAGES>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sc.P);
+  cfg.blockDim = dim3(kWsThreads);
+  cfg.dynamicSmemBytes = C::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mapW, mapH, sc, a);
+}
+
+cudaError_t launch_lmhead(int NT, const CUtensorMap& mapW, const CUtensorMap& mapH, int n_tiles, int kb, int P,
+                          const LmArgs& a, bool pdl, cudaStream_t s) {
+  SkSched sc{n_tiles, kb, P};
+  switch (NT) {
+    case 16: return lm_launch<16>(mapW, mapH, sc, a, pdl, s);
+    case 32: return lm_launch<32>(mapW, mapH, sc, a, pdl, s);
+    case 64: return lm_launch<64>(mapW, mapH, sc, a, pdl, s);
+    case 128: return lm_launch<128>(mapW, mapH, sc, a, pdl, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dvlm

@@ -1,0 +1,132 @@
+// Weight-streaming mainloop shared by the decoder GEMMs and the fused LM head.
+//
+// Batch-1 decoding re-reads every weight once per forward while only 16 token
+// rows flow through it, so these products are bound by HBM, not by the tensor
+// cores.  The layout is "swap-AB": the weight tile (128 output features x 64
+// k) is the 128-row UMMA A operand, the token rows (NT = 16..128) are the
+// N side, and the fp32 accumulator lives in TMEM (128 lanes x NT columns).
+//
+// Work split: the (output tile, 64-wide k block) units are cut into P equal
+// contiguous ranges, one per CTA (stream-K).  A tile whose k range spans two
+// or more CTAs is finished by whichever contributor arrives last (per-tile
+// counter, no spinning), summing the partial tiles in a fixed order so the
+// result is deterministic.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
+// UMMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+#pragma once
+#include "ptx.cuh"
+
+namespace dvlm {
+
+struct SkSched {
+  int n_tiles;  // output tiles of 128 rows
+  int kb;       // 64-wide k blocks per tile
+  int P;        // CTAs
+  __host__ __device__ long long units() const { return static_cast<long long>(n_tiles) * kb; }
+  __host__ __device__ long long begin(int p) const { return units() * p / P; }
+  // CTA whose range holds unit u (largest p with begin(p) <= u).
+  __host__ __device__ int cta_of(long long u) const { return static_cast<int>(((u + 1) * P - 1) / units()); }
+  __host__ __device__ int first_tile(int p) const { return static_cast<int>(begin(p) / kb); }
+};
+
+constexpr int kWsThreads = 192;
+constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
+
+template <int NT>
+__host__ __device__ constexpr int tmem_cols_for() {
+  return (2 * NT < 32) ? 32 : 2 * NT;
+}
+
+// A operand source: one 128-row box, or two 64-row boxes from two tensors
+// (gate rows on top, up rows below) so the SwiGLU epilogue sees matching
+// gate/up features in one tile.
+template <int NT, int STAGES, bool SPLIT_A>
+__device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUtensorMap* mapA2,
+                                            const CUtensorMap* mapB, uint8_t* sA, uint8_t* sB, uint64_t* full,
+                                            uint64_t* empty, const SkSched& sc, long long u0, long long u1,
+                                            int a_row_base, int b_row, int* status, volatile int* abort_flag) {
+  constexpr int B_BYTES = NT * 128;
+  const uint64_t pol_w = l2_policy_evict_first();
+  const uint64_t pol_x = l2_policy_evict_last();
+  const int n = static_cast<int>(u1 - u0);
+  const int pre = n < STAGES ? n : STAGES;
+  auto load_a = [&](int s, long long u) {
+    const int T = static_cast<int>(u / sc.kb), kk = static_cast<int>(u % sc.kb);
+    if (SPLIT_A) {
+      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * 64, a_row_base + T * 64, pol_w);
+      tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, mapA2, &full[s], kk * 64, a_row_base + T * 64, pol_w);
+    } else {
+      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * 64, a_row_base + T * 128, pol_w);
+    }
+  };
+  auto load_b = [&](int s, long long u) {
+    const int kk = static_cast<int>(u % sc.kb);
+    tma_load_2d(sB + s * B_BYTES, mapB, &full[s], kk * 64, b_row, pol_x);
+  };
+  // Weights do not depend on the previous kernel: start streaming them before
+  // waiting for it (programmatic dependent launch).
+  for (int i = 0; i < pre; ++i) {
+    mbar_arrive_expect_tx(&full[i], kATileBytes + B_BYTES);
+    load_a(i, u0 + i);
+  }
+  griddep_wait();
+  for (int i = 0; i < pre; ++i) load_b(i, u0 + i);
+  for (int i = pre; i < n; ++i) {
+    const int s = i % STAGES;
+    if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, status, abort_flag)) return;
+    mbar_arrive_expect_tx(&full[s], kATileBytes + B_BYTES);
+    load_a(s, u0 + i);
+    load_b(s, u0 + i);
+  }
+}
+
+template <int NT, int STAGES>
+__device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty, uint64_t* accf,
+                                       uint64_t* acce, uint32_t tmem, const SkSched& sc, long long u0, long long u1,
+                                       int* status, volatile int* abort_flag) {
+  constexpr int B_BYTES = NT * 128;
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, NT);
+  griddep_wait();
+  int i = 0, seg = 0;
+  for (long long u = u0; u < u1; ++seg) {
+    const int T = static_cast<int>(u / sc.kb);
+    const long long seg_end = (static_cast<long long>(T) + 1) * sc.kb < u1 ? (static_cast<long long>(T) + 1) * sc.kb : u1;
+    const int b = seg & 1;
+    if (seg >= 2 && !mbar_wait(&acce[b], ((seg >> 1) - 1) & 1, status, abort_flag)) return;
+    tc_fence_after();
+    const uint32_t d = tmem + static_cast<uint32_t>(b * NT);
+    for (long long uu = u; uu < seg_end; ++uu, ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait(&full[s], (i / STAGES) & 1, status, abort_flag)) return;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA + s * kATileBytes);
+      const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        umma_bf16_ss(d, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
+                     (uu > u || k > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[s]);
+    }
+    umma_commit(&accf[b]);
+    u = seg_end;
+  }
+}
+
+// Copy the NT accumulator columns of TMEM buffer b for this thread's lane.
+template <int NT>
+__device__ __forceinline__ void ws_load_acc(uint32_t tmem, int b, int quarter, float (&v)[NT]) {
+#pragma unroll
+  for (int c = 0; c < NT; c += 16) {
+    float tmp[16];
+    tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * NT + c), tmp);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[c + k] = tmp[k];
+  }
+  tmem_wait_ld();
+}
+
+__device__ __forceinline__ float bf16_round_f(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+}  // namespace dvlm

@@ -1,0 +1,289 @@
+/*
+ * dvlm.h -- C ABI of the B200 (sm_100a) block-diffusion decode step.
+ *
+ * The method (Fast-dVLM / Fast-dLLM v2 block diffusion):
+ *   - the answer is produced in blocks of B tokens; inside a block every
+ *     masked position is denoised in parallel, blocks follow one another
+ *     autoregressively over an exact KV cache
+ *     [Fast-dVLM technical overview (ocdem.com), sections 1.2 and 2.2.1];
+ *   - attention follows three rules: noisy tokens of one block see each other
+ *     (N2N, bidirectional), noisy tokens see the clean tokens of preceding
+ *     blocks including the vision tokens (N2C), clean tokens are token-level
+ *     causal (C2C) [same page, section 2.2.1; Fast-dVLM walkthrough
+ *     (itsolotime.com), section 4.1];
+ *   - each masked position is scored by its top-1 softmax probability over
+ *     the vocabulary [Look Only When Needed (LOWN), method step (1)] and is
+ *     committed when that confidence reaches the threshold (0.9), at least one
+ *     per step [Fast-dVLM overview, section 4.1 recommended configuration];
+ *   - the linear self-speculative variant drafts the block by diffusion,
+ *     verifies it with a causal pass, keeps the longest agreeing prefix and
+ *     truncates the KV cache [Fast-dVLM overview, section 2.3.1];
+ *   - the certificate scan visits positions by descending anchor confidence
+ *     and stops at the first disagreement [LOWN, method step (2)].
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host".
+ *     The caller owns all memory; the library never allocates or frees device
+ *     memory.  Workspaces are sized with the matching *_workspace_size() call
+ *     and must be zero-filled once before their first use; every successful
+ *     call leaves them ready for the next (counters return to zero).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Arguments are validated on the host before any
+ *     launch; a bad argument returns an error status and launches nothing.
+ *   - Errors found on the device (a bounded wait that ran out, an index out of
+ *     range) are written to `*dev_status` (device int, first error wins, may
+ *     be NULL); nothing traps or aborts.  Read it after synchronising.
+ *   - Results are deterministic: the same inputs give bitwise-identical
+ *     outputs (fixed reduction orders, no floating-point atomics).
+ *   - Layouts are row-major; "[a, b, c]" lists dimensions outermost first.
+ *     bf16 tensors hold IEEE bfloat16, fp32 tensors IEEE binary32.
+ *   - The bf16 path runs on tcgen05 tensor cores with TMA-staged operands and
+ *     needs every tensor base 16-byte aligned; the fp32 path (for the tiny
+ *     fp32 model) runs on CUDA cores.
+ */
+#ifndef DVLM_H_
+#define DVLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DVLM_API __attribute__((visibility("default")))
+#else
+#define DVLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dvlm_status {
+  DVLM_OK = 0,
+  DVLM_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad enum value       */
+  DVLM_ERR_SHAPE = 2,         /* sizes inconsistent or out of the supported range */
+  DVLM_ERR_UNSUPPORTED = 3,   /* valid request this build does not implement      */
+  DVLM_ERR_CACHE_OVERFLOW = 4,/* the step would write past Lmax                   */
+  DVLM_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out               */
+  DVLM_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed                */
+  DVLM_ERR_WORKSPACE = 7,     /* workspace missing or smaller than required       */
+  DVLM_ERR_BOUNDS = 8         /* a device-side index check failed (e.g. token id) */
+} dvlm_status;
+
+typedef enum dvlm_dtype { DVLM_BF16 = 0, DVLM_FP32 = 1 } dvlm_dtype;
+
+typedef void* dvlm_stream; /* cudaStream_t */
+
+/* Human-readable name of a status code (static string). */
+DVLM_API const char* dvlm_status_string(int status);
+/* Library version: major*10000 + minor*100 + patch. */
+DVLM_API int dvlm_version(void);
+/* Number of SMs the kernels size their grids for on the current device
+ * (queried once per process); -1 when no device is visible. */
+DVLM_API int dvlm_device_sm_count(void);
+
+/* ------------------------------------------------------------------------
+ * Block-masked GQA attention of one step's rows against the KV cache.
+ *
+ * q        [n_batch, n_rows, Hq, D]   queries, RoPE already applied.
+ * out      [n_batch, n_rows, Hq, D]   attention output (same dtype).
+ * k_cache  [n_batch, Hkv, Lmax, D]    keys; slots [L, L+n_rows) already hold
+ *                                     this step's keys.
+ * v_cache  [n_batch, Hkv, D, Lmax]    values, stored TRANSPOSED (value
+ *                                     feature-major) so both tensor-core
+ *                                     products read K-major operands.
+ * Rows 0..n_clean-1 are clean and causal: row t sits at slot L+t and sees
+ * slots 0..L+t (C2C).  Rows n_clean..n_rows-1 are the noisy block: each sees
+ * every slot 0..L+n_rows-1, i.e. the whole cache (N2C: vision, prompt and
+ * committed tokens) and the whole block (N2N).  Query head h uses KV head
+ * h / (Hq/Hkv).  scale multiplies q.k (normally 1/sqrt(D)); softmax in fp32.
+ * Slots at or beyond L+n_rows are never read into a result, whatever they
+ * hold (NaN poison included).
+ * bf16 path: D == 128, Hq == 8*Hkv, Lmax % 8 == 0.  fp32 path: D <= 128.
+ * Errors: INVALID_ARG (null/misaligned), SHAPE (L+n_rows > Lmax, n_clean >
+ * n_rows, Hq % Hkv), UNSUPPORTED (bf16 head shapes other than the above).
+ */
+DVLM_API dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const void* v_cache,
+                            int n_batch, int n_rows, int n_clean, int L, int Lmax, int Hq, int Hkv,
+                            int D, float scale, dvlm_dtype dt, int* dev_status, dvlm_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Fused LM head + top-1 confidence + threshold commit (+ certificate scan).
+ *
+ * For each row r < R: logits l = s_r * (hidden[r] . W^T) over the whole
+ * vocabulary, streamed tile by tile and never written to memory; s_r is the
+ * final RMSNorm factor 1/sqrt(mean(hidden[r]^2)+eps) when apply_rmsnorm != 0,
+ * else 1.  Outputs (each pointer may be NULL):
+ *   top1_id[r]   = lowest id attaining max l,
+ *   top1_prob[r] = max softmax probability = 1 / sum_v exp(l_v - max l),
+ *   commit[r]    = 1 if row r is committed this call, else 0,
+ *   n_commit[0]  = number of committed rows.
+ * Commit rule: among rows with masked[r] != 0 (all rows when masked is
+ * NULL), every row with top1_prob >= threshold; if none passes, the masked
+ * row with the highest top1_prob (lowest r on ties).  threshold <= -1
+ * commits every masked row (the speculative draft).  When `tokens` is
+ * non-NULL the commit is applied in place: tokens[r] = top1_id[r] and
+ * masked[r] = 0 for committed rows (masked must then be non-NULL).
+ * Certificate (when anchor_id, anchor_conf and cert_len are all non-NULL):
+ * the rows that are masked on entry are visited in descending anchor_conf
+ * (lower r first on ties); cert_len[0] = number visited before the first
+ * row whose top1_id differs from anchor_id.
+ * hidden [R, H], w [V, H] (same dtype).  1 <= R <= 128.
+ * bf16 path: H % 64 == 0.  Workspace: dvlm_lmhead_workspace_size().
+ */
+DVLM_API size_t dvlm_lmhead_workspace_size(int R, int V, int H, dvlm_dtype dt);
+DVLM_API dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, int R, int H, int V,
+                                    dvlm_dtype dt, int apply_rmsnorm, float eps, uint8_t* masked,
+                                    int32_t* tokens, float threshold, int32_t* top1_id,
+                                    float* top1_prob, uint8_t* commit, int32_t* n_commit,
+                                    const int32_t* anchor_id, const float* anchor_conf,
+                                    int32_t* cert_len, void* workspace, size_t ws_bytes,
+                                    int* dev_status, dvlm_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Speculative verify + longest-prefix accept + in-place KV truncation.
+ *
+ * For each sequence i < b: v_j = argmax_v verify_logits[i, j, :] (lowest id
+ * on ties; NaN logits never win) when verify_logits [b, B, V] (bf16) is
+ * non-NULL, else v_j = verify_ids[i, j] ([b, B] int32).  accept_len[i] = k =
+ * the longest prefix length with v_j == draft_ids[i, j] for all j < k.
+ * When cache_len is non-NULL it is updated in place from L0+B (the verify
+ * pass wrote B slots) to L0+k, i.e. cache_len[i] -= B - k.  When
+ * poison_tail != 0 the truncated slots [L0+k, L0+B) of every layer are
+ * overwritten with bf16 NaN in k_cache [n_layers, b, Hkv, Lmax, D] and
+ * v_cache [n_layers, b, Hkv, D, Lmax] (a debugging aid: attention never reads
+ * them).  Workspace: dvlm_spec_workspace_size().
+ */
+DVLM_API size_t dvlm_spec_workspace_size(int b, int B, int V);
+DVLM_API dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const int32_t* verify_ids,
+                                    const int32_t* draft_ids, int b, int B, int V,
+                                    int32_t* accept_len, int32_t* cache_len, int poison_tail,
+                                    void* k_cache, void* v_cache, int n_layers, int Hkv, int D,
+                                    int Lmax, void* workspace, size_t ws_bytes, int* dev_status,
+                                    dvlm_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Decoder model and decode engine.
+ *
+ * dvlm_model holds non-owning views of device weights, all [out, in]
+ * row-major in the model dtype:
+ *   embed   [V, H]                 token embeddings
+ *   wqkv    [n_layers, (Hq+2*Hkv)*D, H]  rows: Hq query heads, Hkv key
+ *                                  heads, Hkv value heads (D rows each)
+ *   wo      [n_layers, H, Hq*D]
+ *   wgate   [n_layers, I, H]       SwiGLU gate
+ *   wup     [n_layers, I, H]       SwiGLU up
+ *   wdown   [n_layers, H, I]
+ *   lm_head [V, H]                 untied output projection
+ * Each layer: x += Wo.attn(RoPE(Wqkv.rmsnorm(x))); x += Wdown.(silu(Wgate.n)
+ * * Wup.n) with n = rmsnorm(x); RMSNorm gain 1; RoPE rotate-half with base
+ * rope_base at absolute slot positions; final RMSNorm before the LM head.
+ * bf16 storage points: q/k/v after RoPE, attention output, the residual
+ * stream after each add, the SwiGLU activation; all sums in fp32.
+ * bf16 path: H % 128 == 0, I % 64 == 0, D == 128, Hq == 8*Hkv.
+ */
+typedef struct dvlm_model {
+  int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, inter, vocab;
+  int mask_id;       /* id of [MASK]; its embedding row feeds masked positions */
+  float rope_base, eps;
+  int dtype;         /* dvlm_dtype */
+  const void* embed;
+  const void* wqkv;
+  const void* wo;
+  const void* wgate;
+  const void* wup;
+  const void* wdown;
+  const void* lm_head;
+} dvlm_model;
+
+enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2 };
+
+typedef struct dvlm_decode_cfg {
+  int block_size;     /* B, 1..16 */
+  float threshold;    /* commit threshold (0.9) */
+  int mode;           /* DVLM_MODE_* */
+  int ar_seed;        /* 1: the block's first token is the AR prediction, committed outright */
+  int max_new_tokens; /* generation stops after exactly this many tokens */
+  int use_graphs;     /* 1: replay each forward as a captured CUDA graph */
+} dvlm_decode_cfg;
+
+#define DVLM_HIST 17
+typedef struct dvlm_stats {
+  int64_t nfe;                    /* decoder forwards (noisy iterations + causal passes) */
+  int64_t n_tokens;               /* tokens emitted */
+  int64_t n_iters;                /* threshold iterations (noisy passes) */
+  int64_t n_rounds;               /* blocks (threshold/AR) or draft+verify rounds (spec) */
+  int64_t commit_hist[DVLM_HIST]; /* iterations that committed c tokens, c = 0..16 */
+  int64_t accept_hist[DVLM_HIST]; /* spec rounds that accepted k tokens, k = 0..16 */
+  int64_t n_launches;             /* kernel launches issued (graph replays included) */
+} dvlm_stats;
+
+typedef struct dvlm_engine dvlm_engine;
+
+/* Workspace for an engine serving contexts up to Lmax slots, blocks up to
+ * max_block (<= 16) rows and prompts (vision + ids) up to max_ctx rows. */
+DVLM_API size_t dvlm_engine_workspace_size(const dvlm_model* m, int Lmax, int max_block, int max_ctx);
+/* Builds the host-side engine (tensor maps, launch plans) over the caller's
+ * buffers and zero-fills the workspace on `stream`.  k_cache [n_layers, Hkv,
+ * Lmax, D] and v_cache [n_layers, Hkv, D, Lmax] (transposed) hold the exact
+ * KV cache.  The engine keeps pointers, not copies. */
+DVLM_API dvlm_status dvlm_engine_create(const dvlm_model* m, void* k_cache, void* v_cache, int Lmax,
+                               int max_block, int max_ctx, void* workspace, size_t ws_bytes,
+                               dvlm_stream stream, dvlm_engine** out);
+DVLM_API dvlm_status dvlm_engine_destroy(dvlm_engine* e);
+/* Causal pass over the context [vision rows | text ids] starting at slot 0
+ * (vision [n_vision, H] in the model dtype, ids [n_ids] int32, both device),
+ * in chunks of max_block rows; leaves L = n_vision + n_ids and the AR seed
+ * (argmax of the LM head at the last context row) on the device. */
+DVLM_API dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_vision, const int32_t* ids,
+                         int n_ids, dvlm_stream stream);
+/* Decodes one block (threshold/AR modes: B tokens; spec mode: one draft +
+ * verify round, 1..B tokens).  Tokens go to out_tokens (device, >= B
+ * entries); *n_out (host) receives their count.  Synchronises the stream
+ * once per noisy iteration (threshold mode) or round.  stats accumulate. */
+DVLM_API dvlm_status dvlm_decode_block(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_t* out_tokens,
+                              int32_t* n_out, dvlm_stats* stats, dvlm_stream stream);
+/* Decodes exactly cfg->max_new_tokens tokens into out_tokens (device). */
+DVLM_API dvlm_status dvlm_generate(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_t* out_tokens,
+                          dvlm_stats* stats, dvlm_stream stream);
+/* End to end from HOST buffers: copies vision_host [n_vision, H] (model
+ * dtype) and ids_host [n_ids] to the device, prefills, generates
+ * cfg->max_new_tokens tokens and copies them to out_host.  Pinned host
+ * buffers make the copies asynchronous.  Returns after the stream drained. */
+DVLM_API dvlm_status dvlm_generate_host(dvlm_engine* e, const dvlm_decode_cfg* cfg, const void* vision_host,
+                               int n_vision, const int32_t* ids_host, int n_ids,
+                               int32_t* out_host, dvlm_stats* stats, dvlm_stream stream);
+/* Cache length and pending seed token (host copies; synchronises). */
+DVLM_API dvlm_status dvlm_engine_get_position(dvlm_engine* e, int32_t* L, int32_t* seed, dvlm_stream stream);
+/* Rewinds to an earlier (L, seed); slots [0, L) must still hold that context. */
+DVLM_API dvlm_status dvlm_engine_set_position(dvlm_engine* e, int32_t L, int32_t seed, dvlm_stream stream);
+/* Synchronises, returns the first device-side error recorded since the last
+ * call (DVLM_OK if none) and clears it. */
+DVLM_API dvlm_status dvlm_engine_check(dvlm_engine* e, dvlm_stream stream);
+
+/* One forward pass of n_rows rows at slots [L, L+n_rows) through layers
+ * [first_layer, first_layer+n_layers_run) (test and profiling hook).  Input
+ * rows: x_in [n_rows, H] (model dtype) when non-NULL, else the embeddings of
+ * tokens [n_rows] (rows with masked[r] != 0 take the [MASK] embedding).
+ * Rows 0..n_clean-1 are causal, the rest one noisy block.  Writes this
+ * step's K/V to slots [L, L+n_rows) of the layers it runs, the resulting
+ * residual stream to x_out [n_rows, H] (may be NULL) and, when
+ * advance != 0, sets L += n_rows. */
+DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_t* tokens,
+                         const uint8_t* masked, int n_rows, int n_clean, int first_layer,
+                         int n_layers_run, int advance, void* x_out, dvlm_stream stream);
+
+/* Profiling hook: one forward pass like dvlm_forward over all layers (L is
+ * not advanced), launched eagerly with a CUDA event pair around every kernel
+ * on `stream`.  ms_out[7] receives the device time per kernel class summed
+ * over layers and counts_out[7] the launches: [0] embedding, [1] QKV GEMM,
+ * [2] attention, [3] O-projection GEMM, [4] gate/up GEMM, [5] down GEMM,
+ * [6] fused LM head (run when with_lm_head != 0, rows 0..n_rows-1, no
+ * commit).  Synchronises the stream. */
+DVLM_API dvlm_status dvlm_profile_forward(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
+                                          int n_rows, int n_clean, int with_lm_head, float* ms_out,
+                                          int* counts_out, dvlm_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DVLM_H_ */

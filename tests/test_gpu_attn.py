@@ -1,0 +1,100 @@
+"""Block-masked attention (N2N / N2C / C2C): CUDA path vs the oracle.
+
+Bar: max abs error 2e-2 on bf16 outputs (the oracle is fp64 on the same bf16
+inputs), 1e-4 on the fp32 path."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_vlm_b200 as dv
+import dvlm_gen as gen
+import oracle as O
+from gpu_util import assert_ok, f64, max_abs, status
+
+pytestmark = pytest.mark.gpu
+TOL_BF16 = 2e-2
+
+
+def run_attn(q, k, v, n_rows, n_clean, L, dev, dtype=dv.DVLM_BF16, Hq=16, Hkv=2, D=128):
+    """q [nb, n, Hq, D]; k [nb, Hkv, Lmax, D]; v [nb, Hkv, Lmax, D] (transposed here)."""
+    nb, Lmax = k.shape[0], k.shape[2]
+    qd = q.to(dev).contiguous()
+    kd = k.to(dev).contiguous()
+    vt = v.transpose(-1, -2).contiguous().to(dev)
+    out = torch.full_like(qd, float("nan"))
+    st = status(dev)
+    dv.block_attn(qd, out, kd, vt, n_batch=nb, n_rows=n_rows, n_clean=n_clean, L=L, Lmax=Lmax, Hq=Hq, Hkv=Hkv,
+                  D=D, scale=1.0 / math.sqrt(D), dtype=dtype, status=st)
+    assert_ok(st)
+    return out
+
+
+def oracle_attn(q, k, v, n_clean, L):
+    q64, k64, v64 = f64(q), f64(k), f64(v)
+    D = q64.shape[-1]
+    return np.stack([O.block_attention(q64[b], k64[b], v64[b], L, n_clean, 1.0 / math.sqrt(D))
+                     for b in range(q64.shape[0])])
+
+
+def _pad8(n):
+    return (n + 7) // 8 * 8
+
+
+@pytest.mark.parametrize("B", [4, 8, 16, 32])
+@pytest.mark.parametrize("L", [256, 1024, 4096])
+def test_noisy_block_sweep(cuda, B, L):
+    """Block-attention configuration: 16 query / 2 KV heads, head_dim 128,
+    K/V/Q N(0,1), noisy block of B rows over a cache of L slots."""
+    q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=_pad8(L + B)))
+    out = run_attn(q, k, v, B, 0, L, cuda)
+    err = max_abs(f64(out), oracle_attn(q, k, v, 0, L))
+    assert err < TOL_BF16, err
+
+
+@pytest.mark.parametrize("n_rows,n_clean,L", [(16, 16, 1280), (12, 5, 1000), (16, 16, 0), (3, 3, 37),
+                                              (1, 1, 1343), (16, 8, 64), (20, 20, 100)])
+def test_clean_and_mixed_rows(cuda, n_rows, n_clean, L):
+    q, k, v = (t for t, _ in gen.attn_case(2, n_rows, L, Lmax=_pad8(L + n_rows) + 8))
+    out = run_attn(q, k, v, n_rows, n_clean, L, cuda)
+    err = max_abs(f64(out), oracle_attn(q, k, v, n_clean, L))
+    assert err < TOL_BF16, err
+
+
+def test_batched_problems(cuda):
+    q, k, v = (t for t, _ in gen.attn_case(3, 16, 700, Lmax=720, n_batch=3))
+    out = run_attn(q, k, v, 16, 4, 700, cuda)
+    err = max_abs(f64(out), oracle_attn(q, k, v, 4, 700))
+    assert err < TOL_BF16, err
+
+
+def test_slots_past_the_step_are_never_read(cuda):
+    """Stale slots at or beyond L+n_rows (here NaN poison, as the speculative
+    truncation leaves them) do not change any output."""
+    L, n = 300, 16
+    q, k, v = (t for t, _ in gen.attn_case(4, n, L, Lmax=512))
+    ref = run_attn(q, k, v, n, 0, L, cuda)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, L + n:] = float("nan")
+    v2[:, :, L + n:] = float("nan")
+    out = run_attn(q, k2, v2, n, 0, L, cuda)
+    assert torch.isfinite(out).all()
+    assert torch.equal(out, ref)
+
+
+def test_deterministic(cuda):
+    q, k, v = (t for t, _ in gen.attn_case(5, 16, 1024, Lmax=1040))
+    a = run_attn(q, k, v, 16, 0, 1024, cuda)
+    b = run_attn(q, k, v, 16, 0, 1024, cuda)
+    assert torch.equal(a, b)
+
+
+def test_fp32_path(cuda):
+    """Tiny fp32 shapes: 2 query heads, 1 KV head, head_dim 16."""
+    q, k, v = (t for t, _ in gen.attn_case(6, 4, 60, Hq=2, Hkv=1, D=16, Lmax=64, dtype="f32"))
+    out = run_attn(q, k, v, 4, 0, 60, cuda, dtype=dv.DVLM_FP32, Hq=2, Hkv=1, D=16)
+    err = max_abs(f64(out), oracle_attn(q, k, v, 0, 60))
+    assert err < 1e-4, err
+    out = run_attn(q, k, v, 4, 4, 60, cuda, dtype=dv.DVLM_FP32, Hq=2, Hkv=1, D=16)
+    assert max_abs(f64(out), oracle_attn(q, k, v, 4, 60)) < 1e-4

@@ -1,0 +1,124 @@
+"""End-to-end block decoding through the engine vs the oracle's decoders on
+small models: the tiny fp32 model (first configuration: 64-token context of 32
+vision embeddings, 16 prompt and 16 committed ids, one B=4 block, threshold
+0.9) and a reduced-depth bf16 model with the same per-head shapes as the
+Qwen2.5-3B decoder.  Token sequences and commit counts must match exactly
+when every decision on the oracle's trajectory is at least 1e-3 away from its
+threshold / runner-up (the seeds below were chosen for that by running the
+oracle alone); otherwise a mismatch is only allowed when the oracle's
+trajectory does contain such a near-tie."""
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_vlm_b200 as dv
+import dvlm_gen as gen
+import oracle as O
+from dvlm_gen.device import DeviceModel, kv_buffers
+from gpu_util import f64, max_abs, ws_tensor
+
+pytestmark = pytest.mark.gpu
+MARGIN = 1e-3
+
+SMALL_BF16 = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=1024,
+                           vocab=4096, lm_scale=25.0, dtype="bf16")
+
+
+class Setup:
+    def __init__(self, dims, seed, cuda, n_vis, n_prompt, n_comm, Lmax=512):
+        self.dims, self.seed, self.cuda = dims, seed, cuda
+        self.dm = DeviceModel(dims, seed, device=cuda)
+        self.kc, self.vc = kv_buffers(dims, Lmax, device=cuda)
+        cm = self.dm.c_model()
+        self.ws = ws_tensor(dv.engine_workspace_size(cm, Lmax, 16, 128), cuda)
+        self.eng = dv.Engine(cm, self.kc, self.vc, Lmax, 16, 128, self.ws)
+        self.vis_t, self.vis, self.ids = gen.decode_context(dims, seed, n_vis, n_prompt, n_comm)
+        self.w = O.weights_from_generator(gen, dims, seed)
+        self.od = O.dims_from(dims)
+        self.Lmax = Lmax
+
+    def gpu(self, mode, B, tau, n_new, use_graphs=1):
+        eng = self.eng
+        vis = self.vis_t.to(self.cuda)
+        ids = torch.from_numpy(self.ids).to(self.cuda)
+        eng.prefill(vis, vis.shape[0], ids, len(self.ids))
+        cfg = dv.DecodeCfg(B, tau, mode, 1, n_new, use_graphs)
+        out = torch.zeros(n_new, dtype=torch.int32, device=self.cuda)
+        st = dv.Stats()
+        eng.generate(cfg, out, st)
+        eng.check()
+        return out.cpu().numpy().tolist(), st
+
+    def oracle(self, mode, B, tau, n_new):
+        m = O.OracleModel(self.od, weights=self.w, bf16=self.dims.dtype == "bf16", Lmax=self.Lmax)
+        s = O.prefill(m, self.vis.astype(np.float64), self.ids)
+        if mode == dv.MODE_THRESHOLD:
+            return O.decode_threshold(m, s, B, tau, n_new), m
+        if mode == dv.MODE_SPEC_LINEAR:
+            return O.decode_spec_linear(m, s, B, n_new), m
+        return O.decode_ar(m, s, n_new), m
+
+
+def _compare(tokens, st, tr, mode):
+    if tr.min_margin >= MARGIN:
+        assert tokens == tr.tokens
+        assert st.nfe == tr.nfe
+        if mode == dv.MODE_THRESHOLD:
+            hist = np.bincount(tr.commits_per_iter, minlength=dv.binding.HIST)[:dv.binding.HIST]
+            assert list(st.commit_hist) == hist.tolist()
+        if mode == dv.MODE_SPEC_LINEAR:
+            hist = np.bincount(tr.accept_lens, minlength=dv.binding.HIST)[:dv.binding.HIST]
+            assert list(st.accept_hist) == hist.tolist()
+    elif tokens != tr.tokens:
+        assert tr.min_margin < MARGIN
+
+
+@pytest.fixture(scope="module")
+def tiny0(cuda):
+    return Setup(gen.TINY, 0, cuda, 32, 16, 16, Lmax=128)
+
+
+@pytest.fixture(scope="module")
+def tiny4(cuda):
+    return Setup(gen.TINY, 4, cuda, 32, 16, 16, Lmax=128)
+
+
+def test_tiny_fp32_block_step_seed0(tiny0):
+    """The tiny configuration exactly as stated: seed 0, one B=4 block."""
+    tokens, st = tiny0.gpu(dv.MODE_THRESHOLD, 4, 0.9, 4)
+    tr, m = tiny0.oracle(dv.MODE_THRESHOLD, 4, 0.9, 4)
+    _compare(tokens, st, tr, dv.MODE_THRESHOLD)
+    # the exact KV cache after the block (prefill + causal append) within 1e-4
+    L = m.L
+    kc = f64(tiny0.kc[0, 0, :, :L])
+    vc = f64(tiny0.vc[0, 0, :, :, :L]).transpose(0, 2, 1)
+    if tokens == tr.tokens:
+        assert max_abs(kc, m.K[0][:, :L]) < 1e-4
+        assert max_abs(vc, m.V[0][:, :L]) < 1e-4
+
+
+@pytest.mark.parametrize("mode", [dv.MODE_THRESHOLD, dv.MODE_SPEC_LINEAR, dv.MODE_AR])
+def test_tiny_fp32_modes_seed4(tiny4, mode):
+    tokens, st = tiny4.gpu(mode, 4, 0.9, 16)
+    tr, m = tiny4.oracle(mode, 4, 0.9, 16)
+    assert tr.min_margin >= MARGIN  # chosen seed: well-conditioned trajectory
+    _compare(tokens, st, tr, mode)
+
+
+def test_tiny_fp32_graphs_match_eager(tiny4):
+    a, sa = tiny4.gpu(dv.MODE_THRESHOLD, 4, 0.9, 16, use_graphs=1)
+    b, sb = tiny4.gpu(dv.MODE_THRESHOLD, 4, 0.9, 16, use_graphs=0)
+    assert a == b and sa.nfe == sb.nfe
+
+
+@pytest.mark.parametrize("seed,mode", [(1, dv.MODE_THRESHOLD), (3, dv.MODE_THRESHOLD),
+                                       (6, dv.MODE_SPEC_LINEAR)])
+def test_bf16_reduced_model_matches_oracle(cuda, seed, mode):
+    """2 layers, hidden 1024, 8/1 heads of 128, SwiGLU 1024, vocab 4096;
+    48-token context (32 vision + 16 prompt), B=16, threshold 0.9, 32 tokens."""
+    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
+    tokens, st = s.gpu(mode, 16, 0.9, 32)
+    tr, m = s.oracle(mode, 16, 0.9, 32)
+    assert tr.min_margin >= MARGIN
+    _compare(tokens, st, tr, mode)
+    s.eng.close()

@@ -1,0 +1,185 @@
+"""Fused LM head + confidence + threshold commit + certificate: CUDA path vs
+the oracle on the same seeded inputs.
+
+Bar: top-1 ids and commit sets bit-exact except rows whose oracle margin to
+the runner-up (p1 - p2) or to the threshold (|p1 - tau|) is below 1e-3, where
+the GPU's choice must still be one of the tied candidates; p1 within 2e-4
+(fp32 accumulation and exp against the oracle's fp64)."""
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_vlm_b200 as dv
+import dvlm_gen as gen
+import oracle as O
+from gpu_util import assert_ok, f64, status, ws_tensor
+
+pytestmark = pytest.mark.gpu
+MARGIN = 1e-3
+P1_TOL = 2e-4
+
+
+def run_lmhead(h, w, R, H, V, dev, dtype=dv.DVLM_BF16, masked=None, tokens=None, threshold=0.9, anchors=None,
+               apply_rmsnorm=0):
+    out = dict(top1_id=torch.full((R,), -1, dtype=torch.int32, device=dev),
+               top1_prob=torch.full((R,), -1.0, dtype=torch.float32, device=dev),
+               commit=torch.zeros(R, dtype=torch.uint8, device=dev),
+               n_commit=torch.zeros(1, dtype=torch.int32, device=dev))
+    cert = None
+    kw = {}
+    if anchors is not None:
+        cert = torch.full((1,), -1, dtype=torch.int32, device=dev)
+        kw = dict(anchor_id=anchors[0], anchor_conf=anchors[1], cert_len=cert)
+    ws = ws_tensor(dv.lmhead_workspace_size(R, V, H, dtype), dev)
+    st = status(dev)
+    dv.lmhead_conf_commit(h, w, R=R, H=H, V=V, dtype=dtype, apply_rmsnorm=apply_rmsnorm, masked=masked,
+                          tokens=tokens, threshold=threshold, workspace=ws, status=st, **out, **kw)
+    assert_ok(st)
+    res = {k: v.cpu().numpy() for k, v in out.items()}
+    if cert is not None:
+        res["cert_len"] = int(cert.item())
+    return res
+
+
+def check_ids_probs(res, conf: O.Conf, R):
+    np.testing.assert_allclose(res["top1_prob"], conf.p1[:R], atol=P1_TOL, rtol=0)
+    for r in range(R):
+        if conf.p1[r] - conf.p2[r] >= MARGIN:
+            assert res["top1_id"][r] == conf.top1[r], (r, res["top1_id"][r], conf.top1[r])
+
+
+def check_commit(res, conf: O.Conf, masked, tau, R):
+    want = O.threshold_commit(conf.p1[:R], masked, tau)
+    got = [r for r in range(R) if res["commit"][r]]
+    near = [r for r in range(R) if masked[r] and abs(conf.p1[r] - tau) < MARGIN]
+    if not any(masked[r] and conf.p1[r] >= tau for r in range(R)):
+        # force-commit: exactly one row, the best masked p1 (ties within the margin accepted)
+        assert len(got) == 1
+        best = max(conf.p1[r] for r in range(R) if masked[r])
+        assert masked[got[0]] and conf.p1[got[0]] >= best - MARGIN
+    else:
+        assert set(got) - set(near) == set(want) - set(near), (got, want)
+    assert int(res["n_commit"][0]) == len(got)
+
+
+def _case(seed, R, H, V, lm_scale=25.0):
+    (h_t, h), (w_t, w) = gen.lmhead_case(seed, R, H, V, lm_scale=lm_scale, second_set=False)
+    return h_t, h.astype(np.float64), w_t, w.astype(np.float64)
+
+
+@pytest.mark.parametrize("R,H,V", [(1, 128, 384), (5, 256, 1000), (16, 256, 1000), (17, 512, 4099),
+                                   (32, 256, 1000), (100, 128, 2000), (128, 64, 640)])
+def test_lmhead_small_shapes(cuda, R, H, V):
+    h_t, h, w_t, w = _case(11 + R, R, H, V, lm_scale=12.0)
+    res = run_lmhead(h_t.to(cuda), w_t.to(cuda), R, H, V, cuda)
+    conf = O.lm_head_conf(h, w)
+    check_ids_probs(res, conf, R)
+    check_commit(res, conf, [1] * R, 0.9, R)
+
+
+@pytest.mark.parametrize("R", [1, 16, 32, 128])
+def test_lmhead_full_vocab(cuda, R):
+    """Fused LM head configuration: hidden [R, 2048] N(0,1), W [151936, 2048]
+    N(0, 0.02) x 25, threshold 0.9."""
+    H, V = 2048, 151936
+    h_t, h, w_t, w = _case(2, R, H, V)
+    res = run_lmhead(h_t.to(cuda), w_t.to(cuda), R, H, V, cuda)
+    conf = O.lm_head_conf(h, w)
+    check_ids_probs(res, conf, R)
+    check_commit(res, conf, [1] * R, 0.9, R)
+    assert conf.p1.min() < 0.9 < conf.p1.max()  # the x25 scale spreads top-1 probabilities
+
+
+def test_lmhead_ties_take_lowest_id(cuda):
+    R, H, V = 8, 256, 3000
+    h_t, h, w_t, w = _case(5, R, H, V)
+    conf = O.lm_head_conf(h, w)
+    w2 = w_t.clone()
+    for r in range(R):          # duplicate each row's winner at a lower id -> exact tie
+        low = (int(conf.top1[r]) * 7 + 13 + r) % int(conf.top1[r]) if conf.top1[r] > 0 else None
+        if low is not None:
+            w2[low] = w_t[int(conf.top1[r])]
+    conf2 = O.lm_head_conf(h, w2.float().numpy().astype(np.float64))
+    res = run_lmhead(h_t.to(cuda), w2.to(cuda), R, H, V, cuda)
+    np.testing.assert_array_equal(res["top1_id"], conf2.top1)
+    np.testing.assert_allclose(res["top1_prob"], conf2.p1, atol=P1_TOL)
+    assert np.all(conf2.p1 <= 0.5 + 1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.9, 1.5, -1.0, 0.0])
+def test_lmhead_commit_rules_and_in_place_update(cuda, tau):
+    R, H, V = 16, 256, 2048
+    h_t, h, w_t, w = _case(7, R, H, V)
+    conf = O.lm_head_conf(h, w)
+    masked = np.array([1, 1, 0, 1, 1, 1, 0, 1, 1, 1, 1, 1, 0, 1, 1, 1], dtype=np.uint8)
+    tokens0 = np.arange(R, dtype=np.int32) + 10000
+    m_t = torch.from_numpy(masked).to(cuda)
+    tok_t = torch.from_numpy(tokens0).to(cuda)
+    res = run_lmhead(h_t.to(cuda), w_t.to(cuda), R, H, V, cuda, masked=m_t, tokens=tok_t, threshold=tau)
+    check_ids_probs(res, conf, R)
+    check_commit(res, conf, masked, tau, R)
+    got = [r for r in range(R) if res["commit"][r]]
+    m_after, tok_after = m_t.cpu().numpy(), tok_t.cpu().numpy()
+    for r in range(R):
+        if r in got:
+            assert m_after[r] == 0 and tok_after[r] == res["top1_id"][r]
+        else:
+            assert m_after[r] == masked[r] and tok_after[r] == tokens0[r]
+    if tau > 1:
+        assert len(got) == 1
+    if tau <= 0:
+        assert got == [r for r in range(R) if masked[r]]
+
+
+def test_lmhead_certificate_full_vocab(cuda):
+    """Certificate check of the fused LM-head configuration: anchors are the
+    top-1 (id, confidence) of hidden set H1; the kernel scores H2 = H1 + 0.5 N(0,1)
+    and returns the longest certified prefix in descending anchor confidence."""
+    R, H, V = 32, 2048, 151936
+    (h1_t, h1), (w_t, w), (h2_t, h2) = gen.lmhead_case(2, R, H, V)
+    h1, h2, w = (a.astype(np.float64) for a in (h1, h2, w))
+    a = O.lm_head_conf(h1, w)
+    b = O.lm_head_conf(h2, w)
+    aid = torch.from_numpy(a.top1.astype(np.int32)).to(cuda)
+    aconf = torch.from_numpy(a.p1.astype(np.float32)).to(cuda)
+    res = run_lmhead(h2_t.to(cuda), w_t.to(cuda), R, H, V, cuda, anchors=(aid, aconf))
+    check_ids_probs(res, b, R)
+    want = O.certificate_scan(a.top1, a.p1.astype(np.float32), b.top1)
+    order = sorted(range(R), key=lambda i: (-float(np.float32(a.p1[i])), i))
+    # a near-tie in H2's argmax at or before the stop position makes the stop ambiguous
+    ambiguous = any(b.p1[i] - b.p2[i] < MARGIN for i in order[:want + 1])
+    if not ambiguous:
+        assert res["cert_len"] == want
+    assert 0 < sum(a.top1 == b.top1) < R  # partial agreement, as the configuration intends
+
+
+def test_lmhead_final_rmsnorm(cuda):
+    R, H, V = 16, 2048, 8192
+    h_t, h, w_t, w = _case(9, R, H, V)
+    h_t = (h_t.float() * 3.0).to(torch.bfloat16)
+    h = h_t.float().numpy().astype(np.float64)
+    res = run_lmhead(h_t.to(cuda), w_t.to(cuda), R, H, V, cuda, apply_rmsnorm=1)
+    conf = O.lm_head_conf(h, w, O.rms_factor(h)[:, 0])
+    check_ids_probs(res, conf, R)
+
+
+def test_lmhead_deterministic(cuda):
+    R, H, V = 32, 2048, 151936
+    h_t, h, w_t, w = _case(3, R, H, V)
+    hd, wd = h_t.to(cuda), w_t.to(cuda)
+    r1 = run_lmhead(hd, wd, R, H, V, cuda)
+    r2 = run_lmhead(hd, wd, R, H, V, cuda)
+    assert np.array_equal(r1["top1_prob"].view(np.uint32), r2["top1_prob"].view(np.uint32))
+    assert np.array_equal(r1["top1_id"], r2["top1_id"])
+
+
+def test_lmhead_fp32_path(cuda):
+    R, H, V = 4, 32, 256
+    rng = np.random.default_rng(0)
+    h = rng.standard_normal((R, H)).astype(np.float32)
+    w = (rng.standard_normal((V, H)) * 0.8).astype(np.float32)
+    res = run_lmhead(torch.from_numpy(h).to(cuda), torch.from_numpy(w).to(cuda), R, H, V, cuda,
+                     dtype=dv.DVLM_FP32, apply_rmsnorm=1)
+    conf = O.lm_head_conf(h.astype(np.float64), w.astype(np.float64), O.rms_factor(h.astype(np.float64))[:, 0])
+    np.testing.assert_allclose(res["top1_prob"], conf.p1, atol=1e-5)
+    np.testing.assert_array_equal(res["top1_id"], conf.top1)
