@@ -268,9 +268,10 @@ def run_ours(args, rank, world, local, pg):
     import dvlm_gen as gen
     from dvlm_gen.device import DeviceModel, kv_buffers
 
+    import dataclasses
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    dims = gen.QWEN3B
+    dims = gen.QWEN3B if args.layers == 36 else dataclasses.replace(gen.QWEN3B, n_layers=args.layers)
     dm = DeviceModel(dims, SEED, device=dev)
     Lmax = N_VIS + N_PROMPT + N_NEW + 32
     kc, vc = kv_buffers(dims, Lmax, device=dev)
@@ -284,6 +285,16 @@ def run_ours(args, rank, world, local, pg):
     eng.prefill(vis_d, N_VIS, ids_d, N_PROMPT, stream=stream)
     eng.check(stream=stream)
     L0, seed0 = eng.position(stream=stream)
+    if args.profile_forwards:
+        # profiling case for ncu: eager noisy-block forwards only
+        toks = torch.full((BLOCK,), dims.mask_id, dtype=torch.int32, device=dev)
+        for _ in range(args.profile_forwards):
+            eng.profile_forward(toks, BLOCK, 0, stream=stream)
+        eng.check(stream=stream)
+        eng.close()
+        if rank == 0:
+            print(json.dumps({"profile_forwards": args.profile_forwards, "layers": dims.n_layers}), flush=True)
+        return
     mode = {"threshold": dv.MODE_THRESHOLD, "spec": dv.MODE_SPEC_LINEAR, "ar": dv.MODE_AR}[args.mode]
     cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1)
     out = torch.zeros(N_NEW, dtype=torch.int32, device=dev)
@@ -393,6 +404,9 @@ def main():
     ap.add_argument("--mode", choices=["threshold", "spec", "ar"], default="threshold")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the extra speculative-mode run")
+    ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")
+    ap.add_argument("--profile-forwards", type=int, default=0,
+                    help="profiling case: run this many eager forwards after prefill and exit")
     args = ap.parse_args()
     rank, world, local, pg = dist_setup()
     try:

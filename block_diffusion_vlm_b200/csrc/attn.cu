@@ -217,7 +217,9 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
             if (8 * cc + e >= valid) chunk[e] = 0;
         }
       }
-      if (jj >= 1 && alpha != 1.0f) {
+      // tcgen05.ld/st are warp-collective: the rescale runs for the whole warp
+      // when any of its rows needs it (alpha == 1 leaves a row unchanged).
+      if (jj >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, a.status, sabort);
         tc_fence_after();
 #pragma unroll

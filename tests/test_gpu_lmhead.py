@@ -87,7 +87,8 @@ def test_lmhead_full_vocab(cuda, R):
     conf = O.lm_head_conf(h, w)
     check_ids_probs(res, conf, R)
     check_commit(res, conf, [1] * R, 0.9, R)
-    assert conf.p1.min() < 0.9 < conf.p1.max()  # the x25 scale spreads top-1 probabilities
+    if R >= 16:
+        assert conf.p1.min() < 0.9 < conf.p1.max()  # the x25 scale spreads top-1 probabilities
 
 
 def test_lmhead_ties_take_lowest_id(cuda):
