@@ -4,7 +4,9 @@ layer: QKV GEMM + RMSNorm factor + RoPE + KV-slot write, block attention,
 O-proj + residual, gate/up + SwiGLU, down + residual.  Inputs are generator
 draws (cache prefix N(0,1), token embeddings or N(0,1) rows), so nothing
 from the CUDA path feeds the oracle.  Bar: max abs error 2e-2 on every bf16
-output (residual stream and the K/V written)."""
+output (residual stream and the K/V written), plus one bf16 storage ulp of the
+reference where fp32 and fp64 sums round to neighbouring bf16 values (see
+gpu_util.assert_bf16_close)."""
 import dataclasses
 
 import numpy as np
@@ -15,7 +17,7 @@ import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
 import oracle as O
 from dvlm_gen.device import DeviceModel, kv_buffers
-from gpu_util import f64, max_abs, ws_tensor
+from gpu_util import assert_bf16_close, f64, max_abs, ws_tensor
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
@@ -76,8 +78,8 @@ def test_noisy_block_of_tokens(layer_setup, cuda):
     x = E_t[torch.tensor(rows)].float().numpy().astype(np.float64)
     got = _run(s, None, torch.from_numpy(ids).to(cuda), torch.from_numpy(masked).to(cuda), 16, 0, cuda)
     want = _oracle(s, x, 0)
-    errs = [max_abs(g, w) for g, w in zip(got, want)]
-    assert max(errs) < TOL, errs
+    for g, w, what in zip(got, want, ("x", "k", "v")):
+        assert_bf16_close(g, w, TOL, what)
 
 
 @pytest.mark.parametrize("n_rows,n_clean", [(16, 16), (9, 9), (16, 6)])
@@ -87,5 +89,5 @@ def test_clean_rows_from_hidden_states(layer_setup, cuda, n_rows, n_clean):
     x_t, x = gen.normal_bf16(SEED + n_rows, "layer.x", (n_rows, s["dims"].hidden))
     got = _run(s, x_t.to(cuda), None, None, n_rows, n_clean, cuda)
     want = _oracle(s, x.astype(np.float64), n_clean)
-    errs = [max_abs(g, w) for g, w in zip(got, want)]
-    assert max(errs) < TOL, errs
+    for g, w, what in zip(got, want, ("x", "k", "v")):
+        assert_bf16_close(g, w, TOL, what)
