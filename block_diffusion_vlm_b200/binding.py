@@ -88,6 +88,8 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_lmhead_workspace_size": (_sz, [_i, _i, _i, _i]),
         "dvlm_lmhead_conf_commit": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+        "dvlm_lmhead_conf_commit_static": (_i, [_vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _f, _vp, _vp, _vp, _vp,
+                                                _vp, _vp, _vp, _vp, _vp]),
         "dvlm_spec_workspace_size": (_sz, [_i, _i, _i]),
         "dvlm_spec_verify_accept": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp,
                                          _sz, _vp, _vp]),
@@ -161,6 +163,17 @@ def lmhead_conf_commit(hidden, w, *, R, H, V, dtype, apply_rmsnorm=0, eps=1e-6, 
                                          ptr(cert_len), ptr(workspace), ws_bytes, ptr(status),
                                          stream_handle(stream)),
            "dvlm_lmhead_conf_commit")
+
+
+def lmhead_conf_commit_static(hidden, w, *, R, H, V, apply_rmsnorm=0, eps=1e-6, masked=None, tokens=None,
+                              threshold=0.9, top1_id=None, top1_prob=None, commit=None, n_commit=None,
+                              anchor_id=None, anchor_conf=None, cert_len=None, status=None, stream=None) -> None:
+    """bf16 fused LM head with the library's fixed internal scratch (no workspace argument)."""
+    _check(lib().dvlm_lmhead_conf_commit_static(ptr(hidden), ptr(w), R, H, V, int(apply_rmsnorm), float(eps),
+                                                ptr(masked), ptr(tokens), float(threshold), ptr(top1_id),
+                                                ptr(top1_prob), ptr(commit), ptr(n_commit), ptr(anchor_id),
+                                                ptr(anchor_conf), ptr(cert_len), ptr(status), stream_handle(stream)),
+           "dvlm_lmhead_conf_commit_static")
 
 
 def spec_workspace_size(b: int, B: int, V: int) -> int:

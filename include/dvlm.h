@@ -139,6 +139,28 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, 
                                     int32_t* cert_len, void* workspace, size_t ws_bytes,
                                     int* dev_status, dvlm_stream stream);
 
+/* Same computation as dvlm_lmhead_conf_commit on the bf16 path, for callers
+ * that cannot allocate device memory when they call it (a process whose
+ * device memory is reserved up front by another framework's caching
+ * allocator; a real-time control loop that forbids cudaMalloc after start-up
+ * because an allocation can synchronise the device).  No counterpart on the
+ * method's pages: this is a deployment variant.  It takes no workspace: its
+ * scratch is one fixed 6 MiB device array inside the library, present on
+ * every GPU that loads the library until the process exits.  Limits: R <= 32
+ * and a scratch layout (about 33 KiB per SM plus 4 bytes per 128 vocabulary
+ * rows) within 6 MiB, e.g. V <= 262144 and H <= 8192 on a 148-SM B200;
+ * larger requests return DVLM_ERR_WORKSPACE and launch nothing.  The first
+ * call on a device looks the array's device address up (make that first call
+ * before any stream capture).  Every call shares the one array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  Allocates nothing; calls no allocating routine. */
+DVLM_API dvlm_status dvlm_lmhead_conf_commit_static(const void* hidden, const void* w, int R, int H, int V,
+                                                   int apply_rmsnorm, float eps, uint8_t* masked,
+                                                   int32_t* tokens, float threshold, int32_t* top1_id,
+                                                   float* top1_prob, uint8_t* commit, int32_t* n_commit,
+                                                   const int32_t* anchor_id, const float* anchor_conf,
+                                                   int32_t* cert_len, int* dev_status, dvlm_stream stream);
+
 /* ------------------------------------------------------------------------
  * Speculative verify + longest-prefix accept + in-place KV truncation.
  *
