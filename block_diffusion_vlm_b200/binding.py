@@ -107,6 +107,9 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_engine_set_position": (_i, [_vp, ctypes.c_int32, ctypes.c_int32, _vp]),
         "dvlm_engine_check": (_i, [_vp, _vp]),
         "dvlm_forward": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+        "dvlm_engine_set_option": (_i, [_vp, ctypes.c_char_p, _i]),
+        "dvlm_engine_get_option": (_i, [_vp, ctypes.c_char_p]),
+        "dvlm_selftest_wait_timeout": (_i, [ctypes.c_longlong, _vp, _vp, _vp]),
         "dvlm_profile_forward": (_i, [_vp, _vp, _vp, _i, _i, _i, ctypes.POINTER(ctypes.c_float),
                                       ctypes.POINTER(_i), _vp]),
     }
@@ -191,6 +194,11 @@ def spec_verify_accept(*, draft_ids, b, B, V, accept_len, verify_logits=None, ve
            "dvlm_spec_verify_accept")
 
 
+def selftest_wait_timeout(budget_cycles: int, status, gave_up, stream=None) -> None:
+    _check(lib().dvlm_selftest_wait_timeout(int(budget_cycles), ptr(status), ptr(gave_up), stream_handle(stream)),
+           "dvlm_selftest_wait_timeout")
+
+
 # ---------------------------------------------------------------- engine
 def make_model(dims, *, embed, wqkv, wo, wgate, wup, wdown, lm_head, dtype) -> Model:
     return Model(dims.n_layers, dims.hidden, dims.n_q_heads, dims.n_kv_heads, dims.head_dim, dims.inter,
@@ -260,6 +268,12 @@ class Engine:
 
     def check(self, stream=None) -> None:
         _check(lib().dvlm_engine_check(self.h, stream_handle(stream)), "dvlm_engine_check (device status)")
+
+    def set_option(self, name: str, value: int) -> None:
+        _check(lib().dvlm_engine_set_option(self.h, name.encode(), int(value)), f"dvlm_engine_set_option({name})")
+
+    def get_option(self, name: str) -> int:
+        return int(lib().dvlm_engine_get_option(self.h, name.encode()))
 
     KERNEL_KINDS = ("embed", "qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head")
 

@@ -18,7 +18,10 @@ cudaError_t engine_collect_stats(dvlm_engine* e, dvlm_stats* st, cudaStream_t s)
 size_t engine_workspace_bytes(dvlm_engine* e, int P);
 size_t engine_carve(dvlm_engine* e, void* ws, int P);
 bool engine_build_maps(dvlm_engine* e);
+void engine_plan(dvlm_engine* e);
 cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* counts, cudaStream_t s);
+dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v);
+int engine_get_option(dvlm_engine* e, const char* name);
 }  // namespace dvlm
 
 namespace {
@@ -165,7 +168,9 @@ dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const
   a.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
   a.out = static_cast<bf16*>(out);
   a.status = dev_status;
-  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream)));
+  static int cs_attn = 0;  // cluster size, chosen once per process
+  if (cs_attn == 0) cs_attn = attn_max_clusters(16) >= 2 ? 16 : 8;
+  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), cs_attn));
 }
 
 // ------------------------------------------------------------ LM head
@@ -330,6 +335,7 @@ dvlm_status dvlm_engine_create(const dvlm_model* m, void* k_cache, void* v_cache
     delete e;
     return DVLM_ERR_CUDA;
   }
+  engine_plan(e);
   *out = e;
   return DVLM_OK;
 }
@@ -544,6 +550,24 @@ dvlm_status dvlm_profile_forward(dvlm_engine* e, const int32_t* tokens, const ui
   f.lma.R = n_rows;
   f.lma.threshold = -1.0f;
   return cuda_status(engine_profile(e, f, ms_out, counts_out, s));
+}
+
+dvlm_status dvlm_selftest_wait_timeout(long long budget_cycles, int* dev_status, int* gave_up,
+                                       dvlm_stream stream) {
+  if (!dev_status || !gave_up) return DVLM_ERR_INVALID_ARG;
+  if (budget_cycles < 1 || budget_cycles > 4000000000LL) return DVLM_ERR_SHAPE;
+  return cuda_status(launch_selftest_timeout(budget_cycles, dev_status, gave_up, cs(stream)));
+}
+
+dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value) {
+  if (!e || !name) return DVLM_ERR_INVALID_ARG;
+  if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+  return engine_set_option(e, name, value);
+}
+
+int dvlm_engine_get_option(dvlm_engine* e, const char* name) {
+  if (!e || !name) return -1;
+  return engine_get_option(e, name);
 }
 
 }  // extern "C"

@@ -11,16 +11,17 @@
 // TMA box lands).  S = Q K^T (N = 64 keys) and O += P V (V stored
 // value-feature-major so both products read K-major operands) accumulate in
 // TMEM; softmax runs in fp32 registers, one thread per row, with P rounded
-// to bf16 for the second product.  The keys are split over an 8-CTA cluster;
-// the partial (max, sum, O) of the 8 CTAs are merged through distributed
-// shared memory, so there is no second kernel and no global scratch.
+// to bf16 for the second product.  The keys are split over a cluster of 8 or 16 CTAs;
+// the partial (max, sum, O) of the cluster's CTAs are merged through
+// distributed shared memory, so there is no second kernel and no global
+// scratch.  Clusters of 16 CTAs (where the device can co-schedule them) put
+// one or two 64-key chunks on each CTA at decode lengths.
 #include "kernels.h"
 #include "mainloop.cuh"
 
 namespace dvlm {
 
 namespace {
-constexpr int kCS = 8;           // CTAs per cluster (key splits)
 constexpr int kChunk = 64;       // keys per chunk
 constexpr int kTmemCols = 256;   // S: 2 x 64 columns, O: 128 columns
 constexpr int kQBytes = 32768;   // 128 rows x 128 d
@@ -30,16 +31,19 @@ constexpr int kPBytes = 16384;   // 128 rows x 64 keys
 constexpr int oQ = 0;
 constexpr int oK = oQ + kQBytes;
 constexpr int oV = oK + 2 * kKBytes;
-constexpr int oP = oV + 2 * kVBytes;
-constexpr int oML = oP + 2 * kPBytes;      // m[128], l[128]
+constexpr int oP = oV + 2 * kVBytes;       // one P buffer
+constexpr int oML = oP + kPBytes;          // m[128], l[128]
 constexpr int oBar = oML + 2 * 128 * 4;
 constexpr int oMisc = oBar + 16 * 8;
+// ~114 KB: fits on an SM next to one projection-GEMM CTA, so the kernel can
+// start (and fetch its cache tiles) while the QKV projection still runs.
 constexpr int kSmem = oMisc + 64 + 1024;
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChunk);
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128);
 }  // namespace
 
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
+template <int kCS>  // CTAs per cluster (key splits)
+__global__ void __launch_bounds__(192, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                      const __grid_constant__ CUtensorMap mapV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -53,11 +57,11 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   float* sL = sM + 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* p_full = bars + 7;     // [2]
-  uint64_t* pv_done = bars + 9;    // [2]
+  uint64_t* kv_full = bars + 1;    // [2] K and V of a chunk landed (stage = chunk & 1)
+  uint64_t* kv_empty = bars + 3;   // [2] PV of the chunk in that stage done
+  uint64_t* s_full = bars + 5;     // [2] S of the chunk in that TMEM buffer ready
+  uint64_t* p_full = bars + 7;     // P of the next chunk written (one phase per chunk)
+  uint64_t* pv_done = bars + 8;    // PV of a chunk done (one phase per chunk)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + oMisc);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + oMisc + 4);
 
@@ -69,7 +73,7 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   const int t_base = (blockIdx.z % n_groups) * 16;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
+    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], i == 7 ? 128 : 1);
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -84,12 +88,14 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_launch_dependents();
-  griddep_wait();
 
+  // The cache length is final before this kernel's predecessor runs (only the
+  // end of a forward pass moves it), and so are the cache slots below it: both
+  // may be read before waiting for the predecessor.  Slots L.. are written by
+  // the QKV projection this kernel follows.
   const int L = a.d_len ? *a.d_len : a.L_static;
   const int Ltot = L + a.n_rows;
-  // Chunk j of 64 keys belongs to CTA j % 8 (round robin): a row's partial
+  // Chunk j of 64 keys belongs to CTA j % kCS (round robin): a row's partial
   // sums then do not depend on how many rows the step has, so a causal row
   // gives bitwise the same output in a 1-row AR pass and a 16-row verify pass.
   const int n_chunks = (Ltot + kChunk - 1) / kChunk;
@@ -99,35 +105,39 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0 && nc > 0) {
       const uint64_t pol = l2_policy_evict_last();
-      mbar_arrive_expect_tx(q_full, kQBytes);
-      for (int h = 0; h < 2; ++h)
-        tma_load_3d(sQ + h * (kQBytes / 2), &mapQ, q_full, h * 64, g * 8, bidx * a.n_rows + t_base, pol);
-      for (int jj = 0; jj < nc; ++jj) {
+      auto load_kv = [&](int jj) {
         const int st = jj & 1;
-        if (jj >= 2 && !mbar_wait(&kv_empty[st], ((jj >> 1) - 1) & 1, a.status, sabort)) break;
-        mbar_arrive_expect_tx(&kv_full[st], kKBytes + kVBytes);
         const int key0 = (crank + kCS * jj) * kChunk;
+        mbar_arrive_expect_tx(&kv_full[st], kKBytes + kVBytes);
         for (int h = 0; h < 2; ++h)
           tma_load_2d(sK + st * kKBytes + h * (kKBytes / 2), &mapK, &kv_full[st], h * 64, kv_row0 * a.Lmax + key0,
                       pol);
         tma_load_2d(sV + st * kVBytes, &mapV, &kv_full[st], key0, kv_row0 * 128, pol);
+      };
+      const int first = nc < 2 ? nc : 2;
+      bool early[2] = {false, false};
+      for (int jj = 0; jj < first; ++jj) {
+        if ((crank + kCS * jj + 1) * kChunk <= L) {  // entirely below the cache length
+          load_kv(jj);
+          early[jj] = true;
+        }
       }
+      griddep_wait();
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      for (int h = 0; h < 2; ++h)
+        tma_load_3d(sQ + h * (kQBytes / 2), &mapQ, q_full, h * 64, g * 8, bidx * a.n_rows + t_base, pol);
+      for (int jj = 0; jj < first; ++jj)
+        if (!early[jj]) load_kv(jj);
+      for (int jj = 2; jj < nc; ++jj) {
+        if (!mbar_wait(&kv_empty[jj & 1], ((jj >> 1) - 1) & 1, a.status, sabort)) break;
+        load_kv(jj);
+      }
+    } else if (lane == 0) {
+      griddep_wait();
     }
   } else if (warp == 1) {
+    griddep_wait();
     if (lane == 0 && nc > 0) {
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&p_full[st], (j >> 1) & 1, a.status, sabort)) return false;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(sP + st * kPBytes), vb = smem_u32(sV + st * kVBytes);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss(tmem + 128, sdesc_kmajor_sw128(pa + 32 * kk), sdesc_kmajor_sw128(vb + 32 * kk), kIdescO,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&pv_done[st]);
-        umma_commit(&kv_empty[st]);
-        return true;
-      };
       bool ok = mbar_wait(q_full, 0, a.status, sabort);
       for (int jj = 0; ok && jj < nc; ++jj) {
         const int st = jj & 1;
@@ -141,12 +151,27 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
                        sdesc_kmajor_sw128(kb + h * (kKBytes / 2) + off), kIdescS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[st]);
-        if (jj >= 1) ok = issue_pv(jj - 1);
+        if ((jj & 1) == 1 || jj == nc - 1) {  // end of a pair of chunks: their PV products
+          for (int c = jj & ~1; ok && c <= jj; ++c) {
+            if (!mbar_wait(p_full, c & 1, a.status, sabort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pa = smem_u32(sP), vb = smem_u32(sV + (c & 1) * kVBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(tmem + 128, sdesc_kmajor_sw128(pa + 32 * kk), sdesc_kmajor_sw128(vb + 32 * kk), kIdescO,
+                           (c > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(pv_done);
+            umma_commit(&kv_empty[c & 1]);
+          }
+        }
       }
-      if (ok) issue_pv(nc - 1);
     }
   } else {
     // ---------------------------------------------------------------- softmax
+    griddep_wait();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int t = t_base + (row >> 3);
@@ -154,59 +179,34 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int jj = 0; jj < nc; ++jj) {
-      const int st = jj & 1;
+    // Writes P of chunk jj (probabilities exp2(s - m_new), bf16) for this row
+    // into the P buffer and, on the last chunk, zeroes the value rows of keys
+    // past the valid slots (they may hold anything, NaN poison included, and
+    // 0 * NaN is NaN).
+    auto emit_p = [&](int jj, const float (&sc)[64], float m_new) -> float {
       const int key0 = (crank + kCS * jj) * kChunk;
-      mbar_wait(&s_full[st], (jj >> 1) & 1, a.status, sabort);
-      named_bar_sync(1, 128);
-      if (*sabort) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[kChunk];
-#pragma unroll
-      for (int c = 0; c < kChunk; c += 16) {
-        float tmp[16];
-        tmem_ld16(tmem + lane_off + static_cast<uint32_t>(st * kChunk + c), tmp);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) s[c + k] = tmp[k];
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        s[c] = (key0 + c < limit) ? s[c] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
-      }
-      const float m_new = fmaxf(m, mx);
-      float alpha = 1.0f, psum = 0.f;
       uint32_t packed[kChunk / 2];
+      float psum = 0.f;
       if (m_new == -INFINITY) {
 #pragma unroll
         for (int c = 0; c < kChunk / 2; ++c) packed[c] = 0u;
       } else {
-        alpha = exp2f(m - m_new);
 #pragma unroll
         for (int c = 0; c < kChunk; c += 2) {
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(s[c] - m_new), exp2f(s[c + 1] - m_new));
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(sc[c] - m_new), exp2f(sc[c + 1] - m_new));
           const float2 pf = __bfloat1622float2(pb);
           psum += pf.x + pf.y;
           packed[c / 2] = *reinterpret_cast<const uint32_t*>(&pb);
         }
       }
-      l = l * alpha + psum;
-      // P buffer st is free once PV of chunk jj-2 has completed.
-      if (jj >= 2) mbar_wait(&pv_done[st], ((jj >> 1) - 1) & 1, a.status, sabort);
-      uint8_t* prow = sP + st * kPBytes + row * 128;
+      uint8_t* prow = sP + row * 128;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         const uint4 w = make_uint4(packed[cc * 4 + 0], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
         *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) = w;
       }
-      // Keys past the end of the valid slots may hold anything (NaN poison
-      // included); P is exactly 0 there, but 0 * NaN is NaN, so the value
-      // rows of those keys are zeroed before the PV product reads them.
       if (key0 + kChunk > Ltot) {
+        const int st = jj & 1;
         mbar_wait(&kv_full[st], (jj >> 1) & 1, a.status, sabort);
         uint8_t* vrow = sV + st * kVBytes + row * 128;  // value feature `row`, 64 keys
         const int valid = Ltot - key0;
@@ -217,44 +217,94 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
             if (8 * cc + e >= valid) chunk[e] = 0;
         }
       }
-      // tcgen05.ld/st are warp-collective: the rescale runs for the whole warp
-      // when any of its rows needs it (alpha == 1 leaves a row unchanged).
-      if (jj >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, a.status, sabort);
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 128; c += 16) {
-          float o[16];
-          tmem_ld16(tmem + lane_off + 128u + c, o);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[k] *= alpha;
-          tmem_st16(tmem + lane_off + 128u + c, o);
-        }
-      }
-      m = m_new;
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[st]);
+      mbar_arrive(p_full);
+      return psum;
+    };
+    auto load_scores = [&](int jj, float (&sc)[64]) -> float {
+      const int key0 = (crank + kCS * jj) * kChunk;
+      tmem_ld64(tmem + lane_off + static_cast<uint32_t>((jj & 1) * kChunk), sc);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c) {
+        sc[c] = (key0 + c < limit) ? sc[c] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[c]);
+      }
+      return mx;
+    };
+    for (int jj0 = 0; jj0 < nc; jj0 += 2) {
+      const bool two = jj0 + 1 < nc;
+      mbar_wait(&s_full[0], (jj0 >> 1) & 1, a.status, sabort);
+      if (two) mbar_wait(&s_full[1], (jj0 >> 1) & 1, a.status, sabort);
+      named_bar_sync(1, 128);
+      if (*sabort) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // Pass 1: row maxima of the pair (scores re-read from TMEM in pass 2,
+      // so at most one chunk's scores occupy registers at a time).
+      float mx;
+      {
+        float sc[64];
+        mx = load_scores(jj0, sc);
+        if (two) mx = fmaxf(mx, load_scores(jj0 + 1, sc));
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m - m_new);
+      if (jj0 > 0) {
+        // the previous pair's products are complete: O is stable, P is free
+        mbar_wait(pv_done, (jj0 - 1) & 1, a.status, sabort);
+        tc_fence_after();
+        // tcgen05.ld/st are warp-collective: rescale the whole warp when any
+        // of its rows needs it (alpha == 1 leaves a row unchanged)
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 64) {
+            float o[64];
+            tmem_ld64(tmem + lane_off + 128u + c, o);
+#pragma unroll
+            for (int k = 0; k < 64; ++k) o[k] *= alpha;
+#pragma unroll
+            for (int k = 0; k < 64; k += 16) tmem_st16_nowait(tmem + lane_off + 128u + c + k, o + k);
+            tmem_wait_st();
+          }
+        }
+      }
+      // Pass 2: probabilities of each chunk into the P buffer.
+      float psum;
+      {
+        float sc[64];
+        load_scores(jj0, sc);
+        psum = emit_p(jj0, sc, m_new);
+      }
+      if (two) {
+        mbar_wait(pv_done, jj0 & 1, a.status, sabort);  // P buffer free again
+        float sc[64];
+        load_scores(jj0 + 1, sc);
+        psum += emit_p(jj0 + 1, sc, m_new);
+      }
+      l = l * alpha + psum;
+      m = m_new;
     }
     // Final PV done -> unnormalised partial O of this CTA into shared memory
     // (the K/V stages are free by then).
-    if (ok && nc > 0) {
-      mbar_wait(&pv_done[(nc - 1) & 1], ((nc - 1) >> 1) & 1, a.status, sabort);
-    }
+    if (ok && nc > 0) mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort);
     named_bar_sync(1, 128);
     const bool have = ok && nc > 0 && !*sabort;
     if (have) tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < 128; c += 16) {
-      float o[16];
+    for (int c = 0; c < 128; c += 64) {
+      float o[64];
       if (have) {
-        tmem_ld16(tmem + lane_off + 128u + c, o);
+        tmem_ld64(tmem + lane_off + 128u + c, o);
       } else {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = 0.f;
+        for (int k = 0; k < 64; ++k) o[k] = 0.f;
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) sO[row * 128 + ((c + k + 4 * row) & 127)] = o[k];
+      for (int k = 0; k < 64; ++k) sO[row * 128 + ((c + k + 4 * row) & 127)] = o[k];
     }
     sM[row] = have ? m : -INFINITY;
     sL[row] = have ? l : 0.f;
@@ -262,49 +312,72 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   tc_fence_before();
   cluster_sync();
   // ---------------------------------------------------------------- merge
-  // CTA `crank` combines rows [crank*16, crank*16+16) over the 8 partials.
+  // CTA `crank` combines rows [crank*RPC, (crank+1)*RPC) over the kCS partials.
   if (threadIdx.x >= 64) {
+    constexpr int RPC = 128 / kCS;  // rows per CTA
+    constexpr int TPR = 128 / RPC;  // threads per row
+    constexpr int DPT = 128 / TPR;  // value features per thread
     const int et = threadIdx.x - 64;
-    const int r = crank * (128 / kCS) + et / 8;
-    const int d0 = (et % 8) * 16;
+    const int r = crank * RPC + et / TPR;
+    const int d0 = (et % TPR) * DPT;
     const int t = t_base + (r >> 3), hl = r & 7;
-    float ms[kCS], M = -INFINITY;
+    // Maxima and sums of all partials first, then the partial outputs four
+    // sources at a time (all loads of a group in flight together).
+    float ms[kCS], ls[kCS];
+#pragma unroll
     for (int s2 = 0; s2 < kCS; ++s2) {
       ms[s2] = ld_dsmem_f32(map_to_cta(smem_u32(&sM[r]), s2));
-      M = fmaxf(M, ms[s2]);
+      ls[s2] = ld_dsmem_f32(map_to_cta(smem_u32(&sL[r]), s2));
     }
-    float acc[16];
+    float M = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (int s2 = 0; s2 < kCS; ++s2) M = fmaxf(M, ms[s2]);
+    float acc[DPT];
+#pragma unroll
+    for (int k = 0; k < DPT; ++k) acc[k] = 0.f;
     float lsum = 0.f;
     if (M != -INFINITY) {
-      for (int s2 = 0; s2 < kCS; ++s2) {
-        if (ms[s2] == -INFINITY) continue;
-        const float w = exp2f(ms[s2] - M);
-        lsum += w * ld_dsmem_f32(map_to_cta(smem_u32(&sL[r]), s2));
 #pragma unroll
-        for (int k = 0; k < 16; k += 4) {
-          // rows are stored rotated by 4*row floats (bank spread); undo it
-          const int col = (d0 + k + 4 * r) & 127;
-          const float4 f = ld_dsmem_f32x4(map_to_cta(smem_u32(&sO[r * 128 + col]), s2));
-          acc[k] += w * f.x;
-          acc[k + 1] += w * f.y;
-          acc[k + 2] += w * f.z;
-          acc[k + 3] += w * f.w;
+      for (int g0 = 0; g0 < kCS; g0 += 4) {
+        float4 ov[4][DPT / 4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int k = 0; k < DPT / 4; ++k) {
+            // rows are stored rotated by 4*row floats (bank spread); undo it
+            const int col = (d0 + 4 * k + 4 * r) & 127;
+            ov[q][k] = ld_dsmem_f32x4(map_to_cta(smem_u32(&sO[r * 128 + col]), g0 + q));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int s2 = g0 + q;
+          if (ms[s2] == -INFINITY) continue;
+          const float w = exp2f(ms[s2] - M);
+          lsum += w * ls[s2];
+#pragma unroll
+          for (int k = 0; k < DPT / 4; ++k) {
+            acc[4 * k] += w * ov[q][k].x;
+            acc[4 * k + 1] += w * ov[q][k].y;
+            acc[4 * k + 2] += w * ov[q][k].z;
+            acc[4 * k + 3] += w * ov[q][k].w;
+          }
         }
       }
     }
     if (t < a.n_rows) {
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
       bf16* dst = a.out + ((static_cast<size_t>(bidx) * a.n_rows + t) * a.Hq + g * 8 + hl) * 128 + d0;
-      uint32_t w[8];
 #pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
-        w[k / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+      for (int k = 0; k < DPT; k += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 8; q += 2) {
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(acc[k + q] * inv, acc[k + q + 1] * inv);
+          w[q / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+        }
+        reinterpret_cast<uint4*>(dst + k)[0] = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
   cluster_sync();
@@ -314,26 +387,68 @@ __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
-cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                             const AttnArgs& a, bool pdl, cudaStream_t s) {
+template <int CS>
+static cudaError_t attn_launch(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                               const AttnArgs& a, bool pdl, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
+    if (CS > 8) {
+      e = cudaFuncSetAttribute(attn_bf16_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
   const int n_groups = (a.n_rows + 15) / 16;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kCS, a.Hkv, a.n_batch * n_groups);
+  cfg.gridDim = dim3(CS, a.Hkv, a.n_batch * n_groups);
   cfg.blockDim = dim3(192);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, attn_bf16_kernel<CS>, mapQ, mapK, mapV, a);
+}
+
+cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                             const AttnArgs& a, bool pdl, cudaStream_t s, int cs) {
+  if (cs == 16) return attn_launch<16>(mapQ, mapK, mapV, a, pdl, s);
+  return attn_launch<8>(mapQ, mapK, mapV, a, pdl, s);
+}
+
+// Clusters of cs CTAs that can be resident at once (0: cannot launch).
+int attn_max_clusters(int cs) {
+  auto kern = cs == 16 ? attn_bf16_kernel<16> : attn_bf16_kernel<8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess ||
+      (cs > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, 2, 1);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_bf16_kernel, mapQ, mapK, mapV, a);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 }  // namespace dvlm

@@ -13,6 +13,7 @@
 //   AR: one causal row per pass (the comparator).
 #include <cmath>
 #include <cstring>
+#include <string>
 
 #include "engine.h"
 #include "ptx.cuh"
@@ -22,8 +23,8 @@ using namespace dvlm;
 namespace dvlm {
 
 __global__ void advance_kernel(int32_t* d_len, int n) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) *d_len += n;
 }
 
@@ -62,7 +63,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->attn_o = c.take<void>(kNT * HD * es);
   e->act = c.take<void>(static_cast<size_t>(kNT) * I * es);
   e->ssq = c.take<float>((H / 128 + 1) * kNT * 4);
-  e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, P));
+  e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, 2 * P));  // up to two CTAs per SM
   e->gcnt = c.take<int>(num_tiles_max(m) * 4);
   e->lpart = c.take<float>(static_cast<size_t>(P) * 2 * kNT * 128 * 4);
   e->lcnt = c.take<int>(((m.vocab + 127) / 128) * 4);
@@ -138,7 +139,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   const dvlm_model& m = e->m;
   const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
   const int qkv_rows = (Hq + 2 * Hkv) * D;
-  const bool pdl = true;
+  const bool pdl = e->pdl;
   bf16* x = static_cast<bf16*>(e->x);
   KernelTimer* tm = f.timer;
   auto T0 = [&](int k) { if (tm) tm->begin(k); };
@@ -171,8 +172,12 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
     ea.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
     T0(K_QKV);
-    DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
-                           ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s));
+    if (e->s_qkv > 0)
+      DVLM_CK(launch_gemm_cl(kNT, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, e->s_qkv, l * qkv_rows, ea, pdl, s,
+                             5));
+    else
+      DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
+                             ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s, 5));
     T1(K_QKV);
     AttnArgs aa{};
     aa.n_rows = f.n_rows;
@@ -187,27 +192,37 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     aa.out = static_cast<bf16*>(e->attn_o);
     aa.status = e->d_status;
     T0(K_ATTN);
-    DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s));
+    DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s, e->attn_cs));
     T1(K_ATTN);
     ea.epi = EPI_RESID;
     ea.resid = x;
     ea.resid_ld = H;
     ea.ssq_out = e->ssq;
     T0(K_OPROJ);
-    DVLM_CK(launch_gemm_ws(kNT, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64,
-                           ws_ctas(e, (H / 128) * (Hq * D / 64)), l * H, ea, pdl, s));
+    if (e->s_o > 0)
+      DVLM_CK(launch_gemm_cl(kNT, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, e->s_o, l * H, ea, pdl, s, 5));
+    else
+      DVLM_CK(launch_gemm_ws(kNT, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64,
+                             ws_ctas(e, (H / 128) * (Hq * D / 64)), l * H, ea, pdl, s, 5));
     T1(K_OPROJ);
     ea.epi = EPI_SWIGLU;
     ea.out = static_cast<bf16*>(e->act);
     ea.out_ld = I;
     T0(K_GATEUP);
-    DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, ws_ctas(e, (I / 64) * (H / 64)),
-                           l * I, ea, pdl, s));
+    // 10 stages: one CTA per SM; 5 stages: two per SM (same bytes in flight)
+    const long long gu_units = static_cast<long long>(I / 64) * (H / 64);
+    const int gu_ctas = static_cast<int>(std::min<long long>(gu_units, (e->gu_stages == 5 ? 2LL : 1LL) * e->sm));
+    DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, gu_ctas,
+                           l * I, ea, pdl, s, e->gu_stages));
     T1(K_GATEUP);
     ea.epi = EPI_RESID;
     T0(K_DOWN);
-    DVLM_CK(launch_gemm_ws(kNT, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, ws_ctas(e, (H / 128) * (I / 64)),
-                           l * H, ea, pdl, s));
+    if (e->s_down > 0)
+      DVLM_CK(launch_gemm_cl(kNT, e->tm_wd, e->tm_act, H / 128, I / 64, e->s_down, l * H, ea, pdl, s,
+                             e->down_stages));
+    else
+      DVLM_CK(launch_gemm_ws(kNT, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64,
+                             ws_ctas(e, (H / 128) * (I / 64)), l * H, ea, pdl, s, e->down_stages));
     T1(K_DOWN);
   }
   if (f.x_out) DVLM_CK(cudaMemcpyAsync(f.x_out, x, static_cast<size_t>(f.n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
@@ -488,8 +503,77 @@ cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* co
   return err;
 }
 
+// Tuning knobs (cluster sizes, pipeline depths, PDL); invalidates captured graphs.
+dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
+  const dvlm_model& m = e->m;
+  const std::string n(name);
+  auto cluster_ok = [&](int epi, int S, int stages) {
+    return S == 0 || (S >= 2 && S <= 16 && gemm_cl_max_clusters(epi, S, stages) > 0);
+  };
+  if (n == "qkv_cluster") {
+    if (!cluster_ok(EPI_QKV, v, 5) || v > m.hidden / 64) return DVLM_ERR_UNSUPPORTED;
+    e->s_qkv = v;
+  } else if (n == "o_cluster") {
+    if (!cluster_ok(EPI_RESID, v, 5) || v > m.n_q_heads * m.head_dim / 64) return DVLM_ERR_UNSUPPORTED;
+    e->s_o = v;
+  } else if (n == "down_cluster") {
+    if (!cluster_ok(EPI_RESID, v, e->down_stages) || v > m.inter / 64) return DVLM_ERR_UNSUPPORTED;
+    e->s_down = v;
+  } else if (n == "down_stages") {
+    if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
+    if (e->s_down > 0 && gemm_cl_max_clusters(EPI_RESID, e->s_down, v) <= 0) return DVLM_ERR_UNSUPPORTED;
+    e->down_stages = v;
+  } else if (n == "gateup_stages") {
+    if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
+    e->gu_stages = v;
+  } else if (n == "attn_cluster") {
+    if (v != 8 && v != 16) return DVLM_ERR_SHAPE;
+    if (attn_max_clusters(v) <= 0) return DVLM_ERR_UNSUPPORTED;
+    e->attn_cs = v;
+  } else if (n == "pdl") {
+    e->pdl = v != 0;
+  } else {
+    return DVLM_ERR_INVALID_ARG;
+  }
+  for (auto& kv : e->graphs) cudaGraphExecDestroy(kv.second);
+  e->graphs.clear();
+  return DVLM_OK;
+}
+
+int engine_get_option(dvlm_engine* e, const char* name) {
+  const std::string n(name);
+  if (n == "qkv_cluster") return e->s_qkv;
+  if (n == "o_cluster") return e->s_o;
+  if (n == "down_cluster") return e->s_down;
+  if (n == "down_stages") return e->down_stages;
+  if (n == "gateup_stages") return e->gu_stages;
+  if (n == "attn_cluster") return e->attn_cs;
+  if (n == "pdl") return e->pdl ? 1 : 0;
+  return -1;
+}
+
 size_t engine_workspace_bytes(dvlm_engine* e, int P) { return carve(e, nullptr, true, P); }
 size_t engine_carve(dvlm_engine* e, void* ws, int P) { return carve(e, static_cast<uint8_t*>(ws), false, P); }
 bool engine_build_maps(dvlm_engine* e) { return build_maps(e); }
+
+// Cluster size for a projection with n_tiles output tiles: the largest S with
+// n_tiles * S <= SMs whose clusters can all be resident at once (0: use the
+// stream-K kernel instead).
+static int pick_cluster(dvlm_engine* e, int epi, int n_tiles, int kb, int stages) {
+  for (int S = std::min(16, std::min(kb, e->sm / std::max(1, n_tiles))); S >= 2; --S)
+    if (gemm_cl_max_clusters(epi, S, stages) >= n_tiles) return S;
+  return 0;
+}
+
+void engine_plan(dvlm_engine* e) {
+  if (!e->bf16) return;
+  const dvlm_model& m = e->m;
+  const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
+  e->s_qkv = pick_cluster(e, EPI_QKV, qkv_rows / 128, m.hidden / 64, 5);
+  e->s_o = pick_cluster(e, EPI_RESID, m.hidden / 128, m.n_q_heads * m.head_dim / 64, 5);
+  e->s_down = pick_cluster(e, EPI_RESID, m.hidden / 128, m.inter / 64, e->down_stages);
+  // 16-CTA attention clusters when one per KV head can be resident at once
+  e->attn_cs = attn_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
+}
 
 }  // namespace dvlm

@@ -30,11 +30,6 @@ struct GemmSmem {
   static constexpr int kTotal = kMisc + 64 + 1024;  // + alignment slack
 };
 
-template <int NT>
-struct StagesFor {
-  static constexpr int value = NT <= 16 ? 5 : 4;
-};
-
 template <int NT, int STAGES, int EPI>
 __global__ void __launch_bounds__(kWsThreads, 2)
     gemm_ws_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
@@ -82,7 +77,6 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
@@ -96,6 +90,9 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     const int row = quarter * 32 + lane;  // accumulator row = output feature within the tile
     const int et = threadIdx.x - 64;      // 0..127
     griddep_wait();
+    // Dependents may start only once this kernel's own inputs are complete,
+    // so at most two kernels of the chain overlap (see ptx.cuh).
+    if (et == 0) griddep_launch_dependents();
     if (EPI != EPI_RESID) {
       if (et < NT) {
         float s = 0.f;
@@ -232,10 +229,197 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   }
 }
 
-template <int NT, int EPI>
+// ---------------------------------------------------------------------------
+// Cluster split-K variant for the narrow projections (QKV, O-proj, down):
+// one output tile per cluster of S CTAs, CTA c streaming the contiguous k
+// range [c*kb/S, (c+1)*kb/S).  The S fp32 partial tiles meet in distributed
+// shared memory and every CTA finishes a slice of the tile's rows, summing
+// the partials in rank order (deterministic; each token column's arithmetic
+// is independent of how many rows the step has).
+template <int NT, int STAGES>
+struct ClSmem {
+  static constexpr int kA = 0;
+  static constexpr int kB = kA + STAGES * kATileBytes;
+  static constexpr int kP = kB + STAGES * NT * 128;     // partial [128][NT+1]
+  static constexpr int kQ = kP + 128 * (NT + 1) * 4;     // squares [128][NT+1] (residual epilogue)
+  static constexpr int kS = kQ + 128 * (NT + 1) * 4;     // slice sums of squares [NT]
+  static constexpr int kR = kS + 32 * 4;                 // rmsnorm factors [NT]
+  static constexpr int kBar = kR + 32 * 4;
+  static constexpr int kMisc = kBar + (2 * STAGES + 4) * 8;
+  static constexpr int kTotal = kMisc + 64 + 1024;
+};
+
+template <int NT, int STAGES, int EPI>
+__global__ void __launch_bounds__(kWsThreads, 2)
+    gemm_cl_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const int kb,
+                   const int S, const int a_row_base, const GemmEpi ea) {
+  using Sm = ClSmem<NT, STAGES>;
+  constexpr int TMC = tmem_cols_for<NT>();
+  constexpr int PS = NT + 1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem + Sm::kA;
+  uint8_t* sB = smem + Sm::kB;
+  float* sP = reinterpret_cast<float*>(smem + Sm::kP);
+  float* sQ = reinterpret_cast<float*>(smem + Sm::kQ);
+  float* sS = reinterpret_cast<float*>(smem + Sm::kS);
+  float* sR = reinterpret_cast<float*>(smem + Sm::kR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kBar);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Sm::kMisc);
+  volatile int* sabort = reinterpret_cast<volatile int*>(smem + Sm::kMisc + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = static_cast<int>(cluster_ctarank());
+  const int T = blockIdx.x / S;
+  const SkSched sc{static_cast<int>(gridDim.x) / S, kb, 1};
+  const long long u0 = static_cast<long long>(T) * kb + static_cast<long long>(c) * kb / S;
+  const long long u1 = static_cast<long long>(T) * kb + static_cast<long long>(c + 1) * kb / S;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    *sabort = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mapA);
+    tma_prefetch_map(&mapB);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMC);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int et = threadIdx.x - 64;  // epilogue thread 0..127 (warps 2..5)
+  if (warp == 0) {
+    if (lane == 0 && u1 > u0)
+      ws_producer<NT, STAGES, false>(&mapA, &mapA, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base, 0, ea.status,
+                                     sabort);
+  } else if (warp == 1) {
+    if (lane == 0 && u1 > u0) ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort);
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    griddep_wait();
+    // Dependents may start only once this kernel's own inputs are complete,
+    // so at most two kernels of the chain overlap (see ptx.cuh).
+    if (et == 0) griddep_launch_dependents();
+    if (EPI == EPI_QKV && et < NT) {
+      float s2 = 0.f;
+      for (int p = 0; p < ea.n_ssq; ++p) s2 += ea.ssq_in[p * NT + et];
+      sR[et] = 1.0f / sqrtf(s2 * ea.inv_h + ea.eps);
+    }
+    float v[NT];
+    if (u1 > u0) {
+      mbar_wait(&accf[0], 0, ea.status, sabort);
+      tc_fence_after();
+      ws_load_acc<NT>(tmem, 0, quarter, v);
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) v[t] = 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) sP[row * PS + t] = v[t];
+  }
+  tc_fence_before();
+  cluster_sync();  // partials of every CTA of the tile are visible
+
+  if (threadIdx.x >= 64) {
+    uint32_t rp[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) rp[q] = q < S ? map_to_cta(smem_u32(sP), q) : 0u;
+    // Sum of the S partials of element (r, t), in rank order; all S loads
+    // are issued before the first add.
+    auto part_sum = [&](int r, int t) {
+      const uint32_t off = 4u * static_cast<uint32_t>(r * PS + t);
+      float vals[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) vals[q] = q < S ? ld_dsmem_f32(rp[q] + off) : 0.f;
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < S) acc += vals[q];
+      return acc;
+    };
+    if (EPI == EPI_RESID) {
+      const int r0 = c * 128 / S, r1 = (c + 1) * 128 / S;
+      const int nr = r1 - r0;
+      for (int it = et; it < nr * NT; it += 128) {
+        const int r = r0 + it / NT, t = it % NT;
+        const float y = part_sum(r, t);
+        float sq = 0.f;
+        if (t < ea.n_rows) {
+          bf16* px = ea.resid + static_cast<size_t>(t) * ea.resid_ld + T * 128 + r;
+          const float xn = bf16_round_f(__bfloat162float(*px) + y);
+          *px = __float2bfloat16_rn(xn);
+          sq = xn * xn;
+        }
+        sQ[r * PS + t] = sq;
+      }
+      named_bar_sync(1, 128);
+      if (et < NT) {
+        float s2 = 0.f;
+        for (int r = r0; r < r1; ++r) s2 += sQ[r * PS + et];
+        sS[et] = s2;
+      }
+    } else {  // EPI_QKV: pairs (j, j+64) of one head per tile
+      const int p0 = c * 64 / S, p1 = (c + 1) * 64 / S;
+      const int np = p1 - p0;
+      const int nq = ea.n_q_heads, nkv = ea.n_kv_heads;
+      const int L0 = ea.d_len ? *ea.d_len : ea.L_static;
+      for (int it = et; it < np * NT; it += 128) {
+        const int j = p0 + it / NT, t = it % NT;
+        const float x1 = part_sum(j, t) * sR[t];
+        const float x2 = part_sum(j + 64, t) * sR[t];
+        if (t >= ea.n_rows) continue;
+        if (T < nq + nkv) {
+          const double inv_freq = exp2(-(2.0 * j / 128.0) * ea.log2_rope_base);
+          double sn, cs;
+          sincos(static_cast<double>(L0 + t) * inv_freq, &sn, &cs);
+          const float co = static_cast<float>(cs), si = static_cast<float>(sn);
+          const bf16 y1 = __float2bfloat16_rn(x1 * co - x2 * si);
+          const bf16 y2 = __float2bfloat16_rn(x2 * co + x1 * si);
+          bf16* dst = (T < nq) ? ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128
+                               : ea.kcache + (static_cast<size_t>(T - nq) * ea.Lmax + (L0 + t)) * 128;
+          dst[j] = y1;
+          dst[j + 64] = y2;
+        } else {
+          const int h = T - nq - nkv;
+          ea.vcache[(static_cast<size_t>(h) * 128 + j) * ea.Lmax + (L0 + t)] = __float2bfloat16_rn(x1);
+          ea.vcache[(static_cast<size_t>(h) * 128 + j + 64) * ea.Lmax + (L0 + t)] = __float2bfloat16_rn(x2);
+        }
+      }
+    }
+  }
+  if (EPI == EPI_RESID) {
+    cluster_sync();  // slice sums visible
+    if (c == 0 && threadIdx.x >= 64 && et < NT) {
+      float s2 = 0.f;
+      for (int q = 0; q < S; ++q) s2 += ld_dsmem_f32(map_to_cta(smem_u32(&sS[et]), q));
+      ea.ssq_out[T * NT + et] = s2;
+    }
+  }
+  cluster_sync();  // no CTA leaves while another still reads its shared memory
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMC);
+  }
+}
+
+template <int NT, int ST, int EPI>
 static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
                               const SkSched& sc, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
-  constexpr int ST = StagesFor<NT>::value;
   using S = GemmSmem<NT, ST>;
   auto kern = gemm_ws_kernel<NT, ST, EPI>;
   static bool attr_set = false;
@@ -257,22 +441,101 @@ static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2,
   return cudaLaunchKernelEx(&cfg, kern, mapA, mapA2, mapB, sc, a_row_base, ea);
 }
 
+template <int NT, int ST, int EPI>
+static cudaError_t launch_cl(const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
+                             int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
+  using Sm = ClSmem<NT, ST>;
+  auto kern = gemm_cl_kernel<NT, ST, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tiles * S);
+  cfg.blockDim = dim3(kWsThreads);
+  cfg.dynamicSmemBytes = Sm::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = S;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, mapA, mapB, kb, S, a_row_base, ea);
+}
+
+cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
+                           int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s, int stages) {
+  if (S < 1 || S > 16 || NT != 16) return cudaErrorInvalidValue;
+  if (stages == 5) {
+    if (ea.epi == EPI_QKV) return launch_cl<16, 5, EPI_QKV>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);
+    if (ea.epi == EPI_RESID) return launch_cl<16, 5, EPI_RESID>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);
+  }
+  if (stages == 10) {
+    if (ea.epi == EPI_QKV) return launch_cl<16, 10, EPI_QKV>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);
+    if (ea.epi == EPI_RESID) return launch_cl<16, 10, EPI_RESID>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// Clusters of S CTAs of the cluster split-K kernel that can be resident at
+// once (0: that cluster size cannot be launched).
+template <int ST>
+static int cl_max_clusters(int epi, int S) {
+  using Sm = ClSmem<16, ST>;
+  auto kern = epi == EPI_QKV ? gemm_cl_kernel<16, ST, EPI_QKV> : gemm_cl_kernel<16, ST, EPI_RESID>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S * 16);
+  cfg.blockDim = dim3(kWsThreads);
+  cfg.dynamicSmemBytes = Sm::kTotal;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int gemm_cl_max_clusters(int epi, int S, int stages) {
+  return stages == 10 ? cl_max_clusters<10>(epi, S) : cl_max_clusters<5>(epi, S);
+}
+
 size_t gemm_ws_part_bytes(int NT, int P) { return static_cast<size_t>(P) * 2 * NT * 128 * sizeof(float); }
 
 cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
-                           int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl,
-                           cudaStream_t s) {
+                           int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s,
+                           int stages) {
   SkSched sc{n_tiles, kb, P};
-#define DVLM_GEMM_CASE(nt)                                                                       \
-  if (NT == nt) {                                                                                \
-    switch (ea.epi) {                                                                            \
-      case EPI_QKV: return launch_one<nt, EPI_QKV>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s);       \
-      case EPI_RESID: return launch_one<nt, EPI_RESID>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s);   \
-      case EPI_SWIGLU: return launch_one<nt, EPI_SWIGLU>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s); \
-    }                                                                                            \
+#define DVLM_GEMM_CASE(nt, st)                                                                         \
+  if (NT == nt && stages == st) {                                                                      \
+    switch (ea.epi) {                                                                                  \
+      case EPI_QKV: return launch_one<nt, st, EPI_QKV>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s);       \
+      case EPI_RESID: return launch_one<nt, st, EPI_RESID>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s);   \
+      case EPI_SWIGLU: return launch_one<nt, st, EPI_SWIGLU>(mapA, mapA2, mapB, sc, a_row_base, ea, pdl, s); \
+    }                                                                                                  \
   }
-  DVLM_GEMM_CASE(16)
-  DVLM_GEMM_CASE(32)
+  DVLM_GEMM_CASE(16, 5)
+  DVLM_GEMM_CASE(16, 10)
+  DVLM_GEMM_CASE(32, 4)
 #undef DVLM_GEMM_CASE
   return cudaErrorInvalidValue;
 }

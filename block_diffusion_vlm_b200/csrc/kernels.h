@@ -83,9 +83,15 @@ struct Launch {
 };
 
 int device_sm_count();
+// stages: 5 (two CTAs per SM) or 10 (one CTA per SM, deeper stream) for NT=16; 4 for NT=32.
 cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
-                           int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s);
+                           int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s,
+                           int stages);
 size_t gemm_ws_part_bytes(int NT, int P);
+// Cluster split-K (one tile per cluster of S CTAs; QKV and residual epilogues).
+cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
+                           int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s, int stages);
+int gemm_cl_max_clusters(int epi, int S, int stages);
 cudaError_t launch_lmhead(int NT, const CUtensorMap& mapW, const CUtensorMap& mapH, int n_tiles, int kb, int P,
                           const LmArgs& a, bool pdl, cudaStream_t s);
 size_t lmhead_scratch_bytes(int NT, int P, int n_tiles);
@@ -101,8 +107,11 @@ struct AttnArgs {
   bf16* out;                 // [n_batch][n_rows][Hq][128]
   int* status;
 };
+// cs: CTAs per cluster splitting the keys (8, or 16 where the device can
+// co-schedule 16-CTA clusters; see attn_cluster_size()).
 cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                             const AttnArgs& a, bool pdl, cudaStream_t s);
+                             const AttnArgs& a, bool pdl, cudaStream_t s, int cs = 8);
+int attn_max_clusters(int cs);
 
 // Embedding gather / row copy + per-128-feature sums of squares.
 cudaError_t launch_embed_bf16(const bf16* E, const bf16* rows_in, int n_src, const int32_t* tokens,
@@ -120,6 +129,8 @@ cudaError_t launch_spec_ids(const int32_t* vids, const int32_t* draft, int b, in
 cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len,
                                  int32_t* seed, int32_t* out, int32_t* n_out, int max_new, int64_t* accept_hist,
                                  int* status, bool pdl, cudaStream_t s);
+// Failure-detection self-test of the bounded waits.
+cudaError_t launch_selftest_timeout(long long budget, int* status, int* waited_out, cudaStream_t s);
 // Block bookkeeping for the decode driver.
 cudaError_t launch_block_init(int32_t* tokens, uint8_t* masked, const int32_t* seed, int B, int mask_id,
                               int ar_seed, int32_t* n_remaining, cudaStream_t s);

@@ -14,7 +14,9 @@ namespace dvlm {
 
 template <int NT>
 struct LmCfg {
-  static constexpr int STAGES = NT <= 32 ? (NT <= 16 ? 5 : 4) : (NT <= 64 ? 4 : 4);
+  // Bytes in flight per SM bound a streaming kernel at batch 1: one CTA per
+  // SM keeps 160-180 KB of weight tiles in flight for the narrow row counts.
+  static constexpr int STAGES = NT <= 16 ? 10 : (NT <= 32 ? 9 : 4);
   static constexpr int TPT = 128 / NT;     // scan threads per token
   static constexpr int SROW = 128 + TPT;   // padded row of the transposed tile (bank-conflict free)
   static constexpr int kA = 0;
@@ -109,7 +111,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
@@ -123,6 +124,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const int tok = et / TPT, sub = et % TPT;
     auto bar = [] { named_bar_sync(1, 128); };
     griddep_wait();
+    // Dependents may start only once this kernel's own inputs are complete,
+    // so at most two kernels of the chain overlap (see ptx.cuh).
+    if (et == 0) griddep_launch_dependents();
     float rt = 1.0f;  // final RMSNorm factor of this thread's token
     if (a.ssq_in) {
       float s = 0.f;

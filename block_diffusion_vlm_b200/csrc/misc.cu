@@ -16,8 +16,8 @@ __global__ void embed_bf16_kernel(const bf16* __restrict__ E, const bf16* __rest
                                   const int32_t* __restrict__ tokens, const uint8_t* __restrict__ masked,
                                   int mask_id, int H, int V, bf16* __restrict__ x, float* __restrict__ ssq_out,
                                   int NT, int* status) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bf16* src;
@@ -85,8 +85,8 @@ cudaError_t launch_block_init(int32_t* tokens, uint8_t* masked, const int32_t* s
 
 // Append n tokens to the output (capped at max_new) and advance its count.
 __global__ void emit_kernel(const int32_t* tokens, int n, int32_t* out, int32_t* n_out, int max_new) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   const int base = *n_out;
   for (int j = threadIdx.x; j < n; j += blockDim.x)
     if (base + j < max_new) out[base + j] = tokens[j];
@@ -118,8 +118,8 @@ cudaError_t launch_emit(const int32_t* tokens, int n, int32_t* out, int32_t* n_o
 __global__ void decode_accept_kernel(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len,
                                      int32_t* seed, int32_t* out, int32_t* n_out, int max_new,
                                      int64_t* accept_hist, int* status) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x != 0) return;
   int k = 1;
   while (k < B && vids[k] == draft[k]) ++k;
@@ -145,6 +145,28 @@ cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int 
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_accept_kernel, vids, draft, B, d_len, seed, out, n_out, max_new,
                             accept_hist, status);
+}
+
+// Failure-detection self-test: an mbarrier that expects two arrivals gets
+// one, so its phase never completes; the bounded wait must give up after
+// `budget` cycles, record DVLM_ERR_TIMEOUT and let the kernel finish.
+__global__ void selftest_timeout_kernel(long long budget, int* status, int* waited_out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 2);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive(&bar);
+    const bool ok = mbar_wait_budget(&bar, 0, budget, status);
+    *waited_out = ok ? 0 : 1;
+  }
+}
+
+cudaError_t launch_selftest_timeout(long long budget, int* status, int* waited_out, cudaStream_t s) {
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(budget, status, waited_out);
+  return cudaGetLastError();
 }
 
 }  // namespace dvlm

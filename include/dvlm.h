@@ -294,6 +294,31 @@ DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_
                          const uint8_t* masked, int n_rows, int n_clean, int first_layer,
                          int n_layers_run, int advance, void* x_out, dvlm_stream stream);
 
+/* Launch-configuration knobs of a bf16 engine (defaults are chosen at
+ * creation from occupancy queries).  Names and values:
+ *   "qkv_cluster", "o_cluster", "down_cluster": CTAs per cluster of the
+ *       cluster split-K projections (2..16; 0 = stream-K kernel instead);
+ *   "down_stages", "gateup_stages": TMA pipeline depth, 5 or 10;
+ *   "attn_cluster": CTAs per attention cluster, 8 or 16;
+ *   "pdl": 1/0, programmatic dependent launch between kernels.
+ * Results do not depend on the knobs except through fp32 summation order
+ * (cluster sizes).  Changing a knob drops the captured CUDA graphs.
+ * Errors: INVALID_ARG (unknown name), SHAPE (bad value), UNSUPPORTED (the
+ * device cannot launch that configuration, or an fp32 engine). */
+DVLM_API dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value);
+/* Current value of a knob (-1 for an unknown name). */
+DVLM_API int dvlm_engine_get_option(dvlm_engine* e, const char* name);
+
+/* Failure-detection self-test.  Every device-side wait of the library is
+ * bounded: on expiry it writes DVLM_ERR_TIMEOUT to the status word, abandons
+ * the rest of its work and lets the kernel end (no trap, no hang).  This
+ * launches one CTA whose wait can never be satisfied (an mbarrier expecting
+ * two arrivals receives one) with a budget of budget_cycles SM cycles
+ * (1..4e9); afterwards *dev_status (device) holds DVLM_ERR_TIMEOUT and
+ * *gave_up (device int) holds 1. */
+DVLM_API dvlm_status dvlm_selftest_wait_timeout(long long budget_cycles, int* dev_status, int* gave_up,
+                                               dvlm_stream stream);
+
 /* Profiling hook: one forward pass like dvlm_forward over all layers (L is
  * not advanced), launched eagerly with a CUDA event pair around every kernel
  * on `stream`.  ms_out[7] receives the device time per kernel class summed

@@ -39,5 +39,8 @@ def assert_bf16_close(got, want, tol=2e-2, what=""):
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     err = np.abs(got - want)
-    assert np.all(err <= tol + bf16_ulp(want)), (what, float(err.max()))
+    bad = np.argwhere(err > tol + bf16_ulp(want))
+    detail = [(tuple(int(v) for v in i), float(got[tuple(i)]), float(want[tuple(i)]), float(err[tuple(i)]))
+              for i in bad[:8]]
+    assert len(bad) == 0, (what, float(err.max()), detail)
     assert np.mean(err > tol) <= 1e-3, (what, float(np.mean(err > tol)))

@@ -91,3 +91,24 @@ def test_poison_tail_truncates_every_layer(cuda):
         assert torch.isnan(vc[:, i, :, :, lo:L0 + B].float()).all()
         assert torch.equal(kc[:, i, :, :lo], k0[:, i, :, :lo])
         assert torch.equal(vc[:, i, :, :, :lo], v0[:, i, :, :, :lo])
+
+
+def test_accept_on_lm_head_logits(cuda):
+    """Verify logits produced by the LM head of the fused-LM-head configuration
+    (hidden [16, 2048] N(0,1), W [151936, 2048] N(0, 0.02) x 25, bf16 logits):
+    the draft follows the argmax for positions < k and the runner-up after."""
+    B_, V = 16, 151936
+    (h_t, h), (w_t, w) = gen.lmhead_case(2, B_, 2048, V, second_set=False)
+    lg = O.bf16_round(h.astype(np.float64) @ w.astype(np.float64).T)
+    conf = O.confidence_from_logits(lg)
+    order = np.argsort(-lg, axis=-1, kind="stable")
+    k = 9
+    draft = conf.top1.astype(np.int32).copy()
+    draft[k:] = order[k:, 1]                      # runner-up: a different id
+    logits_t = torch.from_numpy(lg.astype(np.float32)).to(torch.bfloat16).reshape(1, B_, V)
+    # the bf16 cast is exact: the oracle already rounded the logits to bf16
+    assert np.array_equal(logits_t.float().numpy().reshape(B_, V), lg)
+    want = O.prefix_accept(conf.top1, draft)
+    assert want == k
+    got = run_spec(cuda, 1, V, torch.from_numpy(draft.reshape(1, B_)).to(cuda), logits=logits_t.to(cuda))
+    np.testing.assert_array_equal(got, [k])
