@@ -11,11 +11,13 @@
 // TMA box lands).  S = Q K^T (N = 64 keys) and O += P V (V stored
 // value-feature-major so both products read K-major operands) accumulate in
 // TMEM; softmax runs in fp32 registers, one thread per row, with P rounded
-// to bf16 for the second product.  The keys are split over a cluster of 8 or 16 CTAs;
+// to fp16 for the second product (the value tile converted to fp16 too).  The keys are split over a cluster of 8 or 16 CTAs;
 // the partial (max, sum, O) of the cluster's CTAs are merged through
 // distributed shared memory, so there is no second kernel and no global
 // scratch.  Clusters of 16 CTAs (where the device can co-schedule them) put
 // one or two 64-key chunks on each CTA at decode lengths.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "mainloop.cuh"
 
@@ -39,7 +41,10 @@ constexpr int oMisc = oBar + 16 * 8;
 // start (and fetch its cache tiles) while the QKV projection still runs.
 constexpr int kSmem = oMisc + 64 + 1024;
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChunk);
-constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128);
+// P V runs in fp16: probabilities in [0, 1] keep 11 significant bits instead
+// of bf16's 8, and the value tile is converted to fp16 in shared memory
+// (exact for |v| within fp16's normal range).
+constexpr uint32_t kIdescO = idesc_f16_f32(128, 128);
 }  // namespace
 
 template <int kCS>  // CTAs per cluster (key splits)
@@ -179,10 +184,8 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // Writes P of chunk jj (probabilities exp2(s - m_new), bf16) for this row
-    // into the P buffer and, on the last chunk, zeroes the value rows of keys
-    // past the valid slots (they may hold anything, NaN poison included, and
-    // 0 * NaN is NaN).
+    // Writes P of chunk jj (probabilities exp2(s - m_new), fp16) for this row
+    // into the P buffer and converts this thread's value row of the chunk.
     auto emit_p = [&](int jj, const float (&sc)[64], float m_new) -> float {
       const int key0 = (crank + kCS * jj) * kChunk;
       uint32_t packed[kChunk / 2];
@@ -193,10 +196,10 @@ __global__ void __launch_bounds__(192, 1)
       } else {
 #pragma unroll
         for (int c = 0; c < kChunk; c += 2) {
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(sc[c] - m_new), exp2f(sc[c + 1] - m_new));
-          const float2 pf = __bfloat1622float2(pb);
+          const __half2 ph = __floats2half2_rn(exp2f(sc[c] - m_new), exp2f(sc[c + 1] - m_new));
+          const float2 pf = __half22float2(ph);
           psum += pf.x + pf.y;
-          packed[c / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+          packed[c / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
       }
       uint8_t* prow = sP + row * 128;
@@ -205,16 +208,27 @@ __global__ void __launch_bounds__(192, 1)
         const uint4 w = make_uint4(packed[cc * 4 + 0], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
         *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) = w;
       }
-      if (key0 + kChunk > Ltot) {
+      // Value row `row` of this chunk (64 keys) to fp16 in place; keys past
+      // the valid slots may hold anything (NaN poison included) and 0 * NaN
+      // is NaN, so they become 0.
+      {
         const int st = jj & 1;
         mbar_wait(&kv_full[st], (jj >> 1) & 1, a.status, sabort);
-        uint8_t* vrow = sV + st * kVBytes + row * 128;  // value feature `row`, 64 keys
+        uint8_t* vrow = sV + st * kVBytes + row * 128;
         const int valid = Ltot - key0;
+#pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
-          if (8 * cc + 7 < valid) continue;
-          uint16_t* chunk = reinterpret_cast<uint16_t*>(vrow + ((cc ^ (row & 7)) << 4));
-          for (int e = 0; e < 8; ++e)
-            if (8 * cc + e >= valid) chunk[e] = 0;
+          uint4* p16 = reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4));
+          uint4 w = *p16;
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            const int k0 = 8 * cc + 2 * e;
+            const __half2 h = __floats2half2_rn(k0 < valid ? f.x : 0.f, k0 + 1 < valid ? f.y : 0.f);
+            wv[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *p16 = w;
         }
       }
       fence_proxy_async_smem();
