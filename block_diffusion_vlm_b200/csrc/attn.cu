@@ -34,11 +34,12 @@ constexpr int oQ = 0;
 constexpr int oK = oQ + kQBytes;
 constexpr int oV = oK + 2 * kKBytes;
 constexpr int oP = oV + 2 * kVBytes;       // one P buffer
-constexpr int oML = oP + kPBytes;          // m[128], l[128]
-constexpr int oBar = oML + 2 * 128 * 4;
+constexpr int kRecvBytes = 128 * 128 * 4;  // partial O rows received from the cluster
+constexpr int oRecv = oP + kPBytes;
+constexpr int oRecvML = oRecv + kRecvBytes;  // (m, l) received: [sources][rows]
+constexpr int oML = oRecvML + 128 * 8;       // (m, l) of this CTA's 128 rows
+constexpr int oBar = oML + 128 * 8;
 constexpr int oMisc = oBar + 16 * 8;
-// ~114 KB: fits on an SM next to one projection-GEMM CTA, so the kernel can
-// start (and fetch its cache tiles) while the QKV projection still runs.
 constexpr int kSmem = oMisc + 64 + 1024;
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChunk);
 // P V runs in fp16: probabilities in [0, 1] keep 11 significant bits instead
@@ -58,8 +59,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sV = smem + oV;
   uint8_t* sP = smem + oP;
   float* sO = reinterpret_cast<float*>(smem + oK);  // reused after the key loop: [128][128]
-  float* sM = reinterpret_cast<float*>(smem + oML);
-  float* sL = sM + 128;
+  float* sRecvO = reinterpret_cast<float*>(smem + oRecv);      // [kCS][128 / kCS rows][128]
+  float2* sRecvML = reinterpret_cast<float2*>(smem + oRecvML);  // [kCS][128 / kCS rows]
+  float2* sML = reinterpret_cast<float2*>(smem + oML);          // [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBar);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;    // [2] K and V of a chunk landed (stage = chunk & 1)
@@ -67,6 +69,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* s_full = bars + 5;     // [2] S of the chunk in that TMEM buffer ready
   uint64_t* p_full = bars + 7;     // P of the next chunk written (one phase per chunk)
   uint64_t* pv_done = bars + 8;    // PV of a chunk done (one phase per chunk)
+  uint64_t* recv_full = bars + 9;  // every cluster CTA's rows of this CTA landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + oMisc);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + oMisc + 4);
 
@@ -77,10 +80,14 @@ __global__ void __launch_bounds__(192, 1)
   const int bidx = blockIdx.z / n_groups;       // batch entry
   const int t_base = (blockIdx.z % n_groups) * 16;
 
+  constexpr int RPC = 128 / kCS;                  // output rows merged by each CTA
+  constexpr uint32_t kSendO = RPC * 128 * 4;      // bytes of partial O per destination
+  constexpr uint32_t kSendML = RPC * 8;           // bytes of (m, l) per destination
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], i == 7 ? 128 : 1);
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], i == 7 ? 128 : 1);
     *sabort = 0;
     fence_mbar_init();
+    mbar_arrive_expect_tx(recv_full, kCS * (kSendO + kSendML));
     tma_prefetch_map(&mapQ);
     tma_prefetch_map(&mapK);
     tma_prefetch_map(&mapV);
@@ -93,6 +100,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Receive barriers initialised cluster-wide before any CTA sends (waited on
+  // just before the sends).
+  cluster_arrive();
 
   // The cache length is final before this kernel's predecessor runs (only the
   // end of a forward pass moves it), and so are the cache slots below it: both
@@ -308,6 +318,10 @@ __global__ void __launch_bounds__(192, 1)
     named_bar_sync(1, 128);
     const bool have = ok && nc > 0 && !*sabort;
     if (have) tc_fence_after();
+    // Partial O row `row` as 32 float4 chunks, chunk c4 stored at slot
+    // c4 ^ (row & 31): conflict-free for the writes here (lanes = rows) and
+    // for the merge's reads.
+    float4* sO4 = reinterpret_cast<float4*>(sO);
 #pragma unroll
     for (int c = 0; c < 128; c += 64) {
       float o[64];
@@ -318,64 +332,64 @@ __global__ void __launch_bounds__(192, 1)
         for (int k = 0; k < 64; ++k) o[k] = 0.f;
       }
 #pragma unroll
-      for (int k = 0; k < 64; ++k) sO[row * 128 + ((c + k + 4 * row) & 127)] = o[k];
+      for (int k = 0; k < 64; k += 4) {
+        const int c4 = (c + k) >> 2;
+        sO4[row * 32 + (c4 ^ (row & 31))] = make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+      }
     }
-    sM[row] = have ? m : -INFINITY;
-    sL[row] = have ? l : 0.f;
+    sML[row] = have ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+    // Rows [d*RPC, (d+1)*RPC) of the partial go to cluster CTA d, which merges
+    // them: copies by the bulk-copy engine into that CTA's receive buffer,
+    // counted on its receive barrier.
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    cluster_wait();
+    if (warp == 2 && lane < kCS) {
+      const uint32_t rb = map_to_cta(smem_u32(recv_full), lane);
+      bulk_s2s_cluster(map_to_cta(smem_u32(sRecvO) + crank * kSendO, lane), sO + lane * RPC * 128, kSendO, rb);
+      bulk_s2s_cluster(map_to_cta(smem_u32(sRecvML) + crank * kSendML, lane), sML + lane * RPC, kSendML, rb);
+      bulk_commit();
+    }
   }
-  tc_fence_before();
-  cluster_sync();
+  if (warp < 2) {
+    __syncwarp();
+    cluster_wait();
+  }
   // ---------------------------------------------------------------- merge
-  // CTA `crank` combines rows [crank*RPC, (crank+1)*RPC) over the kCS partials.
+  // CTA `crank` combines rows [crank*RPC, (crank+1)*RPC) over the kCS partials,
+  // read from its own receive buffer in source order.
   if (threadIdx.x >= 64) {
-    constexpr int RPC = 128 / kCS;  // rows per CTA
     constexpr int TPR = 128 / RPC;  // threads per row
     constexpr int DPT = 128 / TPR;  // value features per thread
     const int et = threadIdx.x - 64;
-    const int r = crank * RPC + et / TPR;
+    const int rl = et / TPR;
+    const int r = crank * RPC + rl;
     const int d0 = (et % TPR) * DPT;
     const int t = t_base + (r >> 3), hl = r & 7;
-    // Maxima and sums of all partials first, then the partial outputs four
-    // sources at a time (all loads of a group in flight together).
-    float ms[kCS], ls[kCS];
-#pragma unroll
-    for (int s2 = 0; s2 < kCS; ++s2) {
-      ms[s2] = ld_dsmem_f32(map_to_cta(smem_u32(&sM[r]), s2));
-      ls[s2] = ld_dsmem_f32(map_to_cta(smem_u32(&sL[r]), s2));
-    }
+    const bool got = mbar_wait(recv_full, 0, a.status, sabort);
     float M = -INFINITY;
 #pragma unroll
-    for (int s2 = 0; s2 < kCS; ++s2) M = fmaxf(M, ms[s2]);
+    for (int s2 = 0; s2 < kCS; ++s2) M = fmaxf(M, sRecvML[s2 * RPC + rl].x);
     float acc[DPT];
 #pragma unroll
     for (int k = 0; k < DPT; ++k) acc[k] = 0.f;
     float lsum = 0.f;
-    if (M != -INFINITY) {
+    if (got && M != -INFINITY) {
+      const float4* rO4 = reinterpret_cast<const float4*>(sRecvO);
+#pragma unroll 4
+      for (int s2 = 0; s2 < kCS; ++s2) {
+        const float2 ml = sRecvML[s2 * RPC + rl];
+        if (ml.x == -INFINITY) continue;
+        const float w = exp2f(ml.x - M);
+        lsum += w * ml.y;
 #pragma unroll
-      for (int g0 = 0; g0 < kCS; g0 += 4) {
-        float4 ov[4][DPT / 4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int k = 0; k < DPT / 4; ++k) {
-            // rows are stored rotated by 4*row floats (bank spread); undo it
-            const int col = (d0 + 4 * k + 4 * r) & 127;
-            ov[q][k] = ld_dsmem_f32x4(map_to_cta(smem_u32(&sO[r * 128 + col]), g0 + q));
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int s2 = g0 + q;
-          if (ms[s2] == -INFINITY) continue;
-          const float w = exp2f(ms[s2] - M);
-          lsum += w * ls[s2];
-#pragma unroll
-          for (int k = 0; k < DPT / 4; ++k) {
-            acc[4 * k] += w * ov[q][k].x;
-            acc[4 * k + 1] += w * ov[q][k].y;
-            acc[4 * k + 2] += w * ov[q][k].z;
-            acc[4 * k + 3] += w * ov[q][k].w;
-          }
+        for (int k = 0; k < DPT / 4; ++k) {
+          const int c4 = (d0 >> 2) + k;
+          const float4 v = rO4[(s2 * RPC + rl) * 32 + (c4 ^ (r & 31))];
+          acc[4 * k] += w * v.x;
+          acc[4 * k + 1] += w * v.y;
+          acc[4 * k + 2] += w * v.z;
+          acc[4 * k + 3] += w * v.w;
         }
       }
     }
@@ -394,6 +408,9 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
+  if (warp == 2 && lane < kCS) bulk_wait_read_all();
+  // No CTA leaves while a copy into or out of its shared memory may run.
+  tc_fence_before();
   cluster_sync();
   if (warp == 0) {
     tc_fence_after();

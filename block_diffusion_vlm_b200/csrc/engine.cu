@@ -62,7 +62,8 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->q = c.take<void>(kNT * HD * es);
   e->attn_o = c.take<void>(kNT * HD * es);
   e->act = c.take<void>(static_cast<size_t>(kNT) * I * es);
-  e->ssq = c.take<float>((H / 128 + 1) * kNT * 4);
+  // sums of squares per (128-feature tile, cluster CTA): up to 16 CTAs per tile
+  e->ssq = c.take<float>(((H / 128) * 16 + 1) * kNT * 4);
   e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, 2 * P));  // up to two CTAs per SM
   e->gcnt = c.take<int>(num_tiles_max(m) * 4);
   e->lpart = c.take<float>(static_cast<size_t>(P) * 2 * kNT * 128 * 4);
@@ -153,7 +154,10 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   GemmEpi ea{};
   ea.n_rows = f.n_rows;
   ea.ssq_in = e->ssq;
-  ea.n_ssq = H / 128;
+  // entries of the sums-of-squares buffer the next RMSNorm adds up: one per
+  // 128-feature tile from the embedding and stream-K projections, one per
+  // (tile, cluster CTA) from the cluster split-K projections
+  int n_ssq = H / 128;
   ea.inv_h = 1.0f / H;
   ea.eps = m.eps;
   ea.Lmax = e->Lmax;
@@ -167,6 +171,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
   for (int l = f.layer0; l < l1; ++l) {
     ea.epi = EPI_QKV;
+    ea.n_ssq = n_ssq;
     ea.out = static_cast<bf16*>(e->q);
     ea.out_ld = Hq * D;
     ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
@@ -205,7 +210,9 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64,
                              ws_ctas(e, (H / 128) * (Hq * D / 64)), l * H, ea, pdl, s, 5));
     T1(K_OPROJ);
+    n_ssq = (H / 128) * (e->s_o > 0 ? e->s_o : 1);
     ea.epi = EPI_SWIGLU;
+    ea.n_ssq = n_ssq;
     ea.out = static_cast<bf16*>(e->act);
     ea.out_ld = I;
     T0(K_GATEUP);
@@ -224,13 +231,14 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64,
                              ws_ctas(e, (H / 128) * (I / 64)), l * H, ea, pdl, s, e->down_stages));
     T1(K_DOWN);
+    n_ssq = (H / 128) * (e->s_down > 0 ? e->s_down : 1);
   }
   if (f.x_out) DVLM_CK(cudaMemcpyAsync(f.x_out, x, static_cast<size_t>(f.n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
   if (f.lm) {
     LmArgs a = f.lma;
     fill_lm_scratch(e, a);
     a.ssq_in = e->ssq;
-    a.n_ssq = H / 128;
+    a.n_ssq = n_ssq;
     a.inv_h = 1.0f / H;
     a.eps = m.eps;
     const int nt = (m.vocab + 127) / 128;

@@ -103,13 +103,38 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     }
     int L0 = 0;
     if (EPI == EPI_QKV) L0 = ea.d_len ? *ea.d_len : ea.L_static;
-    const int first_tile = sc.first_tile(blockIdx.x);
+    // A tile split over CTAs pf < ... < pl is finished by pf, which streams
+    // the tile's first k blocks as its last segment; the others stream their
+    // parts first and leave fp32 partials in global scratch, counted on
+    // cnt[T].  pf fetches those partials while its own last segment is still
+    // in the mainloop and adds them in CTA order.
     int seg = 0;
     for (long long u = u0; u < u1; ++seg) {
       const int T = static_cast<int>(u / sc.kb);
       const long long t_begin = static_cast<long long>(T) * sc.kb, t_end = t_begin + sc.kb;
       const long long seg_end = t_end < u1 ? t_end : u1;
       const int b = seg & 1;
+      const bool whole = (u == t_begin) && (seg_end == t_end);
+      const bool finisher = !whole && (u == t_begin);
+      float o[NT];
+      if (finisher) {
+        const int pl = sc.cta_of(t_end - 1);
+        if (et == 0) {
+          const bool ok = wait_counter(&ea.cnt[T], pl - static_cast<int>(blockIdx.x), ea.status, sabort);
+          if (ok) ea.cnt[T] = 0;  // every part is counted: zero again for the next launch
+          *sflag = ok ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (!*sflag) break;
+        __threadfence();
+#pragma unroll
+        for (int t = 0; t < NT; ++t) o[t] = 0.f;
+        for (int p = static_cast<int>(blockIdx.x) + 1; p <= pl; ++p) {
+          const float* src = ea.part + static_cast<size_t>(p) * 2 * NT * 128;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) o[t] += __ldcg(&src[t * 128 + row]);
+        }
+      }
       mbar_wait(&accf[b], (seg >> 1) & 1, ea.status, sabort);
       named_bar_sync(1, 128);  // leave together if any wait gave up
       if (*sabort) break;
@@ -119,34 +144,20 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[b]);
-      const bool whole = (u == t_begin) && (seg_end == t_end);
-      if (!whole) {
-        const int slot = (T == first_tile) ? 0 : 1;
-        float* mine = ea.part + (static_cast<size_t>(blockIdx.x) * 2 + slot) * NT * 128;
+      if (!whole && !finisher) {
+        // tail or middle part of a tile finished by another CTA
+        float* mine = ea.part + static_cast<size_t>(blockIdx.x) * 2 * NT * 128;
 #pragma unroll
         for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + row], v[t]);
         __threadfence();
         named_bar_sync(1, 128);
-        const int pf = sc.cta_of(t_begin), pl = sc.cta_of(t_end - 1);
-        if (et == 0) {
-          const int old = atomicAdd(&ea.cnt[T], 1);
-          *sflag = (old == pl - pf) ? 1 : 0;
-        }
-        named_bar_sync(1, 128);
-        if (!*sflag) {
-          u = seg_end;
-          continue;
-        }
-        __threadfence();
+        if (et == 0) red_release_gpu_add(&ea.cnt[T], 1);
+        u = seg_end;
+        continue;
+      }
+      if (finisher) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) v[t] = 0.f;
-        for (int p = pf; p <= pl; ++p) {
-          const int sp = (T == sc.first_tile(p)) ? 0 : 1;
-          const float* src = ea.part + (static_cast<size_t>(p) * 2 + sp) * NT * 128;
-#pragma unroll
-          for (int t = 0; t < NT; ++t) v[t] += __ldcg(&src[t * 128 + row]);
-        }
-        if (et == 0) ea.cnt[T] = 0;
+        for (int t = 0; t < NT; ++t) v[t] += o[t];
       }
 
       if (EPI == EPI_RESID) {
@@ -240,12 +251,12 @@ template <int NT, int STAGES>
 struct ClSmem {
   static constexpr int kA = 0;
   static constexpr int kB = kA + STAGES * kATileBytes;
-  static constexpr int kP = kB + STAGES * NT * 128;     // partial [128][NT+1]
-  static constexpr int kQ = kP + 128 * (NT + 1) * 4;     // squares [128][NT+1] (residual epilogue)
-  static constexpr int kS = kQ + 128 * (NT + 1) * 4;     // slice sums of squares [NT]
-  static constexpr int kR = kS + 32 * 4;                 // rmsnorm factors [NT]
+  static constexpr int kSend = kB + STAGES * NT * 128;  // this CTA's partial tile [128][NT] fp32
+  static constexpr int kRecv = kSend + 128 * NT * 4;    // slices received [S][rows][NT] (<= 160 rows)
+  static constexpr int kQ = kRecv + 160 * NT * 4;       // squares of this CTA's rows [64][NT+1]
+  static constexpr int kR = kQ + 64 * (NT + 1) * 4;     // rmsnorm factors [NT]
   static constexpr int kBar = kR + 32 * 4;
-  static constexpr int kMisc = kBar + (2 * STAGES + 4) * 8;
+  static constexpr int kMisc = kBar + (2 * STAGES + 5) * 8;
   static constexpr int kTotal = kMisc + 64 + 1024;
 };
 
@@ -260,14 +271,15 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem + Sm::kA;
   uint8_t* sB = smem + Sm::kB;
-  float* sP = reinterpret_cast<float*>(smem + Sm::kP);
+  float* sSend = reinterpret_cast<float*>(smem + Sm::kSend);
+  float* sRecv = reinterpret_cast<float*>(smem + Sm::kRecv);
   float* sQ = reinterpret_cast<float*>(smem + Sm::kQ);
-  float* sS = reinterpret_cast<float*>(smem + Sm::kS);
   float* sR = reinterpret_cast<float*>(smem + Sm::kR);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kBar);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
+  uint64_t* recv_full = acce + 2;  // every cluster CTA's slice of this CTA's rows landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Sm::kMisc);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + Sm::kMisc + 8);
 
@@ -277,6 +289,20 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   const SkSched sc{static_cast<int>(gridDim.x) / S, kb, 1};
   const long long u0 = static_cast<long long>(T) * kb + static_cast<long long>(c) * kb / S;
   const long long u1 = static_cast<long long>(T) * kb + static_cast<long long>(c + 1) * kb / S;
+  // Rows of the tile finished by cluster CTA d: RESID rows [a0, a0+n); QKV the
+  // RoPE pairs (j, j+64) for j in [a0, a0+n), so a pair never straddles CTAs.
+  auto slice = [&](int d, int& a0, int& n) {
+    const int span = EPI == EPI_RESID ? 128 : 64;
+    a0 = d * span / S;
+    n = (d + 1) * span / S - a0;
+  };
+  constexpr int kPieces = EPI == EPI_RESID ? 1 : 2;  // row ranges per slice
+  int my0, myn;
+  slice(c, my0, myn);
+  // slice elements per epilogue thread: at most 64 rows (S >= 2) x NT over 128
+  constexpr int kMaxPer = (64 * NT + 127) / 128;
+  // The cache length is final before this kernel's predecessor runs.
+  const int L0 = (EPI == EPI_QKV) ? (ea.d_len ? *ea.d_len : ea.L_static) : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -287,8 +313,10 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], 4);
     }
+    mbar_init(recv_full, 1);
     *sabort = 0;
     fence_mbar_init();
+    mbar_arrive_expect_tx(recv_full, static_cast<uint32_t>(S * kPieces * myn * NT * 4));
     tma_prefetch_map(&mapA);
     tma_prefetch_map(&mapB);
   }
@@ -300,8 +328,12 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Receive barriers initialised cluster-wide before any CTA sends (waited on
+  // just before the sends).
+  cluster_arrive();
 
   const int et = threadIdx.x - 64;  // epilogue thread 0..127 (warps 2..5)
+  float pre_a[kMaxPer], pre_b[kMaxPer];
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
       ws_producer<NT, STAGES, false>(&mapA, &mapA, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base, 0, ea.status,
@@ -320,6 +352,28 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       for (int p = 0; p < ea.n_ssq; ++p) s2 += ea.ssq_in[p * NT + et];
       sR[et] = 1.0f / sqrtf(s2 * ea.inv_h + ea.eps);
     }
+    // Operands of this thread's share of the slice epilogue that do not
+    // depend on the product, fetched while the mainloop streams: the residual
+    // entries (RESID) or the RoPE rotation (QKV).
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+      const int it = et + 128 * k;
+      pre_a[k] = 0.f;
+      pre_b[k] = 0.f;
+      if (it >= myn * NT) continue;
+      const int t = it % NT;
+      if (t >= ea.n_rows) continue;
+      if (EPI == EPI_RESID) {
+        pre_a[k] = __bfloat162float(ea.resid[static_cast<size_t>(t) * ea.resid_ld + T * 128 + my0 + it / NT]);
+      } else if (T < ea.n_q_heads + ea.n_kv_heads) {
+        const int j = my0 + it / NT;
+        const double inv_freq = exp2(-(2.0 * j / 128.0) * ea.log2_rope_base);
+        double sn, cs;
+        sincos(static_cast<double>(L0 + t) * inv_freq, &sn, &cs);
+        pre_a[k] = static_cast<float>(cs);
+        pre_b[k] = static_cast<float>(sn);
+      }
+    }
     float v[NT];
     if (u1 > u0) {
       mbar_wait(&accf[0], 0, ea.status, sabort);
@@ -329,65 +383,81 @@ __global__ void __launch_bounds__(kWsThreads, 2)
 #pragma unroll
       for (int t = 0; t < NT; ++t) v[t] = 0.f;
     }
+    float4* s4 = reinterpret_cast<float4*>(sSend + row * NT);
 #pragma unroll
-    for (int t = 0; t < NT; ++t) sP[row * PS + t] = v[t];
+    for (int t = 0; t < NT; t += 4) s4[t / 4] = make_float4(v[t], v[t + 1], v[t + 2], v[t + 3]);
+    // Slice d of the partial goes to cluster CTA d, which sums the S partials
+    // of its rows: bulk copies into that CTA's receive buffer (source-major),
+    // counted on its receive barrier.
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    cluster_wait();
+    if (et < S) {
+      int a0, n;
+      slice(et, a0, n);
+      if (n > 0) {
+        const uint32_t rb = map_to_cta(smem_u32(recv_full), et);
+        const uint32_t bytes = static_cast<uint32_t>(n * NT * 4);
+        const uint32_t dst = map_to_cta(smem_u32(sRecv), et) + static_cast<uint32_t>(c * kPieces) * bytes;
+        bulk_s2s_cluster(dst, sSend + a0 * NT, bytes, rb);
+        if (EPI == EPI_QKV) bulk_s2s_cluster(dst + bytes, sSend + (a0 + 64) * NT, bytes, rb);
+      }
+      bulk_commit();
+    }
   }
-  tc_fence_before();
-  cluster_sync();  // partials of every CTA of the tile are visible
+  if (warp < 2) {
+    __syncwarp();
+    cluster_wait();
+  }
+  // Every CTA has issued its copies once all have arrived here: a CTA leaves
+  // only after that (second barrier, waited on at exit).
+  cluster_arrive();
 
   if (threadIdx.x >= 64) {
-    uint32_t rp[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) rp[q] = q < S ? map_to_cta(smem_u32(sP), q) : 0u;
-    // Sum of the S partials of element (r, t), in rank order; all S loads
-    // are issued before the first add.
-    auto part_sum = [&](int r, int t) {
-      const uint32_t off = 4u * static_cast<uint32_t>(r * PS + t);
-      float vals[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) vals[q] = q < S ? ld_dsmem_f32(rp[q] + off) : 0.f;
+    const bool got = mbar_wait(recv_full, 0, ea.status, sabort);
+    const int rps = kPieces * myn;  // rows from each source
+    // Sum of the S partials of element (rl, t) of this CTA's slice, in rank order.
+    auto part_sum = [&](int rl, int t) {
       float acc = 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (q < S) acc += vals[q];
+      for (int q = 0; q < S; ++q) acc += sRecv[(q * rps + rl) * NT + t];
       return acc;
     };
     if (EPI == EPI_RESID) {
-      const int r0 = c * 128 / S, r1 = (c + 1) * 128 / S;
-      const int nr = r1 - r0;
-      for (int it = et; it < nr * NT; it += 128) {
-        const int r = r0 + it / NT, t = it % NT;
-        const float y = part_sum(r, t);
+#pragma unroll
+      for (int k = 0; k < kMaxPer; ++k) {
+        const int it = et + 128 * k;
+        if (it >= myn * NT) break;
+        const int rl = it / NT, t = it % NT;
+        const float y = got ? part_sum(rl, t) : 0.f;
         float sq = 0.f;
         if (t < ea.n_rows) {
-          bf16* px = ea.resid + static_cast<size_t>(t) * ea.resid_ld + T * 128 + r;
-          const float xn = bf16_round_f(__bfloat162float(*px) + y);
-          *px = __float2bfloat16_rn(xn);
+          const float xn = bf16_round_f(pre_a[k] + y);
+          ea.resid[static_cast<size_t>(t) * ea.resid_ld + T * 128 + my0 + rl] = __float2bfloat16_rn(xn);
           sq = xn * xn;
         }
-        sQ[r * PS + t] = sq;
+        sQ[rl * PS + t] = sq;
       }
       named_bar_sync(1, 128);
+      // Sums of squares per (tile, cluster CTA): the next RMSNorm adds all
+      // n_tiles * S of them in order.
       if (et < NT) {
         float s2 = 0.f;
-        for (int r = r0; r < r1; ++r) s2 += sQ[r * PS + et];
-        sS[et] = s2;
+        for (int rl = 0; rl < myn; ++rl) s2 += sQ[rl * PS + et];
+        ea.ssq_out[(T * S + c) * NT + et] = s2;
       }
     } else {  // EPI_QKV: pairs (j, j+64) of one head per tile
-      const int p0 = c * 64 / S, p1 = (c + 1) * 64 / S;
-      const int np = p1 - p0;
       const int nq = ea.n_q_heads, nkv = ea.n_kv_heads;
-      const int L0 = ea.d_len ? *ea.d_len : ea.L_static;
-      for (int it = et; it < np * NT; it += 128) {
-        const int j = p0 + it / NT, t = it % NT;
-        const float x1 = part_sum(j, t) * sR[t];
-        const float x2 = part_sum(j + 64, t) * sR[t];
+#pragma unroll
+      for (int k = 0; k < kMaxPer; ++k) {
+        const int it = et + 128 * k;
+        if (it >= myn * NT) break;
+        const int jl = it / NT, t = it % NT;
+        const int j = my0 + jl;
+        const float x1 = (got ? part_sum(jl, t) : 0.f) * sR[t];
+        const float x2 = (got ? part_sum(myn + jl, t) : 0.f) * sR[t];
         if (t >= ea.n_rows) continue;
         if (T < nq + nkv) {
-          const double inv_freq = exp2(-(2.0 * j / 128.0) * ea.log2_rope_base);
-          double sn, cs;
-          sincos(static_cast<double>(L0 + t) * inv_freq, &sn, &cs);
-          const float co = static_cast<float>(cs), si = static_cast<float>(sn);
+          const float co = pre_a[k], si = pre_b[k];
           const bf16 y1 = __float2bfloat16_rn(x1 * co - x2 * si);
           const bf16 y2 = __float2bfloat16_rn(x2 * co + x1 * si);
           bf16* dst = (T < nq) ? ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128
@@ -401,16 +471,10 @@ __global__ void __launch_bounds__(kWsThreads, 2)
         }
       }
     }
+    if (et < S) bulk_wait_read_all();
   }
-  if (EPI == EPI_RESID) {
-    cluster_sync();  // slice sums visible
-    if (c == 0 && threadIdx.x >= 64 && et < NT) {
-      float s2 = 0.f;
-      for (int q = 0; q < S; ++q) s2 += ld_dsmem_f32(map_to_cta(smem_u32(&sS[et]), q));
-      ea.ssq_out[T * NT + et] = s2;
-    }
-  }
-  cluster_sync();  // no CTA leaves while another still reads its shared memory
+  tc_fence_before();
+  cluster_wait();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TMC);
@@ -473,7 +537,7 @@ static cudaError_t launch_cl(const CUtensorMap& mapA, const CUtensorMap& mapB, i
 
 cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
                            int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s, int stages) {
-  if (S < 1 || S > 16 || NT != 16) return cudaErrorInvalidValue;
+  if (S < 2 || S > 16 || NT != 16) return cudaErrorInvalidValue;
   if (stages == 5) {
     if (ea.epi == EPI_QKV) return launch_cl<16, 5, EPI_QKV>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);
     if (ea.epi == EPI_RESID) return launch_cl<16, 5, EPI_RESID>(mapA, mapB, n_tiles, kb, S, a_row_base, ea, pdl, s);

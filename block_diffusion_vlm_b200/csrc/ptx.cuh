@@ -116,6 +116,29 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// GPU-scope acquire load / release add of a counter in global memory.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Waits (bounded, like mbar_wait) until *p reaches `target`.
+__device__ __forceinline__ bool wait_counter(const int* p, int target, int* status, volatile int* abort_flag) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(p) < target) {
+    if ((abort_flag && *abort_flag) || clock64() - t0 > kWaitBudgetCycles) {
+      record_error(status, DVLM_ERR_TIMEOUT);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- PDL
 // Programmatic dependent launch.  Every kernel of the library triggers its
 // dependents only after its own griddepcontrol.wait has returned, i.e. after
@@ -264,6 +287,27 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The two halves of a cluster barrier, for every thread of every CTA of the
+// cluster: arrive (release) early, wait (acquire) where the other CTAs' state
+// is first needed.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Bulk copy of `bytes` (multiple of 16, 16-byte aligned ends) from this CTA's
+// shared memory into the shared memory of a CTA of the cluster; the bytes are
+// counted on that CTA's mbarrier.  dst and mbar are cluster addresses
+// (map_to_cta).  One commit group per issuing thread.
+__device__ __forceinline__ void bulk_s2s_cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk copies have read their sources.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
