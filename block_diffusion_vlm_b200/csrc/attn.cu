@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ---------------------------------------------------------------- softmax
     griddep_wait();
+    // The next kernel (the output projection) may launch now and stream its
+    // weights on the SMs this kernel leaves idle; it reads this kernel's
+    // output only after its own wait (at most two kernels overlap).
+    if (threadIdx.x == 64) griddep_launch_dependents();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int t = t_base + (row >> 3);

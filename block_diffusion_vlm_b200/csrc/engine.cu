@@ -216,9 +216,8 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.out = static_cast<bf16*>(e->act);
     ea.out_ld = I;
     T0(K_GATEUP);
-    // 10 stages: one CTA per SM; 5 stages: two per SM (same bytes in flight)
     const long long gu_units = static_cast<long long>(I / 64) * (H / 64);
-    const int gu_ctas = static_cast<int>(std::min<long long>(gu_units, (e->gu_stages == 5 ? 2LL : 1LL) * e->sm));
+    const int gu_ctas = static_cast<int>(std::min<long long>(gu_units, static_cast<long long>(e->gu_cps) * e->sm));
     DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, gu_ctas,
                            l * I, ea, pdl, s, e->gu_stages));
     T1(K_GATEUP);
@@ -515,25 +514,32 @@ cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* co
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
   const dvlm_model& m = e->m;
   const std::string n(name);
-  auto cluster_ok = [&](int epi, int S, int stages) {
-    return S == 0 || (S >= 2 && S <= 16 && gemm_cl_max_clusters(epi, S, stages) > 0);
+  // every cluster of the projection resident at once (one wave)
+  const int qkv_tiles = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim / 128, h_tiles = m.hidden / 128;
+  auto cluster_ok = [&](int epi, int S, int stages, int n_tiles) {
+    return S == 0 || (S >= 2 && S <= 16 && gemm_cl_max_clusters(epi, S, stages) >= n_tiles);
   };
   if (n == "qkv_cluster") {
-    if (!cluster_ok(EPI_QKV, v, 5) || v > m.hidden / 64) return DVLM_ERR_UNSUPPORTED;
+    if (!cluster_ok(EPI_QKV, v, 5, qkv_tiles) || v > m.hidden / 64) return DVLM_ERR_UNSUPPORTED;
     e->s_qkv = v;
   } else if (n == "o_cluster") {
-    if (!cluster_ok(EPI_RESID, v, 5) || v > m.n_q_heads * m.head_dim / 64) return DVLM_ERR_UNSUPPORTED;
+    if (!cluster_ok(EPI_RESID, v, 5, h_tiles) || v > m.n_q_heads * m.head_dim / 64) return DVLM_ERR_UNSUPPORTED;
     e->s_o = v;
   } else if (n == "down_cluster") {
-    if (!cluster_ok(EPI_RESID, v, e->down_stages) || v > m.inter / 64) return DVLM_ERR_UNSUPPORTED;
+    if (!cluster_ok(EPI_RESID, v, e->down_stages, h_tiles) || v > m.inter / 64) return DVLM_ERR_UNSUPPORTED;
     e->s_down = v;
   } else if (n == "down_stages") {
     if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
-    if (e->s_down > 0 && gemm_cl_max_clusters(EPI_RESID, e->s_down, v) <= 0) return DVLM_ERR_UNSUPPORTED;
+    if (!cluster_ok(EPI_RESID, e->s_down, v, h_tiles)) return DVLM_ERR_UNSUPPORTED;
     e->down_stages = v;
   } else if (n == "gateup_stages") {
     if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
+    if (v == 10 && e->gu_cps == 2) return DVLM_ERR_UNSUPPORTED;
     e->gu_stages = v;
+  } else if (n == "gateup_ctas_per_sm") {
+    if (v != 1 && v != 2) return DVLM_ERR_SHAPE;
+    if (v == 2 && e->gu_stages == 10) return DVLM_ERR_UNSUPPORTED;
+    e->gu_cps = v;
   } else if (n == "attn_cluster") {
     if (v != 8 && v != 16) return DVLM_ERR_SHAPE;
     if (attn_max_clusters(v) <= 0) return DVLM_ERR_UNSUPPORTED;
@@ -555,6 +561,7 @@ int engine_get_option(dvlm_engine* e, const char* name) {
   if (n == "down_cluster") return e->s_down;
   if (n == "down_stages") return e->down_stages;
   if (n == "gateup_stages") return e->gu_stages;
+  if (n == "gateup_ctas_per_sm") return e->gu_cps;
   if (n == "attn_cluster") return e->attn_cs;
   if (n == "pdl") return e->pdl ? 1 : 0;
   return -1;

@@ -62,6 +62,7 @@ struct dvlm_engine {
   int s_qkv = 0, s_o = 0, s_down = 0;  // cluster sizes of the split-K projections (0: stream-K)
   int attn_cs = 8;                      // CTAs per attention cluster (8 or 16)
   int gu_stages = 10, down_stages = 10; // pipeline depth of the gate/up and down projections
+  int gu_cps = 1;                       // gate/up CTAs per SM (2 needs 5 stages)
   bool pdl = true;                      // programmatic dependent launch between kernels
   // device buffers carved from the workspace
   void* x = nullptr;        // [NT][H]

@@ -299,6 +299,7 @@ DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_
  *   "qkv_cluster", "o_cluster", "down_cluster": CTAs per cluster of the
  *       cluster split-K projections (2..16; 0 = stream-K kernel instead);
  *   "down_stages", "gateup_stages": TMA pipeline depth, 5 or 10;
+ *   "gateup_ctas_per_sm": 1, or 2 with 5 gate/up stages;
  *   "attn_cluster": CTAs per attention cluster, 8 or 16;
  *   "pdl": 1/0, programmatic dependent launch between kernels.
  * Results do not depend on the knobs except through fp32 summation order
