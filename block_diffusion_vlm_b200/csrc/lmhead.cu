@@ -156,7 +156,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       bar();
       return out;
     };
-    const int first_tile = sc.first_tile(blockIdx.x);
+    // A vocabulary tile split over CTAs pf < ... < pl is finished by pf, which
+    // streams the tile's first k blocks as its last segment; the others
+    // stream their parts first and leave fp32 partial logits in global
+    // scratch, counted on cnt[T].  pf fetches them while its own last
+    // segment is still in the mainloop, adds them in CTA order and scans the
+    // tile into its running record like any whole tile.
     int seg = 0;
     bool ok = true;
     for (long long u = u0; u < u1; ++seg) {
@@ -164,6 +169,30 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       const long long t_begin = static_cast<long long>(T) * sc.kb, t_end = t_begin + sc.kb;
       const long long seg_end = t_end < u1 ? t_end : u1;
       const int b = seg & 1;
+      const bool whole = (u == t_begin) && (seg_end == t_end);
+      const bool finisher = !whole && (u == t_begin);
+      float o[NT];  // the other CTAs' partial logits of row et (finisher)
+      if (finisher) {
+        const int pl = sc.cta_of(t_end - 1);
+        if (et == 0) {
+          const bool got = wait_counter(&a.cnt[T], pl - static_cast<int>(blockIdx.x), a.status, sabort);
+          if (got) a.cnt[T] = 0;  // every part is counted: zero again for the next launch
+          *sflag = got ? 1 : 0;
+        }
+        bar();
+        if (!*sflag) {
+          ok = false;
+          break;
+        }
+        __threadfence();
+#pragma unroll
+        for (int t = 0; t < NT; ++t) o[t] = 0.f;
+        for (int p = static_cast<int>(blockIdx.x) + 1; p <= pl; ++p) {
+          const float* src = a.part + static_cast<size_t>(p) * 2 * NT * 128;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) o[t] += __ldcg(&src[t * 128 + et]);
+        }
+      }
       mbar_wait(&accf[b], (seg >> 1) & 1, a.status, sabort);
       bar();
       if (*sabort) {
@@ -182,42 +211,21 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[b]);
       bar();
-      const bool whole = (u == t_begin) && (seg_end == t_end);
-      if (whole) {
-        scan(T, run);
-      } else {
-        const int slot = (T == first_tile) ? 0 : 1;
-        float* mine = a.part + (static_cast<size_t>(blockIdx.x) * 2 + slot) * NT * 128;
+      if (!whole && !finisher) {
+        // tail or middle part of a tile finished by another CTA
+        float* mine = a.part + static_cast<size_t>(blockIdx.x) * 2 * NT * 128;
+#pragma unroll
         for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + et], sT[t * SROW + et]);
         __threadfence();
         bar();
-        const int pf = sc.cta_of(t_begin), pl = sc.cta_of(t_end - 1);
-        if (et == 0) {
-          const int old = atomicAdd(&a.cnt[T], 1);
-          *sflag = (old == pl - pf) ? 1 : 0;
-        }
-        bar();
-        if (*sflag) {
-          __threadfence();
-          for (int t = 0; t < NT; ++t) {
-            float acc = 0.f;
-            for (int p = pf; p <= pl; ++p) {
-              const int sp = (T == sc.first_tile(p)) ? 0 : 1;
-              acc += __ldcg(&a.part[((static_cast<size_t>(p) * 2 + sp) * NT + t) * 128 + et]);
-            }
-            sT[t * SROW + et] = acc;
-          }
-          if (et == 0) a.cnt[T] = 0;
+        if (et == 0) red_release_gpu_add(&a.cnt[T], 1);
+      } else {
+        if (finisher) {
+#pragma unroll
+          for (int t = 0; t < NT; ++t) sT[t * SROW + et] += o[t];
           bar();
-          Stat st{-INFINITY, 0.0f, 0x7fffffff};
-          scan(T, st);
-          const Stat tile_rec = combine(st);
-          if (sub == 0) {
-            float4* dst = reinterpret_cast<float4*>(a.rec) + (static_cast<size_t>(P) + pf) * NT + tok;
-            __stcg(dst, make_float4(tile_rec.m, tile_rec.s, __int_as_float(tile_rec.idx), 0.f));
-          }
-          if (et == 0) a.split_valid[pf] = 1;
         }
+        scan(T, run);
       }
       bar();  // sT is rewritten by the next segment
       u = seg_end;
@@ -237,15 +245,21 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       bar();
       if (*slast) {
         __threadfence();
+        // The last CTA merges every CTA's record of each token in CTA order;
+        // a thread's records are fetched in batches of 16 loads in flight.
         Stat st{-INFINITY, 0.0f, 0x7fffffff};
         const float4* rec = reinterpret_cast<const float4*>(a.rec);
-        for (int p = sub; p < P; p += TPT) {
-          float4 f = __ldcg(&rec[static_cast<size_t>(p) * NT + tok]);
-          stat_merge(st, Stat{f.x, f.y, __float_as_int(f.z)});
-          if (__ldcg(&a.split_valid[p])) {
-            f = __ldcg(&rec[(static_cast<size_t>(P) + p) * NT + tok]);
-            stat_merge(st, Stat{f.x, f.y, __float_as_int(f.z)});
+        constexpr int kBatch = 16;
+        for (int p0 = sub; p0 < P; p0 += TPT * kBatch) {
+          float4 f[kBatch];
+#pragma unroll
+          for (int q = 0; q < kBatch; ++q) {
+            const int p = p0 + TPT * q;
+            f[q] = p < P ? __ldcg(&rec[static_cast<size_t>(p) * NT + tok]) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+#pragma unroll
+          for (int q = 0; q < kBatch; ++q)
+            if (p0 + TPT * q < P) stat_merge(st, Stat{f[q].x, f[q].y, __float_as_int(f[q].z)});
         }
         const Stat fin = combine(st);
         if (sub == 0 && tok < 128) {
@@ -253,7 +267,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           fs.id[tok] = fin.idx;
         }
         bar();
-        for (int p = et; p < P; p += 128) a.split_valid[p] = 0;
         if (et == 0) *a.done = 0;
         finalize_rows(et, a, fs, bar);
       }
