@@ -34,7 +34,7 @@ constexpr int oQ = 0;
 constexpr int oK = oQ + kQBytes;
 constexpr int oV = oK + 2 * kKBytes;
 constexpr int oP = oV + 2 * kVBytes;       // one P buffer
-constexpr int kRecvBytes = 128 * 128 * 4;  // partial O rows received from the cluster
+constexpr int kRecvBytes = 128 * 128 * 2;  // partial O rows (fp16) received from the cluster
 constexpr int oRecv = oP + kPBytes;
 constexpr int oRecvML = oRecv + kRecvBytes;  // (m, l) received: [sources][rows]
 constexpr int oML = oRecvML + 128 * 8;       // (m, l) of this CTA's 128 rows
@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sK = smem + oK;
   uint8_t* sV = smem + oV;
   uint8_t* sP = smem + oP;
-  float* sO = reinterpret_cast<float*>(smem + oK);  // reused after the key loop: [128][128]
-  float* sRecvO = reinterpret_cast<float*>(smem + oRecv);      // [kCS][128 / kCS rows][128]
+  __half* sO = reinterpret_cast<__half*>(smem + oK);  // reused after the key loop: [128][128] fp16
+  __half* sRecvO = reinterpret_cast<__half*>(smem + oRecv);    // [kCS][128 / kCS rows][128]
   float2* sRecvML = reinterpret_cast<float2*>(smem + oRecvML);  // [kCS][128 / kCS rows]
   float2* sML = reinterpret_cast<float2*>(smem + oML);          // [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oBar);
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(192, 1)
   const int t_base = (blockIdx.z % n_groups) * 16;
 
   constexpr int RPC = 128 / kCS;                  // output rows merged by each CTA
-  constexpr uint32_t kSendO = RPC * 128 * 4;      // bytes of partial O per destination
+  constexpr uint32_t kSendO = RPC * 128 * 2;      // bytes of partial O per destination
   constexpr uint32_t kSendML = RPC * 8;           // bytes of (m, l) per destination
   if (threadIdx.x == 0) {
     for (int i = 0; i < 10; ++i) mbar_init(&bars[i], i == 7 ? 128 : 1);
@@ -322,10 +322,11 @@ __global__ void __launch_bounds__(192, 1)
     named_bar_sync(1, 128);
     const bool have = ok && nc > 0 && !*sabort;
     if (have) tc_fence_after();
-    // Partial O row `row` as 32 float4 chunks, chunk c4 stored at slot
-    // c4 ^ (row & 31): conflict-free for the writes here (lanes = rows) and
-    // for the merge's reads.
-    float4* sO4 = reinterpret_cast<float4*>(sO);
+    // Partial O row `row`, divided by its own sum l (|O / l| <= max |v|), as
+    // fp16: 16 chunks of 8 values, chunk c8 stored at slot c8 ^ (row & 15)
+    // (conflict-free here, lanes = rows, and in the merge's reads).
+    uint4* sO16 = reinterpret_cast<uint4*>(sO);
+    const float inv_l = (have && l > 0.f) ? 1.0f / l : 0.f;
 #pragma unroll
     for (int c = 0; c < 128; c += 64) {
       float o[64];
@@ -336,9 +337,15 @@ __global__ void __launch_bounds__(192, 1)
         for (int k = 0; k < 64; ++k) o[k] = 0.f;
       }
 #pragma unroll
-      for (int k = 0; k < 64; k += 4) {
-        const int c4 = (c + k) >> 2;
-        sO4[row * 32 + (c4 ^ (row & 31))] = make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+      for (int k = 0; k < 64; k += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __half2 h = __floats2half2_rn(o[k + 2 * q] * inv_l, o[k + 2 * q + 1] * inv_l);
+          w[q] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        const int c8 = (c + k) >> 3;
+        sO16[row * 16 + (c8 ^ (row & 15))] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
     sML[row] = have ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
@@ -379,21 +386,25 @@ __global__ void __launch_bounds__(192, 1)
     for (int k = 0; k < DPT; ++k) acc[k] = 0.f;
     float lsum = 0.f;
     if (got && M != -INFINITY) {
-      const float4* rO4 = reinterpret_cast<const float4*>(sRecvO);
+      const uint4* rO16 = reinterpret_cast<const uint4*>(sRecvO);
 #pragma unroll 4
       for (int s2 = 0; s2 < kCS; ++s2) {
         const float2 ml = sRecvML[s2 * RPC + rl];
         if (ml.x == -INFINITY) continue;
-        const float w = exp2f(ml.x - M);
-        lsum += w * ml.y;
+        // weight of this partial: its sum l at the common maximum
+        const float w = exp2f(ml.x - M) * ml.y;
+        lsum += w;
 #pragma unroll
-        for (int k = 0; k < DPT / 4; ++k) {
-          const int c4 = (d0 >> 2) + k;
-          const float4 v = rO4[(s2 * RPC + rl) * 32 + (c4 ^ (r & 31))];
-          acc[4 * k] += w * v.x;
-          acc[4 * k + 1] += w * v.y;
-          acc[4 * k + 2] += w * v.z;
-          acc[4 * k + 3] += w * v.w;
+        for (int k = 0; k < DPT / 8; ++k) {
+          const int c8 = (d0 >> 3) + k;
+          const uint4 v = rO16[(s2 * RPC + rl) * 16 + (c8 ^ (r & 15))];
+          const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vw[q]));
+            acc[8 * k + 2 * q] += w * f.x;
+            acc[8 * k + 2 * q + 1] += w * f.y;
+          }
         }
       }
     }
