@@ -33,9 +33,9 @@ constexpr int kPBytes = 16384;   // 128 rows x 64 keys
 constexpr int oQ = 0;
 constexpr int oK = oQ + kQBytes;
 constexpr int oV = oK + 2 * kKBytes;
-constexpr int oP = oV + 2 * kVBytes;       // one P buffer
+constexpr int oP = oV + 2 * kVBytes;       // two P buffers: the chunks of a pair
 constexpr int kRecvBytes = 128 * 128 * 2;  // partial O rows (fp16) received from the cluster
-constexpr int oRecv = oP + kPBytes;
+constexpr int oRecv = oP + 2 * kPBytes;
 constexpr int oRecvML = oRecv + kRecvBytes;  // (m, l) received: [sources][rows]
 constexpr int oML = oRecvML + 128 * 8;       // (m, l) of this CTA's 128 rows
 constexpr int oBar = oML + 128 * 8;
@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* kv_full = bars + 1;    // [2] K and V of a chunk landed (stage = chunk & 1)
   uint64_t* kv_empty = bars + 3;   // [2] PV of the chunk in that stage done
   uint64_t* s_full = bars + 5;     // [2] S of the chunk in that TMEM buffer ready
-  uint64_t* p_full = bars + 7;     // P of the next chunk written (one phase per chunk)
-  uint64_t* pv_done = bars + 8;    // PV of a chunk done (one phase per chunk)
+  uint64_t* p_full = bars + 7;     // P of a pair of chunks written (one phase per pair)
+  uint64_t* pv_done = bars + 8;    // PV of a pair of chunks done (one phase per pair)
   uint64_t* recv_full = bars + 9;  // every cluster CTA's rows of this CTA landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + oMisc);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + oMisc + 4);
@@ -167,20 +167,20 @@ __global__ void __launch_bounds__(192, 1)
         }
         umma_commit(&s_full[st]);
         if ((jj & 1) == 1 || jj == nc - 1) {  // end of a pair of chunks: their PV products
-          for (int c = jj & ~1; ok && c <= jj; ++c) {
-            if (!mbar_wait(p_full, c & 1, a.status, sabort)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t pa = smem_u32(sP), vb = smem_u32(sV + (c & 1) * kVBytes);
+          if (!mbar_wait(p_full, (jj >> 1) & 1, a.status, sabort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int c = jj & ~1; c <= jj; ++c) {
+            const uint32_t pa = smem_u32(sP + (c & 1) * kPBytes), vb = smem_u32(sV + (c & 1) * kVBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_bf16_ss(tmem + 128, sdesc_kmajor_sw128(pa + 32 * kk), sdesc_kmajor_sw128(vb + 32 * kk), kIdescO,
                            (c > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(pv_done);
             umma_commit(&kv_empty[c & 1]);
           }
+          umma_commit(pv_done);
         }
       }
     }
@@ -199,24 +199,26 @@ __global__ void __launch_bounds__(192, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // Writes P of chunk jj (probabilities exp2(s - m_new), fp16) for this row
-    // into the P buffer and converts this thread's value row of the chunk.
+    // into the chunk's P buffer and converts this thread's value row of the
+    // chunk; returns the row sum of the probabilities.
     auto emit_p = [&](int jj, const float (&sc)[64], float m_new) -> float {
       const int key0 = (crank + kCS * jj) * kChunk;
       uint32_t packed[kChunk / 2];
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       if (m_new == -INFINITY) {
 #pragma unroll
         for (int c = 0; c < kChunk / 2; ++c) packed[c] = 0u;
       } else {
 #pragma unroll
         for (int c = 0; c < kChunk; c += 2) {
-          const __half2 ph = __floats2half2_rn(exp2f(sc[c] - m_new), exp2f(sc[c + 1] - m_new));
-          const float2 pf = __half22float2(ph);
-          psum += pf.x + pf.y;
+          const float p0 = ex2_approx(sc[c] - m_new), p1 = ex2_approx(sc[c + 1] - m_new);
+          ps[(c >> 1) & 3] += p0 + p1;
+          const __half2 ph = __floats2half2_rn(p0, p1);
           packed[c / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
       }
-      uint8_t* prow = sP + row * 128;
+      const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      uint8_t* prow = sP + (jj & 1) * kPBytes + row * 128;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         const uint4 w = make_uint4(packed[cc * 4 + 0], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
@@ -245,21 +247,18 @@ __global__ void __launch_bounds__(192, 1)
           *p16 = w;
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
       return psum;
     };
     auto load_scores = [&](int jj, float (&sc)[64]) -> float {
       const int key0 = (crank + kCS * jj) * kChunk;
       tmem_ld64(tmem + lane_off + static_cast<uint32_t>((jj & 1) * kChunk), sc);
-      float mx = -INFINITY;
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < kChunk; ++c) {
         sc[c] = (key0 + c < limit) ? sc[c] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sc[c]);
+        mq[c & 3] = fmaxf(mq[c & 3], sc[c]);
       }
-      return mx;
+      return fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
     };
     for (int jj0 = 0; jj0 < nc; jj0 += 2) {
       const bool two = jj0 + 1 < nc;
@@ -283,7 +282,7 @@ __global__ void __launch_bounds__(192, 1)
       const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m - m_new);
       if (jj0 > 0) {
         // the previous pair's products are complete: O is stable, P is free
-        mbar_wait(pv_done, (jj0 - 1) & 1, a.status, sabort);
+        mbar_wait(pv_done, ((jj0 >> 1) - 1) & 1, a.status, sabort);
         tc_fence_after();
         // tcgen05.ld/st are warp-collective: rescale the whole warp when any
         // of its rows needs it (alpha == 1 leaves a row unchanged)
@@ -308,17 +307,19 @@ __global__ void __launch_bounds__(192, 1)
         psum = emit_p(jj0, sc, m_new);
       }
       if (two) {
-        mbar_wait(pv_done, jj0 & 1, a.status, sabort);  // P buffer free again
         float sc[64];
         load_scores(jj0 + 1, sc);
         psum += emit_p(jj0 + 1, sc, m_new);
       }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
       l = l * alpha + psum;
       m = m_new;
     }
     // Final PV done -> unnormalised partial O of this CTA into shared memory
     // (the K/V stages are free by then).
-    if (ok && nc > 0) mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort);
+    if (ok && nc > 0) mbar_wait(pv_done, ((nc - 1) >> 1) & 1, a.status, sabort);
     named_bar_sync(1, 128);
     const bool have = ok && nc > 0 && !*sabort;
     if (have) tc_fence_after();

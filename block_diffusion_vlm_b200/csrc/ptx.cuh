@@ -116,6 +116,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx: relative error about
+// 2^-22; -inf gives +0; subnormal results flush to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // GPU-scope acquire load / release add of a counter in global memory.
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
