@@ -387,27 +387,34 @@ __global__ void __launch_bounds__(192, 1)
     for (int k = 0; k < DPT; ++k) acc[k] = 0.f;
     float lsum = 0.f;
     if (got && M != -INFINITY) {
-      const uint4* rO16 = reinterpret_cast<const uint4*>(sRecvO);
-#pragma unroll 4
+      // weight of each partial: its sum l at the common maximum (0 for a
+      // source without keys for this row)
+      float w[kCS];
+#pragma unroll
       for (int s2 = 0; s2 < kCS; ++s2) {
         const float2 ml = sRecvML[s2 * RPC + rl];
-        if (ml.x == -INFINITY) continue;
-        // weight of this partial: its sum l at the common maximum
-        const float w = exp2f(ml.x - M) * ml.y;
-        lsum += w;
+        w[s2] = ml.x == -INFINITY ? 0.f : ex2_approx(ml.x - M) * ml.y;
+      }
+      const uint4* rO16 = reinterpret_cast<const uint4*>(sRecvO);
 #pragma unroll
-        for (int k = 0; k < DPT / 8; ++k) {
-          const int c8 = (d0 >> 3) + k;
-          const uint4 v = rO16[(s2 * RPC + rl) * 16 + (c8 ^ (r & 15))];
-          const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v);
+      for (int k = 0; k < DPT / 8; ++k) {
+        const int c8 = (d0 >> 3) + k;
+        uint4 v[kCS];
+#pragma unroll
+        for (int s2 = 0; s2 < kCS; ++s2) v[s2] = rO16[(s2 * RPC + rl) * 16 + (c8 ^ (r & 15))];
+#pragma unroll
+        for (int s2 = 0; s2 < kCS; ++s2) {
+          const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[s2]);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vw[q]));
-            acc[8 * k + 2 * q] += w * f.x;
-            acc[8 * k + 2 * q + 1] += w * f.y;
+            acc[8 * k + 2 * q] += w[s2] * f.x;
+            acc[8 * k + 2 * q + 1] += w[s2] * f.y;
           }
         }
       }
+#pragma unroll
+      for (int s2 = 0; s2 < kCS; ++s2) lsum += w[s2];
     }
     if (t < a.n_rows) {
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
