@@ -129,10 +129,21 @@ __global__ void __launch_bounds__(kWsThreads, 2)
         __threadfence();
 #pragma unroll
         for (int t = 0; t < NT; ++t) o[t] = 0.f;
-        for (int p = static_cast<int>(blockIdx.x) + 1; p <= pl; ++p) {
-          const float* src = ea.part + static_cast<size_t>(p) * 2 * NT * 128;
+        // the other CTAs' partials in CTA order, four sources' loads in flight
+        for (int p0 = static_cast<int>(blockIdx.x) + 1; p0 <= pl; p0 += 4) {
+          float q4[4][NT];
 #pragma unroll
-          for (int t = 0; t < NT; ++t) o[t] += __ldcg(&src[t * 128 + row]);
+          for (int q = 0; q < 4; ++q) {
+            const float* src = ea.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * 2 * NT * 128;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) q4[q][t] = __ldcg(&src[t * 128 + row]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (p0 + q <= pl) {
+#pragma unroll
+              for (int t = 0; t < NT; ++t) o[t] += q4[q][t];
+            }
         }
       }
       mbar_wait(&accf[b], (seg >> 1) & 1, ea.status, sabort);

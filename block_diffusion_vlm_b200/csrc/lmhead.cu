@@ -187,10 +187,22 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         __threadfence();
 #pragma unroll
         for (int t = 0; t < NT; ++t) o[t] = 0.f;
-        for (int p = static_cast<int>(blockIdx.x) + 1; p <= pl; ++p) {
-          const float* src = a.part + static_cast<size_t>(p) * 2 * NT * 128;
+        // the other CTAs' partials in CTA order, kQ sources' loads in flight
+        constexpr int kQ = NT <= 32 ? 2 : 1;
+        for (int p0 = static_cast<int>(blockIdx.x) + 1; p0 <= pl; p0 += kQ) {
+          float q2[kQ][NT];
 #pragma unroll
-          for (int t = 0; t < NT; ++t) o[t] += __ldcg(&src[t * 128 + et]);
+          for (int q = 0; q < kQ; ++q) {
+            const float* src = a.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * 2 * NT * 128;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) q2[q][t] = __ldcg(&src[t * 128 + et]);
+          }
+#pragma unroll
+          for (int q = 0; q < kQ; ++q)
+            if (p0 + q <= pl) {
+#pragma unroll
+              for (int t = 0; t < NT; ++t) o[t] += q2[q][t];
+            }
         }
       }
       mbar_wait(&accf[b], (seg >> 1) & 1, a.status, sabort);
