@@ -31,7 +31,7 @@ struct GemmSmem {
 };
 
 template <int NT, int STAGES, int EPI>
-__global__ void __launch_bounds__(kWsThreads, 2)
+__global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     gemm_ws_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
                    const __grid_constant__ CUtensorMap mapB, const SkSched sc, const int a_row_base,
                    const GemmEpi ea) {
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf[b], 1);
+      mbar_init(&accf[b], 2);
       mbar_init(&acce[b], 4);
     }
     *sabort = 0;
@@ -82,8 +82,9 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     if (lane == 0 && u1 > u0)
       ws_producer<NT, STAGES, EPI == EPI_SWIGLU>(&mapA, &mapA2, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base,
                                                  0, ea.status, sabort);
-  } else if (warp == 1) {
-    if (lane == 0 && u1 > u0) ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort);
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    if (lane == 0 && u1 > u0)
+      ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort, warp == 1 ? 0 : 1);
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       if (*sabort) break;
       tc_fence_after();
       float v[NT];
-      ws_load_acc<NT>(tmem, b, quarter, v);
+      ws_load_acc<NT>(tmem, b, quarter, v, seg_end - u >= 2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[b]);
@@ -272,7 +273,7 @@ struct ClSmem {
 };
 
 template <int NT, int STAGES, int EPI>
-__global__ void __launch_bounds__(kWsThreads, 2)
+__global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     gemm_cl_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const int kb,
                    const int S, const int a_row_base, const GemmEpi ea) {
   using Sm = ClSmem<NT, STAGES>;
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       mbar_init(&empty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf[b], 1);
+      mbar_init(&accf[b], 2);
       mbar_init(&acce[b], 4);
     }
     mbar_init(recv_full, 1);
@@ -349,8 +350,9 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     if (lane == 0 && u1 > u0)
       ws_producer<NT, STAGES, false>(&mapA, &mapA, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base, 0, ea.status,
                                      sabort);
-  } else if (warp == 1) {
-    if (lane == 0 && u1 > u0) ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort);
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    if (lane == 0 && u1 > u0)
+      ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort, warp == 1 ? 0 : 1);
   } else {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     if (u1 > u0) {
       mbar_wait(&accf[0], 0, ea.status, sabort);
       tc_fence_after();
-      ws_load_acc<NT>(tmem, 0, quarter, v);
+      ws_load_acc<NT>(tmem, 0, quarter, v, u1 - u0 >= 2);
     } else {
 #pragma unroll
       for (int t = 0; t < NT; ++t) v[t] = 0.f;
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
       bulk_commit();
     }
   }
-  if (warp < 2) {
+  if (warp < 2 || warp == kMmaWarp2) {
     __syncwarp();
     cluster_wait();
   }
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   // only after that (second barrier, waited on at exit).
   cluster_arrive();
 
-  if (threadIdx.x >= 64) {
+  if (warp >= 2 && warp < kMmaWarp2) {
     const bool got = mbar_wait(recv_full, 0, ea.status, sabort);
     const int rps = kPieces * myn;  // rows from each source
     // Sum of the S partials of element (rl, t) of this CTA's slice, in rank order.

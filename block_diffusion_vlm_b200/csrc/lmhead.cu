@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf[b], 1);
+      mbar_init(&accf[b], 2);
       mbar_init(&acce[b], 4);
     }
     *sabort = 0;
@@ -115,8 +115,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
       ws_producer<NT, STAGES, false>(&mapW, &mapW, &mapH, sA, sB, full, empty, sc, u0, u1, 0, 0, a.status, sabort);
-  } else if (warp == 1) {
-    if (lane == 0 && u1 > u0) ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, a.status, sabort);
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    if (lane == 0 && u1 > u0)
+      ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, a.status, sabort, warp == 1 ? 0 : 1);
   } else {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -214,10 +215,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < NT; c += 16) {
-        float tmp[16];
-        tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * NT + c), tmp);
+        float acc[16];
+        ws_load_acc16<NT>(tmem, b, quarter, c, acc, seg_end - u >= 2);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) sT[(c + k) * SROW + row] = tmp[k];
+        for (int k = 0; k < 16; ++k) sT[(c + k) * SROW + row] = acc[k];
       }
       tc_fence_before();
       __syncwarp();

@@ -30,12 +30,17 @@ struct SkSched {
   __host__ __device__ int first_tile(int p) const { return static_cast<int>(begin(p) / kb); }
 };
 
-constexpr int kWsThreads = 192;
+// Warp roles of the weight-streaming kernels: 0 TMA producer, 1 and 6 MMA
+// issuers (alternate k blocks of a segment into their own accumulators: one
+// issuing thread cannot keep a 16-column MMA fed at HBM speed), 2..5 epilogue.
+constexpr int kWsThreads = 224;
+constexpr int kMmaWarp2 = 6;
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
 
+// TMEM columns: 2 segment buffers x 2 issuers x NT (a power of two >= 32).
 template <int NT>
 __host__ __device__ constexpr int tmem_cols_for() {
-  return (2 * NT < 32) ? 32 : 2 * NT;
+  return (4 * NT < 32) ? 32 : 4 * NT;
 }
 
 // A operand source: one 128-row box, or two 64-row boxes from two tensors
@@ -84,47 +89,75 @@ __device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUten
 template <int NT, int STAGES>
 __device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty, uint64_t* accf,
                                        uint64_t* acce, uint32_t tmem, const SkSched& sc, long long u0, long long u1,
-                                       int* status, volatile int* abort_flag) {
+                                       int* status, volatile int* abort_flag, int issuer) {
+  // Issuer `issuer` (0 or 1) takes the k blocks j = issuer, issuer + 2, ... of
+  // each segment into accumulator (b, issuer); both commit accf[b] (count 2).
   constexpr int B_BYTES = NT * 128;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, NT);
   griddep_wait();
-  int i = 0, seg = 0;
+  long long i_base = 0;  // pipeline stage index of the segment's first k block
+  int seg = 0;
   for (long long u = u0; u < u1; ++seg) {
     const int T = static_cast<int>(u / sc.kb);
     const long long seg_end = (static_cast<long long>(T) + 1) * sc.kb < u1 ? (static_cast<long long>(T) + 1) * sc.kb : u1;
     const int b = seg & 1;
     if (seg >= 2 && !mbar_wait(&acce[b], ((seg >> 1) - 1) & 1, status, abort_flag)) return;
     tc_fence_after();
-    const uint32_t d = tmem + static_cast<uint32_t>(b * NT);
-    for (long long uu = u; uu < seg_end; ++uu, ++i) {
-      const int s = i % STAGES;
-      if (!mbar_wait(&full[s], (i / STAGES) & 1, status, abort_flag)) return;
+    const uint32_t d = tmem + static_cast<uint32_t>((b * 2 + issuer) * NT);
+    const long long len = seg_end - u;
+    for (long long jj = issuer; jj < len; jj += 2) {
+      const long long i = i_base + jj;
+      const int s = static_cast<int>(i % STAGES);
+      if (!mbar_wait(&full[s], static_cast<uint32_t>((i / STAGES) & 1), status, abort_flag)) return;
       tc_fence_after();
       const uint32_t a0 = smem_u32(sA + s * kATileBytes);
       const uint32_t b0 = smem_u32(sB + s * B_BYTES);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         umma_bf16_ss(d, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
-                     (uu > u || k > 0) ? 1u : 0u);
+                     (jj >= 2 || k > 0) ? 1u : 0u);
       }
       umma_commit(&empty[s]);
     }
     umma_commit(&accf[b]);
+    i_base += len;
     u = seg_end;
   }
 }
 
-// Copy the NT accumulator columns of TMEM buffer b for this thread's lane.
+// The NT accumulator columns of segment buffer b for this thread's lane: the
+// first issuer's accumulator plus, when the segment had two or more k blocks,
+// the second one's (fixed order).
 template <int NT>
-__device__ __forceinline__ void ws_load_acc(uint32_t tmem, int b, int quarter, float (&v)[NT]) {
+__device__ __forceinline__ void ws_load_acc(uint32_t tmem, int b, int quarter, float (&v)[NT], bool two) {
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll
   for (int c = 0; c < NT; c += 16) {
-    float tmp[16];
-    tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * NT + c), tmp);
+    float tmp[16], tmp2[16];
+    tmem_ld16(lane_base + static_cast<uint32_t>(b * 2 * NT + c), tmp);
+    if (two) {
+      tmem_ld16(lane_base + static_cast<uint32_t>((b * 2 + 1) * NT + c), tmp2);
+    } else {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) v[c + k] = tmp[k];
+      for (int k = 0; k < 16; ++k) tmp2[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[c + k] = tmp[k] + tmp2[k];
   }
   tmem_wait_ld();
+}
+
+// Columns [c, c+16) of the same sum.
+template <int NT>
+__device__ __forceinline__ void ws_load_acc16(uint32_t tmem, int b, int quarter, int c, float (&v)[16], bool two) {
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  float tmp2[16];
+  tmem_ld16(lane_base + static_cast<uint32_t>(b * 2 * NT + c), v);
+  if (two) {
+    tmem_ld16(lane_base + static_cast<uint32_t>((b * 2 + 1) * NT + c), tmp2);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] += tmp2[k];
+  }
 }
 
 __device__ __forceinline__ float bf16_round_f(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
