@@ -366,7 +366,7 @@ def _note_argmax_margin(tr: DecodeTrace, c: Conf, rows) -> None:
 
 
 def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, max_new: int,
-                     shift: int = 1, ar_seed: int = 1) -> DecodeTrace:
+                     shift: int = 1, ar_seed: int = 1, on_iter=None, on_block=None) -> DecodeTrace:
     """Threshold (MDM-style) block decoding [FDV §2.2.1, §2.2.2, §4.1].
 
     Per block: the first token is the AR seed (ar_seed=1); the remaining
@@ -375,7 +375,11 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
     scores the still-masked positions (position j from row j-shift; row -1 is
     the previous pass's last row) and commits per ``threshold_commit``.  When
     the block is complete a causal pass over it makes its K/V final, advances
-    L by B and yields the next block's seed from its last row."""
+    L by B and yields the next block's seed from its last row.
+
+    Optional observers (they do not change the trajectory): on_iter(L, toks,
+    masked, p1, top1, p2) before each iteration's commit, with the scores per
+    block position; on_block(L, toks) before each block's causal pass."""
     d = model.d
     tr = DecodeTrace(tokens=[])
     seed = seed_token
@@ -397,6 +401,8 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
                 r = j - shift
                 cc, rr = (prev_conf, 0) if r < 0 else (c, r)
                 p1[j], top[j], p2[j] = cc.p1[rr], cc.top1[rr], cc.p2[rr]
+            if on_iter is not None:
+                on_iter(L, list(toks), list(masked), p1.copy(), top.copy(), p2.copy())
             C = threshold_commit(p1, masked, tau)
             for j in range(B):
                 if masked[j]:
@@ -414,6 +420,8 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
                 masked[j] = False
             tr.commits_per_iter.append(len(C))
             tr.nfe += 1
+        if on_block is not None:
+            on_block(L, list(toks))
         x = model.forward(model.embed(toks), L, n_clean=B)
         model.L = L + B
         c = model.logits_conf(x)
