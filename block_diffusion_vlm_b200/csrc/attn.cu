@@ -367,6 +367,10 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
     cluster_wait();
   }
+  // Every CTA has issued its copies once all have arrived here: a CTA leaves
+  // only after that (second barrier, waited on at exit).
+  __syncwarp();
+  cluster_arrive();
   // ---------------------------------------------------------------- merge
   // CTA `crank` combines rows [crank*RPC, (crank+1)*RPC) over the kCS partials,
   // read from its own receive buffer in source order.
@@ -432,9 +436,11 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   if (warp == 2 && lane < kCS) bulk_wait_read_all();
-  // No CTA leaves while a copy into or out of its shared memory may run.
+  // No CTA leaves while a copy into or out of its shared memory may run: its
+  // own incoming copies landed (receive barrier), its outgoing ones have read
+  // their source, and every other CTA has issued its copies.
   tc_fence_before();
-  cluster_sync();
+  cluster_wait();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
