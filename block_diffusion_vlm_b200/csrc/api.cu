@@ -41,7 +41,6 @@ struct LmWs {
   float* part;
   int* cnt;
   float* rec;
-  int* valid;
   int* done;
   float* ssq;
   float* p1;
@@ -61,10 +60,9 @@ LmWs carve_lm(uint8_t* base, int R, int V, int H, dvlm_dtype dt, int P) {
   if (dt == DVLM_BF16) {
     const int NT = lm_nt(R);
     const int n_tiles = (V + 127) / 128;
-    w.part = reinterpret_cast<float*>(take(static_cast<size_t>(P) * 2 * NT * 128 * 4));
+    w.part = reinterpret_cast<float*>(take(static_cast<size_t>(P) * NT * 128 * 4));
     w.cnt = reinterpret_cast<int*>(take(static_cast<size_t>(n_tiles) * 4));
-    w.rec = reinterpret_cast<float*>(take(static_cast<size_t>(2) * P * NT * 16));
-    w.valid = reinterpret_cast<int*>(take(static_cast<size_t>(P) * 4));
+    w.rec = reinterpret_cast<float*>(take(static_cast<size_t>(P) * NT * 16));
     w.done = reinterpret_cast<int*>(take(4));
     w.ssq = reinterpret_cast<float*>(take(static_cast<size_t>(H / 128 + 1) * NT * 4));
   } else {
@@ -230,7 +228,6 @@ dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, int R, in
   a.part = lw.part;
   a.cnt = lw.cnt;
   a.rec = lw.rec;
-  a.split_valid = lw.valid;
   a.done = lw.done;
   if (apply_rmsnorm) {
     cudaError_t e = launch_embed_bf16(nullptr, static_cast<const bf16*>(hidden), R, nullptr, nullptr, 0, R, H, V,

@@ -66,10 +66,9 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->ssq = c.take<float>(((H / 128) * 16 + 1) * kNT * 4);
   e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, 2 * P));  // up to two CTAs per SM
   e->gcnt = c.take<int>(num_tiles_max(m) * 4);
-  e->lpart = c.take<float>(static_cast<size_t>(P) * 2 * kNT * 128 * 4);
+  e->lpart = c.take<float>(static_cast<size_t>(P) * kNT * 128 * 4);
   e->lcnt = c.take<int>(((m.vocab + 127) / 128) * 4);
-  e->lrec = c.take<float>(static_cast<size_t>(2) * P * kNT * 16);
-  e->lvalid = c.take<int>(P * 4);
+  e->lrec = c.take<float>(static_cast<size_t>(P) * kNT * 16);
   e->ldone = c.take<int>(4);
   e->d_len = c.take<int32_t>(4);
   e->d_seed = c.take<int32_t>(4);
@@ -124,7 +123,6 @@ static void fill_lm_scratch(dvlm_engine* e, LmArgs& a) {
   a.part = e->lpart;
   a.cnt = e->lcnt;
   a.rec = e->lrec;
-  a.split_valid = e->lvalid;
   a.done = e->ldone;
   a.status = e->d_status;
   a.V = e->m.vocab;

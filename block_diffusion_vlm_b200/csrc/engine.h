@@ -75,7 +75,6 @@ struct dvlm_engine {
   float* lpart = nullptr;   // LM head scratch
   int* lcnt = nullptr;
   float* lrec = nullptr;
-  int* lvalid = nullptr;
   int* ldone = nullptr;
   int32_t* d_len = nullptr;
   int32_t* d_seed = nullptr;

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
           float q4[4][NT];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float* src = ea.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * 2 * NT * 128;
+            const float* src = ea.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * NT * 128;
 #pragma unroll
             for (int t = 0; t < NT; ++t) q4[q][t] = __ldcg(&src[t * 128 + row]);
           }
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
       if (lane == 0) mbar_arrive(&acce[b]);
       if (!whole && !finisher) {
         // tail or middle part of a tile finished by another CTA
-        float* mine = ea.part + static_cast<size_t>(blockIdx.x) * 2 * NT * 128;
+        float* mine = ea.part + static_cast<size_t>(blockIdx.x) * NT * 128;
 #pragma unroll
         for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + row], v[t]);
         __threadfence();
@@ -596,7 +596,7 @@ int gemm_cl_max_clusters(int epi, int S, int stages) {
   return stages == 10 ? cl_max_clusters<10>(epi, S) : cl_max_clusters<5>(epi, S);
 }
 
-size_t gemm_ws_part_bytes(int NT, int P) { return static_cast<size_t>(P) * 2 * NT * 128 * sizeof(float); }
+size_t gemm_ws_part_bytes(int NT, int P) { return static_cast<size_t>(P) * NT * 128 * sizeof(float); }
 
 cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
                            int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s,

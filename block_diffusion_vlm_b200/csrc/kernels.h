@@ -50,11 +50,10 @@ struct LmArgs {
   int n_ssq;
   float inv_h, eps;
   // scratch
-  float* part;               // [P][2][NT][128]
-  int* cnt;                  // [n_tiles]
-  float* rec;                // [2][P][NT][4]: per-CTA and per-split-tile (m, s, idx)
-  int* split_valid;          // [P]
-  int* done;                 // [1]
+  float* part;               // [P][NT][128] partial logits of split tiles
+  int* cnt;                  // [n_tiles] (zero between launches)
+  float* rec;                // [P][NT][4]: per-CTA (m, s, idx)
+  int* done;                 // [1] (zero between launches)
   // commit / outputs
   uint8_t* masked;
   int32_t* tokens;

@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           float q2[kQ][NT];
 #pragma unroll
           for (int q = 0; q < kQ; ++q) {
-            const float* src = a.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * 2 * NT * 128;
+            const float* src = a.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * NT * 128;
 #pragma unroll
             for (int t = 0; t < NT; ++t) q2[q][t] = __ldcg(&src[t * 128 + et]);
           }
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       bar();
       if (!whole && !finisher) {
         // tail or middle part of a tile finished by another CTA
-        float* mine = a.part + static_cast<size_t>(blockIdx.x) * 2 * NT * 128;
+        float* mine = a.part + static_cast<size_t>(blockIdx.x) * NT * 128;
 #pragma unroll
         for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + et], sT[t * SROW + et]);
         __threadfence();
@@ -294,9 +294,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 }
 
 size_t lmhead_scratch_bytes(int NT, int P, int n_tiles) {
-  size_t part = static_cast<size_t>(P) * 2 * NT * 128 * 4;
-  size_t rec = static_cast<size_t>(2) * P * NT * 16;
-  size_t ints = (static_cast<size_t>(n_tiles) + P + 1) * 4;
+  size_t part = static_cast<size_t>(P) * NT * 128 * 4;
+  size_t rec = static_cast<size_t>(P) * NT * 16;
+  size_t ints = (static_cast<size_t>(n_tiles) + 1) * 4;
   return part + rec + ints + 256;
 }
 

@@ -45,7 +45,7 @@ cudaError_t scratch_address(void** out) {
 }
 
 struct StaticLayout {
-  size_t part, cnt, valid, done, rec, ssq, bytes;
+  size_t part, cnt, done, rec, ssq, bytes;
   size_t zero_begin, zero_end;  // counters that must start at zero
 };
 
@@ -55,18 +55,16 @@ StaticLayout layout(int NT, int P, int n_tiles, int H) {
   StaticLayout L{};
   size_t off = 0;
   L.part = off;
-  off = up256(off + static_cast<size_t>(P) * 2 * NT * 128 * 4);
+  off = up256(off + static_cast<size_t>(P) * NT * 128 * 4);
   L.cnt = off;
   L.zero_begin = off;
   off += static_cast<size_t>(n_tiles) * 4;
-  L.valid = off;
-  off += static_cast<size_t>(P) * 4;
   L.done = off;
   off += 4;
   L.zero_end = off;
   off = up256(off);
   L.rec = off;
-  off = up256(off + static_cast<size_t>(2) * P * NT * 16);
+  off = up256(off + static_cast<size_t>(P) * NT * 16);
   L.ssq = off;
   off = up256(off + static_cast<size_t>(H / 128 + 1) * NT * 4);
   L.bytes = off;
@@ -119,7 +117,6 @@ extern "C" dvlm_status dvlm_lmhead_conf_commit_static(
   a.part = reinterpret_cast<float*>(s + lay.part);
   a.cnt = reinterpret_cast<int*>(s + lay.cnt);
   a.rec = reinterpret_cast<float*>(s + lay.rec);
-  a.split_valid = reinterpret_cast<int*>(s + lay.valid);
   a.done = reinterpret_cast<int*>(s + lay.done);
   a.masked = masked;
   a.tokens = tokens;

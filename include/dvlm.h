@@ -147,7 +147,7 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, 
  * method's pages: this is a deployment variant.  It takes no workspace: its
  * scratch is one fixed 6 MiB device array inside the library, present on
  * every GPU that loads the library until the process exits.  Limits: R <= 32
- * and a scratch layout (about 33 KiB per SM plus 4 bytes per 128 vocabulary
+ * and a scratch layout (about 17 KiB per SM plus 4 bytes per 128 vocabulary
  * rows) within 6 MiB, e.g. V <= 262144 and H <= 8192 on a 148-SM B200;
  * larger requests return DVLM_ERR_WORKSPACE and launch nothing.  The first
  * call on a device looks the array's device address up (make that first call
