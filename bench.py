@@ -179,12 +179,21 @@ def load_traffic(kernel: str):
 
 
 def source_hash() -> str:
+    """Hash of the kernel sources with comments and white space removed: the
+    recorded DRAM traffic stays attached to the code it was measured on, and a
+    comment-only edit does not detach it."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_diffusion_vlm_b200", "csrc")
     for n in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, n), encoding="utf-8") as f:
+            txt = f.read()
+        txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)
+        txt = re.sub(r"//[^\n]*", " ", txt)
+        txt = re.sub(r"\s+", " ", txt).strip()
+        h.update(n.encode())
+        h.update(txt.encode())
     return h.hexdigest()[:16]
 
 

@@ -11,11 +11,14 @@
 // TMA box lands).  S = Q K^T (N = 64 keys) and O += P V (V stored
 // value-feature-major so both products read K-major operands) accumulate in
 // TMEM; softmax runs in fp32 registers, one thread per row, with P rounded
-// to fp16 for the second product (the value tile converted to fp16 too).  The keys are split over a cluster of 8 or 16 CTAs;
-// the partial (max, sum, O) of the cluster's CTAs are merged through
-// distributed shared memory, so there is no second kernel and no global
-// scratch.  Clusters of 16 CTAs (where the device can co-schedule them) put
-// one or two 64-key chunks on each CTA at decode lengths.
+// to fp16 for the second product (the value tile converted to fp16 too).
+// The keys are split over a cluster of 8 or 16 CTAs in 64-key chunks (chunk j
+// on CTA j mod cluster size); each CTA pushes its partial rows (max, sum and
+// the fp16 output rows divided by their sum) with bulk shared-memory copies to
+// the CTA that owns those rows, which merges them in source order, so there is
+// no second kernel and no global scratch.  Clusters of 16 CTAs (where the
+// device can co-schedule them) put one or two chunks on each CTA at decode
+// lengths.
 #include <cuda_fp16.h>
 
 #include "kernels.h"

@@ -36,7 +36,7 @@ struct GemmEpi {
   const int* d_len;           // slot of row 0 (device); NULL -> L_static
   int L_static;
   double log2_rope_base;
-  // split-tile scratch: part [P][2][NT][128] fp32, cnt [n_tiles] int (zero)
+  // stream-K scratch: part [P][NT][128] fp32 (one partial tile per CTA), cnt [n_tiles] int (zero)
   float* part;
   int* cnt;
   int* status;

@@ -6,14 +6,19 @@
 // k) is the 128-row UMMA A operand, the token rows (NT = 16..128) are the
 // N side, and the fp32 accumulator lives in TMEM (128 lanes x NT columns).
 //
-// Work split: the (output tile, 64-wide k block) units are cut into P equal
-// contiguous ranges, one per CTA (stream-K).  A tile whose k range spans two
-// or more CTAs is finished by whichever contributor arrives last (per-tile
-// counter, no spinning), summing the partial tiles in a fixed order so the
-// result is deterministic.
+// Work split (stream-K kernels): the (output tile, 64-wide k block) units are
+// cut into P equal contiguous ranges, one per CTA.  A tile whose k range spans
+// two or more CTAs is finished by the CTA that streams its first k blocks (the
+// last segment of that CTA's range); the others stream their parts first,
+// store fp32 partial tiles and count them on a per-tile counter, and the
+// finisher adds them in CTA order, so the result is deterministic.  The
+// cluster split-K kernels use the same producer and MMA roles with one tile
+// per cluster.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
-// UMMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Roles (224 threads): warp 0 lane 0 issues TMA loads; warps 1 and 6 (lane 0)
+// issue UMMAs for alternate k blocks of each segment into their own TMEM
+// accumulators; warps 2..5 run the epilogue (warp w reads TMEM lanes
+// 32*(w%4)..+31) and add the two accumulators.
 #pragma once
 #include "ptx.cuh"
 
