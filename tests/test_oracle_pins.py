@@ -279,6 +279,28 @@ def test_threshold_extreme_thresholds():
     assert tr.commits_per_iter == [B - 1, B - 1] and tr.nfe == 4
 
 
+def test_threshold_observers_do_not_change_the_trajectory():
+    """The per-iteration observers used by the teacher-forced GPU checks see
+    every iteration (with the scores the commit is decided on) and every block,
+    and leave tokens, forwards and commits unchanged."""
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s = _fresh(d, w, True, vis, ids)
+    plain = O.decode_threshold(m, s, B, 0.9, 2 * B)
+    seen, blocks = [], []
+
+    def on_iter(L, toks, masked, p1, top, p2):
+        seen.append((L, list(toks), list(masked)))
+        assert len(p1) == len(top) == len(p2) == B and all(p1 >= p2)
+
+    m, s = _fresh(d, w, True, vis, ids)
+    obs = O.decode_threshold(m, s, B, 0.9, 2 * B, on_iter=on_iter, on_block=lambda L, toks: blocks.append((L, toks)))
+    assert obs.tokens == plain.tokens and obs.nfe == plain.nfe and obs.commits_per_iter == plain.commits_per_iter
+    assert len(seen) == sum(1 for _ in plain.commits_per_iter) and len(blocks) == 2
+    assert [b[1] for b in blocks] == [plain.tokens[:B], plain.tokens[B:2 * B]]
+    assert blocks[1][0] == blocks[0][0] + B
+
+
 def test_block_first_token_is_ar_token_and_append_kv_equals_prefill():
     gd, d, w, vis, ids = _tiny()
     B = 4
