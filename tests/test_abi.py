@@ -5,7 +5,6 @@ import ctypes
 import os
 import subprocess
 
-import pytest
 
 import block_diffusion_vlm_b200 as dv
 from block_diffusion_vlm_b200 import binding

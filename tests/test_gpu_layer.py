@@ -17,7 +17,7 @@ import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
 import oracle as O
 from dvlm_gen.device import DeviceModel, kv_buffers
-from gpu_util import assert_bf16_close, f64, max_abs, ws_tensor
+from gpu_util import assert_bf16_close, f64, ws_tensor
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2

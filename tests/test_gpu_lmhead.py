@@ -12,7 +12,7 @@ import torch
 import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
 import oracle as O
-from gpu_util import assert_ok, f64, status, ws_tensor
+from gpu_util import assert_ok, status, ws_tensor
 
 pytestmark = pytest.mark.gpu
 MARGIN = 1e-3
