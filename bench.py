@@ -162,31 +162,45 @@ def algorithmic_bytes(kind: str, dims, L: int, rows: int = 16) -> float:
     return 0.0
 
 
+# Kernel sources (under block_diffusion_vlm_b200/csrc) each recorded DRAM
+# traffic depends on: the kernel's own file, the shared device headers and the
+# engine that plans its launch shape.
+_COMMON_SOURCES = ["ptx.cuh", "mainloop.cuh", "kernels.h", "tmap.cu", "engine.cu", "engine.h"]
+TRAFFIC_SOURCES = {
+    "qkv_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
+    "oproj_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
+    "gateup_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
+    "down_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
+    "lm_head": _COMMON_SOURCES + ["lmhead.cu", "finalize.cuh"],
+    "attention": _COMMON_SOURCES + ["attn.cu"],
+}
+
+
 def load_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, when it was taken
-    on the current kernel source; else None."""
+    on the kernel's current sources; else None."""
     p = os.path.join(PROFILE_DIR, "traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kernel not in TRAFFIC_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
     ent = d.get(kernel)
     if not ent:
         return None
-    if ent.get("source_hash") != source_hash():
+    if ent.get("source_hash") != source_hash(TRAFFIC_SOURCES[kernel]):
         return None
     return ent.get("dram_bytes_per_launch")
 
 
-def source_hash() -> str:
-    """Hash of the kernel sources with comments and white space removed: the
-    recorded DRAM traffic stays attached to the code it was measured on, and a
-    comment-only edit does not detach it."""
+def source_hash(files=None) -> str:
+    """Hash of kernel sources (all of csrc, or the listed files) with comments
+    and white space removed: the recorded DRAM traffic stays attached to the
+    code it was measured on, and a comment-only edit does not detach it."""
     import hashlib
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_diffusion_vlm_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
+    for n in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, n), encoding="utf-8") as f:
             txt = f.read()
         txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)

@@ -21,6 +21,17 @@ def bench_copy(tmp_path, monkeypatch):
     return bench, dst
 
 
+def test_traffic_key_covers_only_the_kernels_sources(bench_copy):
+    bench, csrc = bench_copy
+    h0 = bench.source_hash(bench.TRAFFIC_SOURCES["lm_head"])
+    f = csrc / "spec.cu"
+    f.write_text(f.read_text() + "\nstatic int unrelated_edit;\n")
+    assert bench.source_hash(bench.TRAFFIC_SOURCES["lm_head"]) == h0
+    f = csrc / "lmhead.cu"
+    f.write_text(f.read_text() + "\nstatic int related_edit;\n")
+    assert bench.source_hash(bench.TRAFFIC_SOURCES["lm_head"]) != h0
+
+
 def test_source_hash_ignores_comments_but_not_code(bench_copy):
     bench, csrc = bench_copy
     h0 = bench.source_hash()
