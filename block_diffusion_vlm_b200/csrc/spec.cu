@@ -55,7 +55,30 @@ __global__ void spec_logits_kernel(const bf16* __restrict__ logits, const int32_
   float best = -INFINITY;
   int bidx = 0x7fffffff;
   const bool vec = (V % 8) == 0;  // rows start 16-byte aligned only then
-  for (int v = v0 + threadIdx.x * 8; v < v1; v += blockDim.x * 8) {
+  // Four 16-byte loads in flight per thread, scanned in index order (a tie
+  // keeps the earlier, lower id).
+  const int step = blockDim.x * 8;
+  int v = v0 + threadIdx.x * 8;
+  if (vec) {
+    for (; v + 3 * step + 8 <= v1; v += 4 * step) {
+      uint4 w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint4*>(row + v + u * step);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bf16* e = reinterpret_cast<const bf16*>(&w[u]);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float x = __bfloat162float(e[q]);
+          if (x > best) {
+            best = x;
+            bidx = v + u * step + q;
+          }
+        }
+      }
+    }
+  }
+  for (; v < v1; v += step) {
     if (vec && v + 8 <= v1) {
       const uint4 w = *reinterpret_cast<const uint4*>(row + v);
       const bf16* e = reinterpret_cast<const bf16*>(&w);
@@ -109,13 +132,21 @@ __global__ void spec_logits_kernel(const bf16* __restrict__ logits, const int32_
   if (threadIdx.x < B) {
     float bb = -INFINITY;
     int ii = 0x7fffffff;
-    for (int s = 0; s < splits; ++s) {
-      const float* p = part + ((static_cast<size_t>(i) * B + threadIdx.x) * splits + s) * 2;
-      const float x = __ldcg(&p[0]);
-      const int ix = __float_as_int(__ldcg(&p[1]));
-      if (x > bb || (x == bb && ix < ii)) {
-        bb = x;
-        ii = ix;
+    // the row's split results in split order, eight loads in flight
+    const float2* p = reinterpret_cast<const float2*>(part) + (static_cast<size_t>(i) * B + threadIdx.x) * splits;
+    for (int s0 = 0; s0 < splits; s0 += 8) {
+      float2 r[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) r[q] = s0 + q < splits ? __ldcg(&p[s0 + q]) : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (s0 + q >= splits) break;
+        const float x = r[q].x;
+        const int ix = __float_as_int(r[q].y);
+        if (x > bb || (x == bb && ix < ii)) {
+          bb = x;
+          ii = ix;
+        }
       }
     }
     s_v[threadIdx.x] = ii;
