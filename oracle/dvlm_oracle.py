@@ -28,6 +28,10 @@ its reason in the repository's design notes):
   commit    p1 >= threshold; if none passes, the masked position with the
             highest p1 (lowest position on ties) is committed.
   argmax    lowest vocabulary id among equal maxima.
+  fp8       (next step, not on the bf16 path) W8A8 in E4M3, finite variant,
+            round to nearest even, saturating at 448; one scale per weight
+            output channel and per activation token (amax / 448);
+            SmoothQuant factors with alpha = 0.5.
   norms     RMSNorm gain 1, eps 1e-6, no biases; RoPE rotate-half, base 1e4.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
@@ -56,6 +60,58 @@ def bf16_round(x) -> np.ndarray:
     m, e = np.frexp(x)                    # x = m * 2**e, 0.5 <= |m| < 1
     r = np.round(m * 256.0)               # numpy rounds half to even
     return np.ldexp(r, e - 8)
+
+
+# ----------------------------------------------------------------------------
+# FP8 W8A8 linear layer (next step of the weight stream; not on the bf16 path)
+# ----------------------------------------------------------------------------
+# [FDV §2.3.2] names SmoothQuant W8A8 FP8 as the final serving step.  The pages
+# give no formats or granularity; readings taken: E4M3 (finite variant) for
+# both operands, one scale per weight output channel and per activation token
+# (amax / 448), round to nearest even, SmoothQuant factors with alpha = 0.5.
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round real values to FP8 E4M3 (4 exponent bits with bias 7, 3 mantissa
+    bits, subnormals down to 2^-9, largest finite 448), ties to even, returned
+    as float64.  Magnitudes beyond 448 saturate to 448 (the per-row scales
+    below keep every quantised value within range)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    _, e = np.frexp(a)                     # leading bit of a is 2^(e-1)
+    e = np.maximum(e, -5)                  # below 2^-6: the subnormal spacing 2^-9
+    q = np.ldexp(1.0, e - 4)               # 3 mantissa bits below the leading bit
+    r = np.round(a / q) * q                # numpy rounds half to even
+    return np.sign(x) * np.minimum(r, E4M3_MAX)
+
+
+def fp8_quantize_rows(A: np.ndarray):
+    """Per-row FP8 quantisation: scale s_r = max_k |A[r, k]| / 448 (1 for an
+    all-zero row) and codes A_q = e4m3(A / s_r); A ~ s_r * A_q.  Rows are
+    output channels for weights [out, in] and tokens for activations."""
+    A = np.asarray(A, dtype=np.float64)
+    amax = np.max(np.abs(A), axis=1)
+    s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    return e4m3_round(A / s[:, None]), s
+
+
+def fp8_linear(x: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """W8A8 product y[t, o] = a_t * s_o * sum_k xq[t, k] Wq[o, k] of per-token
+    quantised activations and per-output-channel quantised weights; the
+    products of two E4M3 values and their sums are exact in float64 for the
+    layer sizes here (every term is a multiple of 2^-18 below 2^18)."""
+    xq, a = fp8_quantize_rows(x)
+    wq, s = fp8_quantize_rows(W)
+    return (xq @ wq.T) * a[:, None] * s[None, :]
+
+
+def smooth_factors(x_amax: np.ndarray, w_amax: np.ndarray, alpha: float = 0.5) -> np.ndarray:
+    """SmoothQuant factor per input channel k: m_k = x_amax_k^alpha /
+    w_amax_k^(1 - alpha).  The layer then quantises x / m and W * m (per input
+    channel), whose product equals x W^T before quantisation."""
+    return np.power(np.asarray(x_amax, dtype=np.float64), alpha) / np.power(np.asarray(w_amax, dtype=np.float64),
+                                                                            1.0 - alpha)
 
 
 # ----------------------------------------------------------------------------

@@ -377,6 +377,143 @@ def _check_argmax(fn):
     assert fn(np.array([[1.0, 5.0, 0.0, 5.0, 2.0]])).top1[0] == 1
 
 
+# ----------------------------------------------------------------------------
+# FP8 W8A8 linear layer (next step of the weight stream)
+# ----------------------------------------------------------------------------
+def _e4m3_grid():
+    """Every finite non-negative E4M3 value, from torch's own decoding."""
+    codes = torch.arange(0, 128, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    return np.unique(codes[np.isfinite(codes)])
+
+
+def test_e4m3_round_matches_torch_cast_and_ties():
+    g = _e4m3_grid()
+    assert g.max() == O.E4M3_MAX and g[1] == 2.0 ** -9 and len(g) == 127
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.uniform(-448, 448, 20000), rng.standard_normal(20000) * 2.0 ** -7,
+                        g, -g, (g[1:] + g[:-1]) / 2, -(g[1:] + g[:-1]) / 2,   # every exact midpoint
+                        rng.uniform(448, 463.9, 100)])                       # rounds down to 448
+    x = x.astype(np.float32).astype(np.float64)                             # exact inputs for torch's cast
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    np.testing.assert_array_equal(O.e4m3_round(x), ref)
+    # beyond the finite range the definition saturates (torch's cast gives NaN)
+    np.testing.assert_array_equal(O.e4m3_round(np.array([500.0, -1e6])), [448.0, -448.0])
+
+
+def test_fp8_row_scales_and_power_of_two_invariance():
+    rng = np.random.default_rng(4)
+    A = rng.standard_normal((6, 96))
+    A[2] = 0.0
+    q, s = O.fp8_quantize_rows(A)
+    for r in range(6):
+        if r == 2:
+            assert s[r] == 1.0 and not q[r].any()
+            continue
+        k = np.argmax(np.abs(A[r]))
+        assert abs(q[r, k]) == O.E4M3_MAX                      # the row's largest entry maps to +-448
+        assert np.all(np.isin(np.abs(q[r]), _e4m3_grid()))      # codes are E4M3 values
+    q2, s2 = O.fp8_quantize_rows(A * np.array([1, 2.0 ** 5, 1, 2.0 ** -7, 1, 1])[:, None])
+    np.testing.assert_array_equal(q2, q)                        # scaling a row by 2^k moves only its scale
+    np.testing.assert_allclose(s2 / s, [1, 2.0 ** 5, 1, 2.0 ** -7, 1, 1], rtol=0, atol=0)
+
+
+def test_fp8_linear_exact_when_operands_are_representable():
+    """Rows made of E4M3 values times 2^j that contain +-448 * 2^j have scale
+    2^j and quantise without error: the W8A8 product is then the exact product."""
+    rng = np.random.default_rng(5)
+    g = _e4m3_grid()
+    vals = np.concatenate([g, -g])
+
+    def rows(n, k, jlo, jhi):
+        j = rng.integers(jlo, jhi, (n, 1))
+        A = rng.choice(vals, (n, k))
+        A[:, 0] = O.E4M3_MAX * rng.choice([-1.0, 1.0], n)
+        return A * 2.0 ** j
+
+    x, W = rows(8, 64, -3, 4), rows(16, 64, -6, 2)
+    assert np.array_equal(O.fp8_quantize_rows(x)[0] * O.fp8_quantize_rows(x)[1][:, None], x)
+    np.testing.assert_array_equal(O.fp8_linear(x, W), x @ W.T)
+
+
+def test_fp8_linear_error_bound():
+    """|y_fp8 - x W^T| stays within the bound an E4M3 code error implies:
+    per element at most 2^-4 relative (normal codes) or 2^-10 of the row
+    scale (subnormal codes), so a dropped scale, a wrong axis or truncation
+    would break it by orders of magnitude or on average."""
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((16, 2048))
+    W = rng.standard_normal((256, 2048)) * 0.02
+    y = O.fp8_linear(x, W)
+    exact = x @ W.T
+    xq, a = O.fp8_quantize_rows(x)
+    wq, s = O.fp8_quantize_rows(W)
+    dx = np.maximum(np.abs(x) * 2.0 ** -4, a[:, None] * 2.0 ** -10)
+    dw = np.maximum(np.abs(W) * 2.0 ** -4, s[:, None] * 2.0 ** -10)
+    bound = dx @ np.abs(W).T + np.abs(x) @ dw.T + dx @ dw.T
+    assert np.all(np.abs(y - exact) <= bound)
+    # round to nearest is unbiased: no systematic shrink or growth of |y|
+    # (rounding toward zero would shrink it by about 3%)
+    bias = np.mean(np.sign(exact) * (y - exact)) / np.mean(np.abs(exact))
+    assert abs(bias) < 0.005
+
+
+def test_smooth_factors_balance_channels_and_keep_the_product():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((32, 64)) * rng.uniform(0.1, 20, 64)
+    W = rng.standard_normal((48, 64)) * rng.uniform(0.001, 0.1, 64)
+    xa, wa = np.max(np.abs(x), axis=0), np.max(np.abs(W), axis=0)
+    m = O.smooth_factors(xa, wa, 0.5)
+    np.testing.assert_allclose(xa / m, wa * m, rtol=1e-12)       # alpha 0.5: equal channel ranges
+    np.testing.assert_allclose((x / m) @ (W * m).T, x @ W.T, rtol=1e-12, atol=1e-12)
+    m1 = O.smooth_factors(xa, wa, 1.0)
+    np.testing.assert_allclose(np.max(np.abs(x / m1), axis=0), 1.0, rtol=1e-12)   # alpha 1: all range to W
+
+
+def test_fp8_planted_mistakes_are_caught(monkeypatch):
+    """Each plausible slip in the FP8 definitions fails at least one FP8 pin."""
+    import oracle.dvlm_oracle as OM
+    real_round, real_rows, real_linear = OM.e4m3_round, OM.fp8_quantize_rows, OM.fp8_linear
+
+    def round_toward_zero(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.minimum(np.abs(x), OM.E4M3_MAX)
+        _, e = np.frexp(a)
+        q = np.ldexp(1.0, np.maximum(e, -5) - 4)
+        return np.sign(x) * np.trunc(a / q) * q
+
+    def subnormal_floor_too_low(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.minimum(np.abs(x), OM.E4M3_MAX)
+        _, e = np.frexp(a)
+        q = np.ldexp(1.0, np.maximum(e, -6) - 4)
+        return np.sign(x) * np.minimum(np.round(a / q) * q, OM.E4M3_MAX)
+
+    def scales_per_column(A):
+        q, s = real_rows(np.asarray(A).T)
+        return q.T, s
+
+    def no_activation_scale(x, W):
+        xq, _ = real_rows(x)
+        wq, s = real_rows(W)
+        return (xq @ wq.T) * s[None, :]
+
+    pins = [test_e4m3_round_matches_torch_cast_and_ties, test_fp8_row_scales_and_power_of_two_invariance,
+            test_fp8_linear_exact_when_operands_are_representable, test_fp8_linear_error_bound]
+    for name, mutant in [("e4m3_round", round_toward_zero), ("e4m3_round", subnormal_floor_too_low),
+                         ("fp8_quantize_rows", scales_per_column), ("fp8_linear", no_activation_scale)]:
+        with monkeypatch.context() as mp:
+            mp.setattr(OM, name, mutant)
+            mp.setattr(O, name, mutant)
+            failed = 0
+            for pin in pins:
+                try:
+                    pin()
+                except (AssertionError, ValueError, IndexError):   # wrong values or wrong scale shapes
+                    failed += 1
+            assert failed > 0, name
+    assert OM.e4m3_round is real_round and OM.fp8_linear is real_linear
+
+
 def test_pins_accept_the_oracle():
     _check_rope(O.rope)
     _check_commit(O.threshold_commit)
