@@ -402,7 +402,9 @@ dvlm_status dvlm_decode_block(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_
   if (L + cfg->block_size > e->Lmax) return DVLM_ERR_CACHE_OVERFLOW;
   if (cudaMemsetAsync(e->n_out, 0, 4, s) != cudaSuccess) return DVLM_ERR_CUDA;
   int emitted = 0;
-  if (engine_step(e, *cfg, cfg->block_size, 0, &emitted, stats, s) != cudaSuccess) return DVLM_ERR_CUDA;
+  const cudaError_t r = engine_step(e, *cfg, cfg->block_size, 0, &emitted, stats, s);
+  if (r == cudaErrorLaunchTimeout) return DVLM_ERR_TIMEOUT;
+  if (r != cudaSuccess) return DVLM_ERR_CUDA;
   if (emitted > 0 && cudaMemcpyAsync(out_tokens, e->stage_out, static_cast<size_t>(emitted) * 4,
                                      cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return DVLM_ERR_CUDA;
@@ -423,7 +425,9 @@ static dvlm_status generate_impl(dvlm_engine* e, const dvlm_decode_cfg* cfg, dvl
   int n = 0;
   while (n < cfg->max_new_tokens) {
     int emitted = 0;
-    if (engine_step(e, *cfg, cfg->max_new_tokens, n, &emitted, stats, s) != cudaSuccess) return DVLM_ERR_CUDA;
+    const cudaError_t r = engine_step(e, *cfg, cfg->max_new_tokens, n, &emitted, stats, s);
+    if (r == cudaErrorLaunchTimeout) return DVLM_ERR_TIMEOUT;
+    if (r != cudaSuccess) return DVLM_ERR_CUDA;
     n += emitted;
   }
   if (stats) stats->n_tokens += n;

@@ -378,7 +378,10 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
   DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, e->m.mask_id, 1, e->n_remaining, s));
   if (cfg.mode == DVLM_MODE_THRESHOLD) {
     int rem = B - 1;
-    while (rem > 0) {
+    for (int it = 0; rem > 0; ++it) {
+      // every iteration commits at least one position: a block needing more
+      // than B - 1 means a device-side wait gave up (see the status word)
+      if (it >= B - 1) return cudaErrorLaunchTimeout;
       DVLM_CK(run_graph(e, {G_NOISY, B, fbits(cfg.threshold)}, ug, s, [&]() -> cudaError_t {
         FwdSpec f;
         f.tokens = e->tokens;
@@ -460,6 +463,8 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
   int32_t h = 0;
   DVLM_CK(cudaMemcpyAsync(&h, e->n_out, 4, cudaMemcpyDeviceToHost, s));
   DVLM_CK(cudaStreamSynchronize(s));
+  // a round always keeps at least the AR seed: none means a device-side wait gave up
+  if (h <= n_out_host) return cudaErrorLaunchTimeout;
   if (st) {
     st->nfe += 2;
     st->n_rounds += 1;

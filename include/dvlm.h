@@ -261,10 +261,14 @@ DVLM_API dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_visi
 /* Decodes one block (threshold/AR modes: B tokens; spec mode: one draft +
  * verify round, 1..B tokens).  Tokens go to out_tokens (device, >= B
  * entries); *n_out (host) receives their count.  Synchronises the stream
- * once per noisy iteration (threshold mode) or round.  stats accumulate. */
+ * once per noisy iteration (threshold mode) or round.  stats accumulate.
+ * Returns DVLM_ERR_TIMEOUT when a block needs more than B - 1 noisy
+ * iterations or a speculative round keeps no token: both mean a device-side
+ * wait gave up (the status word, dvlm_engine_check, says where). */
 DVLM_API dvlm_status dvlm_decode_block(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_t* out_tokens,
                               int32_t* n_out, dvlm_stats* stats, dvlm_stream stream);
-/* Decodes exactly cfg->max_new_tokens tokens into out_tokens (device). */
+/* Decodes exactly cfg->max_new_tokens tokens into out_tokens (device).
+ * Errors as dvlm_decode_block. */
 DVLM_API dvlm_status dvlm_generate(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_t* out_tokens,
                           dvlm_stats* stats, dvlm_stream stream);
 /* End to end from HOST buffers: copies vision_host [n_vision, H] (model
