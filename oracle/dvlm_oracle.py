@@ -33,6 +33,11 @@ its reason in the repository's design notes):
             output channel and per activation token (amax / 448);
             SmoothQuant factors with alpha = 0.5.
   norms     RMSNorm gain 1, eps 1e-6, no biases; RoPE rotate-half, base 1e4.
+  lown      (next step) TEXT-ONLY = the vision cache slots hidden from the
+            block's queries, position ids unchanged; each block opens with a
+            FULL pass unmasking min(k, masked) by confidence; the certified
+            prefix is unmasked with the anchor ids; the FULL branch puts
+            divergent positions first, each group by FULL confidence.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against brute force, closed forms, library routines or the pages' printed
@@ -192,14 +197,16 @@ def dense_masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np
 
 
 def block_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, L: int, n_clean: int,
-                    scale: float) -> np.ndarray:
+                    scale: float, hide: int = 0) -> np.ndarray:
     """Attention of one step's rows against the KV cache.
 
     q: [n, Hq, D] for rows at cache slots L .. L+n-1 (their K/V already in the
     cache).  K, V: [Hkv, >= L+n, D].  Rows 0..n_clean-1 are clean (causal:
     row t sees slots 0..L+t); the remaining rows form the noisy block and see
     every slot 0..L+n-1 (the whole cache through N2C plus the whole block
-    through N2N)."""
+    through N2N).  ``hide``: slots 0..hide-1 are invisible to every row (the
+    TEXT-ONLY pass of certificate routing drops the vision tokens, which sit
+    at the front of the cache; positions are unchanged) [LOWN method step (2)]."""
     q = np.asarray(q, dtype=np.float64)
     n, Hq, D = q.shape
     Hkv = K.shape[0]
@@ -209,10 +216,10 @@ def block_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, L: int, n_clean
         vis = (L + t + 1) if t < n_clean else (L + n)
         for h in range(Hq):
             g = h // G
-            s = scale * (K[g, :vis] @ q[t, h])
+            s = scale * (K[g, hide:vis] @ q[t, h])
             p = np.exp(s - s.max())
             p /= p.sum()
-            out[t, h] = p @ V[g, :vis]
+            out[t, h] = p @ V[g, hide:vis]
     return out
 
 
@@ -280,6 +287,24 @@ def certificate_scan(anchor_id: Sequence[int], anchor_conf: Sequence[float],
     return n
 
 
+def certificate_order(anchor_conf: Sequence[float], participants: Sequence[bool]) -> List[int]:
+    """Positions in the order the certificate scan visits them: descending
+    anchor confidence, lower index first on ties [LOWN method step (2)]."""
+    idx = [i for i in range(len(anchor_conf)) if participants[i]]
+    idx.sort(key=lambda i: (-float(anchor_conf[i]), i))
+    return idx
+
+
+def divergence_first_order(full_top1: Sequence[int], full_conf: Sequence[float], text_top1: Sequence[int],
+                           participants: Sequence[bool]) -> List[int]:
+    """Unmasking order of the FULL branch [LOWN method step (3)]: positions
+    whose TEXT-ONLY and FULL top-1 differ first, then the others; each group
+    by descending FULL confidence, lower index first on ties."""
+    idx = [i for i in range(len(full_top1)) if participants[i]]
+    idx.sort(key=lambda i: (int(text_top1[i]) == int(full_top1[i]), -float(full_conf[i]), i))
+    return idx
+
+
 def prefix_accept(verify_ids: Sequence[int], draft_ids: Sequence[int]) -> int:
     """Longest prefix on which the causal pass's argmax equals the draft
     [FDV §2.3.1 longest-prefix acceptance]."""
@@ -341,7 +366,7 @@ class OracleModel:
         return bf16_round(x) if self.bf16 else x
 
     # -- one decoder layer ---------------------------------------------------
-    def layer(self, l: int, x: np.ndarray, L: int, n_clean: int, write_kv: bool = True) -> np.ndarray:
+    def layer(self, l: int, x: np.ndarray, L: int, n_clean: int, write_kv: bool = True, hide: int = 0) -> np.ndarray:
         d = self.d
         n = x.shape[0]
         D, Hq, Hkv = d.head_dim, d.n_q_heads, d.n_kv_heads
@@ -356,7 +381,7 @@ class OracleModel:
         if write_kv:
             self.K[l][:, L:L + n] = k.transpose(1, 0, 2)
             self.V[l][:, L:L + n] = v.transpose(1, 0, 2)
-        a = block_attention(q, self.K[l], self.V[l], L, n_clean, 1.0 / math.sqrt(D))
+        a = block_attention(q, self.K[l], self.V[l], L, n_clean, 1.0 / math.sqrt(D), hide)
         a = self.rnd(a).reshape(n, Hq * D)
         x = self.rnd(x + a @ self.w(f"{l}.wo").T)
         h2 = x * rms_factor(x, d.eps)
@@ -370,12 +395,14 @@ class OracleModel:
         E = self.w("embed")
         return np.asarray(E[np.asarray(ids, dtype=np.int64)], dtype=np.float64)
 
-    def forward(self, x: np.ndarray, L: int, n_clean: int) -> np.ndarray:
+    def forward(self, x: np.ndarray, L: int, n_clean: int, hide: int = 0) -> np.ndarray:
         """Run all layers over rows at slots L..L+n-1; returns the final
         residual stream (before the final norm).  K/V of these rows are
-        written to the cache; the cache length is NOT advanced here."""
+        written to the cache; the cache length is NOT advanced here.  ``hide``:
+        cache slots 0..hide-1 are invisible (TEXT-ONLY pass, see
+        block_attention)."""
         for l in range(self.d.n_layers):
-            x = self.layer(l, x, L, n_clean)
+            x = self.layer(l, x, L, n_clean, hide=hide)
         return x
 
     def logits_conf(self, x: np.ndarray) -> Conf:
@@ -534,6 +561,87 @@ def decode_ar(model: OracleModel, seed_token: int, max_new: int) -> DecodeTrace:
         tr.nfe += 1
         tr.tokens.append(seed)
         seed = int(c.top1[0])
+    return tr
+
+
+@dataclasses.dataclass
+class LownTrace:
+    tokens: List[int]
+    n_full: int = 0          # FULL noisy forwards (vision visible)
+    n_text: int = 0          # TEXT-ONLY noisy forwards (vision hidden)
+    n_causal: int = 0        # causal append passes
+    accepted: List[int] = dataclasses.field(default_factory=list)   # positions unmasked per step
+    text_branch: List[bool] = dataclasses.field(default_factory=list)
+
+
+def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int, max_new: int,
+                shift: int = 1) -> LownTrace:
+    """Certificate-guided visual routing [LOWN method steps (1)-(3)] inside
+    block decoding.  Per block (first token = the AR seed, the rest [MASK]):
+    a FULL noisy forward sets the anchors (top-1 id and confidence of every
+    masked position, position j scored by row j - shift) and unmasks the k
+    most confident positions.  Each later step runs a TEXT-ONLY noisy forward
+    (cache slots 0..n_vis-1, the vision rows, hidden; positions unchanged) and
+    scans the masked positions in descending anchor confidence while the
+    TEXT-ONLY top-1 equals the anchor: if that certified prefix holds at least
+    min(k, masked) positions, all of it is unmasked with the anchor ids;
+    otherwise a FULL forward refreshes the anchors and min(k, masked)
+    positions are unmasked with the FULL ids, divergent positions (TEXT-ONLY
+    top-1 != FULL top-1) first.  A causal pass then appends the block."""
+    d = model.d
+    tr = LownTrace(tokens=[])
+    seed = seed_token
+    prev_conf = model.last_conf
+
+    def scores(c, pc):
+        p1, top = np.zeros(B), np.zeros(B, dtype=np.int64)
+        for j in range(B):
+            r = j - shift
+            cc, rr = (pc, 0) if r < 0 else (c, r)
+            p1[j], top[j] = cc.p1[rr], cc.top1[rr]
+        return p1, top
+
+    while len(tr.tokens) < max_new:
+        L = model.L
+        toks = [d.mask_id] * B
+        masked = [True] * B
+        toks[0], masked[0] = seed, False
+        anchor_id, anchor_conf = None, None
+        text_top = None
+        while any(masked):
+            kk = min(k, sum(masked))
+            if anchor_id is not None:
+                x = model.forward(model.embed(toks), L, n_clean=0, hide=n_vis)
+                _, text_top = scores(model.logits_conf(x), prev_conf)
+                tr.n_text += 1
+                order = certificate_order(anchor_conf, masked)
+                n = certificate_scan(anchor_id, anchor_conf, text_top, masked)
+                if n >= kk:
+                    for j in order[:n]:
+                        toks[j], masked[j] = int(anchor_id[j]), False
+                    tr.accepted.append(n)
+                    tr.text_branch.append(True)
+                    continue
+            x = model.forward(model.embed(toks), L, n_clean=0)
+            full_p1, full_top = scores(model.logits_conf(x), prev_conf)
+            tr.n_full += 1
+            anchor_id, anchor_conf = full_top.copy(), full_p1.copy()
+            if text_top is None:
+                order = certificate_order(full_p1, masked)
+            else:
+                order = divergence_first_order(full_top, full_p1, text_top, masked)
+            for j in order[:kk]:
+                toks[j], masked[j] = int(full_top[j]), False
+            tr.accepted.append(kk)
+            tr.text_branch.append(False)
+        x = model.forward(model.embed(toks), L, n_clean=B)
+        model.L = L + B
+        c = model.logits_conf(x)
+        tr.n_causal += 1
+        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:])
+        seed = int(c.top1[B - 1])
+        take = min(B, max_new - len(tr.tokens))
+        tr.tokens.extend(toks[:take])
     return tr
 
 

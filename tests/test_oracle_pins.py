@@ -4,6 +4,7 @@ bf16 cast, scipy's softmax/expit, numpy's sort), brute force on tiny inputs,
 and invariants of the decoding method.  Each pin is chosen so that a plausible
 slip (dropped term, wrong sign or index, transposed operand, > for >=) fails.
 """
+import inspect
 import math
 import os
 
@@ -512,6 +513,154 @@ def test_fp8_planted_mistakes_are_caught(monkeypatch):
                     failed += 1
             assert failed > 0, name
     assert OM.e4m3_round is real_round and OM.fp8_linear is real_linear
+
+
+# ----------------------------------------------------------------------------
+# Certificate-guided visual routing (LOWN) inside block decoding
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("L,n,n_vis", [(12, 4, 5), (9, 5, 9), (8, 4, 1)])
+def test_text_only_attention_equals_dense_without_vision_keys(L, n, n_vis):
+    """TEXT-ONLY pass: the dense role mask with the vision keys (the first
+    n_vis cache slots) removed, brute force, positions unchanged."""
+    rng = np.random.default_rng(L * 13 + n_vis)
+    q, K, V = _roles_case(rng, L, n, 0)
+    scale = 1 / math.sqrt(q.shape[-1])
+    got = O.block_attention(q, K, V, L, 0, scale, hide=n_vis)
+    k_noisy = [False] * L + [True] * n
+    k_block = [j // 4 for j in range(L)] + [10 ** 6] * n
+    k_pos = list(range(L + n))
+    m = O.mask_from_roles(k_noisy[L:], k_block[L:], k_pos[L:], k_noisy, k_block, k_pos)
+    m[:, :n_vis] = 0
+    want = O.dense_masked_attention(q, K.transpose(1, 0, 2), V.transpose(1, 0, 2), m, scale)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(got, O.block_attention(q, K, V, L, 0, scale))
+
+
+def test_routing_orders_hand_cases():
+    conf = [0.3, 0.9, 0.5, 0.9, 0.7]
+    part = [False, True, True, True, True]
+    assert O.certificate_order(conf, part) == [1, 3, 4, 2]                 # ties: lower position first
+    full_top, text_top = [0, 5, 6, 7, 8], [0, 5, 9, 7, 1]
+    assert O.divergence_first_order(full_top, conf, text_top, part) == [4, 2, 1, 3]
+
+
+class _ScriptedModel:
+    """Stands in for the decoder: hands out scripted confidences per kind of
+    pass (FULL / TEXT-ONLY noisy, causal append) and records the passes."""
+
+    def __init__(self, B, full, text):
+        self.d = O.Dims(n_layers=1, hidden=4, n_q_heads=1, n_kv_heads=1, head_dim=2, inter=4, vocab=100)
+        self.L, self.B = 40, B
+        self.last_conf = O.Conf(p1=np.array([1.0]), top1=np.array([7]), p2=np.array([0.0]))
+        self.full, self.text, self.calls = list(full), list(text), []
+
+    def embed(self, toks):
+        return np.asarray(toks, dtype=np.float64)[:, None]
+
+    def forward(self, x, L, n_clean, hide=0):
+        kind = "causal" if n_clean else ("text" if hide else "full")
+        self.calls.append((kind, L, hide, [int(t) for t in x[:, 0]]))
+        return kind
+
+    def logits_conf(self, kind):
+        if kind == "causal":
+            return O.Conf(p1=np.ones(self.B), top1=np.arange(self.B) + 60, p2=np.zeros(self.B))
+        script = self.full if kind == "full" else self.text
+        assert script, f"one {kind} pass more than scripted"
+        p1, top = script.pop(0)
+        # row r scores position r + 1
+        return O.Conf(p1=np.array(p1[1:] + [0.0]), top1=np.array(top[1:] + [0]), p2=np.zeros(self.B))
+
+
+def test_lown_routing_on_a_scripted_model():
+    B, mk = 5, 99                                   # mask id of the stub's vocabulary
+    full1 = ([0, 0.9, 0.5, 0.8, 0.6], [0, 11, 12, 13, 14])
+    # 1) TEXT-ONLY disagrees at the first scanned position: FULL refresh, divergent first
+    m = _ScriptedModel(B, [full1, ([0, 0, 0.7, 0, 0.95], [0, 0, 22, 0, 44])], [([0] * 5, [0, 0, 12, 0, 98])])
+    tr = O.decode_lown(m, 7, B, 2, n_vis=32, max_new=5)
+    assert tr.tokens == [7, 11, 22, 13, 44]
+    assert (tr.n_full, tr.n_text, tr.n_causal) == (2, 1, 1) and tr.accepted == [2, 2]
+    assert tr.text_branch == [False, False]
+    assert [c[0] for c in m.calls] == ["full", "text", "full", "causal"]
+    assert m.calls[1][2] == 32 and m.calls[1][3] == [7, 11, mk, 13, mk]     # vision hidden, state after step 1
+    # 2) TEXT-ONLY agrees along the scan: the prefix is accepted with the anchor ids
+    m = _ScriptedModel(B, [full1], [([0] * 5, [0, 0, 12, 0, 14])])
+    tr = O.decode_lown(m, 7, B, 2, n_vis=32, max_new=5)
+    assert tr.tokens == [7, 11, 12, 13, 14] and (tr.n_full, tr.n_text) == (1, 1)
+    assert tr.text_branch == [False, True]
+    # 3) a certified prefix longer than k is accepted whole
+    m = _ScriptedModel(6, [([0, 0.9, 0.5, 0.8, 0.6, 0.4], [0, 11, 12, 13, 14, 15])],
+                       [([0] * 6, [0, 0, 12, 0, 14, 15])])
+    tr = O.decode_lown(m, 7, 6, 2, n_vis=32, max_new=6)
+    assert tr.accepted == [2, 3] and tr.tokens == [7, 11, 12, 13, 14, 15]
+    # 4) the FULL branch unmasks the divergent positions (2, 4) before the more
+    # confident agreeing one (5), which the next TEXT-ONLY step certifies
+    # against the refreshed anchor
+    m = _ScriptedModel(6, [([0, 0.9, 0.5, 0.8, 0.6, 0.4], [0, 11, 12, 13, 14, 15]),
+                           ([0, 0, 0.3, 0, 0.2, 0.35], [0, 0, 32, 0, 34, 35])],
+                       [([0] * 6, [0, 0, 12, 0, 97, 35]), ([0] * 6, [0, 0, 0, 0, 0, 35])])
+    tr = O.decode_lown(m, 7, 6, 2, n_vis=32, max_new=6)
+    assert tr.text_branch == [False, False, True] and tr.accepted == [2, 2, 1]
+    assert tr.tokens == [7, 11, 32, 13, 34, 35]
+    # 5) the certificate stops at the first disagreement (position 4, scanned
+    # first) although positions 2 and 5 further down agree, which would reach k
+    m = _ScriptedModel(6, [([0, 0.9, 0.5, 0.8, 0.6, 0.4], [0, 11, 12, 13, 14, 15]),
+                           ([0, 0, 0.3, 0, 0.2, 0.35], [0, 0, 32, 0, 34, 35])],
+                       [([0] * 6, [0, 0, 12, 0, 97, 15]), ([0] * 6, [0, 0, 0, 0, 34, 0])])
+    tr = O.decode_lown(m, 7, 6, 2, n_vis=32, max_new=6)
+    assert tr.text_branch == [False, False, True] and tr.accepted == [2, 2, 1]
+    assert tr.tokens == [7, 11, 32, 13, 34, 35]
+
+
+def test_lown_planted_mistakes_are_caught(monkeypatch):
+    import oracle.dvlm_oracle as OM
+    real_div = OM.divergence_first_order
+
+    def agreeing_first(full_top, full_conf, text_top, part):
+        idx = real_div(full_top, full_conf, text_top, part)
+        return [i for i in idx if text_top[i] == full_top[i]] + [i for i in idx if text_top[i] != full_top[i]]
+
+    def count_all_agreeing(anchor_id, anchor_conf, top1, part=None):
+        return sum(1 for i in range(len(anchor_id)) if (part is None or part[i]) and top1[i] == anchor_id[i])
+
+    for name, mutant in [("divergence_first_order", agreeing_first), ("certificate_scan", count_all_agreeing)]:
+        with monkeypatch.context() as mp:
+            mp.setattr(OM, name, mutant)
+            with pytest.raises(AssertionError):
+                test_lown_routing_on_a_scripted_model()
+
+    # the FULL pass hides the vision rows as well (the routing then never sees them)
+    src = inspect.getsource(OM.decode_lown)
+    full_call = "model.forward(model.embed(toks), L, n_clean=0)\n"
+    assert src.count(full_call) == 1
+    ns = dict(vars(OM))
+    exec(src.replace(full_call, "model.forward(model.embed(toks), L, n_clean=0, hide=n_vis)\n"), ns)
+    with monkeypatch.context() as mp:
+        mp.setattr(O, "decode_lown", ns["decode_lown"])
+        for check in (test_lown_routing_on_a_scripted_model, test_lown_on_the_tiny_model):
+            with pytest.raises(AssertionError):
+                check()
+
+
+def test_lown_on_the_tiny_model():
+    """Invariants on a real (tiny) decoder: every step unmasks at least
+    min(k, masked) positions; with k covering the block, one FULL step per
+    block reproduces threshold decoding with tau 0 (everything commits at
+    once)."""
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s0 = _fresh(d, w, False, vis, ids)
+    tr = O.decode_lown(m, s0, B, B - 1, n_vis=len(vis), max_new=3 * B)
+    m2, s2 = _fresh(d, w, False, vis, ids)
+    th = O.decode_threshold(m2, s2, B, 0.0, 3 * B)
+    assert tr.tokens == th.tokens and tr.n_full == 3 and tr.n_text == 0
+    for k in (1, 2):
+        m, s0 = _fresh(d, w, False, vis, ids)
+        tr = O.decode_lown(m, s0, B, k, n_vis=len(vis), max_new=3 * B)
+        assert len(tr.tokens) == 3 * B and tr.n_causal == 3 and tr.n_full >= 3
+        assert all(a >= 1 for a in tr.accepted) and sum(tr.accepted) == 3 * (B - 1)
+        steps_per_block = len(tr.accepted) / 3
+        assert steps_per_block <= math.ceil((B - 1) / k)
 
 
 def test_pins_accept_the_oracle():
