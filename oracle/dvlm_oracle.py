@@ -38,6 +38,10 @@ its reason in the repository's design notes):
             FULL pass unmasking min(k, masked) by confidence; the certified
             prefix is unmasked with the anchor ids; the FULL branch puts
             divergent positions first, each group by FULL confidence.
+  quadratic (next step) one fused forward = the draft's causal verify rows
+            plus one all-[MASK] candidate block per possible accepted length
+            k, at positions L+k.., seeing the context and verify rows 0..k-1;
+            the next draft = [verifier's token] + the chosen candidate's top-1.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against brute force, closed forms, library routines or the pages' printed
@@ -419,6 +423,7 @@ class DecodeTrace:
     nfe: int = 0
     commits_per_iter: List[int] = dataclasses.field(default_factory=list)
     accept_lens: List[int] = dataclasses.field(default_factory=list)
+    drafts: List[List[int]] = dataclasses.field(default_factory=list)   # speculative drafts, per round
     # smallest decision margin met along the trajectory (for parity exclusion)
     min_margin: float = math.inf
     margins: List[float] = dataclasses.field(default_factory=list)
@@ -561,6 +566,115 @@ def decode_ar(model: OracleModel, seed_token: int, max_new: int) -> DecodeTrace:
         tr.nfe += 1
         tr.tokens.append(seed)
         seed = int(c.top1[0])
+    return tr
+
+
+# ----------------------------------------------------------------------------
+# Quadratic self-speculative decoding  [FDV §2.3.1, the variant that fuses
+# draft and verify into one forward at O(B^2) cost]
+# ----------------------------------------------------------------------------
+def quadratic_attention(q_ver: np.ndarray, q_cand: np.ndarray, K: np.ndarray, V: np.ndarray, L: int,
+                        k_cand: np.ndarray, v_cand: np.ndarray, scale: float) -> np.ndarray:
+    """Attention of one fused forward.
+
+    q_ver [B, Hq, D]: the causal verify rows of the draft at slots L..L+B-1,
+    whose K/V are already in the cache K, V [Hkv, >= L+B, D]; row t sees
+    slots 0..L+t.  q_cand [B, B, Hq, D]: candidate block i (0-based; it
+    stands for "the first i+1 draft tokens accepted") holds B noisy rows at
+    positions L+i+1 .. L+i+B; its K/V k_cand, v_cand [B, B, Hkv, D] stay out
+    of the cache.  A candidate row sees the cache slots 0..L+i (the context
+    and the accepted verify rows, N2C) and the B rows of its own candidate
+    block (N2N), nothing of the other candidates.  Returns [B + B*B, Hq, D]:
+    verify rows, then the candidate blocks in order."""
+    B, Hq, D = q_ver.shape
+    Hkv = K.shape[0]
+    G = Hq // Hkv
+    out = [block_attention(q_ver, K, V, L, B, scale)]
+    for i in range(B):
+        o = np.zeros((B, Hq, D))
+        for r in range(B):
+            for h in range(Hq):
+                g = h // G
+                keys = np.concatenate([K[g, :L + i + 1], k_cand[i, :, g]], axis=0)
+                vals = np.concatenate([V[g, :L + i + 1], v_cand[i, :, g]], axis=0)
+                sc = scale * (keys @ q_cand[i, r, h])
+                p = np.exp(sc - sc.max())
+                p /= p.sum()
+                o[r, h] = p @ vals
+        out.append(o)
+    return np.concatenate(out, axis=0)
+
+
+def forward_quadratic(model: OracleModel, draft: Sequence[int], L: int) -> np.ndarray:
+    """One fused draft+verify forward over B + B*B rows: the draft's verify
+    rows (clean, causal, K/V written to slots L..L+B-1) and B candidate blocks
+    of B [MASK] rows each (candidate i at positions L+i+1 .. L+i+B, K/V kept
+    out of the cache).  Same layer arithmetic and bf16 storage points as
+    OracleModel.layer.  Returns the final residual rows [B + B*B, H]."""
+    d = model.d
+    B = len(draft)
+    D, Hq, Hkv = d.head_dim, d.n_q_heads, d.n_kv_heads
+    x = np.concatenate([model.embed(draft), model.embed([d.mask_id] * (B * B))], axis=0)
+    pos = np.concatenate([np.arange(L, L + B)] + [np.arange(L + i + 1, L + i + 1 + B) for i in range(B)])
+    n = x.shape[0]
+    for l in range(d.n_layers):
+        h = x * rms_factor(x, d.eps)
+        q = (h @ model.w(f"{l}.wq").T).reshape(n, Hq, D)
+        k = (h @ model.w(f"{l}.wk").T).reshape(n, Hkv, D)
+        v = (h @ model.w(f"{l}.wv").T).reshape(n, Hkv, D)
+        q = model.rnd(rope(q, pos, d.rope_base))
+        k = model.rnd(rope(k, pos, d.rope_base))
+        v = model.rnd(v)
+        model.K[l][:, L:L + B] = k[:B].transpose(1, 0, 2)
+        model.V[l][:, L:L + B] = v[:B].transpose(1, 0, 2)
+        a = quadratic_attention(q[:B], q[B:].reshape(B, B, Hq, D), model.K[l], model.V[l], L,
+                                k[B:].reshape(B, B, Hkv, D), v[B:].reshape(B, B, Hkv, D),
+                                1.0 / math.sqrt(D))
+        a = model.rnd(a).reshape(n, Hq * D)
+        x = model.rnd(x + a @ model.w(f"{l}.wo").T)
+        h2 = x * rms_factor(x, d.eps)
+        g = h2 @ model.w(f"{l}.wg").T
+        u = h2 @ model.w(f"{l}.wu").T
+        act = model.rnd(silu(g) * u)
+        x = model.rnd(x + act @ model.w(f"{l}.wd").T)
+    return x
+
+
+def decode_spec_quadratic(model: OracleModel, seed_token: int, B: int, max_new: int) -> DecodeTrace:
+    """Quadratic self-speculative decoding [FDV §2.3.1].  The first draft
+    comes from one diffusion pass as in the linear variant.  Every later
+    forward is fused: it verifies the current draft causally (v_j = top-1 of
+    verify row j-1, v_0 = the seed) and, for every possible accepted length
+    k = 1..B, drafts the next block in candidate block k-1, whose rows sit at
+    positions L+k .. L+k+B-1.  After the longest agreeing prefix k is kept
+    (L advances by k), the next draft is [v_k] followed by the top-1 of
+    candidate block k-1's rows 0..B-2 (shift=1: a row scores the position
+    after it).  One forward per round instead of two; the output equals
+    greedy AR decoding, since only verified tokens are kept."""
+    d = model.d
+    tr = DecodeTrace(tokens=[])
+    L = model.L
+    x = model.forward(model.embed([seed_token] + [d.mask_id] * (B - 1)), L, n_clean=0)
+    c = model.logits_conf(x)
+    _note_argmax_margin(tr, c, range(B - 1))
+    draft = [seed_token] + [int(c.top1[j - 1]) for j in range(1, B)]
+    tr.nfe += 1
+    while len(tr.tokens) < max_new:
+        L = model.L
+        tr.drafts.append(list(draft))
+        x = forward_quadratic(model, draft, L)
+        c = model.logits_conf(x)
+        tr.nfe += 1
+        _note_argmax_margin(tr, c, range(B))
+        verify = [draft[0]] + [int(c.top1[j - 1]) for j in range(1, B)]
+        k = prefix_accept(verify, draft)
+        tr.accept_lens.append(k)
+        tr.tokens.extend(draft[:k])
+        model.L = L + k
+        rows = B + (k - 1) * B
+        _note_argmax_margin(tr, c, range(rows, rows + B - 1))
+        draft = [int(c.top1[k - 1])] + [int(c.top1[rows + j - 1]) for j in range(1, B)]
+    tr.tokens = tr.tokens[:max_new]
     return tr
 
 

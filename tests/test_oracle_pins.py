@@ -4,6 +4,7 @@ bf16 cast, scipy's softmax/expit, numpy's sort), brute force on tiny inputs,
 and invariants of the decoding method.  Each pin is chosen so that a plausible
 slip (dropped term, wrong sign or index, transposed operand, > for >=) fails.
 """
+import copy
 import inspect
 import math
 import os
@@ -661,6 +662,178 @@ def test_lown_on_the_tiny_model():
         assert all(a >= 1 for a in tr.accepted) and sum(tr.accepted) == 3 * (B - 1)
         steps_per_block = len(tr.accepted) / 3
         assert steps_per_block <= math.ceil((B - 1) / k)
+
+
+# ----------------------------------------------------------------------------
+# Quadratic self-speculative decoding [FDV §2.3.1]
+# ----------------------------------------------------------------------------
+def _quad_mask(L, B):
+    """The fused forward's visibility from token roles alone: cache slots are
+    clean tokens of an earlier block; verify row t is the clean token of a
+    block of its own (t) at position L+t; candidate block i holds the noisy
+    tokens of block i+1 at positions L+i+1 ... (so it sees verify rows 0..i)."""
+    k_noisy = [False] * (L + B) + [True] * (B * B)
+    k_block = [-1] * L + list(range(B)) + [i + 1 for i in range(B) for _ in range(B)]
+    k_pos = list(range(L + B)) + [L + i + 1 + r for i in range(B) for r in range(B)]
+    return O.mask_from_roles(k_noisy[L:], k_block[L:], k_pos[L:], k_noisy, k_block, k_pos)
+
+
+@pytest.mark.parametrize("L,B", [(5, 1), (7, 3), (4, 4)])
+def test_quadratic_attention_equals_dense_masked_bruteforce(L, B):
+    rng = np.random.default_rng(10 * L + B)
+    Hq, Hkv, D = 4, 2, 8
+    K, V = rng.standard_normal((2, Hkv, L + B, D))
+    q_ver = rng.standard_normal((B, Hq, D))
+    q_cand = rng.standard_normal((B, B, Hq, D))
+    k_cand, v_cand = rng.standard_normal((2, B, B, Hkv, D))
+    got = O.quadratic_attention(q_ver, q_cand, K, V, L, k_cand, v_cand, 0.3)
+    mask = _quad_mask(L, B)
+    # a candidate row of block i sees the context, verify rows 0..i and its own B rows
+    assert [int(mask[B + i * B].sum()) for i in range(B)] == [L + i + 1 + B for i in range(B)]
+    want = O.dense_masked_attention(np.concatenate([q_ver, q_cand.reshape(B * B, Hq, D)]),
+                                    np.concatenate([K.transpose(1, 0, 2), k_cand.reshape(B * B, Hkv, D)]),
+                                    np.concatenate([V.transpose(1, 0, 2), v_cand.reshape(B * B, Hkv, D)]),
+                                    mask, 0.3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_fused_forward_equals_the_sequential_passes():
+    """Verify rows == one causal pass over the draft (same cache writes);
+    candidate block k-1 == accepting k draft tokens by a causal pass and then
+    running a [MASK] block at L+k as an ordinary noisy pass."""
+    gd, d, w, vis, ids = _tiny()
+    m, s0 = _fresh(d, w, False, vis, ids)
+    B, L = 4, m.L
+    rng = np.random.default_rng(3)
+    draft = [s0] + [int(t) for t in rng.integers(0, d.vocab - 1, B - 1)]
+    mq = copy.deepcopy(m)
+    xq = O.forward_quadratic(mq, draft, L)
+    assert xq.shape == (B + B * B, d.hidden)
+    mv = copy.deepcopy(m)
+    xv = mv.forward(mv.embed(draft), L, n_clean=B)
+    np.testing.assert_allclose(xq[:B], xv, rtol=0, atol=1e-10)
+    for l in range(d.n_layers):
+        np.testing.assert_allclose(mq.K[l], mv.K[l], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(mq.V[l], mv.V[l], rtol=0, atol=1e-10)
+    for k in range(1, B + 1):
+        ms = copy.deepcopy(m)
+        ms.forward(ms.embed(draft[:k]), L, n_clean=k)
+        xs = ms.forward(ms.embed([d.mask_id] * B), L + k, n_clean=0)
+        np.testing.assert_allclose(xq[B + (k - 1) * B:B + k * B], xs, rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_spec_quadratic_equals_greedy_ar(bf16):
+    gd, d, w, vis, ids = _tiny(bf16)
+    m1, s1 = _fresh(d, w, bf16, vis, ids)
+    ar = O.decode_ar(m1, s1, 24)
+    for B in (1, 4):
+        m2, s2 = _fresh(d, w, bf16, vis, ids)
+        qd = O.decode_spec_quadratic(m2, s2, B, 24)
+        assert qd.tokens == ar.tokens
+        assert all(1 <= k <= B for k in qd.accept_lens)
+        assert qd.nfe == 1 + len(qd.accept_lens)          # one fused forward per round
+        assert m2.L == m1.L + sum(qd.accept_lens) - 24
+        if B == 1:
+            assert qd.accept_lens == [1] * 24
+
+
+def test_spec_quadratic_drafts_replayed_by_sequential_passes():
+    """Every round's draft is [the verifier's token after the accepted
+    prefix] + the argmax of an ordinary noisy [MASK] pass placed right after
+    that prefix, shifted by one row; replayed with causal and noisy passes."""
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s0 = _fresh(d, w, False, vis, ids)
+    qd = O.decode_spec_quadratic(copy.deepcopy(m), s0, B, 16)
+    x = m.forward(m.embed([s0] + [d.mask_id] * (B - 1)), m.L, n_clean=0)
+    c = m.logits_conf(x)
+    assert qd.drafts[0] == [s0] + [int(c.top1[j - 1]) for j in range(1, B)]
+    for r, draft in enumerate(qd.drafts[:-1]):
+        L = m.L
+        g = m.logits_conf(m.forward(m.embed(draft), L, n_clean=B))
+        verify = [draft[0]] + [int(g.top1[j - 1]) for j in range(1, B)]
+        k = O.prefix_accept(verify, draft)
+        assert k == qd.accept_lens[r]
+        m.L = L + k
+        probe = copy.deepcopy(m)
+        n = probe.logits_conf(probe.forward(probe.embed([d.mask_id] * B), m.L, n_clean=0))
+        assert qd.drafts[r + 1] == [int(g.top1[k - 1])] + [int(n.top1[j - 1]) for j in range(1, B)]
+
+
+class _IdModel:
+    """Stub decoder whose rows carry token ids: the LM head's top-1 of a row
+    is its first entry.  The first draft's noisy pass predicts 500 + row."""
+
+    def __init__(self):
+        self.d = O.Dims(n_layers=1, hidden=1, n_q_heads=1, n_kv_heads=1, head_dim=2, inter=1, vocab=100000)
+        self.L = 40
+
+    def embed(self, toks):
+        return np.asarray(toks, dtype=np.float64)[:, None]
+
+    def forward(self, x, L, n_clean, hide=0):
+        assert n_clean == 0 and L == self.L
+        return 500.0 + np.arange(x.shape[0])[:, None]
+
+    def logits_conf(self, x):
+        n = x.shape[0]
+        return O.Conf(p1=np.ones(n), top1=x[:, 0].astype(np.int64), p2=np.zeros(n))
+
+
+def test_spec_quadratic_driver_on_a_scripted_model(monkeypatch):
+    """Fused forwards scripted: verify row j predicts script[r][j]; row r of
+    candidate block i predicts 10000*round + 1000 + 100*i + r.  Accepted
+    lengths, seeds, chosen candidate blocks and L worked out by hand."""
+    B, script, calls = 4, [[500, 501, 9, 9], [1200, 5, 5, 5], [11100, 11101, 11102, 77]], []
+
+    def fused(model, draft, L):
+        r = len(calls)
+        assert r < len(script), "one fused forward more than scripted"
+        calls.append((list(draft), L))
+        cand = [10000 * r + 1000 + 100 * i + q for i in range(B) for q in range(B)]
+        return np.asarray(script[r] + cand, dtype=np.float64)[:, None]
+
+    monkeypatch.setitem(O.decode_spec_quadratic.__globals__, "forward_quadratic", fused)
+    m = _IdModel()
+    tr = O.decode_spec_quadratic(m, 7, B, 9)
+    assert tr.drafts == [[7, 500, 501, 502], [9, 1200, 1201, 1202], [5, 11100, 11101, 11102]]
+    assert tr.accept_lens == [3, 2, 4] and tr.nfe == 4
+    assert tr.tokens == [7, 500, 501, 9, 1200, 5, 11100, 11101, 11102]
+    assert [c[1] for c in calls] == [40, 43, 45] and m.L == 49
+
+
+def test_quadratic_planted_mistakes_are_caught(monkeypatch):
+    import oracle.dvlm_oracle as OM
+
+    def mutate(fn_name, old, new, checks, count=1):
+        src = inspect.getsource(getattr(OM, fn_name))
+        assert src.count(old) == count, old
+        ns = dict(vars(OM))
+        exec(src.replace(old, new), ns)
+        with monkeypatch.context() as mp:
+            mp.setattr(OM, fn_name, ns[fn_name])
+            mp.setattr(O, fn_name, ns[fn_name])
+            for check in checks:
+                with pytest.raises(AssertionError):
+                    check()
+
+    attn = lambda: test_quadratic_attention_equals_dense_masked_bruteforce(7, 3)
+    # candidates see every verify row, not only the accepted prefix
+    mutate("quadratic_attention", "[g, :L + i + 1]", "[g, :L + B]", [attn], count=2)
+    # candidates see one verify row too few
+    mutate("quadratic_attention", "[g, :L + i + 1]", "[g, :L + i]", [attn], count=2)
+    # candidate blocks placed one position early (RoPE of the wrong slots)
+    mutate("forward_quadratic", "np.arange(L + i + 1, L + i + 1 + B)", "np.arange(L + i, L + i + B)",
+           [test_fused_forward_equals_the_sequential_passes])
+    scripted = lambda: test_spec_quadratic_driver_on_a_scripted_model(monkeypatch)
+    # the next draft taken from the candidate block of one more accepted token
+    mutate("decode_spec_quadratic", "rows = B + (k - 1) * B", "rows = B + min(k, B - 1) * B", [scripted])
+    # the next draft read without the one-row shift
+    mutate("decode_spec_quadratic", "c.top1[rows + j - 1]", "c.top1[rows + j]", [scripted])
+    # the next seed taken from the verify row of the last accepted token itself
+    mutate("decode_spec_quadratic", "draft = [int(c.top1[k - 1])]", "draft = [int(c.top1[max(k - 2, 0)])]",
+           [scripted, lambda: test_spec_quadratic_equals_greedy_ar(False)])
 
 
 def test_pins_accept_the_oracle():
