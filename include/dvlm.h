@@ -61,7 +61,7 @@ typedef enum dvlm_status {
   DVLM_OK = 0,
   DVLM_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad enum value       */
   DVLM_ERR_SHAPE = 2,         /* sizes inconsistent or out of the supported range */
-  DVLM_ERR_UNSUPPORTED = 3,   /* valid request this build does not implement      */
+  DVLM_ERR_UNSUPPORTED = 3,   /* valid request the library does not implement     */
   DVLM_ERR_CACHE_OVERFLOW = 4,/* the step would write past Lmax                   */
   DVLM_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out               */
   DVLM_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed                */
