@@ -28,6 +28,8 @@ its reason in the repository's design notes):
   commit    p1 >= threshold; if none passes, the masked position with the
             highest p1 (lowest position on ties) is committed.
   argmax    lowest vocabulary id among equal maxima.
+  top-k     (next step) the k most confident masked positions per iteration,
+            lower position first on ties.
   fp8       (next step, not on the bf16 path) W8A8 in E4M3, finite variant,
             round to nearest even, saturating at 448; one scale per weight
             output channel and per activation token (amax / 448);
@@ -275,6 +277,16 @@ def threshold_commit(p1: Sequence[float], masked: Sequence[bool], tau: float) ->
     return C
 
 
+def topk_commit(p1: Sequence[float], masked: Sequence[bool], k: int) -> List[int]:
+    """Commit the k masked rows of highest p1 (all of them when fewer remain),
+    lower index first on ties: the confidence-ordered unmasking of a fixed
+    number of positions per step [LOWN, background on confidence-guided
+    unmasking]."""
+    idx = [r for r in range(len(p1)) if masked[r]]
+    idx.sort(key=lambda r: (-float(p1[r]), r))
+    return sorted(idx[:max(k, 0)])
+
+
 def certificate_scan(anchor_id: Sequence[int], anchor_conf: Sequence[float],
                      top1: Sequence[int], participants: Optional[Sequence[bool]] = None) -> int:
     """Longest certified prefix [LOWN method step (2)]: visit positions in
@@ -454,7 +466,8 @@ def _note_argmax_margin(tr: DecodeTrace, c: Conf, rows) -> None:
 
 
 def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, max_new: int,
-                     shift: int = 1, ar_seed: int = 1, on_iter=None, on_block=None) -> DecodeTrace:
+                     shift: int = 1, ar_seed: int = 1, on_iter=None, on_block=None,
+                     commit_k: Optional[int] = None) -> DecodeTrace:
     """Threshold (MDM-style) block decoding [FDV §2.2.1, §2.2.2, §4.1].
 
     Per block: the first token is the AR seed (ar_seed=1); the remaining
@@ -464,6 +477,9 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
     the previous pass's last row) and commits per ``threshold_commit``.  When
     the block is complete a causal pass over it makes its K/V final, advances
     L by B and yields the next block's seed from its last row.
+
+    ``commit_k``: commit per ``topk_commit`` (the k most confident masked
+    positions each iteration) instead of the threshold rule; tau is unused.
 
     Optional observers (they do not change the trajectory): on_iter(L, toks,
     masked, p1, top1, p2) before each iteration's commit, with the scores per
@@ -491,13 +507,23 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
                 p1[j], top[j], p2[j] = cc.p1[rr], cc.top1[rr], cc.p2[rr]
             if on_iter is not None:
                 on_iter(L, list(toks), list(masked), p1.copy(), top.copy(), p2.copy())
-            C = threshold_commit(p1, masked, tau)
+            if commit_k is not None:
+                C = topk_commit(p1, masked, commit_k)
+                rest = [p1[j] for j in range(B) if masked[j] and j not in C]
+                margins = [p1[j] - p2[j] for j in C]
+                if rest:
+                    margins.append(min(p1[j] for j in C) - max(rest))
+                for mg in margins:
+                    tr.margins.append(float(mg))
+                    tr.min_margin = min(tr.min_margin, float(mg))
+            else:
+                C = threshold_commit(p1, masked, tau)
             for j in range(B):
-                if masked[j]:
+                if commit_k is None and masked[j]:
                     mg = min(abs(p1[j] - tau), p1[j] - p2[j])
                     tr.margins.append(mg)
                     tr.min_margin = min(tr.min_margin, mg)
-            if len(C) == 1 and not (p1[C[0]] >= tau):
+            if commit_k is None and len(C) == 1 and not (p1[C[0]] >= tau):
                 others = [p1[j] for j in range(B) if masked[j] and j != C[0]]
                 if others:
                     mg = float(p1[C[0]] - max(others))

@@ -664,6 +664,62 @@ def test_lown_on_the_tiny_model():
         assert steps_per_block <= math.ceil((B - 1) / k)
 
 
+def test_topk_commit_hand_cases():
+    p = [0.95, 0.5, 0.91, 0.2, 0.91]
+    assert O.topk_commit(p, [True] * 5, 2) == [0, 2]           # tie at 0.91: lower position
+    assert O.topk_commit(p, [True] * 5, 3) == [0, 2, 4]
+    assert O.topk_commit(p, [False, True, True, True, True], 1) == [2]
+    assert O.topk_commit(p, [False, True, False, True, False], 5) == [1, 3]
+    assert O.topk_commit(p, [False] * 5, 2) == []
+    assert O.topk_commit(p, [True] * 5, 0) == []
+    # k = 1 is the threshold rule's force-commit when nothing passes
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        q = rng.choice([0.1, 0.3, 0.5, 0.7], 6)
+        m = list(rng.random(6) < 0.7)
+        assert O.topk_commit(q, m, 1) == O.threshold_commit(q, m, 2.0)
+        assert O.topk_commit(q, m, 6) == O.threshold_commit(q, m, 0.0)
+
+
+def test_topk_planted_mistakes_are_caught(monkeypatch):
+    import oracle.dvlm_oracle as OM
+    real = OM.topk_commit
+
+    def later_on_ties(p1, masked, k):
+        idx = [r for r in range(len(p1)) if masked[r]]
+        idx.sort(key=lambda r: (-float(p1[r]), -r))
+        return sorted(idx[:k])
+
+    def counts_committed_rows(p1, masked, k):       # k taken over all rows, not the masked ones
+        idx = sorted(range(len(p1)), key=lambda r: (-float(p1[r]), r))[:k]
+        return sorted(r for r in idx if masked[r])
+
+    for mutant in (later_on_ties, counts_committed_rows, lambda p1, masked, k: real(p1, masked, k + 1)):
+        with monkeypatch.context() as mp:
+            mp.setattr(OM, "topk_commit", mutant)
+            mp.setattr(O, "topk_commit", mutant)
+            with pytest.raises(AssertionError):
+                test_topk_commit_hand_cases()
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_topk_decoding_limits(bf16):
+    """k = 1 equals threshold decoding with nothing passing (tau > 1); k
+    covering the block equals tau = 0; in between, ceil((B-1)/k) iterations
+    per block, k commits each but the last."""
+    gd, d, w, vis, ids = _tiny(bf16)
+    B = 5
+    runs = {}
+    for name, kw in [("k1", dict(tau=0.9, commit_k=1)), ("t2", dict(tau=2.0)),
+                     ("kB", dict(tau=0.9, commit_k=B)), ("t0", dict(tau=0.0)), ("k3", dict(tau=0.9, commit_k=3))]:
+        m, s0 = _fresh(d, w, bf16, vis, ids)
+        runs[name] = O.decode_threshold(m, s0, B, kw.pop("tau"), 3 * B, **kw)
+    assert runs["k1"].tokens == runs["t2"].tokens and runs["k1"].commits_per_iter == [1] * (3 * (B - 1))
+    assert runs["kB"].tokens == runs["t0"].tokens and runs["kB"].commits_per_iter == [B - 1] * 3
+    assert runs["k3"].commits_per_iter == [3, 1] * 3
+    assert runs["k3"].nfe == 3 * (math.ceil((B - 1) / 3) + 1)
+
+
 # ----------------------------------------------------------------------------
 # Quadratic self-speculative decoding [FDV §2.3.1]
 # ----------------------------------------------------------------------------
