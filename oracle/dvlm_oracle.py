@@ -30,6 +30,8 @@ its reason in the repository's design notes):
   argmax    lowest vocabulary id among equal maxima.
   top-k     (next step) the k most confident masked positions per iteration,
             lower position first on ties.
+  paged     (next step) slot s of a sequence lives in row s mod P of page
+            table[s div P]; a batch is the per-sequence definition per entry.
   fp8       (next step, not on the bf16 path) W8A8 in E4M3, finite variant,
             round to nearest even, saturating at 448; one scale per weight
             output channel and per activation token (amax / 448);
@@ -227,6 +229,28 @@ def block_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, L: int, n_clean
             p /= p.sum()
             out[t, h] = p @ V[g, hide:vis]
     return out
+
+
+def paged_gather(pages: np.ndarray, block_table: Sequence[int], n: int) -> np.ndarray:
+    """Logical cache slots 0..n-1 of one sequence from a paged store [FDV
+    §2.3.2, paged KV cache management].  pages: [n_pages, Hkv, P, D]; logical
+    slot s lives in row s mod P of page block_table[s div P].  Returns
+    [Hkv, n, D] in logical order."""
+    P = pages.shape[2]
+    out = np.zeros((pages.shape[1], n, pages.shape[3]))
+    for s in range(n):
+        out[:, s] = pages[block_table[s // P], :, s % P]
+    return out
+
+
+def paged_block_attention(q: np.ndarray, K_pages: np.ndarray, V_pages: np.ndarray, block_table: Sequence[int],
+                          L: int, n_clean: int, scale: float, hide: int = 0) -> np.ndarray:
+    """block_attention over a paged cache: the step's rows sit at logical
+    slots L..L+n-1 (their K/V already stored through the same table)."""
+    n = q.shape[0]
+    K = paged_gather(K_pages, block_table, L + n)
+    V = paged_gather(V_pages, block_table, L + n)
+    return block_attention(q, K, V, L, n_clean, scale, hide)
 
 
 # ----------------------------------------------------------------------------

@@ -720,6 +720,55 @@ def test_topk_decoding_limits(bf16):
     assert runs["k3"].nfe == 3 * (math.ceil((B - 1) / 3) + 1)
 
 
+def test_paged_gather_hand_case():
+    pages = np.zeros((4, 1, 2, 1))
+    for pg in range(4):
+        for r in range(2):
+            pages[pg, 0, r, 0] = 10 * pg + r
+    # table [3, 0, 2]: slots 0,1 -> page 3; 2,3 -> page 0; 4 -> page 2 row 0
+    got = O.paged_gather(pages, [3, 0, 2], 5)[0, :, 0]
+    assert list(got) == [30, 31, 0, 1, 20]
+
+
+def test_paged_planted_mistakes_are_caught(monkeypatch):
+    import oracle.dvlm_oracle as OM
+    src = inspect.getsource(OM.paged_gather)
+    old = "pages[block_table[s // P], :, s % P]"
+    assert src.count(old) == 1
+    for new in ("pages[block_table[s % P], :, s // P]",          # page and row swapped
+                "pages[s // P, :, s % P]",                         # table ignored
+                "pages[block_table[s // P], :, (s + 1) % P]"):     # row off by one
+        ns = dict(vars(OM))
+        exec(src.replace(old, new), ns)
+        with monkeypatch.context() as mp:
+            mp.setattr(O, "paged_gather", ns["paged_gather"])
+            with pytest.raises((AssertionError, IndexError)):
+                test_paged_gather_hand_case()
+
+
+@pytest.mark.parametrize("P,L,n,n_clean", [(1, 7, 3, 0), (3, 10, 4, 2), (16, 37, 5, 5), (16, 64, 16, 0)])
+def test_paged_attention_equals_contiguous_cache(P, L, n, n_clean):
+    """Scatter a contiguous cache into randomly permuted pages (ragged last
+    page), gather it back, and attend: both equal the contiguous results."""
+    rng = np.random.default_rng(100 * P + L)
+    Hq, Hkv, D = 4, 2, 8
+    K, V = rng.standard_normal((2, Hkv, L + n, D))
+    q = rng.standard_normal((n, Hq, D))
+    n_pages = -(-(L + n) // P)
+    table = [int(t) for t in rng.permutation(n_pages + 3)[:n_pages]]      # spare pages stay unused
+    Kp = rng.standard_normal((n_pages + 3, Hkv, P, D))                     # garbage outside the table
+    Vp = rng.standard_normal((n_pages + 3, Hkv, P, D))
+    for s in range(L + n):
+        Kp[table[s // P], :, s % P] = K[:, s]
+        Vp[table[s // P], :, s % P] = V[:, s]
+    np.testing.assert_array_equal(O.paged_gather(Kp, table, L + n), K)
+    want = O.block_attention(q, K, V, L, n_clean, 0.3)
+    np.testing.assert_array_equal(O.paged_block_attention(q, Kp, Vp, table, L, n_clean, 0.3), want)
+    hide = min(3, L)
+    np.testing.assert_array_equal(O.paged_block_attention(q, Kp, Vp, table, L, n_clean, 0.3, hide),
+                                  O.block_attention(q, K, V, L, n_clean, 0.3, hide))
+
+
 # ----------------------------------------------------------------------------
 # Quadratic self-speculative decoding [FDV §2.3.1]
 # ----------------------------------------------------------------------------
