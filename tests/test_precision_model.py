@@ -1,0 +1,69 @@
+"""How much of the 2e-2 attention bar the GPU's precision choices use.
+
+A numpy model of the arithmetic (not of the code) of the bf16 attention
+path: fp32 scores from bf16 q and k; keys split over 16 cooperating CTAs in
+64-key chunks taken round-robin; each CTA's probabilities exp2(s - m_cta)
+rounded to fp16 and multiplied by the fp16 copy of V with fp32 accumulation;
+each CTA's partial rows divided by its own sum and exchanged in fp16; merged
+with weights exp2(m_cta - M) * l_cta; the output stored in bf16.  Measured
+against the fp64 oracle on the block-attention configuration's inputs: the
+error is the bf16 store's rounding plus well under 1e-3, a small fraction of
+the bar."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dvlm_gen as gen
+import oracle as O
+
+TOL_BF16 = 2e-2
+CHUNK, SPLIT = 64, 16
+
+
+def _bf16(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def model_attention(q, k, v, L, scale):
+    """q [n, Hq, D], k/v [Hkv, >= L+n, D] (bf16 values as float32); noisy rows
+    see slots 0..L+n-1."""
+    n, Hq, D = q.shape
+    G = Hq // k.shape[0]
+    nk = L + n
+    s2 = scale * math.log2(math.e)
+    out = np.zeros((n, Hq, D), dtype=np.float32)
+    chunks = [np.arange(c, min(c + CHUNK, nk)) for c in range(0, nk, CHUNK)]
+    for h in range(Hq):
+        kk, vv = k[h // G, :nk], v[h // G, :nk]
+        s = (q[:, h].astype(np.float32) @ kk.T.astype(np.float32)) * np.float32(s2)     # [n, nk] fp32
+        parts = []
+        for c in range(SPLIT):
+            idx = np.concatenate([chunks[j] for j in range(c, len(chunks), SPLIT)] or [np.zeros(0, int)])
+            if len(idx) == 0:
+                continue
+            m = s[:, idx].max(axis=1, keepdims=True)
+            p = np.exp2(s[:, idx] - m).astype(np.float32)
+            l_ = p.sum(axis=1, keepdims=True, dtype=np.float32)
+            o = p.astype(np.float16).astype(np.float32) @ vv[idx].astype(np.float16).astype(np.float32)
+            parts.append((m, l_, (o / l_).astype(np.float16).astype(np.float32)))
+        M = np.max([m for m, _, _ in parts], axis=0)
+        w = [np.exp2(m - M) * l_ for m, l_, _ in parts]
+        num = sum(wi * oi for wi, (_, _, oi) in zip(w, parts))
+        out[:, h] = num / sum(w)
+    return _bf16(out)
+
+
+@pytest.mark.parametrize("B,L", [(16, 1344), (16, 4096), (32, 4096), (4, 256)])
+def test_attention_precision_uses_a_fraction_of_the_bar(B, L):
+    q, k, v = (t.float().numpy() for t, _ in gen.attn_case(1, B, L))
+    scale = 1.0 / math.sqrt(q.shape[-1])
+    got = model_attention(q[0], k[0], v[0], L, scale)
+    want = O.block_attention(q[0].astype(np.float64), k[0].astype(np.float64), v[0].astype(np.float64), L, 0,
+                             scale)
+    err = float(np.abs(got - want).max())
+    # the bf16 store alone may cost half an ulp, at most 2^-8 of |out|; the
+    # fp16 probabilities and partial rows add at most a few 1e-4 on top
+    assert err <= 2.0 ** -8 * float(np.abs(want).max()) + 2e-4, err
+    assert err < TOL_BF16 / 4, err
