@@ -419,6 +419,120 @@ def run_ours(args, rank, world, local, pg):
         print(json.dumps(line), flush=True)
 
 
+def _device_ms_per_call(fn, reps, dev):
+    """Device time per call of `fn` (launches on the current stream), from CUDA
+    events around a CUDA graph of `reps` calls; eager launches if the capture
+    is refused.  Returns (ms, "graph" | "eager")."""
+    import torch
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):          # warm-up outside the capture (one-time setup)
+            fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    mode = "graph"
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        run = g.replay
+    except RuntimeError:
+        mode = "eager"
+
+        def run():
+            for _ in range(reps):
+                fn()
+    run()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    run()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / reps, mode
+
+
+def run_sweep(args, local):
+    """Timings of the single-kernel configurations, one JSON line per case:
+    block attention for B in {4, 8, 16, 32} x L in {256, 1024, 4096}, both one
+    cache per call (L2-resident after the first call) and 36 distinct caches
+    in one batched launch (one per decoder layer; the working set exceeds L2
+    at L = 4096); the fused LM head + commit for R in {1, 16, 32, 128} rows
+    (its 622 MB of weights exceed L2 on every call)."""
+    import torch
+    import block_diffusion_vlm_b200 as dv
+    import dvlm_gen as gen
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dims = gen.QWEN3B
+    hbm_peak, peak_kind = peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def emit(d):
+        d.update(peak=hbm_peak, peak_source=f"{peak_kind} copy bandwidth")
+        print(json.dumps(d), flush=True)
+
+    if args.sweep in ("attention", "all"):
+        D, Hq, Hkv = dims.head_dim, dims.n_q_heads, dims.n_kv_heads
+        for B in (4, 8, 16, 32):
+            for L in (256, 1024, 4096):
+                Lmax = (L + B + 7) // 8 * 8
+                for nb in (1, dims.n_layers):
+                    q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=Lmax, n_batch=nb))
+                    qd, kd = q.to(dev).contiguous(), k.to(dev).contiguous()
+                    vt = v.transpose(-1, -2).contiguous().to(dev)
+                    out = torch.empty_like(qd)
+
+                    def call():
+                        dv.block_attn(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
+                                      Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, dtype=dv.DVLM_BF16, status=st)
+
+                    ms, mode = _device_ms_per_call(call, 20 if nb > 1 else 200, dev)
+                    b = nb * algorithmic_bytes("attention", dims, L, rows=B)
+                    emit({"sweep": "attention", "B": B, "L": L, "caches_per_launch": nb,
+                          "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
+                          "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
+                          "frac": b / (ms * 1e-3) / 1e9 / hbm_peak,
+                          "working_set_mb": (kd.numel() + vt.numel()) * 2 / 1e6, "timing": mode})
+                    del qd, kd, vt, out
+    if args.sweep in ("lmhead", "all"):
+        H, V = dims.hidden, dims.vocab
+        _, (w_t, _) = gen.lmhead_case(2, 1, H, V, second_set=False)
+        wd = w_t.to(dev)
+        for R in (1, 16, 32, 128):
+            hd = gen.normal_bf16(2, "lm.h1", (R, H))[0].to(dev)
+            o = dict(top1_id=torch.empty(R, dtype=torch.int32, device=dev),
+                     top1_prob=torch.empty(R, dtype=torch.float32, device=dev),
+                     commit=torch.empty(R, dtype=torch.uint8, device=dev),
+                     n_commit=torch.empty(1, dtype=torch.int32, device=dev))
+            ws = torch.zeros((dv.lmhead_workspace_size(R, V, H, dv.DVLM_BF16) + 3) // 4 + 1, dtype=torch.int32,
+                             device=dev)
+
+            def call():
+                dv.lmhead_conf_commit(hd, wd, R=R, H=H, V=V, dtype=dv.DVLM_BF16, threshold=TAU, workspace=ws,
+                                      status=st, **o)
+
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 20
+            e0.record()
+            for _ in range(reps):
+                call()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / reps
+            b = algorithmic_bytes("lm_head", dims, 0, rows=R)
+            emit({"sweep": "lm_head", "R": R, "us_per_launch": 1000 * ms, "bytes_per_launch": b,
+                  "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / hbm_peak, "timing": "eager"})
+    torch.cuda.synchronize(dev)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after the sweep")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -431,10 +545,15 @@ def main():
     ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")
     ap.add_argument("--profile-forwards", type=int, default=0,
                     help="profiling case: run this many eager forwards after prefill and exit")
+    ap.add_argument("--sweep", choices=["attention", "lmhead", "all"], default=None,
+                    help="time the single-kernel configurations (one JSON line per case) instead of the decode")
     args = ap.parse_args()
     rank, world, local, pg = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.sweep:
+            if rank == 0:
+                run_sweep(args, local)
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local, pg)
