@@ -497,6 +497,26 @@ def run_sweep(args, local):
                           "frac": b / (ms * 1e-3) / 1e9 / hbm_peak,
                           "working_set_mb": (kd.numel() + vt.numel()) * 2 / 1e6, "timing": mode})
                     del qd, kd, vt, out
+        # TEXT-ONLY pass of certificate-guided routing at the decode shape: the
+        # 1280 vision slots hidden by viewing the cache from slot 1280 (64 spare
+        # slots keep the last key chunk inside each head's rows)
+        B, L, n_vis = BLOCK, N_VIS + N_PROMPT, N_VIS
+        Lmax = (L + B + 7) // 8 * 8 + 64
+        q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=Lmax, n_batch=dims.n_layers))
+        qd, kd = q.to(dev).contiguous(), k.to(dev).contiguous()
+        vt = v.transpose(-1, -2).contiguous().to(dev)
+        out = torch.empty_like(qd)
+        for hide in (0, n_vis):
+            def call():
+                dv.block_attn(qd, out, kd[:, :, hide:, :], vt[:, :, :, hide:], n_batch=dims.n_layers, n_rows=B,
+                              n_clean=0, L=L - hide, Lmax=Lmax, Hq=Hq, Hkv=Hkv, D=D, scale=1.0 / D ** 0.5,
+                              dtype=dv.DVLM_BF16, status=st)
+
+            ms, mode = _device_ms_per_call(call, 20, dev)
+            emit({"sweep": "attention_text_only" if hide else "attention_full", "B": B, "L": L, "hidden_slots": hide,
+                  "caches_per_launch": dims.n_layers, "us_per_launch": 1000 * ms,
+                  "us_per_cache": 1000 * ms / dims.n_layers, "timing": mode})
+        del qd, kd, vt, out
     if args.sweep in ("lmhead", "all"):
         H, V = dims.hidden, dims.vocab
         _, (w_t, _) = gen.lmhead_case(2, 1, H, V, second_set=False)

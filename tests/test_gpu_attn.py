@@ -69,6 +69,33 @@ def test_batched_problems(cuda):
     assert err < TOL_BF16, err
 
 
+@pytest.mark.parametrize("n_vis,L,n_rows,n_clean,nb", [(1280, 1344, 16, 0, 1), (64, 300, 16, 0, 2),
+                                                       (8, 100, 4, 0, 1), (64, 64, 16, 0, 1), (128, 500, 12, 5, 1)])
+def test_text_only_pass_through_offset_cache_views(cuda, n_vis, L, n_rows, n_clean, nb):
+    """TEXT-ONLY pass of certificate-guided routing: cache slots 0..n_vis-1
+    (the vision rows) hidden from every row, positions unchanged.  Attention
+    reads no positions, so the public entry point computes it over the cache
+    seen from slot n_vis: K and V^T base pointers advanced by n_vis slots
+    (n_vis a multiple of 8 keeps both 16-byte aligned) and length L - n_vis.
+    Lmax keeps 64 spare slots, so the last 64-key chunk of every head stays
+    inside that head's rows."""
+    Lmax = _pad8(L + n_rows) + 64
+    q, k, v = (t for t, _ in gen.attn_case(8, n_rows, L, Lmax=Lmax, n_batch=nb))
+    qd, kd = q.to(cuda).contiguous(), k.to(cuda).contiguous()
+    vt = v.transpose(-1, -2).contiguous().to(cuda)
+    out = torch.full_like(qd, float("nan"))
+    st = status(cuda)
+    D = q.shape[-1]
+    dv.block_attn(qd, out, kd[:, :, n_vis:, :], vt[:, :, :, n_vis:], n_batch=nb, n_rows=n_rows, n_clean=n_clean,
+                  L=L - n_vis, Lmax=Lmax, Hq=16, Hkv=2, D=D, scale=1.0 / math.sqrt(D), dtype=dv.DVLM_BF16, status=st)
+    assert_ok(st)
+    q64, k64, v64 = f64(q), f64(k), f64(v)
+    want = np.stack([O.block_attention(q64[b], k64[b], v64[b], L, n_clean, 1.0 / math.sqrt(D), hide=n_vis)
+                     for b in range(nb)])
+    err = max_abs(f64(out), want)
+    assert err < TOL_BF16, err
+
+
 def test_slots_past_the_step_are_never_read(cuda):
     """Stale slots at or beyond L+n_rows (here NaN poison, as the speculative
     truncation leaves them) do not change any output."""
