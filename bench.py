@@ -34,6 +34,7 @@ N_VIS, N_PROMPT, N_NEW, BLOCK, TAU, SEED = 1280, 64, 256, 16, 0.9, 4
 WORKLOAD = "qwen2.5-3b-shaped block-diffusion decode: 36L h2048 16/2x128 ffn11008 V151936, ctx 1280 vision + 64 prompt, 256 new, B=16, tau 0.9"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # the part's nominal HBM3e bandwidth (context beside the measured copy figure)
 
 
 def peaks():
@@ -385,7 +386,8 @@ def run_ours(args, rank, world, local, pg):
         return {"bound": "hbm", "achieved": per[k]["gbs"], "peak": hbm_peak, "unit": "GB/s",
                 "frac": per[k]["gbs"] / hbm_peak, "traffic": load_traffic(k), "kernel": k,
                 "peak_source": f"{peak_kind} copy bandwidth", "bytes_per_launch": per[k]["bytes_per_launch"],
-                "ms_per_launch": per[k]["ms_per_launch"]}
+                "ms_per_launch": per[k]["ms_per_launch"], "frac_of_nominal": per[k]["gbs"] / NOMINAL_HBM_GBS,
+                "nominal_peak": NOMINAL_HBM_GBS}
 
     fwd_ms = sum(v["ms_per_launch"] * v["launches"] for v in per.values())
     fwd_bytes = dims.n_params() * 2
@@ -399,7 +401,9 @@ def run_ours(args, rank, world, local, pg):
             "gpu_launches": launches, "clocks": clk, "e2e": e2e,
             "decode": {"nfe_per_step": nfe, "tokens_per_nfe": N_NEW / nfe, "commit_hist": hist,
                        "ms_per_forward": 1000 * secs / args.steps / nfe,
-                       "forward_gbs": fwd_bytes / (secs / args.steps / nfe) / 1e9},
+                       "forward_gbs": fwd_bytes / (secs / args.steps / nfe) / 1e9,
+                       "forward_frac": fwd_bytes / (secs / args.steps / nfe) / 1e9 / hbm_peak,
+                       "forward_frac_of_nominal": fwd_bytes / (secs / args.steps / nfe) / 1e9 / NOMINAL_HBM_GBS},
             "kernels": per, "eager_forward_ms": fwd_ms}
 
     # a short run of the linear self-speculative mode for context
