@@ -390,7 +390,7 @@ def run_ours(args, rank, world, local, pg):
                 "nominal_peak": NOMINAL_HBM_GBS}
 
     fwd_ms = sum(v["ms_per_launch"] * v["launches"] for v in per.values())
-    fwd_bytes = dims.n_params() * 2
+    fwd_bytes = dims.streamed_params() * 2
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

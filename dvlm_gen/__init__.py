@@ -60,6 +60,11 @@ class ModelDims:
         per_layer = self.qkv_rows * H + H * self.n_q_heads * self.head_dim + 3 * I * H
         return self.n_layers * per_layer + 2 * V * H
 
+    def streamed_params(self) -> int:
+        """Parameters a forward pass reads in full: every decoder matrix and
+        the LM head; the embedding table is only gathered by row."""
+        return self.n_params() - self.vocab * self.hidden
+
 
 # Tiny fp32 model of the first configuration: LM head scaled x40.
 TINY = ModelDims(n_layers=1, hidden=32, n_q_heads=2, n_kv_heads=1, head_dim=16,
