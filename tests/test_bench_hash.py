@@ -1,6 +1,7 @@
-"""bench.py attaches the committed DRAM traffic to the kernel source it was
-measured on: the key ignores comments and white space but changes with any
-code edit."""
+"""bench.py's roofline bookkeeping: the committed DRAM traffic stays attached
+to the kernel source it was measured on (the key ignores comments and white
+space but changes with any code edit), and the algorithmic bytes per launch
+add up to the weights a forward streams."""
 import importlib
 import os
 import shutil
@@ -41,3 +42,21 @@ def test_source_hash_ignores_comments_but_not_code(bench_copy):
     assert bench.source_hash() == h0
     f.write_text(text.replace("kChunk = 64", "kChunk = 32", 1))
     assert bench.source_hash() != h0
+
+
+def test_algorithmic_bytes_add_up_to_the_streamed_weights():
+    """The per-launch byte counts the roofline uses: the configured figures at
+    16 rows, and the weight bytes of one forward's launches (36 layers of the
+    four projections plus the LM head) equal the streamed parameter bytes."""
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    import dvlm_gen as gen
+    d = gen.QWEN3B
+    ab = {k: bench.algorithmic_bytes(k, d, 1344, rows=16) for k in
+          ("qkv_gemm", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head", "attention")}
+    assert ab["qkv_gemm"] == 10_633_216 and ab["oproj_gemm"] == 8_585_216
+    assert ab["gateup_gemm"] == 90_595_328 and ab["down_gemm"] == 45_572_096
+    assert ab["lm_head"] == 622_395_392 and ab["attention"] == 1_523_712
+    weights = {k: bench.algorithmic_bytes(k, d, 0, rows=0) for k in ab if k != "attention"}
+    assert d.n_layers * sum(v for k, v in weights.items() if k != "lm_head") + weights["lm_head"] == \
+        2 * d.streamed_params() == 6_171_394_048
