@@ -31,9 +31,11 @@ from gpu_util import assert_ok, f64, max_abs, status, ws_tensor
 
 pytestmark = pytest.mark.gpu
 MARGIN = 1e-3
-# bound on |p1(GPU) - p1(oracle)| for the bf16 reduced model on identical inputs
-# (hidden states one storage ulp apart in a few elements; measured up to 0.03)
-DELTA = 0.05
+# bound on |p1(GPU) - p1(oracle)| for the bf16 reduced model on identical inputs:
+# hidden states one storage ulp apart in a few elements move p1 by a few 1e-2
+# (GPU against oracle: up to 0.03 measured; a CPU model of such rounding
+# flips: up to 0.066, tests/test_precision_model.py)
+DELTA = 0.1
 
 SMALL_BF16 = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=1024,
                            vocab=4096, lm_scale=25.0, dtype="bf16")
