@@ -1,6 +1,7 @@
-"""How much of the 2e-2 attention bar the GPU's precision choices use.
+"""numpy models of the GPU path's arithmetic (not of its code) against the
+fp64 oracle: they show how much of each parity bar the precision choices use.
 
-A numpy model of the arithmetic (not of the code) of the bf16 attention
+Attention (bar 2e-2).  A numpy model of the arithmetic of the bf16 attention
 path: fp32 scores from bf16 q and k; keys split over 16 cooperating CTAs in
 64-key chunks taken round-robin; each CTA's probabilities exp2(s - m_cta)
 rounded to fp16 and multiplied by the fp16 copy of V with fp32 accumulation;
@@ -106,3 +107,20 @@ def test_bf16_storage_flips_move_p1_by_hundredths(seed):
 
     O.decode_threshold(ref, s, 16, 0.9, 32, on_iter=on_iter, on_block=on_block)
     assert 0.01 < max(moves) < TEACHER_FORCED_DELTA, max(moves)
+
+
+def test_lmhead_p1_precision_within_its_bar():
+    """The fused LM head's p1 bar (2e-4 against the fp64 oracle): bf16 hidden
+    rows and weights, logits summed in fp32, softmax sum and maximum in fp32.
+    On the configuration's distributions (hidden N(0,1), W N(0, 0.02) x 25,
+    H = 2048; a 16384-row slice of the vocabulary, the per-logit arithmetic
+    being the same) p1 moves by orders of magnitude less than the bar."""
+    H, V, R = 2048, 16384, 16
+    (_, h), (_, w) = gen.lmhead_case(2, R, H, V, second_set=False)
+    lg32 = h.astype(np.float32) @ w.astype(np.float32).T
+    m = lg32.max(axis=1, keepdims=True)
+    p1_32 = 1.0 / np.exp(lg32 - m).sum(axis=1, dtype=np.float32)
+    want = O.lm_head_conf(h.astype(np.float64), w.astype(np.float64))
+    err = float(np.abs(p1_32 - want.p1).max())
+    assert err < 2e-4 / 20, err
+    assert np.array_equal(lg32.argmax(axis=1)[want.p1 - want.p2 >= 1e-3], want.top1[want.p1 - want.p2 >= 1e-3])
