@@ -572,12 +572,17 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
     return tr
 
 
-def decode_spec_linear(model: OracleModel, seed_token: int, B: int, max_new: int) -> DecodeTrace:
+def decode_spec_linear(model: OracleModel, seed_token: int, B: int, max_new: int, on_round=None) -> DecodeTrace:
     """Linear self-speculative decoding [FDV §2.3.1]: a diffusion draft pass
     (every position takes its argmax), then a causal verify pass over the
     draft; the longest prefix on which the verifier agrees is kept (position
     0, the AR seed, always), L advances by its length and the verifier's
-    prediction right after it seeds the next round (shift=1)."""
+    prediction right after it seeds the next round (shift=1).
+
+    Optional observer (it does not change the trajectory): on_round(L,
+    draft_input, draft_conf, draft, verify_conf, k, next_seed) after each
+    round, with the draft pass's input tokens and the per-row confidences of
+    both passes (row r scores position r + 1)."""
     d = model.d
     tr = DecodeTrace(tokens=[])
     seed = seed_token
@@ -599,6 +604,8 @@ def decode_spec_linear(model: OracleModel, seed_token: int, B: int, max_new: int
         tr.tokens.extend(draft[:k])
         model.L = L + k
         seed = int(g.top1[k - 1])
+        if on_round is not None:
+            on_round(L, list(toks), c, list(draft), g, k, seed)
     tr.tokens = tr.tokens[:max_new]
     return tr
 

@@ -190,3 +190,56 @@ def test_bf16_reduced_model_threshold_teacher_forced(cuda, seed):
     assert counts["iters"] == tr.nfe - len(tr.tokens) // B
     assert counts["top1"] > 0 and counts["commit"] > 0
     s.eng.close()
+
+
+@pytest.mark.parametrize("seed", [6, 2])
+def test_bf16_reduced_model_spec_teacher_forced(cuda, seed):
+    """Linear self-speculative decoding (B=16, 32 tokens) of the reduced bf16
+    model, per round and teacher-forced: the oracle's draft pass ([seed,
+    MASK...], noisy) and verify pass (its draft, causal) are replayed on the
+    GPU over the same cache, top-1 ids compared wherever the oracle's margin
+    is at least DELTA and p1 within DELTA, then the cache length and seed are
+    set to the oracle's accepted prefix."""
+    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
+    eng, d, dev = s.eng, SMALL_BF16, cuda
+    B = 16
+    eng.prefill(s.vis_t.to(dev), 32, torch.from_numpy(s.ids).to(dev), 16)
+    _, seed_gpu = eng.position()
+    lw = ws_tensor(dv.lmhead_workspace_size(B, d.vocab, d.hidden, dv.DVLM_BF16), dev)
+    x = torch.zeros((B, d.hidden), dtype=torch.bfloat16, device=dev)
+    counts = {"rounds": 0, "draft": 0, "verify": 0}
+
+    def gpu_rows(toks, n_clean):
+        eng.forward(B, n_clean, d.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=dev), x_out=x)
+        top = torch.zeros(B, dtype=torch.int32, device=dev)
+        p1 = torch.zeros(B, dtype=torch.float32, device=dev)
+        st = status(dev)
+        dv.lmhead_conf_commit(x, s.dm.lm_head, R=B, H=d.hidden, V=d.vocab, dtype=dv.DVLM_BF16, apply_rmsnorm=1,
+                              top1_id=top, top1_prob=p1, workspace=lw, status=st)
+        assert_ok(st)
+        return top.cpu().numpy(), p1.cpu().numpy()
+
+    def check(rows, conf, top, p1, key):
+        for r in range(rows):
+            assert abs(p1[r] - conf.p1[r]) <= DELTA, (key, r, p1[r], conf.p1[r])
+            if conf.p1[r] - conf.p2[r] >= DELTA:
+                assert top[r] == conf.top1[r], (key, r)
+                counts[key] += 1
+
+    def on_round(L, toks, c, draft, g, k, nxt):
+        assert eng.position()[0] == L
+        top, p1 = gpu_rows(toks, 0)
+        check(B - 1, c, top, p1, "draft")        # row r drafts position r + 1
+        top, p1 = gpu_rows(draft, B)
+        check(B, g, top, p1, "verify")
+        eng.set_position(L + k, nxt)
+        counts["rounds"] += 1
+
+    m = O.OracleModel(s.od, weights=s.w, bf16=True, Lmax=s.Lmax)
+    seed_o = O.prefill(m, s.vis.astype(np.float64), s.ids)
+    assert seed_o == seed_gpu
+    tr = O.decode_spec_linear(m, seed_o, B, 32, on_round=on_round)
+    eng.check()
+    assert counts["rounds"] == len(tr.accept_lens)
+    assert counts["draft"] > 0 and counts["verify"] > 0
+    s.eng.close()

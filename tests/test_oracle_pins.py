@@ -303,6 +303,30 @@ def test_threshold_observers_do_not_change_the_trajectory():
     assert blocks[1][0] == blocks[0][0] + B
 
 
+def test_spec_observer_does_not_change_the_trajectory():
+    """The per-round observer of the teacher-forced speculative GPU check sees
+    every round: the draft pass's input, both passes' row scores, the draft,
+    the accepted length and the next seed, consistent with one another."""
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s = _fresh(d, w, False, vis, ids)
+    plain = O.decode_spec_linear(m, s, B, 12)
+    rounds = []
+
+    def on_round(L, toks, c, draft, g, k, nxt):
+        assert toks == [draft[0]] + [d.mask_id] * (B - 1)
+        assert draft[1:] == [int(t) for t in c.top1[:B - 1]]
+        verify = [draft[0]] + [int(t) for t in g.top1[:B - 1]]
+        assert k == O.prefix_accept(verify, draft) and nxt == int(g.top1[k - 1])
+        rounds.append((L, k))
+
+    m, s = _fresh(d, w, False, vis, ids)
+    obs = O.decode_spec_linear(m, s, B, 12, on_round=on_round)
+    assert obs.tokens == plain.tokens and obs.accept_lens == plain.accept_lens and obs.nfe == plain.nfe
+    assert [k for _, k in rounds] == plain.accept_lens
+    assert all(rounds[i + 1][0] == rounds[i][0] + rounds[i][1] for i in range(len(rounds) - 1))
+
+
 def test_block_first_token_is_ar_token_and_append_kv_equals_prefill():
     gd, d, w, vis, ids = _tiny()
     B = 4
