@@ -1,0 +1,116 @@
+"""bench.py's own arm assembles the benchmark's JSON line from measured
+values; here the measuring parts (CUDA, the engine, the device model) are
+replaced by stand-ins with fixed timings, so that the line's assembly runs on
+the CPU and its contract keys are checked before any GPU run."""
+import importlib
+import json
+import os
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+class _Event:
+    def __init__(self, enable_timing=False):
+        pass
+
+    def record(self, stream=None):
+        pass
+
+    def elapsed_time(self, other):
+        return 100.0                                   # ms between any two events
+
+
+class _Stream:
+    cuda_stream = 0
+
+    def __init__(self, device=None):
+        pass
+
+
+class _FakeEngine:
+    def __init__(self, *a, **k):
+        pass
+
+    def prefill(self, *a, **k):
+        pass
+
+    def check(self, stream=None):
+        pass
+
+    def position(self, stream=None):
+        return 1344, 7
+
+    def set_position(self, L, seed, stream=None):
+        pass
+
+    def generate(self, cfg, out, st=None, stream=None):
+        if st is not None:
+            st.nfe, st.n_tokens, st.n_launches = 71, 256, 12954
+            st.commit_hist[1], st.commit_hist[15] = 70, 1
+
+    def generate_host(self, *a, **k):
+        pass
+
+    def profile_forward(self, *a, **k):
+        ms = {"embed": 0.01, "qkv_gemm": 0.47, "attention": 0.56, "oproj_gemm": 0.43, "gateup_gemm": 0.90,
+              "down_gemm": 0.68, "lm_head": 0.107}
+        return {k: (v, 1 if k in ("embed", "lm_head") else 36) for k, v in ms.items()}
+
+    def close(self):
+        pass
+
+
+class _FakeDeviceModel:
+    def __init__(self, *a, **k):
+        pass
+
+    def c_model(self):
+        return None
+
+
+def test_default_arm_line_has_the_contract_keys(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    import block_diffusion_vlm_b200 as dv
+    import dvlm_gen as gen
+    import dvlm_gen.device as gdev
+    real_device = torch.device
+    monkeypatch.setattr(torch, "device", lambda *a, **k: real_device("cpu"))
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "Stream", _Stream)
+    monkeypatch.setattr(torch.cuda, "Event", _Event)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(dv, "Engine", _FakeEngine)
+    monkeypatch.setattr(dv, "engine_workspace_size", lambda *a: 64)
+    monkeypatch.setattr(gdev, "DeviceModel", _FakeDeviceModel)
+    monkeypatch.setattr(gdev, "kv_buffers", lambda *a, **k: (None, None))
+    monkeypatch.setattr(bench, "gpu_uuid", lambda: None)
+    args = bench.argparse.Namespace(steps=5, warmup=3, mode="threshold", quick=True, no_cpu_baseline=True,
+                                    layers=36, profile_forwards=0, impl="ours", gpus=1, sweep=None)
+    bench.run_ours(args, 0, 1, 0, None)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in d, key
+    assert d["value"] == pytest.approx(256 * 5 / 0.1) and d["ms_per_step"] == pytest.approx(20.0)
+    assert d["n_gpus"] == 1 and d["dtype"] == "bf16" and d["higher_is_better"] is True
+    assert "workload" in d["config"] and d["gpu_launches"] == 5 * 12954
+    r = d["roofline"]
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r) and r["kernel"] == "gateup_gemm"
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"]) and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(bench.algorithmic_bytes("gateup_gemm", gen.QWEN3B, 1344) /
+                                          (0.90 / 36 * 1e-3) / 1e9)
+    assert d["lmhead"]["kernel"] == "lm_head"
+    e = d["e2e"]
+    assert e["h2d_bytes_per_step"] == 1280 * 2048 * 2 + 64 * 4 and e["d2h_bytes_per_step"] == 256 * 4
+    dec = d["decode"]
+    assert dec["nfe_per_step"] == 71
+    assert dec["forward_gbs"] == pytest.approx(6_171_394_048 / (0.1 / 5 / 71) / 1e9)
+    assert isinstance(d["clocks"], dict) and "reasons" in d["clocks"]
