@@ -114,3 +114,64 @@ def test_default_arm_line_has_the_contract_keys(monkeypatch, capsys):
     assert dec["nfe_per_step"] == 71
     assert dec["forward_gbs"] == pytest.approx(6_171_394_048 / (0.1 / 5 / 71) / 1e9)
     assert isinstance(d["clocks"], dict) and "reasons" in d["clocks"]
+
+
+class _Graph:
+    def replay(self):
+        pass
+
+
+class _GraphCtx:
+    def __init__(self, g):
+        pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
+    """`bench.py --sweep all` with the entry points, CUDA graphs and large
+    draws replaced by stand-ins: the attention cases (12 shapes, one cache
+    and 36 caches per launch, plus the TEXT-ONLY pair) and the four LM-head
+    row counts each print one line with their bytes, GB/s and fraction."""
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    import block_diffusion_vlm_b200 as dv
+    import dvlm_gen as gen
+    real_device = torch.device
+    monkeypatch.setattr(torch, "device", lambda *a, **k: real_device("cpu"))
+    for name, fake in [("set_device", lambda *a, **k: None), ("synchronize", lambda *a, **k: None),
+                       ("Stream", _Stream), ("Event", _Event), ("CUDAGraph", _Graph), ("graph", _GraphCtx),
+                       ("current_stream", lambda *a, **k: _Stream()), ("stream", lambda s: _GraphCtx(s))]:
+        monkeypatch.setattr(torch.cuda, name, fake)
+    monkeypatch.setattr(_Stream, "wait_stream", lambda self, other: None, raising=False)
+    calls = {"attn": [], "lm": []}
+    monkeypatch.setattr(dv, "block_attn", lambda q, out, k, v, **kw: calls["attn"].append(kw))
+    monkeypatch.setattr(dv, "lmhead_conf_commit", lambda h, w, **kw: calls["lm"].append(kw["R"]))
+    monkeypatch.setattr(dv, "lmhead_workspace_size", lambda *a: 64)
+    small = torch.zeros(2, 2, 2, 2, dtype=torch.bfloat16)
+    monkeypatch.setattr(gen, "attn_case", lambda *a, **k: ((small, None),) * 3)
+    monkeypatch.setattr(gen, "lmhead_case", lambda *a, **k: ((small, None), (small, None)))
+    monkeypatch.setattr(gen, "normal_bf16", lambda *a, **k: (small, None))
+    args = bench.argparse.Namespace(sweep="all")
+    bench.run_sweep(args, 0)
+    lines = [json.loads(ln) for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    attn = [d for d in lines if d["sweep"] == "attention"]
+    assert len(attn) == 4 * 3 * 2
+    assert {(d["B"], d["L"], d["caches_per_launch"]) for d in attn} == \
+        {(B, L, nb) for B in (4, 8, 16, 32) for L in (256, 1024, 4096) for nb in (1, 36)}
+    for d in attn:
+        assert d["bytes_per_launch"] == d["caches_per_launch"] * bench.algorithmic_bytes("attention", gen.QWEN3B,
+                                                                                         d["L"], rows=d["B"])
+        assert d["frac"] == pytest.approx(d["gbs"] / d["peak"]) and d["timing"] == "graph"
+    text = {d["sweep"]: d for d in lines if d["sweep"].startswith("attention_")}
+    assert set(text) == {"attention_full", "attention_text_only"}
+    assert text["attention_text_only"]["hidden_slots"] == 1280 and text["attention_full"]["hidden_slots"] == 0
+    hidden = [kw for kw in calls["attn"] if kw["L"] == 1344 - 1280]
+    assert hidden and all(kw["Lmax"] >= 1344 + 16 + 64 and kw["n_batch"] == 36 for kw in hidden)
+    lm = [d for d in lines if d["sweep"] == "lm_head"]
+    assert [d["R"] for d in lm] == [1, 16, 32, 128]
+    assert all(d["bytes_per_launch"] == bench.algorithmic_bytes("lm_head", gen.QWEN3B, 0, rows=d["R"]) for d in lm)
