@@ -1,10 +1,14 @@
-"""The teacher-forced GPU decode checks, run on the CPU against a stand-in
-engine: a copy of the oracle whose stored bf16 values are perturbed by about
+"""GPU checks whose logic can run on the CPU against stand-ins.
+
+The teacher-forced decode checks run against a stand-in engine: a copy of the oracle whose stored bf16 values are perturbed by about
 5e-7 relative before rounding (the CPU model of the GPU's fp32-sum
 differences), behind the same calls the checks make (prefill, position,
 forward with x_out / advance, set_position, the fused LM head).  This runs
 the checks' own logic -- call order, row-to-position mapping, accepted-prefix
-bookkeeping, tolerances -- before any GPU does."""
+bookkeeping, tolerances -- before any GPU does.  The TEXT-ONLY attention
+check runs against a stand-in that addresses memory as the kernel does, from
+the base pointers it is given, so the offset cache views are shown to reach
+exactly the intended slots and to stay inside their buffers."""
 import numpy as np
 import pytest
 import torch
@@ -124,3 +128,57 @@ def test_threshold_check_catches_a_swapped_row_mapping(standin, monkeypatch):
     monkeypatch.setattr(dv, "lmhead_conf_commit", unshifted)
     with pytest.raises(AssertionError):
         T.test_bf16_reduced_model_threshold_teacher_forced(standin, 1)
+
+
+def _attn_by_kernel_addressing(q, out, k, v, *, n_batch, n_rows, n_clean, L, Lmax, Hq, Hkv, D, scale, dtype,
+                               status=None, **kw):
+    """Block attention computed from raw storage with the kernel's
+    addressing: K row (b*Hkv + g)*Lmax + key from the K base pointer, V^T
+    element ((b*Hkv + g)*D + d)*Lmax + key from the V base pointer, keys
+    0..L+n_rows-1, every 64-key box the kernel requests inside the storage."""
+    kflat = torch.empty(0, dtype=k.dtype).set_(k.untyped_storage()).float()
+    vflat = torch.empty(0, dtype=v.dtype).set_(v.untyped_storage()).float()
+    ko, vo = k.storage_offset(), v.storage_offset()
+    n_keys = L + n_rows
+    boxed = -(-n_keys // 64) * 64
+    qn = q.float().numpy().astype(np.float64)
+    res = np.zeros(qn.shape)
+    for b in range(n_batch):
+        for g in range(Hkv):
+            row0 = (b * Hkv + g) * Lmax
+            assert ko + (row0 + boxed) * D <= kflat.numel()
+            assert vo + ((b * Hkv + g) * D + D - 1) * Lmax + boxed <= vflat.numel()
+            K = kflat[ko + row0 * D: ko + (row0 + n_keys) * D].reshape(n_keys, D).numpy().astype(np.float64)
+            base = vo + (b * Hkv + g) * D * Lmax
+            V = np.stack([vflat[base + d * Lmax: base + d * Lmax + n_keys].numpy() for d in range(D)],
+                         axis=1).astype(np.float64)
+            heads = slice(g * (Hq // Hkv), (g + 1) * (Hq // Hkv))
+            res[b][:, heads] = O.block_attention(qn[b][:, heads], K[None], V[None], L, n_clean, scale)
+    out.copy_(torch.from_numpy(res.astype(np.float32)).to(out.dtype))
+
+
+@pytest.mark.parametrize("case", [(1280, 1344, 16, 0, 1), (64, 300, 16, 0, 2), (8, 100, 4, 0, 1),
+                                  (64, 64, 16, 0, 1), (128, 500, 12, 5, 1)])
+def test_text_only_offset_views_reach_the_intended_slots(standin, monkeypatch, case):
+    import test_gpu_attn as TA
+    monkeypatch.setattr(dv, "block_attn", _attn_by_kernel_addressing)
+    monkeypatch.setattr(TA, "assert_ok", lambda st: None)
+    TA.test_text_only_pass_through_offset_cache_views(standin, *case)
+
+
+def test_text_only_check_catches_unhidden_vision_slots(standin, monkeypatch):
+    """Reading from the cache's own base (the vision slots not hidden) fails
+    the TEXT-ONLY check."""
+    import test_gpu_attn as TA
+
+    def from_base(q, out, k, v, **kw):
+        full_k = torch.empty(0, dtype=k.dtype).set_(k.untyped_storage())
+        full_v = torch.empty(0, dtype=v.dtype).set_(v.untyped_storage())
+        n_vis = k.storage_offset() // kw["D"]
+        kw["L"] += n_vis
+        _attn_by_kernel_addressing(q, out, full_k, full_v, **kw)
+
+    monkeypatch.setattr(dv, "block_attn", from_base)
+    monkeypatch.setattr(TA, "assert_ok", lambda st: None)
+    with pytest.raises(AssertionError):
+        TA.test_text_only_pass_through_offset_cache_views(standin, 64, 300, 16, 0, 1)
