@@ -90,6 +90,7 @@ def _declare(L: ctypes.CDLL) -> None:
                                          _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
         "dvlm_lmhead_conf_commit_static": (_i, [_vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                                 _vp, _vp, _vp, _vp, _vp]),
+        "dvlm_topk_commit": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
         "dvlm_spec_workspace_size": (_sz, [_i, _i, _i]),
         "dvlm_spec_verify_accept": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp,
                                          _sz, _vp, _vp]),
@@ -177,6 +178,14 @@ def lmhead_conf_commit_static(hidden, w, *, R, H, V, apply_rmsnorm=0, eps=1e-6, 
                                                 ptr(top1_prob), ptr(commit), ptr(n_commit), ptr(anchor_id),
                                                 ptr(anchor_conf), ptr(cert_len), ptr(status), stream_handle(stream)),
            "dvlm_lmhead_conf_commit_static")
+
+
+def topk_commit(top1_prob, top1_id, masked, tokens, *, R, k, commit=None, n_commit=None, status=None,
+                stream=None) -> None:
+    """Commit the k most confident masked rows in place (dvlm_topk_commit)."""
+    _check(lib().dvlm_topk_commit(ptr(top1_prob), ptr(top1_id), ptr(masked), ptr(tokens), int(R), int(k),
+                                  ptr(commit), ptr(n_commit), ptr(status), stream_handle(stream)),
+           "dvlm_topk_commit")
 
 
 def spec_workspace_size(b: int, B: int, V: int) -> int:

@@ -22,6 +22,8 @@ void engine_plan(dvlm_engine* e);
 cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* counts, cudaStream_t s);
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v);
 int engine_get_option(dvlm_engine* e, const char* name);
+cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, uint8_t* masked, int32_t* tokens, int R, int k,
+                               uint8_t* commit, int32_t* n_commit, cudaStream_t s);
 }  // namespace dvlm
 
 namespace {
@@ -249,6 +251,14 @@ size_t dvlm_spec_workspace_size(int b, int B, int V) {
   if (b < 1 || B < 1 || V < 1) return 0;
   const size_t part = static_cast<size_t>(b) * B * spec_splits(b, B) * 2 * 4;
   return (part + 255) / 256 * 256 + static_cast<size_t>(b) * 4 + 256;
+}
+
+dvlm_status dvlm_topk_commit(const float* top1_prob, const int32_t* top1_id, uint8_t* masked, int32_t* tokens,
+                             int R, int k, uint8_t* commit, int32_t* n_commit, int* dev_status, dvlm_stream stream) {
+  (void)dev_status;
+  if (!top1_prob || !top1_id || !masked || !tokens) return DVLM_ERR_INVALID_ARG;
+  if (R < 1 || R > 128 || k < 0) return DVLM_ERR_SHAPE;
+  return cuda_status(launch_topk_commit(top1_prob, top1_id, masked, tokens, R, k, commit, n_commit, cs(stream)));
 }
 
 dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const int32_t* verify_ids, const int32_t* draft_ids,

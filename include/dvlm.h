@@ -162,6 +162,25 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit_static(const void* hidden, const vo
                                                    int32_t* cert_len, int* dev_status, dvlm_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Top-k commit [Look Only When Needed, background: the baseline dVLM
+ * schedule unmasks the k most confident masked positions per step].
+ *
+ * Among rows r < R with masked[r] != 0, the k of highest top1_prob[r] (lower
+ * row first on equal values) are committed: tokens[r] = top1_id[r] and
+ * masked[r] = 0; every other row keeps its token and mask.  commit[r] = 1 for
+ * the committed rows, 0 otherwise; *n_commit = min(k, number of masked rows).
+ * top1_prob [R] (finite), top1_id [R]: device, as written by
+ * dvlm_lmhead_conf_commit; masked [R] (uint8, in/out), tokens [R] (int32,
+ * in/out): device; commit [R] and n_commit [1]: device, may be NULL.
+ * 1 <= R <= 128, k >= 0.  Errors: DVLM_ERR_INVALID_ARG (a required pointer is
+ * NULL), DVLM_ERR_SHAPE (R or k out of range).  One small kernel on `stream`,
+ * asynchronous; dev_status is unused (no device-side failure mode).
+ */
+DVLM_API dvlm_status dvlm_topk_commit(const float* top1_prob, const int32_t* top1_id, uint8_t* masked,
+                                      int32_t* tokens, int R, int k, uint8_t* commit, int32_t* n_commit,
+                                      int* dev_status, dvlm_stream stream);
+
+/* ------------------------------------------------------------------------
  * Speculative verify + longest-prefix accept + in-place KV truncation.
  *
  * For each sequence i < b: v_j = argmax_v verify_logits[i, j, :] (lowest id

@@ -99,6 +99,15 @@ def test_spec_host_validation(dvlm_lib):
     assert f(None, 16, 16, 1, 16, 100, 16, None, 1, None, None, 0, 0, 0, 0, None, 0, None, None) == INVALID
 
 
+def test_topk_host_validation(dvlm_lib):
+    f = dv.lib().dvlm_topk_commit
+    assert f(None, 16, 16, 16, 4, 1, None, None, None, None) == INVALID
+    assert f(16, 16, 16, None, 4, 1, None, None, None, None) == INVALID
+    assert f(16, 16, 16, 16, 0, 1, None, None, None, None) == SHAPE
+    assert f(16, 16, 16, 16, 129, 1, None, None, None, None) == SHAPE
+    assert f(16, 16, 16, 16, 4, -1, None, None, None, None) == SHAPE
+
+
 def _dims_model(**kw):
     import dvlm_gen as gen
     m = dv.make_model(gen.QWEN3B, embed=None, wqkv=None, wo=None, wgate=None, wup=None, wdown=None,
