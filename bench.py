@@ -552,6 +552,18 @@ def run_sweep(args, local):
             b = algorithmic_bytes("lm_head", dims, 0, rows=R)
             emit({"sweep": "lm_head", "R": R, "us_per_launch": 1000 * ms, "bytes_per_launch": b,
                   "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / hbm_peak, "timing": "eager"})
+        # top-k commit on the LM head's per-row outputs (a latency-bound launch)
+        R, k = BLOCK, 4
+        p1 = torch.rand(R, device=dev)
+        top = torch.zeros(R, dtype=torch.int32, device=dev)
+        masked = torch.ones(R, dtype=torch.uint8, device=dev)
+        tokens = torch.zeros(R, dtype=torch.int32, device=dev)
+
+        def call():
+            dv.topk_commit(p1, top, masked, tokens, R=R, k=k, status=st)
+
+        ms, mode = _device_ms_per_call(call, 200, dev)
+        emit({"sweep": "topk_commit", "R": R, "k": k, "us_per_launch": 1000 * ms, "timing": mode})
     torch.cuda.synchronize(dev)
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} after the sweep")

@@ -152,6 +152,7 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     monkeypatch.setattr(dv, "block_attn", lambda q, out, k, v, **kw: calls["attn"].append(kw))
     monkeypatch.setattr(dv, "lmhead_conf_commit", lambda h, w, **kw: calls["lm"].append(kw["R"]))
     monkeypatch.setattr(dv, "lmhead_workspace_size", lambda *a: 64)
+    monkeypatch.setattr(dv, "topk_commit", lambda *a, **kw: calls["lm"].append(("topk", kw["R"], kw["k"])))
     small = torch.zeros(2, 2, 2, 2, dtype=torch.bfloat16)
     monkeypatch.setattr(gen, "attn_case", lambda *a, **k: ((small, None),) * 3)
     monkeypatch.setattr(gen, "lmhead_case", lambda *a, **k: ((small, None), (small, None)))
@@ -175,3 +176,5 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     lm = [d for d in lines if d["sweep"] == "lm_head"]
     assert [d["R"] for d in lm] == [1, 16, 32, 128]
     assert all(d["bytes_per_launch"] == bench.algorithmic_bytes("lm_head", gen.QWEN3B, 0, rows=d["R"]) for d in lm)
+    tk = [d for d in lines if d["sweep"] == "topk_commit"]
+    assert len(tk) == 1 and tk[0]["R"] == 16 and tk[0]["us_per_launch"] > 0
