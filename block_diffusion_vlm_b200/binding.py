@@ -91,6 +91,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_lmhead_conf_commit_static": (_i, [_vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                                 _vp, _vp, _vp, _vp, _vp]),
         "dvlm_topk_commit": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
+        "dvlm_divergence_first_commit": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
         "dvlm_spec_workspace_size": (_sz, [_i, _i, _i]),
         "dvlm_spec_verify_accept": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp,
                                          _sz, _vp, _vp]),
@@ -186,6 +187,16 @@ def topk_commit(top1_prob, top1_id, masked, tokens, *, R, k, commit=None, n_comm
     _check(lib().dvlm_topk_commit(ptr(top1_prob), ptr(top1_id), ptr(masked), ptr(tokens), int(R), int(k),
                                   ptr(commit), ptr(n_commit), ptr(status), stream_handle(stream)),
            "dvlm_topk_commit")
+
+
+def divergence_first_commit(full_prob, full_id, text_id, masked, tokens, *, R, k, commit=None, n_commit=None,
+                            status=None, stream=None) -> None:
+    """Commit k masked rows in place, TEXT-ONLY/FULL divergent rows first
+    (dvlm_divergence_first_commit)."""
+    _check(lib().dvlm_divergence_first_commit(ptr(full_prob), ptr(full_id), ptr(text_id), ptr(masked), ptr(tokens),
+                                              int(R), int(k), ptr(commit), ptr(n_commit), ptr(status),
+                                              stream_handle(stream)),
+           "dvlm_divergence_first_commit")
 
 
 def spec_workspace_size(b: int, B: int, V: int) -> int:

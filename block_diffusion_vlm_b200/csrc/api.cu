@@ -22,8 +22,8 @@ void engine_plan(dvlm_engine* e);
 cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* counts, cudaStream_t s);
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v);
 int engine_get_option(dvlm_engine* e, const char* name);
-cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, uint8_t* masked, int32_t* tokens, int R, int k,
-                               uint8_t* commit, int32_t* n_commit, cudaStream_t s);
+cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, const int32_t* other_ids, uint8_t* masked,
+                               int32_t* tokens, int R, int k, uint8_t* commit, int32_t* n_commit, cudaStream_t s);
 }  // namespace dvlm
 
 namespace {
@@ -258,7 +258,18 @@ dvlm_status dvlm_topk_commit(const float* top1_prob, const int32_t* top1_id, uin
   (void)dev_status;
   if (!top1_prob || !top1_id || !masked || !tokens) return DVLM_ERR_INVALID_ARG;
   if (R < 1 || R > 128 || k < 0) return DVLM_ERR_SHAPE;
-  return cuda_status(launch_topk_commit(top1_prob, top1_id, masked, tokens, R, k, commit, n_commit, cs(stream)));
+  return cuda_status(
+      launch_topk_commit(top1_prob, top1_id, nullptr, masked, tokens, R, k, commit, n_commit, cs(stream)));
+}
+
+dvlm_status dvlm_divergence_first_commit(const float* full_prob, const int32_t* full_id, const int32_t* text_id,
+                                         uint8_t* masked, int32_t* tokens, int R, int k, uint8_t* commit,
+                                         int32_t* n_commit, int* dev_status, dvlm_stream stream) {
+  (void)dev_status;
+  if (!full_prob || !full_id || !text_id || !masked || !tokens) return DVLM_ERR_INVALID_ARG;
+  if (R < 1 || R > 128 || k < 0) return DVLM_ERR_SHAPE;
+  return cuda_status(
+      launch_topk_commit(full_prob, full_id, text_id, masked, tokens, R, k, commit, n_commit, cs(stream)));
 }
 
 dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const int32_t* verify_ids, const int32_t* draft_ids,

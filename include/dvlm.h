@@ -180,6 +180,20 @@ DVLM_API dvlm_status dvlm_topk_commit(const float* top1_prob, const int32_t* top
                                       int32_t* tokens, int R, int k, uint8_t* commit, int32_t* n_commit,
                                       int* dev_status, dvlm_stream stream);
 
+/* Divergence-first commit of certificate-guided routing's FULL branch [Look
+ * Only When Needed, method step (3)]: as dvlm_topk_commit over the FULL
+ * pass's rows (full_prob, full_id), except that masked rows whose TEXT-ONLY
+ * top-1 text_id[r] differs from full_id[r] rank before every agreeing row;
+ * inside each group descending full_prob, lower row first.  Committed rows
+ * take full_id.  text_id [R]: device int32.  Same shapes, ownership and
+ * errors as dvlm_topk_commit.  (The certified-prefix branch needs no entry
+ * of its own: dvlm_topk_commit over the anchors' confidences and ids with k
+ * = the certificate length unmasks exactly that prefix.) */
+DVLM_API dvlm_status dvlm_divergence_first_commit(const float* full_prob, const int32_t* full_id,
+                                                  const int32_t* text_id, uint8_t* masked, int32_t* tokens, int R,
+                                                  int k, uint8_t* commit, int32_t* n_commit, int* dev_status,
+                                                  dvlm_stream stream);
+
 /* ------------------------------------------------------------------------
  * Speculative verify + longest-prefix accept + in-place KV truncation.
  *

@@ -106,6 +106,10 @@ def test_topk_host_validation(dvlm_lib):
     assert f(16, 16, 16, 16, 0, 1, None, None, None, None) == SHAPE
     assert f(16, 16, 16, 16, 129, 1, None, None, None, None) == SHAPE
     assert f(16, 16, 16, 16, 4, -1, None, None, None, None) == SHAPE
+    g = dv.lib().dvlm_divergence_first_commit
+    assert g(16, 16, None, 16, 16, 4, 1, None, None, None, None) == INVALID
+    assert g(16, 16, 16, 16, 16, 129, 1, None, None, None, None) == SHAPE
+    assert g(16, 16, 16, 16, 16, 4, -2, None, None, None, None) == SHAPE
 
 
 def _dims_model(**kw):

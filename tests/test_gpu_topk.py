@@ -63,3 +63,33 @@ def test_topk_commit_on_the_lm_head_outputs(cuda):
     conf = O.lm_head_conf(h.astype(np.float64), w.astype(np.float64))
     sure = [r for r in want if conf.p1[r] - conf.p2[r] >= 1e-3]
     assert all(int(tokens[r].item()) == int(conf.top1[r]) for r in sure)
+
+
+@pytest.mark.parametrize("R", [1, 7, 16, 128])
+@pytest.mark.parametrize("k", [0, 2, 5, 200])
+def test_divergence_first_commit_matches_oracle(cuda, R, k):
+    """FULL branch of certificate-guided routing: divergent rows first, each
+    group by FULL confidence; committed rows take the FULL ids."""
+    rng = np.random.default_rng(31 * R + k)
+    p1 = rng.choice(np.array([0.05, 0.3, 0.5, 0.9, 0.91, 1.0], dtype=np.float32), R)
+    masked = (rng.random(R) < 0.7).astype(np.uint8)
+    full = rng.integers(0, 4, R).astype(np.int32)
+    text = rng.integers(0, 4, R).astype(np.int32)
+    tokens0 = (np.arange(R) + 1000).astype(np.int32)
+    m_t, tok_t = torch.from_numpy(masked).to(cuda), torch.from_numpy(tokens0).to(cuda)
+    commit = torch.full((R,), 7, dtype=torch.uint8, device=cuda)
+    n = torch.full((1,), -1, dtype=torch.int32, device=cuda)
+    st = status(cuda)
+    dv.divergence_first_commit(torch.from_numpy(p1).to(cuda), torch.from_numpy(full).to(cuda),
+                               torch.from_numpy(text).to(cuda), m_t, tok_t, R=R, k=k, commit=commit, n_commit=n,
+                               status=st)
+    assert_ok(st)
+    want = sorted(O.divergence_first_order(full, p1.astype(np.float64), text, masked.astype(bool))[:k])
+    assert [r for r in range(R) if commit.cpu().numpy()[r]] == want
+    assert int(n.item()) == min(k, int(masked.sum()))
+    m_after, tok_after = m_t.cpu().numpy(), tok_t.cpu().numpy()
+    for r in range(R):
+        if r in want:
+            assert m_after[r] == 0 and tok_after[r] == full[r]
+        else:
+            assert m_after[r] == masked[r] and tok_after[r] == tokens0[r]
