@@ -70,3 +70,34 @@ def test_spec_case_plants_the_agreeing_prefix(b):
         assert np.array_equal(draft[i, :k[i]], top[i, :k[i]])
         assert np.all(draft[i, k[i]:] != top[i, k[i]:])
         assert draft[i].min() >= 0 and draft[i].max() < V
+
+
+@pytest.mark.parametrize("dims", [gen.TINY, gen.ModelDims(n_layers=2, hidden=256, n_q_heads=8, n_kv_heads=1,
+                                                           head_dim=128, inter=192, vocab=512, dtype="bf16")])
+def test_uploaded_layout_matches_the_abi_and_the_oracle_names(dims):
+    """The uploader stacks each layer's matrices as the C ABI documents
+    (wqkv rows: the Hq query heads, then the Hkv key heads, then the Hkv
+    value heads, D rows each; wo, wgate, wup, wdown [out, in]) from exactly
+    the draws the oracle uses under its own names; caches are K [layers,
+    batch, Hkv, Lmax, D] and V transposed [layers, batch, Hkv, D, Lmax]."""
+    import oracle as O
+    from dvlm_gen.device import DeviceModel, as_f64, kv_buffers
+    dm = DeviceModel(dims, 3, device="cpu")
+    w = O.weights_from_generator(gen, dims, 3)
+    qd, kd = dims.n_q_heads * dims.head_dim, dims.n_kv_heads * dims.head_dim
+    for l in range(dims.n_layers):
+        qkv = as_f64(dm.wqkv[l])
+        assert np.array_equal(qkv[:qd], w[f"{l}.wq"])
+        assert np.array_equal(qkv[qd:qd + kd], w[f"{l}.wk"])
+        assert np.array_equal(qkv[qd + kd:], w[f"{l}.wv"])
+        for name, t in (("wo", dm.wo), ("wg", dm.wgate), ("wu", dm.wup), ("wd", dm.wdown)):
+            assert np.array_equal(as_f64(t[l]), w[f"{l}.{name}"]), name
+    assert np.array_equal(as_f64(dm.embed), w["embed"]) and np.array_equal(as_f64(dm.lm_head), w["lm_head"])
+    k, v = kv_buffers(dims, 40, device="cpu", n_batch=2)
+    assert k.shape == (dims.n_layers, 2, dims.n_kv_heads, 40, dims.head_dim)
+    assert v.shape == (dims.n_layers, 2, dims.n_kv_heads, dims.head_dim, 40)
+    m = dm.c_model()
+    assert (m.n_layers, m.hidden, m.n_q_heads, m.n_kv_heads, m.head_dim, m.inter, m.vocab, m.mask_id) == \
+        (dims.n_layers, dims.hidden, dims.n_q_heads, dims.n_kv_heads, dims.head_dim, dims.inter, dims.vocab,
+         dims.vocab - 1)
+    assert m.wqkv == dm.wqkv.data_ptr() and m.lm_head == dm.lm_head.data_ptr()
