@@ -143,3 +143,14 @@ def test_engine_host_validation(dvlm_lib):
     assert L.dvlm_engine_destroy(None) == INVALID
     assert L.dvlm_prefill(None, None, 0, None, 0, None) == INVALID
     assert L.dvlm_decode_block(None, None, None, None, None, None) == INVALID
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without the built library every entry point raises."""
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libdvlm.so"))
+    import pytest
+    with pytest.raises(RuntimeError, match="missing"):
+        binding.lib()
+    with pytest.raises(RuntimeError, match="missing"):
+        dv.topk_commit(None, None, None, None, R=1, k=1)
