@@ -35,7 +35,10 @@ its reason in the repository's design notes):
   fp8       (next step, not on the bf16 path) W8A8 in E4M3, finite variant,
             round to nearest even, saturating at 448; one scale per weight
             output channel and per activation token (amax / 448);
-            SmoothQuant factors with alpha = 0.5.
+            SmoothQuant factors with alpha = 0.5.  The fp8 model (next
+            step) runs the four projections of every layer W8A8 and keeps
+            the LM head, norms, RoPE, attention and storage points as in
+            the bf16 model.
   norms     RMSNorm gain 1, eps 1e-6, no biases; RoPE rotate-half, base 1e4.
   lown      (next step) TEXT-ONLY = the vision cache slots hidden from the
             block's queries, position ids unchanged; each block opens with a
@@ -387,12 +390,19 @@ class OracleModel:
     activation)."""
 
     def __init__(self, dims: Dims, weights=None, weights_fn=None, bf16: bool = True,
-                 Lmax: int = 4096):
+                 Lmax: int = 4096, fp8: bool = False, smooth: Optional[Dict[str, np.ndarray]] = None):
         self.d = dims
         self._w = weights
         self._wfn = weights_fn
         self.bf16 = bf16
         self.Lmax = Lmax
+        # W8A8 decoder projections (next step of the weight stream): the four
+        # projections of every layer go through fp8_linear on the activations
+        # they consume; the LM head, norms, RoPE, attention and the bf16
+        # storage points stay as in the bf16 model.  `smooth` maps a weight
+        # name to its SmoothQuant factors m (x / m and W * m are quantised).
+        self.fp8 = fp8
+        self.smooth = smooth or {}
         self.K = [np.zeros((dims.n_kv_heads, Lmax, dims.head_dim)) for _ in range(dims.n_layers)]
         self.V = [np.zeros((dims.n_kv_heads, Lmax, dims.head_dim)) for _ in range(dims.n_layers)]
         self.L = 0
@@ -405,6 +415,16 @@ class OracleModel:
     def rnd(self, x: np.ndarray) -> np.ndarray:
         return bf16_round(x) if self.bf16 else x
 
+    def lin(self, a: np.ndarray, name: str) -> np.ndarray:
+        """a W^T for the decoder matrix `name` ([out, in]); W8A8 in fp8 mode."""
+        W = self.w(name)
+        if not self.fp8:
+            return a @ W.T
+        m = self.smooth.get(name)
+        if m is not None:
+            return fp8_linear(a / m[None, :], W * m[None, :])
+        return fp8_linear(a, W)
+
     # -- one decoder layer ---------------------------------------------------
     def layer(self, l: int, x: np.ndarray, L: int, n_clean: int, write_kv: bool = True, hide: int = 0) -> np.ndarray:
         d = self.d
@@ -412,9 +432,9 @@ class OracleModel:
         D, Hq, Hkv = d.head_dim, d.n_q_heads, d.n_kv_heads
         pos = np.arange(L, L + n)
         h = x * rms_factor(x, d.eps)
-        q = (h @ self.w(f"{l}.wq").T).reshape(n, Hq, D)
-        k = (h @ self.w(f"{l}.wk").T).reshape(n, Hkv, D)
-        v = (h @ self.w(f"{l}.wv").T).reshape(n, Hkv, D)
+        q = self.lin(h, f"{l}.wq").reshape(n, Hq, D)
+        k = self.lin(h, f"{l}.wk").reshape(n, Hkv, D)
+        v = self.lin(h, f"{l}.wv").reshape(n, Hkv, D)
         q = self.rnd(rope(q, pos, d.rope_base))
         k = self.rnd(rope(k, pos, d.rope_base))
         v = self.rnd(v)
@@ -423,12 +443,12 @@ class OracleModel:
             self.V[l][:, L:L + n] = v.transpose(1, 0, 2)
         a = block_attention(q, self.K[l], self.V[l], L, n_clean, 1.0 / math.sqrt(D), hide)
         a = self.rnd(a).reshape(n, Hq * D)
-        x = self.rnd(x + a @ self.w(f"{l}.wo").T)
+        x = self.rnd(x + self.lin(a, f"{l}.wo"))
         h2 = x * rms_factor(x, d.eps)
-        g = h2 @ self.w(f"{l}.wg").T
-        u = h2 @ self.w(f"{l}.wu").T
+        g = self.lin(h2, f"{l}.wg")
+        u = self.lin(h2, f"{l}.wu")
         act = self.rnd(silu(g) * u)
-        x = self.rnd(x + act @ self.w(f"{l}.wd").T)
+        x = self.rnd(x + self.lin(act, f"{l}.wd"))
         return x
 
     def embed(self, ids: Sequence[int]) -> np.ndarray:
@@ -676,9 +696,9 @@ def forward_quadratic(model: OracleModel, draft: Sequence[int], L: int) -> np.nd
     n = x.shape[0]
     for l in range(d.n_layers):
         h = x * rms_factor(x, d.eps)
-        q = (h @ model.w(f"{l}.wq").T).reshape(n, Hq, D)
-        k = (h @ model.w(f"{l}.wk").T).reshape(n, Hkv, D)
-        v = (h @ model.w(f"{l}.wv").T).reshape(n, Hkv, D)
+        q = model.lin(h, f"{l}.wq").reshape(n, Hq, D)
+        k = model.lin(h, f"{l}.wk").reshape(n, Hkv, D)
+        v = model.lin(h, f"{l}.wv").reshape(n, Hkv, D)
         q = model.rnd(rope(q, pos, d.rope_base))
         k = model.rnd(rope(k, pos, d.rope_base))
         v = model.rnd(v)
@@ -688,12 +708,12 @@ def forward_quadratic(model: OracleModel, draft: Sequence[int], L: int) -> np.nd
                                 k[B:].reshape(B, B, Hkv, D), v[B:].reshape(B, B, Hkv, D),
                                 1.0 / math.sqrt(D))
         a = model.rnd(a).reshape(n, Hq * D)
-        x = model.rnd(x + a @ model.w(f"{l}.wo").T)
+        x = model.rnd(x + model.lin(a, f"{l}.wo"))
         h2 = x * rms_factor(x, d.eps)
-        g = h2 @ model.w(f"{l}.wg").T
-        u = h2 @ model.w(f"{l}.wu").T
+        g = model.lin(h2, f"{l}.wg")
+        u = model.lin(h2, f"{l}.wu")
         act = model.rnd(silu(g) * u)
-        x = model.rnd(x + act @ model.w(f"{l}.wd").T)
+        x = model.rnd(x + model.lin(act, f"{l}.wd"))
     return x
 
 
