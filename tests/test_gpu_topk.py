@@ -93,3 +93,55 @@ def test_divergence_first_commit_matches_oracle(cuda, R, k):
             assert m_after[r] == 0 and tok_after[r] == full[r]
         else:
             assert m_after[r] == masked[r] and tok_after[r] == tokens0[r]
+
+
+def test_routing_step_decisions_on_the_lm_head_outputs(cuda):
+    """One step of certificate-guided routing on device-resident outputs:
+    the FULL rows' LM head gives the anchors, the TEXT-ONLY rows' LM head
+    (with those anchors and the mask) gives the certified length; the accept
+    branch (top-k over the anchors with k = that length) and the FULL branch
+    (divergent-first, k = 3) are then applied, each to its own copy of the
+    state.  Every decision equals the oracle's routing functions applied to
+    the same kernel outputs (the LM head's own parity is tested elsewhere)."""
+    import dvlm_gen as gen
+    from gpu_util import ws_tensor
+    R, H, V, k = 16, 256, 2048, 3
+    (h1_t, _), (w_t, _), (h2_t, _) = gen.lmhead_case(11, R, H, V)
+    wd = w_t.to(cuda)
+    ws = ws_tensor(dv.lmhead_workspace_size(R, V, H, dv.DVLM_BF16), cuda)
+    st = status(cuda)
+    masked_h = (np.random.default_rng(12).random(R) < 0.75).astype(np.uint8)
+    masked = torch.from_numpy(masked_h).to(cuda)
+
+    def head(h, anchors=None):
+        top = torch.zeros(R, dtype=torch.int32, device=cuda)
+        p1 = torch.zeros(R, dtype=torch.float32, device=cuda)
+        kw = {}
+        if anchors is not None:
+            kw = dict(masked=masked, anchor_id=anchors[0], anchor_conf=anchors[1],
+                      cert_len=torch.full((1,), -1, dtype=torch.int32, device=cuda))
+        dv.lmhead_conf_commit(h.to(cuda), wd, R=R, H=H, V=V, dtype=dv.DVLM_BF16, threshold=0.9, top1_id=top,
+                              top1_prob=p1, workspace=ws, status=st, **kw)
+        return top, p1, kw.get("cert_len")
+
+    a_id, a_p, _ = head(h1_t)
+    t_id, t_p, cert = head(h2_t, anchors=(a_id, a_p))
+    assert_ok(st)
+    assert np.array_equal(masked.cpu().numpy(), masked_h)          # the TEXT-ONLY pass commits nothing
+    aid, ap, tid = a_id.cpu().numpy(), a_p.cpu().numpy().astype(np.float64), t_id.cpu().numpy()
+    n = int(cert.item())
+    assert n == O.certificate_scan(aid, ap, tid, masked_h.astype(bool))
+    tokens0 = torch.arange(R, dtype=torch.int32, device=cuda) + 1000
+
+    m1, tok1 = masked.clone(), tokens0.clone()
+    dv.topk_commit(a_p, a_id, m1, tok1, R=R, k=n, status=st)
+    m2, tok2 = masked.clone(), tokens0.clone()
+    dv.divergence_first_commit(a_p, a_id, t_id, m2, tok2, R=R, k=k, status=st)
+    assert_ok(st)
+    accept = sorted(O.certificate_order(ap, masked_h.astype(bool))[:n])
+    full = sorted(O.divergence_first_order(aid, ap, tid, masked_h.astype(bool))[:k])
+    for m, tok, want in ((m1, tok1, accept), (m2, tok2, full)):
+        m, tok = m.cpu().numpy(), tok.cpu().numpy()
+        assert [r for r in range(R) if masked_h[r] and not m[r]] == want
+        assert all(tok[r] == aid[r] for r in want)
+        assert all(tok[r] == 1000 + r for r in range(R) if r not in want)

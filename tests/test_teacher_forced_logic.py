@@ -182,3 +182,44 @@ def test_text_only_check_catches_unhidden_vision_slots(standin, monkeypatch):
     monkeypatch.setattr(TA, "assert_ok", lambda st: None)
     with pytest.raises(AssertionError):
         TA.test_text_only_pass_through_offset_cache_views(standin, 64, 300, 16, 0, 1)
+
+
+def _lmhead_full(h, w, *, R, H, V, dtype, masked=None, tokens=None, threshold=0.9, top1_id=None, top1_prob=None,
+                 anchor_id=None, anchor_conf=None, cert_len=None, workspace=None, status=None, **kw):
+    """Fused LM head stand-in with the header's contract: outputs, in-place
+    commit only when tokens is given, certificate over the rows masked on
+    entry."""
+    x = h[:R].float().numpy().astype(np.float64)
+    c = O.lm_head_conf(x, w.float().numpy().astype(np.float64))
+    p1 = c.p1.astype(np.float32)
+    if top1_id is not None:
+        top1_id[:R] = torch.from_numpy(c.top1.astype(np.int32))
+    if top1_prob is not None:
+        top1_prob[:R] = torch.from_numpy(p1)
+    part = masked.numpy().astype(bool) if masked is not None else np.ones(R, dtype=bool)
+    if cert_len is not None:
+        cert_len[0] = O.certificate_scan(anchor_id.numpy(), anchor_conf.numpy().astype(np.float64), c.top1, part)
+    if tokens is not None:
+        for r in O.threshold_commit(p1.astype(np.float64), part, threshold):
+            tokens[r], masked[r] = int(c.top1[r]), 0
+
+
+def _commit_standin(order_fn):
+    def run(p, ids, *rest, R, k, commit=None, n_commit=None, status=None, **kw):
+        other = rest[0] if len(rest) == 3 else None
+        masked, tokens = rest[-2], rest[-1]
+        part = masked.numpy().astype(bool)
+        rows = order_fn(p.numpy().astype(np.float64), ids.numpy(), None if other is None else other.numpy(), part, k)
+        for r in rows:
+            tokens[r], masked[r] = int(ids[r]), 0
+    return run
+
+
+def test_routing_step_check_logic(standin, monkeypatch):
+    import test_gpu_topk as TK
+    monkeypatch.setattr(dv, "lmhead_conf_commit", _lmhead_full)
+    monkeypatch.setattr(dv, "topk_commit", _commit_standin(lambda p, ids, other, part, k: O.topk_commit(p, part, k)))
+    monkeypatch.setattr(dv, "divergence_first_commit", _commit_standin(
+        lambda p, ids, other, part, k: O.divergence_first_order(ids, p, other, part)[:k]))
+    monkeypatch.setattr(TK, "assert_ok", lambda st: None)
+    TK.test_routing_step_decisions_on_the_lm_head_outputs(standin)
