@@ -109,6 +109,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_engine_set_position": (_i, [_vp, ctypes.c_int32, ctypes.c_int32, _vp]),
         "dvlm_engine_check": (_i, [_vp, _vp]),
         "dvlm_forward": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+        "dvlm_forward_text_only": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
         "dvlm_engine_set_option": (_i, [_vp, ctypes.c_char_p, _i]),
         "dvlm_engine_get_option": (_i, [_vp, ctypes.c_char_p]),
         "dvlm_selftest_wait_timeout": (_i, [ctypes.c_longlong, _vp, _vp, _vp]),
@@ -306,6 +307,13 @@ class Engine:
                                           cnt, stream_handle(stream)),
                "dvlm_profile_forward")
         return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(self.KERNEL_KINDS)}
+
+    def forward_text_only(self, n_rows: int, n_hidden: int, *, tokens, masked=None, x_out=None,
+                          stream=None) -> None:
+        """Noisy pass with cache slots 0..n_hidden-1 hidden from attention (dvlm_forward_text_only)."""
+        _check(lib().dvlm_forward_text_only(self.h, ptr(tokens), ptr(masked), n_rows, n_hidden, ptr(x_out),
+                                            stream_handle(stream)),
+               "dvlm_forward_text_only")
 
     def forward(self, n_rows: int, n_clean: int, n_layers: int, *, x_in=None, tokens=None, masked=None,
                 first_layer: int = 0, advance: bool = False, x_out=None, stream=None) -> None:

@@ -552,6 +552,30 @@ dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_t* tokens
   return cuda_status(engine_forward(e, f, s));
 }
 
+dvlm_status dvlm_forward_text_only(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked, int n_rows,
+                                   int n_hidden, void* x_out, dvlm_stream stream) {
+  if (!e || !tokens) return DVLM_ERR_INVALID_ARG;
+  if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+  if (n_rows < 1 || n_rows > kNT || n_hidden < 0 || n_hidden % 8) return DVLM_ERR_SHAPE;
+  if (x_out && !al16(x_out)) return DVLM_ERR_INVALID_ARG;
+  cudaStream_t s = cs(stream);
+  int32_t L = 0;
+  if (cudaMemcpyAsync(&L, e->d_len, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DVLM_ERR_CUDA;
+  if (L + n_rows > e->Lmax) return DVLM_ERR_CACHE_OVERFLOW;
+  if (n_hidden > L) return DVLM_ERR_SHAPE;
+  FwdSpec f;
+  f.tokens = tokens;
+  f.masked = masked;
+  f.n_rows = n_rows;
+  f.n_clean = 0;
+  f.x_out = x_out;
+  f.hide = n_hidden;
+  f.L_host = L;
+  return cuda_status(engine_forward(e, f, s));
+}
+
 dvlm_status dvlm_profile_forward(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked, int n_rows,
                                  int n_clean, int with_lm_head, float* ms_out, int* counts_out, dvlm_stream stream) {
   if (!e || !tokens || !ms_out || !counts_out) return DVLM_ERR_INVALID_ARG;

@@ -143,6 +143,22 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   KernelTimer* tm = f.timer;
   auto T0 = [&](int k) { if (tm) tm->begin(k); };
   auto T1 = [&](int k) { if (tm) tm->end(k); };
+  // TEXT-ONLY pass [Look Only When Needed, method step (2): the vision rows
+  // removed, position ids kept]: attention reads the cache from slot f.hide
+  // on.  The K and V^T maps start f.hide slots in and end where the cache
+  // allocation ends (outer rows of K, inner keys of V^T shortened by f.hide),
+  // so a 64-key box past the last valid key is zero-filled instead of read
+  // beyond the allocation; the length is the host-read L minus f.hide.  The
+  // QKV epilogue still writes K/V at the absolute slots.
+  CUtensorMap tm_k_text, tm_v_text;
+  if (f.hide > 0) {
+    const uint64_t k_rows = static_cast<uint64_t>(m.n_layers) * Hkv * e->Lmax;
+    bool ok = make_tmap_2d(&tm_k_text, static_cast<const bf16*>(e->kc) + static_cast<size_t>(f.hide) * D, D,
+                           k_rows - f.hide, D * 2, 64, 64);
+    ok &= make_tmap_2d(&tm_v_text, static_cast<const bf16*>(e->vc) + f.hide, e->Lmax - f.hide,
+                       static_cast<uint64_t>(m.n_layers) * Hkv * D, static_cast<uint64_t>(e->Lmax) * 2, 64, 128);
+    if (!ok) return cudaErrorInvalidValue;
+  }
   T0(K_EMBED);
   DVLM_CK(launch_embed_bf16(static_cast<const bf16*>(m.embed), static_cast<const bf16*>(f.rows_in), f.n_src,
                             f.tokens, f.masked, m.mask_id, f.n_rows, H, m.vocab, x, e->ssq, kNT, e->d_status, pdl,
@@ -195,7 +211,13 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     aa.out = static_cast<bf16*>(e->attn_o);
     aa.status = e->d_status;
     T0(K_ATTN);
-    DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s, e->attn_cs));
+    if (f.hide > 0) {
+      aa.d_len = nullptr;
+      aa.L_static = f.L_host - f.hide;
+      DVLM_CK(launch_attn_bf16(e->tm_q, tm_k_text, tm_v_text, aa, pdl, s, e->attn_cs));
+    } else {
+      DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s, e->attn_cs));
+    }
     T1(K_ATTN);
     ea.epi = EPI_RESID;
     ea.resid = x;

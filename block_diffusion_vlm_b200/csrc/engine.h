@@ -45,6 +45,11 @@ struct FwdSpec {
   LmArgs lma{};              // LM-head outputs (scratch pointers filled by the engine)
   void* x_out = nullptr;     // copy of the residual stream (test hook)
   KernelTimer* timer = nullptr;
+  // TEXT-ONLY pass of certificate-guided routing: cache slots 0..hide-1 (the
+  // vision rows) are hidden from attention, positions unchanged; L_host is
+  // the cache length, read by the caller (eager forwards only).
+  int hide = 0;
+  int L_host = 0;
 };
 
 // Kernel launches of one forward pass over n_layers layers.

@@ -357,6 +357,19 @@ DVLM_API int dvlm_engine_get_option(dvlm_engine* e, const char* name);
 DVLM_API dvlm_status dvlm_selftest_wait_timeout(long long budget_cycles, int* dev_status, int* gave_up,
                                                dvlm_stream stream);
 
+/* TEXT-ONLY noisy pass of certificate-guided routing [Look Only When Needed,
+ * method step (2): the vision rows removed, position ids kept]: one forward
+ * of n_rows noisy rows (tokens, masked as in dvlm_forward) at slots L..L+n-1
+ * over all layers in which attention does not see cache slots
+ * 0..n_hidden-1 (the vision rows at the front of the cache); RoPE positions
+ * and the K/V written for the rows stay absolute.  L is not advanced.
+ * x_out [n_rows, H] (bf16, may be NULL) receives the final residual stream.
+ * bf16 engines only (DVLM_ERR_UNSUPPORTED otherwise); 0 <= n_hidden <= L,
+ * n_hidden % 8 == 0 (DVLM_ERR_SHAPE otherwise).  Reads L to the host
+ * (synchronises the stream) and launches eagerly. */
+DVLM_API dvlm_status dvlm_forward_text_only(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
+                                           int n_rows, int n_hidden, void* x_out, dvlm_stream stream);
+
 /* Profiling hook: one forward pass like dvlm_forward over all layers (L is
  * not advanced), launched eagerly with a CUDA event pair around every kernel
  * on `stream`.  ms_out[7] receives the device time per kernel class summed

@@ -766,7 +766,7 @@ class LownTrace:
 
 
 def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int, max_new: int,
-                shift: int = 1) -> LownTrace:
+                shift: int = 1, on_pass=None, on_block=None) -> LownTrace:
     """Certificate-guided visual routing [LOWN method steps (1)-(3)] inside
     block decoding.  Per block (first token = the AR seed, the rest [MASK]):
     a FULL noisy forward sets the anchors (top-1 id and confidence of every
@@ -778,7 +778,12 @@ def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int,
     min(k, masked) positions, all of it is unmasked with the anchor ids;
     otherwise a FULL forward refreshes the anchors and min(k, masked)
     positions are unmasked with the FULL ids, divergent positions (TEXT-ONLY
-    top-1 != FULL top-1) first.  A causal pass then appends the block."""
+    top-1 != FULL top-1) first.  A causal pass then appends the block.
+
+    Optional observers (they do not change the trajectory): on_pass(kind, L,
+    toks, p1, top1) after each noisy pass ("full" or "text"), with the block
+    tokens it ran on and its scores per block position; on_block(L, toks)
+    before each block's causal pass."""
     d = model.d
     tr = LownTrace(tokens=[])
     seed = seed_token
@@ -803,8 +808,10 @@ def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int,
             kk = min(k, sum(masked))
             if anchor_id is not None:
                 x = model.forward(model.embed(toks), L, n_clean=0, hide=n_vis)
-                _, text_top = scores(model.logits_conf(x), prev_conf)
+                text_p1, text_top = scores(model.logits_conf(x), prev_conf)
                 tr.n_text += 1
+                if on_pass is not None:
+                    on_pass("text", L, list(toks), text_p1.copy(), text_top.copy())
                 order = certificate_order(anchor_conf, masked)
                 n = certificate_scan(anchor_id, anchor_conf, text_top, masked)
                 if n >= kk:
@@ -816,6 +823,8 @@ def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int,
             x = model.forward(model.embed(toks), L, n_clean=0)
             full_p1, full_top = scores(model.logits_conf(x), prev_conf)
             tr.n_full += 1
+            if on_pass is not None:
+                on_pass("full", L, list(toks), full_p1.copy(), full_top.copy())
             anchor_id, anchor_conf = full_top.copy(), full_p1.copy()
             if text_top is None:
                 order = certificate_order(full_p1, masked)
@@ -825,6 +834,8 @@ def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int,
                 toks[j], masked[j] = int(full_top[j]), False
             tr.accepted.append(kk)
             tr.text_branch.append(False)
+        if on_block is not None:
+            on_block(L, list(toks))
         x = model.forward(model.embed(toks), L, n_clean=B)
         model.L = L + B
         c = model.logits_conf(x)

@@ -143,6 +143,7 @@ def test_engine_host_validation(dvlm_lib):
     assert L.dvlm_engine_destroy(None) == INVALID
     assert L.dvlm_prefill(None, None, 0, None, 0, None) == INVALID
     assert L.dvlm_decode_block(None, None, None, None, None, None) == INVALID
+    assert L.dvlm_forward_text_only(None, 4096, None, 16, 32, None, None) == INVALID
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

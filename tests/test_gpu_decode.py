@@ -243,3 +243,53 @@ def test_bf16_reduced_model_spec_teacher_forced(cuda, seed):
     assert counts["rounds"] == len(tr.accept_lens)
     assert counts["draft"] > 0 and counts["verify"] > 0
     s.eng.close()
+
+
+def test_bf16_reduced_model_routing_teacher_forced(cuda):
+    """Certificate-guided routing (B=16, k=2, 32 tokens; the 32 vision rows
+    hidden in TEXT-ONLY passes) of the reduced bf16 model, per pass and
+    teacher-forced: each FULL pass of the oracle's trajectory replayed with
+    the engine's forward, each TEXT-ONLY pass with its TEXT-ONLY forward,
+    then the fused LM head; top-1 ids compared wherever the oracle's margin
+    is at least DELTA, p1 within DELTA; finished blocks appended causally."""
+    s = Setup(SMALL_BF16, 1, cuda, 32, 16, 0)
+    eng, d, dev = s.eng, SMALL_BF16, cuda
+    B, k, n_vis = 16, 2, 32
+    eng.prefill(s.vis_t.to(dev), n_vis, torch.from_numpy(s.ids).to(dev), 16)
+    _, seed_gpu = eng.position()
+    lw = ws_tensor(dv.lmhead_workspace_size(B, d.vocab, d.hidden, dv.DVLM_BF16), dev)
+    x = torch.zeros((B, d.hidden), dtype=torch.bfloat16, device=dev)
+    counts = {"full": 0, "text": 0, "top1": 0}
+
+    def on_pass(kind, L, toks, p1o, topo):
+        assert eng.position()[0] == L
+        t = torch.tensor(toks, dtype=torch.int32, device=dev)
+        if kind == "full":
+            eng.forward(B, 0, d.n_layers, tokens=t, x_out=x)
+        else:
+            eng.forward_text_only(B, n_vis, tokens=t, x_out=x)
+        top = torch.zeros(B, dtype=torch.int32, device=dev)
+        p1 = torch.zeros(B, dtype=torch.float32, device=dev)
+        st = status(dev)
+        dv.lmhead_conf_commit(x, s.dm.lm_head, R=B, H=d.hidden, V=d.vocab, dtype=dv.DVLM_BF16, apply_rmsnorm=1,
+                              top1_id=top, top1_prob=p1, workspace=lw, status=st)
+        assert_ok(st)
+        p1g, topg = p1.cpu().numpy(), top.cpu().numpy()
+        counts[kind] += 1
+        for j in range(1, B):  # position j is scored by row j - 1
+            assert abs(p1g[j - 1] - p1o[j]) <= DELTA, (kind, j)
+            if p1o[j] >= 0.5 + DELTA / 2:          # a p1 above 1/2 leaves the runner-up below 1 - p1
+                assert topg[j - 1] == topo[j], (kind, j)
+                counts["top1"] += 1
+
+    def on_block(L, toks):
+        eng.forward(B, B, d.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=dev), advance=True)
+
+    m = O.OracleModel(s.od, weights=s.w, bf16=True, Lmax=s.Lmax)
+    seed_o = O.prefill(m, s.vis.astype(np.float64), s.ids)
+    assert seed_o == seed_gpu
+    tr = O.decode_lown(m, seed_o, B, k, n_vis=n_vis, max_new=32, on_pass=on_pass, on_block=on_block)
+    eng.check()
+    assert counts["full"] == tr.n_full and counts["text"] == tr.n_text
+    assert counts["text"] > 0 and counts["top1"] > 0
+    s.eng.close()

@@ -694,6 +694,25 @@ def test_lown_routing_on_a_scripted_model():
     assert tr.tokens == [7, 11, 32, 13, 34, 35]
 
 
+def test_lown_observers_do_not_change_the_trajectory():
+    """The per-pass observers of the teacher-forced GPU routing check see
+    every FULL and TEXT-ONLY pass (tokens before the pass's unmasking) and
+    every block, and leave the trajectory unchanged."""
+    gd, d, w, vis, ids = _tiny()
+    B = 4
+    m, s0 = _fresh(d, w, False, vis, ids)
+    plain = O.decode_lown(m, s0, B, 1, n_vis=len(vis), max_new=3 * B)
+    passes, blocks = [], []
+    m, s0 = _fresh(d, w, False, vis, ids)
+    obs = O.decode_lown(m, s0, B, 1, n_vis=len(vis), max_new=3 * B,
+                        on_pass=lambda kind, L, toks, p1, top: passes.append((kind, L, toks)),
+                        on_block=lambda L, toks: blocks.append((L, toks)))
+    assert obs.tokens == plain.tokens and obs.accepted == plain.accepted and obs.text_branch == plain.text_branch
+    assert [p[0] for p in passes].count("full") == plain.n_full and [p[0] for p in passes].count("text") == plain.n_text
+    assert [b[1] for b in blocks] == [plain.tokens[i * B:(i + 1) * B] for i in range(3)]
+    assert all(p[2][0] == blocks[[b[0] for b in blocks].index(p[1])][1][0] for p in passes)   # seed row fixed
+
+
 def test_lown_planted_mistakes_are_caught(monkeypatch):
     import oracle.dvlm_oracle as OM
     real_div = OM.divergence_first_order

@@ -68,6 +68,12 @@ class _Engine:
         if advance:
             self.m.L += n_rows
 
+    def forward_text_only(self, n_rows, n_hidden, *, tokens=None, x_out=None, **kw):
+        assert tokens is not None and n_hidden % 8 == 0 and n_hidden <= self.m.L
+        x = self.m.forward(self.m.embed(tokens.numpy()), self.m.L, n_clean=0, hide=n_hidden)
+        if x_out is not None:
+            x_out[:n_rows] = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+
     def check(self, stream=None):
         pass
 
@@ -223,3 +229,14 @@ def test_routing_step_check_logic(standin, monkeypatch):
         lambda p, ids, other, part, k: O.divergence_first_order(ids, p, other, part)[:k]))
     monkeypatch.setattr(TK, "assert_ok", lambda st: None)
     TK.test_routing_step_decisions_on_the_lm_head_outputs(standin)
+
+
+def test_routing_decode_check_logic(standin):
+    T.test_bf16_reduced_model_routing_teacher_forced(standin)
+
+
+def test_routing_decode_check_catches_a_text_pass_that_sees_the_vision_rows(standin, monkeypatch):
+    monkeypatch.setattr(_Engine, "forward_text_only",
+                        lambda self, n_rows, n_hidden, **kw: _Engine.forward(self, n_rows, 0, self.d.n_layers, **kw))
+    with pytest.raises(AssertionError):
+        T.test_bf16_reduced_model_routing_teacher_forced(standin)
