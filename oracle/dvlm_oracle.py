@@ -755,6 +755,10 @@ def decode_spec_quadratic(model: OracleModel, seed_token: int, B: int, max_new: 
     return tr
 
 
+# ----------------------------------------------------------------------------
+# Certificate-guided visual routing inside block decoding  [LOWN method
+# steps (1)-(3)]
+# ----------------------------------------------------------------------------
 @dataclasses.dataclass
 class LownTrace:
     tokens: List[int]
