@@ -155,3 +155,12 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         binding.lib()
     with pytest.raises(RuntimeError, match="missing"):
         dv.topk_commit(None, None, None, None, R=1, k=1)
+
+
+def test_binding_declares_every_header_entry_point():
+    """Every entry point of include/dvlm.h has a ctypes signature in the
+    binding (so no call goes through ctypes' int defaults)."""
+    import inspect
+    import re
+    src = inspect.getsource(binding._declare)
+    assert set(re.findall(r'"(dvlm_\w+)"', src)) == set(dv.declared_symbols())
