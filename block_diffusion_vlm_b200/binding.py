@@ -115,6 +115,8 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_selftest_wait_timeout": (_i, [ctypes.c_longlong, _vp, _vp, _vp]),
         "dvlm_profile_forward": (_i, [_vp, _vp, _vp, _i, _i, _i, ctypes.POINTER(ctypes.c_float),
                                       ctypes.POINTER(_i), _vp]),
+        "dvlm_engine_trace_record_bytes": (_sz, [ctypes.POINTER(Model)]),
+        "dvlm_engine_set_trace": (_i, [_vp, _vp, _sz, _vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -231,6 +233,11 @@ def engine_workspace_size(model: Model, Lmax: int, max_block: int, max_ctx: int)
     return int(lib().dvlm_engine_workspace_size(ctypes.byref(model), Lmax, max_block, max_ctx))
 
 
+def engine_trace_record_bytes(model: Model) -> int:
+    """Bytes of one forward-trace record (dvlm_engine_trace_record_bytes)."""
+    return int(lib().dvlm_engine_trace_record_bytes(ctypes.byref(model)))
+
+
 class Engine:
     """Decode engine over caller-owned device buffers (see dvlm_engine_create)."""
 
@@ -295,6 +302,13 @@ class Engine:
 
     def get_option(self, name: str) -> int:
         return int(lib().dvlm_engine_get_option(self.h, name.encode()))
+
+    def set_trace(self, buf, count) -> None:
+        """Record every decode-driver forward into buf (device tensor), counting
+        records in count (device int32); buf=None clears (dvlm_engine_set_trace)."""
+        nbytes = buf.numel() * buf.element_size() if buf is not None else 0
+        _check(lib().dvlm_engine_set_trace(self.h, ptr(buf), nbytes, ptr(count) if buf is not None else None),
+               "dvlm_engine_set_trace")
 
     KERNEL_KINDS = ("embed", "qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head")
 

@@ -22,6 +22,10 @@ void engine_plan(dvlm_engine* e);
 cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* counts, cudaStream_t s);
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v);
 int engine_get_option(dvlm_engine* e, const char* name);
+void engine_set_trace(dvlm_engine* e, void* buf, int cap, int32_t* cnt);
+bool prefill_gemm_supported(const dvlm_engine* e);
+cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, const int32_t* ids, int n_ids,
+                                cudaStream_t s);
 cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, const int32_t* other_ids, uint8_t* masked,
                                int32_t* tokens, int R, int k, uint8_t* commit, int32_t* n_commit, cudaStream_t s);
 }  // namespace dvlm
@@ -373,8 +377,10 @@ dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_vision, const
   if (n_vision + n_ids > e->Lmax) return DVLM_ERR_CACHE_OVERFLOW;
   if (e->bf16 && n_vision > 0 && !al16(vision)) return DVLM_ERR_INVALID_ARG;
   cudaStream_t s = cs(stream);
-  if (cudaMemsetAsync(e->d_len, 0, 4, s) != cudaSuccess) return DVLM_ERR_CUDA;
   const int n_ctx = n_vision + n_ids;
+  if (e->prefill_gemm && n_ctx <= e->max_ctx && prefill_gemm_supported(e))
+    return cuda_status(engine_prefill_gemm(e, vision, n_vision, ids, n_ids, s));
+  if (cudaMemsetAsync(e->d_len, 0, 4, s) != cudaSuccess) return DVLM_ERR_CUDA;
   const size_t es = e->bf16 ? 2 : 4;
   for (int c0 = 0; c0 < n_ctx; c0 += kNT) {
     const int n = std::min(kNT, n_ctx - c0);
@@ -609,6 +615,25 @@ dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value) 
   if (!e || !name) return DVLM_ERR_INVALID_ARG;
   if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
   return engine_set_option(e, name, value);
+}
+
+size_t dvlm_engine_trace_record_bytes(const dvlm_model* m) {
+  if (!model_ok(m)) return 0;
+  return trace_record_bytes(m->hidden, m->dtype == DVLM_BF16);
+}
+
+dvlm_status dvlm_engine_set_trace(dvlm_engine* e, void* buf, size_t bytes, int32_t* count) {
+  if (!e) return DVLM_ERR_INVALID_ARG;
+  if (!buf) {
+    engine_set_trace(e, nullptr, 0, nullptr);
+    return DVLM_OK;
+  }
+  if (!count || !al16(buf) || !al16(count)) return DVLM_ERR_INVALID_ARG;
+  const size_t rb = trace_record_bytes(e->m.hidden, e->bf16);
+  if (bytes < rb) return DVLM_ERR_WORKSPACE;
+  const size_t cap = bytes / rb;
+  engine_set_trace(e, buf, static_cast<int>(cap > 1000000 ? 1000000 : cap), count);
+  return DVLM_OK;
 }
 
 int dvlm_engine_get_option(dvlm_engine* e, const char* name) {

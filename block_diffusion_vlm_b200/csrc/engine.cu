@@ -30,6 +30,46 @@ __global__ void advance_kernel(int32_t* d_len, int n) {
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Forward trace (test hook): the block state before a forward ...
+__global__ void trace_begin_kernel(uint8_t* buf, size_t rec_bytes, int cap, const int32_t* cnt, int kind,
+                                   const int32_t* d_len, int n_rows, int n_clean, int R, const int32_t* tokens,
+                                   const uint8_t* masked) {
+  const int idx = *cnt;
+  if (idx >= cap) return;
+  int32_t* w = reinterpret_cast<int32_t*>(buf + static_cast<size_t>(idx) * rec_bytes);
+  const int t = threadIdx.x;
+  if (t < 8) w[t] = t == 0 ? kind : t == 1 ? *d_len : t == 2 ? n_rows : t == 3 ? n_clean : t == 4 ? R : 0;
+  if (t < kNT) {
+    w[8 + t] = t < n_rows ? tokens[t] : -1;
+    w[24 + t] = (t < n_rows && masked) ? static_cast<int32_t>(masked[t]) : 0;
+  }
+}
+
+// ... and after it: LM-head outputs, the block state, the next seed and cache
+// length, and the final residual stream rows; then the record count advances.
+__global__ void trace_end_kernel(uint8_t* buf, size_t rec_bytes, int cap, int32_t* cnt, const int32_t* d_len,
+                                 const int32_t* d_seed, int n_rows, int R, const int32_t* top1, const float* p1,
+                                 const int32_t* tokens, const uint8_t* masked, const uint8_t* x, size_t x_bytes) {
+  const int idx = *cnt;
+  if (idx < cap) {
+    uint8_t* rec = buf + static_cast<size_t>(idx) * rec_bytes;
+    int32_t* w = reinterpret_cast<int32_t*>(rec);
+    const int t = threadIdx.x;
+    if (t < kNT) {
+      w[40 + t] = t < R ? top1[t] : -1;
+      w[56 + t] = t < R ? __float_as_int(p1[t]) : 0;
+      w[72 + t] = t < n_rows ? tokens[t] : -1;
+      w[88 + t] = (t < n_rows && masked) ? static_cast<int32_t>(masked[t]) : 0;
+    }
+    if (t < 8) w[104 + t] = t == 0 ? *d_seed : t == 1 ? *d_len : 0;
+    uint8_t* xr = rec + kTraceWords * 4;
+    for (size_t i = t; i < x_bytes / 4; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(xr)[i] = reinterpret_cast<const uint32_t*>(x)[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && idx < cap) *cnt = idx + 1;
+}
+
 struct Carver {
   uint8_t* base;
   size_t off = 0;
@@ -78,11 +118,21 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->tokens = c.take<int32_t>((kNT + 1) * 4);
   e->vids = c.take<int32_t>((kNT + 1) * 4);
   e->masked = c.take<uint8_t>(kNT + 1);
+  e->tr_top1 = c.take<int32_t>(kNT * 4);
+  e->tr_p1 = c.take<float>(kNT * 4);
   e->hist = c.take<int64_t>(DVLM_HIST * 8);
   e->ahist = c.take<int64_t>(DVLM_HIST * 8);
   e->stage_vis = c.take<void>(static_cast<size_t>(std::max(e->max_ctx, 1)) * H * es);
   e->stage_ids = c.take<int32_t>(std::max(e->max_ctx, 1) * 4);
   e->stage_out = c.take<int32_t>(static_cast<size_t>(e->Lmax) * 4);
+  if (e->bf16 && e->max_ctx > 0) {
+    const size_t C = static_cast<size_t>(e->max_ctx);
+    e->px = c.take<void>(C * H * 2);
+    e->pq = c.take<void>(C * HD * 2);
+    e->pao = c.take<void>(C * HD * 2);
+    e->pact = c.take<void>(C * I * 2);
+    e->pssq = c.take<float>(static_cast<size_t>(H / 128 + 1) * C * 4);
+  }
   if (!e->bf16) {
     e->f_y = c.take<float>(static_cast<size_t>(kNT) * std::max(qkv_rows, H) * 4);
     e->f_r = c.take<float>(kNT * 4);
@@ -112,8 +162,23 @@ static bool build_maps(dvlm_engine* e) {
   ok &= make_tmap_2d(&e->tm_k, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 64);
   ok &= make_tmap_2d(&e->tm_v, e->vc, e->Lmax, static_cast<uint64_t>(L) * Hkv * D,
                      static_cast<uint64_t>(e->Lmax) * 2, 64, 128);
+  if (e->max_ctx > 0) {
+    const uint64_t C = static_cast<uint64_t>(e->max_ctx);
+    ok &= make_tmap_2d(&e->tm_px, e->px, H, C, H * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_pq, e->pq, Hq * D, C, Hq * D * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_pao, e->pao, Hq * D, C, Hq * D * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_pact, e->pact, I, C, static_cast<uint64_t>(I) * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_wqkv_p, m.wqkv, H, static_cast<uint64_t>(L) * qkv_rows, H * 2, 64, 256);
+    ok &= make_tmap_2d(&e->tm_wo_p, m.wo, Hq * D, static_cast<uint64_t>(L) * H, Hq * D * 2, 64, 256);
+    ok &= make_tmap_2d(&e->tm_wd_p, m.wdown, I, static_cast<uint64_t>(L) * H, static_cast<uint64_t>(I) * 2, 64, 256);
+    ok &= make_tmap_2d(&e->tm_wg_p, m.wgate, H, static_cast<uint64_t>(L) * I, H * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_wu_p, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_kp, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 128);
+  }
   return ok;
 }
+
+
 
 static int ws_ctas(dvlm_engine* e, long long units) {
   return static_cast<int>(std::min<long long>(e->sm, units));
@@ -329,8 +394,127 @@ static cudaError_t fwd_f32(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   return cudaSuccess;
 }
 
+// Shapes the compute-bound prefill handles: 256-row weight tiles (two heads
+// of 128 per QKV tile), 128-row gate/up tiles, k in 64-wide blocks.
+bool prefill_gemm_supported(const dvlm_engine* e) {
+  const dvlm_model& m = e->m;
+  const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
+  return e->bf16 && e->max_ctx > 0 && m.head_dim == 128 && m.hidden % 256 == 0 && m.inter % 128 == 0 &&
+         qkv_rows % 256 == 0 && (m.n_q_heads * m.head_dim) % 64 == 0;
+}
+
+// Prefill of n = n_vis + n_ids context rows at slots 0..n-1 [Fast-dVLM
+// technical overview (ocdem.com), section 2.2.1: the exact KV cache of vision
+// and prompt tokens the blocks attend to]: per layer one token-major GEMM per
+// projection over all n rows and one causal attention launch; then the final
+// norm and LM head of row n-1 give the first AR seed, and L = n.
+cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, const int32_t* ids, int n_ids,
+                                cudaStream_t s) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
+  const int qkv_rows = (Hq + 2 * Hkv) * D;
+  const int n = n_vis + n_ids, C = e->max_ctx;
+  bf16* px = static_cast<bf16*>(e->px);
+  DVLM_CK(cudaMemsetAsync(e->d_len, 0, 4, s));
+  DVLM_CK(launch_embed_bf16(static_cast<const bf16*>(m.embed), static_cast<const bf16*>(vision), n_vis, ids, nullptr,
+                            m.mask_id, n, H, m.vocab, px, e->pssq, C, e->d_status, false, s));
+  // V^T as the attention reads it: keys past slot n - 1 are zero-filled by the
+  // load (stale or poisoned cache slots never enter a product)
+  CUtensorMap tm_vp;
+  if (!make_tmap_2d(&tm_vp, e->vc, n, static_cast<uint64_t>(m.n_layers) * Hkv * D, static_cast<uint64_t>(e->Lmax) * 2,
+                    64, 128))
+    return cudaErrorInvalidValue;
+  const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
+  TmArgs ta{};
+  ta.n_tok = n;
+  ta.tok_stride = C;
+  ta.inv_h = 1.0f / H;
+  ta.eps = m.eps;
+  ta.Lmax = e->Lmax;
+  ta.n_q_heads = Hq;
+  ta.n_kv_heads = Hkv;
+  ta.L0 = 0;
+  ta.log2_rope_base = std::log2(static_cast<double>(m.rope_base));
+  ta.status = e->d_status;
+  PrefillAttnArgs pa{};
+  pa.n_tok = n;
+  pa.L0 = 0;
+  pa.Lmax = e->Lmax;
+  pa.Hq = Hq;
+  pa.Hkv = Hkv;
+  pa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  pa.out = static_cast<bf16*>(e->pao);
+  pa.out_ld = Hq * D;
+  pa.status = e->d_status;
+  for (int l = 0; l < m.n_layers; ++l) {
+    ta.epi = EPI_QKV;
+    ta.ssq_in = e->pssq;
+    ta.n_ssq = l == 0 ? H / 128 : H / 256;
+    ta.out = static_cast<bf16*>(e->pq);
+    ta.out_ld = Hq * D;
+    ta.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
+    ta.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
+    DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wqkv_p, e->tm_wqkv_p, H / 64, l * qkv_rows, qkv_rows / 256, ta, s));
+    pa.kv_base = l;
+    DVLM_CK(launch_attn_prefill(e->tm_pq, e->tm_kp, tm_vp, pa, s));
+    ta.epi = EPI_RESID;
+    ta.resid = px;
+    ta.resid_ld = H;
+    ta.ssq_out = e->pssq;
+    DVLM_CK(launch_gemm_tm(e->tm_pao, e->tm_wo_p, e->tm_wo_p, Hq * D / 64, l * H, H / 256, ta, s));
+    ta.epi = EPI_SWIGLU;
+    ta.n_ssq = H / 256;
+    ta.out = static_cast<bf16*>(e->pact);
+    ta.out_ld = I;
+    DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wg_p, e->tm_wu_p, H / 64, l * I, I / 128, ta, s));
+    ta.epi = EPI_RESID;
+    DVLM_CK(launch_gemm_tm(e->tm_pact, e->tm_wd_p, e->tm_wd_p, I / 64, l * H, H / 256, ta, s));
+  }
+  // last context row -> decode buffer row 0 (with its sums of squares), then
+  // the final norm + LM head: the AR seed of the first block, L = n
+  DVLM_CK(launch_embed_bf16(nullptr, px + static_cast<size_t>(n - 1) * H, 1, nullptr, nullptr, 0, 1, H, m.vocab,
+                            static_cast<bf16*>(e->x), e->ssq, kNT, e->d_status, false, s));
+  LmArgs a{};
+  a.R = 1;
+  a.threshold = -1.0f;
+  a.seed_out = e->d_seed;
+  a.seed_row = 0;
+  a.len_ptr = e->d_len;
+  a.len_advance = n;
+  fill_lm_scratch(e, a);
+  a.ssq_in = e->ssq;
+  a.n_ssq = H / 128;
+  a.inv_h = 1.0f / H;
+  a.eps = m.eps;
+  const int nt = (m.vocab + 127) / 128;
+  return launch_lmhead(kNT, e->tm_lm, e->tm_x, nt, H / 64, ws_ctas(e, static_cast<long long>(nt) * (H / 64)), a,
+                       false, s);
+}
+
 cudaError_t engine_forward(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   return e->bf16 ? fwd_bf16(e, f, s) : fwd_f32(e, f, s);
+}
+
+// One forward of the decode driver, bracketed by the trace kernels when a
+// trace buffer is set (the LM head then also reports its rows' ids and
+// probabilities).  `tokens`/`masked` are the block state the trace records.
+static cudaError_t traced_forward(dvlm_engine* e, FwdSpec f, int kind, const int32_t* tokens,
+                                  const uint8_t* masked, cudaStream_t s) {
+  if (!e->trace_buf) return engine_forward(e, f, s);
+  const size_t rb = trace_record_bytes(e->m.hidden, e->bf16);
+  trace_begin_kernel<<<1, 32, 0, s>>>(e->trace_buf, rb, e->trace_cap, e->trace_cnt, kind, e->d_len, f.n_rows,
+                                      f.n_clean, f.lm ? f.lma.R : 0, tokens, masked);
+  DVLM_CK(cudaGetLastError());
+  if (f.lm) {
+    f.lma.top1_id = e->tr_top1;
+    f.lma.top1_prob = e->tr_p1;
+  }
+  DVLM_CK(engine_forward(e, f, s));
+  const size_t xb = static_cast<size_t>(f.n_rows) * e->m.hidden * (e->bf16 ? 2 : 4);
+  trace_end_kernel<<<1, 256, 0, s>>>(e->trace_buf, rb, e->trace_cap, e->trace_cnt, e->d_len, e->d_seed, f.n_rows,
+                                     f.lm ? f.lma.R : 0, e->tr_top1, e->tr_p1, tokens, masked,
+                                     static_cast<const uint8_t*>(e->x), xb);
+  return cudaGetLastError();
 }
 
 // Replays the captured graph for `key`, capturing `body` on first use.
@@ -387,7 +571,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
       f.lma.len_advance = 1;
       // emit the token being fed before the LM head overwrites the seed
       DVLM_CK(launch_emit(e->d_seed, 1, e->stage_out, e->n_out, max_new, false, s));
-      return engine_forward(e, f, s);
+      return traced_forward(e, f, TR_AR, e->d_seed, nullptr, s);
     }));
     if (st) {
       st->nfe += 1;
@@ -418,7 +602,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
         f.lma.threshold = cfg.threshold;
         f.lma.n_remaining = e->n_remaining;
         f.lma.hist = e->hist;
-        return engine_forward(e, f, s);
+        return traced_forward(e, f, TR_NOISY, e->tokens, e->masked, s);
       }));
       int32_t h = 0;
       DVLM_CK(cudaMemcpyAsync(&h, e->n_remaining, 4, cudaMemcpyDeviceToHost, s));
@@ -442,7 +626,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
       f.lma.seed_row = B - 1;
       f.lma.len_ptr = e->d_len;
       f.lma.len_advance = B;
-      DVLM_CK(engine_forward(e, f, s));
+      DVLM_CK(traced_forward(e, f, TR_APPEND, e->tokens, nullptr, s));
       return launch_emit(e->tokens, B, e->stage_out, e->n_out, max_new, true, s);
     }));
     if (st) {
@@ -465,7 +649,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
     f.lma.masked = e->masked + 1;
     f.lma.tokens = e->tokens + 1;
     f.lma.threshold = -1.0f;  // the draft takes every position's argmax
-    return engine_forward(e, f, s);
+    return traced_forward(e, f, TR_DRAFT, e->tokens, e->masked, s);
   }));
   DVLM_CK(run_graph(e, {G_VERIFY, B, max_new}, ug, s, [&]() -> cudaError_t {
     FwdSpec f;
@@ -478,7 +662,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
     f.lma.id_out = e->vids + 1;  // row j predicts position j+1
     f.lma.len_ptr = e->d_len;
     f.lma.len_advance = B;
-    DVLM_CK(engine_forward(e, f, s));
+    DVLM_CK(traced_forward(e, f, TR_VERIFY, e->tokens, nullptr, s));
     return launch_decode_accept(e->vids, e->tokens, B, e->d_len, e->d_seed, e->stage_out, e->n_out, max_new,
                                 e->ahist, e->d_status, true, s);
   }));
@@ -571,6 +755,10 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
     e->attn_cs = v;
   } else if (n == "pdl") {
     e->pdl = v != 0;
+  } else if (n == "prefill_gemm") {
+    if (v != 0 && v != 1) return DVLM_ERR_SHAPE;
+    if (v && !prefill_gemm_supported(e)) return DVLM_ERR_UNSUPPORTED;
+    e->prefill_gemm = v != 0;
   } else {
     return DVLM_ERR_INVALID_ARG;
   }
@@ -589,7 +777,18 @@ int engine_get_option(dvlm_engine* e, const char* name) {
   if (n == "gateup_ctas_per_sm") return e->gu_cps;
   if (n == "attn_cluster") return e->attn_cs;
   if (n == "pdl") return e->pdl ? 1 : 0;
+  if (n == "prefill_gemm") return e->prefill_gemm ? 1 : 0;
   return -1;
+}
+
+// Sets (or clears, buf == NULL) the forward trace; captured graphs are
+// rebuilt with or without the trace kernels.
+void engine_set_trace(dvlm_engine* e, void* buf, int cap, int32_t* cnt) {
+  e->trace_buf = static_cast<uint8_t*>(buf);
+  e->trace_cap = buf ? cap : 0;
+  e->trace_cnt = buf ? cnt : nullptr;
+  for (auto& kv : e->graphs) cudaGraphExecDestroy(kv.second);
+  e->graphs.clear();
 }
 
 size_t engine_workspace_bytes(dvlm_engine* e, int P) { return carve(e, nullptr, true, P); }
@@ -614,6 +813,7 @@ void engine_plan(dvlm_engine* e) {
   e->s_down = pick_cluster(e, EPI_RESID, m.hidden / 128, m.inter / 64, e->down_stages);
   // 16-CTA attention clusters when one per KV head can be resident at once
   e->attn_cs = attn_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
+  e->prefill_gemm = prefill_gemm_supported(e);
 }
 
 }  // namespace dvlm

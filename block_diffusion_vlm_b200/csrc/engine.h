@@ -52,6 +52,24 @@ struct FwdSpec {
   int L_host = 0;
 };
 
+// Trace of the decode driver's forwards (test hook): one record per forward
+// in a caller-owned device buffer, in launch order.  Layout of a record (32-bit
+// words, then the final residual stream of its rows):
+//   [0] kind (TR_*), [1] cache length L at the forward, [2] rows, [3] clean
+//   rows, [4] LM-head rows R, [5..7] zero;
+//   [8..23] block tokens before, [24..39] masked flags before (1 = masked),
+//   [40..55] LM-head top-1 id of rows 0..R-1, [56..71] their top-1
+//   probability (fp32 bits), [72..87] tokens after, [88..103] masked after,
+//   [104] next AR seed after, [105] cache length after, [106..111] zero;
+//   then rows x H residual-stream values (bf16 or fp32, the model's dtype),
+//   before the final RMSNorm.  Records are padded to 256 bytes.
+enum TraceKind { TR_NOISY = 1, TR_APPEND = 2, TR_DRAFT = 3, TR_VERIFY = 4, TR_AR = 5 };
+constexpr int kTraceWords = 112;
+inline size_t trace_record_bytes(int hidden, bool bf16) {
+  const size_t b = kTraceWords * 4 + static_cast<size_t>(kNT) * hidden * (bf16 ? 2 : 4);
+  return (b + 255) / 256 * 256;
+}
+
 // Kernel launches of one forward pass over n_layers layers.
 inline int launches_per_forward(int n_layers) { return 2 + 5 * n_layers; }
 
@@ -69,6 +87,7 @@ struct dvlm_engine {
   int gu_stages = 10, down_stages = 10; // pipeline depth of the gate/up and down projections
   int gu_cps = 1;                       // gate/up CTAs per SM (2 needs 5 stages)
   bool pdl = true;                      // programmatic dependent launch between kernels
+  bool prefill_gemm = true;             // compute-bound prefill (prefill.cu) where the shapes allow it
   // device buffers carved from the workspace
   void* x = nullptr;        // [NT][H]
   void* q = nullptr;        // [NT][Hq*D]
@@ -95,6 +114,18 @@ struct dvlm_engine {
   int32_t* stage_ids = nullptr;  // [max_ctx]
   int32_t* stage_out = nullptr;  // [max_ctx] generated tokens (host path)
   int32_t* h_pinned = nullptr;   // host-mapped scalars (n_remaining, n_out, L, seed)
+  int32_t* tr_top1 = nullptr;    // [NT] LM-head ids while tracing
+  float* tr_p1 = nullptr;        // [NT] LM-head probabilities while tracing
+  // forward trace (test hook, off unless set): records, capacity, device count
+  uint8_t* trace_buf = nullptr;
+  int trace_cap = 0;
+  int32_t* trace_cnt = nullptr;
+  // compute-bound prefill buffers, max_ctx rows each (bf16 engines)
+  void* px = nullptr;            // [max_ctx][H] residual stream
+  void* pq = nullptr;            // [max_ctx][Hq*D]
+  void* pao = nullptr;           // [max_ctx][Hq*D] attention output
+  void* pact = nullptr;          // [max_ctx][I] SwiGLU activation
+  float* pssq = nullptr;         // [H/128][max_ctx] sums of squares
   // fp32 path scratch
   float* f_y = nullptr;          // [NT][max(qkv_rows, H)]
   float* f_r = nullptr;          // [NT]
@@ -104,6 +135,8 @@ struct dvlm_engine {
   int32_t* f_id = nullptr;       // [NT]
   // tensor maps
   CUtensorMap tm_wqkv, tm_wo, tm_wg, tm_wu, tm_wd, tm_lm, tm_x, tm_ao, tm_act, tm_q, tm_k, tm_v;
+  // prefill: activations (128-row boxes), weights (256-row boxes; gate/up 128), K (128-key boxes)
+  CUtensorMap tm_px, tm_pq, tm_pao, tm_pact, tm_wqkv_p, tm_wo_p, tm_wd_p, tm_wg_p, tm_wu_p, tm_kp;
   // captured graphs keyed by (kind, B, threshold bits, max_new)
   std::map<std::vector<long long>, cudaGraphExec_t> graphs;
 };

@@ -112,6 +112,43 @@ cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, c
                              const AttnArgs& a, bool pdl, cudaStream_t s, int cs = 8);
 int attn_max_clusters(int cs);
 
+// Prefill (compute-bound path over the whole context; csrc/prefill.cu).
+// Token-major GEMM epilogue operands: one context row per epilogue thread.
+struct TmArgs {
+  int epi;
+  int n_tok;                  // valid context rows
+  int tok_stride;             // ssq arrays are [entry][tok_stride]
+  const float* ssq_in;        // RMSNorm input sums of squares (QKV, SWIGLU)
+  int n_ssq;
+  float inv_h, eps;
+  bf16* out;                  // QKV: q [n_tok][Hq*128]; SWIGLU: act [n_tok][I]
+  int out_ld;
+  bf16* resid;                // RESID: residual stream [n_tok][H], updated in place
+  int resid_ld;
+  float* ssq_out;             // RESID: [H/256][tok_stride]
+  bf16* kcache;               // QKV: this layer's K [Hkv][Lmax][128] and V^T [Hkv][128][Lmax]
+  bf16* vcache;
+  int Lmax, n_q_heads, n_kv_heads;
+  int L0;                     // cache slot of context row 0
+  double log2_rope_base;
+  int* status;
+};
+// y = x W^T over n_wtiles tiles of 256 weight rows (SWIGLU: 128 rows of W and
+// the same 128 rows of W2) starting at weight row w_row_base; kb = K / 64.
+cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, const CUtensorMap& mapW2, int kb,
+                           int w_row_base, int n_wtiles, const TmArgs& a, cudaStream_t s);
+struct PrefillAttnArgs {
+  int n_tok, L0;              // query rows at slots L0..L0+n_tok-1
+  int kv_base;                // cache entry (the layer)
+  int Lmax, Hq, Hkv;
+  float scale_log2;
+  bf16* out;                  // [n_tok][out_ld], head h at column h * 128
+  int out_ld;
+  int* status;
+};
+cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                const PrefillAttnArgs& a, cudaStream_t s);
+
 // Embedding gather / row copy + per-128-feature sums of squares.
 cudaError_t launch_embed_bf16(const bf16* E, const bf16* rows_in, int n_src, const int32_t* tokens,
                               const uint8_t* masked, int mask_id, int n_rows, int H, int V, bf16* x,

@@ -7,9 +7,13 @@
 // can synchronise the whole device and stall the loop.  For them
 // dvlm_lmhead_conf_commit_static keeps its scratch (split-tile partials,
 // counters, per-CTA records, sums of squares) in one file-scope device array
-// of fixed size.  The array exists on every GPU that loads this library,
-// from module load until the process exits.  The entry point allocates
-// nothing and calls no allocating routine.
+// of fixed size.  The CUDA runtime creates the array on a GPU when it loads
+// this library's device code there (with lazy loading, the default, at the
+// first call that needs that code) and keeps it until the process exits or
+// the device is reset.  The entry point allocates nothing and calls no
+// allocating routine.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "kernels.h"
@@ -23,22 +27,51 @@ static __device__ __align__(256) unsigned char g_lm_scratch[kStaticScratchBytes]
 
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
+unsigned long long g_ctx[kMaxDevices] = {};  // context the address belongs to
+
+// Unique id of the current context (cuCtxGetId, fetched through the runtime
+// so the library does not link libcuda); 0 when unavailable.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    tried = true;
+  }
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_id || !get_cur || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of g_lm_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, never a device address: the
-// runtime returns the real one, looked up once per device with that device
-// current, and that is what the kernels are given.
+// runtime returns the real one, looked up at set-up with that device current
+// (the first call on the device), and that is what the kernels are given.
+// A device reset gives the device a new context, in which the array may sit
+// elsewhere: the address is looked up again when the current context is not
+// the one it was taken in.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
+  if (!g_addr[dev] || ctx == 0 || g_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_lm_scratch);
     if (e != cudaSuccess) return e;
     g_addr[dev] = p;
+    g_ctx[dev] = ctx;
   }
   *out = g_addr[dev];
   return cudaSuccess;

@@ -47,18 +47,23 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
   return r == CUDA_SUCCESS;
 }
 
+// SM count of the current device, queried once per device (a process may
+// drive GPUs with different SM counts).
 int device_sm_count() {
-  static int cached = 0;
-  if (cached == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      return -1;
-    }
-    cached = n;
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return -1;
   }
-  return cached;
+  if (dev < kMaxDev && cached[dev] > 0) return cached[dev];
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (dev < kMaxDev) cached[dev] = n;
+  return n;
 }
 
 }  // namespace dvlm

@@ -145,15 +145,20 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, 
  * allocator; a real-time control loop that forbids cudaMalloc after start-up
  * because an allocation can synchronise the device).  No counterpart on the
  * method's pages: this is a deployment variant.  It takes no workspace: its
- * scratch is one fixed 6 MiB device array inside the library, present on
- * every GPU that loads the library until the process exits.  Limits: R <= 32
+ * scratch is one fixed 6 MiB device array inside the library.  The CUDA
+ * runtime creates that array on a GPU when it loads the library's device
+ * code there -- with lazy module loading, the CUDA default, during the first
+ * call on that GPU -- and keeps it until the process exits.  Limits: R <= 32
  * and a scratch layout (about 17 KiB per SM plus 4 bytes per 128 vocabulary
  * rows) within 6 MiB, e.g. V <= 262144 and H <= 8192 on a 148-SM B200;
  * larger requests return DVLM_ERR_WORKSPACE and launch nothing.  The first
- * call on a device looks the array's device address up (make that first call
- * before any stream capture).  Every call shares the one array: calls that
- * overlap on the GPU (other streams, other threads) race and must be
- * serialised by the caller.  Allocates nothing; calls no allocating routine. */
+ * call on a device (and the first after a device reset) looks the array's
+ * device address up: make one warm-up call at start-up, before any stream
+ * capture.  Every call shares the one array and finds the previous call's
+ * contents there (the counters it needs at zero are cleared on the stream
+ * first): calls that overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller.  Allocates nothing; calls no
+ * allocating routine. */
 DVLM_API dvlm_status dvlm_lmhead_conf_commit_static(const void* hidden, const void* w, int R, int H, int V,
                                                    int apply_rmsnorm, float eps, uint8_t* masked,
                                                    int32_t* tokens, float threshold, int32_t* top1_id,
@@ -369,6 +374,29 @@ DVLM_API dvlm_status dvlm_selftest_wait_timeout(long long budget_cycles, int* de
  * (synchronises the stream) and launches eagerly. */
 DVLM_API dvlm_status dvlm_forward_text_only(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
                                            int n_rows, int n_hidden, void* x_out, dvlm_stream stream);
+
+/* Trace of the decode driver (test hook).  When set, every forward that
+ * dvlm_decode_block / dvlm_generate run (noisy, causal append, draft, verify,
+ * AR) appends one record to buf (device, caller-owned, 16-byte aligned) and
+ * increments *count (device int32, zeroed by the caller); records past the
+ * capacity bytes / dvlm_engine_trace_record_bytes(m) are dropped and the
+ * count stops there.  A record holds 112 int32 words and then the final
+ * residual stream of the forward's rows before the final RMSNorm (16 x H
+ * values in the model's dtype):
+ *   [0] kind (1 noisy, 2 causal append, 3 speculative draft, 4 speculative
+ *   verify, 5 AR), [1] cache length L at the forward, [2] rows, [3] clean
+ *   rows, [4] LM-head rows R; [8..23] block tokens before the forward,
+ *   [24..39] masked flags before (1 = still masked); [40..55] the LM head's
+ *   top-1 id of rows 0..R-1 and [56..71] their top-1 probability (fp32
+ *   bits); [72..87] block tokens after the LM head's commit, [88..103]
+ *   masked flags after; [104] the pending AR seed and [105] the cache length
+ *   after the forward.
+ * The kernels run inside the captured CUDA graphs (setting or clearing the
+ * trace drops them).  buf == NULL clears the trace.  Errors: INVALID_ARG,
+ * WORKSPACE (room for less than one record).  Decisions and outputs of the
+ * decode do not change. */
+DVLM_API size_t dvlm_engine_trace_record_bytes(const dvlm_model* m);
+DVLM_API dvlm_status dvlm_engine_set_trace(dvlm_engine* e, void* buf, size_t bytes, int32_t* count);
 
 /* Profiling hook: one forward pass like dvlm_forward over all layers (L is
  * not advanced), launched eagerly with a CUDA event pair around every kernel

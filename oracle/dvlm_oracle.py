@@ -264,6 +264,8 @@ class Conf:
     p1: np.ndarray     # top-1 probability per row
     top1: np.ndarray   # lowest id attaining the max logit
     p2: np.ndarray     # second-largest probability (margin checks)
+    top2: Optional[np.ndarray] = None   # the runner-up id: lowest id attaining the max
+                                        # logit once top1 is set aside (near-tie checks)
 
 
 def confidence_from_logits(logits: np.ndarray) -> Conf:
@@ -277,7 +279,10 @@ def confidence_from_logits(logits: np.ndarray) -> Conf:
     top1 = np.argmax(lg, axis=-1).astype(np.int64)      # first maximum
     part = np.partition(lg, -2, axis=-1)[..., -2]
     p2 = np.exp(part - m[..., 0]) / s
-    return Conf(p1=p1, top1=top1, p2=p2)
+    rest = lg.copy()
+    np.put_along_axis(rest, top1[..., None], -np.inf, axis=-1)
+    top2 = np.argmax(rest, axis=-1).astype(np.int64)
+    return Conf(p1=p1, top1=top1, p2=p2, top2=top2)
 
 
 def lm_head_conf(hidden: np.ndarray, W: np.ndarray, row_scale: Optional[np.ndarray] = None) -> Conf:
@@ -585,7 +590,8 @@ def decode_threshold(model: OracleModel, seed_token: int, B: int, tau: float, ma
         c = model.logits_conf(x)
         tr.nfe += 1
         _note_argmax_margin(tr, c, [B - 1])
-        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:])
+        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:],
+                         top2=None if c.top2 is None else c.top2[B - 1:])
         seed = int(c.top1[B - 1])
         tr.tokens.extend(toks)
     tr.tokens = tr.tokens[:max_new]
@@ -844,7 +850,8 @@ def decode_lown(model: OracleModel, seed_token: int, B: int, k: int, n_vis: int,
         model.L = L + B
         c = model.logits_conf(x)
         tr.n_causal += 1
-        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:])
+        prev_conf = Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:],
+                         top2=None if c.top2 is None else c.top2[B - 1:])
         seed = int(c.top1[B - 1])
         take = min(B, max_new - len(tr.tokens))
         tr.tokens.extend(toks[:take])

@@ -1,24 +1,25 @@
-"""End-to-end block decoding through the engine vs the oracle's decoders on
-small models: the tiny fp32 model (first configuration: 64-token context of 32
-vision embeddings, 16 prompt and 16 committed ids, one B=4 block, threshold
-0.9) and a reduced-depth bf16 model with the same per-head shapes as the
-Qwen2.5-3B decoder.
+"""End-to-end block decoding through the engine's own CUDA-graph path vs the
+oracle, on small models: the tiny fp32 model (first configuration: 64-token
+context of 32 vision embeddings, 16 prompt and 16 committed ids, one B=4
+block, threshold 0.9) and a reduced-depth bf16 model with the same per-head
+shapes as the Qwen2.5-3B decoder.
 
-fp32: token sequences and commit counts must match exactly when every
-decision on the oracle's trajectory is at least 1e-3 away from its threshold /
-runner-up (GPU and oracle p1 agree to ~1e-6 there; the seeds were chosen by
-running the oracle alone); otherwise a mismatch is only allowed when the
-oracle's trajectory does contain such a near-tie.
+Every forward the engine's decode driver runs is recorded by its trace hook
+(dvlm_engine_set_trace) and replayed against the oracle, teacher-forced
+(tests/decode_replay.py): the oracle runs the same forward over its own cache,
+the hidden rows must agree (1e-4 fp32; 2e-2 plus one storage ulp bf16), and
+every top-1 id, commit set, accepted length and seed must be bit-exact
+wherever its deciding confidences are at least 1e-3 from the boundary; inside
+that margin the GPU may take any of the tied choices and the oracle follows
+it.
 
-bf16: GPU and oracle round to bf16 at the same storage points, but a value
-whose fp32 and fp64 sums fall on either side of a bf16 rounding boundary
-lands one storage ulp apart, and the LM head (N(0, 0.02) x 25 weights) turns
-such a flip into a p1 difference of a few 1e-2.  A whole trajectory can then
-branch at a decision the oracle takes with a margin of 1e-2, so the
-threshold decoder is checked per iteration instead, teacher-forced: every
-noisy forward of the oracle's trajectory is replayed on the GPU with the same
-block tokens over the same cache, and top-1 ids and commit decisions must
-agree wherever the oracle's margin is at least DELTA."""
+fp32: the deciding confidences are the oracle's own (GPU and oracle hidden
+rows agree to ~1e-6).  bf16: a value whose fp32 and fp64 sums fall on either
+side of a bf16 rounding boundary lands one storage ulp apart, and the LM head
+(N(0, 0.02) x 25 weights) turns such a flip into a p1 difference of a few
+1e-2, so the 1e-3 bar is applied to the oracle's LM head on the GPU's own
+final hidden rows (the rows the fused LM head + commit read), and the
+oracle's own rows hold the decisions to DELTA = 0.1."""
 import numpy as np
 import pytest
 import torch
@@ -26,15 +27,16 @@ import torch
 import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
 import oracle as O
+from decode_replay import NOISY, Replay, parse_trace
 from dvlm_gen.device import DeviceModel, kv_buffers
-from gpu_util import assert_ok, f64, max_abs, status, ws_tensor
+from gpu_util import assert_bf16_close, assert_ok, f64, max_abs, status, ws_tensor
 
 pytestmark = pytest.mark.gpu
 MARGIN = 1e-3
-# bound on |p1(GPU) - p1(oracle)| for the bf16 reduced model on identical inputs:
-# hidden states one storage ulp apart in a few elements move p1 by a few 1e-2
-# (GPU against oracle: up to 0.03 measured; a CPU model of such rounding
-# flips: up to 0.066, tests/test_precision_model.py)
+# bound on |p1(GPU) - p1(oracle)| for the bf16 reduced model on the oracle's
+# own hidden rows: hidden states one storage ulp apart in a few elements move
+# p1 by a few 1e-2 (GPU against oracle: up to 0.03 measured; a CPU model of
+# such rounding flips: up to 0.066, tests/test_precision_model.py)
 DELTA = 0.1
 
 SMALL_BF16 = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=1024,
@@ -66,9 +68,29 @@ class Setup:
         eng.check()
         return out.cpu().numpy().tolist(), st
 
-    def oracle(self, mode, B, tau, n_new):
+    def traced(self, mode, B, tau, n_new, use_graphs=1, cap=512):
+        """Decode with the engine's forward trace on: (tokens, stats, records, final L, final seed)."""
+        rb = dv.engine_trace_record_bytes(self.dm.c_model())
+        buf = torch.zeros(cap * rb, dtype=torch.uint8, device=self.cuda)
+        cnt = torch.zeros(4, dtype=torch.int32, device=self.cuda)
+        self.eng.set_trace(buf, cnt)
+        try:
+            tokens, st = self.gpu(mode, B, tau, n_new, use_graphs)
+        finally:
+            self.eng.set_trace(None, None)
+        n = int(cnt[0].item())
+        assert 0 < n < cap
+        L, seed = self.eng.position()
+        recs = parse_trace(buf.cpu().numpy(), n, rb, self.dims.hidden, self.dims.dtype == "bf16")
+        return tokens, st, recs, L, seed
+
+    def oracle_model(self):
         m = O.OracleModel(self.od, weights=self.w, bf16=self.dims.dtype == "bf16", Lmax=self.Lmax)
         s = O.prefill(m, self.vis.astype(np.float64), self.ids)
+        return m, s
+
+    def oracle(self, mode, B, tau, n_new):
+        m, s = self.oracle_model()
         if mode == dv.MODE_THRESHOLD:
             return O.decode_threshold(m, s, B, tau, n_new), m
         if mode == dv.MODE_SPEC_LINEAR:
@@ -76,18 +98,37 @@ class Setup:
         return O.decode_ar(m, s, n_new), m
 
 
-def _compare(tokens, st, tr, mode):
-    if tr.min_margin >= MARGIN:
-        assert tokens == tr.tokens
-        assert st.nfe == tr.nfe
-        if mode == dv.MODE_THRESHOLD:
-            hist = np.bincount(tr.commits_per_iter, minlength=dv.binding.HIST)[:dv.binding.HIST]
-            assert list(st.commit_hist) == hist.tolist()
-        if mode == dv.MODE_SPEC_LINEAR:
-            hist = np.bincount(tr.accept_lens, minlength=dv.binding.HIST)[:dv.binding.HIST]
-            assert list(st.accept_hist) == hist.tolist()
-    elif tokens != tr.tokens:
-        assert tr.min_margin < MARGIN
+def _fp32_hidden(a, b, what):
+    assert max_abs(a, b) < 1e-4, (what, max_abs(a, b))
+
+
+def _bf16_hidden(a, b, what):
+    assert_bf16_close(a, b, 2e-2, what)
+
+
+def replay_trace(s, mode, B, tau, n_new, tokens, st, recs, L, seed):
+    """Holds a traced engine run to the oracle (teacher-forced); returns the
+    replay (its tallies) and the oracle model (its cache)."""
+    m, so = s.oracle_model()
+    if s.dims.dtype == "bf16":
+        rp = Replay(m, so, B, tau, decide="gpu", hidden_check=_bf16_hidden, secondary=DELTA, seed_bar=DELTA)
+    else:
+        rp = Replay(m, so, B, tau, decide="oracle", hidden_check=_fp32_hidden)
+    if mode == dv.MODE_THRESHOLD:
+        got = rp.threshold(recs, n_new)
+    elif mode == dv.MODE_SPEC_LINEAR:
+        got = rp.speculative(recs, n_new, L, seed)
+    else:
+        got = rp.autoregressive(recs, n_new)
+    # the engine's emitted tokens are the committed blocks of its own trace,
+    # and its counters count exactly these forwards
+    assert got == tokens
+    assert rp._next == len(recs) == st.nfe
+    if mode == dv.MODE_THRESHOLD:
+        per_iter = [int(np.sum(r.msk_in & ~r.msk_out)) for r in recs if r.kind == NOISY]
+        hist = np.bincount(per_iter, minlength=dv.binding.HIST)[:dv.binding.HIST]
+        assert list(st.commit_hist) == hist.tolist()
+    return rp, m
 
 
 @pytest.fixture(scope="module")
@@ -101,25 +142,39 @@ def tiny4(cuda):
 
 
 def test_tiny_fp32_block_step_seed0(tiny0):
-    """The tiny configuration exactly as stated: seed 0, one B=4 block."""
-    tokens, st = tiny0.gpu(dv.MODE_THRESHOLD, 4, 0.9, 4)
-    tr, m = tiny0.oracle(dv.MODE_THRESHOLD, 4, 0.9, 4)
-    _compare(tokens, st, tr, dv.MODE_THRESHOLD)
-    # the exact KV cache after the block (prefill + causal append) within 1e-4
-    L = m.L
+    """The tiny configuration exactly as stated: seed 0, one B=4 block,
+    threshold 0.9, every decision bit-exact outside the 1e-3 margin, and the
+    exact KV cache --
+    the 64 prefilled context slots and the appended block -- within 1e-4."""
+    tokens, st, recs, L, seed = tiny0.traced(dv.MODE_THRESHOLD, 4, 0.9, 4)
+    rp, m = replay_trace(tiny0, dv.MODE_THRESHOLD, 4, 0.9, 4, tokens, st, recs, L, seed)
+    assert L == m.L == 68
     kc = f64(tiny0.kc[0, 0, :, :L])
     vc = f64(tiny0.vc[0, 0, :, :, :L]).transpose(0, 2, 1)
-    if tokens == tr.tokens:
-        assert max_abs(kc, m.K[0][:, :L]) < 1e-4
-        assert max_abs(vc, m.V[0][:, :L]) < 1e-4
+    assert max_abs(kc, m.K[0][:, :L]) < 1e-4
+    assert max_abs(vc, m.V[0][:, :L]) < 1e-4
+    # four ids (the AR seed and three commits) and three forced commits; the
+    # oracle's second forced commit picks between two positions whose p1
+    # differ by 7.2e-5, the one decision inside the margin
+    t = rp.t
+    assert t.ids_exact == 4 and t.ids_excluded == 0, t
+    assert t.commits_exact + t.commits_excluded == 3 and t.commits_excluded <= 1, t
+    print(f"config 1: {t}")
 
 
 @pytest.mark.parametrize("mode", [dv.MODE_THRESHOLD, dv.MODE_SPEC_LINEAR, dv.MODE_AR])
 def test_tiny_fp32_modes_seed4(tiny4, mode):
-    tokens, st = tiny4.gpu(mode, 4, 0.9, 16)
-    tr, m = tiny4.oracle(mode, 4, 0.9, 16)
-    assert tr.min_margin >= MARGIN  # chosen seed: well-conditioned trajectory
-    _compare(tokens, st, tr, mode)
+    tokens, st, recs, L, seed = tiny4.traced(mode, 4, 0.9, 16)
+    rp, m = replay_trace(tiny4, mode, 4, 0.9, 16, tokens, st, recs, L, seed)
+    # a well-conditioned trajectory: nothing inside the margin, so the whole
+    # run equals the oracle's own decode
+    tr, _ = tiny4.oracle(mode, 4, 0.9, 16)
+    assert tr.min_margin >= MARGIN
+    assert tokens == tr.tokens and st.nfe == tr.nfe
+    assert rp.t.ids_excluded == rp.t.commits_excluded == 0
+    if mode == dv.MODE_SPEC_LINEAR:
+        hist = np.bincount(tr.accept_lens, minlength=dv.binding.HIST)[:dv.binding.HIST]
+        assert list(st.accept_hist) == hist.tolist()
 
 
 def test_tiny_fp32_graphs_match_eager(tiny4):
@@ -128,120 +183,43 @@ def test_tiny_fp32_graphs_match_eager(tiny4):
     assert a == b and sa.nfe == sb.nfe
 
 
+def test_trace_does_not_change_the_decode(tiny4):
+    a, sa = tiny4.gpu(dv.MODE_SPEC_LINEAR, 4, 0.9, 16)
+    b, sb, _, _, _ = tiny4.traced(dv.MODE_SPEC_LINEAR, 4, 0.9, 16)
+    assert a == b and sa.nfe == sb.nfe and list(sa.accept_hist) == list(sb.accept_hist)
+
+
 @pytest.mark.parametrize("seed,mode", [(6, dv.MODE_SPEC_LINEAR)])
 def test_bf16_reduced_model_matches_oracle(cuda, seed, mode):
     """2 layers, hidden 1024, 8/1 heads of 128, SwiGLU 1024, vocab 4096;
-    48-token context (32 vision + 16 prompt), B=16, 32 tokens, speculative."""
+    48-token context (32 vision + 16 prompt), B=16, 32 tokens, speculative:
+    the whole trajectory equals the oracle's own (its smallest argmax margin
+    is 0.012)."""
     s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
     tokens, st = s.gpu(mode, 16, 0.9, 32)
     tr, m = s.oracle(mode, 16, 0.9, 32)
     assert tr.min_margin >= MARGIN
-    _compare(tokens, st, tr, mode)
+    assert tokens == tr.tokens and st.nfe == tr.nfe
     s.eng.close()
 
 
-@pytest.mark.parametrize("seed", [1, 3])
-def test_bf16_reduced_model_threshold_teacher_forced(cuda, seed):
-    """Threshold decoding (B=16, tau 0.9, 32 tokens) of the reduced bf16 model:
-    each noisy forward of the oracle's trajectory replayed on the GPU (engine
-    forward over the same cache, then the fused LM head with the final
-    RMSNorm), finished blocks appended causally on both sides."""
+@pytest.mark.parametrize("seed,mode", [(1, dv.MODE_THRESHOLD), (3, dv.MODE_THRESHOLD),
+                                       (6, dv.MODE_SPEC_LINEAR), (2, dv.MODE_SPEC_LINEAR)])
+def test_bf16_reduced_model_engine_path(cuda, seed, mode):
+    """The engine's own graph-driven decode of the reduced bf16 model (B=16,
+    tau 0.9, 32 tokens; in-graph commit, shift-1 row mapping, block set-up,
+    emission and, for speculative decoding, the accept kernel), every forward
+    replayed against the oracle: decisions bit-exact at the 1e-3 bar on the
+    rows the LM head read, within DELTA on the oracle's own rows, hidden rows
+    within 2e-2 plus one storage ulp."""
     s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
-    eng, d, dev = s.eng, SMALL_BF16, cuda
-    B, tau = 16, 0.9
-    eng.prefill(s.vis_t.to(dev), 32, torch.from_numpy(s.ids).to(dev), 16)
-    _, seed_gpu = eng.position()
-    lw = ws_tensor(dv.lmhead_workspace_size(B, d.vocab, d.hidden, dv.DVLM_BF16), dev)
-    x = torch.zeros((B, d.hidden), dtype=torch.bfloat16, device=dev)
-    counts = {"iters": 0, "top1": 0, "commit": 0}
-
-    def on_iter(L, toks, masked, p1o, topo, p2o):
-        assert eng.position()[0] == L
-        eng.forward(B, 0, d.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=dev), x_out=x)
-        top = torch.zeros(B, dtype=torch.int32, device=dev)
-        p1 = torch.zeros(B, dtype=torch.float32, device=dev)
-        st = status(dev)
-        dv.lmhead_conf_commit(x, s.dm.lm_head, R=B, H=d.hidden, V=d.vocab, dtype=dv.DVLM_BF16, apply_rmsnorm=1,
-                              top1_id=top, top1_prob=p1, workspace=lw, status=st)
-        assert_ok(st)
-        p1g, topg = p1.cpu().numpy(), top.cpu().numpy()
-        counts["iters"] += 1
-        for j in range(1, B):  # position j is scored by row j - 1
-            if not masked[j]:
-                continue
-            r = j - 1
-            assert abs(p1g[r] - p1o[j]) <= DELTA
-            if p1o[j] - p2o[j] >= DELTA:
-                assert topg[r] == topo[j]
-                counts["top1"] += 1
-            if abs(p1o[j] - tau) >= DELTA:
-                assert (p1g[r] >= tau) == (p1o[j] >= tau)
-                counts["commit"] += 1
-
-    def on_block(L, toks):
-        eng.forward(B, B, d.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=dev), advance=True)
-
-    m = O.OracleModel(s.od, weights=s.w, bf16=True, Lmax=s.Lmax)
-    seed_o = O.prefill(m, s.vis.astype(np.float64), s.ids)
-    assert seed_o == seed_gpu
-    tr = O.decode_threshold(m, seed_o, B, tau, 32, on_iter=on_iter, on_block=on_block)
-    eng.check()
-    # the comparison covered the whole trajectory and most of its decisions
-    assert counts["iters"] == tr.nfe - len(tr.tokens) // B
-    assert counts["top1"] > 0 and counts["commit"] > 0
-    s.eng.close()
-
-
-@pytest.mark.parametrize("seed", [6, 2])
-def test_bf16_reduced_model_spec_teacher_forced(cuda, seed):
-    """Linear self-speculative decoding (B=16, 32 tokens) of the reduced bf16
-    model, per round and teacher-forced: the oracle's draft pass ([seed,
-    MASK...], noisy) and verify pass (its draft, causal) are replayed on the
-    GPU over the same cache, top-1 ids compared wherever the oracle's margin
-    is at least DELTA and p1 within DELTA, then the cache length and seed are
-    set to the oracle's accepted prefix."""
-    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
-    eng, d, dev = s.eng, SMALL_BF16, cuda
-    B = 16
-    eng.prefill(s.vis_t.to(dev), 32, torch.from_numpy(s.ids).to(dev), 16)
-    _, seed_gpu = eng.position()
-    lw = ws_tensor(dv.lmhead_workspace_size(B, d.vocab, d.hidden, dv.DVLM_BF16), dev)
-    x = torch.zeros((B, d.hidden), dtype=torch.bfloat16, device=dev)
-    counts = {"rounds": 0, "draft": 0, "verify": 0}
-
-    def gpu_rows(toks, n_clean):
-        eng.forward(B, n_clean, d.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=dev), x_out=x)
-        top = torch.zeros(B, dtype=torch.int32, device=dev)
-        p1 = torch.zeros(B, dtype=torch.float32, device=dev)
-        st = status(dev)
-        dv.lmhead_conf_commit(x, s.dm.lm_head, R=B, H=d.hidden, V=d.vocab, dtype=dv.DVLM_BF16, apply_rmsnorm=1,
-                              top1_id=top, top1_prob=p1, workspace=lw, status=st)
-        assert_ok(st)
-        return top.cpu().numpy(), p1.cpu().numpy()
-
-    def check(rows, conf, top, p1, key):
-        for r in range(rows):
-            assert abs(p1[r] - conf.p1[r]) <= DELTA, (key, r, p1[r], conf.p1[r])
-            if conf.p1[r] - conf.p2[r] >= DELTA:
-                assert top[r] == conf.top1[r], (key, r)
-                counts[key] += 1
-
-    def on_round(L, toks, c, draft, g, k, nxt):
-        assert eng.position()[0] == L
-        top, p1 = gpu_rows(toks, 0)
-        check(B - 1, c, top, p1, "draft")        # row r drafts position r + 1
-        top, p1 = gpu_rows(draft, B)
-        check(B, g, top, p1, "verify")
-        eng.set_position(L + k, nxt)
-        counts["rounds"] += 1
-
-    m = O.OracleModel(s.od, weights=s.w, bf16=True, Lmax=s.Lmax)
-    seed_o = O.prefill(m, s.vis.astype(np.float64), s.ids)
-    assert seed_o == seed_gpu
-    tr = O.decode_spec_linear(m, seed_o, B, 32, on_round=on_round)
-    eng.check()
-    assert counts["rounds"] == len(tr.accept_lens)
-    assert counts["draft"] > 0 and counts["verify"] > 0
+    tokens, st, recs, L, sd = s.traced(mode, 16, 0.9, 32)
+    rp, m = replay_trace(s, mode, 16, 0.9, 32, tokens, st, recs, L, sd)
+    t = rp.t
+    assert t.ids_exact > 0 and t.secondary_checked > 0, t
+    if mode == dv.MODE_THRESHOLD:
+        assert t.commits_exact > 0, t
+    print(f"seed {seed} mode {mode}: {t}")
     s.eng.close()
 
 

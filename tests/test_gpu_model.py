@@ -1,13 +1,18 @@
 """Full-size decode (Qwen2.5-3B-shaped decoder: 36 layers, hidden 2048, 16/2
 heads, SwiGLU 11008, vocab 151936, random init; 1280 vision + 64 prompt
-context; B=16) in the launch configuration the benchmark times.  The oracle
-cannot run 36 layers over this context in test time, so these tests check
-(a) sampled outputs the oracle computes on its own inputs -- the first layer's
-K/V over the first 64 context slots -- and (b) properties that hold at any
-size: linear self-speculative decoding reproduces greedy AR decoding exactly,
-threshold decoding with B=1 is AR decoding, every block of threshold decoding
-commits B-1 positions over its iterations, runs are deterministic and graph
-replay equals eager launches."""
+context; B=16) in the launch configuration the benchmark times.
+
+(a) The first threshold block through the engine's own graph path, every
+forward replayed against the oracle (prefill and the block's forwards run
+layer-major, each layer's weights drawn once): decisions bit-exact at the
+1e-3 bar on the rows the LM head read and within DELTA on the oracle's own
+rows, the prefilled KV cache of all 36 layers and the block's hidden rows
+against the oracle's.  (b) The first layer's K/V over the first 64 context
+slots.  (c) Properties that hold at any size: linear self-speculative
+decoding reproduces greedy AR decoding exactly, threshold decoding with B=1
+is AR decoding, every block of threshold decoding commits B-1 positions over
+its iterations, runs are deterministic and graph replay equals eager
+launches."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +21,8 @@ import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
 import oracle as O
 from dvlm_gen.device import DeviceModel, kv_buffers
-from gpu_util import f64, max_abs, ws_tensor
+from decode_replay import Replay, layer_major_hidden, parse_trace
+from gpu_util import assert_bf16_close, f64, max_abs, ws_tensor
 
 pytestmark = pytest.mark.gpu
 SEED = 4          # the full decode configuration is the fifth: seed 4
@@ -61,6 +67,74 @@ def test_prefill_first_layer_kv_matches_oracle(full):
     v = f64(full["vc"][0, 0, :, :, :n]).transpose(0, 2, 1)
     assert max_abs(k, m.K[0][:, :n]) < 2e-2
     assert max_abs(v, m.V[0][:, :n]) < 2e-2
+
+
+DELTA = 0.1   # the bar on the oracle's own rows (tests/test_gpu_decode.py gives the derivation)
+
+
+def _hidden_err_profile(got, want):
+    """Largest error, and the largest in units of the oracle value's bf16 ulp."""
+    from gpu_util import bf16_ulp
+    err = np.abs(np.asarray(got) - np.asarray(want))
+    return float(err.max()), float((err / bf16_ulp(want)).max())
+
+
+@pytest.mark.slow
+def test_first_block_matches_oracle_at_full_size(full):
+    """The benchmarked configuration: prefill of 1280 vision rows + 64 prompt
+    ids, then one threshold block (B=16, tau 0.9) through the engine's CUDA
+    graphs with the forward trace on; the oracle prefills on its own and
+    replays every traced forward, teacher-forced."""
+    dims, eng, cuda = full["dims"], full["eng"], full["kc"].device
+    L0, seed0 = full["L0"], full["seed0"]
+    rb = dv.engine_trace_record_bytes(full["cm"])
+    buf = torch.zeros(32 * rb, dtype=torch.uint8, device=cuda)
+    cnt = torch.zeros(4, dtype=torch.int32, device=cuda)
+    eng.set_position(L0, seed0)
+    eng.set_trace(buf, cnt)
+    try:
+        out = torch.zeros(16, dtype=torch.int32, device=cuda)
+        st = dv.Stats()
+        eng.generate(dv.DecodeCfg(16, 0.9, dv.MODE_THRESHOLD, 1, 16, 1), out, st)
+        eng.check()
+    finally:
+        eng.set_trace(None, None)
+    recs = parse_trace(buf.cpu().numpy(), int(cnt[0].item()), rb, dims.hidden, True)
+    assert len(recs) == st.nfe
+    k_gpu = [f64(full["kc"][l, 0, :, :L0]) for l in range(dims.n_layers)]
+    v_gpu = [f64(full["vc"][l, 0, :, :, :L0]).transpose(0, 2, 1) for l in range(dims.n_layers)]
+
+    vis_t, vis, ids = gen.decode_context(dims, SEED, N_VIS, N_PROMPT)
+    E = gen.embedding_weight(dims, SEED)[1]
+    W = gen.lm_head_weight(dims, SEED)[1]
+    m = O.OracleModel(O.dims_from(dims), weights={"embed": E, "lm_head": W}, bf16=True, Lmax=L0 + 16)
+    ctx = np.concatenate([vis.astype(np.float64), m.embed(ids)])
+    passes = [(ctx, 0, L0)] + [(m.embed(r.tok_in), r.L, r.n_clean) for r in recs]
+    names = gen.layer_weight_names()
+    xs = layer_major_hidden(m, passes, lambda l: {f"{l}.{k}": gen.layer_weight(dims, SEED, l, k)[1] for k in names})
+    m.L = L0
+    m.last_conf = m.logits_conf(xs[0][-1:])
+    seed_o = int(m.last_conf.top1[0])
+
+    # the prefilled cache of every layer
+    kv = [(_hidden_err_profile(k_gpu[l], m.K[l][:, :L0]), _hidden_err_profile(v_gpu[l], m.V[l][:, :L0]))
+          for l in range(dims.n_layers)]
+    hid = []
+
+    def hidden_check(a, b, what):
+        hid.append((what, _hidden_err_profile(a, b)))
+        assert_bf16_close(a, b, 2e-2, what)
+
+    rp = Replay(m, seed_o, 16, 0.9, decide="gpu", hidden_check=hidden_check, secondary=DELTA, seed_bar=DELTA,
+                hidden_fn=lambda i, r: xs[i + 1])
+    got = rp.threshold(recs, 16)
+    print(f"full size first block: {rp.t}; hidden (max abs, max ulps) {hid}; "
+          f"K/V layer 0 {kv[0]}, layer 35 {kv[-1]}")
+    assert got == out.cpu().numpy().tolist()
+    assert rp.t.ids_exact >= 8 and rp.t.commits_exact > 0, rp.t
+    for l in range(dims.n_layers):
+        assert_bf16_close(k_gpu[l], m.K[l][:, :L0], 2e-2, f"K layer {l}")
+        assert_bf16_close(v_gpu[l], m.V[l][:, :L0], 2e-2, f"V layer {l}")
 
 
 def test_spec_linear_equals_greedy_ar(full):

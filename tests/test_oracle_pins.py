@@ -175,6 +175,8 @@ def test_confidence_matches_full_softmax_and_sort():
     np.testing.assert_allclose(c.p1, ps[:, -1], rtol=1e-12)
     np.testing.assert_allclose(c.p2, ps[:, -2], rtol=1e-12)
     np.testing.assert_array_equal(c.top1, order[:, 0])
+    np.testing.assert_array_equal(c.top2, order[:, 1])
+    np.testing.assert_allclose(c.p2, p[np.arange(6), order[:, 1]], rtol=1e-12)
 
 
 def test_confidence_closed_forms():
@@ -190,6 +192,7 @@ def test_confidence_closed_forms():
     lg = np.array([[1.0, 5.0, 0.0, 5.0, 2.0]])
     c = O.confidence_from_logits(lg)
     assert c.top1[0] == 1 and c.p1[0] <= 0.5 and abs(c.p1[0] - c.p2[0]) < 1e-15
+    assert c.top2[0] == 3   # the other maximum is the runner-up
     # uniform logits: p1 = 1/V
     c = O.confidence_from_logits(np.zeros((1, 256)))
     assert abs(c.p1[0] - 1 / 256) < 1e-15 and c.top1[0] == 0

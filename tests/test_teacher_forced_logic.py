@@ -1,11 +1,13 @@
 """GPU checks whose logic can run on the CPU against stand-ins.
 
-The teacher-forced decode checks run against a stand-in engine: a copy of the oracle whose stored bf16 values are perturbed by about
-5e-7 relative before rounding (the CPU model of the GPU's fp32-sum
-differences), behind the same calls the checks make (prefill, position,
-forward with x_out / advance, set_position, the fused LM head).  This runs
-the checks' own logic -- call order, row-to-position mapping, accepted-prefix
-bookkeeping, tolerances -- before any GPU does.  The TEXT-ONLY attention
+The teacher-forced routing checks run against a stand-in engine: a copy of
+the oracle whose stored bf16 values are perturbed by about 5e-7 relative
+before rounding (the CPU model of the GPU's fp32-sum differences), behind the
+same calls the checks make (prefill, position, forward with x_out / advance,
+TEXT-ONLY forward, set_position, the fused LM head).  This runs the checks'
+own logic -- call order, row-to-position mapping, tolerances -- before any
+GPU does.  (The threshold and speculative decode checks replay the engine's
+own trace; tests/test_decode_replay_logic.py covers their logic.)  The TEXT-ONLY attention
 check runs against a stand-in that addresses memory as the kernel does, from
 the base pointers it is given, so the offset cache views are shown to reach
 exactly the intended slots and to stay inside their buffers."""
@@ -103,37 +105,6 @@ def standin(monkeypatch):
     monkeypatch.setattr(dv, "lmhead_workspace_size", lambda *a: 64)
     monkeypatch.setattr(dv, "lmhead_conf_commit", _lmhead)
     return torch.device("cpu")
-
-
-@pytest.mark.parametrize("seed", [1, 3])
-def test_threshold_check_logic(standin, seed):
-    T.test_bf16_reduced_model_threshold_teacher_forced(standin, seed)
-
-
-@pytest.mark.parametrize("seed", [6, 2])
-def test_speculative_check_logic(standin, seed):
-    T.test_bf16_reduced_model_spec_teacher_forced(standin, seed)
-
-
-def test_speculative_check_catches_a_stale_cache_length(standin, monkeypatch):
-    """An engine that ignores the accepted-prefix update (keeps L after a
-    round) fails the check: its next round runs over the wrong cache slots."""
-    monkeypatch.setattr(_Engine, "set_position", lambda self, L, seed, stream=None: None)
-    with pytest.raises(AssertionError):
-        T.test_bf16_reduced_model_spec_teacher_forced(standin, 6)
-
-
-def test_threshold_check_catches_a_swapped_row_mapping(standin, monkeypatch):
-    """A fused LM head that reports row r's result for position r (no shift)
-    fails the threshold check."""
-    def unshifted(h, w, **kw):
-        _lmhead(h, w, **kw)
-        kw["top1_id"][:] = torch.roll(kw["top1_id"], 1)
-        kw["top1_prob"][:] = torch.roll(kw["top1_prob"], 1)
-
-    monkeypatch.setattr(dv, "lmhead_conf_commit", unshifted)
-    with pytest.raises(AssertionError):
-        T.test_bf16_reduced_model_threshold_teacher_forced(standin, 1)
 
 
 def _attn_by_kernel_addressing(q, out, k, v, *, n_batch, n_rows, n_clean, L, Lmax, Hq, Hkv, D, scale, dtype,

@@ -9,7 +9,11 @@ scratch in one fixed array inside the library instead of a workspace.
 Checked here through the C ABI: two calls in a row (different shapes, the
 second one after the first left its counters and records in the shared
 array) each match the workspace entry point on the same inputs, within the
-LM-head tests' bars; sizes beyond the fixed scratch are refused on the host.
+LM-head tests' bars, the first with certificate anchors taken from the
+oracle's top-1 of a related hidden set so that the certified prefix is not
+trivially empty; sizes beyond the fixed scratch (too many rows, or a
+vocabulary whose scratch layout overflows the array) are refused on the host;
+and a call after a warm-up call leaves the device's free memory unchanged.
 This file is collected last so that a stop-at-first-failure run has already
 run every other test."""
 import numpy as np
@@ -18,6 +22,7 @@ import torch
 
 import block_diffusion_vlm_b200 as dv
 import dvlm_gen as gen
+import oracle as O
 from gpu_util import assert_ok, status, ws_tensor
 
 pytestmark = pytest.mark.gpu
@@ -39,14 +44,17 @@ def _compare(a, b):
 
 
 def _case(cuda, seed, R, H, V, apply_rmsnorm, with_commit, with_cert):
-    (h_t, _), (w_t, _), (h2_t, _) = gen.lmhead_case(seed, R, H, V)
+    (h_t, h1), (w_t, wv), (h2_t, _) = gen.lmhead_case(seed, R, H, V)
     h, w = h2_t.to(cuda), w_t.to(cuda)
     masked0 = torch.from_numpy((np.arange(R) % 5 != 2).astype(np.uint8)).to(cuda)
     tokens0 = torch.arange(R, dtype=torch.int32, device=cuda) + 7
     kw = {}
     if with_cert:
-        kw = dict(anchor_id=torch.from_numpy(gen.uniform_ids(seed, "anchor", R, V)).to(cuda),
-                  anchor_conf=torch.rand(R, generator=torch.Generator().manual_seed(seed)).to(cuda))
+        # anchors: the oracle's top-1 (id, confidence) of the first hidden set,
+        # which the scored set H2 = H1 + 0.5 N(0,1) partly agrees with
+        a = O.lm_head_conf(h1.astype(np.float64), wv.astype(np.float64))
+        kw = dict(anchor_id=torch.from_numpy(a.top1.astype(np.int32)).to(cuda),
+                  anchor_conf=torch.from_numpy(a.p1.astype(np.float32)).to(cuda))
     results = []
     for variant in ("workspace", "static"):
         out = _outputs(R, cuda)
@@ -67,6 +75,8 @@ def _case(cuda, seed, R, H, V, apply_rmsnorm, with_commit, with_cert):
     _compare(a, b)
     if with_cert:
         assert int(ca.item()) == int(cb.item())
+        # rows masked on entry in descending anchor confidence agree for a while
+        assert int(ca.item()) > 0
     if with_commit:
         assert torch.equal(ma, mb) and torch.equal(ta, tb)
 
@@ -87,3 +97,31 @@ def test_static_scratch_refuses_sizes_beyond_its_capacity(cuda):
     with pytest.raises(dv.DvlmError) as ei:
         dv.lmhead_conf_commit_static(h, w, R=R, H=H, V=V, top1_id=torch.zeros(R, dtype=torch.int32, device=cuda))
     assert ei.value.status == 7  # DVLM_ERR_WORKSPACE
+    # R <= 32 but a vocabulary of 2^27 rows: 4 bytes of counters per 128 rows
+    # (4 MiB) plus the per-SM partial tiles overflow the 6 MiB array.  The
+    # weight tensor is real (17 GB, never read: the call is refused on the
+    # host before any launch).
+    R, H, V = 16, 64, 1 << 27
+    h = torch.zeros((R, H), dtype=torch.bfloat16, device=cuda)
+    w = torch.empty((V, H), dtype=torch.bfloat16, device=cuda)
+    with pytest.raises(dv.DvlmError) as ei:
+        dv.lmhead_conf_commit_static(h, w, R=R, H=H, V=V, top1_id=torch.zeros(R, dtype=torch.int32, device=cuda))
+    assert ei.value.status == 7
+    del w
+    torch.cuda.empty_cache()
+
+
+def test_static_scratch_call_leaves_free_memory_unchanged(cuda):
+    R, H, V = 16, 2048, 151936
+    (h_t, _), (w_t, _), _ = gen.lmhead_case(5, R, H, V)
+    h, w = h_t.to(cuda), w_t.to(cuda)
+    out = _outputs(R, cuda)
+    st = status(cuda)
+    dv.lmhead_conf_commit_static(h, w, R=R, H=H, V=V, status=st, **out)   # warm-up
+    assert_ok(st)
+    free0, _ = torch.cuda.mem_get_info()
+    dv.lmhead_conf_commit_static(h, w, R=R, H=H, V=V, status=st, **out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert_ok(st)
+    assert free1 == free0
