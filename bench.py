@@ -143,19 +143,23 @@ def gpu_uuid():
 
 
 # ----------------------------------------------------------------- algorithmic bytes
-def algorithmic_bytes(kind: str, dims, L: int, rows: int = 16) -> float:
+def algorithmic_bytes(kind: str, dims, L: int, rows: int = 16, fp8: bool = False) -> float:
     """Bytes a kernel must move per launch: its weights once, its inputs and
-    outputs once (bf16)."""
+    outputs once (bf16 activations).  fp8: the decoder projections' weights
+    are E4M3 codes (1 byte each) plus one fp32 scale per weight row."""
     H, I, D, Hq, Hkv, V = dims.hidden, dims.inter, dims.head_dim, dims.n_q_heads, dims.n_kv_heads, dims.vocab
     qkv = (Hq + 2 * Hkv) * D
+
+    def w(n_out, n_in):
+        return n_out * n_in + 4 * n_out if fp8 else 2 * n_out * n_in
     if kind == "qkv_gemm":
-        return 2 * (qkv * H + rows * H + rows * qkv)
+        return w(qkv, H) + 2 * (rows * H + rows * qkv)
     if kind == "oproj_gemm":
-        return 2 * (H * Hq * D + rows * Hq * D + 2 * rows * H)
+        return w(H, Hq * D) + 2 * (rows * Hq * D + 2 * rows * H)
     if kind == "gateup_gemm":
-        return 2 * (2 * I * H + rows * H + rows * I)
+        return 2 * w(I, H) + 2 * (rows * H + rows * I)
     if kind == "down_gemm":
-        return 2 * (H * I + rows * I + 2 * rows * H)
+        return w(H, I) + 2 * (rows * I + 2 * rows * H)
     if kind == "lm_head":
         return 2 * (V * H + rows * H)
     if kind == "attention":
@@ -262,6 +266,28 @@ def workload_nfe() -> float | None:
     return None
 
 
+def forward_bytes(dims, fp8: bool) -> float:
+    """Bytes one decode forward streams: every decoder matrix and the LM head
+    (the embedding table is only gathered by row); fp8: E4M3 projection codes
+    plus their per-row fp32 scales, bf16 LM head."""
+    if not fp8:
+        return dims.streamed_params() * 2
+    H, I, D, Hq = dims.hidden, dims.inter, dims.head_dim, dims.n_q_heads
+    per_layer_params = dims.qkv_rows * H + H * Hq * D + 3 * I * H
+    per_layer_rows = dims.qkv_rows + H + 2 * I + H
+    return dims.n_layers * (per_layer_params + 4 * per_layer_rows) + 2 * dims.vocab * H
+
+
+def workload_config(args, world: int) -> dict:
+    """The `config` object both arms report (same workload, same keys)."""
+    c = {"workload": WORKLOAD, "global_batch": world, "seq_len": N_VIS + N_PROMPT + N_NEW,
+         "parallelism": f"replicas x{world}", "mode": args.mode,
+         "l2": "inputs larger than L2 (6.2 GB of weights streamed per forward)"}
+    if getattr(args, "weights", "bf16") != "bf16":
+        c["weights"] = "fp8-w8a8 (E4M3 projections, per-row / per-token scales; bf16 LM head)"
+    return c
+
+
 # ----------------------------------------------------------------- arms
 def run_reference(args, rank, world):
     if rank != 0:
@@ -280,8 +306,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * elapsed / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": N_VIS + N_PROMPT + N_NEW,
-                                            "parallelism": "replicas", "l2": "weights 6.2 GB > L2"},
+            "data": "synthetic", "config": workload_config(args, world),
             "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -300,7 +325,8 @@ def run_ours(args, rank, world, local, pg):
     dm = DeviceModel(dims, SEED, device=dev)
     Lmax = N_VIS + N_PROMPT + N_NEW + 32
     kc, vc = kv_buffers(dims, Lmax, device=dev)
-    cm = dm.c_model()
+    fp8 = args.weights == "fp8"
+    cm = dm.fp8_c_model() if fp8 else dm.c_model()
     ws = torch.zeros((dv.engine_workspace_size(cm, Lmax, BLOCK, N_VIS + N_PROMPT) + 3) // 4, dtype=torch.int32,
                      device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -377,7 +403,7 @@ def run_ours(args, rank, world, local, pg):
     per = {}
     for k, (ms, cnt) in prof.items():
         if cnt:
-            b = algorithmic_bytes(k, dims, L0)
+            b = algorithmic_bytes(k, dims, L0, fp8=fp8)
             per[k] = {"ms_per_launch": ms / cnt, "launches": cnt, "gbs": b / (ms / cnt * 1e-3) / 1e9,
                       "bytes_per_launch": b}
     dom = max((k for k in per if k != "embed"), key=lambda k: per[k]["ms_per_launch"] * per[k]["launches"])
@@ -390,13 +416,11 @@ def run_ours(args, rank, world, local, pg):
                 "nominal_peak": NOMINAL_HBM_GBS}
 
     fwd_ms = sum(v["ms_per_launch"] * v["launches"] for v in per.values())
-    fwd_bytes = dims.streamed_params() * 2
+    fwd_bytes = forward_bytes(dims, fp8)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": N_VIS + N_PROMPT + N_NEW,
-                       "parallelism": f"replicas x{world}", "mode": args.mode,
-                       "l2": "inputs larger than L2 (6.2 GB of weights streamed per forward)"},
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3+bf16" if fp8 else "bf16", "data": "synthetic",
+            "config": workload_config(args, world),
             "roofline": roof(dom), "lmhead": roof("lm_head") if "lm_head" in per else None,
             "gpu_launches": launches, "clocks": clk, "e2e": e2e,
             "decode": {"nfe_per_step": nfe, "tokens_per_nfe": N_NEW / nfe, "commit_hist": hist,
@@ -416,7 +440,7 @@ def run_ours(args, rank, world, local, pg):
         torch.cuda.synchronize(dev)
         line["spec_linear"] = {"tokens_per_s": N_NEW / (ev0.elapsed_time(ev1) / 1000.0), "nfe": st.nfe,
                                "accept_hist": list(st.accept_hist)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = cpu_baseline(nfe)
     eng.close()
     if rank == 0:
@@ -576,6 +600,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--mode", choices=["threshold", "spec", "ar"], default="threshold")
+    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: the W8A8 decoder (E4M3 projections quantised from the same bf16 weights)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the extra speculative-mode run")
     ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 LIB_PATH = os.path.join(PKG, "libdvlm.so")
 HEADER = os.path.join(ROOT, "include", "dvlm.h")
 
-DVLM_BF16, DVLM_FP32 = 0, 1
+DVLM_BF16, DVLM_FP32, DVLM_FP8_W8A8 = 0, 1, 2
 MODE_THRESHOLD, MODE_SPEC_LINEAR, MODE_AR = 0, 1, 2
 HIST = 17
 
@@ -57,7 +57,9 @@ class Model(ctypes.Structure):
                 ("vocab", ctypes.c_int), ("mask_id", ctypes.c_int), ("rope_base", ctypes.c_float),
                 ("eps", ctypes.c_float), ("dtype", ctypes.c_int), ("embed", ctypes.c_void_p),
                 ("wqkv", ctypes.c_void_p), ("wo", ctypes.c_void_p), ("wgate", ctypes.c_void_p),
-                ("wup", ctypes.c_void_p), ("wdown", ctypes.c_void_p), ("lm_head", ctypes.c_void_p)]
+                ("wup", ctypes.c_void_p), ("wdown", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("sqkv", ctypes.c_void_p), ("so", ctypes.c_void_p), ("sgate", ctypes.c_void_p),
+                ("sup", ctypes.c_void_p), ("sdown", ctypes.c_void_p)]
 
 
 class DecodeCfg(ctypes.Structure):
@@ -116,6 +118,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_profile_forward": (_i, [_vp, _vp, _vp, _i, _i, _i, ctypes.POINTER(ctypes.c_float),
                                       ctypes.POINTER(_i), _vp]),
         "dvlm_engine_trace_record_bytes": (_sz, [ctypes.POINTER(Model)]),
+        "dvlm_quantize_rows_e4m3": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
         "dvlm_engine_set_trace": (_i, [_vp, _vp, _sz, _vp]),
     }
     for name, (res, args) in sigs.items():
@@ -217,16 +220,24 @@ def spec_verify_accept(*, draft_ids, b, B, V, accept_len, verify_logits=None, ve
            "dvlm_spec_verify_accept")
 
 
+def quantize_rows_e4m3(a, codes, scales, *, rows, K, stream=None) -> None:
+    """Per-row FP8 E4M3 codes and scales of a bf16 matrix (dvlm_quantize_rows_e4m3)."""
+    _check(lib().dvlm_quantize_rows_e4m3(ptr(a), int(rows), int(K), ptr(codes), ptr(scales), stream_handle(stream)),
+           "dvlm_quantize_rows_e4m3")
+
+
 def selftest_wait_timeout(budget_cycles: int, status, gave_up, stream=None) -> None:
     _check(lib().dvlm_selftest_wait_timeout(int(budget_cycles), ptr(status), ptr(gave_up), stream_handle(stream)),
            "dvlm_selftest_wait_timeout")
 
 
 # ---------------------------------------------------------------- engine
-def make_model(dims, *, embed, wqkv, wo, wgate, wup, wdown, lm_head, dtype) -> Model:
+def make_model(dims, *, embed, wqkv, wo, wgate, wup, wdown, lm_head, dtype, scales=None) -> Model:
+    """scales: (sqkv, so, sgate, sup, sdown) per-row fp32 scales of an FP8 W8A8 model."""
+    sc = scales or (None,) * 5
     return Model(dims.n_layers, dims.hidden, dims.n_q_heads, dims.n_kv_heads, dims.head_dim, dims.inter,
                  dims.vocab, dims.mask_id, float(dims.rope_base), float(dims.eps), dtype, ptr(embed), ptr(wqkv),
-                 ptr(wo), ptr(wgate), ptr(wup), ptr(wdown), ptr(lm_head))
+                 ptr(wo), ptr(wgate), ptr(wup), ptr(wdown), ptr(lm_head), *(ptr(t) for t in sc))
 
 
 def engine_workspace_size(model: Model, Lmax: int, max_block: int, max_ctx: int) -> int:

@@ -93,7 +93,8 @@ bool model_ok(const dvlm_model* m) {
   if (m->n_q_heads % m->n_kv_heads || m->head_dim % 2) return false;
   if (m->mask_id < 0 || m->mask_id >= m->vocab) return false;
   if (!(m->eps > 0.f) || !(m->rope_base > 0.f)) return false;
-  if (m->dtype != DVLM_BF16 && m->dtype != DVLM_FP32) return false;
+  if (m->dtype != DVLM_BF16 && m->dtype != DVLM_FP32 && m->dtype != DVLM_FP8_W8A8) return false;
+  if (m->dtype == DVLM_FP8_W8A8 && !(m->sqkv && m->so && m->sgate && m->sup && m->sdown)) return false;
   return m->embed && m->wqkv && m->wo && m->wgate && m->wup && m->wdown && m->lm_head;
 }
 
@@ -104,6 +105,9 @@ dvlm_status bf16_model_supported(const dvlm_model* m) {
   const void* p[] = {m->embed, m->wqkv, m->wo, m->wgate, m->wup, m->wdown, m->lm_head};
   for (const void* q : p)
     if (!al16(q)) return DVLM_ERR_INVALID_ARG;
+  // W8A8: 128-wide k blocks of E4M3 codes in every projection
+  if (m->dtype == DVLM_FP8_W8A8 && (m->inter % 128 || (m->n_q_heads * m->head_dim) % 128 || m->hidden % 128))
+    return DVLM_ERR_UNSUPPORTED;
   return DVLM_OK;
 }
 
@@ -305,12 +309,21 @@ dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const int32_t* ve
                                      n_layers, Hkv, D, Lmax, dev_status, cs(stream)));
 }
 
+// ------------------------------------------------------------ FP8 weights
+dvlm_status dvlm_quantize_rows_e4m3(const void* a, int rows, int K, uint8_t* codes, float* scales,
+                                    dvlm_stream stream) {
+  if (!a || !codes || !scales) return DVLM_ERR_INVALID_ARG;
+  if (rows < 1 || K < 1) return DVLM_ERR_SHAPE;
+  return cuda_status(launch_quantize_rows_e4m3(static_cast<const bf16*>(a), rows, K, codes, scales, cs(stream)));
+}
+
 // ------------------------------------------------------------ engine
 size_t dvlm_engine_workspace_size(const dvlm_model* m, int Lmax, int max_block, int max_ctx) {
   if (!model_ok(m) || Lmax < 1 || max_block < 1 || max_block > kNT || max_ctx < 0) return 0;
   dvlm_engine tmp;
   tmp.m = *m;
-  tmp.bf16 = m->dtype == DVLM_BF16;
+  tmp.bf16 = m->dtype != DVLM_FP32;
+  tmp.fp8 = m->dtype == DVLM_FP8_W8A8;
   tmp.Lmax = Lmax;
   tmp.max_block = max_block;
   tmp.max_ctx = max_ctx;
@@ -323,7 +336,7 @@ dvlm_status dvlm_engine_create(const dvlm_model* m, void* k_cache, void* v_cache
   *out = nullptr;
   if (!model_ok(m) || !k_cache || !v_cache) return DVLM_ERR_INVALID_ARG;
   if (Lmax < 1 || max_block < 1 || max_block > kNT || max_ctx < 0) return DVLM_ERR_SHAPE;
-  if (m->dtype == DVLM_BF16) {
+  if (m->dtype != DVLM_FP32) {
     const dvlm_status st = bf16_model_supported(m);
     if (st != DVLM_OK) return st;
     if (Lmax % 8 || !al16(k_cache) || !al16(v_cache)) return DVLM_ERR_INVALID_ARG;
@@ -336,7 +349,8 @@ dvlm_status dvlm_engine_create(const dvlm_model* m, void* k_cache, void* v_cache
   dvlm_engine* e = new (std::nothrow) dvlm_engine();
   if (!e) return DVLM_ERR_CUDA;
   e->m = *m;
-  e->bf16 = m->dtype == DVLM_BF16;
+  e->bf16 = m->dtype != DVLM_FP32;
+  e->fp8 = m->dtype == DVLM_FP8_W8A8;
   e->Lmax = Lmax;
   e->max_block = max_block;
   e->max_ctx = max_ctx;
@@ -619,7 +633,7 @@ dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value) 
 
 size_t dvlm_engine_trace_record_bytes(const dvlm_model* m) {
   if (!model_ok(m)) return 0;
-  return trace_record_bytes(m->hidden, m->dtype == DVLM_BF16);
+  return trace_record_bytes(m->hidden, m->dtype != DVLM_FP32);
 }
 
 dvlm_status dvlm_engine_set_trace(dvlm_engine* e, void* buf, size_t bytes, int32_t* count) {

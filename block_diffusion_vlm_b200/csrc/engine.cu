@@ -125,7 +125,8 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->stage_vis = c.take<void>(static_cast<size_t>(std::max(e->max_ctx, 1)) * H * es);
   e->stage_ids = c.take<int32_t>(std::max(e->max_ctx, 1) * 4);
   e->stage_out = c.take<int32_t>(static_cast<size_t>(e->Lmax) * 4);
-  if (e->bf16 && e->max_ctx > 0) {
+  if (e->fp8) e->amax_act = c.take<float>(static_cast<size_t>(I / 64) * kNT * 4);
+  if (e->bf16 && !e->fp8 && e->max_ctx > 0) {
     const size_t C = static_cast<size_t>(e->max_ctx);
     e->px = c.take<void>(C * H * 2);
     e->pq = c.take<void>(C * HD * 2);
@@ -149,11 +150,19 @@ static bool build_maps(dvlm_engine* e) {
   const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads, L = m.n_layers;
   const int qkv_rows = (Hq + 2 * Hkv) * D;
   bool ok = true;
-  ok &= make_tmap_2d(&e->tm_wqkv, m.wqkv, H, static_cast<uint64_t>(L) * qkv_rows, H * 2, 64, 128);
-  ok &= make_tmap_2d(&e->tm_wo, m.wo, Hq * D, static_cast<uint64_t>(L) * H, Hq * D * 2, 64, 128);
-  ok &= make_tmap_2d(&e->tm_wg, m.wgate, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
-  ok &= make_tmap_2d(&e->tm_wu, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
-  ok &= make_tmap_2d(&e->tm_wd, m.wdown, I, static_cast<uint64_t>(L) * H, static_cast<uint64_t>(I) * 2, 64, 128);
+  if (e->fp8) {  // E4M3 codes: 128-byte (128 k) boxes
+    ok &= make_tmap_2d_u8(&e->tm_wqkv, m.wqkv, H, static_cast<uint64_t>(L) * qkv_rows, H, 128, 128);
+    ok &= make_tmap_2d_u8(&e->tm_wo, m.wo, Hq * D, static_cast<uint64_t>(L) * H, Hq * D, 128, 128);
+    ok &= make_tmap_2d_u8(&e->tm_wg, m.wgate, H, static_cast<uint64_t>(L) * I, H, 128, 64);
+    ok &= make_tmap_2d_u8(&e->tm_wu, m.wup, H, static_cast<uint64_t>(L) * I, H, 128, 64);
+    ok &= make_tmap_2d_u8(&e->tm_wd, m.wdown, I, static_cast<uint64_t>(L) * H, I, 128, 128);
+  } else {
+    ok &= make_tmap_2d(&e->tm_wqkv, m.wqkv, H, static_cast<uint64_t>(L) * qkv_rows, H * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_wo, m.wo, Hq * D, static_cast<uint64_t>(L) * H, Hq * D * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_wg, m.wgate, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
+    ok &= make_tmap_2d(&e->tm_wu, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 64);
+    ok &= make_tmap_2d(&e->tm_wd, m.wdown, I, static_cast<uint64_t>(L) * H, static_cast<uint64_t>(I) * 2, 64, 128);
+  }
   ok &= make_tmap_2d(&e->tm_lm, m.lm_head, H, m.vocab, H * 2, 64, 128);
   ok &= make_tmap_2d(&e->tm_x, e->x, H, kNT, H * 2, 64, kNT);
   ok &= make_tmap_2d(&e->tm_ao, e->attn_o, Hq * D, kNT, Hq * D * 2, 64, kNT);
@@ -162,7 +171,7 @@ static bool build_maps(dvlm_engine* e) {
   ok &= make_tmap_2d(&e->tm_k, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 64);
   ok &= make_tmap_2d(&e->tm_v, e->vc, e->Lmax, static_cast<uint64_t>(L) * Hkv * D,
                      static_cast<uint64_t>(e->Lmax) * 2, 64, 128);
-  if (e->max_ctx > 0) {
+  if (e->max_ctx > 0 && !e->fp8) {
     const uint64_t C = static_cast<uint64_t>(e->max_ctx);
     ok &= make_tmap_2d(&e->tm_px, e->px, H, C, H * 2, 64, 128);
     ok &= make_tmap_2d(&e->tm_pq, e->pq, Hq * D, C, Hq * D * 2, 64, 128);
@@ -256,12 +265,25 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
     ea.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
     T0(K_QKV);
-    if (e->s_qkv > 0)
+    if (e->fp8) {  // W8A8 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]
+      ea.q_src = x;
+      ea.q_ld = H;
+      ea.q_K = H;
+      ea.rms_input = 1;
+      ea.amax_in = nullptr;
+      ea.wscale = m.sqkv;
+      if (e->s_qkv > 0)
+        DVLM_CK(launch_gemm_cl_fp8(e->tm_wqkv, qkv_rows / 128, H / 128, e->s_qkv, l * qkv_rows, ea, pdl, s, 5));
+      else
+        DVLM_CK(launch_gemm_ws_fp8(e->tm_wqkv, e->tm_wqkv, qkv_rows / 128, H / 128,
+                                   ws_ctas(e, (qkv_rows / 128) * (H / 128)), l * qkv_rows, ea, pdl, s));
+    } else if (e->s_qkv > 0) {
       DVLM_CK(launch_gemm_cl(kNT, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, e->s_qkv, l * qkv_rows, ea, pdl, s,
                              5));
-    else
+    } else {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
                              ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s, 5));
+    }
     T1(K_QKV);
     AttnArgs aa{};
     aa.n_rows = f.n_rows;
@@ -289,11 +311,24 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.resid_ld = H;
     ea.ssq_out = e->ssq;
     T0(K_OPROJ);
-    if (e->s_o > 0)
+    if (e->fp8) {
+      ea.q_src = static_cast<bf16*>(e->attn_o);
+      ea.q_ld = Hq * D;
+      ea.q_K = Hq * D;
+      ea.rms_input = 0;
+      ea.amax_in = nullptr;
+      ea.wscale = m.so;
+      if (e->s_o > 0)
+        DVLM_CK(launch_gemm_cl_fp8(e->tm_wo, H / 128, Hq * D / 128, e->s_o, l * H, ea, pdl, s, 5));
+      else
+        DVLM_CK(launch_gemm_ws_fp8(e->tm_wo, e->tm_wo, H / 128, Hq * D / 128, ws_ctas(e, (H / 128) * (Hq * D / 128)),
+                                   l * H, ea, pdl, s));
+    } else if (e->s_o > 0) {
       DVLM_CK(launch_gemm_cl(kNT, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, e->s_o, l * H, ea, pdl, s, 5));
-    else
+    } else {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64,
                              ws_ctas(e, (H / 128) * (Hq * D / 64)), l * H, ea, pdl, s, 5));
+    }
     T1(K_OPROJ);
     n_ssq = (H / 128) * (e->s_o > 0 ? e->s_o : 1);
     ea.epi = EPI_SWIGLU;
@@ -301,19 +336,46 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.out = static_cast<bf16*>(e->act);
     ea.out_ld = I;
     T0(K_GATEUP);
-    const long long gu_units = static_cast<long long>(I / 64) * (H / 64);
-    const int gu_ctas = static_cast<int>(std::min<long long>(gu_units, static_cast<long long>(e->gu_cps) * e->sm));
-    DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, gu_ctas,
-                           l * I, ea, pdl, s, e->gu_stages));
+    if (e->fp8) {
+      ea.q_src = x;
+      ea.q_ld = H;
+      ea.q_K = H;
+      ea.rms_input = 1;
+      ea.amax_in = nullptr;
+      ea.wscale = m.sgate;
+      ea.wscale2 = m.sup;
+      ea.amax_out = e->amax_act;
+      const long long units = static_cast<long long>(I / 64) * (H / 128);
+      DVLM_CK(launch_gemm_ws_fp8(e->tm_wg, e->tm_wu, I / 64, H / 128,
+                                 static_cast<int>(std::min<long long>(units, e->sm)), l * I, ea, pdl, s));
+    } else {
+      const long long gu_units = static_cast<long long>(I / 64) * (H / 64);
+      const int gu_ctas = static_cast<int>(std::min<long long>(gu_units, static_cast<long long>(e->gu_cps) * e->sm));
+      DVLM_CK(launch_gemm_ws(kNT, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, gu_ctas,
+                             l * I, ea, pdl, s, e->gu_stages));
+    }
     T1(K_GATEUP);
     ea.epi = EPI_RESID;
     T0(K_DOWN);
-    if (e->s_down > 0)
+    if (e->fp8) {
+      ea.q_src = static_cast<bf16*>(e->act);
+      ea.q_ld = I;
+      ea.q_K = I;
+      ea.rms_input = 0;
+      ea.amax_in = e->amax_act;
+      ea.n_amax = I / 64;
+      ea.wscale = m.sdown;
+      ea.wscale2 = nullptr;
+      ea.amax_out = nullptr;
+      if (e->s_down <= 0) return cudaErrorInvalidValue;  // the fp8 down projection runs split-K in clusters
+      DVLM_CK(launch_gemm_cl_fp8(e->tm_wd, H / 128, I / 128, e->s_down, l * H, ea, pdl, s, e->down_stages));
+    } else if (e->s_down > 0) {
       DVLM_CK(launch_gemm_cl(kNT, e->tm_wd, e->tm_act, H / 128, I / 64, e->s_down, l * H, ea, pdl, s,
                              e->down_stages));
-    else
+    } else {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64,
                              ws_ctas(e, (H / 128) * (I / 64)), l * H, ea, pdl, s, e->down_stages));
+    }
     T1(K_DOWN);
     n_ssq = (H / 128) * (e->s_down > 0 ? e->s_down : 1);
   }
@@ -399,7 +461,7 @@ static cudaError_t fwd_f32(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
 bool prefill_gemm_supported(const dvlm_engine* e) {
   const dvlm_model& m = e->m;
   const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
-  return e->bf16 && e->max_ctx > 0 && m.head_dim == 128 && m.hidden % 256 == 0 && m.inter % 128 == 0 &&
+  return e->bf16 && !e->fp8 && e->max_ctx > 0 && m.head_dim == 128 && m.hidden % 256 == 0 && m.inter % 128 == 0 &&
          qkv_rows % 256 == 0 && (m.n_q_heads * m.head_dim) % 64 == 0;
 }
 
@@ -723,6 +785,7 @@ cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* co
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
   const dvlm_model& m = e->m;
   const std::string n(name);
+  if (e->fp8 && n != "pdl" && n != "attn_cluster") return DVLM_ERR_UNSUPPORTED;
   // every cluster of the projection resident at once (one wave)
   const int qkv_tiles = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim / 128, h_tiles = m.hidden / 128;
   auto cluster_ok = [&](int epi, int S, int stages, int n_tiles) {
@@ -804,10 +867,26 @@ static int pick_cluster(dvlm_engine* e, int epi, int n_tiles, int kb, int stages
   return 0;
 }
 
+// Same for the W8A8 kernels (kb = 128-wide k blocks; each CTA's share of them
+// must fit its activation-code buffer of 16 blocks).
+static int pick_cluster_fp8(dvlm_engine* e, int epi, int n_tiles, int kb, int stages) {
+  for (int S = std::min(16, std::min(kb, e->sm / std::max(1, n_tiles))); S >= 2; --S)
+    if ((kb + S - 1) / S <= 16 && gemm_cl_max_clusters_fp8(epi, S, stages) >= n_tiles) return S;
+  return 0;
+}
+
 void engine_plan(dvlm_engine* e) {
   if (!e->bf16) return;
   const dvlm_model& m = e->m;
   const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
+  if (e->fp8) {
+    e->s_qkv = pick_cluster_fp8(e, EPI_QKV, qkv_rows / 128, m.hidden / 128, 5);
+    e->s_o = pick_cluster_fp8(e, EPI_RESID, m.hidden / 128, m.n_q_heads * m.head_dim / 128, 5);
+    e->s_down = pick_cluster_fp8(e, EPI_RESID, m.hidden / 128, m.inter / 128, e->down_stages);
+    e->attn_cs = attn_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
+    e->prefill_gemm = false;
+    return;
+  }
   e->s_qkv = pick_cluster(e, EPI_QKV, qkv_rows / 128, m.hidden / 64, 5);
   e->s_o = pick_cluster(e, EPI_RESID, m.hidden / 128, m.n_q_heads * m.head_dim / 64, 5);
   e->s_down = pick_cluster(e, EPI_RESID, m.hidden / 128, m.inter / 64, e->down_stages);

@@ -78,6 +78,7 @@ inline int launches_per_forward(int n_layers) { return 2 + 5 * n_layers; }
 struct dvlm_engine {
   dvlm_model m{};
   bool bf16 = true;
+  bool fp8 = false;                     // FP8 W8A8 projections (bf16 everywhere else)
   int Lmax = 0, max_block = 0, max_ctx = 0;
   void* kc = nullptr;
   void* vc = nullptr;
@@ -126,6 +127,7 @@ struct dvlm_engine {
   void* pao = nullptr;           // [max_ctx][Hq*D] attention output
   void* pact = nullptr;          // [max_ctx][I] SwiGLU activation
   float* pssq = nullptr;         // [H/128][max_ctx] sums of squares
+  float* amax_act = nullptr;     // fp8: [I/64][NT] largest |SwiGLU activation| per gate/up tile
   // fp32 path scratch
   float* f_y = nullptr;          // [NT][max(qkv_rows, H)]
   float* f_r = nullptr;          // [NT]

@@ -19,23 +19,33 @@
 
 namespace dvlm {
 
-template <int NT, int STAGES>
+// Activation code blocks an fp8 CTA can hold (its k range, 128 wide each).
+constexpr int kMaxFp8Blocks = 16;
+
+template <int NT, int STAGES, bool FP8 = false>
 struct GemmSmem {
   static constexpr int kA = 0;
   static constexpr int kB = kA + STAGES * kATileBytes;
-  static constexpr int kE = kB + STAGES * NT * 128;
+  static constexpr int kE = kB + (FP8 ? kMaxFp8Blocks : STAGES) * NT * 128;
   static constexpr int kR = kE + 128 * (NT + 1) * 4;
-  static constexpr int kBar = kR + 32 * 4;
-  static constexpr int kMisc = kBar + (2 * STAGES + 4) * 8;
+  static constexpr int kAt = kR + 32 * 4;  // fp8: token scales [32], quantisation multipliers [32], amax [32]
+  static constexpr int kBar = kAt + 3 * 32 * 4;
+  static constexpr int kMisc = kBar + (2 * STAGES + 5) * 8;
   static constexpr int kTotal = kMisc + 64 + 1024;  // + alignment slack
 };
 
-template <int NT, int STAGES, int EPI>
+// Per-row scale of an E4M3 weight tile row (absolute weight row index).
+__device__ __forceinline__ float fp8_row_scale(const GemmEpi& ea, bool split, int a_row_base, int T, int row) {
+  if (split) return row < 64 ? ea.wscale[a_row_base + T * 64 + row] : ea.wscale2[a_row_base + T * 64 + row - 64];
+  return ea.wscale[a_row_base + T * 128 + row];
+}
+
+template <int NT, int STAGES, int EPI, bool FP8 = false>
 __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     gemm_ws_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
                    const __grid_constant__ CUtensorMap mapB, const SkSched sc, const int a_row_base,
                    const GemmEpi ea) {
-  using S = GemmSmem<NT, STAGES>;
+  using S = GemmSmem<NT, STAGES, FP8>;
   constexpr int TMC = tmem_cols_for<NT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -47,12 +57,22 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
+  uint64_t* b_ready = acce + 2;  // fp8: the activation codes are in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMisc);
   int* sflag = reinterpret_cast<int*>(smem + S::kMisc + 4);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + S::kMisc + 8);
+  float* sAt = reinterpret_cast<float*>(smem + S::kAt);
+  float* sQm = sAt + 32;
+  unsigned* sAmax = reinterpret_cast<unsigned*>(sAt + 64);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+  // fp8: 128-wide k blocks whose activation codes this CTA needs
+  int kb_lo = 0, kb_hi = sc.kb;
+  if (FP8 && u1 > u0 && u0 / sc.kb == (u1 - 1) / sc.kb) {
+    kb_lo = static_cast<int>(u0 % sc.kb);
+    kb_hi = static_cast<int>((u1 - 1) % sc.kb) + 1;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -63,6 +83,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
       mbar_init(&accf[b], 2);
       mbar_init(&acce[b], 4);
     }
+    mbar_init(b_ready, 1);
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapA);
@@ -80,11 +101,12 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
-      ws_producer<NT, STAGES, EPI == EPI_SWIGLU>(&mapA, &mapA2, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base,
-                                                 0, ea.status, sabort);
+      ws_producer<NT, STAGES, EPI == EPI_SWIGLU, FP8>(&mapA, &mapA2, &mapB, sA, sB, full, empty, sc, u0, u1,
+                                                      a_row_base, 0, ea.status, sabort);
   } else if (warp == 1 || warp == kMmaWarp2) {
     if (lane == 0 && u1 > u0)
-      ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort, warp == 1 ? 0 : 1);
+      ws_mma<NT, STAGES, FP8>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort,
+                              warp == 1 ? 0 : 1, b_ready, kb_lo);
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
@@ -102,6 +124,9 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
       }
       named_bar_sync(1, 128);
     }
+    if (FP8)
+      fp8_quantize_activations<NT>(et, ea.q_src, ea.q_ld, ea.q_K, ea.n_rows, ea.rms_input ? sR : nullptr,
+                                   ea.amax_in, ea.n_amax, kb_lo, kb_hi, sB, sAt, sQm, b_ready);
     int L0 = 0;
     if (EPI == EPI_QKV) L0 = ea.d_len ? *ea.d_len : ea.L_static;
     // A tile split over CTAs pf < ... < pl is finished by pf, which streams
@@ -171,6 +196,11 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 #pragma unroll
         for (int t = 0; t < NT; ++t) v[t] += o[t];
       }
+      if (FP8) {  // W8A8 dequantisation: weight row scale x token scale
+        const float sr = fp8_row_scale(ea, EPI == EPI_SWIGLU, a_row_base, T, row);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) v[t] *= sr * sAt[t];
+      }
 
       if (EPI == EPI_RESID) {
         const int col = T * 128 + row;
@@ -195,7 +225,8 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
         named_bar_sync(1, 128);
       } else {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) sE[row * (NT + 1) + t] = v[t] * sR[t];
+        for (int t = 0; t < NT; ++t) sE[row * (NT + 1) + t] = FP8 ? v[t] : v[t] * sR[t];
+        if (FP8 && EPI == EPI_SWIGLU && et < NT) sAmax[et] = 0u;
         named_bar_sync(1, 128);
         const int j = et & 63;
         const int half = et >> 6;
@@ -205,7 +236,13 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
             const float g = sE[j * (NT + 1) + t];
             const float up = sE[(j + 64) * (NT + 1) + t];
             const float a = g / (1.0f + expf(-g)) * up;
-            ea.out[static_cast<size_t>(t) * ea.out_ld + T * 64 + j] = __float2bfloat16_rn(a);
+            const bf16 ab = __float2bfloat16_rn(a);
+            ea.out[static_cast<size_t>(t) * ea.out_ld + T * 64 + j] = ab;
+            if (FP8) atomicMax(&sAmax[t], __float_as_uint(fabsf(__bfloat162float(ab))));
+          }
+          if (FP8) {
+            named_bar_sync(1, 128);
+            if (et < NT) ea.amax_out[T * NT + et] = __uint_as_float(sAmax[et]);
           }
         } else {  // EPI_QKV, one head (128 rows) per tile
           const int nq = ea.n_q_heads, nkv = ea.n_kv_heads;
@@ -259,24 +296,25 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 // shared memory and every CTA finishes a slice of the tile's rows, summing
 // the partials in rank order (deterministic; each token column's arithmetic
 // is independent of how many rows the step has).
-template <int NT, int STAGES>
+template <int NT, int STAGES, bool FP8 = false>
 struct ClSmem {
   static constexpr int kA = 0;
   static constexpr int kB = kA + STAGES * kATileBytes;
-  static constexpr int kSend = kB + STAGES * NT * 128;  // this CTA's partial tile [128][NT] fp32
+  static constexpr int kSend = kB + (FP8 ? kMaxFp8Blocks : STAGES) * NT * 128;  // partial tile [128][NT] fp32
   static constexpr int kRecv = kSend + 128 * NT * 4;    // slices received [S][rows][NT] (<= 160 rows)
   static constexpr int kQ = kRecv + 160 * NT * 4;       // squares of this CTA's rows [64][NT+1]
   static constexpr int kR = kQ + 64 * (NT + 1) * 4;     // rmsnorm factors [NT]
-  static constexpr int kBar = kR + 32 * 4;
-  static constexpr int kMisc = kBar + (2 * STAGES + 5) * 8;
+  static constexpr int kAt = kR + 32 * 4;               // fp8: token scales [32], multipliers [32]
+  static constexpr int kBar = kAt + 2 * 32 * 4;
+  static constexpr int kMisc = kBar + (2 * STAGES + 6) * 8;
   static constexpr int kTotal = kMisc + 64 + 1024;
 };
 
-template <int NT, int STAGES, int EPI>
+template <int NT, int STAGES, int EPI, bool FP8 = false>
 __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     gemm_cl_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const int kb,
                    const int S, const int a_row_base, const GemmEpi ea) {
-  using Sm = ClSmem<NT, STAGES>;
+  using Sm = ClSmem<NT, STAGES, FP8>;
   constexpr int TMC = tmem_cols_for<NT>();
   constexpr int PS = NT + 1;
   extern __shared__ uint8_t smem_raw[];
@@ -292,8 +330,11 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
   uint64_t* recv_full = acce + 2;  // every cluster CTA's slice of this CTA's rows landed
+  uint64_t* b_ready = recv_full + 1;  // fp8: the activation codes are in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Sm::kMisc);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + Sm::kMisc + 8);
+  float* sAt = reinterpret_cast<float*>(smem + Sm::kAt);
+  float* sQm = sAt + 32;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = static_cast<int>(cluster_ctarank());
@@ -326,6 +367,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
       mbar_init(&acce[b], 4);
     }
     mbar_init(recv_full, 1);
+    mbar_init(b_ready, 1);
     *sabort = 0;
     fence_mbar_init();
     mbar_arrive_expect_tx(recv_full, static_cast<uint32_t>(S * kPieces * myn * NT * 4));
@@ -346,13 +388,15 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 
   const int et = threadIdx.x - 64;  // epilogue thread 0..127 (warps 2..5)
   float pre_a[kMaxPer], pre_b[kMaxPer];
+  const int kb_lo = c * kb / S, kb_hi = (c + 1) * kb / S;  // fp8: this CTA's k blocks
   if (warp == 0) {
     if (lane == 0 && u1 > u0)
-      ws_producer<NT, STAGES, false>(&mapA, &mapA, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base, 0, ea.status,
-                                     sabort);
+      ws_producer<NT, STAGES, false, FP8>(&mapA, &mapA, &mapB, sA, sB, full, empty, sc, u0, u1, a_row_base, 0,
+                                          ea.status, sabort);
   } else if (warp == 1 || warp == kMmaWarp2) {
     if (lane == 0 && u1 > u0)
-      ws_mma<NT, STAGES>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort, warp == 1 ? 0 : 1);
+      ws_mma<NT, STAGES, FP8>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ea.status, sabort,
+                              warp == 1 ? 0 : 1, b_ready, kb_lo);
   } else {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -365,6 +409,9 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
       for (int p = 0; p < ea.n_ssq; ++p) s2 += ea.ssq_in[p * NT + et];
       sR[et] = 1.0f / sqrtf(s2 * ea.inv_h + ea.eps);
     }
+    if (FP8)
+      fp8_quantize_activations<NT>(et, ea.q_src, ea.q_ld, ea.q_K, ea.n_rows, ea.rms_input ? sR : nullptr,
+                                   ea.amax_in, ea.n_amax, kb_lo, kb_hi, sB, sAt, sQm, b_ready);
     // Operands of this thread's share of the slice epilogue that do not
     // depend on the product, fetched while the mainloop streams: the residual
     // entries (RESID) or the RoPE rotation (QKV).
@@ -441,7 +488,8 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
         const int it = et + 128 * k;
         if (it >= myn * NT) break;
         const int rl = it / NT, t = it % NT;
-        const float y = got ? part_sum(rl, t) : 0.f;
+        float y = got ? part_sum(rl, t) : 0.f;
+        if (FP8) y *= ea.wscale[a_row_base + T * 128 + my0 + rl] * sAt[t];
         float sq = 0.f;
         if (t < ea.n_rows) {
           const float xn = bf16_round_f(pre_a[k] + y);
@@ -466,8 +514,10 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
         if (it >= myn * NT) break;
         const int jl = it / NT, t = it % NT;
         const int j = my0 + jl;
-        const float x1 = (got ? part_sum(jl, t) : 0.f) * sR[t];
-        const float x2 = (got ? part_sum(myn + jl, t) : 0.f) * sR[t];
+        const float f1 = FP8 ? ea.wscale[a_row_base + T * 128 + j] * sAt[t] : sR[t];
+        const float f2 = FP8 ? ea.wscale[a_row_base + T * 128 + j + 64] * sAt[t] : sR[t];
+        const float x1 = (got ? part_sum(jl, t) : 0.f) * f1;
+        const float x2 = (got ? part_sum(myn + jl, t) : 0.f) * f2;
         if (t >= ea.n_rows) continue;
         if (T < nq + nkv) {
           const float co = pre_a[k], si = pre_b[k];
@@ -494,11 +544,11 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
   }
 }
 
-template <int NT, int ST, int EPI>
+template <int NT, int ST, int EPI, bool FP8 = false>
 static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
                               const SkSched& sc, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
-  using S = GemmSmem<NT, ST>;
-  auto kern = gemm_ws_kernel<NT, ST, EPI>;
+  using S = GemmSmem<NT, ST, FP8>;
+  auto kern = gemm_ws_kernel<NT, ST, EPI, FP8>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
@@ -518,11 +568,11 @@ static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2,
   return cudaLaunchKernelEx(&cfg, kern, mapA, mapA2, mapB, sc, a_row_base, ea);
 }
 
-template <int NT, int ST, int EPI>
+template <int NT, int ST, int EPI, bool FP8 = false>
 static cudaError_t launch_cl(const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
                              int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
-  using Sm = ClSmem<NT, ST>;
-  auto kern = gemm_cl_kernel<NT, ST, EPI>;
+  using Sm = ClSmem<NT, ST, FP8>;
+  auto kern = gemm_cl_kernel<NT, ST, EPI, FP8>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
@@ -562,12 +612,41 @@ cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& m
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_gemm_cl_fp8(const CUtensorMap& mapA, int n_tiles, int kb, int S, int a_row_base, const GemmEpi& ea,
+                               bool pdl, cudaStream_t s, int stages) {
+  if (S < 2 || S > 16 || (kb + S - 1) / S > kMaxFp8Blocks) return cudaErrorInvalidValue;
+  if (stages == 5) {
+    if (ea.epi == EPI_QKV) return launch_cl<16, 5, EPI_QKV, true>(mapA, mapA, n_tiles, kb, S, a_row_base, ea, pdl, s);
+    if (ea.epi == EPI_RESID)
+      return launch_cl<16, 5, EPI_RESID, true>(mapA, mapA, n_tiles, kb, S, a_row_base, ea, pdl, s);
+  }
+  if (stages == 10) {
+    if (ea.epi == EPI_QKV)
+      return launch_cl<16, 10, EPI_QKV, true>(mapA, mapA, n_tiles, kb, S, a_row_base, ea, pdl, s);
+    if (ea.epi == EPI_RESID)
+      return launch_cl<16, 10, EPI_RESID, true>(mapA, mapA, n_tiles, kb, S, a_row_base, ea, pdl, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// Stream-K W8A8 kernel: every CTA's range must need at most kMaxFp8Blocks
+// activation code blocks (a range that crosses a tile boundary needs all kb).
+cudaError_t launch_gemm_ws_fp8(const CUtensorMap& mapA, const CUtensorMap& mapA2, int n_tiles, int kb, int P,
+                               int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
+  if (kb > kMaxFp8Blocks) return cudaErrorInvalidValue;
+  SkSched sc{n_tiles, kb, P};
+  if (ea.epi == EPI_SWIGLU) return launch_one<16, 10, EPI_SWIGLU, true>(mapA, mapA2, mapA, sc, a_row_base, ea, pdl, s);
+  if (ea.epi == EPI_RESID) return launch_one<16, 10, EPI_RESID, true>(mapA, mapA2, mapA, sc, a_row_base, ea, pdl, s);
+  if (ea.epi == EPI_QKV) return launch_one<16, 10, EPI_QKV, true>(mapA, mapA2, mapA, sc, a_row_base, ea, pdl, s);
+  return cudaErrorInvalidValue;
+}
+
 // Clusters of S CTAs of the cluster split-K kernel that can be resident at
 // once (0: that cluster size cannot be launched).
-template <int ST>
+template <int ST, bool FP8 = false>
 static int cl_max_clusters(int epi, int S) {
-  using Sm = ClSmem<16, ST>;
-  auto kern = epi == EPI_QKV ? gemm_cl_kernel<16, ST, EPI_QKV> : gemm_cl_kernel<16, ST, EPI_RESID>;
+  using Sm = ClSmem<16, ST, FP8>;
+  auto kern = epi == EPI_QKV ? gemm_cl_kernel<16, ST, EPI_QKV, FP8> : gemm_cl_kernel<16, ST, EPI_RESID, FP8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
@@ -594,6 +673,10 @@ static int cl_max_clusters(int epi, int S) {
 
 int gemm_cl_max_clusters(int epi, int S, int stages) {
   return stages == 10 ? cl_max_clusters<10>(epi, S) : cl_max_clusters<5>(epi, S);
+}
+
+int gemm_cl_max_clusters_fp8(int epi, int S, int stages) {
+  return stages == 10 ? cl_max_clusters<10, true>(epi, S) : cl_max_clusters<5, true>(epi, S);
 }
 
 size_t gemm_ws_part_bytes(int NT, int P) { return static_cast<size_t>(P) * NT * 128 * sizeof(float); }

@@ -40,6 +40,20 @@ struct GemmEpi {
   float* part;
   int* cnt;
   int* status;
+  // W8A8 (fp8 kernels only): the projection's input rows q_src [NT][q_ld]
+  // (K wide; with rms_input the projection consumes their RMSNorm) are
+  // quantised per token in the CTA; amax_in [n_amax][NT] gives their largest
+  // magnitudes (else the rows are scanned); wscale / wscale2 are the E4M3
+  // weights' per-row scales indexed by absolute weight row (wscale2: the up
+  // rows of gate/up tiles); amax_out [n_tiles][NT] receives the SwiGLU
+  // activation's largest magnitude per tile (the down projection's amax_in).
+  const bf16* q_src;
+  int q_ld, q_K, rms_input;
+  const float* amax_in;
+  int n_amax;
+  const float* wscale;
+  const float* wscale2;
+  float* amax_out;
 };
 
 // Fused LM head operands.
@@ -86,6 +100,13 @@ int device_sm_count();
 cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
                            int n_tiles, int kb, int P, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s,
                            int stages);
+// W8A8 variants (E4M3 weight maps with 128-byte k boxes; kb = K / 128): the
+// stream-K gate/up kernel (10 stages) and the cluster split-K kernels.
+cudaError_t launch_gemm_ws_fp8(const CUtensorMap& mapA, const CUtensorMap& mapA2, int n_tiles, int kb, int P,
+                               int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s);
+cudaError_t launch_gemm_cl_fp8(const CUtensorMap& mapA, int n_tiles, int kb, int S, int a_row_base, const GemmEpi& ea,
+                               bool pdl, cudaStream_t s, int stages);
+int gemm_cl_max_clusters_fp8(int epi, int S, int stages);
 size_t gemm_ws_part_bytes(int NT, int P);
 // Cluster split-K (one tile per cluster of S CTAs; QKV and residual epilogues).
 cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
@@ -149,6 +170,9 @@ struct PrefillAttnArgs {
 cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                 const PrefillAttnArgs& a, cudaStream_t s);
 
+// FP8 E4M3 row quantisation (csrc/fp8.cu): codes [rows][K], scales [rows].
+cudaError_t launch_quantize_rows_e4m3(const bf16* a, int rows, int K, uint8_t* codes, float* scales, cudaStream_t s);
+
 // Embedding gather / row copy + per-128-feature sums of squares.
 cudaError_t launch_embed_bf16(const bf16* E, const bf16* rows_in, int n_src, const int32_t* tokens,
                               const uint8_t* masked, int mask_id, int n_rows, int H, int V, bf16* x,
@@ -193,6 +217,9 @@ cudaError_t f32_lmhead(const float* hidden, const float* w, int R, int H, int V,
 // Tensor maps (host).
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                   uint32_t box_inner, uint32_t box_outer);
+// Same for a byte matrix (E4M3 codes), 128-byte swizzle.
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
                   uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 

@@ -51,12 +51,18 @@ __host__ __device__ constexpr int tmem_cols_for() {
 // A operand source: one 128-row box, or two 64-row boxes from two tensors
 // (gate rows on top, up rows below) so the SwiGLU epilogue sees matching
 // gate/up features in one tile.
-template <int NT, int STAGES, bool SPLIT_A>
+//
+// FP8 (W8A8): the weight tiles are E4M3 codes, 128 rows x 128 k (the same 16 KB
+// per stage, twice the k of a bf16 stage), and the producer streams only
+// them; the activation codes for the CTA's k range are written into shared
+// memory once by the epilogue warps (fp8_quantize_activations).
+template <int NT, int STAGES, bool SPLIT_A, bool FP8 = false>
 __device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUtensorMap* mapA2,
                                             const CUtensorMap* mapB, uint8_t* sA, uint8_t* sB, uint64_t* full,
                                             uint64_t* empty, const SkSched& sc, long long u0, long long u1,
                                             int a_row_base, int b_row, int* status, volatile int* abort_flag) {
-  constexpr int B_BYTES = NT * 128;
+  constexpr int B_BYTES = FP8 ? 0 : NT * 128;
+  constexpr int KW = FP8 ? 128 : 64;  // k elements of one stage
   const uint64_t pol_w = l2_policy_evict_first();
   const uint64_t pol_x = l2_policy_evict_last();
   const int n = static_cast<int>(u1 - u0);
@@ -64,13 +70,14 @@ __device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUten
   auto load_a = [&](int s, long long u) {
     const int T = static_cast<int>(u / sc.kb), kk = static_cast<int>(u % sc.kb);
     if (SPLIT_A) {
-      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * 64, a_row_base + T * 64, pol_w);
-      tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, mapA2, &full[s], kk * 64, a_row_base + T * 64, pol_w);
+      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * KW, a_row_base + T * 64, pol_w);
+      tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, mapA2, &full[s], kk * KW, a_row_base + T * 64, pol_w);
     } else {
-      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * 64, a_row_base + T * 128, pol_w);
+      tma_load_2d(sA + s * kATileBytes, mapA, &full[s], kk * KW, a_row_base + T * 128, pol_w);
     }
   };
   auto load_b = [&](int s, long long u) {
+    if (FP8) return;
     const int kk = static_cast<int>(u % sc.kb);
     tma_load_2d(sB + s * B_BYTES, mapB, &full[s], kk * 64, b_row, pol_x);
   };
@@ -91,15 +98,19 @@ __device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUten
   }
 }
 
-template <int NT, int STAGES>
+// FP8: B is the activation code block of k block kk at sB + (kk - kb_lo) *
+// NT * 128, written once before b_ready completes.
+template <int NT, int STAGES, bool FP8 = false>
 __device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty, uint64_t* accf,
                                        uint64_t* acce, uint32_t tmem, const SkSched& sc, long long u0, long long u1,
-                                       int* status, volatile int* abort_flag, int issuer) {
+                                       int* status, volatile int* abort_flag, int issuer, uint64_t* b_ready = nullptr,
+                                       int kb_lo = 0) {
   // Issuer `issuer` (0 or 1) takes the k blocks j = issuer, issuer + 2, ... of
   // each segment into accumulator (b, issuer); both commit accf[b] (count 2).
   constexpr int B_BYTES = NT * 128;
-  constexpr uint32_t IDESC = idesc_bf16_f32(128, NT);
+  constexpr uint32_t IDESC = FP8 ? idesc_e4m3_f32(128, NT) : idesc_bf16_f32(128, NT);
   griddep_wait();
+  if (FP8 && !mbar_wait(b_ready, 0, status, abort_flag)) return;
   long long i_base = 0;  // pipeline stage index of the segment's first k block
   int seg = 0;
   for (long long u = u0; u < u1; ++seg) {
@@ -116,11 +127,16 @@ __device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full,
       if (!mbar_wait(&full[s], static_cast<uint32_t>((i / STAGES) & 1), status, abort_flag)) return;
       tc_fence_after();
       const uint32_t a0 = smem_u32(sA + s * kATileBytes);
-      const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+      const uint32_t b0 = FP8 ? smem_u32(sB + (static_cast<int>((u + jj) % sc.kb) - kb_lo) * B_BYTES)
+                              : smem_u32(sB + s * B_BYTES);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        umma_bf16_ss(d, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
-                     (jj >= 2 || k > 0) ? 1u : 0u);
+        if (FP8)
+          umma_e4m3_ss(d, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
+                       (jj >= 2 || k > 0) ? 1u : 0u);
+        else
+          umma_bf16_ss(d, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
+                       (jj >= 2 || k > 0) ? 1u : 0u);
       }
       umma_commit(&empty[s]);
     }
@@ -166,5 +182,84 @@ __device__ __forceinline__ void ws_load_acc16(uint32_t tmem, int b, int quarter,
 }
 
 __device__ __forceinline__ float bf16_round_f(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// W8A8 activations [Fast-dVLM technical overview (ocdem.com), section 2.3.2;
+// per-token scale a_t = max_k |h_tk| / 448, codes E4M3(h_tk / a_t)]: run by
+// the 128 epilogue threads (et = 0..127) of a weight-streaming CTA before its
+// first UMMA.  The projection's input h is src (bf16 [NT rows][src_ld]) or,
+// with rms != NULL, RMSNorm(src) = rms[t] * src (then a_t = rms[t] * amax /
+// 448 and the codes need only src * 448 / amax: the factor cancels).  The
+// per-token largest magnitude comes from amax_in ([n_amax][NT], written by
+// the producing kernel) or from reading the rows.  Codes of the 128-wide k
+// blocks [kb_lo, kb_hi) go to sB (block i at i * NT * 128, rows of 128 bytes,
+// 128-byte swizzle); a_t to sAt[t] (0 for rows >= n_rows).  Then one arrival
+// on b_ready.
+template <int NT>
+__device__ void fp8_quantize_activations(int et, const bf16* __restrict__ src, int src_ld, int K, int n_rows,
+                                         const float* rms, const float* amax_in, int n_amax, int kb_lo, int kb_hi,
+                                         uint8_t* sB, float* sAt, float* sQm, uint64_t* b_ready) {
+  constexpr int TPT = 128 / NT;  // threads per token for the row scan
+  if (amax_in) {
+    if (et < NT) {
+      float m = 0.f;
+      for (int p = 0; p < n_amax; ++p) m = fmaxf(m, amax_in[p * NT + et]);
+      sQm[et] = m;
+    }
+  } else {
+    const int t = et / TPT, part = et % TPT;
+    const int per = K / TPT;
+    float m = 0.f;
+    if (t < n_rows) {
+      const uint4* row = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld + part * per);
+      for (int i = 0; i < per / 8; ++i) {
+        const uint4 w = row[i];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h[q]);
+          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+    }
+#pragma unroll
+    for (int o = TPT / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (part == 0) sQm[t] = m;
+  }
+  named_bar_sync(1, 128);
+  if (et < NT) {
+    const float m = sQm[et];
+    const bool live = et < n_rows && m > 0.f;
+    sAt[et] = live ? m / 448.0f * (rms ? rms[et] : 1.0f) : 0.f;
+    sQm[et] = live ? 448.0f / m : 0.f;
+  }
+  named_bar_sync(1, 128);
+  const int n_items = (kb_hi - kb_lo) * NT * 8;  // (k block, row, 16-byte chunk)
+  for (int i = et; i < n_items; i += 128) {
+    const int c = i & 7, t = (i >> 3) % NT, b = i / (8 * NT);
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    const float q = sQm[t];
+    if (q != 0.f) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld + (kb_lo + b) * 128 + c * 16);
+      const uint4 w0 = p[0], w1 = p[1];
+      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&w0);
+      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&w1);
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float2 a = __bfloat1622float2(h0[2 * j]), bb = __bfloat1622float2(h0[2 * j + 1]);
+        o[j] = static_cast<uint32_t>(cvt_e4m3x2(a.y * q, a.x * q)) |
+               (static_cast<uint32_t>(cvt_e4m3x2(bb.y * q, bb.x * q)) << 16);
+        const float2 a2 = __bfloat1622float2(h1[2 * j]), b2 = __bfloat1622float2(h1[2 * j + 1]);
+        o[2 + j] = static_cast<uint32_t>(cvt_e4m3x2(a2.y * q, a2.x * q)) |
+                   (static_cast<uint32_t>(cvt_e4m3x2(b2.y * q, b2.x * q)) << 16);
+      }
+      out = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    *reinterpret_cast<uint4*>(sB + b * NT * 128 + (t >> 3) * 1024 + (t & 7) * 128 + ((c ^ (t & 7)) << 4)) = out;
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(1, 128);
+  if (et == 0) mbar_arrive(b_ready);
+}
 
 }  // namespace dvlm

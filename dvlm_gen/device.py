@@ -48,6 +48,24 @@ class DeviceModel:
                           dtype=DVLM_BF16 if self.dims.dtype == "bf16" else DVLM_FP32)
 
 
+    def fp8_c_model(self):
+        """The W8A8 version of this model: each projection's E4M3 codes and
+        per-row scales, quantised from these bf16 weights on the device by the
+        library (dvlm_quantize_rows_e4m3); embedding and LM head stay bf16."""
+        from block_diffusion_vlm_b200 import DVLM_FP8_W8A8, make_model, quantize_rows_e4m3
+        q = {}
+        for name in ("wqkv", "wo", "wgate", "wup", "wdown"):
+            w = getattr(self, name)
+            codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+            scales = torch.empty(w.shape[:2], dtype=torch.float32, device=w.device)
+            quantize_rows_e4m3(w, codes, scales, rows=w.shape[0] * w.shape[1], K=w.shape[2])
+            q[name] = (codes, scales)
+        self.fp8 = q
+        return make_model(self.dims, embed=self.embed, wqkv=q["wqkv"][0], wo=q["wo"][0], wgate=q["wgate"][0],
+                          wup=q["wup"][0], wdown=q["wdown"][0], lm_head=self.lm_head, dtype=DVLM_FP8_W8A8,
+                          scales=tuple(q[n][1] for n in ("wqkv", "wo", "wgate", "wup", "wdown")))
+
+
 def kv_buffers(dims: ModelDims, Lmax: int, device="cuda", n_batch: int = 1):
     """Zeroed K cache [n_layers, n_batch, Hkv, Lmax, D] and transposed V cache
     [n_layers, n_batch, Hkv, D, Lmax]."""

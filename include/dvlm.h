@@ -69,7 +69,11 @@ typedef enum dvlm_status {
   DVLM_ERR_BOUNDS = 8         /* a device-side index check failed (e.g. token id) */
 } dvlm_status;
 
-typedef enum dvlm_dtype { DVLM_BF16 = 0, DVLM_FP32 = 1 } dvlm_dtype;
+/* DVLM_FP8_W8A8: the four projections of every layer are FP8 W8A8 (E4M3
+ * weight codes with one scale per output row, activations quantised per
+ * token on the fly); embedding, LM head, activations and the KV cache are
+ * bf16 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]. */
+typedef enum dvlm_dtype { DVLM_BF16 = 0, DVLM_FP32 = 1, DVLM_FP8_W8A8 = 2 } dvlm_dtype;
 
 typedef void* dvlm_stream; /* cudaStream_t */
 
@@ -240,6 +244,11 @@ DVLM_API dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const in
  * bf16 storage points: q/k/v after RoPE, attention output, the residual
  * stream after each add, the SwiGLU activation; all sums in fp32.
  * bf16 path: H % 128 == 0, I % 64 == 0, D == 128, Hq == 8*Hkv.
+ * FP8 W8A8 path: the bf16 path's shapes with I % 128 == 0; the projection
+ * y = x W^T becomes y[t,o] = a_t * s_o * sum_k E4M3(h_tk / a_t) * code_ok
+ * with a_t = max_k |h_tk| / 448 over the projection's input row h_t (the
+ * RMS-normed row, the attention output or the SwiGLU activation) and s_o the
+ * weight row scale; prefill runs in 16-row forwards.
  */
 typedef struct dvlm_model {
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, inter, vocab;
@@ -253,6 +262,14 @@ typedef struct dvlm_model {
   const void* wup;
   const void* wdown;
   const void* lm_head;
+  /* DVLM_FP8_W8A8 only: wqkv..wdown hold E4M3 codes (uint8, same shapes) and
+   * these their per-row fp32 scales ([n_layers, rows] each, e.g. from
+   * dvlm_quantize_rows_e4m3); NULL otherwise. */
+  const float* sqkv;
+  const float* so;
+  const float* sgate;
+  const float* sup;
+  const float* sdown;
 } dvlm_model;
 
 enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2 };
@@ -374,6 +391,17 @@ DVLM_API dvlm_status dvlm_selftest_wait_timeout(long long budget_cycles, int* de
  * (synchronises the stream) and launches eagerly. */
 DVLM_API dvlm_status dvlm_forward_text_only(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
                                            int n_rows, int n_hidden, void* x_out, dvlm_stream stream);
+
+/* FP8 row quantisation for the W8A8 projections [Fast-dVLM technical
+ * overview (ocdem.com), section 2.3.2: the served model is quantised to W8A8
+ * FP8].  For each row r of a (bf16 [rows, K], device, row-major): scales[r]
+ * = max_k |a[r,k]| / 448 (1 for an all-zero row; fp32, device [rows]) and
+ * codes[r,k] = E4M3(a[r,k] / scales[r]) (device uint8 [rows, K]; E4M3 finite
+ * variant, round to nearest even, formed from the exact quotient in fp64).
+ * Rows are a weight matrix's output channels.  Errors: INVALID_ARG (NULL
+ * pointer), SHAPE (rows or K < 1).  One launch on `stream`, asynchronous. */
+DVLM_API dvlm_status dvlm_quantize_rows_e4m3(const void* a, int rows, int K, uint8_t* codes, float* scales,
+                                            dvlm_stream stream);
 
 /* Trace of the decode driver (test hook).  When set, every forward that
  * dvlm_decode_block / dvlm_generate run (noisy, causal append, draft, verify,

@@ -22,6 +22,11 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0
     assert d["unit"] == "tokens/s" and d["higher_is_better"] is True and d["value"] > 0
     assert d["vs_baseline"] is None and d["data"] == "synthetic" and "workload" in d["config"]
+    # the same config object as our arm prints for the same arguments
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench.argparse.Namespace(mode="threshold", weights="bf16")
+    assert d["config"] == bench.workload_config(args, 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -1,0 +1,129 @@
+"""FP8 W8A8 weight streaming against the oracle's W8A8 definitions
+[Fast-dVLM technical overview (ocdem.com), section 2.3.2: the served model is
+quantised to W8A8 FP8; readings: E4M3 finite variant, round to nearest even,
+one scale per weight output row and per activation token, amax / 448].
+
+* dvlm_quantize_rows_e4m3: codes bit-exact with the oracle's e4m3_round of the
+  exact quotient (random rows, an all-zero row, and a row whose quotients sit
+  exactly on E4M3 rounding midpoints, so every tie is exercised), scales
+  within fp32 rounding of amax / 448.
+* The W8A8 decoder (reduced model: 2 layers, hidden 1024, 8/1 heads of 128,
+  SwiGLU 1024) against OracleModel(fp8=True): the prefilled KV cache and a
+  noisy forward's hidden rows within the bf16 bar (2e-2 plus one storage ulp);
+  then threshold decoding through the engine's own graph path, every forward
+  replayed against the oracle's W8A8 model, decisions bit-exact at the 1e-3
+  bar on the rows the LM head read and within DELTA on the oracle's own rows.
+  The activations are quantised on the GPU from an fp32 quotient (the oracle
+  forms it in fp64): a code can differ where the quotient sits within fp32
+  rounding of an E4M3 midpoint, a one-code change of one of the K terms of a
+  sum, which the bf16 bar covers."""
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_vlm_b200 as dv
+import dvlm_gen as gen
+import oracle as O
+from decode_replay import Replay, parse_trace
+from dvlm_gen.device import DeviceModel, kv_buffers
+from gpu_util import assert_bf16_close, f64, ws_tensor
+
+pytestmark = pytest.mark.gpu
+DELTA = 0.1
+SMALL = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=1024, vocab=4096,
+                      lm_scale=25.0, dtype="bf16")
+
+
+def _e4m3_values():
+    return torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+
+
+def test_quantize_rows_matches_oracle(cuda):
+    rows, K = 64, 1024
+    a = gen.normal(3, "fp8.a", (rows, K), 0.02)
+    a[5] = 0.0
+    # row 7: amax 448 (scale exactly 1) and every midpoint between adjacent
+    # E4M3 values, both signs: each quotient is a tie
+    g = _e4m3_values()
+    mids = (g[:-1] + g[1:]) / 2
+    r7 = np.zeros(K)
+    r7[0] = 448.0
+    r7[1:1 + len(mids)] = mids
+    r7[1 + len(mids):1 + 2 * len(mids)] = -mids
+    a[7] = r7
+    a_t = gen.bf16_tensor(a)
+    assert np.array_equal(a_t.float().numpy()[7].astype(np.float64), r7)   # midpoints are bf16 values
+    a_d = a_t.to(cuda)
+    codes = torch.empty((rows, K), dtype=torch.uint8, device=cuda)
+    scales = torch.empty(rows, dtype=torch.float32, device=cuda)
+    dv.quantize_rows_e4m3(a_d, codes, scales, rows=rows, K=K)
+    torch.cuda.synchronize()
+    got = codes.cpu().view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    want, s = O.fp8_quantize_rows(a_t.float().numpy().astype(np.float64))
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_allclose(scales.cpu().numpy().astype(np.float64), s, rtol=2 ** -23, atol=0)
+
+
+class Fp8Setup:
+    def __init__(self, cuda, seed, n_vis=32, n_prompt=16, Lmax=256):
+        self.cuda, self.seed = cuda, seed
+        self.dm = DeviceModel(SMALL, seed, device=cuda)
+        self.cm = self.dm.fp8_c_model()
+        self.kc, self.vc = kv_buffers(SMALL, Lmax, device=cuda)
+        self.ws = ws_tensor(dv.engine_workspace_size(self.cm, Lmax, 16, 64), cuda)
+        self.eng = dv.Engine(self.cm, self.kc, self.vc, Lmax, 16, 64, self.ws)
+        self.vis_t, self.vis, self.ids = gen.decode_context(SMALL, seed, n_vis, n_prompt)
+        self.n_vis, self.n_prompt, self.Lmax = n_vis, n_prompt, Lmax
+
+    def prefill(self):
+        self.eng.prefill(self.vis_t.to(self.cuda), self.n_vis, torch.from_numpy(self.ids).to(self.cuda),
+                         self.n_prompt)
+        self.eng.check()
+        return self.eng.position()
+
+    def oracle(self):
+        m = O.OracleModel(O.dims_from(SMALL), weights=O.weights_from_generator(gen, SMALL, self.seed), bf16=True,
+                          Lmax=self.Lmax, fp8=True)
+        s = O.prefill(m, self.vis.astype(np.float64), self.ids)
+        return m, s
+
+
+def test_fp8_prefill_and_forward_match_oracle(cuda):
+    st = Fp8Setup(cuda, 5)
+    L, seed = st.prefill()
+    m, s = st.oracle()
+    assert L == m.L == 48
+    for l in range(SMALL.n_layers):
+        assert_bf16_close(f64(st.kc[l, 0, :, :L]), m.K[l][:, :L], 2e-2, f"K layer {l}")
+        assert_bf16_close(f64(st.vc[l, 0, :, :, :L]).transpose(0, 2, 1), m.V[l][:, :L], 2e-2, f"V layer {l}")
+    toks = [seed] + [SMALL.mask_id] * 15
+    x = torch.zeros((16, SMALL.hidden), dtype=torch.bfloat16, device=cuda)
+    st.eng.forward(16, 0, SMALL.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=cuda), x_out=x)
+    st.eng.check()
+    xo = m.forward(m.embed(toks), L, n_clean=0)
+    assert_bf16_close(f64(x), xo, 2e-2, "noisy forward")
+    st.eng.close()
+
+
+@pytest.mark.parametrize("seed", [1, 3])
+def test_fp8_threshold_decode_engine_path(cuda, seed):
+    st = Fp8Setup(cuda, seed)
+    rb = dv.engine_trace_record_bytes(st.cm)
+    buf = torch.zeros(128 * rb, dtype=torch.uint8, device=cuda)
+    cnt = torch.zeros(4, dtype=torch.int32, device=cuda)
+    st.prefill()
+    st.eng.set_trace(buf, cnt)
+    out = torch.zeros(32, dtype=torch.int32, device=cuda)
+    stats = dv.Stats()
+    st.eng.generate(dv.DecodeCfg(16, 0.9, dv.MODE_THRESHOLD, 1, 32, 1), out, stats)
+    st.eng.check()
+    st.eng.set_trace(None, None)
+    recs = parse_trace(buf.cpu().numpy(), int(cnt[0].item()), rb, SMALL.hidden, True)
+    m, s = st.oracle()
+    rp = Replay(m, s, 16, 0.9, decide="gpu", hidden_check=lambda a, b, w: assert_bf16_close(a, b, 2e-2, w),
+                secondary=DELTA, seed_bar=DELTA)
+    assert rp.threshold(recs, 32) == out.cpu().numpy().tolist()
+    assert rp._next == len(recs) == stats.nfe
+    assert rp.t.ids_exact > 0 and rp.t.commits_exact > 0 and rp.t.secondary_checked > 0, rp.t
+    print(f"fp8 seed {seed}: {rp.t}")
+    st.eng.close()
