@@ -346,7 +346,8 @@ def run_ours(args, rank, world, local, pg):
         if rank == 0:
             print(json.dumps({"profile_forwards": args.profile_forwards, "layers": dims.n_layers}), flush=True)
         return
-    mode = {"threshold": dv.MODE_THRESHOLD, "spec": dv.MODE_SPEC_LINEAR, "ar": dv.MODE_AR}[args.mode]
+    mode = {"threshold": dv.MODE_THRESHOLD, "spec": dv.MODE_SPEC_LINEAR, "ar": dv.MODE_AR,
+            "quad": dv.MODE_SPEC_QUAD}[args.mode]
     cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1)
     out = torch.zeros(N_NEW, dtype=torch.int32, device=dev)
 
@@ -430,16 +431,18 @@ def run_ours(args, rank, world, local, pg):
                        "forward_frac_of_nominal": fwd_bytes / (secs / args.steps / nfe) / 1e9 / NOMINAL_HBM_GBS},
             "kernels": per, "eager_forward_ms": fwd_ms}
 
-    # a short run of the linear self-speculative mode for context
+    # short runs of the speculative modes for context (same model and context)
     if args.mode == "threshold" and not args.quick:
-        sc = dv.DecodeCfg(BLOCK, TAU, dv.MODE_SPEC_LINEAR, 1, N_NEW, 1)
-        step(sc)
-        ev0.record(stream)
-        st = step(sc)
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        line["spec_linear"] = {"tokens_per_s": N_NEW / (ev0.elapsed_time(ev1) / 1000.0), "nfe": st.nfe,
-                               "accept_hist": list(st.accept_hist)}
+        for key, md in (("spec_linear", dv.MODE_SPEC_LINEAR), ("spec_quadratic", dv.MODE_SPEC_QUAD)):
+            sc = dv.DecodeCfg(BLOCK, TAU, md, 1, N_NEW, 1)
+            step(sc)
+            ev0.record(stream)
+            st = step(sc)
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+            secs_sc = ev0.elapsed_time(ev1) / 1000.0
+            line[key] = {"tokens_per_s": N_NEW / secs_sc, "nfe": st.nfe, "ms_per_forward": 1000 * secs_sc / st.nfe,
+                         "accept_hist": list(st.accept_hist)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = cpu_baseline(nfe)
     eng.close()
@@ -599,7 +602,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", choices=["threshold", "spec", "ar"], default="threshold")
+    ap.add_argument("--mode", choices=["threshold", "spec", "ar", "quad"], default="threshold")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: the W8A8 decoder (E4M3 projections quantised from the same bf16 weights)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(PKG, "libdvlm.so")
 HEADER = os.path.join(ROOT, "include", "dvlm.h")
 
 DVLM_BF16, DVLM_FP32, DVLM_FP8_W8A8 = 0, 1, 2
-MODE_THRESHOLD, MODE_SPEC_LINEAR, MODE_AR = 0, 1, 2
+MODE_THRESHOLD, MODE_SPEC_LINEAR, MODE_AR, MODE_SPEC_QUAD = 0, 1, 2, 3
 HIST = 17
 
 _lib: Optional[ctypes.CDLL] = None
@@ -119,6 +119,7 @@ def _declare(L: ctypes.CDLL) -> None:
                                       ctypes.POINTER(_i), _vp]),
         "dvlm_engine_trace_record_bytes": (_sz, [ctypes.POINTER(Model)]),
         "dvlm_quantize_rows_e4m3": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+        "dvlm_forward_quad": (_i, [_vp, _vp, _i, _vp, _vp]),
         "dvlm_engine_set_trace": (_i, [_vp, _vp, _sz, _vp]),
     }
     for name, (res, args) in sigs.items():
@@ -313,6 +314,11 @@ class Engine:
 
     def get_option(self, name: str) -> int:
         return int(lib().dvlm_engine_get_option(self.h, name.encode()))
+
+    def forward_quad(self, draft, B: int, x_out, stream=None) -> None:
+        """The fused draft+verify forward alone (dvlm_forward_quad)."""
+        _check(lib().dvlm_forward_quad(self.h, ptr(draft), int(B), ptr(x_out), stream_handle(stream)),
+               "dvlm_forward_quad")
 
     def set_trace(self, buf, count) -> None:
         """Record every decode-driver forward into buf (device tensor), counting

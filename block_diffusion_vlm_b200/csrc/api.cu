@@ -24,6 +24,8 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v);
 int engine_get_option(dvlm_engine* e, const char* name);
 void engine_set_trace(dvlm_engine* e, void* buf, int cap, int32_t* cnt);
 bool prefill_gemm_supported(const dvlm_engine* e);
+bool quad_supported(const dvlm_engine* e, int B);
+cudaError_t engine_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out, cudaStream_t s);
 cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, const int32_t* ids, int n_ids,
                                 cudaStream_t s);
 cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, const int32_t* other_ids, uint8_t* masked,
@@ -392,6 +394,7 @@ dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_vision, const
   if (e->bf16 && n_vision > 0 && !al16(vision)) return DVLM_ERR_INVALID_ARG;
   cudaStream_t s = cs(stream);
   const int n_ctx = n_vision + n_ids;
+  e->quad_ready = false;
   if (e->prefill_gemm && n_ctx <= e->max_ctx && prefill_gemm_supported(e))
     return cuda_status(engine_prefill_gemm(e, vision, n_vision, ids, n_ids, s));
   if (cudaMemsetAsync(e->d_len, 0, 4, s) != cudaSuccess) return DVLM_ERR_CUDA;
@@ -423,7 +426,8 @@ dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_vision, const
 static dvlm_status check_cfg(dvlm_engine* e, const dvlm_decode_cfg* cfg) {
   if (!e || !cfg) return DVLM_ERR_INVALID_ARG;
   if (cfg->block_size < 1 || cfg->block_size > e->max_block) return DVLM_ERR_SHAPE;
-  if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_AR) return DVLM_ERR_INVALID_ARG;
+  if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_SPEC_QUAD) return DVLM_ERR_INVALID_ARG;
+  if (cfg->mode == DVLM_MODE_SPEC_QUAD && !quad_supported(e, cfg->block_size)) return DVLM_ERR_UNSUPPORTED;
   if (std::isnan(cfg->threshold)) return DVLM_ERR_INVALID_ARG;
   if (cfg->ar_seed != 1) return DVLM_ERR_UNSUPPORTED;
   if (cfg->max_new_tokens < 1 || cfg->max_new_tokens > e->Lmax) return DVLM_ERR_SHAPE;
@@ -456,6 +460,7 @@ dvlm_status dvlm_decode_block(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_
 }
 
 static dvlm_status generate_impl(dvlm_engine* e, const dvlm_decode_cfg* cfg, dvlm_stats* stats, cudaStream_t s) {
+  e->quad_ready = false;  // a run starts from the pending seed: the quadratic mode drafts afresh
   int32_t L = 0;
   if (cudaMemcpyAsync(&L, e->d_len, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
@@ -527,6 +532,7 @@ dvlm_status dvlm_engine_set_position(dvlm_engine* e, int32_t L, int32_t seed, dv
   if (!e) return DVLM_ERR_INVALID_ARG;
   if (L < 0 || L > e->Lmax) return DVLM_ERR_SHAPE;
   if (seed < 0 || seed >= e->m.vocab) return DVLM_ERR_INVALID_ARG;
+  e->quad_ready = false;
   cudaStream_t s = cs(stream);
   if (cudaMemcpyAsync(e->d_len, &L, 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(e->d_seed, &seed, 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
@@ -629,6 +635,21 @@ dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value) 
   if (!e || !name) return DVLM_ERR_INVALID_ARG;
   if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
   return engine_set_option(e, name, value);
+}
+
+dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out, dvlm_stream stream) {
+  if (!e || !draft || !x_out) return DVLM_ERR_INVALID_ARG;
+  if (B < 1 || B > kNT || B + B * B > e->max_ctx) return DVLM_ERR_SHAPE;
+  if (!quad_supported(e, B)) return DVLM_ERR_UNSUPPORTED;
+  if (!al16(x_out)) return DVLM_ERR_INVALID_ARG;
+  cudaStream_t s = cs(stream);
+  int32_t L = 0;
+  if (cudaMemcpyAsync(&L, e->d_len, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DVLM_ERR_CUDA;
+  if (L + 2 * B > e->Lmax) return DVLM_ERR_CACHE_OVERFLOW;
+  e->quad_ready = false;
+  return cuda_status(engine_forward_quad(e, draft, B, x_out, s));
 }
 
 size_t dvlm_engine_trace_record_bytes(const dvlm_model* m) {

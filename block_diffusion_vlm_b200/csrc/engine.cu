@@ -133,6 +133,12 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
     e->pao = c.take<void>(C * HD * 2);
     e->pact = c.take<void>(C * I * 2);
     e->pssq = c.take<float>(static_cast<size_t>(H / 128 + 1) * C * 4);
+    e->qtok = c.take<int32_t>(C * 4);
+    e->d_k = c.take<int32_t>(4);
+    e->kside = c.take<void>(static_cast<size_t>(m.n_kv_heads) * kQuadSideKeys * 128 * 2);
+    e->vside = c.take<void>(static_cast<size_t>(m.n_kv_heads) * kQuadSideKeys * 128 * 2);
+    e->qpart = c.take<float>(static_cast<size_t>(P) * 128 * 256 * 4);
+    e->qcnt = c.take<int>(1024 * 4);
   }
   if (!e->bf16) {
     e->f_y = c.take<float>(static_cast<size_t>(kNT) * std::max(qkv_rows, H) * 4);
@@ -183,6 +189,10 @@ static bool build_maps(dvlm_engine* e) {
     ok &= make_tmap_2d(&e->tm_wg_p, m.wgate, H, static_cast<uint64_t>(L) * I, H * 2, 64, 128);
     ok &= make_tmap_2d(&e->tm_wu_p, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 128);
     ok &= make_tmap_2d(&e->tm_kp, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 128);
+    ok &= make_tmap_3d(&e->tm_q3, e->pq, D, Hq, C, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
+    ok &= make_tmap_2d(&e->tm_ks, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_vs, e->vside, kQuadSideKeys, static_cast<uint64_t>(Hkv) * D, kQuadSideKeys * 2, 64,
+                       128);
   }
   return ok;
 }
@@ -553,6 +563,193 @@ cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, c
                        false, s);
 }
 
+// Split-K factor of a token-major GEMM with n_tiles output tiles and kb k
+// blocks: enough CTAs to cover the SMs, at least 4 k blocks each.
+static int tm_splits(const dvlm_engine* e, int n_tiles, int kb) {
+  if (n_tiles >= e->sm) return 1;
+  return std::max(1, std::min(kb / 4, e->sm / n_tiles));
+}
+
+bool quad_supported(const dvlm_engine* e, int B) {
+  return prefill_gemm_supported(e) && B >= 1 && B <= 16 && B + B * B <= e->max_ctx &&
+         e->m.n_q_heads == 8 * e->m.n_kv_heads;
+}
+
+// The fused forward of quadratic self-speculative decoding [Fast-dVLM
+// technical overview (ocdem.com), section 2.3.1: draft and verify in one
+// forward at O(B^2) cost] over the draft in e->tokens at slots L..L+B-1:
+// B verify rows (causal; K/V to the cache) and B candidate blocks of B
+// [MASK] rows (block i at positions L+i+1..; K/V to the side buffers, one
+// layer at a time), all through the token-major GEMMs; the final residual
+// rows end in e->px.  L is not advanced.
+static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
+  const int qkv_rows = (Hq + 2 * Hkv) * D;
+  const int n = B + B * B, C = e->max_ctx;
+  const int n_tt = (n + 127) / 128;
+  bf16* px = static_cast<bf16*>(e->px);
+  DVLM_CK(launch_quad_tokens(e->tokens, B, m.mask_id, e->qtok, s));
+  DVLM_CK(launch_embed_bf16(static_cast<const bf16*>(m.embed), nullptr, 0, e->qtok, nullptr, m.mask_id, n, H,
+                            m.vocab, px, e->pssq, C, e->d_status, false, s));
+  const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  TmArgs ta{};
+  ta.n_tok = n;
+  ta.tok_stride = C;
+  ta.inv_h = 1.0f / H;
+  ta.eps = m.eps;
+  ta.Lmax = e->Lmax;
+  ta.n_q_heads = Hq;
+  ta.n_kv_heads = Hkv;
+  ta.d_len = e->d_len;
+  ta.log2_rope_base = std::log2(static_cast<double>(m.rope_base));
+  ta.status = e->d_status;
+  ta.part = e->qpart;
+  ta.cnt = e->qcnt;
+  ta.quad_B = B;
+  ta.kside = static_cast<bf16*>(e->kside);
+  ta.vside = static_cast<bf16*>(e->vside);
+  AttnArgs aa{};
+  aa.n_rows = B;
+  aa.n_clean = B;
+  aa.n_batch = 1;
+  aa.d_len = e->d_len;
+  aa.Lmax = e->Lmax;
+  aa.Hq = Hq;
+  aa.Hkv = Hkv;
+  aa.scale_log2 = scale_log2;
+  aa.out = static_cast<bf16*>(e->pao);
+  aa.status = e->d_status;
+  PrefillAttnArgs pa{};
+  pa.n_tok = n;
+  pa.Lmax = e->Lmax;
+  pa.Hq = Hq;
+  pa.Hkv = Hkv;
+  pa.scale_log2 = scale_log2;
+  pa.out = static_cast<bf16*>(e->pao);
+  pa.out_ld = Hq * D;
+  pa.status = e->d_status;
+  pa.quad_B = B;
+  pa.d_len = e->d_len;
+  pa.side_n = kQuadSideKeys;
+  for (int l = 0; l < m.n_layers; ++l) {
+    ta.epi = EPI_QKV;
+    ta.ssq_in = e->pssq;
+    ta.n_ssq = l == 0 ? H / 128 : H / 256;
+    ta.out = static_cast<bf16*>(e->pq);
+    ta.out_ld = Hq * D;
+    ta.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
+    ta.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
+    ta.splits = tm_splits(e, n_tt * (qkv_rows / 256), H / 64);
+    DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wqkv_p, e->tm_wqkv_p, H / 64, l * qkv_rows, qkv_rows / 256, ta, s));
+    aa.kv_base = l;
+    DVLM_CK(launch_attn_bf16(e->tm_q3, e->tm_k, e->tm_v, aa, false, s, e->attn_cs));
+    pa.kv_base = l;
+    DVLM_CK(launch_attn_cand(e->tm_q3, e->tm_kp, e->tm_v, e->tm_ks, e->tm_vs, pa, s));
+    ta.epi = EPI_RESID;
+    ta.resid = px;
+    ta.resid_ld = H;
+    ta.ssq_out = e->pssq;
+    ta.splits = tm_splits(e, n_tt * (H / 256), Hq * D / 64);
+    DVLM_CK(launch_gemm_tm(e->tm_pao, e->tm_wo_p, e->tm_wo_p, Hq * D / 64, l * H, H / 256, ta, s));
+    ta.epi = EPI_SWIGLU;
+    ta.n_ssq = H / 256;
+    ta.out = static_cast<bf16*>(e->pact);
+    ta.out_ld = I;
+    ta.splits = tm_splits(e, n_tt * (I / 128), H / 64);
+    DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wg_p, e->tm_wu_p, H / 64, l * I, I / 128, ta, s));
+    ta.epi = EPI_RESID;
+    ta.splits = tm_splits(e, n_tt * (H / 256), I / 64);
+    DVLM_CK(launch_gemm_tm(e->tm_pact, e->tm_wd_p, e->tm_wd_p, I / 64, l * H, H / 256, ta, s));
+  }
+  return cudaSuccess;
+}
+
+// Trace records around an LM head the fused round runs directly.
+static void quad_trace_begin(dvlm_engine* e, int kind, int n_rows, int n_clean, int R, const uint8_t* masked,
+                             cudaStream_t s) {
+  if (!e->trace_buf) return;
+  trace_begin_kernel<<<1, 32, 0, s>>>(e->trace_buf, trace_record_bytes(e->m.hidden, e->bf16), e->trace_cap,
+                                      e->trace_cnt, kind, e->d_len, n_rows, n_clean, R, e->tokens, masked);
+}
+static void quad_trace_end(dvlm_engine* e, int n_rows, int R, const uint8_t* masked, cudaStream_t s) {
+  if (!e->trace_buf) return;
+  trace_end_kernel<<<1, 256, 0, s>>>(e->trace_buf, trace_record_bytes(e->m.hidden, e->bf16), e->trace_cap,
+                                     e->trace_cnt, e->d_len, e->d_seed, n_rows, R, e->tr_top1, e->tr_p1, e->tokens,
+                                     masked, static_cast<const uint8_t*>(e->x),
+                                     static_cast<size_t>(n_rows) * e->m.hidden * 2);
+}
+
+// One round of quadratic self-speculative decoding: the fused forward over
+// the draft, the verify rows' LM head (row j predicts position j+1, L += B),
+// the longest agreeing prefix k (L -= B - k, seed v_k, accepted tokens
+// emitted), then the next draft: [v_k] followed by the top-1 of candidate
+// block k-1's rows 0..B-2 (shift 1).
+static cudaError_t quad_round(dvlm_engine* e, int B, int max_new, cudaStream_t s) {
+  const dvlm_model& m = e->m;
+  const int H = m.hidden;
+  DVLM_CK(quad_forward(e, B, s));
+  const int nt = (m.vocab + 127) / 128;
+  const int lm_ctas = ws_ctas(e, static_cast<long long>(nt) * (H / 64));
+  // verify rows -> decode rows (+ sums of squares), LM head over them
+  DVLM_CK(launch_embed_bf16(nullptr, static_cast<const bf16*>(e->px), B, nullptr, nullptr, 0, B, H, m.vocab,
+                            static_cast<bf16*>(e->x), e->ssq, kNT, e->d_status, false, s));
+  quad_trace_begin(e, TR_QUAD_VERIFY, B, B, B, nullptr, s);
+  LmArgs a{};
+  a.R = B;
+  a.threshold = -1.0f;
+  a.id_out = e->vids + 1;
+  a.len_ptr = e->d_len;
+  a.len_advance = B;
+  fill_lm_scratch(e, a);
+  a.ssq_in = e->ssq;
+  a.n_ssq = H / 128;
+  a.inv_h = 1.0f / H;
+  a.eps = m.eps;
+  if (e->trace_buf) {
+    a.top1_id = e->tr_top1;
+    a.top1_prob = e->tr_p1;
+  }
+  DVLM_CK(launch_lmhead(kNT, e->tm_lm, e->tm_x, nt, H / 64, lm_ctas, a, false, s));
+  quad_trace_end(e, B, B, nullptr, s);
+  DVLM_CK(launch_decode_accept(e->vids, e->tokens, B, e->d_len, e->d_seed, e->stage_out, e->n_out, max_new, e->ahist,
+                               e->d_k, e->d_status, false, s));
+  // next draft from candidate block k-1
+  DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, m.mask_id, 1, e->n_remaining, s));
+  DVLM_CK(launch_select_cand_rows(static_cast<const bf16*>(e->px), H, e->d_k, B, static_cast<bf16*>(e->x), e->ssq,
+                                  kNT, s));
+  if (B > 1) {
+    quad_trace_begin(e, TR_QUAD_CAND, B, 0, B - 1, e->masked, s);
+    LmArgs c{};
+    c.R = B - 1;
+    c.masked = e->masked + 1;
+    c.tokens = e->tokens + 1;
+    c.threshold = -1.0f;  // the draft takes every position's argmax
+    fill_lm_scratch(e, c);
+    c.ssq_in = e->ssq;
+    c.n_ssq = H / 128;
+    c.inv_h = 1.0f / H;
+    c.eps = m.eps;
+    if (e->trace_buf) {
+      c.top1_id = e->tr_top1;
+      c.top1_prob = e->tr_p1;
+    }
+    DVLM_CK(launch_lmhead(kNT, e->tm_lm, e->tm_x, nt, H / 64, lm_ctas, c, false, s));
+    quad_trace_end(e, B, B - 1, e->masked, s);
+  }
+  return cudaGetLastError();
+}
+
+// Test hook: the fused forward alone over the draft tokens (device [B]),
+// its final residual rows [B + B*B][H] copied to x_out.
+cudaError_t engine_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out, cudaStream_t s) {
+  DVLM_CK(cudaMemcpyAsync(e->tokens, draft, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToDevice, s));
+  DVLM_CK(quad_forward(e, B, s));
+  return cudaMemcpyAsync(x_out, e->px, static_cast<size_t>(B + B * B) * e->m.hidden * 2, cudaMemcpyDeviceToDevice,
+                         s);
+}
+
 cudaError_t engine_forward(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   return e->bf16 ? fwd_bf16(e, f, s) : fwd_f32(e, f, s);
 }
@@ -609,7 +806,7 @@ static long long fbits(float v) {
   return u;
 }
 
-enum { G_NOISY = 1, G_APPEND, G_DRAFT, G_VERIFY, G_AR };
+enum { G_NOISY = 1, G_APPEND, G_DRAFT, G_VERIFY, G_AR, G_QUAD };
 
 // One block (threshold / AR) or one round (spec).  Tokens are emitted into
 // stage_out at n_out (capped at max_new).  Returns the number of tokens this
@@ -641,6 +838,48 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
       st->n_launches += launches_per_forward(e->m.n_layers) + 1;
     }
     *emitted = std::min(1, max_new - n_out_host);
+    return cudaSuccess;
+  }
+  auto draft_pass = [&]() -> cudaError_t {
+    return run_graph(e, {G_DRAFT, B}, ug, s, [&]() -> cudaError_t {
+      FwdSpec f;
+      f.tokens = e->tokens;
+      f.masked = e->masked;
+      f.n_rows = B;
+      f.n_clean = 0;
+      f.lm = B > 1;
+      f.lma.R = B - 1;
+      f.lma.masked = e->masked + 1;
+      f.lma.tokens = e->tokens + 1;
+      f.lma.threshold = -1.0f;  // the draft takes every position's argmax
+      return traced_forward(e, f, TR_DRAFT, e->tokens, e->masked, s);
+    });
+  };
+  if (cfg.mode == DVLM_MODE_SPEC_QUAD) {
+    // quadratic self-speculative round [Fast-dVLM technical overview
+    // (ocdem.com), section 2.3.1]: the first round of a run drafts with one
+    // diffusion pass; every round is then one fused draft+verify forward
+    if (!e->quad_ready || e->quad_B != B) {
+      DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, e->m.mask_id, 1, e->n_remaining, s));
+      DVLM_CK(draft_pass());
+      e->quad_ready = true;
+      e->quad_B = B;
+      if (st) {
+        st->nfe += 1;
+        st->n_launches += 1 + (B > 1 ? 1 : 0) * launches_per_forward(e->m.n_layers);
+      }
+    }
+    DVLM_CK(run_graph(e, {G_QUAD, B, max_new}, ug, s, [&]() { return quad_round(e, B, max_new, s); }));
+    int32_t h = 0;
+    DVLM_CK(cudaMemcpyAsync(&h, e->n_out, 4, cudaMemcpyDeviceToHost, s));
+    DVLM_CK(cudaStreamSynchronize(s));
+    if (h <= n_out_host) return cudaErrorLaunchTimeout;
+    if (st) {
+      st->nfe += 1;
+      st->n_rounds += 1;
+      st->n_launches += 8 + 6 * e->m.n_layers + (B > 1 ? 1 : 0);
+    }
+    *emitted = h - n_out_host;
     return cudaSuccess;
   }
   DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, e->m.mask_id, 1, e->n_remaining, s));
@@ -700,19 +939,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
     return cudaSuccess;
   }
   // linear self-speculative round
-  DVLM_CK(run_graph(e, {G_DRAFT, B}, ug, s, [&]() -> cudaError_t {
-    FwdSpec f;
-    f.tokens = e->tokens;
-    f.masked = e->masked;
-    f.n_rows = B;
-    f.n_clean = 0;
-    f.lm = B > 1;
-    f.lma.R = B - 1;
-    f.lma.masked = e->masked + 1;
-    f.lma.tokens = e->tokens + 1;
-    f.lma.threshold = -1.0f;  // the draft takes every position's argmax
-    return traced_forward(e, f, TR_DRAFT, e->tokens, e->masked, s);
-  }));
+  DVLM_CK(draft_pass());
   DVLM_CK(run_graph(e, {G_VERIFY, B, max_new}, ug, s, [&]() -> cudaError_t {
     FwdSpec f;
     f.tokens = e->tokens;
@@ -726,7 +953,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
     f.lma.len_advance = B;
     DVLM_CK(traced_forward(e, f, TR_VERIFY, e->tokens, nullptr, s));
     return launch_decode_accept(e->vids, e->tokens, B, e->d_len, e->d_seed, e->stage_out, e->n_out, max_new,
-                                e->ahist, e->d_status, true, s);
+                                e->ahist, nullptr, e->d_status, true, s);
   }));
   int32_t h = 0;
   DVLM_CK(cudaMemcpyAsync(&h, e->n_out, 4, cudaMemcpyDeviceToHost, s));

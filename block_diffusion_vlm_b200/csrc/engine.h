@@ -63,7 +63,9 @@ struct FwdSpec {
 //   [104] next AR seed after, [105] cache length after, [106..111] zero;
 //   then rows x H residual-stream values (bf16 or fp32, the model's dtype),
 //   before the final RMSNorm.  Records are padded to 256 bytes.
-enum TraceKind { TR_NOISY = 1, TR_APPEND = 2, TR_DRAFT = 3, TR_VERIFY = 4, TR_AR = 5 };
+enum TraceKind { TR_NOISY = 1, TR_APPEND = 2, TR_DRAFT = 3, TR_VERIFY = 4, TR_AR = 5, TR_QUAD_VERIFY = 6,
+                 TR_QUAD_CAND = 7 };
+constexpr int kQuadSideKeys = 16 * 64;  // side-buffer keys per head: candidate block i at i * 64
 constexpr int kTraceWords = 112;
 inline size_t trace_record_bytes(int hidden, bool bf16) {
   const size_t b = kTraceWords * 4 + static_cast<size_t>(kNT) * hidden * (bf16 ? 2 : 4);
@@ -128,6 +130,15 @@ struct dvlm_engine {
   void* pact = nullptr;          // [max_ctx][I] SwiGLU activation
   float* pssq = nullptr;         // [H/128][max_ctx] sums of squares
   float* amax_act = nullptr;     // fp8: [I/64][NT] largest |SwiGLU activation| per gate/up tile
+  // quadratic self-speculative decoding (fused draft + verify forward)
+  int32_t* qtok = nullptr;       // [max_ctx] input tokens of the fused forward
+  int32_t* d_k = nullptr;        // accepted length of the last fused round
+  void* kside = nullptr;         // candidate K [Hkv][16*64][128] (one layer at a time)
+  void* vside = nullptr;         // candidate V^T [Hkv][128][16*64]
+  float* qpart = nullptr;        // split-K partial tiles of the token-major GEMMs
+  int* qcnt = nullptr;           // their per-tile counters (zero between launches)
+  bool quad_ready = false;       // the next fused round's draft is in `tokens`
+  int quad_B = 0;
   // fp32 path scratch
   float* f_y = nullptr;          // [NT][max(qkv_rows, H)]
   float* f_r = nullptr;          // [NT]
@@ -139,6 +150,8 @@ struct dvlm_engine {
   CUtensorMap tm_wqkv, tm_wo, tm_wg, tm_wu, tm_wd, tm_lm, tm_x, tm_ao, tm_act, tm_q, tm_k, tm_v;
   // prefill: activations (128-row boxes), weights (256-row boxes; gate/up 128), K (128-key boxes)
   CUtensorMap tm_px, tm_pq, tm_pao, tm_pact, tm_wqkv_p, tm_wo_p, tm_wd_p, tm_wg_p, tm_wu_p, tm_kp;
+  // fused forward: q rows as 16-row x 8-head boxes, candidate side buffers
+  CUtensorMap tm_q3, tm_ks, tm_vs;
   // captured graphs keyed by (kind, B, threshold bits, max_new)
   std::map<std::vector<long long>, cudaGraphExec_t> graphs;
 };

@@ -150,9 +150,24 @@ struct TmArgs {
   bf16* kcache;               // QKV: this layer's K [Hkv][Lmax][128] and V^T [Hkv][128][Lmax]
   bf16* vcache;
   int Lmax, n_q_heads, n_kv_heads;
-  int L0;                     // cache slot of context row 0
+  int L0;                     // cache slot of context row 0 (d_len != NULL: *d_len)
+  const int* d_len;
   double log2_rope_base;
   int* status;
+  // split-K: grid z = splits CTAs per output tile, each over k blocks
+  // [z*kb/splits, (z+1)*kb/splits); fp32 partial tiles part[(tile*splits+z)]
+  // [128][256] and per-tile arrival counters cnt (zero between launches): the
+  // last CTA of a tile adds the partials in z order and runs the epilogue.
+  int splits;
+  float* part;
+  int* cnt;
+  // QKV of the fused draft+verify forward (quad_B = B > 0): rows 0..B-1 are
+  // the verify rows (slots L..L+B-1, K/V to the cache); row B + i*B + r is row
+  // r of candidate block i at position L+i+1+r, its K/V to kside
+  // [Hkv][B*64][128] / vside [Hkv][128][B*64] at key i*64 + r.
+  int quad_B;
+  bf16* kside;
+  bf16* vside;
 };
 // y = x W^T over n_wtiles tiles of 256 weight rows (SWIGLU: 128 rows of W and
 // the same 128 rows of W2) starting at weight row w_row_base; kb = K / 64.
@@ -166,9 +181,22 @@ struct PrefillAttnArgs {
   bf16* out;                  // [n_tok][out_ld], head h at column h * 128
   int out_ld;
   int* status;
+  // candidate blocks of the fused draft+verify forward (launch_attn_cand):
+  // B = quad_B, cache length *d_len, side buffers with side_n keys per head
+  int quad_B;
+  const int* d_len;
+  int side_n;
 };
 cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                 const PrefillAttnArgs& a, cudaStream_t s);
+// Candidate block i (B noisy rows at positions L+i+1..) of the fused forward
+// sees cache slots 0..L+i and its own B keys from the side buffers
+// [Fast-dVLM technical overview (ocdem.com), section 2.3.1].  mapQ: 3-D map
+// of the q rows (box 64 x 8 heads x 16 rows); mapK/mapV: the cache maps
+// (128-key K boxes, 64-key V^T boxes); mapKs/mapVs: the side buffers.
+cudaError_t launch_attn_cand(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                             const CUtensorMap& mapKs, const CUtensorMap& mapVs, const PrefillAttnArgs& a,
+                             cudaStream_t s);
 
 // FP8 E4M3 row quantisation (csrc/fp8.cu): codes [rows][K], scales [rows].
 cudaError_t launch_quantize_rows_e4m3(const bf16* a, int rows, int K, uint8_t* codes, float* scales, cudaStream_t s);
@@ -188,7 +216,12 @@ cudaError_t launch_spec_ids(const int32_t* vids, const int32_t* draft, int b, in
 // Decode-driver accept: k over (verify ids, draft), L = L - B + k, seed, emit.
 cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len,
                                  int32_t* seed, int32_t* out, int32_t* n_out, int max_new, int64_t* accept_hist,
-                                 int* status, bool pdl, cudaStream_t s);
+                                 int32_t* k_out, int* status, bool pdl, cudaStream_t s);
+// Fused draft+verify forward helpers: its input tokens, and the chosen
+// candidate block's rows into the decode rows.
+cudaError_t launch_quad_tokens(const int32_t* draft, int B, int mask_id, int32_t* qtok, cudaStream_t s);
+cudaError_t launch_select_cand_rows(const bf16* src, int H, const int32_t* k_dev, int B, bf16* x, float* ssq_out,
+                                    int NT, cudaStream_t s);
 // Failure-detection self-test of the bounded waits.
 cudaError_t launch_selftest_timeout(long long budget, int* status, int* waited_out, cudaStream_t s);
 // Block bookkeeping for the decode driver.

@@ -117,12 +117,13 @@ cudaError_t launch_emit(const int32_t* tokens, int n, int32_t* out, int32_t* n_o
 // [Fast-dVLM technical overview (ocdem.com), section 2.3.1].
 __global__ void decode_accept_kernel(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len,
                                      int32_t* seed, int32_t* out, int32_t* n_out, int max_new,
-                                     int64_t* accept_hist, int* status) {
+                                     int64_t* accept_hist, int32_t* k_out, int* status) {
   griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x != 0) return;
   int k = 1;
   while (k < B && vids[k] == draft[k]) ++k;
+  if (k_out) *k_out = k;
   *d_len -= B - k;
   *seed = vids[k];
   const int base = *n_out;
@@ -132,8 +133,8 @@ __global__ void decode_accept_kernel(const int32_t* vids, const int32_t* draft, 
 }
 
 cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int B, int32_t* d_len, int32_t* seed,
-                                 int32_t* out, int32_t* n_out, int max_new, int64_t* accept_hist, int* status,
-                                 bool pdl, cudaStream_t s) {
+                                 int32_t* out, int32_t* n_out, int max_new, int64_t* accept_hist, int32_t* k_out,
+                                 int* status, bool pdl, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(32);
@@ -144,7 +145,48 @@ cudaError_t launch_decode_accept(const int32_t* vids, const int32_t* draft, int 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_accept_kernel, vids, draft, B, d_len, seed, out, n_out, max_new,
-                            accept_hist, status);
+                            accept_hist, k_out, status);
+}
+
+// Input tokens of the fused draft+verify forward: the draft's B tokens, then
+// B candidate blocks of B [MASK] tokens [Fast-dVLM technical overview
+// (ocdem.com), section 2.3.1].
+__global__ void quad_tokens_kernel(const int32_t* draft, int B, int mask_id, int32_t* qtok) {
+  for (int j = threadIdx.x; j < B + B * B; j += blockDim.x) qtok[j] = j < B ? draft[j] : mask_id;
+}
+
+cudaError_t launch_quad_tokens(const int32_t* draft, int B, int mask_id, int32_t* qtok, cudaStream_t s) {
+  quad_tokens_kernel<<<1, 256, 0, s>>>(draft, B, mask_id, qtok);
+  return cudaGetLastError();
+}
+
+// Rows of the chosen candidate block (k accepted: block k - 1, rows
+// B + (k-1)*B + r of src) into the decode rows x[r], r < B, with each row's
+// sum of squares per 128 features (ssq_out[p * NT + r]) for the final norm.
+__global__ void select_cand_rows_kernel(const bf16* __restrict__ src, int H, const int32_t* k_dev, int B,
+                                        bf16* __restrict__ x, float* __restrict__ ssq_out, int NT) {
+  const int r = blockIdx.x;
+  const int k = *k_dev;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bf16* row = src + static_cast<size_t>(B + (k - 1) * B + r) * H;
+  bf16* dst = x + static_cast<size_t>(r) * H;
+  for (int p = warp; p < H / 128; p += 4) {
+    const int c = p * 128 + lane * 4;
+    const uint2 w = *reinterpret_cast<const uint2*>(row + c);
+    *reinterpret_cast<uint2*>(dst + c) = w;
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const float2 a = __bfloat1622float2(h2[0]), b = __bfloat1622float2(h2[1]);
+    float sq = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) ssq_out[p * NT + r] = sq;
+  }
+}
+
+cudaError_t launch_select_cand_rows(const bf16* src, int H, const int32_t* k_dev, int B, bf16* x, float* ssq_out,
+                                    int NT, cudaStream_t s) {
+  select_cand_rows_kernel<<<B, 128, 0, s>>>(src, H, k_dev, B, x, ssq_out, NT);
+  return cudaGetLastError();
 }
 
 // Failure-detection self-test: an mbarrier that expects two arrivals gets

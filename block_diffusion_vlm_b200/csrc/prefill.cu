@@ -100,6 +100,9 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tt = blockIdx.x;  // token tile (fastest: the CTAs of one weight tile run together, sharing it in L2)
   const int T = blockIdx.y;   // weight tile
+  const int S = gridDim.z, z = blockIdx.z;
+  const int k_lo = z * kb / S, k_hi = (z + 1) * kb / S;
+  int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTmStages; ++s) {
@@ -125,25 +128,25 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_normal();
-      for (int i = 0; i < kb; ++i) {
-        const int s = i % kTmStages;
+      for (int i = 0; i < k_hi - k_lo; ++i) {
+        const int s = i % kTmStages, kk = k_lo + i;
         if (i >= kTmStages && !mbar_wait(&empty[s], ((i / kTmStages) & 1) ^ 1, a.status, sabort)) break;
         uint8_t* sA = smem + s * kTmStage;
         uint8_t* sB = sA + kTmA;
         mbar_arrive_expect_tx(&full[s], kTmStage);
-        tma_load_2d(sA, &mapX, &full[s], i * 64, tt * 128, pol);
+        tma_load_2d(sA, &mapX, &full[s], kk * 64, tt * 128, pol);
         if (EPI == EPI_SWIGLU) {
-          tma_load_2d(sB, &mapW, &full[s], i * 64, w_row_base + T * 128, pol);
-          tma_load_2d(sB + kTmB / 2, &mapW2, &full[s], i * 64, w_row_base + T * 128, pol);
+          tma_load_2d(sB, &mapW, &full[s], kk * 64, w_row_base + T * 128, pol);
+          tma_load_2d(sB + kTmB / 2, &mapW2, &full[s], kk * 64, w_row_base + T * 128, pol);
         } else {
-          tma_load_2d(sB, &mapW, &full[s], i * 64, w_row_base + T * 256, pol);
+          tma_load_2d(sB, &mapW, &full[s], kk * 64, w_row_base + T * 256, pol);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = true;
-      for (int i = 0; i < kb; ++i) {
+      for (int i = 0; i < k_hi - k_lo; ++i) {
         const int s = i % kTmStages;
         if (!mbar_wait(&full[s], (i / kTmStages) & 1, a.status, sabort)) {
           ok = false;
@@ -171,17 +174,65 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       for (int p = 0; p < a.n_ssq; ++p) s2 += a.ssq_in[static_cast<size_t>(p) * a.tok_stride + tok];
       r = 1.0f / sqrtf(s2 * a.inv_h + a.eps);
     }
-    const bool got = mbar_wait(accf, 0, a.status, sabort);
+    bool got = mbar_wait(accf, 0, a.status, sabort);
     __syncwarp();
+    if (got) tc_fence_after();
+    // Split-K: every CTA stores its fp32 partial tile; the last to arrive on
+    // the tile's counter adds all partials in z order (deterministic) and runs
+    // the epilogue on the sums.
+    const int tile = tt * gridDim.y + T;
+    if (S > 1) {
+      if (got) {
+        float* mine = a.part + (static_cast<size_t>(tile) * S + z) * 128 * 256 + static_cast<size_t>(row) * 256;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 16) {
+          float v[16];
+          acc16(tmem, quarter, c, v);
+#pragma unroll
+          for (int q = 0; q < 16; q += 4)
+            __stcg(reinterpret_cast<float4*>(mine + c + q), make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]));
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) *sflag = (atomicAdd(&a.cnt[tile], 1) == S - 1) ? 1 : 0;
+      named_bar_sync(1, 128);
+      got = got && *sflag;
+      if (got) {
+        __threadfence();
+        if (threadIdx.x == 64) a.cnt[tile] = 0;  // every partial arrived: zero for the next launch
+      }
+    }
+    // Columns [c, c+16) of this thread's row: the accumulator, or the sum of
+    // the split partials.
+    auto cols = [&](int c, float (&v)[16]) {
+      if (S == 1) {
+        acc16(tmem, quarter, c, v);
+        return;
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) v[q] = 0.f;
+      for (int zz = 0; zz < S; ++zz) {
+        const float4* src = reinterpret_cast<const float4*>(
+            a.part + (static_cast<size_t>(tile) * S + zz) * 128 * 256 + static_cast<size_t>(row) * 256 + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = __ldcg(src + q);
+          v[4 * q] += f.x;
+          v[4 * q + 1] += f.y;
+          v[4 * q + 2] += f.z;
+          v[4 * q + 3] += f.w;
+        }
+      }
+    };
     if (got) {
-      tc_fence_after();
       if (EPI == EPI_RESID) {
         bf16* x = a.resid + static_cast<size_t>(tok) * a.resid_ld + T * 256;
         float sq = 0.f;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 16) {
           float v[16];
-          acc16(tmem, quarter, c, v);  // warp-collective: every lane loads
+          cols(c, v);  // TMEM loads are warp-collective: every lane loads
           if (valid) {
             const uint4 xa = reinterpret_cast<const uint4*>(x + c)[0];
             const uint4 xb = reinterpret_cast<const uint4*>(x + c)[1];
@@ -207,8 +258,8 @@ __global__ void __launch_bounds__(kTmThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < 128; c += 16) {
           float g[16], u[16];
-          acc16(tmem, quarter, c, g);
-          acc16(tmem, quarter, 128 + c, u);
+          cols(c, g);
+          cols(128 + c, u);
           float o[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -219,18 +270,25 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         }
       } else {  // EPI_QKV: the tile holds heads 2T and 2T+1 of the [q | k | v] rows
         const int nq = a.n_q_heads, nkv = a.n_kv_heads;
-        const int pos = a.L0 + tok;
+        const int L0 = a.d_len ? *a.d_len : a.L0;
+        // candidate rows of a fused draft+verify forward: block ci, row cr
+        const int Bq = a.quad_B;
+        const bool cand = Bq > 0 && tok >= Bq;
+        const int ci = cand ? (tok - Bq) / Bq : 0, cr = cand ? (tok - Bq) % Bq : 0;
+        const int pos = cand ? L0 + ci + 1 + cr : L0 + tok;
+        const int side_n = Bq * 64;  // keys per head in the side buffers
 #pragma unroll 1
         for (int i = 0; i < 2; ++i) {
           const int hh = 2 * T + i;
           if (hh < nq + nkv) {
             bf16* dst = hh < nq ? a.out + static_cast<size_t>(tok) * a.out_ld + hh * 128
-                                : a.kcache + (static_cast<size_t>(hh - nq) * a.Lmax + pos) * 128;
+                        : cand ? a.kside + (static_cast<size_t>(hh - nq) * side_n + ci * 64 + cr) * 128
+                               : a.kcache + (static_cast<size_t>(hh - nq) * a.Lmax + pos) * 128;
 #pragma unroll 1
             for (int j0 = 0; j0 < 64; j0 += 16) {
               float x1[16], x2[16], y1[16], y2[16];
-              acc16(tmem, quarter, i * 128 + j0, x1);
-              acc16(tmem, quarter, i * 128 + 64 + j0, x2);
+              cols(i * 128 + j0, x1);
+              cols(i * 128 + 64 + j0, x2);
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
                 const int j = j0 + k;
@@ -252,11 +310,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
 #pragma unroll 1
             for (int c = 0; c < 128; c += 16) {
               float v[16];
-              acc16(tmem, quarter, i * 128 + c, v);
+              cols(i * 128 + c, v);
               if (valid) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                  a.vcache[(static_cast<size_t>(h) * 128 + c + k) * a.Lmax + pos] = __float2bfloat16_rn(v[k] * r);
+                for (int k = 0; k < 16; ++k) {
+                  const bf16 vb = __float2bfloat16_rn(v[k] * r);
+                  if (cand)
+                    a.vside[(static_cast<size_t>(h) * 128 + c + k) * side_n + ci * 64 + cr] = vb;
+                  else
+                    a.vcache[(static_cast<size_t>(h) * 128 + c + k) * a.Lmax + pos] = vb;
+                }
               }
             }
           }
@@ -273,10 +336,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
 }
 
 // Causal attention of n_tok prefill rows (slots L0..L0+n_tok-1, their K/V
-// already in the cache) over the cache slots 0..L0+n_tok-1.
+// already in the cache) over the cache slots 0..L0+n_tok-1 (CAND = false:
+// one CTA per 128 rows of one query head).  CAND = true: candidate block
+// blockIdx.x of the fused draft+verify forward, one CTA per (block, KV head),
+// its 16 rows x 8 query heads as the 128-row tile; it sees cache slots
+// 0..L+i (chunks of 128 keys) and then its own B keys (one side chunk).
+template <bool CAND>
 __global__ void __launch_bounds__(kPaThreads, 1)
-    attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                        const __grid_constant__ CUtensorMap mapV, const PrefillAttnArgs a) {
+    attn_tile_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapKs,
+                     const __grid_constant__ CUtensorMap mapVs, const PrefillAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem + oPaQ;
@@ -295,11 +364,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y;
-  const int g = h / (a.Hq / a.Hkv);
+  const int qt = blockIdx.x;                              // query tile (CAND: candidate block)
+  const int h = CAND ? 0 : blockIdx.y;                    // query head (prefill)
+  const int g = CAND ? blockIdx.y : h / (a.Hq / a.Hkv);   // KV head
   const int Ltot = a.L0 + a.n_tok;
-  const int q_last = min(a.L0 + qt * 128 + 127, Ltot - 1);  // last query slot of the tile
-  const int nc = q_last / kPaKeys + 1;
+  const int Lc = CAND ? *a.d_len + qt + 1 : 0;            // cache slots a candidate block sees
+  const int q_last = min(a.L0 + qt * 128 + 127, Ltot - 1);  // last query slot of a prefill tile
+  const int n_cache = CAND ? (Lc + kPaKeys - 1) / kPaKeys : q_last / kPaKeys + 1;
+  const int nc = n_cache + (CAND ? 1 : 0);                // + the candidate's own keys
   const int kv_row0 = a.kv_base * a.Hkv + g;  // (layer, KV head) entry of the cache
 
   if (threadIdx.x == 0) {
@@ -309,6 +381,10 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     tma_prefetch_map(&mapQ);
     tma_prefetch_map(&mapK);
     tma_prefetch_map(&mapV);
+    if (CAND) {
+      tma_prefetch_map(&mapKs);
+      tma_prefetch_map(&mapVs);
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kPaTmem);
@@ -323,16 +399,28 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_last();
       mbar_arrive_expect_tx(q_full, 2 * kPaAtom);
-      for (int d = 0; d < 2; ++d) tma_load_2d(sQ + d * kPaAtom, &mapQ, q_full, h * 128 + d * 64, qt * 128, pol);
+      for (int d = 0; d < 2; ++d) {
+        if (CAND)  // 16 rows x 8 heads of the block: row r*8 + hl of the tile
+          tma_load_3d(sQ + d * kPaAtom, &mapQ, q_full, d * 64, g * 8, a.quad_B + qt * a.quad_B, pol);
+        else
+          tma_load_2d(sQ + d * kPaAtom, &mapQ, q_full, h * 128 + d * 64, qt * 128, pol);
+      }
       for (int c = 0; c < nc; ++c) {
         const int st = c & 1;
         if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
         mbar_arrive_expect_tx(&kv_full[st], 4 * kPaAtom);
-        const int key0 = c * kPaKeys;
-        for (int d = 0; d < 2; ++d)
-          tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapK, &kv_full[st], d * 64, kv_row0 * a.Lmax + key0, pol);
-        for (int k = 0; k < 2; ++k)
-          tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapV, &kv_full[st], key0 + k * 64, kv_row0 * 128, pol);
+        if (CAND && c == n_cache) {  // the block's own keys: side entries qt*64 .. qt*64 + B - 1
+          for (int d = 0; d < 2; ++d)
+            tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapKs, &kv_full[st], d * 64, g * a.side_n + qt * 64, pol);
+          for (int k = 0; k < 2; ++k)
+            tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapVs, &kv_full[st], qt * 64 + k * 64, g * 128, pol);
+        } else {
+          const int key0 = c * kPaKeys;
+          for (int d = 0; d < 2; ++d)
+            tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapK, &kv_full[st], d * 64, kv_row0 * a.Lmax + key0, pol);
+          for (int k = 0; k < 2; ++k)
+            tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapV, &kv_full[st], key0 + k * 64, kv_row0 * 128, pol);
+        }
       }
     }
   } else if (warp == 1) {
@@ -374,8 +462,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int tok = qt * 128 + row;
-    const bool valid = tok < a.n_tok;
-    const int qslot = valid ? a.L0 + tok : Ltot - 1;  // rows past the end: finite, never written
+    const int cr = row >> 3, hl = row & 7;      // CAND: block row and query head within the group
+    const bool valid = CAND ? cr < a.quad_B : tok < a.n_tok;
+    const int qslot = valid ? a.L0 + tok : Ltot - 1;  // prefill rows past the end: finite, never written
+    // key j of chunk c is visible to this row
+    auto visible = [&](int c, int j) -> bool {
+      if (CAND) return c == n_cache ? j < a.quad_B : c * kPaKeys + j < Lc;
+      return c * kPaKeys + j <= qslot;
+    };
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -395,7 +489,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
         tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kPaKeys + hf * 64), sc);
 #pragma unroll
         for (int k = 0; k < 64; ++k)
-          if (key0 + hf * 64 + k <= qslot) mx = fmaxf(mx, sc[k] * a.scale_log2);
+          if (visible(c, hf * 64 + k)) mx = fmaxf(mx, sc[k] * a.scale_log2);
       }
       const float m_new = fmaxf(m, mx);
       const float alpha = (m == -INFINITY) ? (m_new == -INFINITY ? 1.f : 0.f) : exp2f(m - m_new);
@@ -407,7 +501,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
         tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kPaKeys + hf * 64), sc);
 #pragma unroll
         for (int k = 0; k < 64; k += 2) {
-          const bool v0 = key0 + hf * 64 + k <= qslot, v1 = key0 + hf * 64 + k + 1 <= qslot;
+          const bool v0 = visible(c, hf * 64 + k), v1 = visible(c, hf * 64 + k + 1);
           const float p0 = v0 ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
           const float p1 = v1 ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
           psum += p0 + p1;
@@ -451,7 +545,10 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       }
       // value row `row` (feature d = row) of this chunk to fp16 in place;
       // keys past the cache's valid slots were zero-filled by the load
+      // (prefill) or are zeroed here (candidate blocks: stale or poisoned
+      // slots past L+i, padding of the side chunk)
       {
+        const int n_valid = CAND ? (c == n_cache ? a.quad_B : Lc - c * kPaKeys) : kPaKeys;
         if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) {
           ok = false;
           break;
@@ -467,7 +564,9 @@ __global__ void __launch_bounds__(kPaThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
-              const __half2 hh = __floats2half2_rn(f.x, f.y);
+              // 16-byte chunk cc of this 128-byte row holds keys ((cc ^ (row & 7)) * 8 + 2e, +1)
+              const int kk = at * 64 + ((cc ^ (row & 7)) << 3) + 2 * e;
+              const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
               wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
             }
             *p16 = w;
@@ -484,7 +583,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     if (ok && mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      bf16* dst = a.out + static_cast<size_t>(tok) * a.out_ld + h * 128;
+      bf16* dst = CAND ? a.out + static_cast<size_t>(a.quad_B + qt * a.quad_B + cr) * a.out_ld + (g * 8 + hl) * 128
+                       : a.out + static_cast<size_t>(tok) * a.out_ld + h * 128;
 #pragma unroll 1
       for (int cc = 0; cc < 128; cc += 64) {
         float o[64];
@@ -516,7 +616,9 @@ static cudaError_t tm_launch(const CUtensorMap& mapX, const CUtensorMap& mapW, c
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmSmem);
   if (e != cudaSuccess) return e;
   const int n_tt = (a.n_tok + 127) / 128;
-  kern<<<dim3(n_tt, n_wtiles), kTmThreads, kTmSmem, s>>>(mapX, mapW, mapW2, kb, w_row_base, a);
+  const int S = a.splits > 1 ? a.splits : 1;
+  if (S > 1 && (!a.part || !a.cnt || S > kb)) return cudaErrorInvalidValue;
+  kern<<<dim3(n_tt, n_wtiles, S), kTmThreads, kTmSmem, s>>>(mapX, mapW, mapW2, kb, w_row_base, a);
   return cudaGetLastError();
 }
 
@@ -534,9 +636,20 @@ cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, con
 cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                 const PrefillAttnArgs& a, cudaStream_t s) {
   if (a.n_tok < 1 || a.Hq % a.Hkv) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
+  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
   if (e != cudaSuccess) return e;
-  attn_prefill_kernel<<<dim3((a.n_tok + 127) / 128, a.Hq), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, a);
+  attn_tile_kernel<false><<<dim3((a.n_tok + 127) / 128, a.Hq), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, mapK,
+                                                                                         mapV, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_cand(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                             const CUtensorMap& mapKs, const CUtensorMap& mapVs, const PrefillAttnArgs& a,
+                             cudaStream_t s) {
+  if (a.quad_B < 1 || a.quad_B > 16 || !a.d_len || a.Hq != 8 * a.Hkv) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
+  if (e != cudaSuccess) return e;
+  attn_tile_kernel<true><<<dim3(a.quad_B, a.Hkv), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, mapKs, mapVs, a);
   return cudaGetLastError();
 }
 

@@ -272,7 +272,18 @@ typedef struct dvlm_model {
   const float* sdown;
 } dvlm_model;
 
-enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2 };
+/* DVLM_MODE_SPEC_QUAD: quadratic self-speculative decoding [Fast-dVLM
+ * technical overview (ocdem.com), section 2.3.1: draft and verify fused into
+ * one forward at O(B^2) cost].  The first round of a run drafts with one
+ * diffusion pass; every round then runs one forward over B + B*B rows: the
+ * draft's B verify rows (causal, K/V to the cache) and, for each possible
+ * accepted length k = 1..B, a candidate block of B [MASK] rows at positions
+ * L+k..L+k+B-1 that sees the context, the verify rows 0..k-1 and itself (its
+ * K/V stay out of the cache).  The longest agreeing prefix k is kept (L += k)
+ * and the next draft is the verifier's token v_k followed by the top-1 of
+ * candidate block k-1's rows 0..B-2.  Output = greedy AR output.  bf16
+ * engines whose compute-bound prefill is supported, with B + B*B <= max_ctx. */
+enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2, DVLM_MODE_SPEC_QUAD = 3 };
 
 typedef struct dvlm_decode_cfg {
   int block_size;     /* B, 1..16 */
@@ -352,6 +363,16 @@ DVLM_API dvlm_status dvlm_engine_check(dvlm_engine* e, dvlm_stream stream);
 DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_t* tokens,
                          const uint8_t* masked, int n_rows, int n_clean, int first_layer,
                          int n_layers_run, int advance, void* x_out, dvlm_stream stream);
+
+/* Test hook: the fused draft+verify forward of quadratic self-speculative
+ * decoding alone, over draft [B] (device int32, copied into the engine's
+ * block tokens) at slots L..L+B-1: writes the verify rows' K/V to the cache
+ * (L is not advanced) and the final residual stream of all B + B*B rows
+ * (verify rows, then candidate blocks 0..B-1) to x_out [B + B*B, H] (bf16,
+ * device).  UNSUPPORTED where DVLM_MODE_SPEC_QUAD is; SHAPE for B outside
+ * 1..16 or B + B*B > max_ctx; CACHE_OVERFLOW if L + B + B > Lmax. */
+DVLM_API dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out,
+                                      dvlm_stream stream);
 
 /* Launch-configuration knobs of a bf16 engine (defaults are chosen at
  * creation from occupancy queries).  Names and values:

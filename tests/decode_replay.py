@@ -43,7 +43,7 @@ import numpy as np
 import oracle as O
 
 MARGIN = 1e-3
-NOISY, APPEND, DRAFT, VERIFY, AR = 1, 2, 3, 4, 5
+NOISY, APPEND, DRAFT, VERIFY, AR, QUAD_VERIFY, QUAD_CAND = 1, 2, 3, 4, 5, 6, 7
 NT = 16
 WORDS = 112
 
@@ -298,6 +298,63 @@ class Replay:
             self.seed_conf = O.Conf(p1=g.p1[k - 1:k], top1=g.top1[k - 1:k], p2=g.p2[k - 1:k],
                                     top2=g.top2[k - 1:k])
             i += 2
+        self._next = i
+        return self.tokens[:max_new]
+
+    def quadratic(self, recs: List[Rec], max_new: int, final_L: int, final_seed: int) -> List[int]:
+        """Quadratic self-speculative decoding: a diffusion draft pass, then per
+        round one fused forward (the oracle's forward_quadratic over the
+        draft) recorded as its verify rows (QUAD_VERIFY) and the chosen
+        candidate block's rows (QUAD_CAND, cache length already L + k)."""
+        B, mask_id = self.B, self.m.d.mask_id
+        assert B >= 2
+        dr = recs[0]
+        assert dr.kind == DRAFT, dr.kind
+        self._seed_check(int(dr.tok_in[0]))
+        toks = [self.seed] + [mask_id] * (B - 1)
+        assert list(dr.tok_in) == toks and list(dr.msk_in) == [False] + [True] * (B - 1)
+        c, c_o = self._forward(dr, 0, "draft #0")
+        self._row_checks(dr, range(B - 1), c, c_o, "draft #0")
+        draft = [self.seed] + [int(dr.top1[j - 1]) for j in range(1, B)]
+        assert list(dr.tok_out) == draft
+        for j in range(1, B):
+            self._id(draft[j], c, j - 1, "draft #0")
+        i = 1
+        while len(self.tokens) < max_new:
+            rv, rc = recs[i], recs[i + 1]
+            assert rv.kind == QUAD_VERIFY and rc.kind == QUAD_CAND, (i, rv.kind, rc.kind)
+            L = self.m.L
+            assert rv.L == L and list(rv.tok_in) == draft, (i, rv.L, L)
+            x_all = O.forward_quadratic(self.m, draft, L)
+            self.hidden_check(rv.x, x_all[:B], f"quad verify #{i}")
+            self.t.hidden_max_err = max(self.t.hidden_max_err, float(np.max(np.abs(rv.x - x_all[:B]))))
+            self.t.forwards += 1
+            g, g_o = self._confs(rv, x_all[:B])
+            self._row_checks(rv, range(B), g, g_o, f"quad verify #{i}")
+            ver = [draft[0]] + [int(rv.top1[j - 1]) for j in range(1, B)]
+            k = O.prefix_accept(ver, draft)
+            sure = all(g.p1[j - 1] - g.p2[j - 1] >= MARGIN for j in range(1, min(k + 1, B)))
+            for j in range(1, min(k + 1, B)):
+                self._id(ver[j], g, j - 1, f"quad verify #{i}")
+            self.t.accepts_exact += 1 if sure else 0
+            self.t.accepts_excluded += 0 if sure else 1
+            # the engine kept k tokens and seeded the next draft with v_k
+            assert rc.L == L + k, (i, rc.L, L, k)
+            v_k = int(rv.top1[k - 1])
+            assert int(rc.tok_in[0]) == v_k and list(rc.msk_in) == [False] + [True] * (B - 1)
+            xc = x_all[B + (k - 1) * B:B + k * B]
+            self.hidden_check(rc.x, xc, f"quad candidate #{i + 1}")
+            cc, cc_o = self._confs(rc, xc)
+            self._row_checks(rc, range(B - 1), cc, cc_o, f"quad candidate #{i + 1}")
+            nd = [v_k] + [int(rc.top1[j - 1]) for j in range(1, B)]
+            assert list(rc.tok_out) == nd, (i, list(rc.tok_out), nd)
+            for j in range(1, B):
+                self._id(nd[j], cc, j - 1, f"quad candidate #{i + 1}")
+            self.tokens.extend(draft[:k])
+            self.m.L = L + k
+            draft = nd
+            i += 2
+        assert self.m.L == final_L and draft[0] == final_seed, (self.m.L, final_L, draft[0], final_seed)
         self._next = i
         return self.tokens[:max_new]
 

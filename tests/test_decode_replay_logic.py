@@ -16,7 +16,8 @@ import pytest
 
 import dvlm_gen as gen
 import oracle as O
-from decode_replay import APPEND, AR, DRAFT, NOISY, VERIFY, Rec, Replay, layer_major_hidden, parse_trace
+from decode_replay import (APPEND, AR, DRAFT, NOISY, QUAD_CAND, QUAD_VERIFY, VERIFY, Rec, Replay,
+                           layer_major_hidden, parse_trace)
 
 DIMS = gen.TINY
 SEED = 4
@@ -109,6 +110,39 @@ def standin_spec(B=4, n_new=12, fault=None):
         seed = int(g.top1[k - 1])
         out.extend(draft[:k])
     return recs, out[:n_new], m.L, seed
+
+
+def standin_quad(B=4, n_new=12, fault=None):
+    """Quadratic self-speculative decoding with the oracle's fused forward,
+    recorded as the engine does (draft, then QUAD_VERIFY / QUAD_CAND pairs)."""
+    m, seed = _prefilled()
+    recs, out = [], []
+    L = m.L
+    toks = [seed] + [DIMS.mask_id] * (B - 1)
+    x = m.forward(m.embed(toks), L, 0)
+    c = m.logits_conf(x)
+    draft = [seed] + [int(c.top1[j - 1]) for j in range(1, B)]
+    recs.append(_rec(DRAFT, L, toks, [False] + [True] * (B - 1), 0, B - 1, c, draft, [False] * B, seed, L, x))
+    while len(out) < n_new:
+        L = m.L
+        xa = O.forward_quadratic(m, draft, L)
+        g = m.logits_conf(xa[:B])
+        recs.append(_rec(QUAD_VERIFY, L, draft, [False] * B, B, B, g, draft, [False] * B, draft[0], L + B, xa[:B]))
+        ver = [draft[0]] + [int(g.top1[j - 1]) for j in range(1, B)]
+        k = O.prefix_accept(ver, draft)
+        if fault == "accept" and k < B:
+            k += 1
+        vk = int(g.top1[k - 1])
+        blk = k if fault == "block" and k < B else k - 1
+        xc = xa[B + blk * B:B + (blk + 1) * B]
+        cc = m.logits_conf(xc)
+        nd = [vk] + [int(cc.top1[j - 1]) for j in range(1, B)]
+        recs.append(_rec(QUAD_CAND, L + k, [vk] + [DIMS.mask_id] * (B - 1), [False] + [True] * (B - 1), 0, B - 1,
+                         cc, nd, [False] * B, vk, L + k, xc))
+        out.extend(draft[:k])
+        m.L = L + k
+        draft = nd
+    return recs, out[:n_new], m.L, draft[0]
 
 
 def standin_ar(n_new=6):
@@ -220,3 +254,14 @@ def test_parse_trace_layout():
     assert list(r.tok_out) == [5, 9, 12, 9] and list(r.msk_out) == [False, True, False, True]
     assert (r.seed_out, r.len_out) == (7, 70)
     np.testing.assert_array_equal(r.x, xs[:4])
+
+
+def test_replay_quadratic_accepts_the_oracle_and_rejects_faults():
+    recs, out, L, s0 = standin_quad()
+    rp = _replay()
+    assert rp.quadratic(recs, 12, L, s0) == out and rp._next == len(recs)
+    assert rp.t.ids_exact > 0
+    for fault in ("accept", "block"):
+        recs, out, L, s0 = standin_quad(fault=fault)
+        with pytest.raises(AssertionError):
+            _replay().quadratic(recs, 12, L, s0)

@@ -97,11 +97,11 @@ def test_static_scratch_refuses_sizes_beyond_its_capacity(cuda):
     with pytest.raises(dv.DvlmError) as ei:
         dv.lmhead_conf_commit_static(h, w, R=R, H=H, V=V, top1_id=torch.zeros(R, dtype=torch.int32, device=cuda))
     assert ei.value.status == 7  # DVLM_ERR_WORKSPACE
-    # R <= 32 but a vocabulary of 2^27 rows: 4 bytes of counters per 128 rows
-    # (4 MiB) plus the per-SM partial tiles overflow the 6 MiB array.  The
-    # weight tensor is real (17 GB, never read: the call is refused on the
-    # host before any launch).
-    R, H, V = 16, 64, 1 << 27
+    # R <= 32 but a vocabulary of 2^28 rows: its counters alone (4 bytes per
+    # 128 rows, 8 MiB) overflow the 6 MiB array on any device.  The weight
+    # tensor is real (34 GB, never read: the call is refused on the host
+    # before any launch).
+    R, H, V = 16, 64, 1 << 28
     h = torch.zeros((R, H), dtype=torch.bfloat16, device=cuda)
     w = torch.empty((V, H), dtype=torch.bfloat16, device=cuda)
     with pytest.raises(dv.DvlmError) as ei:
