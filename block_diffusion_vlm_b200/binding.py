@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(PKG, "libdvlm.so")
 HEADER = os.path.join(ROOT, "include", "dvlm.h")
 
 DVLM_BF16, DVLM_FP32, DVLM_FP8_W8A8 = 0, 1, 2
-MODE_THRESHOLD, MODE_SPEC_LINEAR, MODE_AR, MODE_SPEC_QUAD = 0, 1, 2, 3
+MODE_THRESHOLD, MODE_SPEC_LINEAR, MODE_AR, MODE_SPEC_QUAD, MODE_ROUTE = 0, 1, 2, 3, 4
 HIST = 17
 
 _lib: Optional[ctypes.CDLL] = None
@@ -64,18 +64,20 @@ class Model(ctypes.Structure):
 
 class DecodeCfg(ctypes.Structure):
     _fields_ = [("block_size", ctypes.c_int), ("threshold", ctypes.c_float), ("mode", ctypes.c_int),
-                ("ar_seed", ctypes.c_int), ("max_new_tokens", ctypes.c_int), ("use_graphs", ctypes.c_int)]
+                ("ar_seed", ctypes.c_int), ("max_new_tokens", ctypes.c_int), ("use_graphs", ctypes.c_int),
+                ("route_k", ctypes.c_int), ("route_n_vis", ctypes.c_int)]
 
 
 class Stats(ctypes.Structure):
     _fields_ = [("nfe", ctypes.c_int64), ("n_tokens", ctypes.c_int64), ("n_iters", ctypes.c_int64),
                 ("n_rounds", ctypes.c_int64), ("commit_hist", ctypes.c_int64 * HIST),
-                ("accept_hist", ctypes.c_int64 * HIST), ("n_launches", ctypes.c_int64)]
+                ("accept_hist", ctypes.c_int64 * HIST), ("n_launches", ctypes.c_int64),
+                ("n_text_passes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {"nfe": self.nfe, "n_tokens": self.n_tokens, "n_iters": self.n_iters, "n_rounds": self.n_rounds,
                 "commit_hist": list(self.commit_hist), "accept_hist": list(self.accept_hist),
-                "n_launches": self.n_launches}
+                "n_launches": self.n_launches, "n_text_passes": self.n_text_passes}
 
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

@@ -428,6 +428,10 @@ static dvlm_status check_cfg(dvlm_engine* e, const dvlm_decode_cfg* cfg) {
   if (cfg->block_size < 1 || cfg->block_size > e->max_block) return DVLM_ERR_SHAPE;
   if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_SPEC_QUAD) return DVLM_ERR_INVALID_ARG;
   if (cfg->mode == DVLM_MODE_SPEC_QUAD && !quad_supported(e, cfg->block_size)) return DVLM_ERR_UNSUPPORTED;
+  if (cfg->mode == DVLM_MODE_ROUTE) {
+    if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+    if (cfg->route_k < 1 || cfg->route_n_vis < 0 || cfg->route_n_vis % 8 || cfg->block_size < 2) return DVLM_ERR_SHAPE;
+  }
   if (std::isnan(cfg->threshold)) return DVLM_ERR_INVALID_ARG;
   if (cfg->ar_seed != 1) return DVLM_ERR_UNSUPPORTED;
   if (cfg->max_new_tokens < 1 || cfg->max_new_tokens > e->Lmax) return DVLM_ERR_SHAPE;
@@ -467,6 +471,7 @@ static dvlm_status generate_impl(dvlm_engine* e, const dvlm_decode_cfg* cfg, dvl
     return DVLM_ERR_CUDA;
   // worst case: every block/round ends B slots further (spec truncates back)
   if (static_cast<long long>(L) + cfg->max_new_tokens + cfg->block_size > e->Lmax) return DVLM_ERR_CACHE_OVERFLOW;
+  if (cfg->mode == DVLM_MODE_ROUTE && cfg->route_n_vis > L) return DVLM_ERR_SHAPE;
   if (cudaMemsetAsync(e->n_out, 0, 4, s) != cudaSuccess) return DVLM_ERR_CUDA;
   int n = 0;
   while (n < cfg->max_new_tokens) {

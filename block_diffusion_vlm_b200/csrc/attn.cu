@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(192, 1)
   // end of a forward pass moves it), and so are the cache slots below it: both
   // may be read before waiting for the predecessor.  Slots L.. are written by
   // the QKV projection this kernel follows.
-  const int L = a.d_len ? *a.d_len : a.L_static;
+  const int L = (a.d_len ? *a.d_len : a.L_static) - a.len_sub;
   const int Ltot = L + a.n_rows;
   // Chunk j of 64 keys belongs to CTA j % kCS (round robin): a row's partial
   // sums then do not depend on how many rows the step has, so a causal row

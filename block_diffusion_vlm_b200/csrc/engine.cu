@@ -22,6 +22,9 @@ using namespace dvlm;
 
 namespace dvlm {
 
+cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, const int32_t* other_ids, uint8_t* masked,
+                               int32_t* tokens, int R, int k, uint8_t* commit, int32_t* n_commit, cudaStream_t s);
+
 __global__ void advance_kernel(int32_t* d_len, int n) {
   griddep_wait();
   griddep_launch_dependents();
@@ -120,6 +123,11 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->masked = c.take<uint8_t>(kNT + 1);
   e->tr_top1 = c.take<int32_t>(kNT * 4);
   e->tr_p1 = c.take<float>(kNT * 4);
+  e->anc_id = c.take<int32_t>(kNT * 4);
+  e->anc_p1 = c.take<float>(kNT * 4);
+  e->txt_id = c.take<int32_t>(kNT * 4);
+  e->txt_p1 = c.take<float>(kNT * 4);
+  e->cert = c.take<int32_t>(4);
   e->hist = c.take<int64_t>(DVLM_HIST * 8);
   e->ahist = c.take<int64_t>(DVLM_HIST * 8);
   e->stage_vis = c.take<void>(static_cast<size_t>(std::max(e->max_ctx, 1)) * H * es);
@@ -309,8 +317,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     aa.status = e->d_status;
     T0(K_ATTN);
     if (f.hide > 0) {
-      aa.d_len = nullptr;
-      aa.L_static = f.L_host - f.hide;
+      aa.len_sub = f.hide;  // the view starts f.hide slots into the cache
       DVLM_CK(launch_attn_bf16(e->tm_q, tm_k_text, tm_v_text, aa, pdl, s, e->attn_cs));
     } else {
       DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s, e->attn_cs));
@@ -806,7 +813,7 @@ static long long fbits(float v) {
   return u;
 }
 
-enum { G_NOISY = 1, G_APPEND, G_DRAFT, G_VERIFY, G_AR, G_QUAD };
+enum { G_NOISY = 1, G_APPEND, G_DRAFT, G_VERIFY, G_AR, G_QUAD, G_RFULL, G_RTEXT };
 
 // One block (threshold / AR) or one round (spec).  Tokens are emitted into
 // stage_out at n_out (capped at max_new).  Returns the number of tokens this
@@ -883,7 +890,79 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
     return cudaSuccess;
   }
   DVLM_CK(launch_block_init(e->tokens, e->masked, e->d_seed, B, e->m.mask_id, 1, e->n_remaining, s));
-  if (cfg.mode == DVLM_MODE_THRESHOLD) {
+  if (cfg.mode == DVLM_MODE_ROUTE || cfg.mode == DVLM_MODE_THRESHOLD) {
+  if (cfg.mode == DVLM_MODE_ROUTE) {
+    // certificate-guided visual routing [Look Only When Needed, method
+    // steps (1)-(3)]; position j is scored by row j-1 (rows 0..B-2)
+    const int k = cfg.route_k, nv = cfg.route_n_vis;
+    int n_masked = B - 1;
+    bool have_anchors = false;
+    for (int step = 0; n_masked > 0; ++step) {
+      // every step unmasks at least one position
+      if (step >= 2 * (B - 1)) return cudaErrorLaunchTimeout;
+      const int kk = std::min(k, n_masked);
+      if (have_anchors) {
+        DVLM_CK(run_graph(e, {G_RTEXT, B, nv}, ug, s, [&]() -> cudaError_t {
+          FwdSpec f;
+          f.tokens = e->tokens;
+          f.masked = e->masked;
+          f.n_rows = B;
+          f.n_clean = 0;
+          f.hide = nv;
+          f.lm = true;
+          f.lma.R = B - 1;
+          f.lma.masked = e->masked + 1;
+          f.lma.threshold = 2.0f;
+          f.lma.top1_id = e->txt_id;
+          f.lma.top1_prob = e->txt_p1;
+          f.lma.anchor_id = e->anc_id;
+          f.lma.anchor_conf = e->anc_p1;
+          f.lma.cert_len = e->cert;
+          return traced_forward(e, f, TR_ROUTE_TEXT, e->tokens, e->masked, s);
+        }));
+        int32_t cert = 0;
+        DVLM_CK(cudaMemcpyAsync(&cert, e->cert, 4, cudaMemcpyDeviceToHost, s));
+        DVLM_CK(cudaStreamSynchronize(s));
+        if (st) {
+          st->nfe += 1;
+          st->n_iters += 1;
+          st->n_text_passes += 1;
+          st->n_launches += launches_per_forward(e->m.n_layers);
+        }
+        if (cert >= kk) {  // the certified prefix, with the anchor ids
+          DVLM_CK(launch_topk_commit(e->anc_p1, e->anc_id, nullptr, e->masked + 1, e->tokens + 1, B - 1, cert,
+                                     nullptr, nullptr, s));
+          n_masked -= cert;
+          if (st && cert < DVLM_HIST) st->commit_hist[cert] += 1;
+          continue;
+        }
+      }
+      DVLM_CK(run_graph(e, {G_RFULL, B}, ug, s, [&]() -> cudaError_t {
+        FwdSpec f;
+        f.tokens = e->tokens;
+        f.masked = e->masked;
+        f.n_rows = B;
+        f.n_clean = 0;
+        f.lm = true;
+        f.lma.R = B - 1;
+        f.lma.masked = e->masked + 1;
+        f.lma.threshold = 2.0f;
+        f.lma.top1_id = e->anc_id;  // the FULL pass replaces every anchor
+        f.lma.top1_prob = e->anc_p1;
+        return traced_forward(e, f, TR_ROUTE_FULL, e->tokens, e->masked, s);
+      }));
+      DVLM_CK(launch_topk_commit(e->anc_p1, e->anc_id, have_anchors ? e->txt_id : nullptr, e->masked + 1,
+                                 e->tokens + 1, B - 1, kk, nullptr, nullptr, s));
+      n_masked -= kk;
+      have_anchors = true;
+      if (st) {
+        st->nfe += 1;
+        st->n_iters += 1;
+        st->n_launches += launches_per_forward(e->m.n_layers) + 1;
+        if (kk < DVLM_HIST) st->commit_hist[kk] += 1;
+      }
+    }
+  } else {
     int rem = B - 1;
     for (int it = 0; rem > 0; ++it) {
       // every iteration commits at least one position: a block needing more
@@ -915,6 +994,7 @@ cudaError_t engine_step(dvlm_engine* e, const dvlm_decode_cfg& cfg, int max_new,
         st->n_launches += launches_per_forward(e->m.n_layers);
       }
     }
+  }
     DVLM_CK(run_graph(e, {G_APPEND, B, max_new}, ug, s, [&]() -> cudaError_t {
       FwdSpec f;
       f.tokens = e->tokens;

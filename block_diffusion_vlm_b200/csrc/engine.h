@@ -64,7 +64,7 @@ struct FwdSpec {
 //   then rows x H residual-stream values (bf16 or fp32, the model's dtype),
 //   before the final RMSNorm.  Records are padded to 256 bytes.
 enum TraceKind { TR_NOISY = 1, TR_APPEND = 2, TR_DRAFT = 3, TR_VERIFY = 4, TR_AR = 5, TR_QUAD_VERIFY = 6,
-                 TR_QUAD_CAND = 7 };
+                 TR_QUAD_CAND = 7, TR_ROUTE_FULL = 8, TR_ROUTE_TEXT = 9 };
 constexpr int kQuadSideKeys = 16 * 64;  // side-buffer keys per head: candidate block i at i * 64
 constexpr int kTraceWords = 112;
 inline size_t trace_record_bytes(int hidden, bool bf16) {
@@ -117,6 +117,12 @@ struct dvlm_engine {
   int32_t* stage_ids = nullptr;  // [max_ctx]
   int32_t* stage_out = nullptr;  // [max_ctx] generated tokens (host path)
   int32_t* h_pinned = nullptr;   // host-mapped scalars (n_remaining, n_out, L, seed)
+  // certificate-guided routing: anchors (FULL pass), TEXT-ONLY outputs, certified length
+  int32_t* anc_id = nullptr;     // [NT]
+  float* anc_p1 = nullptr;       // [NT]
+  int32_t* txt_id = nullptr;     // [NT]
+  float* txt_p1 = nullptr;       // [NT]
+  int32_t* cert = nullptr;       // [1]
   int32_t* tr_top1 = nullptr;    // [NT] LM-head ids while tracing
   float* tr_p1 = nullptr;        // [NT] LM-head probabilities while tracing
   // forward trace (test hook, off unless set): records, capacity, device count

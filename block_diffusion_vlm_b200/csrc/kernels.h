@@ -126,6 +126,7 @@ struct AttnArgs {
   float scale_log2;          // scale * log2(e)
   bf16* out;                 // [n_batch][n_rows][Hq][128]
   int* status;
+  int len_sub;               // the length used is (*d_len or L_static) - len_sub (offset cache views)
 };
 // cs: CTAs per cluster splitting the keys (8, or 16 where the device can
 // co-schedule 16-CTA clusters; see attn_cluster_size()).

@@ -283,7 +283,21 @@ typedef struct dvlm_model {
  * and the next draft is the verifier's token v_k followed by the top-1 of
  * candidate block k-1's rows 0..B-2.  Output = greedy AR output.  bf16
  * engines whose compute-bound prefill is supported, with B + B*B <= max_ctx. */
-enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2, DVLM_MODE_SPEC_QUAD = 3 };
+/* DVLM_MODE_ROUTE: certificate-guided visual routing inside block decoding
+ * [Look Only When Needed, method steps (1)-(3)].  Per block (first token the
+ * AR seed): a FULL noisy pass sets the anchors (top-1 id and probability of
+ * every masked position) and unmasks the route_k most confident; each later
+ * step runs a TEXT-ONLY pass (cache slots 0..route_n_vis-1 hidden, positions
+ * unchanged) and scans the masked positions in descending anchor confidence
+ * while its top-1 equals the anchor: a certified prefix of at least
+ * min(route_k, masked) positions is unmasked whole with the anchor ids;
+ * otherwise a FULL pass refreshes every anchor and min(route_k, masked)
+ * positions are unmasked with the FULL ids, those whose TEXT-ONLY top-1
+ * differs first (each group by confidence, lower position first on ties).
+ * A causal pass appends the block.  bf16 engines; one host read of the
+ * certified length per TEXT-ONLY pass. */
+enum { DVLM_MODE_THRESHOLD = 0, DVLM_MODE_SPEC_LINEAR = 1, DVLM_MODE_AR = 2, DVLM_MODE_SPEC_QUAD = 3,
+       DVLM_MODE_ROUTE = 4 };
 
 typedef struct dvlm_decode_cfg {
   int block_size;     /* B, 1..16 */
@@ -292,6 +306,8 @@ typedef struct dvlm_decode_cfg {
   int ar_seed;        /* 1: the block's first token is the AR prediction, committed outright */
   int max_new_tokens; /* generation stops after exactly this many tokens */
   int use_graphs;     /* 1: replay each forward as a captured CUDA graph */
+  int route_k;        /* DVLM_MODE_ROUTE: positions unmasked per step (>= 1) */
+  int route_n_vis;    /* DVLM_MODE_ROUTE: vision rows at the front of the cache (multiple of 8) */
 } dvlm_decode_cfg;
 
 #define DVLM_HIST 17
@@ -303,6 +319,7 @@ typedef struct dvlm_stats {
   int64_t commit_hist[DVLM_HIST]; /* iterations that committed c tokens, c = 0..16 */
   int64_t accept_hist[DVLM_HIST]; /* spec rounds that accepted k tokens, k = 0..16 */
   int64_t n_launches;             /* kernel launches issued (graph replays included) */
+  int64_t n_text_passes;          /* DVLM_MODE_ROUTE: TEXT-ONLY noisy passes (counted in nfe too) */
 } dvlm_stats;
 
 typedef struct dvlm_engine dvlm_engine;

@@ -43,7 +43,7 @@ import numpy as np
 import oracle as O
 
 MARGIN = 1e-3
-NOISY, APPEND, DRAFT, VERIFY, AR, QUAD_VERIFY, QUAD_CAND = 1, 2, 3, 4, 5, 6, 7
+NOISY, APPEND, DRAFT, VERIFY, AR, QUAD_VERIFY, QUAD_CAND, ROUTE_FULL, ROUTE_TEXT = 1, 2, 3, 4, 5, 6, 7, 8, 9
 NT = 16
 WORDS = 112
 
@@ -355,6 +355,102 @@ class Replay:
             draft = nd
             i += 2
         assert self.m.L == final_L and draft[0] == final_seed, (self.m.L, final_L, draft[0], final_seed)
+        self._next = i
+        return self.tokens[:max_new]
+
+    def _append(self, recs: List[Rec], i: int, toks) -> None:
+        B = self.B
+        rec = recs[i]
+        assert rec.kind == APPEND and rec.n_clean == B and list(rec.tok_in) == toks, (i, rec.kind)
+        c, c_o = self._forward(rec, i, f"append #{i}")
+        self.m.L += B
+        assert rec.len_out == self.m.L, (i, rec.len_out, self.m.L)
+        self._row_checks(rec, [B - 1], c, c_o, f"append #{i}")
+        assert rec.seed_out == rec.top1[B - 1]
+        self.seed_conf = O.Conf(p1=c.p1[B - 1:], top1=c.top1[B - 1:], p2=c.p2[B - 1:], top2=c.top2[B - 1:])
+        self.tokens.extend(toks)
+
+    def _set_check(self, chosen, p1_oracle, masked, n, what) -> None:
+        """The n positions the engine chose by its own confidences, against the
+        choice the deciding confidences make, wherever the n-th and (n+1)-th
+        largest are at least MARGIN apart (the choice is then unique)."""
+        live = sorted((-p1_oracle[j], j) for j in range(self.B) if masked[j])
+        if n < len(live) and -live[n - 1][0] - (-live[n][0]) < MARGIN:
+            self.t.commits_excluded += 1
+            return
+        assert sorted(chosen) == sorted(j for _, j in live[:n]), (what, sorted(chosen), live[:n + 1])
+        self.t.commits_exact += 1
+
+    def routing(self, recs: List[Rec], max_new: int, k: int, n_vis: int) -> List[int]:
+        """Certificate-guided routing [LOWN steps (1)-(3)]: FULL passes set the
+        anchors, TEXT-ONLY passes (vision slots hidden) are certified against
+        them.  The engine's own rule on its own values is held exactly (the
+        certified length, the committed positions and ids, read from the next
+        record's block state); its values are held to the oracle."""
+        B, mask_id = self.B, self.m.d.mask_id
+        i = 0
+        while len(self.tokens) < max_new:
+            self._seed_check(int(recs[i].tok_in[0]))
+            toks = [self.seed] + [mask_id] * (B - 1)
+            masked = [False] + [True] * (B - 1)
+            anc_id = anc_p1 = text_top = None
+            while any(masked):
+                kk = min(k, sum(masked))
+                rec, nxt = recs[i], recs[i + 1]
+                assert list(rec.tok_in) == toks and list(rec.msk_in) == masked, (i, list(rec.tok_in), toks)
+                L = self.m.L
+                assert rec.L == L
+                top = np.array([-1] + [int(rec.top1[j - 1]) for j in range(1, B)])
+                p1g = np.array([0.0] + [float(rec.p1[j - 1]) for j in range(1, B)])
+                live = [j for j in range(B) if masked[j]]
+                if anc_id is not None:
+                    assert rec.kind == ROUTE_TEXT, (i, rec.kind)
+                    x_o = self.m.forward(self.m.embed(toks), L, 0, hide=n_vis)
+                    self.hidden_check(rec.x, x_o, f"text #{i}")
+                    self.t.forwards += 1
+                    c, c_o = self._confs(rec, x_o)
+                    self._row_checks(rec, [j - 1 for j in live], c, c_o, f"text #{i}")
+                    text_top = top
+                    order = O.certificate_order(anc_p1, masked)
+                    n = O.certificate_scan(anc_id, anc_p1, text_top, masked)
+                    for j in order[:n + 1]:           # the scanned rows decide the certificate
+                        self._id(int(text_top[j]), c, j - 1, f"text #{i}")
+                    if n >= kk:
+                        want_t, want_m = list(toks), list(masked)
+                        for j in order[:n]:
+                            want_t[j], want_m[j] = int(anc_id[j]), False
+                        assert list(nxt.tok_in) == want_t and list(nxt.msk_in) == want_m, (i, "certified commit")
+                        toks, masked = want_t, want_m
+                        i += 1
+                        continue
+                    rec, nxt = recs[i + 1], recs[i + 2]
+                    i += 1
+                    assert list(rec.tok_in) == toks and list(rec.msk_in) == masked
+                    top = np.array([-1] + [int(rec.top1[j - 1]) for j in range(1, B)])
+                    p1g = np.array([0.0] + [float(rec.p1[j - 1]) for j in range(1, B)])
+                assert rec.kind == ROUTE_FULL, (i, rec.kind)
+                x_o = self.m.forward(self.m.embed(toks), L, 0)
+                self.hidden_check(rec.x, x_o, f"full #{i}")
+                self.t.forwards += 1
+                c, c_o = self._confs(rec, x_o)
+                self._row_checks(rec, [j - 1 for j in live], c, c_o, f"full #{i}")
+                if text_top is None:
+                    order = O.certificate_order(p1g, masked)
+                else:
+                    order = O.divergence_first_order(top, p1g, text_top, masked)
+                want_t, want_m = list(toks), list(masked)
+                for j in order[:kk]:
+                    want_t[j], want_m[j] = int(top[j]), False
+                    self._id(int(top[j]), c, j - 1, f"full #{i}")
+                assert list(nxt.tok_in) == want_t and list(nxt.msk_in) == want_m, (i, "FULL commit")
+                if text_top is None:   # the plain top-k choice, also by the deciding confidences
+                    po = np.array([0.0] + [float(c.p1[j - 1]) for j in range(1, B)])
+                    self._set_check(order[:kk], po, masked, kk, f"full #{i}")
+                anc_id, anc_p1 = top, p1g
+                toks, masked = want_t, want_m
+                i += 1
+            self._append(recs, i, toks)
+            i += 1
         self._next = i
         return self.tokens[:max_new]
 

@@ -16,8 +16,8 @@ import pytest
 
 import dvlm_gen as gen
 import oracle as O
-from decode_replay import (APPEND, AR, DRAFT, NOISY, QUAD_CAND, QUAD_VERIFY, VERIFY, Rec, Replay,
-                           layer_major_hidden, parse_trace)
+from decode_replay import (APPEND, AR, DRAFT, NOISY, QUAD_CAND, QUAD_VERIFY, ROUTE_FULL, ROUTE_TEXT, VERIFY, Rec,
+                           Replay, layer_major_hidden, parse_trace)
 
 DIMS = gen.TINY
 SEED = 4
@@ -145,6 +145,54 @@ def standin_quad(B=4, n_new=12, fault=None):
     return recs, out[:n_new], m.L, draft[0]
 
 
+def standin_route(B=4, k=1, n_vis=32, n_new=12, fault=None):
+    """Certificate-guided routing with the oracle's forward, recorded as the
+    engine does (FULL / TEXT-ONLY passes, then the causal append)."""
+    m, seed = _prefilled()
+    recs, out = [], []
+    while len(out) < n_new:
+        L = m.L
+        toks = [seed] + [DIMS.mask_id] * (B - 1)
+        masked = [False] + [True] * (B - 1)
+        anc_id = anc_p1 = text_top = None
+
+        def pass_(hide):
+            x = m.forward(m.embed(toks), L, 0, hide=hide)
+            c = m.logits_conf(x)
+            top = np.array([-1] + [int(c.top1[j - 1]) for j in range(1, B)])
+            p1 = np.array([0.0] + [float(np.float32(c.p1[j - 1])) for j in range(1, B)])
+            return x, c, top, p1
+
+        while any(masked):
+            kk = min(k, sum(masked))
+            if anc_id is not None:
+                x, c, top, p1 = pass_(0 if fault == "sees_vision" else n_vis)
+                recs.append(_rec(ROUTE_TEXT, L, toks, masked, 0, B - 1, c, toks, masked, seed, L, x))
+                text_top = top
+                n = O.certificate_scan(anc_id, anc_p1, text_top, masked)
+                if n >= kk:
+                    order = O.certificate_order(anc_p1, masked)
+                    if fault == "reverse":
+                        order = order[::-1]
+                    for j in order[:n]:
+                        toks[j], masked[j] = int(anc_id[j]), False
+                    continue
+            x, c, top, p1 = pass_(0)
+            recs.append(_rec(ROUTE_FULL, L, toks, masked, 0, B - 1, c, toks, masked, seed, L, x))
+            order = (O.certificate_order(p1, masked) if text_top is None
+                     else O.divergence_first_order(top, p1, text_top, masked))
+            for j in order[:kk]:
+                toks[j], masked[j] = int(top[j]), False
+            anc_id, anc_p1 = top, p1
+        x = m.forward(m.embed(toks), L, B)
+        m.L = L + B
+        c = m.logits_conf(x)
+        seed = int(c.top1[B - 1])
+        recs.append(_rec(APPEND, L, toks, [False] * B, B, B, c, toks, [False] * B, seed, m.L, x))
+        out.extend(toks)
+    return recs, out[:n_new]
+
+
 def standin_ar(n_new=6):
     m, seed = _prefilled()
     recs, out = [], []
@@ -265,3 +313,17 @@ def test_replay_quadratic_accepts_the_oracle_and_rejects_faults():
         recs, out, L, s0 = standin_quad(fault=fault)
         with pytest.raises(AssertionError):
             _replay().quadratic(recs, 12, L, s0)
+
+
+def test_replay_routing_accepts_the_oracle_and_rejects_faults():
+    recs, out = standin_route(B=8, k=1, n_new=24)
+    rp = Replay(*_prefilled(), 8, 0.9, decide="oracle", hidden_check=_fp32_check)
+    assert rp.routing(recs, 24, 1, 32) == out and rp._next == len(recs)
+    kinds = [r.kind for r in recs]
+    assert ROUTE_TEXT in kinds and ROUTE_FULL in kinds
+    sig = lambda rs: [list(r.tok_in) for r in rs]
+    for fault in ("sees_vision", "reverse"):
+        bad, _ = standin_route(B=8, k=1, n_new=24, fault=fault)
+        assert sig(bad) != sig(recs) or fault == "sees_vision"   # the fault did fire
+        with pytest.raises(AssertionError):
+            Replay(*_prefilled(), 8, 0.9, decide="oracle", hidden_check=_fp32_check).routing(bad, 24, 1, 32)

@@ -271,3 +271,35 @@ def test_bf16_reduced_model_routing_teacher_forced(cuda):
     assert counts["full"] == tr.n_full and counts["text"] == tr.n_text
     assert counts["text"] > 0 and counts["top1"] > 0
     s.eng.close()
+
+
+@pytest.mark.parametrize("seed,k", [(1, 2), (3, 1)])
+def test_bf16_reduced_model_routing_engine_path(cuda, seed, k):
+    """Certificate-guided routing driven by the engine itself (mode
+    DVLM_MODE_ROUTE: anchors kept on the device, FULL and TEXT-ONLY passes
+    captured in CUDA graphs, certified and divergence-first commits), B=16,
+    32 tokens, the 32 vision rows hidden in TEXT-ONLY passes; every pass
+    replayed against the oracle (the TEXT-ONLY ones with the vision slots
+    hidden), the engine's certificate and commits held to the routing rules."""
+    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
+    rb = dv.engine_trace_record_bytes(s.dm.c_model())
+    buf = torch.zeros(256 * rb, dtype=torch.uint8, device=cuda)
+    cnt = torch.zeros(4, dtype=torch.int32, device=cuda)
+    s.eng.set_trace(buf, cnt)
+    try:
+        s.eng.prefill(s.vis_t.to(cuda), 32, torch.from_numpy(s.ids).to(cuda), 16)
+        out = torch.zeros(32, dtype=torch.int32, device=cuda)
+        st = dv.Stats()
+        s.eng.generate(dv.DecodeCfg(16, 0.9, dv.MODE_ROUTE, 1, 32, 1, k, 32), out, st)
+        s.eng.check()
+    finally:
+        s.eng.set_trace(None, None)
+    recs = parse_trace(buf.cpu().numpy(), int(cnt[0].item()), rb, SMALL_BF16.hidden, True)
+    m, so = s.oracle_model()
+    rp = Replay(m, so, 16, 0.9, decide="gpu", hidden_check=_bf16_hidden, secondary=DELTA, seed_bar=DELTA)
+    got = rp.routing(recs, 32, k, 32)
+    assert got == out.cpu().numpy().tolist()
+    assert rp._next == len(recs) == st.nfe
+    assert st.n_text_passes == sum(r.kind == 9 for r in recs) > 0
+    print(f"routing seed {seed} k {k}: {rp.t}, text passes {st.n_text_passes} of {st.nfe}")
+    s.eng.close()
