@@ -122,6 +122,8 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_engine_trace_record_bytes": (_sz, [ctypes.POINTER(Model)]),
         "dvlm_quantize_rows_e4m3": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
         "dvlm_forward_quad": (_i, [_vp, _vp, _i, _vp, _vp]),
+        "dvlm_engine_set_paged": (_i, [_vp, _vp, _vp, _vp, _i, _i]),
+        "dvlm_block_attn_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
         "dvlm_engine_set_trace": (_i, [_vp, _vp, _sz, _vp]),
     }
     for name, (res, args) in sigs.items():
@@ -161,6 +163,15 @@ def block_attn(q, out, k_cache, v_cache, *, n_batch, n_rows, n_clean, L, Lmax, H
     _check(lib().dvlm_block_attn(ptr(q), ptr(out), ptr(k_cache), ptr(v_cache), n_batch, n_rows, n_clean, L, Lmax,
                                  Hq, Hkv, D, float(scale), dtype, ptr(status), stream_handle(stream)),
            "dvlm_block_attn")
+
+
+def block_attn_paged(q, out, k_pages, v_pages, block_table, lens, *, n_batch, n_rows, n_clean, n_pages, max_pages,
+                     Hq, Hkv, D, scale, status=None, stream=None) -> None:
+    """Attention over paged KV caches (dvlm_block_attn_paged)."""
+    _check(lib().dvlm_block_attn_paged(ptr(q), ptr(out), ptr(k_pages), ptr(v_pages), ptr(block_table), ptr(lens),
+                                       n_batch, n_rows, n_clean, n_pages, max_pages, Hq, Hkv, D, float(scale),
+                                       ptr(status), stream_handle(stream)),
+           "dvlm_block_attn_paged")
 
 
 def lmhead_workspace_size(R: int, V: int, H: int, dtype: int) -> int:
@@ -316,6 +327,13 @@ class Engine:
 
     def get_option(self, name: str) -> int:
         return int(lib().dvlm_engine_get_option(self.h, name.encode()))
+
+    def set_paged(self, k_pages, v_pages, block_table, n_pages: int, max_pages: int) -> None:
+        """Switch to a paged KV cache (dvlm_engine_set_paged)."""
+        self._keep = self._keep + (k_pages, v_pages, block_table)
+        _check(lib().dvlm_engine_set_paged(self.h, ptr(k_pages), ptr(v_pages), ptr(block_table), int(n_pages),
+                                           int(max_pages)),
+               "dvlm_engine_set_paged")
 
     def forward_quad(self, draft, B: int, x_out, stream=None) -> None:
         """The fused draft+verify forward alone (dvlm_forward_quad)."""

@@ -26,6 +26,8 @@ void engine_set_trace(dvlm_engine* e, void* buf, int cap, int32_t* cnt);
 bool prefill_gemm_supported(const dvlm_engine* e);
 bool quad_supported(const dvlm_engine* e, int B);
 cudaError_t engine_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out, cudaStream_t s);
+bool engine_set_paged(dvlm_engine* e, void* k_pages, void* v_pages, const int32_t* table, int n_pages,
+                      int max_pages);
 cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, const int32_t* ids, int n_ids,
                                 cudaStream_t s);
 cudaError_t launch_topk_commit(const float* p1, const int32_t* ids, const int32_t* other_ids, uint8_t* masked,
@@ -42,6 +44,15 @@ inline dvlm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DVLM_O
 inline int sms_or_default() {
   const int n = device_sm_count();
   return n > 0 ? n : kDefaultSms;
+}
+// Attention cluster size for the current device: 16 CTAs where two such
+// clusters can be resident at once, else 8 (queried once per device).
+inline int attn_cluster_for_device() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return attn_max_clusters(16) >= 2 ? 16 : 8;
+  if (cached[dev] == 0) cached[dev] = attn_max_clusters(16) >= 2 ? 16 : 8;
+  return cached[dev];
 }
 inline int lm_nt(int R) { return R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128; }
 
@@ -178,9 +189,45 @@ dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const
   a.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
   a.out = static_cast<bf16*>(out);
   a.status = dev_status;
-  static int cs_attn = 0;  // cluster size, chosen once per process
-  if (cs_attn == 0) cs_attn = attn_max_clusters(16) >= 2 ? 16 : 8;
-  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), cs_attn));
+  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), attn_cluster_for_device()));
+}
+
+dvlm_status dvlm_block_attn_paged(const void* q, void* out, const void* k_pages, const void* v_pages,
+                                  const int32_t* block_table, const int32_t* lens, int n_batch, int n_rows,
+                                  int n_clean, int n_pages, int max_pages, int Hq, int Hkv, int D, float scale,
+                                  int* dev_status, dvlm_stream stream) {
+  if (!q || !out || !k_pages || !v_pages || !block_table || !lens) return DVLM_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return DVLM_ERR_INVALID_ARG;
+  if (n_batch < 1 || n_rows < 1 || n_rows > 64 || n_clean < 0 || n_clean > n_rows || n_pages < 1 || max_pages < 1 ||
+      Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv)
+    return DVLM_ERR_SHAPE;
+  if (D != 128 || Hq != 8 * Hkv) return DVLM_ERR_UNSUPPORTED;
+  if (!al16(q) || !al16(out) || !al16(k_pages) || !al16(v_pages)) return DVLM_ERR_INVALID_ARG;
+  const int n_groups = (n_rows + 15) / 16;
+  if (static_cast<long long>(n_batch) * n_groups > 65535) return DVLM_ERR_SHAPE;
+  CUtensorMap mq, mk, mv;
+  const uint64_t rows_total = static_cast<uint64_t>(n_batch) * n_rows;
+  const uint64_t page_rows = static_cast<uint64_t>(n_pages) * Hkv;
+  bool ok = make_tmap_3d(&mq, q, D, Hq, rows_total, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
+  ok &= make_tmap_2d(&mk, k_pages, D, page_rows * 64, D * 2, 64, 64);
+  ok &= make_tmap_2d(&mv, v_pages, 64, page_rows * D, 64 * 2, 64, 128);
+  if (!ok) return DVLM_ERR_CUDA;
+  AttnArgs a{};
+  a.n_rows = n_rows;
+  a.n_clean = n_clean;
+  a.n_batch = n_batch;
+  a.Lmax = 64;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.kv_base = 0;
+  a.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  a.out = static_cast<bf16*>(out);
+  a.status = dev_status;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.n_pages = n_pages;
+  a.d_lens = lens;
+  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), attn_cluster_for_device()));
 }
 
 // ------------------------------------------------------------ LM head
@@ -429,7 +476,7 @@ static dvlm_status check_cfg(dvlm_engine* e, const dvlm_decode_cfg* cfg) {
   if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_SPEC_QUAD) return DVLM_ERR_INVALID_ARG;
   if (cfg->mode == DVLM_MODE_SPEC_QUAD && !quad_supported(e, cfg->block_size)) return DVLM_ERR_UNSUPPORTED;
   if (cfg->mode == DVLM_MODE_ROUTE) {
-    if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+    if (!e->bf16 || e->paged) return DVLM_ERR_UNSUPPORTED;
     if (cfg->route_k < 1 || cfg->route_n_vis < 0 || cfg->route_n_vis % 8 || cfg->block_size < 2) return DVLM_ERR_SHAPE;
   }
   if (std::isnan(cfg->threshold)) return DVLM_ERR_INVALID_ARG;
@@ -586,7 +633,7 @@ dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_t* tokens
 dvlm_status dvlm_forward_text_only(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked, int n_rows,
                                    int n_hidden, void* x_out, dvlm_stream stream) {
   if (!e || !tokens) return DVLM_ERR_INVALID_ARG;
-  if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+  if (!e->bf16 || e->paged) return DVLM_ERR_UNSUPPORTED;
   if (n_rows < 1 || n_rows > kNT || n_hidden < 0 || n_hidden % 8) return DVLM_ERR_SHAPE;
   if (x_out && !al16(x_out)) return DVLM_ERR_INVALID_ARG;
   cudaStream_t s = cs(stream);
@@ -640,6 +687,15 @@ dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value) 
   if (!e || !name) return DVLM_ERR_INVALID_ARG;
   if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
   return engine_set_option(e, name, value);
+}
+
+dvlm_status dvlm_engine_set_paged(dvlm_engine* e, void* k_pages, void* v_pages, const int32_t* block_table,
+                                  int n_pages, int max_pages) {
+  if (!e || !k_pages || !v_pages || !block_table) return DVLM_ERR_INVALID_ARG;
+  if (!e->bf16) return DVLM_ERR_UNSUPPORTED;
+  if (n_pages < 1 || max_pages < 1 || static_cast<long long>(max_pages) * 64 < e->Lmax) return DVLM_ERR_SHAPE;
+  if (!al16(k_pages) || !al16(v_pages)) return DVLM_ERR_INVALID_ARG;
+  return engine_set_paged(e, k_pages, v_pages, block_table, n_pages, max_pages) ? DVLM_OK : DVLM_ERR_CUDA;
 }
 
 dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int B, void* x_out, dvlm_stream stream) {

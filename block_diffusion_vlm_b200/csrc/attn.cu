@@ -111,7 +111,11 @@ __global__ void __launch_bounds__(192, 1)
   // end of a forward pass moves it), and so are the cache slots below it: both
   // may be read before waiting for the predecessor.  Slots L.. are written by
   // the QKV projection this kernel follows.
-  const int L = (a.d_len ? *a.d_len : a.L_static) - a.len_sub;
+  int L = (a.d_lens ? a.d_lens[bidx] : a.d_len ? *a.d_len : a.L_static) - a.len_sub;
+  if (a.block_table && L + a.n_rows > a.max_pages * kChunk) {  // the table cannot hold this length
+    record_error(a.status, DVLM_ERR_BOUNDS);
+    L = a.max_pages * kChunk - a.n_rows;
+  }
   const int Ltot = L + a.n_rows;
   // Chunk j of 64 keys belongs to CTA j % kCS (round robin): a row's partial
   // sums then do not depend on how many rows the step has, so a causal row
@@ -127,10 +131,21 @@ __global__ void __launch_bounds__(192, 1)
         const int st = jj & 1;
         const int key0 = (crank + kCS * jj) * kChunk;
         mbar_arrive_expect_tx(&kv_full[st], kKBytes + kVBytes);
+        int krow = kv_row0 * a.Lmax + key0, vrow = kv_row0 * 128, vx = key0;
+        if (a.block_table) {  // chunk = one 64-slot page
+          int page = a.block_table[bidx * a.max_pages + key0 / kChunk];
+          if (page < 0 || page >= a.n_pages) {
+            record_error(a.status, DVLM_ERR_BOUNDS);
+            page = 0;
+          }
+          const int pe = (a.kv_base * a.n_pages + page) * a.Hkv + g;  // (layer, page, KV head)
+          krow = pe * kChunk;
+          vrow = pe * 128;
+          vx = 0;
+        }
         for (int h = 0; h < 2; ++h)
-          tma_load_2d(sK + st * kKBytes + h * (kKBytes / 2), &mapK, &kv_full[st], h * 64, kv_row0 * a.Lmax + key0,
-                      pol);
-        tma_load_2d(sV + st * kVBytes, &mapV, &kv_full[st], key0, kv_row0 * 128, pol);
+          tma_load_2d(sK + st * kKBytes + h * (kKBytes / 2), &mapK, &kv_full[st], h * 64, krow, pol);
+        tma_load_2d(sV + st * kVBytes, &mapV, &kv_full[st], vx, vrow, pol);
       };
       const int first = nc < 2 ? nc : 2;
       bool early[2] = {false, false};
@@ -453,15 +468,18 @@ __global__ void __launch_bounds__(192, 1)
 template <int CS>
 static cudaError_t attn_launch(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                const AttnArgs& a, bool pdl, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  // function attributes are per device: set once on each device that launches
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     if (CS > 8) {
       e = cudaFuncSetAttribute(attn_bf16_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
     }
-    attr_set = true;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int n_groups = (a.n_rows + 15) / 16;
   cudaLaunchConfig_t cfg = {};

@@ -274,7 +274,13 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   ea.part = e->gpart;
   ea.cnt = e->gcnt;
   ea.status = e->d_status;
-  const size_t kv_layer = static_cast<size_t>(Hkv) * e->Lmax * D;
+  // per-layer cache stride: contiguous [Hkv][Lmax][D], or paged [n_pages][Hkv][64][D]
+  const size_t kv_layer = e->paged ? static_cast<size_t>(e->n_pages) * Hkv * 64 * D
+                                   : static_cast<size_t>(Hkv) * e->Lmax * D;
+  if (e->paged) {
+    ea.block_table = e->block_table;
+    ea.n_pages = e->n_pages;
+  }
   for (int l = f.layer0; l < l1; ++l) {
     ea.epi = EPI_QKV;
     ea.n_ssq = n_ssq;
@@ -315,6 +321,11 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     aa.out = static_cast<bf16*>(e->attn_o);
     aa.status = e->d_status;
+    if (e->paged) {
+      aa.block_table = e->block_table;
+      aa.max_pages = e->max_pages;
+      aa.n_pages = e->n_pages;
+    }
     T0(K_ATTN);
     if (f.hide > 0) {
       aa.len_sub = f.hide;  // the view starts f.hide slots into the cache
@@ -478,7 +489,7 @@ static cudaError_t fwd_f32(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
 bool prefill_gemm_supported(const dvlm_engine* e) {
   const dvlm_model& m = e->m;
   const int qkv_rows = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim;
-  return e->bf16 && !e->fp8 && e->max_ctx > 0 && m.head_dim == 128 && m.hidden % 256 == 0 && m.inter % 128 == 0 &&
+  return e->bf16 && !e->fp8 && !e->paged && e->max_ctx > 0 && m.head_dim == 128 && m.hidden % 256 == 0 && m.inter % 128 == 0 &&
          qkv_rows % 256 == 0 && (m.n_q_heads * m.head_dim) % 64 == 0;
 }
 
@@ -1159,6 +1170,34 @@ void engine_set_trace(dvlm_engine* e, void* buf, int cap, int32_t* cnt) {
   e->trace_cnt = buf ? cnt : nullptr;
   for (auto& kv : e->graphs) cudaGraphExecDestroy(kv.second);
   e->graphs.clear();
+}
+
+// Switches the engine to a paged KV cache [Fast-dVLM technical overview
+// (ocdem.com), section 2.3.2: paged KV cache management]: attention reads
+// 64-key chunks through the block table, the QKV epilogue writes each new
+// K/V row through it; the compute-bound prefill, the fused quadratic forward
+// and the TEXT-ONLY views (contiguous layouts) are not used.
+bool engine_set_paged(dvlm_engine* e, void* k_pages, void* v_pages, const int32_t* table, int n_pages,
+                      int max_pages) {
+  const dvlm_model& m = e->m;
+  const uint64_t rows = static_cast<uint64_t>(m.n_layers) * n_pages * m.n_kv_heads;
+  CUtensorMap tk, tv;
+  if (!make_tmap_2d(&tk, k_pages, m.head_dim, rows * 64, m.head_dim * 2, 64, 64) ||
+      !make_tmap_2d(&tv, v_pages, 64, rows * m.head_dim, 64 * 2, 64, 128))
+    return false;
+  e->tm_k = tk;
+  e->tm_v = tv;
+  e->kc = k_pages;
+  e->vc = v_pages;
+  e->block_table = table;
+  e->n_pages = n_pages;
+  e->max_pages = max_pages;
+  e->paged = true;
+  e->prefill_gemm = false;
+  e->quad_ready = false;
+  for (auto& kv : e->graphs) cudaGraphExecDestroy(kv.second);
+  e->graphs.clear();
+  return true;
 }
 
 size_t engine_workspace_bytes(dvlm_engine* e, int P) { return carve(e, nullptr, true, P); }

@@ -91,6 +91,11 @@ struct dvlm_engine {
   int gu_cps = 1;                       // gate/up CTAs per SM (2 needs 5 stages)
   bool pdl = true;                      // programmatic dependent launch between kernels
   bool prefill_gemm = true;             // compute-bound prefill (prefill.cu) where the shapes allow it
+  // paged KV cache (dvlm_engine_set_paged): kc / vc are 64-slot pages
+  // [n_layers][n_pages][Hkv][64][D] and [n_layers][n_pages][Hkv][D][64]
+  bool paged = false;
+  const int32_t* block_table = nullptr;  // [max_pages] page of each 64-slot chunk
+  int n_pages = 0, max_pages = 0;
   // device buffers carved from the workspace
   void* x = nullptr;        // [NT][H]
   void* q = nullptr;        // [NT][Hq*D]

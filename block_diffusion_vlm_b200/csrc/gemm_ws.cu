@@ -260,19 +260,24 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
                 bf16* q = ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128;
                 q[j] = y1;
                 q[j + 64] = y2;
-              } else {
-                bf16* k = ea.kcache + (static_cast<size_t>(T - nq) * ea.Lmax + (L0 + t)) * 128;
+              } else if (bf16* k = kv_k_ptr(ea, T - nq, L0 + t)) {
                 k[j] = y1;
                 k[j + 64] = y2;
+              } else {
+                record_error(ea.status, DVLM_ERR_BOUNDS);
               }
             }
           } else {
             const int h = T - nq - nkv;
             for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
-              ea.vcache[(static_cast<size_t>(h) * 128 + j) * ea.Lmax + (L0 + t)] =
-                  __float2bfloat16_rn(sE[j * (NT + 1) + t]);
-              ea.vcache[(static_cast<size_t>(h) * 128 + j + 64) * ea.Lmax + (L0 + t)] =
-                  __float2bfloat16_rn(sE[(j + 64) * (NT + 1) + t]);
+              bf16* v1 = kv_v_ptr(ea, h, j, L0 + t);
+              bf16* v2 = kv_v_ptr(ea, h, j + 64, L0 + t);
+              if (!v1 || !v2) {
+                record_error(ea.status, DVLM_ERR_BOUNDS);
+                continue;
+              }
+              *v1 = __float2bfloat16_rn(sE[j * (NT + 1) + t]);
+              *v2 = __float2bfloat16_rn(sE[(j + 64) * (NT + 1) + t]);
             }
           }
         }
@@ -523,14 +528,23 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
           const float co = pre_a[k], si = pre_b[k];
           const bf16 y1 = __float2bfloat16_rn(x1 * co - x2 * si);
           const bf16 y2 = __float2bfloat16_rn(x2 * co + x1 * si);
-          bf16* dst = (T < nq) ? ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128
-                               : ea.kcache + (static_cast<size_t>(T - nq) * ea.Lmax + (L0 + t)) * 128;
+          bf16* dst = (T < nq) ? ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128 : kv_k_ptr(ea, T - nq, L0 + t);
+          if (!dst) {
+            record_error(ea.status, DVLM_ERR_BOUNDS);
+            continue;
+          }
           dst[j] = y1;
           dst[j + 64] = y2;
         } else {
           const int h = T - nq - nkv;
-          ea.vcache[(static_cast<size_t>(h) * 128 + j) * ea.Lmax + (L0 + t)] = __float2bfloat16_rn(x1);
-          ea.vcache[(static_cast<size_t>(h) * 128 + j + 64) * ea.Lmax + (L0 + t)] = __float2bfloat16_rn(x2);
+          bf16* v1 = kv_v_ptr(ea, h, j, L0 + t);
+          bf16* v2 = kv_v_ptr(ea, h, j + 64, L0 + t);
+          if (!v1 || !v2) {
+            record_error(ea.status, DVLM_ERR_BOUNDS);
+            continue;
+          }
+          *v1 = __float2bfloat16_rn(x1);
+          *v2 = __float2bfloat16_rn(x2);
         }
       }
     }
@@ -549,11 +563,14 @@ static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2,
                               const SkSched& sc, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
   using S = GemmSmem<NT, ST, FP8>;
   auto kern = gemm_ws_kernel<NT, ST, EPI, FP8>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // function attributes are per device: set once on each device that launches
+  static bool attr_set[64] = {};
+  int dev_ = 0;
+  if (cudaGetDevice(&dev_) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev_ < 0 || dev_ >= 64 || !attr_set[dev_]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev_ >= 0 && dev_ < 64) attr_set[dev_] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sc.P);
@@ -573,13 +590,16 @@ static cudaError_t launch_cl(const CUtensorMap& mapA, const CUtensorMap& mapB, i
                              int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
   using Sm = ClSmem<NT, ST, FP8>;
   auto kern = gemm_cl_kernel<NT, ST, EPI, FP8>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // function attributes are per device: set once on each device that launches
+  static bool attr_set[64] = {};
+  int dev_ = 0;
+  if (cudaGetDevice(&dev_) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev_ < 0 || dev_ >= 64 || !attr_set[dev_]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev_ >= 0 && dev_ < 64) attr_set[dev_] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles * S);

@@ -54,7 +54,27 @@ struct GemmEpi {
   const float* wscale;
   const float* wscale2;
   float* amax_out;
+  // Paged cache (block_table != NULL): slot s of the sequence is row s % 64 of
+  // page block_table[s / 64] (n_pages pages); kcache / vcache then point at
+  // this layer's pages, K [n_pages][Hkv][64][128], V^T [n_pages][Hkv][128][64].
+  const int* block_table;
+  int n_pages;
 };
+
+// Destination of cache slot `slot`, KV head h (value feature j) in a
+// contiguous or paged cache (see GemmEpi); NULL for a page id out of range.
+__device__ __forceinline__ bf16* kv_k_ptr(const GemmEpi& ea, int h, int slot) {
+  if (!ea.block_table) return ea.kcache + (static_cast<size_t>(h) * ea.Lmax + slot) * 128;
+  const int page = ea.block_table[slot >> 6];
+  if (page < 0 || page >= ea.n_pages) return nullptr;
+  return ea.kcache + (static_cast<size_t>(page * ea.n_kv_heads + h) * 64 + (slot & 63)) * 128;
+}
+__device__ __forceinline__ bf16* kv_v_ptr(const GemmEpi& ea, int h, int j, int slot) {
+  if (!ea.block_table) return ea.vcache + (static_cast<size_t>(h) * 128 + j) * ea.Lmax + slot;
+  const int page = ea.block_table[slot >> 6];
+  if (page < 0 || page >= ea.n_pages) return nullptr;
+  return ea.vcache + (static_cast<size_t>(page * ea.n_kv_heads + h) * 128 + j) * 64 + (slot & 63);
+}
 
 // Fused LM head operands.
 struct LmArgs {
@@ -127,6 +147,13 @@ struct AttnArgs {
   bf16* out;                 // [n_batch][n_rows][Hq][128]
   int* status;
   int len_sub;               // the length used is (*d_len or L_static) - len_sub (offset cache views)
+  // Paged cache (block_table != NULL): 64-slot pages; logical slot s of batch
+  // entry b lives in row s % 64 of page block_table[b * max_pages + s / 64].
+  // K pages [kv_base layers][n_pages][Hkv][64][128], V^T pages
+  // [layers][n_pages][Hkv][128][64]; d_lens[b] (device) is entry b's length.
+  const int* block_table;
+  int max_pages, n_pages;
+  const int* d_lens;
 };
 // cs: CTAs per cluster splitting the keys (8, or 16 where the device can
 // co-schedule 16-CTA clusters; see attn_cluster_size()).

@@ -305,11 +305,14 @@ static cudaError_t lm_launch(const CUtensorMap& mapW, const CUtensorMap& mapH, c
                              bool pdl, cudaStream_t s) {
   using C = LmCfg<NT>;
   auto kern = lmhead_kernel<NT, C::STAGES>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // function attributes are per device: set once on each device that launches
+  static bool attr_set[64] = {};
+  int dev_ = 0;
+  if (cudaGetDevice(&dev_) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev_ < 0 || dev_ >= 64 || !attr_set[dev_]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kTotal);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev_ >= 0 && dev_ < 64) attr_set[dev_] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sc.P);

@@ -170,6 +170,24 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit_static(const void* hidden, const vo
                                                    const int32_t* anchor_id, const float* anchor_conf,
                                                    int32_t* cert_len, int* dev_status, dvlm_stream stream);
 
+/* Block-masked attention over PAGED KV caches [Fast-dVLM technical overview
+ * (ocdem.com), section 2.3.2: paged KV cache management], bf16: the rules of
+ * dvlm_block_attn for each of n_batch sequences, whose caches live in 64-slot
+ * pages.  Logical slot s of sequence b is row s % 64 of page
+ * block_table[b * max_pages + s / 64] (device int32 [n_batch, max_pages]);
+ * k_pages [n_pages, Hkv, 64, D], v_pages [n_pages, Hkv, D, 64] (transposed);
+ * lens (device int32 [n_batch]) gives each sequence's cache length L_b, its
+ * rows' K/V already at slots L_b..L_b+n_rows-1; q [n_batch, n_rows, Hq, D],
+ * out likewise.  Ragged lengths are the point: every sequence is the
+ * per-sequence definition and sees only its own pages.  D == 128, Hq == 8 *
+ * Hkv, n_rows <= 64.  A page id outside 0..n_pages-1 or a length the table
+ * cannot hold sets DVLM_ERR_BOUNDS in *dev_status (that chunk then reads page
+ * 0 / the length is clamped; no out-of-range access).  Asynchronous. */
+DVLM_API dvlm_status dvlm_block_attn_paged(const void* q, void* out, const void* k_pages, const void* v_pages,
+                                          const int32_t* block_table, const int32_t* lens, int n_batch,
+                                          int n_rows, int n_clean, int n_pages, int max_pages, int Hq, int Hkv,
+                                          int D, float scale, int* dev_status, dvlm_stream stream);
+
 /* ------------------------------------------------------------------------
  * Top-k commit [Look Only When Needed, background: the baseline dVLM
  * schedule unmasks the k most confident masked positions per step].
@@ -380,6 +398,21 @@ DVLM_API dvlm_status dvlm_engine_check(dvlm_engine* e, dvlm_stream stream);
 DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_t* tokens,
                          const uint8_t* masked, int n_rows, int n_clean, int first_layer,
                          int n_layers_run, int advance, void* x_out, dvlm_stream stream);
+
+/* Paged KV cache for an engine [Fast-dVLM technical overview (ocdem.com),
+ * section 2.3.2: paged KV cache management]: from now on the engine's cache
+ * is k_pages [n_layers, n_pages, Hkv, 64, D] and v_pages [n_layers, n_pages,
+ * Hkv, D, 64] (bf16, device, caller-owned), logical slot s living in row
+ * s % 64 of page block_table[s / 64] (device int32 [max_pages], read at each
+ * launch: the caller may extend it between calls).  Attention reads 64-key
+ * chunks through the table and the QKV projection writes each new K/V row
+ * through it; results equal those of the contiguous cache bit for bit.
+ * Prefill runs in 16-row forwards; DVLM_MODE_SPEC_QUAD, DVLM_MODE_ROUTE and
+ * dvlm_forward_text_only are unsupported on a paged engine.  max_pages * 64
+ * must cover the engine's Lmax (DVLM_ERR_SHAPE).  A page id outside
+ * 0..n_pages-1 is reported as DVLM_ERR_BOUNDS in the status word. */
+DVLM_API dvlm_status dvlm_engine_set_paged(dvlm_engine* e, void* k_pages, void* v_pages,
+                                          const int32_t* block_table, int n_pages, int max_pages);
 
 /* Test hook: the fused draft+verify forward of quadratic self-speculative
  * decoding alone, over draft [B] (device int32, copied into the engine's

@@ -109,7 +109,8 @@ class Replay:
     hidden_check(x_gpu, x_oracle, what) asserts the hidden bar.  p1_tol
     bounds |p1(GPU) - p1(deciding oracle)|.  seed_bar: margin for the first
     AR seed, which comes from the prefill (scored by the oracle's own rows:
-    the prefill is not traced).  hidden_fn(index, record) returns the
+    the prefill is not traced; None: not checked, only teacher-forced).
+    hidden_fn(index, record) returns the
     oracle's final rows of a record computed beforehand (layer-major replay,
     see layer_major_hidden); by default each record runs model.forward."""
 
@@ -166,6 +167,8 @@ class Replay:
 
     def _seed_check(self, gpu_seed: int) -> None:
         c = self.seed_conf
+        if self.seed_bar is None:   # the first seed is only teacher-forced
+            c = None
         if c is not None:
             if c.p1[0] - c.p2[0] >= self.seed_bar:
                 assert gpu_seed == c.top1[0], ("seed", gpu_seed, int(c.top1[0]))
