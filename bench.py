@@ -522,12 +522,29 @@ def run_sweep(args, local):
 
                     ms, mode = _device_ms_per_call(call, 20 if nb > 1 else 200, dev)
                     b = nb * algorithmic_bytes("attention", dims, L, rows=B)
-                    emit({"sweep": "attention", "B": B, "L": L, "caches_per_launch": nb,
+                    emit({"sweep": "attention", "kernel": "cluster", "B": B, "L": L, "caches_per_launch": nb,
                           "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
                           "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
                           "frac": b / (ms * 1e-3) / 1e9 / hbm_peak,
                           "working_set_mb": (kd.numel() + vt.numel()) * 2 / 1e6, "timing": mode})
-                    del qd, kd, vt, out
+                    # the split form: enough CTAs to fill the SMs (one CTA per 128-key chunk at most)
+                    n_chunks = (L + B + 127) // 128
+                    groups = nb * ((B + 15) // 16) * Hkv
+                    splits = max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
+                    ws = torch.zeros((dv.block_attn_split_workspace_size(nb, B, Hkv, splits) + 3) // 4,
+                                     dtype=torch.int32, device=dev)
+
+                    def call_split():
+                        dv.block_attn_split(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
+                                            Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, splits=splits, workspace=ws,
+                                            status=st)
+
+                    ms, mode = _device_ms_per_call(call_split, 20 if nb > 1 else 200, dev)
+                    emit({"sweep": "attention", "kernel": "split", "splits": splits, "B": B, "L": L,
+                          "caches_per_launch": nb, "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
+                          "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
+                          "frac": b / (ms * 1e-3) / 1e9 / hbm_peak, "timing": mode})
+                    del qd, kd, vt, out, ws
         # TEXT-ONLY pass of certificate-guided routing at the decode shape: the
         # 1280 vision slots hidden by viewing the cache from slot 1280 (64 spare
         # slots keep the last key chunk inside each head's rows)

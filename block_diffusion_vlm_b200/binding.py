@@ -123,6 +123,9 @@ def _declare(L: ctypes.CDLL) -> None:
         "dvlm_quantize_rows_e4m3": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
         "dvlm_forward_quad": (_i, [_vp, _vp, _i, _vp, _vp]),
         "dvlm_engine_set_paged": (_i, [_vp, _vp, _vp, _vp, _i, _i]),
+        "dvlm_block_attn_split_workspace_size": (_sz, [_i, _i, _i, _i]),
+        "dvlm_block_attn_split": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp,
+                                       _vp]),
         "dvlm_block_attn_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
         "dvlm_engine_set_trace": (_i, [_vp, _vp, _sz, _vp]),
     }
@@ -163,6 +166,20 @@ def block_attn(q, out, k_cache, v_cache, *, n_batch, n_rows, n_clean, L, Lmax, H
     _check(lib().dvlm_block_attn(ptr(q), ptr(out), ptr(k_cache), ptr(v_cache), n_batch, n_rows, n_clean, L, Lmax,
                                  Hq, Hkv, D, float(scale), dtype, ptr(status), stream_handle(stream)),
            "dvlm_block_attn")
+
+
+def block_attn_split_workspace_size(n_batch: int, n_rows: int, Hkv: int, splits: int) -> int:
+    return int(lib().dvlm_block_attn_split_workspace_size(n_batch, n_rows, Hkv, splits))
+
+
+def block_attn_split(q, out, k_cache, v_cache, *, n_batch, n_rows, n_clean, L, Lmax, Hq, Hkv, D, scale, splits,
+                     workspace, status=None, stream=None) -> None:
+    """Split-CTA block attention (dvlm_block_attn_split)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().dvlm_block_attn_split(ptr(q), ptr(out), ptr(k_cache), ptr(v_cache), n_batch, n_rows, n_clean, L,
+                                       Lmax, Hq, Hkv, D, float(scale), int(splits), ptr(workspace), ws_bytes,
+                                       ptr(status), stream_handle(stream)),
+           "dvlm_block_attn_split")
 
 
 def block_attn_paged(q, out, k_pages, v_pages, block_table, lens, *, n_batch, n_rows, n_clean, n_pages, max_pages,

@@ -192,6 +192,48 @@ dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const
   return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), attn_cluster_for_device()));
 }
 
+size_t dvlm_block_attn_split_workspace_size(int n_batch, int n_rows, int Hkv, int splits) {
+  if (n_batch < 1 || n_rows < 1 || Hkv < 1 || splits < 1 || splits > 64) return 0;
+  return attn_split_scratch_bytes(n_batch * ((n_rows + 15) / 16) * Hkv, splits);
+}
+
+dvlm_status dvlm_block_attn_split(const void* q, void* out, const void* k_cache, const void* v_cache, int n_batch,
+                                  int n_rows, int n_clean, int L, int Lmax, int Hq, int Hkv, int D, float scale,
+                                  int splits, void* workspace, size_t ws_bytes, int* dev_status,
+                                  dvlm_stream stream) {
+  if (!q || !out || !k_cache || !v_cache) return DVLM_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return DVLM_ERR_INVALID_ARG;
+  if (n_batch < 1 || n_rows < 1 || n_clean < 0 || n_clean > n_rows || L < 0 || Lmax < 1 || Hq < 1 || Hkv < 1 ||
+      D < 1 || Hq % Hkv || splits < 1 || splits > 64)
+    return DVLM_ERR_SHAPE;
+  if (static_cast<long long>(L) + n_rows > Lmax) return DVLM_ERR_CACHE_OVERFLOW;
+  if (D != 128 || Hq != 8 * Hkv) return DVLM_ERR_UNSUPPORTED;
+  if (Lmax % 8) return DVLM_ERR_SHAPE;
+  if (!al16(q) || !al16(out) || !al16(k_cache) || !al16(v_cache) || !al16(workspace)) return DVLM_ERR_INVALID_ARG;
+  const int n_groups = (n_rows + 15) / 16;
+  if (static_cast<long long>(n_batch) * n_groups > 65535) return DVLM_ERR_SHAPE;
+  if (!workspace || ws_bytes < attn_split_scratch_bytes(n_batch * n_groups * Hkv, splits)) return DVLM_ERR_WORKSPACE;
+  CUtensorMap mq, mk, mv;
+  const uint64_t rows_total = static_cast<uint64_t>(n_batch) * n_rows;
+  bool ok = make_tmap_3d(&mq, q, D, Hq, rows_total, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
+  ok &= make_tmap_2d(&mk, k_cache, D, static_cast<uint64_t>(n_batch) * Hkv * Lmax, D * 2, 64, 64);
+  ok &= make_tmap_2d(&mv, v_cache, Lmax, static_cast<uint64_t>(n_batch) * Hkv * D, static_cast<uint64_t>(Lmax) * 2,
+                     64, 128);
+  if (!ok) return DVLM_ERR_CUDA;
+  AttnArgs a{};
+  a.n_rows = n_rows;
+  a.n_clean = n_clean;
+  a.n_batch = n_batch;
+  a.L_static = L;
+  a.Lmax = Lmax;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  a.out = static_cast<bf16*>(out);
+  a.status = dev_status;
+  return cuda_status(launch_attn_split(mq, mk, mv, a, splits, workspace, false, cs(stream)));
+}
+
 dvlm_status dvlm_block_attn_paged(const void* q, void* out, const void* k_pages, const void* v_pages,
                                   const int32_t* block_table, const int32_t* lens, int n_batch, int n_rows,
                                   int n_clean, int n_pages, int max_pages, int Hq, int Hkv, int D, float scale,

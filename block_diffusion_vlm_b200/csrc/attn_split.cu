@@ -1,0 +1,408 @@
+// Block-masked GQA attention split over independent CTAs (flash-decoding
+// style), bf16, tcgen05: the bandwidth-bound form of the decode attention.
+//
+// Visibility [Fast-dVLM technical overview (ocdem.com), section 2.2.1;
+// Fast-dVLM walkthrough (itsolotime.com), section 4.1]: a clean row t (slot
+// L+t) sees slots 0..L+t (C2C); a noisy row sees slots 0..L+n_rows-1 (N2C and
+// N2N).  The same rules as attn_bf16_kernel; only the work split differs.
+//
+// Tile: one KV head's 8 query heads x 16 step rows = 128 rows (token-major,
+// head-minor, as a 3-D TMA box lands).  Keys go in 128-key chunks, chunk j
+// to split j % S (round robin by absolute key position, so a causal row's
+// arithmetic is the same whatever the number of rows in the step: a 1-row AR
+// pass and a 16-row verify pass give bitwise the same output).  Each of the S
+// CTAs of a (batch entry, row group, KV head) streams its chunks through a
+// 2-stage TMA pipeline (S = Q K^T and O += P V in TMEM, online softmax in
+// fp32 with one thread per row, P and V in fp16 for the second product),
+// then stores its partial rows (O / l in fp32, and (m, l)) to global scratch
+// and counts itself on the group's counter; the last CTA to arrive merges the
+// S partials in split order (deterministic) and writes the bf16 output.  No
+// CTA waits for another.  Paged caches read each 64-key half chunk through
+// the block table.
+#include <cuda_fp16.h>
+
+#include "kernels.h"
+#include "mainloop.cuh"
+
+namespace dvlm {
+
+namespace {
+constexpr int kSpThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one row each)
+constexpr int kSpKeys = 128;           // keys per chunk
+constexpr int kSpAtom = 128 * 128;     // one 128-byte-swizzled 128-row operand atom (16 KB)
+constexpr int oSpQ = 0;                // Q: 2 atoms (d 0..63, 64..127)
+constexpr int oSpK = oSpQ + 2 * kSpAtom;   // K: 2 stages x 2 d-atoms
+constexpr int oSpV = oSpK + 4 * kSpAtom;   // V^T: 2 stages x 2 key-atoms
+constexpr int oSpP = oSpV + 4 * kSpAtom;   // P: 2 key-atoms
+constexpr int oSpBar = oSpP + 2 * kSpAtom;
+constexpr int kSpSmem = oSpBar + 256 + 1024;
+constexpr uint32_t kSpIdescS = idesc_bf16_f32(128, kSpKeys);
+constexpr uint32_t kSpIdescO = idesc_f16_f32(128, 128);
+constexpr int kSpTmem = 512;           // S: 2 x 128 columns, O: 128 columns
+}  // namespace
+
+size_t attn_split_scratch_bytes(int n_groups_total, int S) {
+  const size_t part = static_cast<size_t>(n_groups_total) * S * 128 * 128 * 4;
+  const size_t ml = static_cast<size_t>(n_groups_total) * S * 128 * 8;
+  return (part + 255) / 256 * 256 + (ml + 255) / 256 * 256 + (static_cast<size_t>(n_groups_total) * 4 + 255) / 256 * 256;
+}
+
+__global__ void __launch_bounds__(kSpThreads, 1)
+    attn_split_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                      const __grid_constant__ CUtensorMap mapV, const AttnArgs a, float* part, float2* ml,
+                      int* cnt) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem + oSpQ;
+  uint8_t* sK = smem + oSpK;
+  uint8_t* sV = smem + oSpV;
+  uint8_t* sP = smem + oSpP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oSpBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2] PV of the chunk in that stage done
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_empty = bars + 7;   // [2] the softmax warps have read S of that buffer
+  uint64_t* p_full = bars + 9;    // P of the current chunk written, O rescaled (one phase per chunk)
+  uint64_t* pv_done = bars + 10;  // PV of a chunk done (one phase per chunk)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = gridDim.x, sp = blockIdx.x, g = blockIdx.y;
+  const int n_groups = (a.n_rows + 15) / 16;
+  const int bidx = blockIdx.z / n_groups;
+  const int t_base = (blockIdx.z % n_groups) * 16;
+  const int grp = blockIdx.z * a.Hkv + g;  // one merge group per (batch entry, row group, KV head)
+
+  griddep_wait();
+  int L = (a.d_lens ? a.d_lens[bidx] : a.d_len ? *a.d_len : a.L_static) - a.len_sub;
+  if (a.block_table && L + a.n_rows > a.max_pages * 64) {
+    record_error(a.status, DVLM_ERR_BOUNDS);
+    L = a.max_pages * 64 - a.n_rows;
+  }
+  const int Ltot = L + a.n_rows;
+  const int n_all = (Ltot + kSpKeys - 1) / kSpKeys;
+  const int nc = sp < n_all ? (n_all - sp + S - 1) / S : 0;  // this CTA's chunks sp, sp+S, ...
+  const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 4 : 1);
+    *sabort = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mapQ);
+    tma_prefetch_map(&mapK);
+    tma_prefetch_map(&mapV);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kSpTmem);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // (layer, page, head) entry holding logical slot `key` of a paged cache
+  auto page_entry = [&](int key) -> int {
+    int page = a.block_table[bidx * a.max_pages + key / 64];
+    if (page < 0 || page >= a.n_pages) {
+      record_error(a.status, DVLM_ERR_BOUNDS);
+      page = 0;
+    }
+    return (a.kv_base * a.n_pages + page) * a.Hkv + g;
+  };
+
+  if (warp == 0) {
+    if (lane == 0 && nc > 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      mbar_arrive_expect_tx(q_full, 2 * kSpAtom);
+      for (int d = 0; d < 2; ++d)
+        tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, bidx * a.n_rows + t_base, pol);
+      for (int c = 0; c < nc; ++c) {
+        const int st = c & 1;
+        if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
+        mbar_arrive_expect_tx(&kv_full[st], 4 * kSpAtom);
+        const int key0 = (sp + c * S) * kSpKeys;
+        for (int hf = 0; hf < 2; ++hf) {  // 64-key halves: one page each in a paged cache
+          const int key = key0 + hf * 64;
+          int krow, vrow, vx;
+          if (a.block_table) {
+            const int pe = page_entry(key);
+            krow = pe * 64;
+            vrow = pe * 128;
+            vx = 0;
+          } else {
+            krow = kv_row0 * a.Lmax + key;
+            vrow = kv_row0 * 128;
+            vx = key;
+          }
+          for (int d = 0; d < 2; ++d)
+            tma_load_2d(sK + (2 * st + d) * kSpAtom + hf * (kSpAtom / 2), &mapK, &kv_full[st], d * 64, krow, pol);
+          tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &kv_full[st], vx, vrow, pol);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nc > 0) {
+      bool ok = mbar_wait(q_full, 0, a.status, sabort);
+      auto issue_pv = [&](int c) -> bool {
+        if (!mbar_wait(p_full, c & 1, a.status, sabort)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sP), vb = smem_u32(sV + 2 * (c & 1) * kSpAtom);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
+          umma_bf16_ss(tmem + 256, sdesc_kmajor_sw128(pa + off), sdesc_kmajor_sw128(vb + off), kSpIdescO,
+                       (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[c & 1]);
+        umma_commit(pv_done);
+        return true;
+      };
+      for (int c = 0; ok && c < nc; ++c) {
+        const int st = c & 1;
+        if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) break;
+        if (c >= 2 && !mbar_wait(&s_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kSpAtom);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
+          umma_bf16_ss(tmem + st * kSpKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off), kSpIdescS,
+                       kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        if (c >= 1) ok = issue_pv(c - 1);
+      }
+      if (ok) issue_pv(nc - 1);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    // The next kernel (the output projection) may launch now and stream its
+    // weights on idle SMs; it reads this kernel's output only after its own
+    // wait (at most two kernels overlap).
+    if (threadIdx.x == 64) griddep_launch_dependents();
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int t = t_base + (row >> 3);
+    const int limit = (t < a.n_clean) ? (L + t + 1) : Ltot;  // keys below `limit` are visible
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = nc > 0;
+    for (int c = 0; ok && c < nc; ++c) {
+      const int st = c & 1;
+      const int key0 = (sp + c * S) * kSpKeys;
+      if (!mbar_wait(&s_full[st], (c >> 1) & 1, a.status, sabort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        float sc[64];
+        tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (key0 + hf * 64 + k < limit) mx = fmaxf(mx, sc[k] * a.scale_log2);
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m == -INFINITY) ? (m_new == -INFINITY ? 1.f : 0.f) : exp2f(m - m_new);
+      uint32_t packed[64];
+      float psum = 0.f;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float sc[64];
+        tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const int key = key0 + hf * 64 + k;
+          const float p0 = (key < limit && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
+          const float p1 =
+              (key + 1 < limit && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
+          psum += p0 + p1;
+          const __half2 ph = __floats2half2_rn(p0, p1);
+          packed[hf * 32 + k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[st]);
+      if (c > 0) {
+        if (!mbar_wait(pv_done, (c - 1) & 1, a.status, sabort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+          for (int cc = 0; cc < 128; cc += 64) {
+            float o[64];
+            tmem_ld64(tmem + lane_off + 256u + cc, o);
+#pragma unroll
+            for (int k = 0; k < 64; ++k) o[k] *= alpha;
+#pragma unroll
+            for (int k = 0; k < 64; k += 16) tmem_st16_nowait(tmem + lane_off + 256u + cc + k, o + k);
+            tmem_wait_st();
+          }
+        }
+      }
+#pragma unroll
+      for (int at = 0; at < 2; ++at) {
+        uint8_t* prow = sP + at * kSpAtom + row * 128;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
+              make_uint4(packed[at * 32 + cc * 4], packed[at * 32 + cc * 4 + 1], packed[at * 32 + cc * 4 + 2],
+                         packed[at * 32 + cc * 4 + 3]);
+      }
+      // value row `row` (feature d = row) of this chunk to fp16 in place; keys
+      // past the valid slots (stale, poisoned, other pages' rows) become 0
+      if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) {
+        ok = false;
+        break;
+      }
+      {
+        const int n_valid = Ltot - key0;
+#pragma unroll
+        for (int at = 0; at < 2; ++at) {
+          uint8_t* vrow = sV + (2 * st + at) * kSpAtom + row * 128;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint4* p16 = reinterpret_cast<uint4*>(vrow + (cc << 4));
+            uint4 w = *p16;
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+              const int kk = at * 64 + ((cc ^ (row & 7)) << 3) + 2 * e;
+              const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
+              wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            *p16 = w;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      l = l * alpha + psum;
+      m = m_new;
+    }
+    // this split's partial rows: O / l (fp32) and (m, l)
+    const size_t pidx = static_cast<size_t>(grp) * S + sp;
+    float* prow = part + (pidx * 128 + row) * 128;
+    const bool have = ok && nc > 0 && mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort);
+    if (have) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < 128; cc += 64) {
+        float o[64];
+        tmem_ld64(tmem + lane_off + 256u + cc, o);
+#pragma unroll
+        for (int k = 0; k < 64; k += 4)
+          __stcg(reinterpret_cast<float4*>(prow + cc + k),
+                 make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l));
+      }
+    }
+    ml[pidx * 128 + row] = (have && l > 0.f) ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+    __threadfence();
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 64) *sflag = (atomicAdd(&cnt[grp], 1) == S - 1) ? 1 : 0;
+    named_bar_sync(1, 128);
+    if (*sflag) {
+      // ------------------------------------------------------------ merge
+      __threadfence();
+      if (threadIdx.x == 64) cnt[grp] = 0;  // every split arrived: zero for the next launch
+      const size_t p0 = static_cast<size_t>(grp) * S;
+      float M = -INFINITY;
+      for (int q = 0; q < S; ++q) M = fmaxf(M, __ldcg(&ml[(p0 + q) * 128 + row]).x);
+      float wsum = 0.f;
+      for (int q = 0; q < S; ++q) {
+        const float2 v = __ldcg(&ml[(p0 + q) * 128 + row]);
+        wsum += v.y > 0.f ? ex2_approx(v.x - M) * v.y : 0.f;
+      }
+      const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+      const int hl = row & 7;
+      bf16* dst = a.out + ((static_cast<size_t>(bidx) * a.n_rows + t) * a.Hq + g * 8 + hl) * 128;
+#pragma unroll 1
+      for (int d0 = 0; d0 < 128; d0 += 32) {
+        float acc[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+        for (int q = 0; q < S; ++q) {
+          const float2 v = __ldcg(&ml[(p0 + q) * 128 + row]);
+          if (!(v.y > 0.f)) continue;
+          const float w = ex2_approx(v.x - M) * v.y;
+          const float4* src = reinterpret_cast<const float4*>(part + ((p0 + q) * 128 + row) * 128 + d0);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 f = __ldcg(src + k);
+            acc[4 * k] += w * f.x;
+            acc[4 * k + 1] += w * f.y;
+            acc[4 * k + 2] += w * f.z;
+            acc[4 * k + 3] += w * f.w;
+          }
+        }
+        if (t < a.n_rows) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 8) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const __nv_bfloat162 b = __floats2bfloat162_rn(acc[k + 2 * q] * inv, acc[k + 2 * q + 1] * inv);
+              wv[q] = *reinterpret_cast<const uint32_t*>(&b);
+            }
+            *reinterpret_cast<uint4*>(dst + d0 + k) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kSpTmem);
+  }
+}
+
+// S CTAs per (batch entry, row group, KV head); scratch from
+// attn_split_scratch_bytes(n_batch * n_groups * Hkv, S), counters zero.
+cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                              const AttnArgs& a, int S, void* scratch, bool pdl, cudaStream_t s) {
+  if (S < 1 || S > 64 || !scratch) return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int n_groups = (a.n_rows + 15) / 16;
+  const int groups_total = a.n_batch * n_groups * a.Hkv;
+  const size_t part = static_cast<size_t>(groups_total) * S * 128 * 128 * 4;
+  const size_t ml = static_cast<size_t>(groups_total) * S * 128 * 8;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  float* p = reinterpret_cast<float*>(base);
+  float2* m = reinterpret_cast<float2*>(base + (part + 255) / 256 * 256);
+  int* c = reinterpret_cast<int*>(base + (part + 255) / 256 * 256 + (ml + 255) / 256 * 256);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, a.Hkv, a.n_batch * n_groups);
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = kSpSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_split_kernel, mapQ, mapK, mapV, a, p, m, c);
+}
+
+}  // namespace dvlm

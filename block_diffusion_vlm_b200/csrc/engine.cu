@@ -134,6 +134,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->stage_ids = c.take<int32_t>(std::max(e->max_ctx, 1) * 4);
   e->stage_out = c.take<int32_t>(static_cast<size_t>(e->Lmax) * 4);
   if (e->fp8) e->amax_act = c.take<float>(static_cast<size_t>(I / 64) * kNT * 4);
+  if (e->bf16) e->attn_scratch = c.take<void>(attn_split_scratch_bytes(m.n_kv_heads, kMaxAttnSplit));
   if (e->bf16 && !e->fp8 && e->max_ctx > 0) {
     const size_t C = static_cast<size_t>(e->max_ctx);
     e->px = c.take<void>(C * H * 2);
@@ -327,12 +328,13 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
       aa.n_pages = e->n_pages;
     }
     T0(K_ATTN);
-    if (f.hide > 0) {
-      aa.len_sub = f.hide;  // the view starts f.hide slots into the cache
-      DVLM_CK(launch_attn_bf16(e->tm_q, tm_k_text, tm_v_text, aa, pdl, s, e->attn_cs));
-    } else {
-      DVLM_CK(launch_attn_bf16(e->tm_q, e->tm_k, e->tm_v, aa, pdl, s, e->attn_cs));
-    }
+    if (f.hide > 0) aa.len_sub = f.hide;  // the view starts f.hide slots into the cache
+    const CUtensorMap& mk = f.hide > 0 ? tm_k_text : e->tm_k;
+    const CUtensorMap& mv = f.hide > 0 ? tm_v_text : e->tm_v;
+    if (e->attn_split > 0)
+      DVLM_CK(launch_attn_split(e->tm_q, mk, mv, aa, e->attn_split, e->attn_scratch, pdl, s));
+    else
+      DVLM_CK(launch_attn_bf16(e->tm_q, mk, mv, aa, pdl, s, e->attn_cs));
     T1(K_ATTN);
     ea.epi = EPI_RESID;
     ea.resid = x;
@@ -1103,7 +1105,7 @@ cudaError_t engine_profile(dvlm_engine* e, const FwdSpec& f0, float* ms, int* co
 dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
   const dvlm_model& m = e->m;
   const std::string n(name);
-  if (e->fp8 && n != "pdl" && n != "attn_cluster") return DVLM_ERR_UNSUPPORTED;
+  if (e->fp8 && n != "pdl" && n != "attn_cluster" && n != "attn_split") return DVLM_ERR_UNSUPPORTED;
   // every cluster of the projection resident at once (one wave)
   const int qkv_tiles = (m.n_q_heads + 2 * m.n_kv_heads) * m.head_dim / 128, h_tiles = m.hidden / 128;
   auto cluster_ok = [&](int epi, int S, int stages, int n_tiles) {
@@ -1136,6 +1138,9 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
     e->attn_cs = v;
   } else if (n == "pdl") {
     e->pdl = v != 0;
+  } else if (n == "attn_split") {
+    if (v < 0 || v > kMaxAttnSplit) return DVLM_ERR_SHAPE;
+    e->attn_split = v;
   } else if (n == "prefill_gemm") {
     if (v != 0 && v != 1) return DVLM_ERR_SHAPE;
     if (v && !prefill_gemm_supported(e)) return DVLM_ERR_UNSUPPORTED;
@@ -1158,6 +1163,7 @@ int engine_get_option(dvlm_engine* e, const char* name) {
   if (n == "gateup_ctas_per_sm") return e->gu_cps;
   if (n == "attn_cluster") return e->attn_cs;
   if (n == "pdl") return e->pdl ? 1 : 0;
+  if (n == "attn_split") return e->attn_split;
   if (n == "prefill_gemm") return e->prefill_gemm ? 1 : 0;
   return -1;
 }

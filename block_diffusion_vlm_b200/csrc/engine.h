@@ -65,7 +65,8 @@ struct FwdSpec {
 //   before the final RMSNorm.  Records are padded to 256 bytes.
 enum TraceKind { TR_NOISY = 1, TR_APPEND = 2, TR_DRAFT = 3, TR_VERIFY = 4, TR_AR = 5, TR_QUAD_VERIFY = 6,
                  TR_QUAD_CAND = 7, TR_ROUTE_FULL = 8, TR_ROUTE_TEXT = 9 };
-constexpr int kQuadSideKeys = 16 * 64;  // side-buffer keys per head: candidate block i at i * 64
+constexpr int kQuadSideKeys = 16 * 64;
+constexpr int kMaxAttnSplit = 32;  // side-buffer keys per head: candidate block i at i * 64
 constexpr int kTraceWords = 112;
 inline size_t trace_record_bytes(int hidden, bool bf16) {
   const size_t b = kTraceWords * 4 + static_cast<size_t>(kNT) * hidden * (bf16 ? 2 : 4);
@@ -87,6 +88,7 @@ struct dvlm_engine {
   int sm = 0;
   int s_qkv = 0, s_o = 0, s_down = 0;  // cluster sizes of the split-K projections (0: stream-K)
   int attn_cs = 8;                      // CTAs per attention cluster (8 or 16)
+  int attn_split = 0;                   // > 0: split attention with this many CTAs per KV head
   int gu_stages = 10, down_stages = 10; // pipeline depth of the gate/up and down projections
   int gu_cps = 1;                       // gate/up CTAs per SM (2 needs 5 stages)
   bool pdl = true;                      // programmatic dependent launch between kernels
@@ -141,6 +143,7 @@ struct dvlm_engine {
   void* pact = nullptr;          // [max_ctx][I] SwiGLU activation
   float* pssq = nullptr;         // [H/128][max_ctx] sums of squares
   float* amax_act = nullptr;     // fp8: [I/64][NT] largest |SwiGLU activation| per gate/up tile
+  void* attn_scratch = nullptr;  // split attention partials (up to kMaxAttnSplit CTAs per KV head)
   // quadratic self-speculative decoding (fused draft + verify forward)
   int32_t* qtok = nullptr;       // [max_ctx] input tokens of the fused forward
   int32_t* d_k = nullptr;        // accepted length of the last fused round

@@ -160,6 +160,13 @@ struct AttnArgs {
 cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                              const AttnArgs& a, bool pdl, cudaStream_t s, int cs = 8);
 int attn_max_clusters(int cs);
+// Split form of the same attention (csrc/attn_split.cu): S independent CTAs
+// per (batch entry, 16-row group, KV head), merged by the last to finish;
+// scratch of attn_split_scratch_bytes(n_batch * n_groups * Hkv, S) bytes whose
+// counters start at zero (they are zero again after each launch).
+size_t attn_split_scratch_bytes(int n_groups_total, int S);
+cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                              const AttnArgs& a, int S, void* scratch, bool pdl, cudaStream_t s);
 
 // Prefill (compute-bound path over the whole context; csrc/prefill.cu).
 // Token-major GEMM epilogue operands: one context row per epilogue thread.

@@ -170,6 +170,23 @@ DVLM_API dvlm_status dvlm_lmhead_conf_commit_static(const void* hidden, const vo
                                                    const int32_t* anchor_id, const float* anchor_conf,
                                                    int32_t* cert_len, int* dev_status, dvlm_stream stream);
 
+/* dvlm_block_attn computed by `splits` independent CTAs per (batch entry,
+ * 16-row group, KV head), bf16 only: the keys are dealt to the splits in
+ * 128-key chunks (chunk j to split j % splits, by absolute slot, so a causal
+ * row's result does not depend on n_rows), each split streams its chunks,
+ * and the last split to finish merges all partials in split order.  The
+ * bandwidth-bound form, for long caches and batches of caches.  workspace
+ * (device, 16-byte aligned, zero-filled before the first call; it is zero
+ * again after each call) of dvlm_block_attn_split_workspace_size bytes;
+ * calls sharing a workspace must not overlap.  Arguments and errors
+ * otherwise as dvlm_block_attn (DVLM_ERR_WORKSPACE for a small workspace;
+ * splits 1..64). */
+DVLM_API size_t dvlm_block_attn_split_workspace_size(int n_batch, int n_rows, int Hkv, int splits);
+DVLM_API dvlm_status dvlm_block_attn_split(const void* q, void* out, const void* k_cache, const void* v_cache,
+                                          int n_batch, int n_rows, int n_clean, int L, int Lmax, int Hq, int Hkv,
+                                          int D, float scale, int splits, void* workspace, size_t ws_bytes,
+                                          int* dev_status, dvlm_stream stream);
+
 /* Block-masked attention over PAGED KV caches [Fast-dVLM technical overview
  * (ocdem.com), section 2.3.2: paged KV cache management], bf16: the rules of
  * dvlm_block_attn for each of n_batch sequences, whose caches live in 64-slot
@@ -431,7 +448,10 @@ DVLM_API dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int
  *   "down_stages", "gateup_stages": TMA pipeline depth, 5 or 10;
  *   "gateup_ctas_per_sm": 1, or 2 with 5 gate/up stages;
  *   "attn_cluster": CTAs per attention cluster, 8 or 16;
- *   "pdl": 1/0, programmatic dependent launch between kernels.
+ *   "pdl": 1/0, programmatic dependent launch between kernels;
+ *   "attn_split": 0 = cluster attention, 1..32 = split attention with that
+ *       many CTAs per KV head (dvlm_block_attn_split);
+ *   "prefill_gemm": 1/0, the compute-bound prefill (where supported).
  * Results do not depend on the knobs except through fp32 summation order
  * (cluster sizes).  Changing a knob drops the captured CUDA graphs.
  * Errors: INVALID_ARG (unknown name), SHAPE (bad value), UNSUPPORTED (the

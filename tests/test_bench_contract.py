@@ -150,6 +150,8 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     monkeypatch.setattr(_Stream, "wait_stream", lambda self, other: None, raising=False)
     calls = {"attn": [], "lm": []}
     monkeypatch.setattr(dv, "block_attn", lambda q, out, k, v, **kw: calls["attn"].append(kw))
+    monkeypatch.setattr(dv, "block_attn_split", lambda q, out, k, v, **kw: calls["attn"].append(kw))
+    monkeypatch.setattr(dv, "block_attn_split_workspace_size", lambda *a: 64)
     monkeypatch.setattr(dv, "lmhead_conf_commit", lambda h, w, **kw: calls["lm"].append(kw["R"]))
     monkeypatch.setattr(dv, "lmhead_workspace_size", lambda *a: 64)
     monkeypatch.setattr(dv, "topk_commit", lambda *a, **kw: calls["lm"].append(("topk", kw["R"], kw["k"])))
@@ -161,9 +163,10 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     bench.run_sweep(args, 0)
     lines = [json.loads(ln) for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
     attn = [d for d in lines if d["sweep"] == "attention"]
-    assert len(attn) == 4 * 3 * 2
-    assert {(d["B"], d["L"], d["caches_per_launch"]) for d in attn} == \
-        {(B, L, nb) for B in (4, 8, 16, 32) for L in (256, 1024, 4096) for nb in (1, 36)}
+    assert len(attn) == 4 * 3 * 2 * 2
+    for kern in ("cluster", "split"):
+        assert {(d["B"], d["L"], d["caches_per_launch"]) for d in attn if d["kernel"] == kern} == \
+            {(B, L, nb) for B in (4, 8, 16, 32) for L in (256, 1024, 4096) for nb in (1, 36)}
     for d in attn:
         assert d["bytes_per_launch"] == d["caches_per_launch"] * bench.algorithmic_bytes("attention", gen.QWEN3B,
                                                                                          d["L"], rows=d["B"])

@@ -125,3 +125,60 @@ def test_fp32_path(cuda):
     assert err < 1e-4, err
     out = run_attn(q, k, v, 4, 4, 60, cuda, dtype=dv.DVLM_FP32, Hq=2, Hkv=1, D=16)
     assert max_abs(f64(out), oracle_attn(q, k, v, 4, 60)) < 1e-4
+
+
+# ---------------------------------------------------------------- split form
+def run_attn_split(q, k, v, n_rows, n_clean, L, dev, splits, Hq=16, Hkv=2, D=128):
+    nb, Lmax = k.shape[0], k.shape[2]
+    qd = q.to(dev).contiguous()
+    kd = k.to(dev).contiguous()
+    vt = v.transpose(-1, -2).contiguous().to(dev)
+    out = torch.full_like(qd, float("nan"))
+    ws = torch.zeros((dv.block_attn_split_workspace_size(nb, n_rows, Hkv, splits) + 3) // 4, dtype=torch.int32,
+                     device=dev)
+    st = status(dev)
+    dv.block_attn_split(qd, out, kd, vt, n_batch=nb, n_rows=n_rows, n_clean=n_clean, L=L, Lmax=Lmax, Hq=Hq, Hkv=Hkv,
+                        D=D, scale=1.0 / math.sqrt(D), splits=splits, workspace=ws, status=st)
+    assert_ok(st)
+    return out
+
+
+@pytest.mark.parametrize("B,L,splits", [(16, 1344, 8), (16, 4096, 2), (4, 256, 3), (32, 1024, 5), (8, 4096, 16),
+                                        (16, 0, 4)])
+def test_split_attention_matches_oracle(cuda, B, L, splits):
+    q, k, v = (t for t, _ in gen.attn_case(7, B, L, Lmax=_pad8(L + B)))
+    out = run_attn_split(q, k, v, B, 0, L, cuda, splits)
+    err = max_abs(f64(out), oracle_attn(q, k, v, 0, L))
+    assert err < TOL_BF16, err
+
+
+@pytest.mark.parametrize("n_rows,n_clean,L", [(16, 16, 1280), (12, 5, 1000), (3, 3, 37), (20, 20, 100)])
+def test_split_attention_clean_and_mixed_rows_with_poisoned_stale_slots(cuda, n_rows, n_clean, L):
+    Lmax = _pad8(L + n_rows) + 136
+    q, k, v = (t for t, _ in gen.attn_case(8, n_rows, L, Lmax=Lmax))
+    k[:, :, L + n_rows:] = float("nan")
+    v[:, :, L + n_rows:] = float("nan")
+    out = run_attn_split(q, k, v, n_rows, n_clean, L, cuda, 6)
+    err = max_abs(f64(out), oracle_attn(q, k, v, n_clean, L))
+    assert err < TOL_BF16, err
+
+
+def test_split_attention_causal_row_independent_of_rows_in_step(cuda):
+    """A causal row gives bitwise the same output in a 16-row pass (verify)
+    as in a 1-row pass at its own slot (AR): chunks go to splits by absolute
+    key position, so the split sums do not depend on the step's rows."""
+    L, n = 1300, 16
+    q, k, v = (t for t, _ in gen.attn_case(9, n, L, Lmax=_pad8(L + n)))
+    full = run_attn_split(q, k, v, n, n, L, cuda, 8)
+    for t in (0, 5, 15):
+        one = run_attn_split(q[:, t:t + 1].contiguous(), k, v, 1, 1, L + t, cuda, 8)
+        assert torch.equal(one[0, 0], full[0, t]), t
+
+
+def test_split_attention_batch_of_caches(cuda):
+    """36 distinct caches in one launch (one per decoder layer)."""
+    B, L, nb = 16, 1024, 36
+    q, k, v = (t for t, _ in gen.attn_case(10, B, L, Lmax=_pad8(L + B), n_batch=nb))
+    out = run_attn_split(q, k, v, B, 0, L, cuda, 2)
+    err = max_abs(f64(out), oracle_attn(q, k, v, 0, L))
+    assert err < TOL_BF16, err
