@@ -331,6 +331,9 @@ def run_ours(args, rank, world, local, pg):
                      device=dev)
     stream = torch.cuda.Stream(device=dev)
     eng = dv.Engine(cm, kc, vc, Lmax, BLOCK, N_VIS + N_PROMPT, ws, stream=stream)
+    for opt in args.option or []:
+        name, val = opt.split("=")
+        eng.set_option(name, int(val))
     vis_t, vis, ids = gen.decode_context(dims, SEED, N_VIS, N_PROMPT)
     vis_d, ids_d = vis_t.to(dev), torch.from_numpy(ids).to(dev)
     eng.prefill(vis_d, N_VIS, ids_d, N_PROMPT, stream=stream)
@@ -421,7 +424,7 @@ def run_ours(args, rank, world, local, pg):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3+bf16" if fp8 else "bf16", "data": "synthetic",
-            "config": workload_config(args, world),
+            "config": dict(workload_config(args, world), **({"options": args.option} if args.option else {})),
             "roofline": roof(dom), "lmhead": roof("lm_head") if "lm_head" in per else None,
             "gpu_launches": launches, "clocks": clk, "e2e": e2e,
             "decode": {"nfe_per_step": nfe, "tokens_per_nfe": N_NEW / nfe, "commit_hist": hist,
@@ -620,6 +623,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--mode", choices=["threshold", "spec", "ar", "quad"], default="threshold")
+    ap.add_argument("--option", action="append", default=None, metavar="NAME=VALUE",
+                    help="engine launch knob (dvlm_engine_set_option), e.g. attn_split=8; repeatable")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: the W8A8 decoder (E4M3 projections quantised from the same bf16 weights)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -105,6 +105,9 @@ DVLM_API int dvlm_device_sm_count(void);
  * bf16 path: D == 128, Hq == 8*Hkv, Lmax % 8 == 0.  fp32 path: D <= 128.
  * Errors: INVALID_ARG (null/misaligned), SHAPE (L+n_rows > Lmax, n_clean >
  * n_rows, Hq % Hkv), UNSUPPORTED (bf16 head shapes other than the above).
+ * Defined by: Fast-dVLM technical overview (ocdem.com), section 2.2.1 (the
+ * N2N / N2C / C2C attention rules of block diffusion over an exact KV
+ * cache); Fast-dVLM walkthrough (itsolotime.com), section 4.1.
  */
 DVLM_API dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const void* v_cache,
                             int n_batch, int n_rows, int n_clean, int L, int Lmax, int Hq, int Hkv,
@@ -133,6 +136,10 @@ DVLM_API dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cac
  * row whose top1_id differs from anchor_id.
  * hidden [R, H], w [V, H] (same dtype).  1 <= R <= 128.
  * bf16 path: H % 64 == 0.  Workspace: dvlm_lmhead_workspace_size().
+ * Defined by: Look Only When Needed, method step (1) (top-1 confidence = the
+ * largest softmax probability) and step (2) (the certificate scan);
+ * Fast-dVLM technical overview (ocdem.com), section 4.1 (threshold 0.9,
+ * at least one position committed per step).
  */
 DVLM_API size_t dvlm_lmhead_workspace_size(int R, int V, int H, dvlm_dtype dt);
 DVLM_API dvlm_status dvlm_lmhead_conf_commit(const void* hidden, const void* w, int R, int H, int V,
@@ -251,6 +258,9 @@ DVLM_API dvlm_status dvlm_divergence_first_commit(const float* full_prob, const 
  * overwritten with bf16 NaN in k_cache [n_layers, b, Hkv, Lmax, D] and
  * v_cache [n_layers, b, Hkv, D, Lmax] (a debugging aid: attention never reads
  * them).  Workspace: dvlm_spec_workspace_size().
+ * Defined by: Fast-dVLM technical overview (ocdem.com), section 2.3.1
+ * (linear self-speculative decoding: a causal verify pass, the longest
+ * agreeing prefix kept, the KV cache truncated to it).
  */
 DVLM_API size_t dvlm_spec_workspace_size(int b, int B, int V);
 DVLM_API dvlm_status dvlm_spec_verify_accept(const void* verify_logits, const int32_t* verify_ids,
@@ -382,7 +392,11 @@ DVLM_API dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_visi
  * once per noisy iteration (threshold mode) or round.  stats accumulate.
  * Returns DVLM_ERR_TIMEOUT when a block needs more than B - 1 noisy
  * iterations or a speculative round keeps no token: both mean a device-side
- * wait gave up (the status word, dvlm_engine_check, says where). */
+ * wait gave up (the status word, dvlm_engine_check, says where).
+ * Defined by: Fast-dVLM technical overview (ocdem.com), sections 2.2.1-2.2.2
+ * (block-wise decoding over the KV cache, the block's first token the AR
+ * prediction), 2.3.1 (self-speculative variants) and 4.1 (block 16,
+ * threshold 0.9); Look Only When Needed, method steps (1)-(3) (routing). */
 DVLM_API dvlm_status dvlm_decode_block(dvlm_engine* e, const dvlm_decode_cfg* cfg, int32_t* out_tokens,
                               int32_t* n_out, dvlm_stats* stats, dvlm_stream stream);
 /* Decodes exactly cfg->max_new_tokens tokens into out_tokens (device).

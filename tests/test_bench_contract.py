@@ -91,7 +91,7 @@ def test_default_arm_line_has_the_contract_keys(monkeypatch, capsys):
     monkeypatch.setattr(gdev, "kv_buffers", lambda *a, **k: (None, None))
     monkeypatch.setattr(bench, "gpu_uuid", lambda: None)
     args = bench.argparse.Namespace(steps=5, warmup=3, mode="threshold", quick=True, no_cpu_baseline=True,
-                                    layers=36, profile_forwards=0, impl="ours", gpus=1, sweep=None, weights="bf16")
+                                    layers=36, profile_forwards=0, impl="ours", gpus=1, sweep=None, weights="bf16", option=None)
     bench.run_ours(args, 0, 1, 0, None)
     lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
