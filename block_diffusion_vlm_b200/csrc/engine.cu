@@ -630,6 +630,7 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
   ta.quad_B = B;
   ta.kside = static_cast<bf16*>(e->kside);
   ta.vside = static_cast<bf16*>(e->vside);
+  ta.side_n = kQuadSideKeys;
   AttnArgs aa{};
   aa.n_rows = B;
   aa.n_clean = B;

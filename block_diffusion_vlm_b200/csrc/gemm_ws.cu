@@ -40,6 +40,180 @@ __device__ __forceinline__ float fp8_row_scale(const GemmEpi& ea, bool split, in
   return ea.wscale[a_row_base + T * 128 + row];
 }
 
+// The epilogue warps' work for the stream-K units [u0, u1) of one GEMM:
+// partial tiles stored for the CTAs that finish them, split tiles finished
+// (partials added in CTA order), the fused epilogue on every tile this CTA
+// owns.  gseg counts the CTA's segments across consecutive GEMMs (it selects
+// the accumulator buffer and its phase); L0 is the QKV rows' first slot.
+// Returns false when a wait gave up.
+template <int NT, int EPI, bool FP8>
+__device__ __forceinline__ bool ws_epilogue_units(const SkSched& sc, long long u0, long long u1, int a_row_base,
+                                                  const GemmEpi& ea, uint32_t tmem, uint64_t* accf,
+                                                  uint64_t* acce, float* sE, const float* sR, const float* sAt,
+                                                  unsigned* sAmax, int* sflag, volatile int* sabort, int& gseg,
+                                                  int L0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;  // accumulator row = output feature within the tile
+  const int et = threadIdx.x - 64;      // 0..127
+  // A tile split over CTAs pf < ... < pl is finished by pf, which streams
+  // the tile's first k blocks as its last segment; the others stream their
+  // parts first and leave fp32 partials in global scratch, counted on
+  // cnt[T].  pf fetches those partials while its own last segment is still
+  // in the mainloop and adds them in CTA order.
+  for (long long u = u0; u < u1; ++gseg) {
+    const int T = static_cast<int>(u / sc.kb);
+    const long long t_begin = static_cast<long long>(T) * sc.kb, t_end = t_begin + sc.kb;
+    const long long seg_end = t_end < u1 ? t_end : u1;
+    const int b = gseg & 1;
+    const bool whole = (u == t_begin) && (seg_end == t_end);
+    const bool finisher = !whole && (u == t_begin);
+    float o[NT];
+    if (finisher) {
+      const int pl = sc.cta_of(t_end - 1);
+      if (et == 0) {
+        const bool ok = wait_counter(&ea.cnt[T], pl - static_cast<int>(blockIdx.x), ea.status, sabort);
+        if (ok) ea.cnt[T] = 0;  // every part is counted: zero again for the next launch
+        *sflag = ok ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (!*sflag) return false;
+      __threadfence();
+#pragma unroll
+      for (int t = 0; t < NT; ++t) o[t] = 0.f;
+      // the other CTAs' partials in CTA order, four sources' loads in flight
+      for (int p0 = static_cast<int>(blockIdx.x) + 1; p0 <= pl; p0 += 4) {
+        float q4[4][NT];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float* src = ea.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * NT * 128;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) q4[q][t] = __ldcg(&src[t * 128 + row]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (p0 + q <= pl) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) o[t] += q4[q][t];
+          }
+      }
+    }
+    mbar_wait(&accf[b], (gseg >> 1) & 1, ea.status, sabort);
+    named_bar_sync(1, 128);  // leave together if any wait gave up
+    if (*sabort) return false;
+    tc_fence_after();
+    float v[NT];
+    ws_load_acc<NT>(tmem, b, quarter, v, seg_end - u >= 2);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&acce[b]);
+    if (!whole && !finisher) {
+      // tail or middle part of a tile finished by another CTA
+      float* mine = ea.part + static_cast<size_t>(blockIdx.x) * NT * 128;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + row], v[t]);
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (et == 0) red_release_gpu_add(&ea.cnt[T], 1);
+      u = seg_end;
+      continue;
+    }
+    if (finisher) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) v[t] += o[t];
+    }
+    if (FP8) {  // W8A8 dequantisation: weight row scale x token scale
+      const float sr = fp8_row_scale(ea, EPI == EPI_SWIGLU, a_row_base, T, row);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) v[t] *= sr * sAt[t];
+    }
+
+    if (EPI == EPI_RESID) {
+      const int col = T * 128 + row;
+      float sq[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        sq[t] = 0.f;
+        if (t < ea.n_rows) {
+          bf16* px = ea.resid + static_cast<size_t>(t) * ea.resid_ld + col;
+          const float xn = bf16_round_f(__bfloat162float(*px) + v[t]);
+          *px = __float2bfloat16_rn(xn);
+          sq[t] = xn * xn;
+        }
+        sE[row * (NT + 1) + t] = sq[t];
+      }
+      named_bar_sync(1, 128);
+      if (et < NT) {
+        float s = 0.f;
+        for (int r = 0; r < 128; ++r) s += sE[r * (NT + 1) + et];
+        ea.ssq_out[T * NT + et] = s;
+      }
+      named_bar_sync(1, 128);
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) sE[row * (NT + 1) + t] = FP8 ? v[t] : v[t] * sR[t];
+      if (FP8 && EPI == EPI_SWIGLU && et < NT) sAmax[et] = 0u;
+      named_bar_sync(1, 128);
+      const int j = et & 63;
+      const int half = et >> 6;
+      const int t0 = half * (NT / 2), t1 = t0 + NT / 2;
+      if (EPI == EPI_SWIGLU) {
+        for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
+          const float g = sE[j * (NT + 1) + t];
+          const float up = sE[(j + 64) * (NT + 1) + t];
+          const float a = g / (1.0f + expf(-g)) * up;
+          const bf16 ab = __float2bfloat16_rn(a);
+          ea.out[static_cast<size_t>(t) * ea.out_ld + T * 64 + j] = ab;
+          if (FP8) atomicMax(&sAmax[t], __float_as_uint(fabsf(__bfloat162float(ab))));
+        }
+        if (FP8) {
+          named_bar_sync(1, 128);
+          if (et < NT) ea.amax_out[T * NT + et] = __uint_as_float(sAmax[et]);
+        }
+      } else {  // EPI_QKV, one head (128 rows) per tile
+        const int nq = ea.n_q_heads, nkv = ea.n_kv_heads;
+        if (T < nq + nkv) {
+          const double inv_freq = exp2(-(2.0 * j / 128.0) * ea.log2_rope_base);
+          for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
+            const float x1 = sE[j * (NT + 1) + t];
+            const float x2 = sE[(j + 64) * (NT + 1) + t];
+            double sn, cs;
+            sincos(static_cast<double>(L0 + t) * inv_freq, &sn, &cs);
+            const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+            const bf16 y1 = __float2bfloat16_rn(x1 * c - x2 * s);
+            const bf16 y2 = __float2bfloat16_rn(x2 * c + x1 * s);
+            if (T < nq) {
+              bf16* q = ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128;
+              q[j] = y1;
+              q[j + 64] = y2;
+            } else if (bf16* k = kv_k_ptr(ea, T - nq, L0 + t)) {
+              k[j] = y1;
+              k[j + 64] = y2;
+            } else {
+              record_error(ea.status, DVLM_ERR_BOUNDS);
+            }
+          }
+        } else {
+          const int h = T - nq - nkv;
+          for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
+            bf16* v1 = kv_v_ptr(ea, h, j, L0 + t);
+            bf16* v2 = kv_v_ptr(ea, h, j + 64, L0 + t);
+            if (!v1 || !v2) {
+              record_error(ea.status, DVLM_ERR_BOUNDS);
+              continue;
+            }
+            *v1 = __float2bfloat16_rn(sE[j * (NT + 1) + t]);
+            *v2 = __float2bfloat16_rn(sE[(j + 64) * (NT + 1) + t]);
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+    u = seg_end;
+  }
+  return true;
+}
+
 template <int NT, int STAGES, int EPI, bool FP8 = false>
 __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     gemm_ws_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
@@ -129,162 +303,9 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
                                    ea.amax_in, ea.n_amax, kb_lo, kb_hi, sB, sAt, sQm, b_ready);
     int L0 = 0;
     if (EPI == EPI_QKV) L0 = ea.d_len ? *ea.d_len : ea.L_static;
-    // A tile split over CTAs pf < ... < pl is finished by pf, which streams
-    // the tile's first k blocks as its last segment; the others stream their
-    // parts first and leave fp32 partials in global scratch, counted on
-    // cnt[T].  pf fetches those partials while its own last segment is still
-    // in the mainloop and adds them in CTA order.
-    int seg = 0;
-    for (long long u = u0; u < u1; ++seg) {
-      const int T = static_cast<int>(u / sc.kb);
-      const long long t_begin = static_cast<long long>(T) * sc.kb, t_end = t_begin + sc.kb;
-      const long long seg_end = t_end < u1 ? t_end : u1;
-      const int b = seg & 1;
-      const bool whole = (u == t_begin) && (seg_end == t_end);
-      const bool finisher = !whole && (u == t_begin);
-      float o[NT];
-      if (finisher) {
-        const int pl = sc.cta_of(t_end - 1);
-        if (et == 0) {
-          const bool ok = wait_counter(&ea.cnt[T], pl - static_cast<int>(blockIdx.x), ea.status, sabort);
-          if (ok) ea.cnt[T] = 0;  // every part is counted: zero again for the next launch
-          *sflag = ok ? 1 : 0;
-        }
-        named_bar_sync(1, 128);
-        if (!*sflag) break;
-        __threadfence();
-#pragma unroll
-        for (int t = 0; t < NT; ++t) o[t] = 0.f;
-        // the other CTAs' partials in CTA order, four sources' loads in flight
-        for (int p0 = static_cast<int>(blockIdx.x) + 1; p0 <= pl; p0 += 4) {
-          float q4[4][NT];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float* src = ea.part + static_cast<size_t>(p0 + q <= pl ? p0 + q : p0) * NT * 128;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) q4[q][t] = __ldcg(&src[t * 128 + row]);
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (p0 + q <= pl) {
-#pragma unroll
-              for (int t = 0; t < NT; ++t) o[t] += q4[q][t];
-            }
-        }
-      }
-      mbar_wait(&accf[b], (seg >> 1) & 1, ea.status, sabort);
-      named_bar_sync(1, 128);  // leave together if any wait gave up
-      if (*sabort) break;
-      tc_fence_after();
-      float v[NT];
-      ws_load_acc<NT>(tmem, b, quarter, v, seg_end - u >= 2);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[b]);
-      if (!whole && !finisher) {
-        // tail or middle part of a tile finished by another CTA
-        float* mine = ea.part + static_cast<size_t>(blockIdx.x) * NT * 128;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) __stcg(&mine[t * 128 + row], v[t]);
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (et == 0) red_release_gpu_add(&ea.cnt[T], 1);
-        u = seg_end;
-        continue;
-      }
-      if (finisher) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) v[t] += o[t];
-      }
-      if (FP8) {  // W8A8 dequantisation: weight row scale x token scale
-        const float sr = fp8_row_scale(ea, EPI == EPI_SWIGLU, a_row_base, T, row);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) v[t] *= sr * sAt[t];
-      }
-
-      if (EPI == EPI_RESID) {
-        const int col = T * 128 + row;
-        float sq[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          sq[t] = 0.f;
-          if (t < ea.n_rows) {
-            bf16* px = ea.resid + static_cast<size_t>(t) * ea.resid_ld + col;
-            const float xn = bf16_round_f(__bfloat162float(*px) + v[t]);
-            *px = __float2bfloat16_rn(xn);
-            sq[t] = xn * xn;
-          }
-          sE[row * (NT + 1) + t] = sq[t];
-        }
-        named_bar_sync(1, 128);
-        if (et < NT) {
-          float s = 0.f;
-          for (int r = 0; r < 128; ++r) s += sE[r * (NT + 1) + et];
-          ea.ssq_out[T * NT + et] = s;
-        }
-        named_bar_sync(1, 128);
-      } else {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) sE[row * (NT + 1) + t] = FP8 ? v[t] : v[t] * sR[t];
-        if (FP8 && EPI == EPI_SWIGLU && et < NT) sAmax[et] = 0u;
-        named_bar_sync(1, 128);
-        const int j = et & 63;
-        const int half = et >> 6;
-        const int t0 = half * (NT / 2), t1 = t0 + NT / 2;
-        if (EPI == EPI_SWIGLU) {
-          for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
-            const float g = sE[j * (NT + 1) + t];
-            const float up = sE[(j + 64) * (NT + 1) + t];
-            const float a = g / (1.0f + expf(-g)) * up;
-            const bf16 ab = __float2bfloat16_rn(a);
-            ea.out[static_cast<size_t>(t) * ea.out_ld + T * 64 + j] = ab;
-            if (FP8) atomicMax(&sAmax[t], __float_as_uint(fabsf(__bfloat162float(ab))));
-          }
-          if (FP8) {
-            named_bar_sync(1, 128);
-            if (et < NT) ea.amax_out[T * NT + et] = __uint_as_float(sAmax[et]);
-          }
-        } else {  // EPI_QKV, one head (128 rows) per tile
-          const int nq = ea.n_q_heads, nkv = ea.n_kv_heads;
-          if (T < nq + nkv) {
-            const double inv_freq = exp2(-(2.0 * j / 128.0) * ea.log2_rope_base);
-            for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
-              const float x1 = sE[j * (NT + 1) + t];
-              const float x2 = sE[(j + 64) * (NT + 1) + t];
-              double sn, cs;
-              sincos(static_cast<double>(L0 + t) * inv_freq, &sn, &cs);
-              const float c = static_cast<float>(cs), s = static_cast<float>(sn);
-              const bf16 y1 = __float2bfloat16_rn(x1 * c - x2 * s);
-              const bf16 y2 = __float2bfloat16_rn(x2 * c + x1 * s);
-              if (T < nq) {
-                bf16* q = ea.out + static_cast<size_t>(t) * ea.out_ld + T * 128;
-                q[j] = y1;
-                q[j + 64] = y2;
-              } else if (bf16* k = kv_k_ptr(ea, T - nq, L0 + t)) {
-                k[j] = y1;
-                k[j + 64] = y2;
-              } else {
-                record_error(ea.status, DVLM_ERR_BOUNDS);
-              }
-            }
-          } else {
-            const int h = T - nq - nkv;
-            for (int t = t0; t < t1 && t < ea.n_rows; ++t) {
-              bf16* v1 = kv_v_ptr(ea, h, j, L0 + t);
-              bf16* v2 = kv_v_ptr(ea, h, j + 64, L0 + t);
-              if (!v1 || !v2) {
-                record_error(ea.status, DVLM_ERR_BOUNDS);
-                continue;
-              }
-              *v1 = __float2bfloat16_rn(sE[j * (NT + 1) + t]);
-              *v2 = __float2bfloat16_rn(sE[(j + 64) * (NT + 1) + t]);
-            }
-          }
-        }
-        named_bar_sync(1, 128);
-      }
-      u = seg_end;
-    }
+    int gseg = 0;
+    ws_epilogue_units<NT, EPI, FP8>(sc, u0, u1, a_row_base, ea, tmem, accf, acce, sE, sR, sAt, sAmax, sflag,
+                                    sabort, gseg, L0);
   }
   tc_fence_before();
   __syncthreads();

@@ -199,10 +199,12 @@ struct TmArgs {
   // QKV of the fused draft+verify forward (quad_B = B > 0): rows 0..B-1 are
   // the verify rows (slots L..L+B-1, K/V to the cache); row B + i*B + r is row
   // r of candidate block i at position L+i+1+r, its K/V to kside
-  // [Hkv][B*64][128] / vside [Hkv][128][B*64] at key i*64 + r.
+  // [Hkv][side_n][128] / vside [Hkv][128][side_n] at key i*64 + r
+  // (side_n >= 64 * B keys per KV head).
   int quad_B;
   bf16* kside;
   bf16* vside;
+  int side_n;
 };
 // y = x W^T over n_wtiles tiles of 256 weight rows (SWIGLU: 128 rows of W and
 // the same 128 rows of W2) starting at weight row w_row_base; kb = K / 64.

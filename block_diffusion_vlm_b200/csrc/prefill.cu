@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         const bool cand = Bq > 0 && tok >= Bq;
         const int ci = cand ? (tok - Bq) / Bq : 0, cr = cand ? (tok - Bq) % Bq : 0;
         const int pos = cand ? L0 + ci + 1 + cr : L0 + tok;
-        const int side_n = Bq * 64;  // keys per head in the side buffers
+        const int side_n = a.side_n;  // keys per KV head in the side buffers
 #pragma unroll 1
         for (int i = 0; i < 2; ++i) {
           const int hh = 2 * T + i;
@@ -625,6 +625,7 @@ static cudaError_t tm_launch(const CUtensorMap& mapX, const CUtensorMap& mapW, c
 cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, const CUtensorMap& mapW2, int kb,
                            int w_row_base, int n_wtiles, const TmArgs& a, cudaStream_t s) {
   if (a.n_tok < 1 || kb < 1 || n_wtiles < 1) return cudaErrorInvalidValue;
+  if (a.quad_B > 0 && (a.side_n < 64 * a.quad_B || !a.kside || !a.vside)) return cudaErrorInvalidValue;
   switch (a.epi) {
     case EPI_QKV: return tm_launch<EPI_QKV>(mapX, mapW, mapW2, kb, w_row_base, n_wtiles, a, s);
     case EPI_RESID: return tm_launch<EPI_RESID>(mapX, mapW, mapW2, kb, w_row_base, n_wtiles, a, s);
@@ -646,7 +647,8 @@ cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK
 cudaError_t launch_attn_cand(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                              const CUtensorMap& mapKs, const CUtensorMap& mapVs, const PrefillAttnArgs& a,
                              cudaStream_t s) {
-  if (a.quad_B < 1 || a.quad_B > 16 || !a.d_len || a.Hq != 8 * a.Hkv) return cudaErrorInvalidValue;
+  if (a.quad_B < 1 || a.quad_B > 16 || !a.d_len || a.Hq != 8 * a.Hkv || a.side_n < 64 * a.quad_B)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
   if (e != cudaSuccess) return e;
   attn_tile_kernel<true><<<dim3(a.quad_B, a.Hkv), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, mapKs, mapVs, a);
