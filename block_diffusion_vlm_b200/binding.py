@@ -364,13 +364,14 @@ class Engine:
         _check(lib().dvlm_engine_set_trace(self.h, ptr(buf), nbytes, ptr(count) if buf is not None else None),
                "dvlm_engine_set_trace")
 
-    KERNEL_KINDS = ("embed", "qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head")
+    KERNEL_KINDS = ("embed", "qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head",
+                    "gemm_chain")
 
     def profile_forward(self, tokens, n_rows: int, n_clean: int, *, masked=None, with_lm_head=True,
                         stream=None) -> dict:
         """Per-kernel-class device time (ms, summed over layers) and launch count of one eager forward."""
-        ms = (ctypes.c_float * 7)()
-        cnt = (ctypes.c_int * 7)()
+        ms = (ctypes.c_float * len(self.KERNEL_KINDS))()
+        cnt = (ctypes.c_int * len(self.KERNEL_KINDS))()
         _check(lib().dvlm_profile_forward(self.h, ptr(tokens), ptr(masked), n_rows, n_clean, int(with_lm_head), ms,
                                           cnt, stream_handle(stream)),
                "dvlm_profile_forward")

@@ -108,7 +108,9 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   // sums of squares per (128-feature tile, cluster CTA): up to 16 CTAs per tile
   e->ssq = c.take<float>(((H / 128) * 16 + 1) * kNT * 4);
   e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, 2 * P));  // up to two CTAs per SM
-  e->gcnt = c.take<int>(num_tiles_max(m) * 4);
+  e->gcnt_stride = num_tiles_max(m);
+  e->gcnt = c.take<int>(static_cast<size_t>(e->gcnt_stride) * kMaxChainPhases * 4);
+  e->chain_bar = c.take<int>(2 * 4);
   e->lpart = c.take<float>(static_cast<size_t>(P) * kNT * 128 * 4);
   e->lcnt = c.take<int>(((m.vocab + 127) / 128) * 4);
   e->lrec = c.take<float>(static_cast<size_t>(P) * kNT * 16);
@@ -227,6 +229,37 @@ static void fill_lm_scratch(dvlm_engine* e, LmArgs& a) {
     if (err__ != cudaSuccess) return err__;   \
   } while (0)
 
+// Persistent GEMM chain (gemm_chain): bf16 weights, 128-wide heads, feature
+// counts in whole tiles, and one resident CTA on every SM.
+static bool chain_supported(dvlm_engine* e) {
+  const dvlm_model& m = e->m;
+  return e->bf16 && !e->fp8 && m.head_dim == 128 && m.hidden % 128 == 0 && m.inter % 64 == 0 &&
+         (m.n_q_heads * m.head_dim) % 64 == 0 && e->sm >= 1 && e->sm <= gemm_chain_max_ctas();
+}
+
+static ChainArgs chain_args(dvlm_engine* e) {
+  ChainArgs ca{};
+  ca.P = e->sm;
+  ca.bar = e->chain_bar;
+  ca.status = e->d_status;
+  return ca;
+}
+
+// Appends a phase; each phase counts its split tiles in its own block of gcnt.
+static void chain_push(dvlm_engine* e, ChainArgs& ca, const CUtensorMap& a, const CUtensorMap& a2,
+                       const CUtensorMap& b, int n_tiles, int kb, int a_row_base, const GemmEpi& ea) {
+  ChainPhase& ph = ca.ph[ca.n_phases];
+  ph.mapA = a;
+  ph.mapA2 = a2;
+  ph.mapB = b;
+  ph.ea = ea;
+  ph.ea.cnt = e->gcnt + static_cast<size_t>(ca.n_phases) * e->gcnt_stride;
+  ph.n_tiles = n_tiles;
+  ph.kb = kb;
+  ph.a_row_base = a_row_base;
+  ++ca.n_phases;
+}
+
 static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
   const dvlm_model& m = e->m;
   const int H = m.hidden, I = m.inter, D = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
@@ -282,15 +315,38 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.block_table = e->block_table;
     ea.n_pages = e->n_pages;
   }
+  // persistent chain: [QKV(first layer)], then per layer attention followed
+  // by one launch of [O, gate/up, down, QKV(next layer)]
+  const bool chain = e->chain && !e->fp8;
+  const GemmEpi base = ea;
+  auto qkv_epi = [&](int layer) {
+    GemmEpi q = base;
+    q.epi = EPI_QKV;
+    q.n_ssq = H / 128;
+    q.out = static_cast<bf16*>(e->q);
+    q.out_ld = Hq * D;
+    q.kcache = static_cast<bf16*>(e->kc) + layer * kv_layer;
+    q.vcache = static_cast<bf16*>(e->vc) + layer * kv_layer;
+    return q;
+  };
   for (int l = f.layer0; l < l1; ++l) {
+    if (chain && l == f.layer0) {
+      ChainArgs ca = chain_args(e);
+      chain_push(e, ca, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, l * qkv_rows, qkv_epi(l));
+      T0(K_CHAIN);
+      DVLM_CK(launch_gemm_chain(ca, pdl, s));
+      T1(K_CHAIN);
+    }
     ea.epi = EPI_QKV;
     ea.n_ssq = n_ssq;
     ea.out = static_cast<bf16*>(e->q);
     ea.out_ld = Hq * D;
     ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
     ea.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
-    T0(K_QKV);
-    if (e->fp8) {  // W8A8 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]
+    if (!chain) T0(K_QKV);
+    if (chain) {
+      // written by the previous chain launch
+    } else if (e->fp8) {  // W8A8 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]
       ea.q_src = x;
       ea.q_ld = H;
       ea.q_K = H;
@@ -309,7 +365,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
                              ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s, 5));
     }
-    T1(K_QKV);
+    if (!chain) T1(K_QKV);
     AttnArgs aa{};
     aa.n_rows = f.n_rows;
     aa.n_clean = f.n_clean;
@@ -336,6 +392,30 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     else
       DVLM_CK(launch_attn_bf16(e->tm_q, mk, mv, aa, pdl, s, e->attn_cs));
     T1(K_ATTN);
+    if (chain) {
+      ChainArgs ca = chain_args(e);
+      GemmEpi o = base;  // O-projection and down: residual add + sums of squares
+      o.epi = EPI_RESID;
+      o.resid = x;
+      o.resid_ld = H;
+      o.ssq_out = e->ssq;
+      GemmEpi g = base;
+      g.epi = EPI_SWIGLU;
+      g.n_ssq = H / 128;
+      g.out = static_cast<bf16*>(e->act);
+      g.out_ld = I;
+      chain_push(e, ca, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, l * H, o);
+      chain_push(e, ca, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, l * I, g);
+      chain_push(e, ca, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, l * H, o);
+      if (l + 1 < l1)
+        chain_push(e, ca, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, (l + 1) * qkv_rows,
+                   qkv_epi(l + 1));
+      T0(K_CHAIN);
+      DVLM_CK(launch_gemm_chain(ca, pdl, s));
+      T1(K_CHAIN);
+      n_ssq = H / 128;
+      continue;
+    }
     ea.epi = EPI_RESID;
     ea.resid = x;
     ea.resid_ld = H;
@@ -1142,6 +1222,10 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
   } else if (n == "attn_split") {
     if (v < 0 || v > kMaxAttnSplit) return DVLM_ERR_SHAPE;
     e->attn_split = v;
+  } else if (n == "persistent") {
+    if (v != 0 && v != 1) return DVLM_ERR_SHAPE;
+    if (v && !chain_supported(e)) return DVLM_ERR_UNSUPPORTED;
+    e->chain = v != 0;
   } else if (n == "prefill_gemm") {
     if (v != 0 && v != 1) return DVLM_ERR_SHAPE;
     if (v && !prefill_gemm_supported(e)) return DVLM_ERR_UNSUPPORTED;
@@ -1166,6 +1250,7 @@ int engine_get_option(dvlm_engine* e, const char* name) {
   if (n == "pdl") return e->pdl ? 1 : 0;
   if (n == "attn_split") return e->attn_split;
   if (n == "prefill_gemm") return e->prefill_gemm ? 1 : 0;
+  if (n == "persistent") return e->chain ? 1 : 0;
   return -1;
 }
 

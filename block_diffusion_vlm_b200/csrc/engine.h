@@ -13,7 +13,7 @@ namespace dvlm {
 constexpr int kNT = 16;  // token rows per forward (block size <= 16)
 
 // Per-kernel-class CUDA-event timing of one eager forward (profiling hook).
-enum KernelKind { K_EMBED = 0, K_QKV, K_ATTN, K_OPROJ, K_GATEUP, K_DOWN, K_LMHEAD, K_KINDS };
+enum KernelKind { K_EMBED = 0, K_QKV, K_ATTN, K_OPROJ, K_GATEUP, K_DOWN, K_LMHEAD, K_CHAIN, K_KINDS };
 struct KernelTimer {
   std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> marks;
   cudaStream_t s = nullptr;
@@ -105,7 +105,10 @@ struct dvlm_engine {
   void* act = nullptr;      // [NT][I]
   float* ssq = nullptr;     // [H/128][NT]
   float* gpart = nullptr;   // GEMM split scratch
-  int* gcnt = nullptr;
+  int* gcnt = nullptr;      // split-tile counters, one block of gcnt_stride per chain phase
+  int gcnt_stride = 0;
+  int* chain_bar = nullptr; // persistent chain: barrier and exit counters
+  bool chain = false;       // post-attention GEMMs + next QKV as one persistent launch
   float* lpart = nullptr;   // LM head scratch
   int* lcnt = nullptr;
   float* lrec = nullptr;

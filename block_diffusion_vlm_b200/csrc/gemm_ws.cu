@@ -579,6 +579,222 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent GEMM chain.  The products that follow a layer's attention --
+// O-projection (+ residual), gate/up (SwiGLU), down (+ residual) -- and the
+// next layer's QKV run as consecutive stream-K phases of one launch on every
+// SM, instead of one kernel each.  A phase reads what the previous phase's
+// epilogues wrote (all CTAs), so a grid barrier separates the phases: every
+// CTA bumps a counter after its phase epilogue, and phase p's inputs are
+// ready once the counter reaches p * P.  The weight stream never waits for
+// it: the A loader runs through the phases back to back, so while the last
+// split tiles of one phase are being reduced and finished, the next phase's
+// weight tiles already fill the pipeline stages.  Only the activation tiles
+// (2 KB a stage, L2-resident) wait for the barrier, issued by a loader warp
+// of their own that polls it.  One A loader arrival per stage arms the
+// stage's full barrier with A + B bytes (a B copy may complete before that
+// arrival; the phase still needs the arrival).
+//
+// Roles (256 threads): warp 0 A loader, warps 1 and 6 MMA issuers, warps
+// 2..5 epilogue, warp 7 B loader.  All P CTAs must be resident together
+// (one per SM; the launcher checks the occupancy), and every wait is
+// bounded: a CTA that gives up records DVLM_ERR_TIMEOUT and still arrives
+// at the remaining barriers, so the others do not wait on it.
+constexpr int kChainThreads = 256;
+constexpr int kChainStages = 12;
+constexpr int kChainNT = 16;
+
+template <int STAGES>
+__device__ __forceinline__ void chain_load_a(const ChainArgs& ca, uint8_t* sA, uint64_t* full, uint64_t* empty,
+                                             volatile int* abort_flag) {
+  constexpr int B_BYTES = kChainNT * 128;
+  const uint64_t pol_w = l2_policy_evict_first();
+  long long i = 0;
+  for (int p = 0; p < ca.n_phases; ++p) {
+    const ChainPhase& ph = ca.ph[p];
+    const SkSched sc{ph.n_tiles, ph.kb, ca.P};
+    const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+    const bool split = ph.ea.epi == EPI_SWIGLU;
+    for (long long u = u0; u < u1; ++u, ++i) {
+      const int s = static_cast<int>(i % STAGES);
+      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, ca.status, abort_flag)) return;
+      mbar_arrive_expect_tx(&full[s], kATileBytes + B_BYTES);
+      const int T = static_cast<int>(u / sc.kb), kk = static_cast<int>(u % sc.kb);
+      if (split) {
+        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, ph.a_row_base + T * 64, pol_w);
+        tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, &ph.mapA2, &full[s], kk * 64, ph.a_row_base + T * 64,
+                    pol_w);
+      } else {
+        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, ph.a_row_base + T * 128, pol_w);
+      }
+    }
+  }
+}
+
+template <int STAGES>
+__device__ __forceinline__ void chain_load_b(const ChainArgs& ca, uint8_t* sB, uint64_t* full, uint64_t* empty,
+                                             volatile int* abort_flag) {
+  constexpr int B_BYTES = kChainNT * 128;
+  const uint64_t pol_x = l2_policy_evict_last();
+  long long i = 0;
+  for (int p = 0; p < ca.n_phases; ++p) {
+    // inputs of phase p: the kernel before this one (p = 0), else every CTA's phase p-1
+    if (p == 0)
+      griddep_wait();
+    else if (!wait_counter(ca.bar, p * ca.P, ca.status, abort_flag))
+      return;
+    fence_proxy_async_global();
+    const ChainPhase& ph = ca.ph[p];
+    const SkSched sc{ph.n_tiles, ph.kb, ca.P};
+    const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+    for (long long u = u0; u < u1; ++u, ++i) {
+      const int s = static_cast<int>(i % STAGES);
+      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, ca.status, abort_flag)) return;
+      tma_load_2d(sB + s * B_BYTES, &ph.mapB, &full[s], static_cast<int>(u % sc.kb) * 64, 0, pol_x);
+    }
+  }
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __grid_constant__ ChainArgs ca) {
+  constexpr int NT = kChainNT;
+  using S = GemmSmem<NT, STAGES, false>;
+  constexpr int TMC = tmem_cols_for<NT>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem + S::kA;
+  uint8_t* sB = smem + S::kB;
+  float* sE = reinterpret_cast<float*>(smem + S::kE);
+  float* sR = reinterpret_cast<float*>(smem + S::kR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMisc);
+  int* sflag = reinterpret_cast<int*>(smem + S::kMisc + 4);
+  volatile int* sabort = reinterpret_cast<volatile int*>(smem + S::kMisc + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 2);
+      mbar_init(&acce[b], 4);
+    }
+    *sabort = 0;
+    fence_mbar_init();
+    for (int p = 0; p < ca.n_phases; ++p) {
+      tma_prefetch_map(&ca.ph[p].mapA);
+      tma_prefetch_map(&ca.ph[p].mapB);
+      if (ca.ph[p].ea.epi == EPI_SWIGLU) tma_prefetch_map(&ca.ph[p].mapA2);
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMC);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) chain_load_a<STAGES>(ca, sA, full, empty, sabort);
+  } else if (warp == 7) {
+    if (lane == 0) chain_load_b<STAGES>(ca, sB, full, empty, sabort);
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    if (lane == 0) {
+      long long i_base = 0;
+      int seg = 0;
+      for (int p = 0; p < ca.n_phases; ++p) {
+        const SkSched sc{ca.ph[p].n_tiles, ca.ph[p].kb, ca.P};
+        if (!ws_mma_units<NT, STAGES, false>(sA, sB, full, empty, accf, acce, tmem, sc, sc.begin(blockIdx.x),
+                                             sc.begin(blockIdx.x + 1), ca.status, sabort, warp == 1 ? 0 : 1, 0,
+                                             i_base, seg))
+          break;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int et = threadIdx.x - 64;  // 0..127
+    griddep_wait();
+    // dependents start only once this kernel's own inputs are complete
+    if (et == 0) griddep_launch_dependents();
+    int gseg = 0;
+    bool ok = true;
+    for (int p = 0; p < ca.n_phases; ++p) {
+      const ChainPhase& ph = ca.ph[p];
+      const GemmEpi& ea = ph.ea;
+      if (p > 0) {
+        if (et == 0) {
+          *sflag = ok && wait_counter(ca.bar, p * ca.P, ca.status, sabort) ? 1 : 0;
+          __threadfence();
+        }
+        named_bar_sync(1, 128);
+        ok = *sflag != 0;
+        named_bar_sync(1, 128);  // sflag is read before the phase may reuse it
+      }
+      if (ok) {
+        if (ea.epi != EPI_RESID) {
+          if (et < NT) {
+            float sq = 0.f;
+            for (int q = 0; q < ea.n_ssq; ++q) sq += __ldcg(&ea.ssq_in[q * NT + et]);
+            sR[et] = 1.0f / sqrtf(sq * ea.inv_h + ea.eps);
+          }
+          named_bar_sync(1, 128);
+        }
+        const SkSched sc{ph.n_tiles, ph.kb, ca.P};
+        const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+        if (ea.epi == EPI_QKV)
+          ok = ws_epilogue_units<NT, EPI_QKV, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
+                                                     nullptr, nullptr, sflag, sabort, gseg,
+                                                     ea.d_len ? *ea.d_len : ea.L_static);
+        else if (ea.epi == EPI_SWIGLU)
+          ok = ws_epilogue_units<NT, EPI_SWIGLU, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
+                                                        nullptr, nullptr, sflag, sabort, gseg, 0);
+        else
+          ok = ws_epilogue_units<NT, EPI_RESID, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
+                                                       nullptr, nullptr, sflag, sabort, gseg, 0);
+      }
+      if (p + 1 < ca.n_phases) {
+        // this CTA's phase outputs, plain stores, are read by TMA in other CTAs
+        fence_proxy_async_global();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          __threadfence();
+          red_release_gpu_add(ca.bar, 1);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*sabort) {
+    // a wait gave up: let copies already issued land before the CTA's shared
+    // memory is released (they complete in microseconds)
+    const long long t0 = clock64();
+    while (clock64() - t0 < 4000000) {
+    }
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMC);
+  }
+  if (threadIdx.x == 0) {
+    // every thread of this CTA is past its last barrier wait; the last CTA
+    // out zeroes both counters for the next launch
+    __threadfence();
+    if (atomicAdd(ca.bar + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      ca.bar[0] = 0;
+      ca.bar[1] = 0;
+      __threadfence();
+    }
+  }
+}
+
 template <int NT, int ST, int EPI, bool FP8 = false>
 static cudaError_t launch_one(const CUtensorMap& mapA, const CUtensorMap& mapA2, const CUtensorMap& mapB,
                               const SkSched& sc, int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s) {
@@ -739,6 +955,52 @@ cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& m
   DVLM_GEMM_CASE(32, 4)
 #undef DVLM_GEMM_CASE
   return cudaErrorInvalidValue;
+}
+
+static int chain_cap[64] = {};  // resident CTAs per device (0: not yet queried)
+
+int gemm_chain_max_ctas() {
+  using S = GemmSmem<kChainNT, kChainStages, false>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (chain_cap[dev] == 0) {
+    auto kern = gemm_chain_kernel<kChainStages>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal) != cudaSuccess) return 0;
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kChainThreads, S::kTotal) != cudaSuccess)
+      return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    chain_cap[dev] = per_sm * sms;
+  }
+  return chain_cap[dev];
+}
+
+cudaError_t launch_gemm_chain(const ChainArgs& ca, bool pdl, cudaStream_t s) {
+  using S = GemmSmem<kChainNT, kChainStages, false>;
+  if (ca.n_phases < 1 || ca.n_phases > kMaxChainPhases || ca.P < 1 || !ca.bar || !ca.status)
+    return cudaErrorInvalidValue;
+  for (int p = 0; p < ca.n_phases; ++p) {
+    const ChainPhase& ph = ca.ph[p];
+    const int epi = ph.ea.epi;
+    if ((epi != EPI_QKV && epi != EPI_RESID && epi != EPI_SWIGLU) || ph.n_tiles < 1 || ph.kb < 1 ||
+        ph.ea.n_rows < 1 || ph.ea.n_rows > kChainNT || !ph.ea.part || !ph.ea.cnt || ph.ea.status != ca.status)
+      return cudaErrorInvalidValue;
+  }
+  // every CTA must be resident at once: the phases meet at grid barriers
+  const int cap = gemm_chain_max_ctas();
+  if (cap < 1) return cudaErrorInvalidConfiguration;
+  if (ca.P > cap) return cudaErrorCooperativeLaunchTooLarge;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ca.P);
+  cfg.blockDim = dim3(kChainThreads);
+  cfg.dynamicSmemBytes = S::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_chain_kernel<kChainStages>, ca);
 }
 
 }  // namespace dvlm

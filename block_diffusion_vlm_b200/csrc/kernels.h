@@ -132,6 +132,30 @@ size_t gemm_ws_part_bytes(int NT, int P);
 cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& mapB, int n_tiles, int kb, int S,
                            int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s, int stages);
 int gemm_cl_max_clusters(int epi, int S, int stages);
+
+// Persistent chain of bf16 weight-streaming GEMMs over 16 token rows: up to
+// kMaxChainPhases products run as consecutive stream-K phases of one launch
+// of P CTAs (one per SM, all resident at once), each phase's inputs the
+// previous phases' outputs (a grid barrier between phases).  Phase p streams
+// weights mapA (mapA2: the up rows of a gate/up product) against activations
+// mapB over n_tiles x kb units with the fused epilogue ea (ea.cnt: n_tiles
+// zeroed ints of its own; ea.part: P partial tiles, shared by the phases).
+struct ChainPhase {
+  CUtensorMap mapA, mapA2, mapB;
+  GemmEpi ea;
+  int n_tiles, kb, a_row_base;
+};
+constexpr int kMaxChainPhases = 4;
+struct ChainArgs {
+  ChainPhase ph[kMaxChainPhases];
+  int n_phases;
+  int P;
+  int* bar;     // [2] barrier and exit counters: zero before the first launch, zero again after each
+  int* status;
+};
+cudaError_t launch_gemm_chain(const ChainArgs& ca, bool pdl, cudaStream_t s);
+// CTAs of the chain kernel that can be resident at once on the current device (0 on error).
+int gemm_chain_max_ctas();
 cudaError_t launch_lmhead(int NT, const CUtensorMap& mapW, const CUtensorMap& mapH, int n_tiles, int kb, int P,
                           const LmArgs& a, bool pdl, cudaStream_t s);
 size_t lmhead_scratch_bytes(int NT, int P, int n_tiles);

@@ -98,33 +98,33 @@ __device__ __forceinline__ void ws_producer(const CUtensorMap* mapA, const CUten
   }
 }
 
-// FP8: B is the activation code block of k block kk at sB + (kk - kb_lo) *
-// NT * 128, written once before b_ready completes.
+// The MMA issuer's work for the stream-K units [u0, u1) of one GEMM.  i_base
+// is the pipeline stage index of the first unit and seg the CTA's segment
+// count (accumulator buffer and phase); both carry over to a following GEMM
+// of the same kernel.  FP8: B is the activation code block of k block kk at
+// sB + (kk - kb_lo) * NT * 128, written before the units start.  Returns
+// false when a wait gave up.
 template <int NT, int STAGES, bool FP8 = false>
-__device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty, uint64_t* accf,
-                                       uint64_t* acce, uint32_t tmem, const SkSched& sc, long long u0, long long u1,
-                                       int* status, volatile int* abort_flag, int issuer, uint64_t* b_ready = nullptr,
-                                       int kb_lo = 0) {
+__device__ __forceinline__ bool ws_mma_units(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty,
+                                             uint64_t* accf, uint64_t* acce, uint32_t tmem, const SkSched& sc,
+                                             long long u0, long long u1, int* status, volatile int* abort_flag,
+                                             int issuer, int kb_lo, long long& i_base, int& seg) {
   // Issuer `issuer` (0 or 1) takes the k blocks j = issuer, issuer + 2, ... of
   // each segment into accumulator (b, issuer); both commit accf[b] (count 2).
   constexpr int B_BYTES = NT * 128;
   constexpr uint32_t IDESC = FP8 ? idesc_e4m3_f32(128, NT) : idesc_bf16_f32(128, NT);
-  griddep_wait();
-  if (FP8 && !mbar_wait(b_ready, 0, status, abort_flag)) return;
-  long long i_base = 0;  // pipeline stage index of the segment's first k block
-  int seg = 0;
   for (long long u = u0; u < u1; ++seg) {
     const int T = static_cast<int>(u / sc.kb);
     const long long seg_end = (static_cast<long long>(T) + 1) * sc.kb < u1 ? (static_cast<long long>(T) + 1) * sc.kb : u1;
     const int b = seg & 1;
-    if (seg >= 2 && !mbar_wait(&acce[b], ((seg >> 1) - 1) & 1, status, abort_flag)) return;
+    if (seg >= 2 && !mbar_wait(&acce[b], ((seg >> 1) - 1) & 1, status, abort_flag)) return false;
     tc_fence_after();
     const uint32_t d = tmem + static_cast<uint32_t>((b * 2 + issuer) * NT);
     const long long len = seg_end - u;
     for (long long jj = issuer; jj < len; jj += 2) {
       const long long i = i_base + jj;
       const int s = static_cast<int>(i % STAGES);
-      if (!mbar_wait(&full[s], static_cast<uint32_t>((i / STAGES) & 1), status, abort_flag)) return;
+      if (!mbar_wait(&full[s], static_cast<uint32_t>((i / STAGES) & 1), status, abort_flag)) return false;
       tc_fence_after();
       const uint32_t a0 = smem_u32(sA + s * kATileBytes);
       const uint32_t b0 = FP8 ? smem_u32(sB + (static_cast<int>((u + jj) % sc.kb) - kb_lo) * B_BYTES)
@@ -144,6 +144,20 @@ __device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full,
     i_base += len;
     u = seg_end;
   }
+  return true;
+}
+
+template <int NT, int STAGES, bool FP8 = false>
+__device__ __forceinline__ void ws_mma(uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty, uint64_t* accf,
+                                       uint64_t* acce, uint32_t tmem, const SkSched& sc, long long u0, long long u1,
+                                       int* status, volatile int* abort_flag, int issuer, uint64_t* b_ready = nullptr,
+                                       int kb_lo = 0) {
+  griddep_wait();
+  if (FP8 && !mbar_wait(b_ready, 0, status, abort_flag)) return;
+  long long i_base = 0;
+  int seg = 0;
+  ws_mma_units<NT, STAGES, FP8>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, status, abort_flag, issuer, kb_lo,
+                                i_base, seg);
 }
 
 // The NT accumulator columns of segment buffer b for this thread's lane: the

@@ -115,6 +115,11 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Generic-proxy accesses to global memory ordered with async-proxy (TMA)
+// accesses: a writer's plain stores before a TMA load of them (by any CTA).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // 2^x by the hardware approximation (PTX ex2.approx: relative error about
 // 2^-22; -inf gives +0; subnormal results flush to zero).

@@ -465,9 +465,14 @@ DVLM_API dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int
  *   "pdl": 1/0, programmatic dependent launch between kernels;
  *   "attn_split": 0 = cluster attention, 1..32 = split attention with that
  *       many CTAs per KV head (dvlm_block_attn_split);
- *   "prefill_gemm": 1/0, the compute-bound prefill (where supported).
+ *   "prefill_gemm": 1/0, the compute-bound prefill (where supported);
+ *   "persistent": 1/0, the decoder GEMMs as a persistent chain: per layer,
+ *       after attention, one launch on every SM runs the O-projection,
+ *       gate/up, down and the next layer's QKV as stream-K phases separated
+ *       by grid barriers (bf16 weights, 128-wide heads; UNSUPPORTED where
+ *       one CTA per SM cannot be resident on all SMs).
  * Results do not depend on the knobs except through fp32 summation order
- * (cluster sizes).  Changing a knob drops the captured CUDA graphs.
+ * (cluster sizes, stream-K splits).  Changing a knob drops the captured CUDA graphs.
  * Errors: INVALID_ARG (unknown name), SHAPE (bad value), UNSUPPORTED (the
  * device cannot launch that configuration, or an fp32 engine). */
 DVLM_API dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value);
@@ -533,11 +538,14 @@ DVLM_API dvlm_status dvlm_engine_set_trace(dvlm_engine* e, void* buf, size_t byt
 
 /* Profiling hook: one forward pass like dvlm_forward over all layers (L is
  * not advanced), launched eagerly with a CUDA event pair around every kernel
- * on `stream`.  ms_out[7] receives the device time per kernel class summed
- * over layers and counts_out[7] the launches: [0] embedding, [1] QKV GEMM,
+ * on `stream`.  ms_out[8] receives the device time per kernel class summed
+ * over layers and counts_out[8] the launches: [0] embedding, [1] QKV GEMM,
  * [2] attention, [3] O-projection GEMM, [4] gate/up GEMM, [5] down GEMM,
  * [6] fused LM head (run when with_lm_head != 0, rows 0..n_rows-1, no
- * commit).  Synchronises the stream. */
+ * commit), [7] persistent GEMM chain (option "persistent": the first
+ * layer's QKV, then per layer O-projection, gate/up, down and the next
+ * layer's QKV in one launch; classes 1, 3, 4 and 5 are then empty).
+ * Synchronises the stream. */
 DVLM_API dvlm_status dvlm_profile_forward(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
                                           int n_rows, int n_clean, int with_lm_head, float* ms_out,
                                           int* counts_out, dvlm_stream stream);

@@ -44,13 +44,16 @@ SMALL_BF16 = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, h
 
 
 class Setup:
-    def __init__(self, dims, seed, cuda, n_vis, n_prompt, n_comm, Lmax=512):
+    def __init__(self, dims, seed, cuda, n_vis, n_prompt, n_comm, Lmax=512, options=None):
         self.dims, self.seed, self.cuda = dims, seed, cuda
         self.dm = DeviceModel(dims, seed, device=cuda)
         self.kc, self.vc = kv_buffers(dims, Lmax, device=cuda)
         cm = self.dm.c_model()
         self.ws = ws_tensor(dv.engine_workspace_size(cm, Lmax, 16, 128), cuda)
         self.eng = dv.Engine(cm, self.kc, self.vc, Lmax, 16, 128, self.ws)
+        for name, value in (options or {}).items():
+            self.eng.set_option(name, value)
+            assert self.eng.get_option(name) == value
         self.vis_t, self.vis, self.ids = gen.decode_context(dims, seed, n_vis, n_prompt, n_comm)
         self.w = O.weights_from_generator(gen, dims, seed)
         self.od = O.dims_from(dims)
@@ -203,16 +206,21 @@ def test_bf16_reduced_model_matches_oracle(cuda, seed, mode):
     s.eng.close()
 
 
-@pytest.mark.parametrize("seed,mode", [(1, dv.MODE_THRESHOLD), (3, dv.MODE_THRESHOLD),
-                                       (6, dv.MODE_SPEC_LINEAR), (2, dv.MODE_SPEC_LINEAR)])
-def test_bf16_reduced_model_engine_path(cuda, seed, mode):
+@pytest.mark.parametrize("seed,mode,persistent", [(1, dv.MODE_THRESHOLD, 0), (3, dv.MODE_THRESHOLD, 0),
+                                                  (6, dv.MODE_SPEC_LINEAR, 0), (2, dv.MODE_SPEC_LINEAR, 0),
+                                                  (1, dv.MODE_THRESHOLD, 1), (6, dv.MODE_SPEC_LINEAR, 1)])
+def test_bf16_reduced_model_engine_path(cuda, seed, mode, persistent):
     """The engine's own graph-driven decode of the reduced bf16 model (B=16,
     tau 0.9, 32 tokens; in-graph commit, shift-1 row mapping, block set-up,
     emission and, for speculative decoding, the accept kernel), every forward
     replayed against the oracle: decisions bit-exact at the 1e-3 bar on the
     rows the LM head read, within DELTA on the oracle's own rows, hidden rows
-    within 2e-2 plus one storage ulp."""
-    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0)
+    within 2e-2 plus one storage ulp.  persistent=1: the decoder GEMMs run as
+    the persistent chain (first layer's QKV; then O-projection, gate/up,
+    down and the next layer's QKV per launch); at this size most CTAs of a
+    phase hold one k block or none, so every output tile is split over many
+    CTAs."""
+    s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0, options={"persistent": persistent} if persistent else None)
     tokens, st, recs, L, sd = s.traced(mode, 16, 0.9, 32)
     rp, m = replay_trace(s, mode, 16, 0.9, 32, tokens, st, recs, L, sd)
     t = rp.t

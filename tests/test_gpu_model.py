@@ -202,6 +202,81 @@ def test_every_layer_matches_oracle_on_identical_inputs(full):
     print("per-layer max abs error:", worst)
 
 
+def test_persistent_chain_matches_oracle_per_layer(full):
+    """The persistent GEMM chain at full size (option "persistent"): layers
+    0, 1, 17 and 35 run one at a time on identical inputs (the first
+    layer's QKV as a one-phase chain, attention, then O-projection, gate/up
+    and down as one three-phase launch), each against the oracle's layer at
+    the 2e-2 bar; the input of layer l is the per-kernel path's output of
+    layers 0..l-1.  Then layers 17 and 18 in one forward, whose first chain
+    launch has all four phases (O, gate/up, down, layer 18's QKV), against
+    the per-kernel path on the same input."""
+    dims, eng, cuda = full["dims"], full["eng"], full["kc"].device
+    L0 = full["L0"]
+    names = gen.layer_weight_names()
+    toks = torch.tensor([full["seed0"]] + [dims.mask_id] * 15, dtype=torch.int32, device=cuda)
+    x_in = torch.zeros((16, dims.hidden), dtype=torch.bfloat16, device=cuda)
+    x_out = torch.zeros_like(x_in)
+    assert eng.get_option("persistent") == 0
+    try:
+        for l in (0, 1, 17, 35):
+            eng.set_position(L0, full["seed0"])
+            if l > 0:
+                eng.set_option("persistent", 0)
+                eng.forward(16, 0, l, tokens=toks, first_layer=0, x_out=x_in)
+                eng.check()
+            eng.set_option("persistent", 1)
+            if l == 0:
+                eng.forward(16, 0, 1, tokens=toks, first_layer=0, x_out=x_out)
+                E = gen.embedding_weight(dims, SEED)[1]
+                xin64 = np.asarray(E[toks.cpu().numpy()], dtype=np.float64)
+                del E
+            else:
+                eng.forward(16, 0, 1, x_in=x_in, first_layer=l, x_out=x_out)
+                xin64 = f64(x_in)
+            eng.check()
+            w = {f"{l}.{k}": gen.layer_weight(dims, SEED, l, k)[1] for k in names}
+            m = O.OracleModel(O.dims_from(dims), weights=w, bf16=True, Lmax=L0 + 16)
+            m.K[l][:, :L0] = f64(full["kc"][l, 0, :, :L0])
+            m.V[l][:, :L0] = f64(full["vc"][l, 0, :, :, :L0]).transpose(0, 2, 1)
+            xo = m.layer(l, xin64, L0, 0)
+            assert_bf16_close(f64(x_out), xo, 2e-2, f"chain layer {l} output")
+            assert_bf16_close(f64(full["kc"][l, 0, :, L0:L0 + 16]), m.K[l][:, L0:L0 + 16], 2e-2, f"chain layer {l} K")
+            assert_bf16_close(f64(full["vc"][l, 0, :, :, L0:L0 + 16]).transpose(0, 2, 1), m.V[l][:, L0:L0 + 16],
+                              2e-2, f"chain layer {l} V")
+        # two layers: the four-phase launch against the per-kernel path
+        eng.set_option("persistent", 0)
+        eng.forward(16, 0, 17, tokens=toks, first_layer=0, x_out=x_in)
+        outs = []
+        for persistent in (0, 1):
+            eng.set_option("persistent", persistent)
+            eng.forward(16, 0, 2, x_in=x_in, first_layer=17, x_out=x_out)
+            eng.check()
+            outs.append((f64(x_out), f64(full["kc"][18, 0, :, L0:L0 + 16])))
+        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, chain vs per-kernel")
+        assert_bf16_close(outs[1][1], outs[0][1], 2e-2, "layer 18 K, chain vs per-kernel")
+    finally:
+        eng.set_option("persistent", 0)
+    eng.set_position(L0, full["seed0"])
+
+
+def test_persistent_chain_decode_properties(full):
+    """Properties of the persistent chain's decode at full size: linear
+    self-speculative decoding equals greedy AR decoding, and graph replay
+    equals eager launches."""
+    eng = full["eng"]
+    eng.set_option("persistent", 1)
+    try:
+        ar, _ = _gen(full, dv.MODE_AR, 16, 32)
+        sp, _ = _gen(full, dv.MODE_SPEC_LINEAR, 16, 32)
+        assert sp == ar
+        a, sa = _gen(full, dv.MODE_THRESHOLD, 16, 32)
+        b, sb = _gen(full, dv.MODE_THRESHOLD, 16, 32, graphs=0)
+        assert a == b and sa.nfe == sb.nfe
+    finally:
+        eng.set_option("persistent", 0)
+
+
 def test_spec_linear_equals_greedy_ar(full):
     ar, st_ar = _gen(full, dv.MODE_AR, 16, 48)
     sp, st_sp = _gen(full, dv.MODE_SPEC_LINEAR, 16, 48)
