@@ -514,46 +514,62 @@ def run_sweep(args, local):
         d.update(peak=hbm_peak, peak_source=f"{peak_kind} copy bandwidth")
         print(json.dumps(d), flush=True)
 
+    D, Hq, Hkv = dims.head_dim, dims.n_q_heads, dims.n_kv_heads
+
+    def attn_case(B, L, nb, split_list):
+        """Times the cluster kernel and the split kernel (each S in split_list)
+        on one shape; prints one line per kernel configuration."""
+        Lmax = (L + B + 7) // 8 * 8
+        q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=Lmax, n_batch=nb))
+        qd, kd = q.to(dev).contiguous(), k.to(dev).contiguous()
+        vt = v.transpose(-1, -2).contiguous().to(dev)
+        out = torch.empty_like(qd)
+        b = nb * algorithmic_bytes("attention", dims, L, rows=B)
+        reps = 20 if nb > 1 else 200
+
+        def call():
+            dv.block_attn(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
+                          Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, dtype=dv.DVLM_BF16, status=st)
+
+        ms, mode = _device_ms_per_call(call, reps, dev)
+        emit({"sweep": "attention", "kernel": "cluster", "B": B, "L": L, "caches_per_launch": nb,
+              "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
+              "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
+              "frac": b / (ms * 1e-3) / 1e9 / hbm_peak,
+              "working_set_mb": (kd.numel() + vt.numel()) * 2 / 1e6, "timing": mode})
+        for splits in split_list:
+            ws = torch.zeros((dv.block_attn_split_workspace_size(nb, B, Hkv, splits) + 3) // 4,
+                             dtype=torch.int32, device=dev)
+
+            def call_split():
+                dv.block_attn_split(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
+                                    Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, splits=splits, workspace=ws,
+                                    status=st)
+
+            ms, mode = _device_ms_per_call(call_split, reps, dev)
+            emit({"sweep": "attention", "kernel": "split", "splits": splits, "B": B, "L": L,
+                  "caches_per_launch": nb, "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
+                  "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
+                  "frac": b / (ms * 1e-3) / 1e9 / hbm_peak, "timing": mode})
+            del ws
+        del qd, kd, vt, out
+
+    def auto_splits(B, L, nb):
+        # enough CTAs to fill the SMs (one CTA per 128-key chunk at most)
+        n_chunks = (L + B + 127) // 128
+        groups = nb * ((B + 15) // 16) * Hkv
+        return max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
+
+    if args.sweep == "attn_decode":
+        # the decode shape (one cache per launch) and the long batched case,
+        # split counts around the automatic choice
+        attn_case(BLOCK, N_VIS + N_PROMPT, 1, [2, 4, 8, 16])
+        attn_case(BLOCK, 4096, dims.n_layers, [1, 2, 3, 4])
     if args.sweep in ("attention", "all"):
-        D, Hq, Hkv = dims.head_dim, dims.n_q_heads, dims.n_kv_heads
         for B in (4, 8, 16, 32):
             for L in (256, 1024, 4096):
-                Lmax = (L + B + 7) // 8 * 8
                 for nb in (1, dims.n_layers):
-                    q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=Lmax, n_batch=nb))
-                    qd, kd = q.to(dev).contiguous(), k.to(dev).contiguous()
-                    vt = v.transpose(-1, -2).contiguous().to(dev)
-                    out = torch.empty_like(qd)
-
-                    def call():
-                        dv.block_attn(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
-                                      Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, dtype=dv.DVLM_BF16, status=st)
-
-                    ms, mode = _device_ms_per_call(call, 20 if nb > 1 else 200, dev)
-                    b = nb * algorithmic_bytes("attention", dims, L, rows=B)
-                    emit({"sweep": "attention", "kernel": "cluster", "B": B, "L": L, "caches_per_launch": nb,
-                          "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
-                          "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
-                          "frac": b / (ms * 1e-3) / 1e9 / hbm_peak,
-                          "working_set_mb": (kd.numel() + vt.numel()) * 2 / 1e6, "timing": mode})
-                    # the split form: enough CTAs to fill the SMs (one CTA per 128-key chunk at most)
-                    n_chunks = (L + B + 127) // 128
-                    groups = nb * ((B + 15) // 16) * Hkv
-                    splits = max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
-                    ws = torch.zeros((dv.block_attn_split_workspace_size(nb, B, Hkv, splits) + 3) // 4,
-                                     dtype=torch.int32, device=dev)
-
-                    def call_split():
-                        dv.block_attn_split(qd, out, kd, vt, n_batch=nb, n_rows=B, n_clean=0, L=L, Lmax=Lmax, Hq=Hq,
-                                            Hkv=Hkv, D=D, scale=1.0 / D ** 0.5, splits=splits, workspace=ws,
-                                            status=st)
-
-                    ms, mode = _device_ms_per_call(call_split, 20 if nb > 1 else 200, dev)
-                    emit({"sweep": "attention", "kernel": "split", "splits": splits, "B": B, "L": L,
-                          "caches_per_launch": nb, "us_per_launch": 1000 * ms, "us_per_cache": 1000 * ms / nb,
-                          "bytes_per_launch": b, "gbs": b / (ms * 1e-3) / 1e9,
-                          "frac": b / (ms * 1e-3) / 1e9 / hbm_peak, "timing": mode})
-                    del qd, kd, vt, out, ws
+                    attn_case(B, L, nb, [auto_splits(B, L, nb)])
         # TEXT-ONLY pass of certificate-guided routing at the decode shape: the
         # 1280 vision slots hidden by viewing the cache from slot 1280 (64 spare
         # slots keep the last key chunk inside each head's rows)
@@ -617,6 +633,81 @@ def run_sweep(args, local):
 
         ms, mode = _device_ms_per_call(call, 200, dev)
         emit({"sweep": "topk_commit", "R": R, "k": k, "us_per_launch": 1000 * ms, "timing": mode})
+    if args.sweep in ("spec", "all"):
+        # speculative verify + accept on bf16 logits [b, 16, 151936] (cache
+        # lengths updated in place); four input sets in turn, so that b = 8
+        # (4 x 38.9 MB) does not run from L2
+        V = dims.vocab
+        for b in (1, 8):
+            sets = []
+            for i in range(4):
+                logits_t, _, _, draft, _ = gen.spec_case(4 + i, b, BLOCK, V)
+                sets.append((logits_t.to(dev), torch.from_numpy(draft).to(dev)))
+            acc = torch.zeros(b, dtype=torch.int32, device=dev)
+            cl = torch.full((b,), 1 << 30, dtype=torch.int32, device=dev)
+            ws = torch.zeros((dv.spec_workspace_size(b, BLOCK, V) + 3) // 4 + 1, dtype=torch.int32, device=dev)
+            calls = [0]
+
+            def call():
+                lg, dr = sets[calls[0] % 4]
+                calls[0] += 1
+                dv.spec_verify_accept(draft_ids=dr, b=b, B=BLOCK, V=V, accept_len=acc, verify_logits=lg,
+                                      cache_len=cl, workspace=ws, status=st)
+
+            for _ in range(4):
+                call()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 64
+            e0.record()
+            for _ in range(reps):
+                call()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / reps
+            nbytes = b * BLOCK * V * 2 + 2 * b * BLOCK * 4
+            emit({"sweep": "spec_accept", "b": b, "B": BLOCK, "V": V, "us_per_launch": 1000 * ms,
+                  "bytes_per_launch": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                  "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "timing": "eager", "input_sets": 4})
+            del sets, ws
+    if args.sweep in ("tiny", "all"):
+        # the tiny fp32 configuration: 1 layer, hidden 32, 64 context slots,
+        # one block of B = 4 to completion (threshold 0.9), graph-driven
+        from dvlm_gen.device import DeviceModel, kv_buffers
+        td = gen.TINY
+        dm = DeviceModel(td, 0, device=dev)
+        Lmax = 128
+        kc, vc = kv_buffers(td, Lmax, device=dev)
+        cm = dm.c_model()
+        ws = torch.zeros(dv.engine_workspace_size(cm, Lmax, 16, 128) // 4 + 1, dtype=torch.int32, device=dev)
+        eng = dv.Engine(cm, kc, vc, Lmax, 16, 128, ws)
+        vis_t, _, ids = gen.decode_context(td, 0, 32, 16, 16)
+        eng.prefill(vis_t.to(dev), 32, torch.from_numpy(ids).to(dev), len(ids))
+        eng.check()
+        L0, seed0 = eng.position()
+        cfg = dv.DecodeCfg(4, TAU, dv.MODE_THRESHOLD, 1, 4, 1)
+        out = torch.zeros(4, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            eng.set_position(L0, seed0)
+            eng.generate(cfg, out)
+        torch.cuda.synchronize(dev)
+        reps = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        total = 0.0
+        for _ in range(reps):
+            stt = dv.Stats()
+            eng.set_position(L0, seed0)
+            e0.record()
+            eng.generate(cfg, out, stt)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            total += e0.elapsed_time(e1)
+        eng.check()
+        ms = total / reps
+        emit({"sweep": "tiny_step", "B": 4, "context": L0, "nfe": stt.nfe, "ms_per_block": ms,
+              "us_per_forward": 1000 * ms / max(stt.nfe, 1), "tokens_per_s": 4 / (ms * 1e-3),
+              "timing": "graph replay per forward, host-driven block loop"})
+        eng.close()
     torch.cuda.synchronize(dev)
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} after the sweep")
@@ -638,7 +729,7 @@ def main():
     ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")
     ap.add_argument("--profile-forwards", type=int, default=0,
                     help="profiling case: run this many eager forwards after prefill and exit")
-    ap.add_argument("--sweep", choices=["attention", "lmhead", "all"], default=None,
+    ap.add_argument("--sweep", choices=["attention", "attn_decode", "lmhead", "spec", "tiny", "all"], default=None,
                     help="time the single-kernel configurations (one JSON line per case) instead of the decode")
     args = ap.parse_args()
     rank, world, local, pg = dist_setup()

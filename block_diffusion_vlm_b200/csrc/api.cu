@@ -515,7 +515,7 @@ dvlm_status dvlm_prefill(dvlm_engine* e, const void* vision, int n_vision, const
 static dvlm_status check_cfg(dvlm_engine* e, const dvlm_decode_cfg* cfg) {
   if (!e || !cfg) return DVLM_ERR_INVALID_ARG;
   if (cfg->block_size < 1 || cfg->block_size > e->max_block) return DVLM_ERR_SHAPE;
-  if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_SPEC_QUAD) return DVLM_ERR_INVALID_ARG;
+  if (cfg->mode < DVLM_MODE_THRESHOLD || cfg->mode > DVLM_MODE_ROUTE) return DVLM_ERR_INVALID_ARG;
   if (cfg->mode == DVLM_MODE_SPEC_QUAD && !quad_supported(e, cfg->block_size)) return DVLM_ERR_UNSUPPORTED;
   if (cfg->mode == DVLM_MODE_ROUTE) {
     if (!e->bf16 || e->paged) return DVLM_ERR_UNSUPPORTED;

@@ -316,49 +316,51 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     named_bar_sync(1, 128);
     if (*sflag) {
       // ------------------------------------------------------------ merge
+      // (m, l) of every split and row into shared memory (the K stages are
+      // free now), each row's weights w_q = 2^(m_q - M) l_q in place of m_q;
+      // then one warp per row, its 128 values as 32 lanes x 4, the splits'
+      // partials (independent, coalesced 512-byte loads) summed in split order
       __threadfence();
       if (threadIdx.x == 64) cnt[grp] = 0;  // every split arrived: zero for the next launch
+      const int et = threadIdx.x - 64;
       const size_t p0 = static_cast<size_t>(grp) * S;
-      float M = -INFINITY;
-      for (int q = 0; q < S; ++q) M = fmaxf(M, __ldcg(&ml[(p0 + q) * 128 + row]).x);
-      float wsum = 0.f;
-      for (int q = 0; q < S; ++q) {
-        const float2 v = __ldcg(&ml[(p0 + q) * 128 + row]);
-        wsum += v.y > 0.f ? ex2_approx(v.x - M) * v.y : 0.f;
-      }
-      const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
-      const int hl = row & 7;
-      bf16* dst = a.out + ((static_cast<size_t>(bidx) * a.n_rows + t) * a.Hq + g * 8 + hl) * 128;
-#pragma unroll 1
-      for (int d0 = 0; d0 < 128; d0 += 32) {
-        float acc[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+      float2* sml = reinterpret_cast<float2*>(sK);  // [S][128]
+      float* sinv = reinterpret_cast<float*>(sV);   // [128]
+      for (int i = et; i < S * 128; i += 128) sml[i] = __ldcg(&ml[p0 * 128 + i]);
+      named_bar_sync(1, 128);
+      {
+        float M = -INFINITY;
+        for (int q = 0; q < S; ++q) M = fmaxf(M, sml[q * 128 + row].x);
+        float wsum = 0.f;
         for (int q = 0; q < S; ++q) {
-          const float2 v = __ldcg(&ml[(p0 + q) * 128 + row]);
-          if (!(v.y > 0.f)) continue;
-          const float w = ex2_approx(v.x - M) * v.y;
-          const float4* src = reinterpret_cast<const float4*>(part + ((p0 + q) * 128 + row) * 128 + d0);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float4 f = __ldcg(src + k);
-            acc[4 * k] += w * f.x;
-            acc[4 * k + 1] += w * f.y;
-            acc[4 * k + 2] += w * f.z;
-            acc[4 * k + 3] += w * f.w;
-          }
+          const float2 v = sml[q * 128 + row];
+          const float w = v.y > 0.f ? ex2_approx(v.x - M) * v.y : 0.f;
+          sml[q * 128 + row].x = w;
+          wsum += w;
         }
-        if (t < a.n_rows) {
-#pragma unroll
-          for (int k = 0; k < 32; k += 8) {
-            uint32_t wv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const __nv_bfloat162 b = __floats2bfloat162_rn(acc[k + 2 * q] * inv, acc[k + 2 * q + 1] * inv);
-              wv[q] = *reinterpret_cast<const uint32_t*>(&b);
-            }
-            *reinterpret_cast<uint4*>(dst + d0 + k) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          }
+        sinv[row] = wsum > 0.f ? 1.0f / wsum : 0.f;
+      }
+      named_bar_sync(1, 128);
+      for (int r = et >> 5; r < 128; r += 4) {
+        const int tr = t_base + (r >> 3);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4* src = reinterpret_cast<const float4*>(part + (p0 * 128 + r) * 128) + lane;
+#pragma unroll 4
+        for (int q = 0; q < S; ++q) {
+          const float w = sml[q * 128 + r].x;
+          const float4 f = __ldcg(src + static_cast<size_t>(q) * 128 * 32);
+          acc.x += w * f.x;
+          acc.y += w * f.y;
+          acc.z += w * f.z;
+          acc.w += w * f.w;
+        }
+        if (tr < a.n_rows) {
+          const float inv = sinv[r];
+          bf16* dst = a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + lane * 4;
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+          const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+          *reinterpret_cast<uint2*>(dst) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
         }
       }
     }

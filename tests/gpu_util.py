@@ -35,12 +35,20 @@ def assert_bf16_close(got, want, tol=2e-2, what=""):
     """Max abs error `tol`, plus one bf16 storage ulp of the reference: both
     sides round a nearly equal real to bf16, and where that real sits next to
     a rounding boundary the two roundings differ by one ulp (0.03125 for
-    |x| in [4, 8)).  At most 0.1% of elements may use that allowance."""
+    |x| in [4, 8)).  How many elements may use that allowance: a flip needs
+    the two reals (which differ by delta, the fp32-against-fp64 arithmetic
+    difference, at most about 3e-3 here) to straddle a boundary, probability
+    delta / ulp, so at most 10% of the elements whose ulp exceeds tol (the
+    only ones a flip can take past tol), or 0.1% of all elements where that
+    is more."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     err = np.abs(got - want)
-    bad = np.argwhere(err > tol + bf16_ulp(want))
+    ulp = bf16_ulp(want)
+    bad = np.argwhere(err > tol + ulp)
     detail = [(tuple(int(v) for v in i), float(got[tuple(i)]), float(want[tuple(i)]), float(err[tuple(i)]))
               for i in bad[:8]]
     assert len(bad) == 0, (what, float(err.max()), detail)
-    assert np.mean(err > tol) <= 1e-3, (what, float(np.mean(err > tol)))
+    n_allow = int(np.sum(err > tol))
+    budget = max(1e-3 * err.size, 0.1 * int(np.sum(ulp > tol)))
+    assert n_allow <= budget, (what, n_allow, budget, err.size)

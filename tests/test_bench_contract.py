@@ -135,8 +135,9 @@ class _GraphCtx:
 def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     """`bench.py --sweep all` with the entry points, CUDA graphs and large
     draws replaced by stand-ins: the attention cases (12 shapes, one cache
-    and 36 caches per launch, plus the TEXT-ONLY pair) and the four LM-head
-    row counts each print one line with their bytes, GB/s and fraction."""
+    and 36 caches per launch, plus the TEXT-ONLY pair), the four LM-head
+    row counts and the speculative accept at b = 1 and 8 each print one line
+    with their bytes, GB/s and fraction; the tiny step prints its block time."""
     sys.path.insert(0, ROOT)
     bench = importlib.import_module("bench")
     import block_diffusion_vlm_b200 as dv
@@ -159,6 +160,17 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     monkeypatch.setattr(gen, "attn_case", lambda *a, **k: ((small, None),) * 3)
     monkeypatch.setattr(gen, "lmhead_case", lambda *a, **k: ((small, None), (small, None)))
     monkeypatch.setattr(gen, "normal_bf16", lambda *a, **k: (small, None))
+    import numpy as np
+    import dvlm_gen.device as gdev
+    monkeypatch.setattr(gen, "spec_case", lambda *a, **k: (small, None, None, np.zeros((1, 16), np.int32), None))
+    monkeypatch.setattr(dv, "spec_verify_accept", lambda **kw: calls["spec"].append(kw["b"]))
+    monkeypatch.setattr(dv, "spec_workspace_size", lambda *a: 64)
+    monkeypatch.setattr(gdev, "DeviceModel", _FakeDeviceModel)
+    monkeypatch.setattr(gdev, "kv_buffers", lambda *a, **k: (None, None))
+    monkeypatch.setattr(gen, "decode_context", lambda *a, **k: (small, None, np.zeros(16, np.int32)))
+    monkeypatch.setattr(dv, "Engine", _FakeEngine)
+    monkeypatch.setattr(dv, "engine_workspace_size", lambda *a: 64)
+    calls["spec"] = []
     args = bench.argparse.Namespace(sweep="all")
     bench.run_sweep(args, 0)
     lines = [json.loads(ln) for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
@@ -181,3 +193,8 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     assert all(d["bytes_per_launch"] == bench.algorithmic_bytes("lm_head", gen.QWEN3B, 0, rows=d["R"]) for d in lm)
     tk = [d for d in lines if d["sweep"] == "topk_commit"]
     assert len(tk) == 1 and tk[0]["R"] == 16 and tk[0]["us_per_launch"] > 0
+    sp = [d for d in lines if d["sweep"] == "spec_accept"]
+    assert [d["b"] for d in sp] == [1, 8] and set(calls["spec"]) == {1, 8}
+    assert all(d["bytes_per_launch"] == d["b"] * 16 * 151936 * 2 + 2 * d["b"] * 16 * 4 for d in sp)
+    tiny = [d for d in lines if d["sweep"] == "tiny_step"]
+    assert len(tiny) == 1 and tiny[0]["B"] == 4 and tiny[0]["ms_per_block"] > 0

@@ -8,15 +8,33 @@ one scale per weight output row and per activation token, amax / 448].
   exactly on E4M3 rounding midpoints, so every tie is exercised), scales
   within fp32 rounding of amax / 448.
 * The W8A8 decoder (reduced model: 2 layers, hidden 1024, 8/1 heads of 128,
-  SwiGLU 1024) against OracleModel(fp8=True): the prefilled KV cache and a
-  noisy forward's hidden rows within the bf16 bar (2e-2 plus one storage ulp);
-  then threshold decoding through the engine's own graph path, every forward
+  SwiGLU 1024) against OracleModel(fp8=True): the prefilled KV cache, a
+  noisy forward's hidden rows, and each layer on identical inputs (bars
+  below); then threshold decoding through the engine's own graph path, every forward
   replayed against the oracle's W8A8 model, decisions bit-exact at the 1e-3
-  bar on the rows the LM head read and within DELTA on the oracle's own rows.
+  bar on the rows the LM head read.
   The activations are quantised on the GPU from an fp32 quotient (the oracle
   forms it in fp64): a code can differ where the quotient sits within fp32
   rounding of an E4M3 midpoint, a one-code change of one of the K terms of a
-  sum, which the bf16 bar covers."""
+  sum, which the bf16 bar covers.
+
+Where the two sides' inputs to a quantisation differ (a bf16 value one ulp
+apart, from fp32-against-fp64 arithmetic or the attention's fp16 P and V
+upstream), a code moves by one E4M3 step (1/16 to 1/8 relative), and a token
+whose largest magnitude moves shifts all its codes' quotients: W8A8 turns
+storage-level differences into code-level ones.  A CPU model of exactly this
+(the oracle's W8A8 model against a copy whose values are perturbed by 2^-20
+relative before each bf16 rounding and by 2^-11 on the attention output,
+eight seeds) gives, on the reduced model: layer outputs on identical inputs
+within 0.041 (4.9% of the rows' largest magnitude), layer-1 K/V after the
+prefill within 0.195 (6.9% of the largest key), and a 2-layer noisy forward
+within 0.073 (8.1%); the bf16 model under the same perturbation stays within
+0.016.  The bars: the first layer's K/V and each layer's block K/V on
+identical inputs at the bf16 bar (their codes come from identical rows);
+layer outputs on identical inputs within 8% and everything downstream of a
+quantised layer within 12% of the compared rows' largest magnitude; the
+decisions themselves stay bit-exact at the 1e-3 bar on the rows the LM head
+read."""
 import numpy as np
 import pytest
 import torch
@@ -29,7 +47,6 @@ from dvlm_gen.device import DeviceModel, kv_buffers
 from gpu_util import assert_bf16_close, f64, ws_tensor
 
 pytestmark = pytest.mark.gpu
-DELTA = 0.1
 SMALL = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=1024, vocab=4096,
                       lm_scale=25.0, dtype="bf16")
 
@@ -88,20 +105,54 @@ class Fp8Setup:
         return m, s
 
 
+FP8_LAYER_REL = 0.08   # a layer on identical inputs
+FP8_DRIFT_REL = 0.12   # downstream of a quantised layer
+
+
+def _assert_rel(got, want, bar, what):
+    got, want = np.asarray(got, dtype=np.float64), np.asarray(want, dtype=np.float64)
+    err, mag = float(np.max(np.abs(got - want))), float(np.max(np.abs(want)))
+    assert err <= bar * mag, (what, err, mag)
+
+
 def test_fp8_prefill_and_forward_match_oracle(cuda):
     st = Fp8Setup(cuda, 5)
     L, seed = st.prefill()
     m, s = st.oracle()
     assert L == m.L == 48
     for l in range(SMALL.n_layers):
-        assert_bf16_close(f64(st.kc[l, 0, :, :L]), m.K[l][:, :L], 2e-2, f"K layer {l}")
-        assert_bf16_close(f64(st.vc[l, 0, :, :, :L]).transpose(0, 2, 1), m.V[l][:, :L], 2e-2, f"V layer {l}")
+        k_gpu, v_gpu = f64(st.kc[l, 0, :, :L]), f64(st.vc[l, 0, :, :, :L]).transpose(0, 2, 1)
+        if l == 0:   # codes from the identical context rows
+            assert_bf16_close(k_gpu, m.K[l][:, :L], 2e-2, f"K layer {l}")
+            assert_bf16_close(v_gpu, m.V[l][:, :L], 2e-2, f"V layer {l}")
+        _assert_rel(k_gpu, m.K[l][:, :L], FP8_DRIFT_REL, f"K layer {l}")
+        _assert_rel(v_gpu, m.V[l][:, :L], FP8_DRIFT_REL, f"V layer {l}")
     toks = [seed] + [SMALL.mask_id] * 15
+    tok_d = torch.tensor(toks, dtype=torch.int32, device=cuda)
     x = torch.zeros((16, SMALL.hidden), dtype=torch.bfloat16, device=cuda)
-    st.eng.forward(16, 0, SMALL.n_layers, tokens=torch.tensor(toks, dtype=torch.int32, device=cuda), x_out=x)
+    st.eng.forward(16, 0, SMALL.n_layers, tokens=tok_d, x_out=x)
     st.eng.check()
     xo = m.forward(m.embed(toks), L, n_clean=0)
-    assert_bf16_close(f64(x), xo, 2e-2, "noisy forward")
+    _assert_rel(f64(x), xo, FP8_DRIFT_REL, "noisy forward")
+    # layer by layer on identical inputs: the oracle's layer gets the GPU's
+    # input rows and the GPU's prefilled cache of that layer
+    x_in = None
+    for l in range(SMALL.n_layers):
+        if l == 0:
+            st.eng.forward(16, 0, 1, tokens=tok_d, first_layer=0, x_out=x)
+            xin64 = m.embed(toks)
+        else:
+            st.eng.forward(16, 0, 1, x_in=x_in, first_layer=l, x_out=x)
+            xin64 = f64(x_in)
+        st.eng.check()
+        m.K[l][:, :L] = f64(st.kc[l, 0, :, :L])
+        m.V[l][:, :L] = f64(st.vc[l, 0, :, :, :L]).transpose(0, 2, 1)
+        xo = m.layer(l, xin64, L, 0)
+        _assert_rel(f64(x), xo, FP8_LAYER_REL, f"layer {l} output")
+        assert_bf16_close(f64(st.kc[l, 0, :, L:L + 16]), m.K[l][:, L:L + 16], 2e-2, f"layer {l} block K")
+        assert_bf16_close(f64(st.vc[l, 0, :, :, L:L + 16]).transpose(0, 2, 1), m.V[l][:, L:L + 16], 2e-2,
+                          f"layer {l} block V")
+        x_in = x.clone()
     st.eng.close()
 
 
@@ -120,10 +171,13 @@ def test_fp8_threshold_decode_engine_path(cuda, seed):
     st.eng.set_trace(None, None)
     recs = parse_trace(buf.cpu().numpy(), int(cnt[0].item()), rb, SMALL.hidden, True)
     m, s = st.oracle()
-    rp = Replay(m, s, 16, 0.9, decide="gpu", hidden_check=lambda a, b, w: assert_bf16_close(a, b, 2e-2, w),
-                secondary=DELTA, seed_bar=DELTA)
+    # decisions on the GPU's rows only: the oracle's own rows of a W8A8 model
+    # drift too far for a bar on their decisions (same CPU model: p1 up to
+    # 0.40 apart, top-1 different in up to 5 of 16 rows)
+    rp = Replay(m, s, 16, 0.9, decide="gpu", hidden_check=lambda a, b, w: _assert_rel(a, b, FP8_DRIFT_REL, w),
+                secondary=None, seed_bar=None)
     assert rp.threshold(recs, 32) == out.cpu().numpy().tolist()
     assert rp._next == len(recs) == stats.nfe
-    assert rp.t.ids_exact > 0 and rp.t.commits_exact > 0 and rp.t.secondary_checked > 0, rp.t
+    assert rp.t.ids_exact > 0 and rp.t.commits_exact > 0, rp.t
     print(f"fp8 seed {seed}: {rp.t}")
     st.eng.close()
