@@ -865,14 +865,18 @@ static cudaError_t traced_forward(dvlm_engine* e, FwdSpec f, int kind, const int
   trace_begin_kernel<<<1, 32, 0, s>>>(e->trace_buf, rb, e->trace_cap, e->trace_cnt, kind, e->d_len, f.n_rows,
                                       f.n_clean, f.lm ? f.lma.R : 0, tokens, masked);
   DVLM_CK(cudaGetLastError());
+  // the LM head's per-row top-1 ids and probabilities are recorded from
+  // where the forward puts them (a routing pass keeps them as anchors), or
+  // from the trace's own buffers when the forward has no use for them
   if (f.lm) {
-    f.lma.top1_id = e->tr_top1;
-    f.lma.top1_prob = e->tr_p1;
+    if (!f.lma.top1_id) f.lma.top1_id = e->tr_top1;
+    if (!f.lma.top1_prob) f.lma.top1_prob = e->tr_p1;
   }
   DVLM_CK(engine_forward(e, f, s));
   const size_t xb = static_cast<size_t>(f.n_rows) * e->m.hidden * (e->bf16 ? 2 : 4);
   trace_end_kernel<<<1, 256, 0, s>>>(e->trace_buf, rb, e->trace_cap, e->trace_cnt, e->d_len, e->d_seed, f.n_rows,
-                                     f.lm ? f.lma.R : 0, e->tr_top1, e->tr_p1, tokens, masked,
+                                     f.lm ? f.lma.R : 0, f.lm ? f.lma.top1_id : e->tr_top1,
+                                     f.lm ? f.lma.top1_prob : e->tr_p1, tokens, masked,
                                      static_cast<const uint8_t*>(e->x), xb);
   return cudaGetLastError();
 }

@@ -604,6 +604,22 @@ constexpr int kChainThreads = 256;
 constexpr int kChainStages = 12;
 constexpr int kChainNT = 16;
 
+// A phase's stream-K schedule: its units over min(P, units) CTAs (a CTA with
+// an empty range between the CTAs of a split tile would be counted as one of
+// its contributors); CTAs past those have no units in the phase.
+__device__ __forceinline__ SkSched chain_sched(const ChainPhase& ph, int P) {
+  const long long units = static_cast<long long>(ph.n_tiles) * ph.kb;
+  return SkSched{ph.n_tiles, ph.kb, static_cast<int>(units < P ? units : P)};
+}
+__device__ __forceinline__ void chain_range(const SkSched& sc, long long& u0, long long& u1) {
+  if (static_cast<int>(blockIdx.x) >= sc.P) {
+    u0 = u1 = 0;
+    return;
+  }
+  u0 = sc.begin(blockIdx.x);
+  u1 = sc.begin(blockIdx.x + 1);
+}
+
 template <int STAGES>
 __device__ __forceinline__ void chain_load_a(const ChainArgs& ca, uint8_t* sA, uint64_t* full, uint64_t* empty,
                                              volatile int* abort_flag) {
@@ -612,8 +628,9 @@ __device__ __forceinline__ void chain_load_a(const ChainArgs& ca, uint8_t* sA, u
   long long i = 0;
   for (int p = 0; p < ca.n_phases; ++p) {
     const ChainPhase& ph = ca.ph[p];
-    const SkSched sc{ph.n_tiles, ph.kb, ca.P};
-    const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+    const SkSched sc = chain_sched(ph, ca.P);
+    long long u0, u1;
+    chain_range(sc, u0, u1);
     const bool split = ph.ea.epi == EPI_SWIGLU;
     for (long long u = u0; u < u1; ++u, ++i) {
       const int s = static_cast<int>(i % STAGES);
@@ -645,8 +662,9 @@ __device__ __forceinline__ void chain_load_b(const ChainArgs& ca, uint8_t* sB, u
       return;
     fence_proxy_async_global();
     const ChainPhase& ph = ca.ph[p];
-    const SkSched sc{ph.n_tiles, ph.kb, ca.P};
-    const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+    const SkSched sc = chain_sched(ph, ca.P);
+    long long u0, u1;
+    chain_range(sc, u0, u1);
     for (long long u = u0; u < u1; ++u, ++i) {
       const int s = static_cast<int>(i % STAGES);
       if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, ca.status, abort_flag)) return;
@@ -710,10 +728,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
       long long i_base = 0;
       int seg = 0;
       for (int p = 0; p < ca.n_phases; ++p) {
-        const SkSched sc{ca.ph[p].n_tiles, ca.ph[p].kb, ca.P};
-        if (!ws_mma_units<NT, STAGES, false>(sA, sB, full, empty, accf, acce, tmem, sc, sc.begin(blockIdx.x),
-                                             sc.begin(blockIdx.x + 1), ca.status, sabort, warp == 1 ? 0 : 1, 0,
-                                             i_base, seg))
+        const SkSched sc = chain_sched(ca.ph[p], ca.P);
+        long long u0, u1;
+        chain_range(sc, u0, u1);
+        if (!ws_mma_units<NT, STAGES, false>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ca.status, sabort,
+                                             warp == 1 ? 0 : 1, 0, i_base, seg))
           break;
       }
     }
@@ -746,8 +765,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
           }
           named_bar_sync(1, 128);
         }
-        const SkSched sc{ph.n_tiles, ph.kb, ca.P};
-        const long long u0 = sc.begin(blockIdx.x), u1 = sc.begin(blockIdx.x + 1);
+        const SkSched sc = chain_sched(ph, ca.P);
+        long long u0, u1;
+        chain_range(sc, u0, u1);
         if (ea.epi == EPI_QKV)
           ok = ws_epilogue_units<NT, EPI_QKV, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
                                                      nullptr, nullptr, sflag, sabort, gseg,

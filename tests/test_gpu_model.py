@@ -194,7 +194,7 @@ def test_every_layer_matches_oracle_on_identical_inputs(full):
         xo = m.layer(l, xin64, L0, 0)
         got = f64(x_out)
         worst.append((l, float(np.max(np.abs(got - xo)))))
-        assert_bf16_close(got, xo, 2e-2, f"layer {l} output")
+        assert_bf16_close(got, xo, 2e-2, f"layer {l} output", ulps=2)
         assert_bf16_close(f64(full["kc"][l, 0, :, L0:L0 + 16]), m.K[l][:, L0:L0 + 16], 2e-2, f"layer {l} K")
         assert_bf16_close(f64(full["vc"][l, 0, :, :, L0:L0 + 16]).transpose(0, 2, 1), m.V[l][:, L0:L0 + 16], 2e-2,
                           f"layer {l} V")
@@ -240,7 +240,7 @@ def test_persistent_chain_matches_oracle_per_layer(full):
             m.K[l][:, :L0] = f64(full["kc"][l, 0, :, :L0])
             m.V[l][:, :L0] = f64(full["vc"][l, 0, :, :, :L0]).transpose(0, 2, 1)
             xo = m.layer(l, xin64, L0, 0)
-            assert_bf16_close(f64(x_out), xo, 2e-2, f"chain layer {l} output")
+            assert_bf16_close(f64(x_out), xo, 2e-2, f"chain layer {l} output", ulps=2)
             assert_bf16_close(f64(full["kc"][l, 0, :, L0:L0 + 16]), m.K[l][:, L0:L0 + 16], 2e-2, f"chain layer {l} K")
             assert_bf16_close(f64(full["vc"][l, 0, :, :, L0:L0 + 16]).transpose(0, 2, 1), m.V[l][:, L0:L0 + 16],
                               2e-2, f"chain layer {l} V")
@@ -253,7 +253,8 @@ def test_persistent_chain_matches_oracle_per_layer(full):
             eng.forward(16, 0, 2, x_in=x_in, first_layer=17, x_out=x_out)
             eng.check()
             outs.append((f64(x_out), f64(full["kc"][18, 0, :, L0:L0 + 16])))
-        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, chain vs per-kernel")
+        # two layers: a flip in layer 17's output is carried through layer 18's two stores
+        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, chain vs per-kernel", ulps=3)
         assert_bf16_close(outs[1][1], outs[0][1], 2e-2, "layer 18 K, chain vs per-kernel")
     finally:
         eng.set_option("persistent", 0)
