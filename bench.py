@@ -560,6 +560,9 @@ def run_sweep(args, local):
         groups = nb * ((B + 15) // 16) * Hkv
         return max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
 
+    if args.sweep == "attn_long":
+        # the bandwidth case alone: 36 caches of 4096 slots in one launch
+        attn_case(BLOCK, 4096, dims.n_layers, [2])
     if args.sweep == "attn_decode":
         # the decode shape (one cache per launch) and the long batched case,
         # split counts around the automatic choice
@@ -729,7 +732,7 @@ def main():
     ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")
     ap.add_argument("--profile-forwards", type=int, default=0,
                     help="profiling case: run this many eager forwards after prefill and exit")
-    ap.add_argument("--sweep", choices=["attention", "attn_decode", "lmhead", "spec", "tiny", "all"], default=None,
+    ap.add_argument("--sweep", choices=["attention", "attn_decode", "attn_long", "lmhead", "spec", "tiny", "all"], default=None,
                     help="time the single-kernel configurations (one JSON line per case) instead of the decode")
     args = ap.parse_args()
     rank, world, local, pg = dist_setup()

@@ -40,6 +40,27 @@ __device__ __forceinline__ float fp8_row_scale(const GemmEpi& ea, bool split, in
   return ea.wscale[a_row_base + T * 128 + row];
 }
 
+// RMSNorm factors of the NT input rows from the producers' per-tile sums of
+// squares (ssq_in [n_ssq][NT]), run by the 128 epilogue threads: 128 / NT
+// partial sums per row with independent loads, then one thread per row adds
+// the partials in order.  sPart: 128 floats of scratch.
+template <int NT>
+__device__ __forceinline__ void ws_rms_factors(const GemmEpi& ea, int et, float* sR, float* sPart) {
+  constexpr int G = 128 / NT;
+  const int t = et % NT, g = et / NT;
+  float s = 0.f;
+  for (int q = g; q < ea.n_ssq; q += G) s += __ldcg(&ea.ssq_in[q * NT + t]);
+  sPart[g * NT + t] = s;
+  named_bar_sync(1, 128);
+  if (et < NT) {
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < G; ++k) tot += sPart[k * NT + et];
+    sR[et] = 1.0f / sqrtf(tot * ea.inv_h + ea.eps);
+  }
+  named_bar_sync(1, 128);
+}
+
 // The epilogue warps' work for the stream-K units [u0, u1) of one GEMM:
 // partial tiles stored for the CTAs that finish them, split tiles finished
 // (partials added in CTA order), the fused epilogue on every tile this CTA
@@ -69,6 +90,15 @@ __device__ __forceinline__ bool ws_epilogue_units(const SkSched& sc, long long u
     const bool whole = (u == t_begin) && (seg_end == t_end);
     const bool finisher = !whole && (u == t_begin);
     float o[NT];
+    // residual rows of the tile's columns, fetched before the accumulator is
+    // ready (independent loads; only this tile's epilogue writes them)
+    float xr[NT];
+    if (EPI == EPI_RESID && (whole || finisher)) {
+      const int col = T * 128 + row;
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        xr[t] = t < ea.n_rows ? __bfloat162float(__ldcg(ea.resid + static_cast<size_t>(t) * ea.resid_ld + col)) : 0.f;
+    }
     if (finisher) {
       const int pl = sc.cta_of(t_end - 1);
       if (et == 0) {
@@ -135,9 +165,8 @@ __device__ __forceinline__ bool ws_epilogue_units(const SkSched& sc, long long u
       for (int t = 0; t < NT; ++t) {
         sq[t] = 0.f;
         if (t < ea.n_rows) {
-          bf16* px = ea.resid + static_cast<size_t>(t) * ea.resid_ld + col;
-          const float xn = bf16_round_f(__bfloat162float(*px) + v[t]);
-          *px = __float2bfloat16_rn(xn);
+          const float xn = bf16_round_f(xr[t] + v[t]);
+          ea.resid[static_cast<size_t>(t) * ea.resid_ld + col] = __float2bfloat16_rn(xn);
           sq[t] = xn * xn;
         }
         sE[row * (NT + 1) + t] = sq[t];
@@ -290,14 +319,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     // Dependents may start only once this kernel's own inputs are complete,
     // so at most two kernels of the chain overlap (see ptx.cuh).
     if (et == 0) griddep_launch_dependents();
-    if (EPI != EPI_RESID) {
-      if (et < NT) {
-        float s = 0.f;
-        for (int p = 0; p < ea.n_ssq; ++p) s += ea.ssq_in[p * NT + et];
-        sR[et] = 1.0f / sqrtf(s * ea.inv_h + ea.eps);
-      }
-      named_bar_sync(1, 128);
-    }
+    if (EPI != EPI_RESID) ws_rms_factors<NT>(ea, et, sR, sE);
     if (FP8)
       fp8_quantize_activations<NT>(et, ea.q_src, ea.q_ld, ea.q_K, ea.n_rows, ea.rms_input ? sR : nullptr,
                                    ea.amax_in, ea.n_amax, kb_lo, kb_hi, sB, sAt, sQm, b_ready);
@@ -757,14 +779,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
         named_bar_sync(1, 128);  // sflag is read before the phase may reuse it
       }
       if (ok) {
-        if (ea.epi != EPI_RESID) {
-          if (et < NT) {
-            float sq = 0.f;
-            for (int q = 0; q < ea.n_ssq; ++q) sq += __ldcg(&ea.ssq_in[q * NT + et]);
-            sR[et] = 1.0f / sqrtf(sq * ea.inv_h + ea.eps);
-          }
-          named_bar_sync(1, 128);
-        }
+        if (ea.epi != EPI_RESID) ws_rms_factors<NT>(ea, et, sR, sE);
         const SkSched sc = chain_sched(ph, ca.P);
         long long u0, u1;
         chain_range(sc, u0, u1);

@@ -47,7 +47,9 @@ def assert_bf16_close(got, want, tol=2e-2, what="", ulps=1):
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     err = np.abs(got - want)
-    ulp = bf16_ulp(want)
+    # the larger of the two values' spacings: across a power of two the steps
+    # of a flip are those of the upper binade
+    ulp = bf16_ulp(np.maximum(np.abs(got), np.abs(want)))
     bad = np.argwhere(err > tol + ulps * ulp)
     detail = [(tuple(int(v) for v in i), float(got[tuple(i)]), float(want[tuple(i)]), float(err[tuple(i)]))
               for i in bad[:8]]
