@@ -160,9 +160,9 @@ def algorithmic_bytes(kind: str, dims, L: int, rows: int = 16, fp8: bool = False
         return 2 * w(I, H) + 2 * (rows * H + rows * I)
     if kind == "down_gemm":
         return w(H, I) + 2 * (rows * I + 2 * rows * H)
-    if kind == "gemm_chain":   # one per-layer launch: O-projection, gate/up, down, next layer's QKV
-        return sum(algorithmic_bytes(k, dims, L, rows, fp8) for k in ("oproj_gemm", "gateup_gemm", "down_gemm",
-                                                                       "qkv_gemm"))
+    if kind == "persistent_forward":   # every decoder layer of a forward in one launch
+        return dims.n_layers * sum(algorithmic_bytes(k, dims, L, rows, fp8)
+                                   for k in ("qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm"))
     if kind == "lm_head":
         return 2 * (V * H + rows * H)
     if kind == "attention":
@@ -180,7 +180,7 @@ TRAFFIC_SOURCES = {
     "oproj_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
     "gateup_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
     "down_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
-    "gemm_chain": _COMMON_SOURCES + ["gemm_ws.cu"],
+    "persistent_forward": _COMMON_SOURCES + ["gemm_ws.cu"],
     "lm_head": _COMMON_SOURCES + ["lmhead.cu", "finalize.cuh"],
     "attention": _COMMON_SOURCES + ["attn.cu"],
 }
@@ -412,8 +412,6 @@ def run_ours(args, rank, world, local, pg):
     for k, (ms, cnt) in prof.items():
         if cnt:
             b = algorithmic_bytes(k, dims, L0, fp8=fp8)
-            if k == "gemm_chain":   # n_layers chains' worth of products over n_layers + 1 launches
-                b = b * dims.n_layers / cnt
             per[k] = {"ms_per_launch": ms / cnt, "launches": cnt, "gbs": b / (ms / cnt * 1e-3) / 1e9,
                       "bytes_per_launch": b}
     dom = max((k for k in per if k != "embed"), key=lambda k: per[k]["ms_per_launch"] * per[k]["launches"])

@@ -365,7 +365,7 @@ class Engine:
                "dvlm_engine_set_trace")
 
     KERNEL_KINDS = ("embed", "qkv_gemm", "attention", "oproj_gemm", "gateup_gemm", "down_gemm", "lm_head",
-                    "gemm_chain")
+                    "persistent_forward")
 
     def profile_forward(self, tokens, n_rows: int, n_clean: int, *, masked=None, with_lm_head=True,
                         stream=None) -> dict:

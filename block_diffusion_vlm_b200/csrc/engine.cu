@@ -109,7 +109,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->ssq = c.take<float>(((H / 128) * 16 + 1) * kNT * 4);
   e->gpart = c.take<float>(gemm_ws_part_bytes(kNT, 2 * P));  // up to two CTAs per SM
   e->gcnt_stride = num_tiles_max(m);
-  e->gcnt = c.take<int>(static_cast<size_t>(e->gcnt_stride) * kMaxChainPhases * 4);
+  e->gcnt = c.take<int>(static_cast<size_t>(e->gcnt_stride) * 4 * 4);  // one block per GEMM kind of the persistent forward
   e->chain_bar = c.take<int>(2 * 4);
   e->lpart = c.take<float>(static_cast<size_t>(P) * kNT * 128 * 4);
   e->lcnt = c.take<int>(((m.vocab + 127) / 128) * 4);
@@ -137,6 +137,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
   e->stage_out = c.take<int32_t>(static_cast<size_t>(e->Lmax) * 4);
   if (e->fp8) e->amax_act = c.take<float>(static_cast<size_t>(I / 64) * kNT * 4);
   if (e->bf16) e->attn_scratch = c.take<void>(attn_split_scratch_bytes(m.n_kv_heads, kMaxAttnSplit));
+  if (e->bf16 && !e->fp8) e->fwd_att = c.take<void>(fwd_attn_scratch_bytes(m.n_kv_heads, e->Lmax));
   if (e->bf16 && !e->fp8 && e->max_ctx > 0) {
     const size_t C = static_cast<size_t>(e->max_ctx);
     e->px = c.take<void>(C * H * 2);
@@ -229,35 +230,26 @@ static void fill_lm_scratch(dvlm_engine* e, LmArgs& a) {
     if (err__ != cudaSuccess) return err__;   \
   } while (0)
 
-// Persistent GEMM chain (gemm_chain): bf16 weights, 128-wide heads, feature
-// counts in whole tiles, and one resident CTA on every SM.
-static bool chain_supported(dvlm_engine* e) {
+// Persistent forward (one launch for all layers): bf16 weights, 128-wide
+// heads, 8 query heads per KV head, feature counts in whole tiles, and one
+// resident CTA on every SM.
+static bool persistent_supported(dvlm_engine* e) {
   const dvlm_model& m = e->m;
   return e->bf16 && !e->fp8 && m.head_dim == 128 && m.hidden % 128 == 0 && m.inter % 64 == 0 &&
-         (m.n_q_heads * m.head_dim) % 64 == 0 && e->sm >= 1 && e->sm <= gemm_chain_max_ctas();
+         m.n_q_heads == 8 * m.n_kv_heads && e->fwd_att && e->sm >= 1 && e->sm <= fwd_persistent_max_ctas();
 }
 
-static ChainArgs chain_args(dvlm_engine* e) {
-  ChainArgs ca{};
-  ca.P = e->sm;
-  ca.bar = e->chain_bar;
-  ca.status = e->d_status;
-  return ca;
-}
-
-// Appends a phase; each phase counts its split tiles in its own block of gcnt.
-static void chain_push(dvlm_engine* e, ChainArgs& ca, const CUtensorMap& a, const CUtensorMap& a2,
-                       const CUtensorMap& b, int n_tiles, int kb, int a_row_base, const GemmEpi& ea) {
-  ChainPhase& ph = ca.ph[ca.n_phases];
+static ChainPhase chain_phase(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, int n_tiles, int kb,
+                              const GemmEpi& ea, int* cnt) {
+  ChainPhase ph{};
   ph.mapA = a;
   ph.mapA2 = a2;
   ph.mapB = b;
   ph.ea = ea;
-  ph.ea.cnt = e->gcnt + static_cast<size_t>(ca.n_phases) * e->gcnt_stride;
+  ph.ea.cnt = cnt;
   ph.n_tiles = n_tiles;
   ph.kb = kb;
-  ph.a_row_base = a_row_base;
-  ++ca.n_phases;
+  return ph;
 }
 
 static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
@@ -315,38 +307,70 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     ea.block_table = e->block_table;
     ea.n_pages = e->n_pages;
   }
-  // persistent chain: [QKV(first layer)], then per layer attention followed
-  // by one launch of [O, gate/up, down, QKV(next layer)]
-  const bool chain = e->chain && !e->fp8;
-  const GemmEpi base = ea;
-  auto qkv_epi = [&](int layer) {
+  // the whole forward as one persistent launch (contiguous cache, no hidden
+  // slots): first layer's QKV, then per layer attention, merge, O, gate/up,
+  // down and the next layer's QKV
+  const bool persistent = e->chain && !e->fp8 && !e->paged && f.hide == 0;
+  if (persistent) {
+    const GemmEpi base = ea;
+    FwdProgram fp{};
     GemmEpi q = base;
     q.epi = EPI_QKV;
     q.n_ssq = H / 128;
     q.out = static_cast<bf16*>(e->q);
     q.out_ld = Hq * D;
-    q.kcache = static_cast<bf16*>(e->kc) + layer * kv_layer;
-    q.vcache = static_cast<bf16*>(e->vc) + layer * kv_layer;
-    return q;
-  };
-  for (int l = f.layer0; l < l1; ++l) {
-    if (chain && l == f.layer0) {
-      ChainArgs ca = chain_args(e);
-      chain_push(e, ca, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, l * qkv_rows, qkv_epi(l));
-      T0(K_CHAIN);
-      DVLM_CK(launch_gemm_chain(ca, pdl, s));
-      T1(K_CHAIN);
-    }
+    q.kcache = static_cast<bf16*>(e->kc);
+    q.vcache = static_cast<bf16*>(e->vc);
+    GemmEpi o = base;  // O-projection and down: residual add + sums of squares
+    o.epi = EPI_RESID;
+    o.resid = x;
+    o.resid_ld = H;
+    o.ssq_out = e->ssq;
+    GemmEpi g = base;
+    g.epi = EPI_SWIGLU;
+    g.n_ssq = H / 128;
+    g.out = static_cast<bf16*>(e->act);
+    g.out_ld = I;
+    const int cs = e->gcnt_stride;
+    fp.qkv = chain_phase(e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, q, e->gcnt);
+    fp.o = chain_phase(e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, o, e->gcnt + cs);
+    fp.gu = chain_phase(e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, g, e->gcnt + 2 * cs);
+    fp.down = chain_phase(e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, o, e->gcnt + 3 * cs);
+    fp.qkv_rows = qkv_rows;
+    fp.H = H;
+    fp.I = I;
+    fp.kv_layer = kv_layer;
+    fp.mapQ = e->tm_q;
+    fp.mapK = e->tm_k;
+    fp.mapV = e->tm_v;
+    fp.Hq = Hq;
+    fp.Hkv = Hkv;
+    fp.Lmax = e->Lmax;
+    fp.n_clean = f.n_clean;
+    fp.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    fp.apart = static_cast<float*>(e->fwd_att);
+    fp.n_chunks_max = (e->Lmax + 63) / 64;
+    fp.aml = reinterpret_cast<float2*>(static_cast<uint8_t*>(e->fwd_att) +
+                                       (static_cast<size_t>(Hkv) * fp.n_chunks_max * 128 * 128 * 4 + 255) / 256 * 256);
+    fp.attn_o = static_cast<bf16*>(e->attn_o);
+    fp.layer0 = f.layer0;
+    fp.n_layers = l1 - f.layer0;
+    fp.bar = e->chain_bar;
+    fp.status = e->d_status;
+    T0(K_CHAIN);
+    DVLM_CK(launch_fwd_persistent(fp, e->sm, pdl, s));
+    T1(K_CHAIN);
+    n_ssq = H / 128;
+  }
+  for (int l = f.layer0; l < l1 && !persistent; ++l) {
     ea.epi = EPI_QKV;
     ea.n_ssq = n_ssq;
     ea.out = static_cast<bf16*>(e->q);
     ea.out_ld = Hq * D;
     ea.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
     ea.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
-    if (!chain) T0(K_QKV);
-    if (chain) {
-      // written by the previous chain launch
-    } else if (e->fp8) {  // W8A8 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]
+    T0(K_QKV);
+    if (e->fp8) {  // W8A8 [Fast-dVLM technical overview (ocdem.com), section 2.3.2]
       ea.q_src = x;
       ea.q_ld = H;
       ea.q_K = H;
@@ -365,7 +389,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
       DVLM_CK(launch_gemm_ws(kNT, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64,
                              ws_ctas(e, (qkv_rows / 128) * (H / 64)), l * qkv_rows, ea, pdl, s, 5));
     }
-    if (!chain) T1(K_QKV);
+    T1(K_QKV);
     AttnArgs aa{};
     aa.n_rows = f.n_rows;
     aa.n_clean = f.n_clean;
@@ -392,30 +416,6 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     else
       DVLM_CK(launch_attn_bf16(e->tm_q, mk, mv, aa, pdl, s, e->attn_cs));
     T1(K_ATTN);
-    if (chain) {
-      ChainArgs ca = chain_args(e);
-      GemmEpi o = base;  // O-projection and down: residual add + sums of squares
-      o.epi = EPI_RESID;
-      o.resid = x;
-      o.resid_ld = H;
-      o.ssq_out = e->ssq;
-      GemmEpi g = base;
-      g.epi = EPI_SWIGLU;
-      g.n_ssq = H / 128;
-      g.out = static_cast<bf16*>(e->act);
-      g.out_ld = I;
-      chain_push(e, ca, e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, l * H, o);
-      chain_push(e, ca, e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, l * I, g);
-      chain_push(e, ca, e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, l * H, o);
-      if (l + 1 < l1)
-        chain_push(e, ca, e->tm_wqkv, e->tm_wqkv, e->tm_x, qkv_rows / 128, H / 64, (l + 1) * qkv_rows,
-                   qkv_epi(l + 1));
-      T0(K_CHAIN);
-      DVLM_CK(launch_gemm_chain(ca, pdl, s));
-      T1(K_CHAIN);
-      n_ssq = H / 128;
-      continue;
-    }
     ea.epi = EPI_RESID;
     ea.resid = x;
     ea.resid_ld = H;
@@ -1228,7 +1228,7 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
     e->attn_split = v;
   } else if (n == "persistent") {
     if (v != 0 && v != 1) return DVLM_ERR_SHAPE;
-    if (v && !chain_supported(e)) return DVLM_ERR_UNSUPPORTED;
+    if (v && !persistent_supported(e)) return DVLM_ERR_UNSUPPORTED;
     e->chain = v != 0;
   } else if (n == "prefill_gemm") {
     if (v != 0 && v != 1) return DVLM_ERR_SHAPE;

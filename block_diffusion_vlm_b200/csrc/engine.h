@@ -107,8 +107,9 @@ struct dvlm_engine {
   float* gpart = nullptr;   // GEMM split scratch
   int* gcnt = nullptr;      // split-tile counters, one block of gcnt_stride per chain phase
   int gcnt_stride = 0;
-  int* chain_bar = nullptr; // persistent chain: barrier and exit counters
-  bool chain = false;       // post-attention GEMMs + next QKV as one persistent launch
+  int* chain_bar = nullptr; // persistent forward: barrier and exit counters
+  void* fwd_att = nullptr;  // persistent forward: attention partials and (max, sum) per 64-key chunk
+  bool chain = false;       // the whole forward as one persistent launch (option "persistent")
   float* lpart = nullptr;   // LM head scratch
   int* lcnt = nullptr;
   float* lrec = nullptr;

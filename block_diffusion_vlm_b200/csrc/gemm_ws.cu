@@ -30,7 +30,7 @@ struct GemmSmem {
   static constexpr int kR = kE + 128 * (NT + 1) * 4;
   static constexpr int kAt = kR + 32 * 4;  // fp8: token scales [32], quantisation multipliers [32], amax [32]
   static constexpr int kBar = kAt + 3 * 32 * 4;
-  static constexpr int kMisc = kBar + (2 * STAGES + 5) * 8;
+  static constexpr int kMisc = kBar + (2 * STAGES + 8) * 8;  // + the persistent forward's attention barriers
   static constexpr int kTotal = kMisc + 64 + 1024;  // + alignment slack
 };
 
@@ -602,29 +602,78 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 }
 
 // ---------------------------------------------------------------------------
-// Persistent GEMM chain.  The products that follow a layer's attention --
-// O-projection (+ residual), gate/up (SwiGLU), down (+ residual) -- and the
-// next layer's QKV run as consecutive stream-K phases of one launch on every
-// SM, instead of one kernel each.  A phase reads what the previous phase's
-// epilogues wrote (all CTAs), so a grid barrier separates the phases: every
-// CTA bumps a counter after its phase epilogue, and phase p's inputs are
-// ready once the counter reaches p * P.  The weight stream never waits for
-// it: the A loader runs through the phases back to back, so while the last
-// split tiles of one phase are being reduced and finished, the next phase's
-// weight tiles already fill the pipeline stages.  Only the activation tiles
-// (2 KB a stage, L2-resident) wait for the barrier, issued by a loader warp
-// of their own that polls it.  One A loader arrival per stage arms the
-// stage's full barrier with A + B bytes (a B copy may complete before that
+// Persistent forward.  All decoder layers of one forward run in a single
+// launch on every SM, phase by phase: the first layer's QKV, then for each
+// layer l the attention partials, the attention merge, the O-projection
+// (+ residual), gate/up (SwiGLU), down (+ residual) and layer l+1's QKV.  A
+// phase reads what the previous phase's epilogues wrote (all CTAs), so a
+// grid barrier separates the phases: every CTA bumps a counter after its
+// phase epilogue, and phase p's inputs are ready once the counter reaches
+// p * gridDim.x.
+//
+// The weight stream never waits for a barrier: the A loader runs through the
+// phases back to back, so while one phase's split tiles are being reduced,
+// or the merge runs, or attention computes, the next phases' weight tiles
+// are already filling the pipeline stages.  Loads that depend on a phase's
+// inputs (a GEMM's activation tiles; attention's query, key and value
+// tiles) come from a loader warp of their own that waits for the barrier.
+// One A-loader arrival per stage arms the stage's full barrier with all of
+// the stage's bytes (a copy from the other loader may complete before that
 // arrival; the phase still needs the arrival).
 //
-// Roles (256 threads): warp 0 A loader, warps 1 and 6 MMA issuers, warps
-// 2..5 epilogue, warp 7 B loader.  All P CTAs must be resident together
-// (one per SM; the launcher checks the occupancy), and every wait is
-// bounded: a CTA that gives up records DVLM_ERR_TIMEOUT and still arrives
-// at the remaining barriers, so the others do not wait on it.
-constexpr int kChainThreads = 256;
-constexpr int kChainStages = 12;
-constexpr int kChainNT = 16;
+// Attention [Fast-dVLM technical overview (ocdem.com), section 2.2.1:
+// N2N / N2C / C2C visibility]: units of (KV head g, 64-key chunk c), dealt
+// round robin over the CTAs.  A unit takes five pipeline stages -- the
+// query tile (8 heads x 16 rows = 128 rows, two 64-wide halves), the
+// chunk's keys, its values (transposed) and P -- and leaves, for each row,
+// the chunk's unnormalised output O_c = sum_k p_k v_k with p_k = 2^(s_k - m_c)
+// (P in bf16; l_c sums the same bf16 values), the row max m_c and l_c.  The
+// merge phase combines a row's chunks in chunk order:
+// out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.  A row's arithmetic
+// depends only on its own query and keys (chunks by absolute key position),
+// so a 1-row pass and a 16-row pass give bitwise the same rows.
+//
+// Roles (256 threads): warp 0 A loader, warps 1 and 6 MMA issuers (warp 1
+// issues attention too), warps 2..5 epilogue / softmax / merge, warp 7 B
+// loader.  All CTAs must be resident at once (one per SM; the launcher checks
+// the occupancy), and every wait is bounded: a CTA that gives up records
+// DVLM_ERR_TIMEOUT and still arrives at the remaining barriers.
+constexpr int kFwdThreads = 256;
+constexpr int kFwdStages = 12;
+constexpr int kFwdNT = 16;
+constexpr int kAttKeys = 64;   // keys per attention unit
+constexpr int kAttSlots = 5;   // stages of an attention unit: Q (2 halves), K, V^T, P
+constexpr uint32_t kAttIdescS = idesc_bf16_f32(128, kAttKeys);
+constexpr uint32_t kAttIdescO = idesc_bf16_f32(128, 128);
+constexpr int kFwdTmem = 256;  // GEMM accumulators [0, 64), S [64, 128), O [128, 256)
+constexpr uint32_t kTmemS = 64, kTmemO = 128;
+
+enum FwdKind { FK_QKV = 0, FK_ATT, FK_MERGE, FK_O, FK_GU, FK_DOWN };
+
+// Kind and layer of phase p.
+__device__ __forceinline__ int fwd_kind(const FwdProgram& fp, int p, int& layer) {
+  if (p == 0) {
+    layer = fp.layer0;
+    return FK_QKV;
+  }
+  const int q = p - 1, r = q % 6;
+  layer = fp.layer0 + q / 6 + (r == 5 ? 1 : 0);
+  return r == 0 ? FK_ATT : r == 1 ? FK_MERGE : r == 2 ? FK_O : r == 3 ? FK_GU : r == 4 ? FK_DOWN : FK_QKV;
+}
+__device__ __forceinline__ const ChainPhase& fwd_gemm(const FwdProgram& fp, int kind) {
+  return kind == FK_QKV ? fp.qkv : kind == FK_O ? fp.o : kind == FK_GU ? fp.gu : fp.down;
+}
+__device__ __forceinline__ int fwd_row_base(const FwdProgram& fp, int kind, int layer) {
+  return layer * (kind == FK_QKV ? fp.qkv_rows : kind == FK_GU ? fp.I : fp.H);
+}
+// Cache length of the forward (the previous kernels have completed).
+__device__ __forceinline__ int fwd_cache_len(const FwdProgram& fp) {
+  griddep_wait();
+  return fp.qkv.ea.d_len ? *fp.qkv.ea.d_len : fp.qkv.ea.L_static;
+}
+__device__ __forceinline__ int att_chunks(const FwdProgram& fp, int L) {
+  return (L + fp.qkv.ea.n_rows + kAttKeys - 1) / kAttKeys;
+}
 
 // A phase's stream-K schedule: its units over min(P, units) CTAs (a CTA with
 // an empty range between the CTAs of a split tile would be counted as one of
@@ -643,63 +692,312 @@ __device__ __forceinline__ void chain_range(const SkSched& sc, long long& u0, lo
 }
 
 template <int STAGES>
-__device__ __forceinline__ void chain_load_a(const ChainArgs& ca, uint8_t* sA, uint64_t* full, uint64_t* empty,
-                                             volatile int* abort_flag) {
-  constexpr int B_BYTES = kChainNT * 128;
+__device__ __forceinline__ void fwd_load_a(const FwdProgram& fp, uint8_t* sA, uint64_t* full, uint64_t* empty,
+                                           volatile int* abort_flag) {
+  constexpr int B_BYTES = kFwdNT * 128;
   const uint64_t pol_w = l2_policy_evict_first();
+  const int n_phases = 6 * fp.n_layers;
   long long i = 0;
-  for (int p = 0; p < ca.n_phases; ++p) {
-    const ChainPhase& ph = ca.ph[p];
-    const SkSched sc = chain_sched(ph, ca.P);
+  int L = -1;
+  // the next stage, once its previous contents are consumed; arms its full
+  // barrier for `bytes` (0: a plain arrival, the stage P of attention)
+  auto take = [&](int bytes) -> int {
+    const int s = static_cast<int>(i % STAGES);
+    if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, fp.status, abort_flag)) return -1;
+    if (bytes)
+      mbar_arrive_expect_tx(&full[s], bytes);
+    else
+      mbar_arrive(&full[s]);
+    ++i;
+    return s;
+  };
+  for (int p = 0; p < n_phases; ++p) {
+    int layer;
+    const int kind = fwd_kind(fp, p, layer);
+    if (kind == FK_MERGE) continue;
+    if (kind == FK_ATT) {
+      if (L < 0) L = fwd_cache_len(fp);
+      const int n_units = fp.Hkv * att_chunks(fp, L);
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x)
+        for (int j = 0; j < kAttSlots; ++j)
+          if (take(j < kAttSlots - 1 ? kATileBytes : 0) < 0) return;
+      continue;
+    }
+    const ChainPhase& ph = fwd_gemm(fp, kind);
+    const int base = fwd_row_base(fp, kind, layer);
+    const SkSched sc = chain_sched(ph, gridDim.x);
     long long u0, u1;
     chain_range(sc, u0, u1);
-    const bool split = ph.ea.epi == EPI_SWIGLU;
-    for (long long u = u0; u < u1; ++u, ++i) {
-      const int s = static_cast<int>(i % STAGES);
-      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, ca.status, abort_flag)) return;
-      mbar_arrive_expect_tx(&full[s], kATileBytes + B_BYTES);
+    const bool split = kind == FK_GU;
+    for (long long u = u0; u < u1; ++u) {
+      const int s = take(kATileBytes + B_BYTES);
+      if (s < 0) return;
       const int T = static_cast<int>(u / sc.kb), kk = static_cast<int>(u % sc.kb);
       if (split) {
-        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, ph.a_row_base + T * 64, pol_w);
-        tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, &ph.mapA2, &full[s], kk * 64, ph.a_row_base + T * 64,
-                    pol_w);
+        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, base + T * 64, pol_w);
+        tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, &ph.mapA2, &full[s], kk * 64, base + T * 64, pol_w);
       } else {
-        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, ph.a_row_base + T * 128, pol_w);
+        tma_load_2d(sA + s * kATileBytes, &ph.mapA, &full[s], kk * 64, base + T * 128, pol_w);
       }
     }
   }
 }
 
 template <int STAGES>
-__device__ __forceinline__ void chain_load_b(const ChainArgs& ca, uint8_t* sB, uint64_t* full, uint64_t* empty,
-                                             volatile int* abort_flag) {
-  constexpr int B_BYTES = kChainNT * 128;
+__device__ __forceinline__ void fwd_load_b(const FwdProgram& fp, uint8_t* sA, uint8_t* sB, uint64_t* full,
+                                           uint64_t* empty, volatile int* abort_flag) {
+  constexpr int B_BYTES = kFwdNT * 128;
   const uint64_t pol_x = l2_policy_evict_last();
+  const int n_phases = 6 * fp.n_layers;
   long long i = 0;
-  for (int p = 0; p < ca.n_phases; ++p) {
+  int L = -1;
+  auto next = [&]() -> int {  // the next stage, once its previous contents are consumed
+    const int s = static_cast<int>(i % STAGES);
+    if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, fp.status, abort_flag)) return -1;
+    ++i;
+    return s;
+  };
+  for (int p = 0; p < n_phases; ++p) {
+    int layer;
+    const int kind = fwd_kind(fp, p, layer);
     // inputs of phase p: the kernel before this one (p = 0), else every CTA's phase p-1
     if (p == 0)
       griddep_wait();
-    else if (!wait_counter(ca.bar, p * ca.P, ca.status, abort_flag))
+    else if (!wait_counter(fp.bar, p * static_cast<int>(gridDim.x), fp.status, abort_flag))
       return;
     fence_proxy_async_global();
-    const ChainPhase& ph = ca.ph[p];
-    const SkSched sc = chain_sched(ph, ca.P);
+    if (kind == FK_MERGE) continue;
+    if (kind == FK_ATT) {
+      if (L < 0) L = fwd_cache_len(fp);
+      const int n_chunks = att_chunks(fp, L);
+      const int n_units = fp.Hkv * n_chunks;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int g = u / n_chunks, c = u % n_chunks;
+        const int entry = layer * fp.Hkv + g;  // (layer, KV head) of the cache
+        for (int j = 0; j < 2; ++j) {          // query halves: 16 rows x 8 heads x 64
+          const int s = next();
+          if (s < 0) return;
+          tma_load_3d(sA + s * kATileBytes, &fp.mapQ, &full[s], j * 64, g * 8, 0, pol_x);
+        }
+        int s = next();  // keys of the chunk, two 64-wide halves
+        if (s < 0) return;
+        const int krow = entry * fp.Lmax + c * kAttKeys;
+        tma_load_2d(sA + s * kATileBytes, &fp.mapK, &full[s], 0, krow, pol_x);
+        tma_load_2d(sA + s * kATileBytes + kATileBytes / 2, &fp.mapK, &full[s], 64, krow, pol_x);
+        s = next();  // values, transposed: 128 rows (d) x 64 keys
+        if (s < 0) return;
+        tma_load_2d(sA + s * kATileBytes, &fp.mapV, &full[s], c * kAttKeys, entry * 128, pol_x);
+        if (next() < 0) return;  // P: written by the softmax warps
+      }
+      continue;
+    }
+    const ChainPhase& ph = fwd_gemm(fp, kind);
+    const SkSched sc = chain_sched(ph, gridDim.x);
     long long u0, u1;
     chain_range(sc, u0, u1);
-    for (long long u = u0; u < u1; ++u, ++i) {
-      const int s = static_cast<int>(i % STAGES);
-      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, ca.status, abort_flag)) return;
+    for (long long u = u0; u < u1; ++u) {
+      const int s = next();
+      if (s < 0) return;
       tma_load_2d(sB + s * B_BYTES, &ph.mapB, &full[s], static_cast<int>(u % sc.kb) * 64, 0, pol_x);
     }
   }
 }
 
+// Attention MMAs of one unit whose stages start at pipeline index iq:
+// S = Q K^T into TMEM columns [64, 128), then O = P V^T into [128, 256).
 template <int STAGES>
-__global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __grid_constant__ ChainArgs ca) {
-  constexpr int NT = kChainNT;
+__device__ __forceinline__ bool fwd_att_mma(const FwdProgram& fp, uint8_t* sA, uint64_t* full, uint64_t* empty,
+                                            uint64_t* att, uint32_t tmem, long long iq, int au,
+                                            volatile int* abort_flag) {
+  uint64_t* s_full = att;
+  uint64_t* p_full = att + 1;
+  uint64_t* o_full = att + 2;
+  uint64_t* att_free = att + 3;
+  auto st = [&](int j) { return static_cast<int>((iq + j) % STAGES); };
+  auto par = [&](int j) { return static_cast<uint32_t>(((iq + j) / STAGES) & 1); };
+  if (au >= 1 && !mbar_wait(att_free, (au - 1) & 1, fp.status, abort_flag)) return false;
+  for (int j = 0; j < 3; ++j)
+    if (!mbar_wait(&full[st(j)], par(j), fp.status, abort_flag)) return false;
+  tc_fence_after();
+  const uint32_t q0 = smem_u32(sA + st(0) * kATileBytes), q1 = smem_u32(sA + st(1) * kATileBytes);
+  const uint32_t kb = smem_u32(sA + st(2) * kATileBytes);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t a = (kk < 4 ? q0 : q1) + (kk & 3) * 32;
+    const uint32_t b = kb + (kk >> 2) * (kATileBytes / 2) + (kk & 3) * 32;
+    umma_bf16_ss(tmem + kTmemS, sdesc_kmajor_sw128(a), sdesc_kmajor_sw128(b), kAttIdescS, kk > 0 ? 1u : 0u);
+  }
+  umma_commit(&empty[st(0)]);
+  umma_commit(&empty[st(1)]);
+  umma_commit(&empty[st(2)]);
+  umma_commit(s_full);
+  if (!mbar_wait(p_full, au & 1, fp.status, abort_flag)) return false;
+  if (!mbar_wait(&full[st(3)], par(3), fp.status, abort_flag)) return false;
+  tc_fence_after();
+  const uint32_t pa = smem_u32(sA + st(4) * kATileBytes), vb = smem_u32(sA + st(3) * kATileBytes);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    umma_bf16_ss(tmem + kTmemO, sdesc_kmajor_sw128(pa + kk * 32), sdesc_kmajor_sw128(vb + kk * 32), kAttIdescO,
+                 kk > 0 ? 1u : 0u);
+  umma_commit(&empty[st(3)]);
+  umma_commit(&empty[st(4)]);
+  umma_commit(o_full);
+  return true;
+}
+
+// Softmax of one attention unit (128 epilogue threads, thread = row r of the
+// query tile: token r / 8, query head g * 8 + r % 8), P into its stage, the
+// row's partial output to global scratch.
+template <int STAGES>
+__device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* sA, uint64_t* full, uint64_t* att,
+                                                uint32_t tmem, long long iq, int au, int L, int g, int c,
+                                                volatile int* abort_flag) {
+  uint64_t* s_full = att;
+  uint64_t* p_full = att + 1;
+  uint64_t* o_full = att + 2;
+  uint64_t* att_free = att + 3;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int et = threadIdx.x - 64;
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const int n_rows = fp.qkv.ea.n_rows;
+  const int t = row >> 3;
+  const int limit = t < fp.n_clean ? L + t + 1 : L + n_rows;  // keys below `limit` are visible
+  const int key0 = c * kAttKeys;
+  auto st = [&](int j) { return static_cast<int>((iq + j) % STAGES); };
+  auto par = [&](int j) { return static_cast<uint32_t>(((iq + j) / STAGES) & 1); };
+  bool ok = mbar_wait(s_full, au & 1, fp.status, abort_flag);
+  float mx = -INFINITY, lsum = 0.f;
+  uint32_t packed[kAttKeys / 2];
+  if (ok) {
+    tc_fence_after();
+    float sc[64];
+    tmem_ld64(tmem + lane_off + kTmemS, sc);
+#pragma unroll
+    for (int k = 0; k < kAttKeys; ++k)
+      if (key0 + k < limit) mx = fmaxf(mx, sc[k] * fp.scale_log2);
+#pragma unroll
+    for (int k = 0; k < kAttKeys; k += 2) {
+      const float p0 = (key0 + k < limit) ? ex2_approx(sc[k] * fp.scale_log2 - mx) : 0.f;
+      const float p1 = (key0 + k + 1 < limit) ? ex2_approx(sc[k + 1] * fp.scale_log2 - mx) : 0.f;
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+      const float2 pr = __bfloat1622float2(pb);
+      lsum += pr.x + pr.y;
+      packed[k / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+    }
+    ok = mbar_wait(&full[st(4)], par(4), fp.status, abort_flag);  // the P stage is free
+  }
+  if (ok) {
+    uint8_t* prow = sA + st(4) * kATileBytes + row * 128;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+      *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
+          make_uint4(packed[cc * 4], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
+    // value row d = row: keys past the cache's valid slots (stale or
+    // poisoned, other heads' rows, zero fill) become 0, so that P = 0 there
+    // contributes exactly 0
+    const int n_valid = L + n_rows - key0;
+    if (n_valid < kAttKeys) {
+      ok = mbar_wait(&full[st(3)], par(3), fp.status, abort_flag);
+      if (ok) {
+        uint8_t* vrow = sA + st(3) * kATileBytes + row * 128;
+#pragma unroll
+        for (int pos = 0; pos < 8; ++pos) {
+          const int k0 = ((pos ^ (row & 7)) << 3);  // keys k0 .. k0+7 of this 16-byte chunk
+          if (k0 + 8 > n_valid) {
+            uint4 w = *reinterpret_cast<uint4*>(vrow + (pos << 4));
+            uint16_t* e = reinterpret_cast<uint16_t*>(&w);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (k0 + q >= n_valid) e[q] = 0;
+            *reinterpret_cast<uint4*>(vrow + (pos << 4)) = w;
+          }
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  named_bar_sync(1, 128);
+  if (et == 0) mbar_arrive(p_full);
+  ok = ok && mbar_wait(o_full, au & 1, fp.status, abort_flag);
+  named_bar_sync(1, 128);  // leave together if a wait gave up
+  if (*abort_flag) return false;
+  tc_fence_after();
+  const size_t pr = static_cast<size_t>(g * fp.n_chunks_max + c) * 128 + row;
+  float* dst = fp.apart + pr * 128;
+#pragma unroll 1
+  for (int cc = 0; cc < 128; cc += 64) {
+    float o[64];
+    tmem_ld64(tmem + lane_off + kTmemO + cc, o);
+#pragma unroll
+    for (int k = 0; k < 64; k += 4)
+      __stcg(reinterpret_cast<float4*>(dst + cc + k), make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]));
+  }
+  fp.aml[pr] = make_float2(mx, lsum);
+  tc_fence_before();
+  named_bar_sync(1, 128);
+  if (et == 0) mbar_arrive(att_free);
+  return true;
+}
+
+// Merge of attention rows: warp w of CTA b takes output rows (token t, query
+// head h) v = b + (w + 4 j) * gridDim.x; lanes hold 4 of the 128 features.
+__device__ __forceinline__ void fwd_att_merge(const FwdProgram& fp, int L, float* sW) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w = (threadIdx.x - 64) >> 5;  // 0..3
+  const int n_rows = fp.qkv.ea.n_rows;
+  const int n_chunks = att_chunks(fp, L);
+  float* wts = sW + w * fp.n_chunks_max;
+  (void)warp;
+  for (int v = blockIdx.x + w * gridDim.x; v < n_rows * fp.Hq; v += 4 * gridDim.x) {
+    const int t = v / fp.Hq, h = v % fp.Hq;
+    const int g = h >> 3, r = t * 8 + (h & 7);
+    const size_t base = static_cast<size_t>(g) * fp.n_chunks_max * 128 + r;
+    float M = -INFINITY;
+    for (int c = lane; c < n_chunks; c += 32) {
+      const float2 ml = __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]);
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float wl = 0.f;
+    for (int c = lane; c < n_chunks; c += 32) {
+      const float2 ml = __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]);
+      const float wc = ml.y > 0.f ? ex2_approx(ml.x - M) : 0.f;
+      wts[c] = wc;
+      wl += wc * ml.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
+    __syncwarp();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int c = 0; c < n_chunks; ++c) {
+      const float wc = wts[c];
+      if (wc != 0.f) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(fp.apart + (base + static_cast<size_t>(c) * 128) * 128) + lane);
+        acc.x += wc * f.x;
+        acc.y += wc * f.y;
+        acc.z += wc * f.z;
+        acc.w += wc * f.w;
+      }
+    }
+    const float inv = wl > 0.f ? 1.0f / wl : 0.f;
+    const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    bf16* out = fp.attn_o + static_cast<size_t>(t) * fp.Hq * 128 + h * 128 + lane * 4;
+    *reinterpret_cast<uint2*>(out) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+    __syncwarp();
+  }
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kFwdThreads, 1) fwd_persistent_kernel(const __grid_constant__ FwdProgram fp) {
+  constexpr int NT = kFwdNT;
   using S = GemmSmem<NT, STAGES, false>;
-  constexpr int TMC = tmem_cols_for<NT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem + S::kA;
@@ -710,9 +1008,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
+  uint64_t* att = acce + 2;  // s_full, p_full, o_full, att_free
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMisc);
   int* sflag = reinterpret_cast<int*>(smem + S::kMisc + 4);
   volatile int* sabort = reinterpret_cast<volatile int*>(smem + S::kMisc + 8);
+  const int n_phases = 6 * fp.n_layers;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -724,16 +1024,20 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
       mbar_init(&accf[b], 2);
       mbar_init(&acce[b], 4);
     }
+    for (int k = 0; k < 4; ++k) mbar_init(&att[k], 1);
     *sabort = 0;
     fence_mbar_init();
-    for (int p = 0; p < ca.n_phases; ++p) {
-      tma_prefetch_map(&ca.ph[p].mapA);
-      tma_prefetch_map(&ca.ph[p].mapB);
-      if (ca.ph[p].ea.epi == EPI_SWIGLU) tma_prefetch_map(&ca.ph[p].mapA2);
+    for (const ChainPhase* ph : {&fp.qkv, &fp.o, &fp.gu, &fp.down}) {
+      tma_prefetch_map(&ph->mapA);
+      tma_prefetch_map(&ph->mapB);
     }
+    tma_prefetch_map(&fp.gu.mapA2);
+    tma_prefetch_map(&fp.mapQ);
+    tma_prefetch_map(&fp.mapK);
+    tma_prefetch_map(&fp.mapV);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, TMC);
+    tmem_alloc(tmem_slot, kFwdTmem);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -742,65 +1046,101 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) chain_load_a<STAGES>(ca, sA, full, empty, sabort);
+    if (lane == 0) fwd_load_a<STAGES>(fp, sA, full, empty, sabort);
   } else if (warp == 7) {
-    if (lane == 0) chain_load_b<STAGES>(ca, sB, full, empty, sabort);
+    if (lane == 0) fwd_load_b<STAGES>(fp, sA, sB, full, empty, sabort);
   } else if (warp == 1 || warp == kMmaWarp2) {
     if (lane == 0) {
+      const int issuer = warp == 1 ? 0 : 1;
       long long i_base = 0;
-      int seg = 0;
-      for (int p = 0; p < ca.n_phases; ++p) {
-        const SkSched sc = chain_sched(ca.ph[p], ca.P);
+      int seg = 0, au = 0, L = -1;
+      for (int p = 0; p < n_phases; ++p) {
+        int layer;
+        const int kind = fwd_kind(fp, p, layer);
+        if (kind == FK_MERGE) continue;
+        if (kind == FK_ATT) {
+          if (L < 0) L = fwd_cache_len(fp);
+          const int n_units = fp.Hkv * att_chunks(fp, L);
+          bool ok = true;
+          for (int u = blockIdx.x; u < n_units; u += gridDim.x, i_base += kAttSlots, ++au)
+            if (issuer == 0 && !fwd_att_mma<STAGES>(fp, sA, full, empty, att, tmem, i_base, au, sabort)) {
+              ok = false;
+              break;
+            }
+          if (!ok) break;
+          continue;
+        }
+        const SkSched sc = chain_sched(fwd_gemm(fp, kind), gridDim.x);
         long long u0, u1;
         chain_range(sc, u0, u1);
-        if (!ws_mma_units<NT, STAGES, false>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, ca.status, sabort,
-                                             warp == 1 ? 0 : 1, 0, i_base, seg))
+        if (!ws_mma_units<NT, STAGES, false>(sA, sB, full, empty, accf, acce, tmem, sc, u0, u1, fp.status, sabort,
+                                             issuer, 0, i_base, seg))
           break;
       }
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ------------------------------------------------- epilogue, softmax, merge
     const int et = threadIdx.x - 64;  // 0..127
     griddep_wait();
     // dependents start only once this kernel's own inputs are complete
     if (et == 0) griddep_launch_dependents();
-    int gseg = 0;
+    const int L = fp.qkv.ea.d_len ? *fp.qkv.ea.d_len : fp.qkv.ea.L_static;
+    int gseg = 0, au = 0;
+    long long i_base = 0;
     bool ok = true;
-    for (int p = 0; p < ca.n_phases; ++p) {
-      const ChainPhase& ph = ca.ph[p];
-      const GemmEpi& ea = ph.ea;
+    for (int p = 0; p < n_phases; ++p) {
+      int layer;
+      const int kind = fwd_kind(fp, p, layer);
       if (p > 0) {
         if (et == 0) {
-          *sflag = ok && wait_counter(ca.bar, p * ca.P, ca.status, sabort) ? 1 : 0;
+          *sflag = ok && wait_counter(fp.bar, p * static_cast<int>(gridDim.x), fp.status, sabort) ? 1 : 0;
           __threadfence();
         }
         named_bar_sync(1, 128);
         ok = *sflag != 0;
         named_bar_sync(1, 128);  // sflag is read before the phase may reuse it
       }
-      if (ok) {
-        if (ea.epi != EPI_RESID) ws_rms_factors<NT>(ea, et, sR, sE);
-        const SkSched sc = chain_sched(ph, ca.P);
+      if (kind == FK_ATT) {
+        const int n_chunks = att_chunks(fp, L);
+        const int n_units = fp.Hkv * n_chunks;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, i_base += kAttSlots, ++au)
+          if (ok)
+            ok = fwd_att_softmax<STAGES>(fp, sA, full, att, tmem, i_base, au, L, u / n_chunks, u % n_chunks,
+                                         sabort);
+      } else if (kind == FK_MERGE) {
+        if (ok) fwd_att_merge(fp, L, sE);
+      } else {
+        const ChainPhase& ph = fwd_gemm(fp, kind);
+        const SkSched sc = chain_sched(ph, gridDim.x);
         long long u0, u1;
         chain_range(sc, u0, u1);
-        if (ea.epi == EPI_QKV)
-          ok = ws_epilogue_units<NT, EPI_QKV, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
-                                                     nullptr, nullptr, sflag, sabort, gseg,
-                                                     ea.d_len ? *ea.d_len : ea.L_static);
-        else if (ea.epi == EPI_SWIGLU)
-          ok = ws_epilogue_units<NT, EPI_SWIGLU, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
-                                                        nullptr, nullptr, sflag, sabort, gseg, 0);
-        else
-          ok = ws_epilogue_units<NT, EPI_RESID, false>(sc, u0, u1, ph.a_row_base, ea, tmem, accf, acce, sE, sR,
-                                                       nullptr, nullptr, sflag, sabort, gseg, 0);
+        if (ok) {
+          GemmEpi ea = ph.ea;
+          if (kind == FK_QKV) {
+            ea.kcache += layer * fp.kv_layer;
+            ea.vcache += layer * fp.kv_layer;
+          }
+          if (kind != FK_O && kind != FK_DOWN) ws_rms_factors<NT>(ea, et, sR, sE);
+          const int base = fwd_row_base(fp, kind, layer);
+          if (kind == FK_QKV)
+            ok = ws_epilogue_units<NT, EPI_QKV, false>(sc, u0, u1, base, ea, tmem, accf, acce, sE, sR, nullptr,
+                                                       nullptr, sflag, sabort, gseg, L);
+          else if (kind == FK_GU)
+            ok = ws_epilogue_units<NT, EPI_SWIGLU, false>(sc, u0, u1, base, ea, tmem, accf, acce, sE, sR, nullptr,
+                                                          nullptr, sflag, sabort, gseg, 0);
+          else
+            ok = ws_epilogue_units<NT, EPI_RESID, false>(sc, u0, u1, base, ea, tmem, accf, acce, sE, sR, nullptr,
+                                                         nullptr, sflag, sabort, gseg, 0);
+        }
+        i_base += u1 - u0;
       }
-      if (p + 1 < ca.n_phases) {
+      if (p + 1 < n_phases) {
         // this CTA's phase outputs, plain stores, are read by TMA in other CTAs
         fence_proxy_async_global();
         named_bar_sync(1, 128);
         if (et == 0) {
           __threadfence();
-          red_release_gpu_add(ca.bar, 1);
+          red_release_gpu_add(fp.bar, 1);
         }
       }
     }
@@ -816,15 +1156,15 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemm_chain_kernel(const __gr
   }
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMC);
+    tmem_dealloc(tmem, kFwdTmem);
   }
   if (threadIdx.x == 0) {
     // every thread of this CTA is past its last barrier wait; the last CTA
     // out zeroes both counters for the next launch
     __threadfence();
-    if (atomicAdd(ca.bar + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-      ca.bar[0] = 0;
-      ca.bar[1] = 0;
+    if (atomicAdd(fp.bar + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      fp.bar[0] = 0;
+      fp.bar[1] = 0;
       __threadfence();
     }
   }
@@ -992,42 +1332,53 @@ cudaError_t launch_gemm_ws(int NT, const CUtensorMap& mapA, const CUtensorMap& m
   return cudaErrorInvalidValue;
 }
 
-static int chain_cap[64] = {};  // resident CTAs per device (0: not yet queried)
+static int fwd_cap[64] = {};  // resident CTAs per device (0: not yet queried)
 
-int gemm_chain_max_ctas() {
-  using S = GemmSmem<kChainNT, kChainStages, false>;
+int fwd_persistent_max_ctas() {
+  using S = GemmSmem<kFwdNT, kFwdStages, false>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (chain_cap[dev] == 0) {
-    auto kern = gemm_chain_kernel<kChainStages>;
+  if (fwd_cap[dev] == 0) {
+    auto kern = fwd_persistent_kernel<kFwdStages>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal) != cudaSuccess) return 0;
     int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kChainThreads, S::kTotal) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, S::kTotal) != cudaSuccess)
       return 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    chain_cap[dev] = per_sm * sms;
+    fwd_cap[dev] = per_sm * sms;
   }
-  return chain_cap[dev];
+  return fwd_cap[dev];
 }
 
-cudaError_t launch_gemm_chain(const ChainArgs& ca, bool pdl, cudaStream_t s) {
-  using S = GemmSmem<kChainNT, kChainStages, false>;
-  if (ca.n_phases < 1 || ca.n_phases > kMaxChainPhases || ca.P < 1 || !ca.bar || !ca.status)
+size_t fwd_attn_scratch_bytes(int Hkv, int Lmax) {
+  const size_t n_chunks = (static_cast<size_t>(Lmax) + kAttKeys - 1) / kAttKeys;
+  const size_t part = static_cast<size_t>(Hkv) * n_chunks * 128 * 128 * 4;
+  const size_t ml = static_cast<size_t>(Hkv) * n_chunks * 128 * 8;
+  return (part + 255) / 256 * 256 + (ml + 255) / 256 * 256;
+}
+
+cudaError_t launch_fwd_persistent(const FwdProgram& fp, int P, bool pdl, cudaStream_t s) {
+  using S = GemmSmem<kFwdNT, kFwdStages, false>;
+  if (fp.n_layers < 1 || P < 1 || !fp.bar || !fp.status || !fp.apart || !fp.aml || !fp.attn_o)
     return cudaErrorInvalidValue;
-  for (int p = 0; p < ca.n_phases; ++p) {
-    const ChainPhase& ph = ca.ph[p];
-    const int epi = ph.ea.epi;
-    if ((epi != EPI_QKV && epi != EPI_RESID && epi != EPI_SWIGLU) || ph.n_tiles < 1 || ph.kb < 1 ||
-        ph.ea.n_rows < 1 || ph.ea.n_rows > kChainNT || !ph.ea.part || !ph.ea.cnt || ph.ea.status != ca.status)
+  if (fp.Hq != 8 * fp.Hkv || fp.n_chunks_max < (fp.Lmax + kAttKeys - 1) / kAttKeys ||
+      fp.n_chunks_max * 4 > 128 * (kFwdNT + 1))
+    return cudaErrorInvalidValue;
+  for (const ChainPhase* ph : {&fp.qkv, &fp.o, &fp.gu, &fp.down}) {
+    if (ph->n_tiles < 1 || ph->kb < 1 || ph->ea.n_rows < 1 || ph->ea.n_rows > kFwdNT || !ph->ea.part ||
+        !ph->ea.cnt || ph->ea.status != fp.status)
       return cudaErrorInvalidValue;
   }
+  if (fp.qkv.ea.epi != EPI_QKV || fp.o.ea.epi != EPI_RESID || fp.gu.ea.epi != EPI_SWIGLU ||
+      fp.down.ea.epi != EPI_RESID)
+    return cudaErrorInvalidValue;
   // every CTA must be resident at once: the phases meet at grid barriers
-  const int cap = gemm_chain_max_ctas();
+  const int cap = fwd_persistent_max_ctas();
   if (cap < 1) return cudaErrorInvalidConfiguration;
-  if (ca.P > cap) return cudaErrorCooperativeLaunchTooLarge;
+  if (P > cap) return cudaErrorCooperativeLaunchTooLarge;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ca.P);
-  cfg.blockDim = dim3(kChainThreads);
+  cfg.gridDim = dim3(P);
+  cfg.blockDim = dim3(kFwdThreads);
   cfg.dynamicSmemBytes = S::kTotal;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1035,7 +1386,7 @@ cudaError_t launch_gemm_chain(const ChainArgs& ca, bool pdl, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_chain_kernel<kChainStages>, ca);
+  return cudaLaunchKernelEx(&cfg, fwd_persistent_kernel<kFwdStages>, fp);
 }
 
 }  // namespace dvlm

@@ -133,29 +133,43 @@ cudaError_t launch_gemm_cl(int NT, const CUtensorMap& mapA, const CUtensorMap& m
                            int a_row_base, const GemmEpi& ea, bool pdl, cudaStream_t s, int stages);
 int gemm_cl_max_clusters(int epi, int S, int stages);
 
-// Persistent chain of bf16 weight-streaming GEMMs over 16 token rows: up to
-// kMaxChainPhases products run as consecutive stream-K phases of one launch
-// of P CTAs (one per SM, all resident at once), each phase's inputs the
-// previous phases' outputs (a grid barrier between phases).  Phase p streams
-// weights mapA (mapA2: the up rows of a gate/up product) against activations
-// mapB over n_tiles x kb units with the fused epilogue ea (ea.cnt: n_tiles
-// zeroed ints of its own; ea.part: P partial tiles, shared by the phases).
+// Persistent forward (bf16 weights, 16 token rows): every decoder layer of
+// one forward in a single launch of one CTA per SM, phase by phase -- the
+// first layer's QKV, then per layer l: attention partials, attention merge,
+// O-projection, gate/up, down, and QKV of layer l+1 (not after the last
+// layer) -- with a grid barrier between phases.  The four GEMM phases are
+// given in their first-layer form: weight rows of layer l start at
+// l * (qkv_rows | H | I | H); the QKV phase's cache pointers move by
+// kv_layer elements per layer.  Each GEMM phase's ea.cnt is its own block of
+// n_tiles zeroed ints; ea.part holds one partial tile per CTA.
 struct ChainPhase {
   CUtensorMap mapA, mapA2, mapB;
   GemmEpi ea;
   int n_tiles, kb, a_row_base;
 };
-constexpr int kMaxChainPhases = 4;
-struct ChainArgs {
-  ChainPhase ph[kMaxChainPhases];
-  int n_phases;
-  int P;
-  int* bar;     // [2] barrier and exit counters: zero before the first launch, zero again after each
+struct FwdProgram {
+  ChainPhase qkv, o, gu, down;
+  int qkv_rows, H, I;
+  size_t kv_layer;
+  // attention: q [16][Hq][128] (3-D map, 64 x 8 x 16 box), the cache's K
+  // rows ((layer * Hkv + g) * Lmax + slot, 64 x 64 box) and V^T rows
+  // ((layer * Hkv + g) * 128 + d, 64-key x 128 box); Hq = 8 * Hkv
+  CUtensorMap mapQ, mapK, mapV;
+  int Hq, Hkv, Lmax, n_clean;
+  float scale_log2;
+  float* apart;   // [Hkv][n_chunks_max][128 rows][128] unnormalised partial rows (fp32)
+  float2* aml;    // [Hkv][n_chunks_max][128 rows] (row max, row sum) per 64-key chunk
+  int n_chunks_max;
+  bf16* attn_o;   // [16][Hq * 128] merged attention rows, the O-projection's input
+  int layer0, n_layers;
+  int* bar;       // [2] barrier and exit counters: zero before the first launch, zero again after each
   int* status;
 };
-cudaError_t launch_gemm_chain(const ChainArgs& ca, bool pdl, cudaStream_t s);
-// CTAs of the chain kernel that can be resident at once on the current device (0 on error).
-int gemm_chain_max_ctas();
+cudaError_t launch_fwd_persistent(const FwdProgram& fp, int P, bool pdl, cudaStream_t s);
+// CTAs of the persistent forward that can be resident at once on the current device (0 on error).
+int fwd_persistent_max_ctas();
+// Scratch of the attention phases for caches of Lmax slots: apart, then aml.
+size_t fwd_attn_scratch_bytes(int Hkv, int Lmax);
 cudaError_t launch_lmhead(int NT, const CUtensorMap& mapW, const CUtensorMap& mapH, int n_tiles, int kb, int P,
                           const LmArgs& a, bool pdl, cudaStream_t s);
 size_t lmhead_scratch_bytes(int NT, int P, int n_tiles);

@@ -466,13 +466,17 @@ DVLM_API dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int
  *   "attn_split": 0 = cluster attention, 1..32 = split attention with that
  *       many CTAs per KV head (dvlm_block_attn_split);
  *   "prefill_gemm": 1/0, the compute-bound prefill (where supported);
- *   "persistent": 1/0, the decoder GEMMs as a persistent chain: per layer,
- *       after attention, one launch on every SM runs the O-projection,
- *       gate/up, down and the next layer's QKV as stream-K phases separated
- *       by grid barriers (bf16 weights, 128-wide heads; UNSUPPORTED where
- *       one CTA per SM cannot be resident on all SMs).
+ *   "persistent": 1/0, every decoder layer of a forward in one launch on
+ *       all SMs: the first layer's QKV, then per layer attention (64-key
+ *       chunk units), its merge, O-projection, gate/up, down and the next
+ *       layer's QKV as phases separated by grid barriers, the weight stream
+ *       running ahead across them (bf16 weights, 128-wide heads, 8 query
+ *       heads per KV head, contiguous cache; TEXT-ONLY passes and paged
+ *       caches use the per-kernel path; UNSUPPORTED where one CTA per SM
+ *       cannot be resident on all SMs).
  * Results do not depend on the knobs except through fp32 summation order
- * (cluster sizes, stream-K splits).  Changing a knob drops the captured CUDA graphs.
+ * (cluster sizes, stream-K splits) and, with "persistent", attention's P
+ * held in bf16 (fp16 in the per-kernel attention).  Changing a knob drops the captured CUDA graphs.
  * Errors: INVALID_ARG (unknown name), SHAPE (bad value), UNSUPPORTED (the
  * device cannot launch that configuration, or an fp32 engine). */
 DVLM_API dvlm_status dvlm_engine_set_option(dvlm_engine* e, const char* name, int value);
@@ -542,9 +546,8 @@ DVLM_API dvlm_status dvlm_engine_set_trace(dvlm_engine* e, void* buf, size_t byt
  * over layers and counts_out[8] the launches: [0] embedding, [1] QKV GEMM,
  * [2] attention, [3] O-projection GEMM, [4] gate/up GEMM, [5] down GEMM,
  * [6] fused LM head (run when with_lm_head != 0, rows 0..n_rows-1, no
- * commit), [7] persistent GEMM chain (option "persistent": the first
- * layer's QKV, then per layer O-projection, gate/up, down and the next
- * layer's QKV in one launch; classes 1, 3, 4 and 5 are then empty).
+ * commit), [7] persistent forward (option "persistent": every decoder
+ * layer in one launch; classes 1 to 5 are then empty).
  * Synchronises the stream. */
 DVLM_API dvlm_status dvlm_profile_forward(dvlm_engine* e, const int32_t* tokens, const uint8_t* masked,
                                           int n_rows, int n_clean, int with_lm_head, float* ms_out,

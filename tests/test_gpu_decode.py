@@ -215,11 +215,10 @@ def test_bf16_reduced_model_engine_path(cuda, seed, mode, persistent):
     emission and, for speculative decoding, the accept kernel), every forward
     replayed against the oracle: decisions bit-exact at the 1e-3 bar on the
     rows the LM head read, within DELTA on the oracle's own rows, hidden rows
-    within 2e-2 plus one storage ulp.  persistent=1: the decoder GEMMs run as
-    the persistent chain (first layer's QKV; then O-projection, gate/up,
-    down and the next layer's QKV per launch); at this size most CTAs of a
-    phase hold one k block or none, so every output tile is split over many
-    CTAs."""
+    within 2e-2 plus one storage ulp.  persistent=1: each forward is one
+    persistent launch (QKV, attention, merge, O-projection, gate/up, down
+    per layer); at this size most CTAs of a GEMM phase hold one k block or
+    none, so every output tile is split over many CTAs."""
     s = Setup(SMALL_BF16, seed, cuda, 32, 16, 0, options={"persistent": persistent} if persistent else None)
     tokens, st, recs, L, sd = s.traced(mode, 16, 0.9, 32)
     rp, m = replay_trace(s, mode, 16, 0.9, 32, tokens, st, recs, L, sd)

@@ -202,15 +202,15 @@ def test_every_layer_matches_oracle_on_identical_inputs(full):
     print("per-layer max abs error:", worst)
 
 
-def test_persistent_chain_matches_oracle_per_layer(full):
-    """The persistent GEMM chain at full size (option "persistent"): layers
-    0, 1, 17 and 35 run one at a time on identical inputs (the first
-    layer's QKV as a one-phase chain, attention, then O-projection, gate/up
-    and down as one three-phase launch), each against the oracle's layer at
-    the 2e-2 bar; the input of layer l is the per-kernel path's output of
-    layers 0..l-1.  Then layers 17 and 18 in one forward, whose first chain
-    launch has all four phases (O, gate/up, down, layer 18's QKV), against
-    the per-kernel path on the same input."""
+def test_persistent_forward_matches_oracle_per_layer(full):
+    """The persistent forward at full size (option "persistent": every
+    layer of a forward in one launch): layers 0, 1, 17 and 35 run one at a
+    time on identical inputs (QKV, attention over 64-key chunks, the merge,
+    O-projection, gate/up and down as phases of one launch), each against
+    the oracle's layer at the 2e-2 bar (two storage ulps on the output rows),
+    K/V included; the input of layer l is the per-kernel path's output of
+    layers 0..l-1.  Then layers 17 and 18 in one launch (the next layer's QKV
+    between them) against the per-kernel path on the same input."""
     dims, eng, cuda = full["dims"], full["eng"], full["kc"].device
     L0 = full["L0"]
     names = gen.layer_weight_names()
@@ -240,10 +240,10 @@ def test_persistent_chain_matches_oracle_per_layer(full):
             m.K[l][:, :L0] = f64(full["kc"][l, 0, :, :L0])
             m.V[l][:, :L0] = f64(full["vc"][l, 0, :, :, :L0]).transpose(0, 2, 1)
             xo = m.layer(l, xin64, L0, 0)
-            assert_bf16_close(f64(x_out), xo, 2e-2, f"chain layer {l} output", ulps=2)
-            assert_bf16_close(f64(full["kc"][l, 0, :, L0:L0 + 16]), m.K[l][:, L0:L0 + 16], 2e-2, f"chain layer {l} K")
+            assert_bf16_close(f64(x_out), xo, 2e-2, f"persistent layer {l} output", ulps=2)
+            assert_bf16_close(f64(full["kc"][l, 0, :, L0:L0 + 16]), m.K[l][:, L0:L0 + 16], 2e-2, f"persistent layer {l} K")
             assert_bf16_close(f64(full["vc"][l, 0, :, :, L0:L0 + 16]).transpose(0, 2, 1), m.V[l][:, L0:L0 + 16],
-                              2e-2, f"chain layer {l} V")
+                              2e-2, f"persistent layer {l} V")
         # two layers: the four-phase launch against the per-kernel path
         eng.set_option("persistent", 0)
         eng.forward(16, 0, 17, tokens=toks, first_layer=0, x_out=x_in)
@@ -254,17 +254,18 @@ def test_persistent_chain_matches_oracle_per_layer(full):
             eng.check()
             outs.append((f64(x_out), f64(full["kc"][18, 0, :, L0:L0 + 16])))
         # two layers: a flip in layer 17's output is carried through layer 18's two stores
-        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, chain vs per-kernel", ulps=3)
-        assert_bf16_close(outs[1][1], outs[0][1], 2e-2, "layer 18 K, chain vs per-kernel")
+        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, persistent vs per-kernel", ulps=3)
+        assert_bf16_close(outs[1][1], outs[0][1], 2e-2, "layer 18 K, persistent vs per-kernel")
     finally:
         eng.set_option("persistent", 0)
     eng.set_position(L0, full["seed0"])
 
 
-def test_persistent_chain_decode_properties(full):
-    """Properties of the persistent chain's decode at full size: linear
-    self-speculative decoding equals greedy AR decoding, and graph replay
-    equals eager launches."""
+def test_persistent_forward_decode_properties(full):
+    """Properties of the persistent forward's decode at full size: linear
+    self-speculative decoding equals greedy AR decoding (attention's rows do
+    not depend on the number of rows in the pass), and graph replay equals
+    eager launches."""
     eng = full["eng"]
     eng.set_option("persistent", 1)
     try:
