@@ -627,7 +627,8 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
 // query tile (8 heads x 16 rows = 128 rows, two 64-wide halves), the
 // chunk's keys, its values (transposed) and P -- and leaves, for each row,
 // the chunk's unnormalised output O_c = sum_k p_k v_k with p_k = 2^(s_k - m_c)
-// (P in bf16; l_c sums the same bf16 values), the row max m_c and l_c.  The
+// (P and V in fp16 for the second product; l_c sums the same fp16 values),
+// the row max m_c and l_c.  The
 // merge phase combines a row's chunks in chunk order:
 // out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.  A row's arithmetic
 // depends only on its own query and keys (chunks by absolute key position),
@@ -644,7 +645,7 @@ constexpr int kFwdNT = 16;
 constexpr int kAttKeys = 64;   // keys per attention unit
 constexpr int kAttSlots = 5;   // stages of an attention unit: Q (2 halves), K, V^T, P
 constexpr uint32_t kAttIdescS = idesc_bf16_f32(128, kAttKeys);
-constexpr uint32_t kAttIdescO = idesc_bf16_f32(128, 128);
+constexpr uint32_t kAttIdescO = idesc_f16_f32(128, 128);  // P and V in fp16
 constexpr int kFwdTmem = 256;  // GEMM accumulators [0, 64), S [64, 128), O [128, 256)
 constexpr uint32_t kTmemS = 64, kTmemO = 128;
 
@@ -881,10 +882,10 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
     for (int k = 0; k < kAttKeys; k += 2) {
       const float p0 = (key0 + k < limit) ? ex2_approx(sc[k] * fp.scale_log2 - mx) : 0.f;
       const float p1 = (key0 + k + 1 < limit) ? ex2_approx(sc[k + 1] * fp.scale_log2 - mx) : 0.f;
-      const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-      const float2 pr = __bfloat1622float2(pb);
+      const __half2 ph = __floats2half2_rn(p0, p1);
+      const float2 pr = __half22float2(ph);
       lsum += pr.x + pr.y;
-      packed[k / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+      packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
     }
     ok = mbar_wait(&full[st(4)], par(4), fp.status, abort_flag);  // the P stage is free
   }
@@ -894,26 +895,25 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
     for (int cc = 0; cc < 8; ++cc)
       *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
           make_uint4(packed[cc * 4], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
-    // value row d = row: keys past the cache's valid slots (stale or
-    // poisoned, other heads' rows, zero fill) become 0, so that P = 0 there
-    // contributes exactly 0
+    // value row d = row to fp16 in place; keys past the cache's valid slots
+    // (stale or poisoned, other heads' rows, zero fill) become 0, so that
+    // P = 0 there contributes exactly 0
     const int n_valid = L + n_rows - key0;
-    if (n_valid < kAttKeys) {
-      ok = mbar_wait(&full[st(3)], par(3), fp.status, abort_flag);
-      if (ok) {
-        uint8_t* vrow = sA + st(3) * kATileBytes + row * 128;
+    ok = mbar_wait(&full[st(3)], par(3), fp.status, abort_flag);
+    if (ok) {
+      uint8_t* vrow = sA + st(3) * kATileBytes + row * 128;
 #pragma unroll
-        for (int pos = 0; pos < 8; ++pos) {
-          const int k0 = ((pos ^ (row & 7)) << 3);  // keys k0 .. k0+7 of this 16-byte chunk
-          if (k0 + 8 > n_valid) {
-            uint4 w = *reinterpret_cast<uint4*>(vrow + (pos << 4));
-            uint16_t* e = reinterpret_cast<uint16_t*>(&w);
+      for (int pos = 0; pos < 8; ++pos) {
+        const int k0 = ((pos ^ (row & 7)) << 3);  // keys k0 .. k0+7 of this 16-byte chunk
+        uint4 w = *reinterpret_cast<uint4*>(vrow + (pos << 4));
+        uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (k0 + q >= n_valid) e[q] = 0;
-            *reinterpret_cast<uint4*>(vrow + (pos << 4)) = w;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+          const __half2 hh = __floats2half2_rn(k0 + 2 * e < n_valid ? f.x : 0.f, k0 + 2 * e + 1 < n_valid ? f.y : 0.f);
+          wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
         }
+        *reinterpret_cast<uint4*>(vrow + (pos << 4)) = w;
       }
     }
   }

@@ -253,9 +253,11 @@ def test_persistent_forward_matches_oracle_per_layer(full):
             eng.forward(16, 0, 2, x_in=x_in, first_layer=17, x_out=x_out)
             eng.check()
             outs.append((f64(x_out), f64(full["kc"][18, 0, :, L0:L0 + 16])))
-        # two layers: a flip in layer 17's output is carried through layer 18's two stores
-        assert_bf16_close(outs[1][0], outs[0][0], 2e-2, "layers 17-18 output, persistent vs per-kernel", ulps=3)
-        assert_bf16_close(outs[1][1], outs[0][1], 2e-2, "layer 18 K, persistent vs per-kernel")
+        # two layers: each path's storage flips (and their attention
+        # arithmetic, chunked differently) compound through layer 18, so the
+        # end-to-end drift bar applies
+        _assert_drift(outs[1][0], outs[0][0], "layers 17-18 output, persistent vs per-kernel")
+        _assert_drift(outs[1][1], outs[0][1], "layer 18 K, persistent vs per-kernel")
     finally:
         eng.set_option("persistent", 0)
     eng.set_position(L0, full["seed0"])
