@@ -236,7 +236,8 @@ static void fill_lm_scratch(dvlm_engine* e, LmArgs& a) {
 static bool persistent_supported(dvlm_engine* e) {
   const dvlm_model& m = e->m;
   return e->bf16 && !e->fp8 && m.head_dim == 128 && m.hidden % 128 == 0 && m.inter % 64 == 0 &&
-         m.n_q_heads == 8 * m.n_kv_heads && e->fwd_att && e->sm >= 1 && e->sm <= fwd_persistent_max_ctas();
+         m.n_q_heads == 8 * m.n_kv_heads && e->Lmax <= 8192 && e->fwd_att && e->sm >= 1 &&
+         e->sm <= fwd_persistent_max_ctas();
 }
 
 static ChainPhase chain_phase(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, int n_tiles, int kb,

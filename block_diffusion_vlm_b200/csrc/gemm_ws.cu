@@ -943,46 +943,52 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
 }
 
 // Merge of attention rows: warp w of CTA b takes output rows (token t, query
-// head h) v = b + (w + 4 j) * gridDim.x; lanes hold 4 of the 128 features.
+// head h) v = b + (w + 4 j) * gridDim.x; lanes hold a row's (m, l) pairs
+// (chunks lane, lane + 32, ...), then 4 of its 128 features each, the
+// chunks' partial rows read with independent loads (every chunk below
+// n_chunks holds a finite partial row: 0 where the row sees none of its keys).
+constexpr int kMergeChunksPerLane = 4;  // chunks of a row: at most 128 (8192 cache slots)
 __device__ __forceinline__ void fwd_att_merge(const FwdProgram& fp, int L, float* sW) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int w = (threadIdx.x - 64) >> 5;  // 0..3
   const int n_rows = fp.qkv.ea.n_rows;
   const int n_chunks = att_chunks(fp, L);
   float* wts = sW + w * fp.n_chunks_max;
-  (void)warp;
   for (int v = blockIdx.x + w * gridDim.x; v < n_rows * fp.Hq; v += 4 * gridDim.x) {
     const int t = v / fp.Hq, h = v % fp.Hq;
     const int g = h >> 3, r = t * 8 + (h & 7);
     const size_t base = static_cast<size_t>(g) * fp.n_chunks_max * 128 + r;
+    float2 ml[kMergeChunksPerLane];
     float M = -INFINITY;
-    for (int c = lane; c < n_chunks; c += 32) {
-      const float2 ml = __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]);
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+#pragma unroll
+    for (int j = 0; j < kMergeChunksPerLane; ++j) {
+      const int c = lane + 32 * j;
+      ml[j] = c < n_chunks ? __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]) : make_float2(-INFINITY, 0.f);
+      if (ml[j].y > 0.f) M = fmaxf(M, ml[j].x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float wl = 0.f;
-    for (int c = lane; c < n_chunks; c += 32) {
-      const float2 ml = __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]);
-      const float wc = ml.y > 0.f ? ex2_approx(ml.x - M) : 0.f;
-      wts[c] = wc;
-      wl += wc * ml.y;
+#pragma unroll
+    for (int j = 0; j < kMergeChunksPerLane; ++j) {
+      const int c = lane + 32 * j;
+      const float wc = ml[j].y > 0.f ? ex2_approx(ml[j].x - M) : 0.f;
+      if (c < n_chunks) wts[c] = wc;
+      wl += wc * ml[j].y;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
     __syncwarp();
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* src = reinterpret_cast<const float4*>(fp.apart + base * 128) + lane;
 #pragma unroll 8
     for (int c = 0; c < n_chunks; ++c) {
       const float wc = wts[c];
-      if (wc != 0.f) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(fp.apart + (base + static_cast<size_t>(c) * 128) * 128) + lane);
-        acc.x += wc * f.x;
-        acc.y += wc * f.y;
-        acc.z += wc * f.z;
-        acc.w += wc * f.w;
-      }
+      const float4 f = __ldcg(src + static_cast<size_t>(c) * 128 * 32);
+      acc.x += wc * f.x;
+      acc.y += wc * f.y;
+      acc.z += wc * f.z;
+      acc.w += wc * f.w;
     }
     const float inv = wl > 0.f ? 1.0f / wl : 0.f;
     const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
@@ -1362,7 +1368,7 @@ cudaError_t launch_fwd_persistent(const FwdProgram& fp, int P, bool pdl, cudaStr
   if (fp.n_layers < 1 || P < 1 || !fp.bar || !fp.status || !fp.apart || !fp.aml || !fp.attn_o)
     return cudaErrorInvalidValue;
   if (fp.Hq != 8 * fp.Hkv || fp.n_chunks_max < (fp.Lmax + kAttKeys - 1) / kAttKeys ||
-      fp.n_chunks_max * 4 > 128 * (kFwdNT + 1))
+      fp.n_chunks_max > 32 * kMergeChunksPerLane)
     return cudaErrorInvalidValue;
   for (const ChainPhase* ph : {&fp.qkv, &fp.o, &fp.gu, &fp.down}) {
     if (ph->n_tiles < 1 || ph->kb < 1 || ph->ea.n_rows < 1 || ph->ea.n_rows > kFwdNT || !ph->ea.part ||
