@@ -681,7 +681,8 @@ __device__ __forceinline__ int att_chunks(const FwdProgram& fp, int L) {
 // its contributors); CTAs past those have no units in the phase.
 __device__ __forceinline__ SkSched chain_sched(const ChainPhase& ph, int P) {
   const long long units = static_cast<long long>(ph.n_tiles) * ph.kb;
-  return SkSched{ph.n_tiles, ph.kb, static_cast<int>(units < P ? units : P)};
+  const int ctas = ph.ctas > 0 && ph.ctas < P ? ph.ctas : P;
+  return SkSched{ph.n_tiles, ph.kb, static_cast<int>(units < ctas ? units : ctas)};
 }
 __device__ __forceinline__ void chain_range(const SkSched& sc, long long& u0, long long& u1) {
   if (static_cast<int>(blockIdx.x) >= sc.P) {
@@ -875,18 +876,29 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
     tc_fence_after();
     float sc[64];
     tmem_ld64(tmem + lane_off + kTmemS, sc);
+    // row max as 8 independent partial maxima (a short dependency chain)
+    float m8[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
 #pragma unroll
     for (int k = 0; k < kAttKeys; ++k)
-      if (key0 + k < limit) mx = fmaxf(mx, sc[k] * fp.scale_log2);
+      if (key0 + k < limit) m8[k & 7] = fmaxf(m8[k & 7], sc[k] * fp.scale_log2);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) mx = fmaxf(mx, m8[q]);
+    float l8[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) l8[q] = 0.f;
 #pragma unroll
     for (int k = 0; k < kAttKeys; k += 2) {
       const float p0 = (key0 + k < limit) ? ex2_approx(sc[k] * fp.scale_log2 - mx) : 0.f;
       const float p1 = (key0 + k + 1 < limit) ? ex2_approx(sc[k + 1] * fp.scale_log2 - mx) : 0.f;
       const __half2 ph = __floats2half2_rn(p0, p1);
       const float2 pr = __half22float2(ph);
-      lsum += pr.x + pr.y;
+      l8[(k >> 1) & 7] += pr.x + pr.y;
       packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) lsum += l8[q];
     ok = mbar_wait(&full[st(4)], par(4), fp.status, abort_flag);  // the P stage is free
   }
   if (ok) {
@@ -903,7 +915,10 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
     if (ok) {
       uint8_t* vrow = sA + st(3) * kATileBytes + row * 128;
 #pragma unroll
-      for (int pos = 0; pos < 8; ++pos) {
+      for (int i = 0; i < 8; ++i) {
+        // lanes start at different 16-byte chunks of their rows (rows are
+        // 128 bytes apart: the same banks)
+        const int pos = (i + lane) & 7;
         const int k0 = ((pos ^ (row & 7)) << 3);  // keys k0 .. k0+7 of this 16-byte chunk
         uint4 w = *reinterpret_cast<uint4*>(vrow + (pos << 4));
         uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
@@ -925,78 +940,96 @@ __device__ __forceinline__ bool fwd_att_softmax(const FwdProgram& fp, uint8_t* s
   named_bar_sync(1, 128);  // leave together if a wait gave up
   if (*abort_flag) return false;
   tc_fence_after();
-  const size_t pr = static_cast<size_t>(g * fp.n_chunks_max + c) * 128 + row;
-  float* dst = fp.apart + pr * 128;
+  // the unit's partial rows feature-major: each store of the warp covers 32
+  // consecutive rows of one feature (128 contiguous bytes)
+  const size_t unit = static_cast<size_t>(g * fp.n_chunks_max + c);
+  float* dst = fp.apart + unit * 128 * 128 + row;
 #pragma unroll 1
   for (int cc = 0; cc < 128; cc += 64) {
     float o[64];
     tmem_ld64(tmem + lane_off + kTmemO + cc, o);
 #pragma unroll
-    for (int k = 0; k < 64; k += 4)
-      __stcg(reinterpret_cast<float4*>(dst + cc + k), make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]));
+    for (int k = 0; k < 64; ++k) __stcg(dst + static_cast<size_t>(cc + k) * 128, o[k]);
   }
-  fp.aml[pr] = make_float2(mx, lsum);
+  fp.aml[unit * 128 + row] = make_float2(mx, lsum);
   tc_fence_before();
   named_bar_sync(1, 128);
   if (et == 0) mbar_arrive(att_free);
   return true;
 }
 
-// Merge of attention rows: warp w of CTA b takes output rows (token t, query
-// head h) v = b + (w + 4 j) * gridDim.x; lanes hold a row's (m, l) pairs
-// (chunks lane, lane + 32, ...), then 4 of its 128 features each, the
-// chunks' partial rows read with independent loads (every chunk below
-// n_chunks holds a finite partial row: 0 where the row sees none of its keys).
-constexpr int kMergeChunksPerLane = 4;  // chunks of a row: at most 128 (8192 cache slots)
+// Merge of attention rows: CTA b takes the (token t, KV group g) units
+// v = b, b + gridDim.x, ... -- 8 rows r = 8 t + (query head within the group)
+// -- and warp w their features [32 w, 32 w + 32); lane = (feature quad q,
+// row hl), so that one load of the warp covers 4 features x 8 rows (four
+// 32-byte pieces).  The rows' weights come first: w_c = 2^(m_c - M), M the
+// row's largest chunk max, and l = sum_c w_c l_c; every chunk below
+// n_chunks holds a finite partial row (0 where the row sees none of its keys).
+constexpr int kMergeMaxChunks = 128;  // 8192 cache slots
 __device__ __forceinline__ void fwd_att_merge(const FwdProgram& fp, int L, float* sW) {
   const int lane = threadIdx.x & 31;
-  const int w = (threadIdx.x - 64) >> 5;  // 0..3
+  const int et = threadIdx.x - 64;
+  const int w = et >> 5;  // 0..3
   const int n_rows = fp.qkv.ea.n_rows;
   const int n_chunks = att_chunks(fp, L);
-  float* wts = sW + w * fp.n_chunks_max;
-  for (int v = blockIdx.x + w * gridDim.x; v < n_rows * fp.Hq; v += 4 * gridDim.x) {
-    const int t = v / fp.Hq, h = v % fp.Hq;
-    const int g = h >> 3, r = t * 8 + (h & 7);
-    const size_t base = static_cast<size_t>(g) * fp.n_chunks_max * 128 + r;
-    float2 ml[kMergeChunksPerLane];
-    float M = -INFINITY;
+  float* wts = sW;                      // [8 rows][n_chunks]
+  float* inv = sW + 8 * n_chunks;       // [8 rows]
+  const int hl = lane & 7, q = lane >> 3;
+  for (int v = blockIdx.x; v < n_rows * fp.Hkv; v += gridDim.x) {
+    const int t = v / fp.Hkv, g = v % fp.Hkv;
+    // weights: thread et takes row et & 7 and chunks et >> 3, + 16, ...
+    {
+      const int r8 = et & 7;
+      const float2* ml = fp.aml + static_cast<size_t>(g) * fp.n_chunks_max * 128 + t * 8 + r8;
+      float M = -INFINITY;
+      for (int c = et >> 3; c < n_chunks; c += 16) {
+        const float2 x = __ldcg(&ml[static_cast<size_t>(c) * 128]);
+        if (x.y > 0.f) M = fmaxf(M, x.x);
+      }
+      // lanes of one row: et, et + 8, ... (the same row in each of the 16 groups of 8)
 #pragma unroll
-    for (int j = 0; j < kMergeChunksPerLane; ++j) {
-      const int c = lane + 32 * j;
-      ml[j] = c < n_chunks ? __ldcg(&fp.aml[base + static_cast<size_t>(c) * 128]) : make_float2(-INFINITY, 0.f);
-      if (ml[j].y > 0.f) M = fmaxf(M, ml[j].x);
+      for (int o = 8; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      sW[1152 + et] = M;  // the four warps' maxima, combined below
+      named_bar_sync(1, 128);
+      M = fmaxf(fmaxf(sW[1152 + r8], sW[1152 + 32 + r8]), fmaxf(sW[1152 + 64 + r8], sW[1152 + 96 + r8]));
+      float wl = 0.f;
+      for (int c = et >> 3; c < n_chunks; c += 16) {
+        const float2 x = __ldcg(&ml[static_cast<size_t>(c) * 128]);
+        const float wc = x.y > 0.f ? ex2_approx(x.x - M) : 0.f;
+        wts[r8 * n_chunks + c] = wc;
+        wl += wc * x.y;
+      }
+#pragma unroll
+      for (int o = 8; o < 32; o <<= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
+      named_bar_sync(1, 128);
+      sW[1152 + et] = wl;
+      named_bar_sync(1, 128);
+      if (et < 8) {
+        const float tot = sW[1152 + et] + sW[1152 + 32 + et] + sW[1152 + 64 + et] + sW[1152 + 96 + et];
+        inv[et] = tot > 0.f ? 1.0f / tot : 0.f;
+      }
+      named_bar_sync(1, 128);
     }
+    // features d = 32 w + 4 k + q (k = 0..7) of row hl
+    float acc[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float wl = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMergeChunksPerLane; ++j) {
-      const int c = lane + 32 * j;
-      const float wc = ml[j].y > 0.f ? ex2_approx(ml[j].x - M) : 0.f;
-      if (c < n_chunks) wts[c] = wc;
-      wl += wc * ml[j].y;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
-    __syncwarp();
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* src = reinterpret_cast<const float4*>(fp.apart + base * 128) + lane;
-#pragma unroll 8
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    const float* src = fp.apart + static_cast<size_t>(g) * fp.n_chunks_max * 128 * 128 + t * 8 + hl;
+#pragma unroll 2
     for (int c = 0; c < n_chunks; ++c) {
-      const float wc = wts[c];
-      const float4 f = __ldcg(src + static_cast<size_t>(c) * 128 * 32);
-      acc.x += wc * f.x;
-      acc.y += wc * f.y;
-      acc.z += wc * f.z;
-      acc.w += wc * f.w;
+      const float wc = wts[hl * n_chunks + c];
+      const float* sc = src + static_cast<size_t>(c) * 128 * 128;
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = __ldcg(sc + static_cast<size_t>(32 * w + 4 * k + q) * 128);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] += wc * f[k];
     }
-    const float inv = wl > 0.f ? 1.0f / wl : 0.f;
-    const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    bf16* out = fp.attn_o + static_cast<size_t>(t) * fp.Hq * 128 + h * 128 + lane * 4;
-    *reinterpret_cast<uint2*>(out) =
-        make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
-    __syncwarp();
+    const float iv = inv[hl];
+    bf16* out = fp.attn_o + static_cast<size_t>(t) * fp.Hq * 128 + (g * 8 + hl) * 128 + 32 * w + q;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[4 * k] = __float2bfloat16_rn(acc[k] * iv);
+    named_bar_sync(1, 128);  // the weights are rewritten by the next unit
   }
 }
 
@@ -1368,7 +1401,7 @@ cudaError_t launch_fwd_persistent(const FwdProgram& fp, int P, bool pdl, cudaStr
   if (fp.n_layers < 1 || P < 1 || !fp.bar || !fp.status || !fp.apart || !fp.aml || !fp.attn_o)
     return cudaErrorInvalidValue;
   if (fp.Hq != 8 * fp.Hkv || fp.n_chunks_max < (fp.Lmax + kAttKeys - 1) / kAttKeys ||
-      fp.n_chunks_max > 32 * kMergeChunksPerLane)
+      fp.n_chunks_max > kMergeMaxChunks)
     return cudaErrorInvalidValue;
   for (const ChainPhase* ph : {&fp.qkv, &fp.o, &fp.gu, &fp.down}) {
     if (ph->n_tiles < 1 || ph->kb < 1 || ph->ea.n_rows < 1 || ph->ea.n_rows > kFwdNT || !ph->ea.part ||

@@ -146,6 +146,8 @@ struct ChainPhase {
   CUtensorMap mapA, mapA2, mapB;
   GemmEpi ea;
   int n_tiles, kb, a_row_base;
+  int ctas;  // CTAs that stream the phase (at most the grid): fewer for the narrow products, so that
+             // their split tiles have fewer parts to add (their weights are prefetched anyway)
 };
 struct FwdProgram {
   ChainPhase qkv, o, gu, down;
@@ -157,7 +159,7 @@ struct FwdProgram {
   CUtensorMap mapQ, mapK, mapV;
   int Hq, Hkv, Lmax, n_clean;
   float scale_log2;
-  float* apart;   // [Hkv][n_chunks_max][128 rows][128] unnormalised partial rows (fp32)
+  float* apart;   // [Hkv][n_chunks_max][128 features][128 rows] unnormalised partial rows (fp32)
   float2* aml;    // [Hkv][n_chunks_max][128 rows] (row max, row sum) per 64-key chunk
   int n_chunks_max;
   bf16* attn_o;   // [16][Hq * 128] merged attention rows, the O-projection's input
