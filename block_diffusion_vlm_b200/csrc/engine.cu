@@ -337,9 +337,10 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     fp.o = chain_phase(e->tm_wo, e->tm_wo, e->tm_ao, H / 128, Hq * D / 64, o, e->gcnt + cs);
     fp.gu = chain_phase(e->tm_wg, e->tm_wu, e->tm_x, I / 64, H / 64, g, e->gcnt + 2 * cs);
     fp.down = chain_phase(e->tm_wd, e->tm_wd, e->tm_act, H / 128, I / 64, o, e->gcnt + 3 * cs);
-    // the narrow QKV and O products on half the SMs: half as many parts per
-    // split tile to add, while their weights are prefetched either way
-    fp.qkv.ctas = fp.o.ctas = (e->sm + 1) / 2;
+    // the narrow QKV and O products one tile per CTA (no split tiles to add
+    // up across CTAs; their weights are prefetched during the phases before)
+    fp.qkv.ctas = qkv_rows / 128;
+    fp.o.ctas = H / 128;
     fp.qkv_rows = qkv_rows;
     fp.H = H;
     fp.I = I;

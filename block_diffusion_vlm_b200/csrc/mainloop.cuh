@@ -213,6 +213,7 @@ __device__ void fp8_quantize_activations(int et, const bf16* __restrict__ src, i
                                          const float* rms, const float* amax_in, int n_amax, int kb_lo, int kb_hi,
                                          uint8_t* sB, float* sAt, float* sQm, uint64_t* b_ready) {
   constexpr int TPT = 128 / NT;  // threads per token for the row scan
+  constexpr int SCAN_UNROLL = 16, CODE_UNROLL = 8;  // independent loads in flight per thread
   if (amax_in) {
     if (et < NT) {
       float m = 0.f;
@@ -220,18 +221,27 @@ __device__ void fp8_quantize_activations(int et, const bf16* __restrict__ src, i
       sQm[et] = m;
     }
   } else {
+    // the TPT threads of a token read consecutive 16-byte pieces of its row
     const int t = et / TPT, part = et % TPT;
-    const int per = K / TPT;
+    const int n16 = K / 8;
     float m = 0.f;
     if (t < n_rows) {
-      const uint4* row = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld + part * per);
-      for (int i = 0; i < per / 8; ++i) {
-        const uint4 w = row[i];
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+      const uint4* row = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld);
+      for (int i0 = part; i0 < n16; i0 += TPT * SCAN_UNROLL) {
+        uint4 w[SCAN_UNROLL];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h[q]);
-          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        for (int j = 0; j < SCAN_UNROLL; ++j) {
+          const int i = i0 + j * TPT;
+          w[j] = i < n16 ? row[i] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < SCAN_UNROLL; ++j) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h[q]);
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
         }
       }
     }
@@ -248,28 +258,40 @@ __device__ void fp8_quantize_activations(int et, const bf16* __restrict__ src, i
   }
   named_bar_sync(1, 128);
   const int n_items = (kb_hi - kb_lo) * NT * 8;  // (k block, row, 16-byte chunk)
-  for (int i = et; i < n_items; i += 128) {
-    const int c = i & 7, t = (i >> 3) % NT, b = i / (8 * NT);
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    const float q = sQm[t];
-    if (q != 0.f) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld + (kb_lo + b) * 128 + c * 16);
-      const uint4 w0 = p[0], w1 = p[1];
-      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&w0);
-      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&w1);
+  for (int i0 = et; i0 < n_items; i0 += 128 * CODE_UNROLL) {
+    uint4 w0[CODE_UNROLL], w1[CODE_UNROLL];
+#pragma unroll
+    for (int j = 0; j < CODE_UNROLL; ++j) {
+      const int i = i0 + j * 128;
+      const int c = i & 7, t = (i >> 3) % NT, b = i / (8 * NT);
+      w0[j] = w1[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < n_items && sQm[t] != 0.f) {
+        const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * src_ld + (kb_lo + b) * 128 + c * 16);
+        w0[j] = p[0];
+        w1[j] = p[1];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < CODE_UNROLL; ++j) {
+      const int i = i0 + j * 128;
+      if (i >= n_items) continue;
+      const int c = i & 7, t = (i >> 3) % NT, b = i / (8 * NT);
+      const float q = sQm[t];
+      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&w0[j]);
+      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&w1[j]);
       uint32_t o[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float2 a = __bfloat1622float2(h0[2 * j]), bb = __bfloat1622float2(h0[2 * j + 1]);
-        o[j] = static_cast<uint32_t>(cvt_e4m3x2(a.y * q, a.x * q)) |
+      for (int k = 0; k < 2; ++k) {
+        const float2 a = __bfloat1622float2(h0[2 * k]), bb = __bfloat1622float2(h0[2 * k + 1]);
+        o[k] = static_cast<uint32_t>(cvt_e4m3x2(a.y * q, a.x * q)) |
                (static_cast<uint32_t>(cvt_e4m3x2(bb.y * q, bb.x * q)) << 16);
-        const float2 a2 = __bfloat1622float2(h1[2 * j]), b2 = __bfloat1622float2(h1[2 * j + 1]);
-        o[2 + j] = static_cast<uint32_t>(cvt_e4m3x2(a2.y * q, a2.x * q)) |
+        const float2 a2 = __bfloat1622float2(h1[2 * k]), b2 = __bfloat1622float2(h1[2 * k + 1]);
+        o[2 + k] = static_cast<uint32_t>(cvt_e4m3x2(a2.y * q, a2.x * q)) |
                    (static_cast<uint32_t>(cvt_e4m3x2(b2.y * q, b2.x * q)) << 16);
       }
-      out = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(sB + b * NT * 128 + (t >> 3) * 1024 + (t & 7) * 128 + ((c ^ (t & 7)) << 4)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *reinterpret_cast<uint4*>(sB + b * NT * 128 + (t >> 3) * 1024 + (t & 7) * 128 + ((c ^ (t & 7)) << 4)) = out;
   }
   fence_proxy_async_smem();
   named_bar_sync(1, 128);
