@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-decode tokens/sec at batch 1 (B=16); fused LM-head+commit HBM GB/s vs peak"
 N_VIS, N_PROMPT, N_NEW, BLOCK, TAU, SEED = 1280, 64, 256, 16, 0.9, 4
+ROUTE_K = 2   # certificate-guided routing: positions unmasked per step
 WORKLOAD = "qwen2.5-3b-shaped block-diffusion decode: 36L h2048 16/2x128 ffn11008 V151936, ctx 1280 vision + 64 prompt, 256 new, B=16, tau 0.9"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 FALLBACK_HBM_GBS = 6650.0
@@ -354,8 +355,10 @@ def run_ours(args, rank, world, local, pg):
             print(json.dumps({"profile_forwards": args.profile_forwards, "layers": dims.n_layers}), flush=True)
         return
     mode = {"threshold": dv.MODE_THRESHOLD, "spec": dv.MODE_SPEC_LINEAR, "ar": dv.MODE_AR,
-            "quad": dv.MODE_SPEC_QUAD}[args.mode]
-    cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1)
+            "quad": dv.MODE_SPEC_QUAD, "route": dv.MODE_ROUTE}[args.mode]
+    # routing: k = ROUTE_K positions unmasked per step, the 1280 vision rows
+    # hidden in TEXT-ONLY passes
+    cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1, ROUTE_K, N_VIS)
     out = torch.zeros(N_NEW, dtype=torch.int32, device=dev)
 
     def step(c=cfg):
@@ -440,8 +443,9 @@ def run_ours(args, rank, world, local, pg):
 
     # short runs of the speculative modes for context (same model and context)
     if args.mode == "threshold" and not args.quick:
-        for key, md in (("spec_linear", dv.MODE_SPEC_LINEAR), ("spec_quadratic", dv.MODE_SPEC_QUAD)):
-            sc = dv.DecodeCfg(BLOCK, TAU, md, 1, N_NEW, 1)
+        for key, md in (("spec_linear", dv.MODE_SPEC_LINEAR), ("spec_quadratic", dv.MODE_SPEC_QUAD),
+                        ("route", dv.MODE_ROUTE)):
+            sc = dv.DecodeCfg(BLOCK, TAU, md, 1, N_NEW, 1, ROUTE_K, N_VIS)
             step(sc)
             ev0.record(stream)
             st = step(sc)
@@ -450,9 +454,18 @@ def run_ours(args, rank, world, local, pg):
             secs_sc = ev0.elapsed_time(ev1) / 1000.0
             line[key] = {"tokens_per_s": N_NEW / secs_sc, "nfe": st.nfe, "ms_per_forward": 1000 * secs_sc / st.nfe,
                          "accept_hist": list(st.accept_hist)}
+            if md == dv.MODE_ROUTE:
+                line[key].update(route_k=ROUTE_K, hidden_vision_slots=N_VIS, text_only_passes=st.n_text_passes)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = cpu_baseline(nfe)
     eng.close()
+    # compact single-kernel set (decode-shape and long-cache attention, LM
+    # head rows, speculative accept) on the same GPU, after the decode
+    if rank == 0 and world == 1 and args.mode == "threshold" and not args.quick:
+        cases = []
+        run_sweep(argparse.Namespace(sweep="compact"), local, sink=cases.append)
+        line["sweep"] = [{k: v for k, v in d.items() if k not in ("peak", "peak_source", "timing", "working_set_mb")}
+                         for d in cases]
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -492,13 +505,15 @@ def _device_ms_per_call(fn, reps, dev):
     return e0.elapsed_time(e1) / reps, mode
 
 
-def run_sweep(args, local):
+def run_sweep(args, local, sink=None):
     """Timings of the single-kernel configurations, one JSON line per case:
     block attention for B in {4, 8, 16, 32} x L in {256, 1024, 4096}, both one
     cache per call (L2-resident after the first call) and 36 distinct caches
     in one batched launch (one per decoder layer; the working set exceeds L2
     at L = 4096); the fused LM head + commit for R in {1, 16, 32, 128} rows
-    (its 622 MB of weights exceed L2 on every call)."""
+    (its 622 MB of weights exceed L2 on every call).  `sink`: a callable that
+    receives each case's dict instead of printing it (the compact set that the
+    decode line carries)."""
     import torch
     import block_diffusion_vlm_b200 as dv
     import dvlm_gen as gen
@@ -510,7 +525,10 @@ def run_sweep(args, local):
 
     def emit(d):
         d.update(peak=hbm_peak, peak_source=f"{peak_kind} copy bandwidth")
-        print(json.dumps(d), flush=True)
+        if sink is not None:
+            sink(d)
+        else:
+            print(json.dumps(d), flush=True)
 
     D, Hq, Hkv = dims.head_dim, dims.n_q_heads, dims.n_kv_heads
 
@@ -558,6 +576,10 @@ def run_sweep(args, local):
         groups = nb * ((B + 15) // 16) * Hkv
         return max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
 
+    if args.sweep == "compact":
+        # the decode shape and the bandwidth case, one line each per kernel
+        attn_case(BLOCK, N_VIS + N_PROMPT, 1, [4])
+        attn_case(BLOCK, 4096, dims.n_layers, [2])
     if args.sweep == "attn_long":
         # the bandwidth case alone: 36 caches of 4096 slots in one launch
         attn_case(BLOCK, 4096, dims.n_layers, [2])
@@ -591,7 +613,7 @@ def run_sweep(args, local):
                   "caches_per_launch": dims.n_layers, "us_per_launch": 1000 * ms,
                   "us_per_cache": 1000 * ms / dims.n_layers, "timing": mode})
         del qd, kd, vt, out
-    if args.sweep in ("lmhead", "all"):
+    if args.sweep in ("lmhead", "all", "compact"):
         H, V = dims.hidden, dims.vocab
         _, (w_t, _) = gen.lmhead_case(2, 1, H, V, second_set=False)
         wd = w_t.to(dev)
@@ -634,7 +656,7 @@ def run_sweep(args, local):
 
         ms, mode = _device_ms_per_call(call, 200, dev)
         emit({"sweep": "topk_commit", "R": R, "k": k, "us_per_launch": 1000 * ms, "timing": mode})
-    if args.sweep in ("spec", "all"):
+    if args.sweep in ("spec", "all", "compact"):
         # speculative verify + accept on bf16 logits [b, 16, 151936] (cache
         # lengths updated in place); four input sets in turn, so that b = 8
         # (4 x 38.9 MB) does not run from L2
@@ -720,7 +742,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", choices=["threshold", "spec", "ar", "quad"], default="threshold")
+    ap.add_argument("--mode", choices=["threshold", "spec", "ar", "quad", "route"], default="threshold")
     ap.add_argument("--option", action="append", default=None, metavar="NAME=VALUE",
                     help="engine launch knob (dvlm_engine_set_option), e.g. attn_split=8; repeatable")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
@@ -730,7 +752,7 @@ def main():
     ap.add_argument("--layers", type=int, default=36, help="decoder depth (36 = the benchmarked model)")
     ap.add_argument("--profile-forwards", type=int, default=0,
                     help="profiling case: run this many eager forwards after prefill and exit")
-    ap.add_argument("--sweep", choices=["attention", "attn_decode", "attn_long", "lmhead", "spec", "tiny", "all"], default=None,
+    ap.add_argument("--sweep", choices=["attention", "attn_decode", "attn_long", "compact", "lmhead", "spec", "tiny", "all"], default=None,
                     help="time the single-kernel configurations (one JSON line per case) instead of the decode")
     args = ap.parse_args()
     rank, world, local, pg = dist_setup()

@@ -198,3 +198,42 @@ def test_sweep_prints_one_line_per_case(monkeypatch, capsys):
     assert all(d["bytes_per_launch"] == d["b"] * 16 * 151936 * 2 + 2 * d["b"] * 16 * 4 for d in sp)
     tiny = [d for d in lines if d["sweep"] == "tiny_step"]
     assert len(tiny) == 1 and tiny[0]["B"] == 4 and tiny[0]["ms_per_block"] > 0
+
+
+def test_full_line_carries_modes_and_compact_sweep(monkeypatch, capsys):
+    """Without --quick the decode line also times the speculative modes and
+    routing on the same engine, and carries the compact single-kernel set
+    (run_sweep in collecting mode, here a stand-in)."""
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    import block_diffusion_vlm_b200 as dv
+    import dvlm_gen.device as gdev
+    real_device = torch.device
+    monkeypatch.setattr(torch, "device", lambda *a, **k: real_device("cpu"))
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "Stream", _Stream)
+    monkeypatch.setattr(torch.cuda, "Event", _Event)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(dv, "Engine", _FakeEngine)
+    monkeypatch.setattr(dv, "engine_workspace_size", lambda *a: 64)
+    monkeypatch.setattr(gdev, "DeviceModel", _FakeDeviceModel)
+    monkeypatch.setattr(gdev, "kv_buffers", lambda *a, **k: (None, None))
+    monkeypatch.setattr(bench, "gpu_uuid", lambda: None)
+    seen = []
+
+    def fake_sweep(a, local, sink=None):
+        seen.append(a.sweep)
+        sink({"sweep": "lm_head", "R": 16, "us_per_launch": 100.0, "peak": 1.0, "timing": "eager"})
+
+    monkeypatch.setattr(bench, "run_sweep", fake_sweep)
+    args = bench.argparse.Namespace(steps=5, warmup=3, mode="threshold", quick=False, no_cpu_baseline=True,
+                                    layers=36, profile_forwards=0, impl="ours", gpus=1, sweep=None, weights="bf16",
+                                    option=None)
+    bench.run_ours(args, 0, 1, 0, None)
+    d = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")][0])
+    assert seen == ["compact"]
+    assert d["sweep"] == [{"sweep": "lm_head", "R": 16, "us_per_launch": 100.0}]
+    for key in ("spec_linear", "spec_quadratic", "route"):
+        assert d[key]["nfe"] == 71 and d[key]["tokens_per_s"] > 0
+    assert d["route"]["route_k"] == bench.ROUTE_K and d["route"]["hidden_vision_slots"] == 1280
