@@ -42,23 +42,39 @@ __device__ __forceinline__ float fp8_row_scale(const GemmEpi& ea, bool split, in
 
 // RMSNorm factors of the NT input rows from the producers' per-tile sums of
 // squares (ssq_in [n_ssq][NT]), run by the 128 epilogue threads: 128 / NT
-// partial sums per row with independent loads, then one thread per row adds
-// the partials in order.  sPart: 128 floats of scratch.
+// partial sums per row, each thread's loads issued together (up to 16 of
+// them in flight), then one thread per row adds the partials in order.
+// sPart: 128 floats of scratch.
 template <int NT>
-__device__ __forceinline__ void ws_rms_factors(const GemmEpi& ea, int et, float* sR, float* sPart) {
+__device__ __forceinline__ void rms_factors(const float* ssq_in, int n_ssq, float inv_h, float eps, int et,
+                                            float* sR, float* sPart) {
   constexpr int G = 128 / NT;
+  constexpr int BATCH = 16;
   const int t = et % NT, g = et / NT;
   float s = 0.f;
-  for (int q = g; q < ea.n_ssq; q += G) s += __ldcg(&ea.ssq_in[q * NT + t]);
+  for (int q0 = g; q0 < n_ssq; q0 += G * BATCH) {
+    float v[BATCH];
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int q = q0 + j * G;
+      v[j] = q < n_ssq ? __ldcg(&ssq_in[q * NT + t]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) s += v[j];
+  }
   sPart[g * NT + t] = s;
   named_bar_sync(1, 128);
   if (et < NT) {
     float tot = 0.f;
 #pragma unroll
     for (int k = 0; k < G; ++k) tot += sPart[k * NT + et];
-    sR[et] = 1.0f / sqrtf(tot * ea.inv_h + ea.eps);
+    sR[et] = 1.0f / sqrtf(tot * inv_h + eps);
   }
   named_bar_sync(1, 128);
+}
+template <int NT>
+__device__ __forceinline__ void ws_rms_factors(const GemmEpi& ea, int et, float* sR, float* sPart) {
+  rms_factors<NT>(ea.ssq_in, ea.n_ssq, ea.inv_h, ea.eps, et, sR, sPart);
 }
 
 // The epilogue warps' work for the stream-K units [u0, u1) of one GEMM:
@@ -452,11 +468,7 @@ __global__ void __launch_bounds__(kWsThreads, NT <= 16 ? 2 : 1)
     // Dependents may start only once this kernel's own inputs are complete,
     // so at most two kernels of the chain overlap (see ptx.cuh).
     if (et == 0) griddep_launch_dependents();
-    if (EPI == EPI_QKV && et < NT) {
-      float s2 = 0.f;
-      for (int p = 0; p < ea.n_ssq; ++p) s2 += ea.ssq_in[p * NT + et];
-      sR[et] = 1.0f / sqrtf(s2 * ea.inv_h + ea.eps);
-    }
+    if (EPI == EPI_QKV) rms_factors<NT>(ea.ssq_in, ea.n_ssq, ea.inv_h, ea.eps, et, sR, sQ);
     if (FP8)
       fp8_quantize_activations<NT>(et, ea.q_src, ea.q_ld, ea.q_K, ea.n_rows, ea.rms_input ? sR : nullptr,
                                    ea.amax_in, ea.n_amax, kb_lo, kb_hi, sB, sAt, sQm, b_ready);
