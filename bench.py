@@ -288,6 +288,8 @@ def workload_config(args, world: int) -> dict:
     c = {"workload": WORKLOAD, "global_batch": world, "seq_len": N_VIS + N_PROMPT + N_NEW,
          "parallelism": f"replicas x{world}", "mode": args.mode,
          "l2": "inputs larger than L2 (6.2 GB of weights streamed per forward)"}
+    if getattr(args, "block", BLOCK) != BLOCK:
+        c["block"] = args.block
     if getattr(args, "weights", "bf16") != "bf16":
         c["weights"] = "fp8-w8a8 (E4M3 projections, per-row / per-token scales; bf16 LM head)"
     return c
@@ -358,7 +360,8 @@ def run_ours(args, rank, world, local, pg):
             "quad": dv.MODE_SPEC_QUAD, "route": dv.MODE_ROUTE}[args.mode]
     # routing: k = ROUTE_K positions unmasked per step, the 1280 vision rows
     # hidden in TEXT-ONLY passes
-    cfg = dv.DecodeCfg(BLOCK, TAU, mode, 1, N_NEW, 1, ROUTE_K, N_VIS)
+    block = getattr(args, "block", BLOCK)
+    cfg = dv.DecodeCfg(block, TAU, mode, 1, N_NEW, 1, ROUTE_K, N_VIS)
     out = torch.zeros(N_NEW, dtype=torch.int32, device=dev)
 
     def step(c=cfg):
@@ -743,6 +746,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--mode", choices=["threshold", "spec", "ar", "quad", "route"], default="threshold")
+    ap.add_argument("--block", type=int, default=BLOCK,
+                    help="block size B of the timed decode (the benchmarked configuration: 16)")
     ap.add_argument("--option", action="append", default=None, metavar="NAME=VALUE",
                     help="engine launch knob (dvlm_engine_set_option), e.g. attn_split=8; repeatable")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
