@@ -13,7 +13,10 @@
 // pass and a 16-row verify pass give bitwise the same output).  Each of the S
 // CTAs of a (batch entry, row group, KV head) streams its chunks through a
 // 2-stage TMA pipeline (S = Q K^T and O += P V in TMEM, online softmax in
-// fp32 with one thread per row, P and V in fp16 for the second product),
+// fp32 with two threads per row, one per 64-key half, P and V in fp16 for
+// the second product; the running maximum moves only when a score passes it
+// by more than 2^8, which leaves the result exact up to rounding and skips
+// most rescales of O),
 // then stores its partial rows (O / l in fp32, and (m, l)) to global scratch
 // and counts itself on the group's counter; the last CTA to arrive merges the
 // S partials in split order (deterministic) and writes the bf16 output.  No
@@ -27,7 +30,9 @@
 namespace dvlm {
 
 namespace {
-constexpr int kSpThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one row each)
+constexpr int kSpThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (two per TMEM lane quarter)
+constexpr int kSpSoftmax = 256;        // softmax threads: row = quarter * 32 + lane, key half = (warp - 2) / 4
+constexpr float kSpLazy = 8.0f;        // log2 headroom before the running maximum moves
 constexpr int kSpKeys = 128;           // keys per chunk
 constexpr int kSpAtom = 128 * 128;     // one 128-byte-swizzled 128-row operand atom (16 KB)
 constexpr int oSpQ = 0;                // Q: 2 atoms (d 0..63, 64..127)
@@ -35,7 +40,8 @@ constexpr int oSpK = oSpQ + 2 * kSpAtom;   // K: 2 stages x 2 d-atoms
 constexpr int oSpV = oSpK + 4 * kSpAtom;   // V^T: 2 stages x 2 key-atoms
 constexpr int oSpP = oSpV + 4 * kSpAtom;   // P: 2 key-atoms
 constexpr int oSpBar = oSpP + 2 * kSpAtom;
-constexpr int kSpSmem = oSpBar + 256 + 1024;
+constexpr int oSpL = oSpBar + 256;     // [2][128] row sums of the two key halves
+constexpr int kSpSmem = oSpL + 1024 + 1024;
 constexpr uint32_t kSpIdescS = idesc_bf16_f32(128, kSpKeys);
 constexpr uint32_t kSpIdescO = idesc_f16_f32(128, 128);
 constexpr int kSpTmem = 512;           // S: 2 x 128 columns, O: 128 columns
@@ -68,6 +74,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
+  float* sLh = reinterpret_cast<float*>(smem + oSpL);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = gridDim.x, sp = blockIdx.x, g = blockIdx.y;
@@ -88,7 +95,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 4 : 1);
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 8 : 1);
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -161,30 +168,58 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         umma_commit(pv_done);
         return true;
       };
-      for (int c = 0; ok && c < nc; ++c) {
-        const int st = c & 1;
-        if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) break;
-        if (c >= 2 && !mbar_wait(&s_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kSpAtom);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
-          umma_bf16_ss(tmem + st * kSpKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off), kSpIdescS,
-                       kk > 0 ? 1u : 0u);
+      // Issue whichever product is ready: PV of the oldest chunk with its P
+      // written (that frees its K/V stage for the load two chunks ahead), else
+      // S of the next chunk with its keys landed and its S buffer free.  A
+      // fixed S(c), PV(c-1) order would hold every load back until the
+      // previous one landed.
+      int cs = 0, cp = 0;
+      long long t0 = clock64();
+      while (ok && cp < nc) {
+        if (cp < cs && mbar_test_wait(p_full, cp & 1)) {
+          ok = issue_pv(cp);
+          ++cp;
+          t0 = clock64();
+          continue;
         }
-        umma_commit(&s_full[st]);
-        if (c >= 1) ok = issue_pv(c - 1);
+        if (cs < nc && cs <= cp + 1) {
+          const int st = cs & 1;
+          if (mbar_test_wait(&kv_full[st], (cs >> 1) & 1) &&
+              (cs < 2 || mbar_test_wait(&s_empty[st], ((cs >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kSpAtom);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
+              umma_bf16_ss(tmem + st * kSpKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off),
+                           kSpIdescS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[st]);
+            ++cs;
+            t0 = clock64();
+            continue;
+          }
+        }
+        if (*sabort || clock64() - t0 > kWaitBudgetCycles) {
+          record_error(a.status, DVLM_ERR_TIMEOUT);
+          *sabort = 1;
+          ok = false;
+        }
       }
-      if (ok) issue_pv(nc - 1);
     }
   } else {
     // ---------------------------------------------------------------- softmax
+    // Two warps per TMEM lane quarter: warp half `hf` exponentiates keys
+    // 64 hf .. 64 hf + 63 of each chunk (P atom hf), rescales output features
+    // 64 hf .. 64 hf + 63 and converts value atom hf.  Both warps of a quarter
+    // take the row maximum over all 128 keys, so they hold the same (m, alpha)
+    // without exchanging it; each keeps the row sum of its own keys.
     // The next kernel (the output projection) may launch now and stream its
     // weights on idle SMs; it reads this kernel's output only after its own
     // wait (at most two kernels overlap).
     if (threadIdx.x == 64) griddep_launch_dependents();
     const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const int t = t_base + (row >> 3);
     const int limit = (t < a.n_clean) ? (L + t + 1) : Ltot;  // keys below `limit` are visible
@@ -194,37 +229,56 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     for (int c = 0; ok && c < nc; ++c) {
       const int st = c & 1;
       const int key0 = (sp + c * S) * kSpKeys;
+      const bool full = key0 + kSpKeys <= limit;  // every key of the chunk visible to this row
       if (!mbar_wait(&s_full[st], (c >> 1) & 1, a.status, sabort)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float sc[64], so[64];  // this warp's keys; the other half's keys (maximum only)
+      tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
+      tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + (hf ^ 1) * 64), so);
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        float sc[64];
-        tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
+      if (full) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (key0 + hf * 64 + k < limit) mx = fmaxf(mx, sc[k] * a.scale_log2);
+        for (int k = 0; k < 64; ++k) mx = fmaxf(mx, fmaxf(sc[k], so[k]));
+      } else {
+        const int kme = key0 + hf * 64, koth = key0 + (hf ^ 1) * 64;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          if (kme + k < limit) mx = fmaxf(mx, sc[k]);
+          if (koth + k < limit) mx = fmaxf(mx, so[k]);
+        }
       }
-      const float m_new = fmaxf(m, mx);
+      // scale_log2 > 0, so the maximum of the scaled scores is the scaled
+      // maximum (rounding is monotonic).  The reference maximum moves only
+      // when a score exceeds it by more than 2^kLazy: below that the
+      // probabilities stay <= 2^kLazy (exact range for fp16 P and the fp32
+      // sums), and the output needs no rescale.
+      const float m_cand = fmaxf(m, mx * a.scale_log2);
+      const float m_new = (m == -INFINITY || m_cand > m + kSpLazy) ? m_cand : m;
       const float alpha = (m == -INFINITY) ? (m_new == -INFINITY ? 1.f : 0.f) : exp2f(m - m_new);
-      uint32_t packed[64];
+      uint32_t packed[32];
       float psum = 0.f;
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float sc[64];
-        tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
+      if (full) {
 #pragma unroll
         for (int k = 0; k < 64; k += 2) {
-          const int key = key0 + hf * 64 + k;
-          const float p0 = (key < limit && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
-          const float p1 =
-              (key + 1 < limit && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
+          const float p0 = ex2_approx(sc[k] * a.scale_log2 - m_new);
+          const float p1 = ex2_approx(sc[k + 1] * a.scale_log2 - m_new);
           psum += p0 + p1;
           const __half2 ph = __floats2half2_rn(p0, p1);
-          packed[hf * 32 + k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
+          packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
+        }
+      } else {
+        const int kme = key0 + hf * 64;
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float p0 = (kme + k < limit && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
+          const float p1 =
+              (kme + k + 1 < limit && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
+          psum += p0 + p1;
+          const __half2 ph = __floats2half2_rn(p0, p1);
+          packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
       }
       tc_fence_before();
@@ -237,52 +291,45 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll 1
-          for (int cc = 0; cc < 128; cc += 64) {
-            float o[64];
-            tmem_ld64(tmem + lane_off + 256u + cc, o);
+          float o[64];
+          tmem_ld64(tmem + lane_off + 256u + static_cast<uint32_t>(hf * 64), o);
 #pragma unroll
-            for (int k = 0; k < 64; ++k) o[k] *= alpha;
+          for (int k = 0; k < 64; ++k) o[k] *= alpha;
 #pragma unroll
-            for (int k = 0; k < 64; k += 16) tmem_st16_nowait(tmem + lane_off + 256u + cc + k, o + k);
-            tmem_wait_st();
-          }
+          for (int k = 0; k < 64; k += 16) tmem_st16_nowait(tmem + lane_off + 256u + hf * 64 + k, o + k);
+          tmem_wait_st();
         }
       }
-#pragma unroll
-      for (int at = 0; at < 2; ++at) {
-        uint8_t* prow = sP + at * kSpAtom + row * 128;
+      {
+        uint8_t* prow = sP + hf * kSpAtom + row * 128;
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
-              make_uint4(packed[at * 32 + cc * 4], packed[at * 32 + cc * 4 + 1], packed[at * 32 + cc * 4 + 2],
-                         packed[at * 32 + cc * 4 + 3]);
+              make_uint4(packed[cc * 4], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
       }
-      // value row `row` (feature d = row) of this chunk to fp16 in place; keys
-      // past the valid slots (stale, poisoned, other pages' rows) become 0
+      // value row `row` (feature d = row) of this warp's 64 keys to fp16 in
+      // place; keys past the valid slots (stale, poisoned, other pages' rows)
+      // become 0
       if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) {
         ok = false;
         break;
       }
       {
-        const int n_valid = Ltot - key0;
+        const int n_valid = Ltot - key0 - hf * 64;
+        uint8_t* vrow = sV + (2 * st + hf) * kSpAtom + row * 128;
 #pragma unroll
-        for (int at = 0; at < 2; ++at) {
-          uint8_t* vrow = sV + (2 * st + at) * kSpAtom + row * 128;
+        for (int cc = 0; cc < 8; ++cc) {
+          uint4* p16 = reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4));
+          uint4 w = *p16;
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint4* p16 = reinterpret_cast<uint4*>(vrow + (cc << 4));
-            uint4 w = *p16;
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
-              const int kk = at * 64 + ((cc ^ (row & 7)) << 3) + 2 * e;
-              const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
-              wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
-            }
-            *p16 = w;
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            const int kk = (cc << 3) + 2 * e;
+            const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
+            wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
           }
+          *p16 = w;
         }
       }
       fence_proxy_async_smem();
@@ -292,75 +339,93 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       l = l * alpha + psum;
       m = m_new;
     }
-    // this split's partial rows: O / l (fp32) and (m, l)
+    // this split's partial rows: O / l (fp32, each warp its 64 features) and
+    // (m, l), l the two halves' sums added in half order
     const size_t pidx = static_cast<size_t>(grp) * S + sp;
-    float* prow = part + (pidx * 128 + row) * 128;
+    float* prow = part + (pidx * 128 + row) * 128 + hf * 64;
     const bool have = ok && nc > 0 && mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort);
+    sLh[hf * 128 + row] = l;
+    named_bar_sync(1, kSpSoftmax);
+    l = sLh[row] + sLh[128 + row];
     if (have) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 64) {
-        float o[64];
-        tmem_ld64(tmem + lane_off + 256u + cc, o);
+      float o[64];
+      tmem_ld64(tmem + lane_off + 256u + static_cast<uint32_t>(hf * 64), o);
 #pragma unroll
-        for (int k = 0; k < 64; k += 4)
-          __stcg(reinterpret_cast<float4*>(prow + cc + k),
-                 make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l));
-      }
+      for (int k = 0; k < 64; k += 4)
+        __stcg(reinterpret_cast<float4*>(prow + k),
+               make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l));
     }
-    ml[pidx * 128 + row] = (have && l > 0.f) ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+    if (hf == 0) ml[pidx * 128 + row] = (have && l > 0.f) ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
     __threadfence();
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kSpSoftmax);
     if (threadIdx.x == 64) *sflag = (atomicAdd(&cnt[grp], 1) == S - 1) ? 1 : 0;
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kSpSoftmax);
     if (*sflag) {
       // ------------------------------------------------------------ merge
       // (m, l) of every split and row into shared memory (the K stages are
       // free now), each row's weights w_q = 2^(m_q - M) l_q in place of m_q;
-      // then one warp per row, its 128 values as 32 lanes x 4, the splits'
-      // partials (independent, coalesced 512-byte loads) summed in split order
+      // then the partials (independent, coalesced 512-byte loads) summed in
+      // split order
       __threadfence();
       if (threadIdx.x == 64) cnt[grp] = 0;  // every split arrived: zero for the next launch
       const int et = threadIdx.x - 64;
       const size_t p0 = static_cast<size_t>(grp) * S;
       float2* sml = reinterpret_cast<float2*>(sK);  // [S][128]
       float* sinv = reinterpret_cast<float*>(sV);   // [128]
-      for (int i = et; i < S * 128; i += 128) sml[i] = __ldcg(&ml[p0 * 128 + i]);
-      named_bar_sync(1, 128);
-      {
+      for (int i = et; i < S * 128; i += kSpSoftmax) sml[i] = __ldcg(&ml[p0 * 128 + i]);
+      named_bar_sync(1, kSpSoftmax);
+      if (et < 128) {
         float M = -INFINITY;
-        for (int q = 0; q < S; ++q) M = fmaxf(M, sml[q * 128 + row].x);
+        for (int q = 0; q < S; ++q) M = fmaxf(M, sml[q * 128 + et].x);
         float wsum = 0.f;
         for (int q = 0; q < S; ++q) {
-          const float2 v = sml[q * 128 + row];
+          const float2 v = sml[q * 128 + et];
           const float w = v.y > 0.f ? ex2_approx(v.x - M) * v.y : 0.f;
-          sml[q * 128 + row].x = w;
+          sml[q * 128 + et].x = w;
           wsum += w;
         }
-        sinv[row] = wsum > 0.f ? 1.0f / wsum : 0.f;
+        sinv[et] = wsum > 0.f ? 1.0f / wsum : 0.f;
       }
-      named_bar_sync(1, 128);
-      for (int r = et >> 5; r < 128; r += 4) {
-        const int tr = t_base + (r >> 3);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4* src = reinterpret_cast<const float4*>(part + (p0 * 128 + r) * 128) + lane;
-#pragma unroll 4
+      named_bar_sync(1, kSpSoftmax);
+      // warp w merges rows 16w .. 16w+15, eight rows at a time, so each warp
+      // keeps 8 (x 2 splits) independent loads in flight
+      constexpr int kRB = 8;
+      const int wq = et >> 5;
+#pragma unroll 1
+      for (int r0 = wq * 16; r0 < wq * 16 + 16; r0 += kRB) {
+        float4 acc[kRB];
+#pragma unroll
+        for (int j = 0; j < kRB; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4* src = reinterpret_cast<const float4*>(part + (p0 * 128 + r0) * 128) + lane;
+#pragma unroll 2
         for (int q = 0; q < S; ++q) {
-          const float w = sml[q * 128 + r].x;
-          const float4 f = __ldcg(src + static_cast<size_t>(q) * 128 * 32);
-          acc.x += w * f.x;
-          acc.y += w * f.y;
-          acc.z += w * f.z;
-          acc.w += w * f.w;
+          float4 f[kRB];
+#pragma unroll
+          for (int j = 0; j < kRB; ++j) f[j] = __ldcg(src + (static_cast<size_t>(q) * 128 + j) * 32);
+#pragma unroll
+          for (int j = 0; j < kRB; ++j) {
+            const float w = sml[q * 128 + r0 + j].x;
+            acc[j].x += w * f[j].x;
+            acc[j].y += w * f[j].y;
+            acc[j].z += w * f[j].z;
+            acc[j].w += w * f[j].w;
+          }
         }
-        if (tr < a.n_rows) {
-          const float inv = sinv[r];
-          bf16* dst = a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + lane * 4;
-          const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-          const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2*>(dst) =
-              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+#pragma unroll
+        for (int j = 0; j < kRB; ++j) {
+          const int r = r0 + j;
+          const int tr = t_base + (r >> 3);
+          if (tr < a.n_rows) {
+            const float inv = sinv[r];
+            bf16* dst =
+                a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + lane * 4;
+            const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[j].x * inv, acc[j].y * inv);
+            const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[j].z * inv, acc[j].w * inv);
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+          }
         }
       }
     }

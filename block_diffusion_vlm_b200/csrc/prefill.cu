@@ -440,22 +440,42 @@ __global__ void __launch_bounds__(kPaThreads, 1)
         umma_commit(pv_done);
         return true;
       };
-      for (int c = 0; ok && c < nc; ++c) {
-        const int st = c & 1;
-        if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) break;
-        if (c >= 2 && !mbar_wait(&s_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kPaAtom);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kPaAtom + (kk & 3) * 32;
-          umma_bf16_ss(tmem + st * kPaKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off), kPaIdescS,
-                       kk > 0 ? 1u : 0u);
+      // Issue whichever product is ready (PV of the oldest chunk with its P
+      // written first: that frees its K/V stage for the load two chunks
+      // ahead), so consecutive loads overlap instead of queueing behind S.
+      int cs = 0, cp = 0;
+      long long t0 = clock64();
+      while (ok && cp < nc) {
+        if (cp < cs && mbar_test_wait(p_full, cp & 1)) {
+          ok = issue_pv(cp);
+          ++cp;
+          t0 = clock64();
+          continue;
         }
-        umma_commit(&s_full[st]);
-        if (c >= 1) ok = issue_pv(c - 1);
+        if (cs < nc && cs <= cp + 1) {
+          const int st = cs & 1;
+          if (mbar_test_wait(&kv_full[st], (cs >> 1) & 1) &&
+              (cs < 2 || mbar_test_wait(&s_empty[st], ((cs >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kPaAtom);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kPaAtom + (kk & 3) * 32;
+              umma_bf16_ss(tmem + st * kPaKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off),
+                           kPaIdescS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[st]);
+            ++cs;
+            t0 = clock64();
+            continue;
+          }
+        }
+        if (*sabort || clock64() - t0 > kWaitBudgetCycles) {
+          record_error(a.status, DVLM_ERR_TIMEOUT);
+          *sabort = 1;
+          ok = false;
+        }
       }
-      if (ok) issue_pv(nc - 1);
     }
   } else {
     // ---------------------------------------------------------------- softmax
@@ -558,14 +578,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
           uint8_t* vrow = sV + (2 * st + at) * kPaAtom + row * 128;
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
-            uint4* p16 = reinterpret_cast<uint4*>(vrow + (cc << 4));
+            uint4* p16 = reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4));
             uint4 w = *p16;
             uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
-              // 16-byte chunk cc of this 128-byte row holds keys ((cc ^ (row & 7)) * 8 + 2e, +1)
-              const int kk = at * 64 + ((cc ^ (row & 7)) << 3) + 2 * e;
+              // keys 8 cc + 2e, +1 sit in 16-byte chunk cc ^ (row & 7) of this 128-byte row
+              const int kk = at * 64 + (cc << 3) + 2 * e;
               const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
               wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
             }
