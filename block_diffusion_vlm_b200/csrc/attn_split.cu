@@ -33,6 +33,7 @@ namespace {
 constexpr int kSpThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (two per TMEM lane quarter)
 constexpr int kSpSoftmax = 256;        // softmax threads: row = quarter * 32 + lane, key half = (warp - 2) / 4
 constexpr float kSpLazy = 8.0f;        // log2 headroom before the running maximum moves
+constexpr int kSpPrefetch = 4;         // L2 prefetch distance in chunks past the newest load
 constexpr int kSpKeys = 128;           // keys per chunk
 constexpr int kSpAtom = 128 * 128;     // one 128-byte-swizzled 128-row operand atom (16 KB)
 constexpr int oSpQ = 0;                // Q: 2 atoms (d 0..63, 64..127)
@@ -65,13 +66,15 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint8_t* sP = smem + oSpP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oSpBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2] PV of the chunk in that stage done
+  uint64_t* k_full = bars + 1;    // [2] keys of the chunk in that stage landed
+  uint64_t* k_empty = bars + 3;   // [2] S of the chunk in that stage done (its keys are free)
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_empty = bars + 7;   // [2] the softmax warps have read S of that buffer
   uint64_t* p_full = bars + 9;    // P of the current chunk written, O rescaled (one phase per chunk)
   uint64_t* pv_done = bars + 10;  // PV of a chunk done (one phase per chunk)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* v_full = bars + 11;   // [2] values of the chunk in that stage landed
+  uint64_t* v_empty = bars + 13;  // [2] PV of the chunk in that stage done (its values are free)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
   float* sLh = reinterpret_cast<float*>(smem + oSpL);
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 8 : 1);
+    for (int i = 0; i < 15; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 8 : 1);
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -127,27 +130,64 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       mbar_arrive_expect_tx(q_full, 2 * kSpAtom);
       for (int d = 0; d < 2; ++d)
         tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, bidx * a.n_rows + t_base, pol);
-      for (int c = 0; c < nc; ++c) {
+      // coordinates of 64-key half `hf` of this CTA's chunk c (one page each
+      // in a paged cache)
+      auto coords = [&](int c, int hf, int& krow, int& vrow, int& vx) {
+        const int key = (sp + c * S) * kSpKeys + hf * 64;
+        if (a.block_table) {
+          const int pe = page_entry(key);
+          krow = pe * 64;
+          vrow = pe * 128;
+          vx = 0;
+        } else {
+          krow = kv_row0 * a.Lmax + key;
+          vrow = kv_row0 * 128;
+          vx = key;
+        }
+      };
+      // Keys and values have two stages each, released separately: a key
+      // stage as soon as S of its chunk is done, a value stage once PV is.
+      // Keys therefore run one chunk ahead of values (K(i) is issued before
+      // V(i - 1), the order in which their stages free up).  The chunks after
+      // the loaded ones are prefetched into L2 (up to kSpPrefetch ahead of the
+      // newest key load), so a refill reads L2 instead of DRAM.
+      auto load_k = [&](int c) {
         const int st = c & 1;
-        if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
-        mbar_arrive_expect_tx(&kv_full[st], 4 * kSpAtom);
-        const int key0 = (sp + c * S) * kSpKeys;
-        for (int hf = 0; hf < 2; ++hf) {  // 64-key halves: one page each in a paged cache
-          const int key = key0 + hf * 64;
+        mbar_arrive_expect_tx(&k_full[st], 2 * kSpAtom);
+        for (int hf = 0; hf < 2; ++hf) {
           int krow, vrow, vx;
-          if (a.block_table) {
-            const int pe = page_entry(key);
-            krow = pe * 64;
-            vrow = pe * 128;
-            vx = 0;
-          } else {
-            krow = kv_row0 * a.Lmax + key;
-            vrow = kv_row0 * 128;
-            vx = key;
-          }
+          coords(c, hf, krow, vrow, vx);
           for (int d = 0; d < 2; ++d)
-            tma_load_2d(sK + (2 * st + d) * kSpAtom + hf * (kSpAtom / 2), &mapK, &kv_full[st], d * 64, krow, pol);
-          tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &kv_full[st], vx, vrow, pol);
+            tma_load_2d(sK + (2 * st + d) * kSpAtom + hf * (kSpAtom / 2), &mapK, &k_full[st], d * 64, krow, pol);
+        }
+      };
+      auto load_v = [&](int c) {
+        const int st = c & 1;
+        mbar_arrive_expect_tx(&v_full[st], 2 * kSpAtom);
+        for (int hf = 0; hf < 2; ++hf) {
+          int krow, vrow, vx;
+          coords(c, hf, krow, vrow, vx);
+          tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &v_full[st], vx, vrow, pol);
+        }
+      };
+      int pf = 2;
+      for (int i = 0; i <= nc; ++i) {
+        if (i < nc) {
+          if (i >= 2 && !mbar_wait(&k_empty[i & 1], ((i >> 1) - 1) & 1, a.status, sabort)) break;
+          load_k(i);
+          for (; pf < nc && pf <= i + kSpPrefetch; ++pf) {
+            for (int hf = 0; hf < 2; ++hf) {
+              int krow, vrow, vx;
+              coords(pf, hf, krow, vrow, vx);
+              for (int d = 0; d < 2; ++d) tma_prefetch_2d(&mapK, d * 64, krow);
+              tma_prefetch_2d(&mapV, vx, vrow);
+            }
+          }
+        }
+        if (i >= 1) {
+          const int c = i - 1;
+          if (c >= 2 && !mbar_wait(&v_empty[c & 1], ((c >> 1) - 1) & 1, a.status, sabort)) break;
+          load_v(c);
         }
       }
     }
@@ -164,7 +204,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           umma_bf16_ss(tmem + 256, sdesc_kmajor_sw128(pa + off), sdesc_kmajor_sw128(vb + off), kSpIdescO,
                        (c > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[c & 1]);
+        umma_commit(&v_empty[c & 1]);
         umma_commit(pv_done);
         return true;
       };
@@ -184,7 +224,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         if (cs < nc && cs <= cp + 1) {
           const int st = cs & 1;
-          if (mbar_test_wait(&kv_full[st], (cs >> 1) & 1) &&
+          if (mbar_test_wait(&k_full[st], (cs >> 1) & 1) &&
               (cs < 2 || mbar_test_wait(&s_empty[st], ((cs >> 1) - 1) & 1))) {
             tc_fence_after();
             const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kSpAtom);
@@ -194,6 +234,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
               umma_bf16_ss(tmem + st * kSpKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off),
                            kSpIdescS, kk > 0 ? 1u : 0u);
             }
+            umma_commit(&k_empty[st]);
             umma_commit(&s_full[st]);
             ++cs;
             t0 = clock64();
@@ -310,27 +351,39 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       // value row `row` (feature d = row) of this warp's 64 keys to fp16 in
       // place; keys past the valid slots (stale, poisoned, other pages' rows)
       // become 0
-      if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) {
+      if (!mbar_wait(&v_full[st], (c >> 1) & 1, a.status, sabort)) {
         ok = false;
         break;
       }
       {
+        // all eight 16-byte pieces loaded first, then converted, then stored
+        // (independent shared-memory round trips)
         const int n_valid = Ltot - key0 - hf * 64;
         uint8_t* vrow = sV + (2 * st + hf) * kSpAtom + row * 128;
+        uint4 w[8];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint4* p16 = reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4));
-          uint4 w = *p16;
-          uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+        for (int cc = 0; cc < 8; ++cc) w[cc] = *reinterpret_cast<const uint4*>(vrow + ((cc ^ (row & 7)) << 4));
+        if (n_valid >= 64) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
-            const int kk = (cc << 3) + 2 * e;
-            const __half2 hh = __floats2half2_rn(kk < n_valid ? f.x : 0.f, kk + 1 < n_valid ? f.y : 0.f);
-            wv[e] = *reinterpret_cast<const uint32_t*>(&hh);
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wv[e] = bf16x2_to_f16x2(wv[e]);
           }
-          *p16 = w;
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int kk = (cc << 3) + 2 * e;
+              const uint32_t keep = (kk < n_valid ? 0x0000FFFFu : 0u) | (kk + 1 < n_valid ? 0xFFFF0000u : 0u);
+              wv[e] = bf16x2_to_f16x2(wv[e] & keep);
+            }
+          }
         }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4)) = w[cc];
       }
       fence_proxy_async_smem();
       tc_fence_before();
