@@ -39,13 +39,16 @@ constexpr int kSpAtom = 128 * 128;     // one 128-byte-swizzled 128-row operand 
 constexpr int oSpQ = 0;                // Q: 2 atoms (d 0..63, 64..127)
 constexpr int oSpK = oSpQ + 2 * kSpAtom;   // K: 2 stages x 2 d-atoms
 constexpr int oSpV = oSpK + 4 * kSpAtom;   // V^T: 2 stages x 2 key-atoms
-constexpr int oSpP = oSpV + 4 * kSpAtom;   // P: 2 key-atoms
-constexpr int oSpBar = oSpP + 2 * kSpAtom;
+constexpr int oSpBar = oSpV + 4 * kSpAtom;
 constexpr int oSpL = oSpBar + 256;     // [2][128] row sums of the two key halves
 constexpr int kSpSmem = oSpL + 1024 + 1024;
 constexpr uint32_t kSpIdescS = idesc_bf16_f32(128, kSpKeys);
 constexpr uint32_t kSpIdescO = idesc_f16_f32(128, 128);
-constexpr int kSpTmem = 512;           // S: 2 x 128 columns, O: 128 columns
+constexpr int kSpTmem = 512;
+// TMEM columns: S of the two buffers, O (fp32), and the two operands the
+// products take from TMEM instead of shared memory: P (fp16, two keys per
+// column) and Q (bf16, two features per column, staged once per CTA)
+constexpr uint32_t kSpColO = 256, kSpColP = 384, kSpColQ = 448;
 }  // namespace
 
 size_t attn_split_scratch_bytes(int n_groups_total, int S) {
@@ -63,7 +66,6 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint8_t* sQ = smem + oSpQ;
   uint8_t* sK = smem + oSpK;
   uint8_t* sV = smem + oSpV;
-  uint8_t* sP = smem + oSpP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oSpBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;    // [2] keys of the chunk in that stage landed
@@ -74,7 +76,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint64_t* pv_done = bars + 10;  // PV of a chunk done (one phase per chunk)
   uint64_t* v_full = bars + 11;   // [2] values of the chunk in that stage landed
   uint64_t* v_empty = bars + 13;  // [2] PV of the chunk in that stage done (its values are free)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* q_tmem = bars + 15;   // Q staged into TMEM by the softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
   float* sLh = reinterpret_cast<float*>(smem + oSpL);
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 15; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9) ? 8 : 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9 || i == 15) ? 8 : 1);
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -193,16 +196,16 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && nc > 0) {
-      bool ok = mbar_wait(q_full, 0, a.status, sabort);
+      bool ok = mbar_wait(q_tmem, 0, a.status, sabort);
       auto issue_pv = [&](int c) -> bool {
         if (!mbar_wait(p_full, c & 1, a.status, sabort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sP), vb = smem_u32(sV + 2 * (c & 1) * kSpAtom);
+        const uint32_t vb = smem_u32(sV + 2 * (c & 1) * kSpAtom);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
-          umma_bf16_ss(tmem + 256, sdesc_kmajor_sw128(pa + off), sdesc_kmajor_sw128(vb + off), kSpIdescO,
-                       (c > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tmem + kSpColO, tmem + kSpColP + kk * 8, sdesc_kmajor_sw128(vb + off), kSpIdescO,
+                      (c > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&v_empty[c & 1]);
         umma_commit(pv_done);
@@ -227,12 +230,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           if (mbar_test_wait(&k_full[st], (cs >> 1) & 1) &&
               (cs < 2 || mbar_test_wait(&s_empty[st], ((cs >> 1) - 1) & 1))) {
             tc_fence_after();
-            const uint32_t qa = smem_u32(sQ), kb = smem_u32(sK + 2 * st * kSpAtom);
+            const uint32_t kb = smem_u32(sK + 2 * st * kSpAtom);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
-              umma_bf16_ss(tmem + st * kSpKeys, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(kb + off),
-                           kSpIdescS, kk > 0 ? 1u : 0u);
+              umma_f16_ts(tmem + st * kSpKeys, tmem + kSpColQ + kk * 8, sdesc_kmajor_sw128(kb + off), kSpIdescS,
+                          kk > 0 ? 1u : 0u);
             }
             umma_commit(&k_empty[st]);
             umma_commit(&s_full[st]);
@@ -267,6 +270,29 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float m = -INFINITY, l = 0.f;
     bool ok = nc > 0;
+    if (ok) {
+      // Q row `row`, features 64 hf .. 64 hf + 63 (atom hf), into TMEM
+      // columns kSpColQ + 32 hf .. + 31 for the S products
+      ok = mbar_wait(q_full, 0, a.status, sabort);
+      if (ok) {
+        const uint8_t* qrow = sQ + hf * kSpAtom + row * 128;
+        uint32_t qw[32];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + ((cc ^ (row & 7)) << 4));
+          qw[4 * cc] = v.x;
+          qw[4 * cc + 1] = v.y;
+          qw[4 * cc + 2] = v.z;
+          qw[4 * cc + 3] = v.w;
+        }
+        tmem_st16u_nowait(tmem + lane_off + kSpColQ + hf * 32, qw);
+        tmem_st16u_nowait(tmem + lane_off + kSpColQ + hf * 32 + 16, qw + 16);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_tmem);
+    }
     for (int c = 0; ok && c < nc; ++c) {
       const int st = c & 1;
       const int key0 = (sp + c * S) * kSpKeys;
@@ -341,13 +367,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           tmem_wait_st();
         }
       }
-      {
-        uint8_t* prow = sP + hf * kSpAtom + row * 128;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
-              make_uint4(packed[cc * 4], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
-      }
+      // P of this warp's 64 keys into TMEM columns kSpColP + 32 hf .. + 31
+      tmem_st16u_nowait(tmem + lane_off + kSpColP + hf * 32, packed);
+      tmem_st16u_nowait(tmem + lane_off + kSpColP + hf * 32 + 16, packed + 16);
       // value row `row` (feature d = row) of this warp's 64 keys to fp16 in
       // place; keys past the valid slots (stale, poisoned, other pages' rows)
       // become 0
@@ -385,6 +407,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4)) = w[cc];
       }
+      tmem_wait_st();  // P (and any rescaled O) in TMEM
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
