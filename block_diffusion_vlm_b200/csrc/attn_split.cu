@@ -30,18 +30,20 @@
 namespace dvlm {
 
 namespace {
-constexpr int kSpThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (two per TMEM lane quarter)
+constexpr int kSpThreads = 384;        // warp 0 TMA, 1 MMA, 2..9 softmax (two per TMEM lane quarter), 10..11 value conversion
 constexpr int kSpSoftmax = 256;        // softmax threads: row = quarter * 32 + lane, key half = (warp - 2) / 4
 constexpr float kSpLazy = 8.0f;        // log2 headroom before the running maximum moves
 constexpr int kSpPrefetch = 4;         // L2 prefetch distance in chunks past the newest load
 constexpr int kSpKeys = 128;           // keys per chunk
 constexpr int kSpAtom = 128 * 128;     // one 128-byte-swizzled 128-row operand atom (16 KB)
 constexpr int oSpQ = 0;                // Q: 2 atoms (d 0..63, 64..127)
-constexpr int oSpK = oSpQ + 2 * kSpAtom;   // K: 2 stages x 2 d-atoms
-constexpr int oSpV = oSpK + 4 * kSpAtom;   // V^T: 2 stages x 2 key-atoms
-constexpr int oSpBar = oSpV + 4 * kSpAtom;
+constexpr int kSpStages = 2;           // key stages and value stages (each)
+constexpr int oSpK = oSpQ + 2 * kSpAtom;   // K: kSpStages x 2 d-atoms
+constexpr int oSpV = oSpK + 2 * kSpStages * kSpAtom;   // V^T: kSpStages x 2 key-atoms
+constexpr int oSpBar = oSpV + 2 * kSpStages * kSpAtom;
 constexpr int oSpL = oSpBar + 256;     // [2][128] row sums of the two key halves
-constexpr int kSpSmem = oSpL + 1024 + 1024;
+constexpr int oSpMx = oSpL + 1024;     // [2 chunk parities][2 halves][128] half-chunk row maxima
+constexpr int kSpSmem = oSpMx + 2048 + 1024;
 constexpr uint32_t kSpIdescS = idesc_bf16_f32(128, kSpKeys);
 constexpr uint32_t kSpIdescO = idesc_f16_f32(128, 128);
 constexpr int kSpTmem = 512;
@@ -68,19 +70,23 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint8_t* sV = smem + oSpV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + oSpBar);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;    // [2] keys of the chunk in that stage landed
-  uint64_t* k_empty = bars + 3;   // [2] S of the chunk in that stage done (its keys are free)
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_empty = bars + 7;   // [2] the softmax warps have read S of that buffer
-  uint64_t* p_full = bars + 9;    // P of the current chunk written, O rescaled (one phase per chunk)
-  uint64_t* pv_done = bars + 10;  // PV of a chunk done (one phase per chunk)
-  uint64_t* v_full = bars + 11;   // [2] values of the chunk in that stage landed
-  uint64_t* v_empty = bars + 13;  // [2] PV of the chunk in that stage done (its values are free)
-  uint64_t* q_tmem = bars + 15;   // Q staged into TMEM by the softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* s_full = bars + 1;    // [2]
+  uint64_t* s_empty = bars + 3;   // [2] the softmax warps have read S of that buffer
+  uint64_t* p_full = bars + 5;    // P of the current chunk written, O rescaled (one phase per chunk)
+  uint64_t* pv_done = bars + 6;   // PV of a chunk done (one phase per chunk)
+  uint64_t* q_tmem = bars + 7;    // Q staged into TMEM by the softmax warps
+  uint64_t* k_full = bars + 8;                   // [kSpStages] keys of the chunk in that stage landed
+  uint64_t* k_empty = k_full + kSpStages;        // [kSpStages] S of that chunk done (its keys are free)
+  uint64_t* v_full = k_empty + kSpStages;        // [kSpStages] values of the chunk in that stage landed
+  uint64_t* v_empty = v_full + kSpStages;        // [kSpStages] PV of that chunk done (its values are free)
+  uint64_t* v_conv = v_empty + kSpStages;        // [kSpStages] values of that chunk converted to fp16
+  uint64_t* mx_bar = v_conv + kSpStages;         // [4 quarters][2 chunk parities] both halves' maxima written
+  constexpr int kSpBars = 8 + 5 * kSpStages + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kSpBars);
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
   float* sLh = reinterpret_cast<float*>(smem + oSpL);
+  float* sMx = reinterpret_cast<float*>(smem + oSpMx);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = gridDim.x, sp = blockIdx.x, g = blockIdx.y;
@@ -101,7 +107,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == 7 || i == 8 || i == 9 || i == 15) ? 8 : 1);
+    for (int i = 0; i < kSpBars; ++i)
+      mbar_init(&bars[i], (i >= 3 && i <= 5) || i == 7 ? 8 : (i >= kSpBars - 8 - kSpStages ? 2 : 1));
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       // the loaded ones are prefetched into L2 (up to kSpPrefetch ahead of the
       // newest key load), so a refill reads L2 instead of DRAM.
       auto load_k = [&](int c) {
-        const int st = c & 1;
+        const int st = c % kSpStages;
         mbar_arrive_expect_tx(&k_full[st], 2 * kSpAtom);
         for (int hf = 0; hf < 2; ++hf) {
           int krow, vrow, vx;
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
       };
       auto load_v = [&](int c) {
-        const int st = c & 1;
+        const int st = c % kSpStages;
         mbar_arrive_expect_tx(&v_full[st], 2 * kSpAtom);
         for (int hf = 0; hf < 2; ++hf) {
           int krow, vrow, vx;
@@ -173,10 +180,11 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &v_full[st], vx, vrow, pol);
         }
       };
-      int pf = 2;
+      int pf = kSpStages;
       for (int i = 0; i <= nc; ++i) {
         if (i < nc) {
-          if (i >= 2 && !mbar_wait(&k_empty[i & 1], ((i >> 1) - 1) & 1, a.status, sabort)) break;
+          if (i >= kSpStages && !mbar_wait(&k_empty[i % kSpStages], ((i / kSpStages) - 1) & 1, a.status, sabort))
+            break;
           load_k(i);
           for (; pf < nc && pf <= i + kSpPrefetch; ++pf) {
             for (int hf = 0; hf < 2; ++hf) {
@@ -189,7 +197,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         if (i >= 1) {
           const int c = i - 1;
-          if (c >= 2 && !mbar_wait(&v_empty[c & 1], ((c >> 1) - 1) & 1, a.status, sabort)) break;
+          if (c >= kSpStages && !mbar_wait(&v_empty[c % kSpStages], ((c / kSpStages) - 1) & 1, a.status, sabort))
+            break;
           load_v(c);
         }
       }
@@ -197,17 +206,18 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && nc > 0) {
       bool ok = mbar_wait(q_tmem, 0, a.status, sabort);
+      // descriptors of stage 0's K and V tiles; a stage or K-step offset adds
+      // (bytes >> 4) to the start-address field (addresses stay below 2^18)
+      const uint64_t kdesc0 = sdesc_kmajor_sw128(smem_u32(sK)), vdesc0 = sdesc_kmajor_sw128(smem_u32(sV));
       auto issue_pv = [&](int c) -> bool {
         if (!mbar_wait(p_full, c & 1, a.status, sabort)) return false;
         tc_fence_after();
-        const uint32_t vb = smem_u32(sV + 2 * (c & 1) * kSpAtom);
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>((2 * (c % kSpStages) * kSpAtom) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
-          umma_f16_ts(tmem + kSpColO, tmem + kSpColP + kk * 8, sdesc_kmajor_sw128(vb + off), kSpIdescO,
-                      (c > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&v_empty[c & 1]);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(tmem + kSpColO, tmem + kSpColP + kk * 8, vd + (((kk >> 2) * kSpAtom + (kk & 3) * 32) >> 4),
+                      kSpIdescO, (c > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&v_empty[c % kSpStages]);
         umma_commit(pv_done);
         return true;
       };
@@ -219,25 +229,24 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       int cs = 0, cp = 0;
       long long t0 = clock64();
       while (ok && cp < nc) {
-        if (cp < cs && mbar_test_wait(p_full, cp & 1)) {
+        if (cp < cs && mbar_test_wait(p_full, cp & 1) &&
+            mbar_test_wait(&v_conv[cp % kSpStages], (cp / kSpStages) & 1)) {
           ok = issue_pv(cp);
           ++cp;
           t0 = clock64();
           continue;
         }
         if (cs < nc && cs <= cp + 1) {
-          const int st = cs & 1;
-          if (mbar_test_wait(&k_full[st], (cs >> 1) & 1) &&
+          const int st = cs & 1, ks = cs % kSpStages;
+          if (mbar_test_wait(&k_full[ks], (cs / kSpStages) & 1) &&
               (cs < 2 || mbar_test_wait(&s_empty[st], ((cs >> 1) - 1) & 1))) {
             tc_fence_after();
-            const uint32_t kb = smem_u32(sK + 2 * st * kSpAtom);
+            const uint64_t kd = kdesc0 + static_cast<uint64_t>((2 * ks * kSpAtom) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kSpAtom + (kk & 3) * 32;
-              umma_f16_ts(tmem + st * kSpKeys, tmem + kSpColQ + kk * 8, sdesc_kmajor_sw128(kb + off), kSpIdescS,
-                          kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&k_empty[st]);
+            for (int kk = 0; kk < 8; ++kk)
+              umma_f16_ts(tmem + st * kSpKeys, tmem + kSpColQ + kk * 8,
+                          kd + (((kk >> 2) * kSpAtom + (kk & 3) * 32) >> 4), kSpIdescS, kk > 0 ? 1u : 0u);
+            umma_commit(&k_empty[ks]);
             umma_commit(&s_full[st]);
             ++cs;
             t0 = clock64();
@@ -250,6 +259,52 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           ok = false;
         }
       }
+    }
+  } else if (warp >= 10) {
+    // ------------------------------------------------------ value conversion
+    // Warp 10 + cw turns value rows (features) 64 cw .. 64 cw + 63 of each
+    // chunk's two key atoms from bf16 to fp16 in place, two rows per lane;
+    // keys past the valid slots (stale, poisoned, other pages' rows) become
+    // 0.  All eight 16-byte pieces of a row are loaded first, then converted,
+    // then stored.
+    const int cw = warp - 10;
+    for (int c = 0; c < nc; ++c) {
+      const int vs = c % kSpStages;
+      if (!mbar_wait(&v_full[vs], (c / kSpStages) & 1, a.status, sabort)) break;
+      const int key0 = (sp + c * S) * kSpKeys;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int at = j & 1, d = 64 * cw + 32 * (j >> 1) + lane;
+        const int n_valid = Ltot - key0 - at * 64;
+        uint8_t* vrow = sV + (2 * vs + at) * kSpAtom + d * 128;
+        uint4 w[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) w[cc] = *reinterpret_cast<const uint4*>(vrow + ((cc ^ (d & 7)) << 4));
+        if (n_valid >= 64) {
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wv[e] = bf16x2_to_f16x2(wv[e]);
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int kk = (cc << 3) + 2 * e;
+              const uint32_t keep = (kk < n_valid ? 0x0000FFFFu : 0u) | (kk + 1 < n_valid ? 0xFFFF0000u : 0u);
+              wv[e] = bf16x2_to_f16x2(wv[e] & keep);
+            }
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + ((cc ^ (d & 7)) << 4)) = w[cc];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_conv[vs]);
     }
   } else {
     // ---------------------------------------------------------------- softmax
@@ -302,21 +357,33 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         break;
       }
       tc_fence_after();
-      float sc[64], so[64];  // this warp's keys; the other half's keys (maximum only)
+      float sc[64];  // this warp's 64 keys
       tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + hf * 64), sc);
-      tmem_ld64(tmem + lane_off + static_cast<uint32_t>(st * kSpKeys + (hf ^ 1) * 64), so);
-      float mx = -INFINITY;
+      // maximum over this half (eight independent chains), then over the
+      // row's two halves through shared memory (max is exact in any order,
+      // so both warps hold the same value)
+      float mv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mv[j] = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) mx = fmaxf(mx, fmaxf(sc[k], so[k]));
+        for (int k = 0; k < 64; ++k) mv[k & 7] = fmaxf(mv[k & 7], sc[k]);
       } else {
-        const int kme = key0 + hf * 64, koth = key0 + (hf ^ 1) * 64;
+        const int kme = key0 + hf * 64;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          if (kme + k < limit) mx = fmaxf(mx, sc[k]);
-          if (koth + k < limit) mx = fmaxf(mx, so[k]);
-        }
+        for (int k = 0; k < 64; ++k)
+          if (kme + k < limit) mv[k & 7] = fmaxf(mv[k & 7], sc[k]);
       }
+      const float mh = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                             fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+      sMx[((c & 1) * 2 + hf) * 128 + row] = mh;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mx_bar[quarter * 2 + (c & 1)]);
+      if (!mbar_wait(&mx_bar[quarter * 2 + (c & 1)], (c >> 1) & 1, a.status, sabort)) {
+        ok = false;
+        break;
+      }
+      const float mx = fmaxf(mh, sMx[((c & 1) * 2 + (hf ^ 1)) * 128 + row]);
       // scale_log2 > 0, so the maximum of the scaled scores is the scaled
       // maximum (rounding is monotonic).  The reference maximum moves only
       // when a score exceeds it by more than 2^kLazy: below that the
@@ -326,13 +393,13 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       const float m_new = (m == -INFINITY || m_cand > m + kSpLazy) ? m_cand : m;
       const float alpha = (m == -INFINITY) ? (m_new == -INFINITY ? 1.f : 0.f) : exp2f(m - m_new);
       uint32_t packed[32];
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
       if (full) {
 #pragma unroll
         for (int k = 0; k < 64; k += 2) {
           const float p0 = ex2_approx(sc[k] * a.scale_log2 - m_new);
           const float p1 = ex2_approx(sc[k + 1] * a.scale_log2 - m_new);
-          psum += p0 + p1;
+          ps[(k >> 1) & 3] += p0 + p1;
           const __half2 ph = __floats2half2_rn(p0, p1);
           packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
@@ -343,7 +410,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           const float p0 = (kme + k < limit && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
           const float p1 =
               (kme + k + 1 < limit && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
-          psum += p0 + p1;
+          ps[(k >> 1) & 3] += p0 + p1;
           const __half2 ph = __floats2half2_rn(p0, p1);
           packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
         }
@@ -370,49 +437,11 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       // P of this warp's 64 keys into TMEM columns kSpColP + 32 hf .. + 31
       tmem_st16u_nowait(tmem + lane_off + kSpColP + hf * 32, packed);
       tmem_st16u_nowait(tmem + lane_off + kSpColP + hf * 32 + 16, packed + 16);
-      // value row `row` (feature d = row) of this warp's 64 keys to fp16 in
-      // place; keys past the valid slots (stale, poisoned, other pages' rows)
-      // become 0
-      if (!mbar_wait(&v_full[st], (c >> 1) & 1, a.status, sabort)) {
-        ok = false;
-        break;
-      }
-      {
-        // all eight 16-byte pieces loaded first, then converted, then stored
-        // (independent shared-memory round trips)
-        const int n_valid = Ltot - key0 - hf * 64;
-        uint8_t* vrow = sV + (2 * st + hf) * kSpAtom + row * 128;
-        uint4 w[8];
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) w[cc] = *reinterpret_cast<const uint4*>(vrow + ((cc ^ (row & 7)) << 4));
-        if (n_valid >= 64) {
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) wv[e] = bf16x2_to_f16x2(wv[e]);
-          }
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[cc]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int kk = (cc << 3) + 2 * e;
-              const uint32_t keep = (kk < n_valid ? 0x0000FFFFu : 0u) | (kk + 1 < n_valid ? 0xFFFF0000u : 0u);
-              wv[e] = bf16x2_to_f16x2(wv[e] & keep);
-            }
-          }
-        }
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + ((cc ^ (row & 7)) << 4)) = w[cc];
-      }
       tmem_wait_st();  // P (and any rescaled O) in TMEM
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      l = l * alpha + psum;
+      l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       m = m_new;
     }
     // this split's partial rows: O / l (fp32, each warp its 64 features) and
