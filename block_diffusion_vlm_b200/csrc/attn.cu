@@ -501,12 +501,12 @@ static cudaError_t attn_launch(const CUtensorMap& mapQ, const CUtensorMap& mapK,
 
 cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                              const AttnArgs& a, bool pdl, cudaStream_t s, int cs) {
-  if (cs == 16) return attn_launch<16>(mapQ, mapK, mapV, a, pdl, s);
-  return attn_launch<8>(mapQ, mapK, mapV, a, pdl, s);
+  return launch_attn_split_cl(mapQ, mapK, mapV, a, cs, pdl, s);
 }
 
 // Clusters of cs CTAs that can be resident at once (0: cannot launch).
 int attn_max_clusters(int cs) {
+  return attn_split_cl_max_clusters(cs);
   auto kern = cs == 16 ? attn_bf16_kernel<16> : attn_bf16_kernel<8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess ||
       (cs > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {

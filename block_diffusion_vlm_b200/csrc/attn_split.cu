@@ -43,7 +43,9 @@ constexpr int oSpV = oSpK + 2 * kSpStages * kSpAtom;   // V^T: kSpStages x 2 key
 constexpr int oSpBar = oSpV + 2 * kSpStages * kSpAtom;
 constexpr int oSpL = oSpBar + 256;     // [2][128] row sums of the two key halves
 constexpr int oSpMx = oSpL + 1024;     // [2 chunk parities][2 halves][128] half-chunk row maxima
-constexpr int kSpSmem = oSpMx + 2048 + 1024;
+constexpr int oSpRecv = oSpMx + 2048;  // cluster merge: [source CTA][row of this CTA][128] fp16 O / l
+constexpr int oSpRecvML = oSpRecv + 128 * 128 * 2;  // and [source CTA][row] (m, l)
+constexpr int kSpSmem = oSpRecvML + 128 * 8 + 1024;
 constexpr uint32_t kSpIdescS = idesc_bf16_f32(128, kSpKeys);
 constexpr uint32_t kSpIdescO = idesc_f16_f32(128, 128);
 constexpr int kSpTmem = 512;
@@ -59,6 +61,13 @@ size_t attn_split_scratch_bytes(int n_groups_total, int S) {
   return (part + 255) / 256 * 256 + (ml + 255) / 256 * 256 + (static_cast<size_t>(n_groups_total) * 4 + 255) / 256 * 256;
 }
 
+// kCL = 0: S = gridDim.x independent CTAs, partials through global scratch,
+// merged by the last CTA of the group.  kCL = 8 or 16: the S = kCL CTAs of a
+// group form one thread-block cluster; each sends its fp16 partial rows
+// O / l and (m, l) straight into the shared memory of the CTA that owns
+// those rows (128 / kCL rows each), which merges them after one cluster
+// barrier: no global scratch, no counter.
+template <int kCL>
 __global__ void __launch_bounds__(kSpThreads, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                       const __grid_constant__ CUtensorMap mapV, const AttnArgs a, float* part, float2* ml,
@@ -81,7 +90,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint64_t* v_empty = v_full + kSpStages;        // [kSpStages] PV of that chunk done (its values are free)
   uint64_t* v_conv = v_empty + kSpStages;        // [kSpStages] values of that chunk converted to fp16
   uint64_t* mx_bar = v_conv + kSpStages;         // [4 quarters][2 chunk parities] both halves' maxima written
-  constexpr int kSpBars = 8 + 5 * kSpStages + 8;
+  uint64_t* recv_full = mx_bar + 8;              // cluster merge: every sending CTA's rows landed
+  constexpr int kSpBars = 8 + 5 * kSpStages + 8 + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kSpBars);
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* sflag = reinterpret_cast<int*>(tmem_slot + 2);
@@ -107,8 +117,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSpBars; ++i)
-      mbar_init(&bars[i], (i >= 3 && i <= 5) || i == 7 ? 8 : (i >= kSpBars - 8 - kSpStages ? 2 : 1));
+    for (int i = 0; i < kSpBars; ++i) {
+      const bool pair = &bars[i] >= v_conv && &bars[i] < recv_full;  // v_conv, mx_bar: two arrivals
+      mbar_init(&bars[i], (i >= 3 && i <= 5) || i == 7 ? 8 : (pair ? 2 : 1));
+    }
+    if constexpr (kCL > 0)  // the CTAs with keys send RPC rows of fp16 O / l and of (m, l) each
+      mbar_arrive_expect_tx(recv_full, static_cast<uint32_t>(min(kCL, n_all)) * (128 / kCL) * (256 + 8));
     *sabort = 0;
     fence_mbar_init();
     tma_prefetch_map(&mapQ);
@@ -123,6 +137,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // every CTA of the cluster is running before any sends into it (the wait
+  // sits just before the sends)
+  if constexpr (kCL > 0) cluster_arrive();
 
   // (layer, page, head) entry holding logical slot `key` of a paged cache
   auto page_entry = [&](int key) -> int {
@@ -444,14 +461,111 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       m = m_new;
     }
-    // this split's partial rows: O / l (fp32, each warp its 64 features) and
-    // (m, l), l the two halves' sums added in half order
-    const size_t pidx = static_cast<size_t>(grp) * S + sp;
-    float* prow = part + (pidx * 128 + row) * 128 + hf * 64;
     const bool have = ok && nc > 0 && mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort);
     sLh[hf * 128 + row] = l;
     named_bar_sync(1, kSpSoftmax);
     l = sLh[row] + sLh[128 + row];
+    if constexpr (kCL > 0) {
+      // ------------------------------------------------------ cluster merge
+      // This CTA's O / l of row `row` (features 64 hf .. 64 hf + 63) as fp16
+      // (|O / l| <= max |v|) and (m, l) into shared memory (the key stages
+      // are free), 16-byte pieces of a 256-byte row at piece ^ (row & 15)
+      // (conflict-free for lanes = rows); then one bulk copy per owner CTA
+      // of its RPC rows into that CTA's slot for this source, counted on its
+      // receive barrier.  CTAs without keys send nothing and every owner
+      // expects the min(kCL, chunks) CTAs that have keys.  Each CTA then
+      // combines its RPC rows over the sources in source order.
+      constexpr int RPC = 128 / kCL;
+      constexpr uint32_t kSendO = RPC * 256, kSendML = RPC * 8;
+      const int crank = sp;
+      const int n_src = min(kCL, n_all);
+      uint8_t* sSend = sK;                                           // [128][256 B]
+      float2* sSendML = reinterpret_cast<float2*>(sK + 128 * 256);  // [128]
+      if (nc > 0) {
+        float o[64];
+        if (have) {
+          tc_fence_after();
+          tmem_ld64(tmem + lane_off + kSpColO + static_cast<uint32_t>(hf * 64), o);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) o[k] = 0.f;
+        }
+        const float inv_l = (have && l > 0.f) ? 1.0f / l : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 h = __floats2half2_rn(o[8 * q + 2 * e] * inv_l, o[8 * q + 2 * e + 1] * inv_l);
+            w[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(sSend + row * 256 + (((hf * 8 + q) ^ (row & 15)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (hf == 0) sSendML[row] = (have && l > 0.f) ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(1, kSpSoftmax);
+      __syncwarp();
+      cluster_wait();  // every CTA of the cluster runs, its receive barrier initialised
+      const int et = threadIdx.x - 64;
+      if (nc > 0 && et < kCL) {
+        const uint32_t rb = map_to_cta(smem_u32(recv_full), et);
+        bulk_s2s_cluster(map_to_cta(smem_u32(smem + oSpRecv) + crank * kSendO, et), sSend + et * kSendO, kSendO, rb);
+        bulk_s2s_cluster(map_to_cta(smem_u32(smem + oSpRecvML) + crank * kSendML, et), sSendML + et * RPC, kSendML,
+                         rb);
+        bulk_commit();
+      }
+      const bool got = mbar_wait(recv_full, 0, a.status, sabort);
+      constexpr int TPR = kSpSoftmax / RPC;  // threads per merged row
+      constexpr int FPT = 128 / TPR;         // features per thread
+      const int rl = et / TPR, f0 = (et % TPR) * FPT;
+      const int r = crank * RPC + rl;        // row of the tile
+      const uint8_t* rO = smem + oSpRecv;
+      const float2* rML = reinterpret_cast<const float2*>(smem + oSpRecvML);
+      // piece of features f0.. in a row sent as tile row r, and the offset in it
+      const int piece = ((f0 >> 3) ^ (r & 15)) << 4, poff = (f0 & 7) * 2;
+      float M = -INFINITY;
+      for (int q = 0; q < n_src; ++q) M = fmaxf(M, rML[q * RPC + rl].x);
+      float acc[FPT];
+#pragma unroll
+      for (int k = 0; k < FPT; ++k) acc[k] = 0.f;
+      float wsum = 0.f;
+      if (got && M != -INFINITY) {
+#pragma unroll 4
+        for (int q = 0; q < n_src; ++q) {
+          const float2 v = rML[q * RPC + rl];
+          const float w = v.y > 0.f ? ex2_approx(v.x - M) * v.y : 0.f;
+          wsum += w;
+          const __half2* src = reinterpret_cast<const __half2*>(rO + (q * RPC + rl) * 256 + piece + poff);
+#pragma unroll
+          for (int k = 0; k < FPT; k += 2) {
+            const float2 f = __half22float2(src[k / 2]);
+            acc[k] += w * f.x;
+            acc[k + 1] += w * f.y;
+          }
+        }
+      }
+      const int tr = t_base + (r >> 3);
+      if (tr < a.n_rows) {
+        const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+        bf16* dst_o = a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + f0;
+#pragma unroll
+        for (int k = 0; k < FPT; k += 4) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
+          const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[k + 2] * inv, acc[k + 3] * inv);
+          *reinterpret_cast<uint2*>(dst_o + k) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        }
+      }
+      // no CTA leaves before its outgoing copies have read their source (its
+      // incoming ones have landed: receive barrier above)
+      if (nc > 0 && et < kCL) bulk_wait_read_all();
+    } else {
+    // this split's partial rows: O / l (fp32, each warp its 64 features) and
+    // (m, l), l the two halves' sums added in half order
+    const size_t pidx = static_cast<size_t>(grp) * S + sp;
+    float* prow = part + (pidx * 128 + row) * 128 + hf * 64;
     if (have) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
@@ -534,6 +648,15 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
       }
     }
+    }
+  }
+  if constexpr (kCL > 0) {
+    // the loader, MMA and conversion warps take part in the cluster barrier
+    // the softmax warps pass before their sends
+    if (warp < 2 || warp >= 10) {
+      __syncwarp();
+      cluster_wait();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -552,7 +675,7 @@ cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -574,7 +697,79 @@ cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, 
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_split_kernel, mapQ, mapK, mapV, a, p, m, c);
+  return cudaLaunchKernelEx(&cfg, attn_split_kernel<0>, mapQ, mapK, mapV, a, p, m, c);
+}
+
+template <int CL>
+static cudaError_t split_cl_attr() {
+  cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+  if (e == cudaSuccess && CL > 8)
+    e = cudaFuncSetAttribute(attn_split_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+// One cluster of cs CTAs (8 or 16) per (batch entry, row group, KV head);
+// no scratch.
+cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                 const AttnArgs& a, int cs, bool pdl, cudaStream_t s) {
+  if (cs != 8 && cs != 16) return cudaErrorInvalidValue;
+  static bool attr_set[2][64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const int ci = cs == 16 ? 1 : 0;
+  if (dev < 0 || dev >= 64 || !attr_set[ci][dev]) {
+    cudaError_t e = cs == 16 ? split_cl_attr<16>() : split_cl_attr<8>();
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[ci][dev] = true;
+  }
+  const int n_groups = (a.n_rows + 15) / 16;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, a.Hkv, a.n_batch * n_groups);
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = kSpSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cs;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cs == 16)
+    return cudaLaunchKernelEx(&cfg, attn_split_kernel<16>, mapQ, mapK, mapV, a, static_cast<float*>(nullptr),
+                              static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
+  return cudaLaunchKernelEx(&cfg, attn_split_kernel<8>, mapQ, mapK, mapV, a, static_cast<float*>(nullptr),
+                            static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
+}
+
+// Clusters of cs CTAs of the cluster-merge form that can be resident at once
+// (0: cannot launch).
+int attn_split_cl_max_clusters(int cs) {
+  if ((cs == 16 ? split_cl_attr<16>() : split_cl_attr<8>()) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, 2, 1);
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = kSpSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = cs == 16 ? cudaOccupancyMaxActiveClusters(&n, attn_split_kernel<16>, &cfg)
+                                 : cudaOccupancyMaxActiveClusters(&n, attn_split_kernel<8>, &cfg);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 }  // namespace dvlm

@@ -207,6 +207,11 @@ int attn_max_clusters(int cs);
 size_t attn_split_scratch_bytes(int n_groups_total, int S);
 cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                               const AttnArgs& a, int S, void* scratch, bool pdl, cudaStream_t s);
+// The same kernel with the S = cs (8 or 16) splits of a group in one
+// thread-block cluster, merged through distributed shared memory.
+cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                 const AttnArgs& a, int cs, bool pdl, cudaStream_t s);
+int attn_split_cl_max_clusters(int cs);
 
 // Prefill (compute-bound path over the whole context; csrc/prefill.cu).
 // Token-major GEMM epilogue operands: one context row per epilogue thread.
