@@ -183,7 +183,7 @@ TRAFFIC_SOURCES = {
     "down_gemm": _COMMON_SOURCES + ["gemm_ws.cu"],
     "persistent_forward": _COMMON_SOURCES + ["gemm_ws.cu"],
     "lm_head": _COMMON_SOURCES + ["lmhead.cu", "finalize.cuh"],
-    "attention": _COMMON_SOURCES + ["attn.cu"],
+    "attention": _COMMON_SOURCES + ["attn_split.cu"],
 }
 
 

@@ -50,8 +50,8 @@ inline int sms_or_default() {
 inline int attn_cluster_for_device() {
   static int cached[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return attn_max_clusters(16) >= 2 ? 16 : 8;
-  if (cached[dev] == 0) cached[dev] = attn_max_clusters(16) >= 2 ? 16 : 8;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return attn_split_cl_max_clusters(16) >= 2 ? 16 : 8;
+  if (cached[dev] == 0) cached[dev] = attn_split_cl_max_clusters(16) >= 2 ? 16 : 8;
   return cached[dev];
 }
 inline int lm_nt(int R) { return R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128; }
@@ -189,7 +189,7 @@ dvlm_status dvlm_block_attn(const void* q, void* out, const void* k_cache, const
   a.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
   a.out = static_cast<bf16*>(out);
   a.status = dev_status;
-  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), attn_cluster_for_device()));
+  return cuda_status(launch_attn_split_cl(mq, mk, mv, a, attn_cluster_for_device(), false, cs(stream)));
 }
 
 size_t dvlm_block_attn_split_workspace_size(int n_batch, int n_rows, int Hkv, int splits) {
@@ -269,7 +269,7 @@ dvlm_status dvlm_block_attn_paged(const void* q, void* out, const void* k_pages,
   a.max_pages = max_pages;
   a.n_pages = n_pages;
   a.d_lens = lens;
-  return cuda_status(launch_attn_bf16(mq, mk, mv, a, false, cs(stream), attn_cluster_for_device()));
+  return cuda_status(launch_attn_split_cl(mq, mk, mv, a, attn_cluster_for_device(), false, cs(stream)));
 }
 
 // ------------------------------------------------------------ LM head

@@ -1,27 +1,33 @@
-// Block-masked GQA attention split over independent CTAs (flash-decoding
-// style), bf16, tcgen05: the bandwidth-bound form of the decode attention.
+// Block-masked GQA attention against the exact KV cache, bf16, tcgen05.
 //
 // Visibility [Fast-dVLM technical overview (ocdem.com), section 2.2.1;
 // Fast-dVLM walkthrough (itsolotime.com), section 4.1]: a clean row t (slot
-// L+t) sees slots 0..L+t (C2C); a noisy row sees slots 0..L+n_rows-1 (N2C and
-// N2N).  The same rules as attn_bf16_kernel; only the work split differs.
+// L+t) sees slots 0..L+t (C2C, causal); a noisy row sees every slot
+// 0..L+n_rows-1 -- the whole cache of vision, prompt and committed tokens
+// (N2C) and its own block in both directions (N2N).
 //
 // Tile: one KV head's 8 query heads x 16 step rows = 128 rows (token-major,
 // head-minor, as a 3-D TMA box lands).  Keys go in 128-key chunks, chunk j
 // to split j % S (round robin by absolute key position, so a causal row's
 // arithmetic is the same whatever the number of rows in the step: a 1-row AR
 // pass and a 16-row verify pass give bitwise the same output).  Each of the S
-// CTAs of a (batch entry, row group, KV head) streams its chunks through a
-// 2-stage TMA pipeline (S = Q K^T and O += P V in TMEM, online softmax in
-// fp32 with two threads per row, one per 64-key half, P and V in fp16 for
-// the second product; the running maximum moves only when a score passes it
-// by more than 2^8, which leaves the result exact up to rounding and skips
-// most rescales of O),
-// then stores its partial rows (O / l in fp32, and (m, l)) to global scratch
-// and counts itself on the group's counter; the last CTA to arrive merges the
-// S partials in split order (deterministic) and writes the bf16 output.  No
-// CTA waits for another.  Paged caches read each 64-key half chunk through
-// the block table.
+// CTAs of a (batch entry, row group, KV head) streams its chunks through
+// two key and two value stages (TMA); S = Q K^T and O += P V accumulate in
+// TMEM with Q and P as TMEM operands; the online softmax runs in fp32 with
+// two threads per row, one per 64-key half, P in fp16 (the value tile
+// converted to fp16 in shared memory by two dedicated warps); the running
+// maximum moves only when a score passes it by more than 2^8, which leaves
+// the result exact up to rounding and skips most rescales of O.
+//
+// Two ways to merge the S partials (O / l and (m, l) per row):
+//   split form (kCL = 0, the bandwidth-bound form): fp32 partial rows to
+//   global scratch, a counter per group, the last CTA to arrive merges in
+//   split order; no CTA waits for another;
+//   cluster form (kCL = S = 8 or 16, the decode path): the S CTAs are one
+//   thread-block cluster; fp16 partial rows go by bulk copies straight into
+//   the shared memory of the CTA owning those rows, which merges them in
+//   source order; no scratch, no second kernel.
+// Paged caches read each 64-key half chunk through the block table.
 #include <cuda_fp16.h>
 
 #include "kernels.h"

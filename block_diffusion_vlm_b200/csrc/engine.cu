@@ -419,7 +419,7 @@ static cudaError_t fwd_bf16(dvlm_engine* e, const FwdSpec& f, cudaStream_t s) {
     if (e->attn_split > 0)
       DVLM_CK(launch_attn_split(e->tm_q, mk, mv, aa, e->attn_split, e->attn_scratch, pdl, s));
     else
-      DVLM_CK(launch_attn_bf16(e->tm_q, mk, mv, aa, pdl, s, e->attn_cs));
+      DVLM_CK(launch_attn_split_cl(e->tm_q, mk, mv, aa, e->attn_cs, pdl, s));
     T1(K_ATTN);
     ea.epi = EPI_RESID;
     ea.resid = x;
@@ -750,7 +750,7 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
     ta.splits = tm_splits(e, n_tt * (qkv_rows / 256), H / 64);
     DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wqkv_p, e->tm_wqkv_p, H / 64, l * qkv_rows, qkv_rows / 256, ta, s));
     aa.kv_base = l;
-    DVLM_CK(launch_attn_bf16(e->tm_q3, e->tm_k, e->tm_v, aa, false, s, e->attn_cs));
+    DVLM_CK(launch_attn_split_cl(e->tm_q3, e->tm_k, e->tm_v, aa, e->attn_cs, false, s));
     pa.kv_base = l;
     DVLM_CK(launch_attn_cand(e->tm_q3, e->tm_kp, e->tm_v, e->tm_ks, e->tm_vs, pa, s));
     ta.epi = EPI_RESID;
@@ -1224,7 +1224,7 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
     e->gu_cps = v;
   } else if (n == "attn_cluster") {
     if (v != 8 && v != 16) return DVLM_ERR_SHAPE;
-    if (attn_max_clusters(v) <= 0) return DVLM_ERR_UNSUPPORTED;
+    if (attn_split_cl_max_clusters(v) <= 0) return DVLM_ERR_UNSUPPORTED;
     e->attn_cs = v;
   } else if (n == "pdl") {
     e->pdl = v != 0;
@@ -1330,7 +1330,7 @@ void engine_plan(dvlm_engine* e) {
     e->s_qkv = pick_cluster_fp8(e, EPI_QKV, qkv_rows / 128, m.hidden / 128, 5);
     e->s_o = pick_cluster_fp8(e, EPI_RESID, m.hidden / 128, m.n_q_heads * m.head_dim / 128, 5);
     e->s_down = pick_cluster_fp8(e, EPI_RESID, m.hidden / 128, m.inter / 128, e->down_stages);
-    e->attn_cs = attn_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
+    e->attn_cs = attn_split_cl_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
     e->prefill_gemm = false;
     return;
   }
@@ -1338,7 +1338,7 @@ void engine_plan(dvlm_engine* e) {
   e->s_o = pick_cluster(e, EPI_RESID, m.hidden / 128, m.n_q_heads * m.head_dim / 64, 5);
   e->s_down = pick_cluster(e, EPI_RESID, m.hidden / 128, m.inter / 64, e->down_stages);
   // 16-CTA attention clusters when one per KV head can be resident at once
-  e->attn_cs = attn_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
+  e->attn_cs = attn_split_cl_max_clusters(16) >= m.n_kv_heads ? 16 : 8;
   e->prefill_gemm = prefill_gemm_supported(e);
 }
 

@@ -195,20 +195,18 @@ struct AttnArgs {
   int max_pages, n_pages;
   const int* d_lens;
 };
-// cs: CTAs per cluster splitting the keys (8, or 16 where the device can
-// co-schedule 16-CTA clusters; see attn_cluster_size()).
-cudaError_t launch_attn_bf16(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                             const AttnArgs& a, bool pdl, cudaStream_t s, int cs = 8);
-int attn_max_clusters(int cs);
-// Split form of the same attention (csrc/attn_split.cu): S independent CTAs
-// per (batch entry, 16-row group, KV head), merged by the last to finish;
-// scratch of attn_split_scratch_bytes(n_batch * n_groups * Hkv, S) bytes whose
-// counters start at zero (they are zero again after each launch).
+// Block attention (csrc/attn_split.cu), two forms of one kernel.  Split form:
+// S independent CTAs per (batch entry, 16-row group, KV head), merged by the
+// last to finish; scratch of attn_split_scratch_bytes(n_batch * n_groups *
+// Hkv, S) bytes whose counters start at zero (they are zero again after each
+// launch).
 size_t attn_split_scratch_bytes(int n_groups_total, int S);
 cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                               const AttnArgs& a, int S, void* scratch, bool pdl, cudaStream_t s);
-// The same kernel with the S = cs (8 or 16) splits of a group in one
-// thread-block cluster, merged through distributed shared memory.
+// Cluster form (the decode path): the S = cs splits of a group are one
+// thread-block cluster (cs = 8, or 16 where two 16-CTA clusters can be
+// resident at once: attn_split_cl_max_clusters), merged through distributed
+// shared memory; no scratch.
 cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                  const AttnArgs& a, int cs, bool pdl, cudaStream_t s);
 int attn_split_cl_max_clusters(int cs);

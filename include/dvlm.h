@@ -435,8 +435,8 @@ DVLM_API dvlm_status dvlm_forward(dvlm_engine* e, const void* x_in, const int32_
  * is k_pages [n_layers, n_pages, Hkv, 64, D] and v_pages [n_layers, n_pages,
  * Hkv, D, 64] (bf16, device, caller-owned), logical slot s living in row
  * s % 64 of page block_table[s / 64] (device int32 [max_pages], read at each
- * launch: the caller may extend it between calls).  Attention reads 64-key
- * chunks through the table and the QKV projection writes each new K/V row
+ * launch: the caller may extend it between calls).  Attention reads each
+ * 64-slot page through the table and the QKV projection writes each new K/V row
  * through it; results equal those of the contiguous cache bit for bit.
  * Prefill runs in 16-row forwards; DVLM_MODE_SPEC_QUAD, DVLM_MODE_ROUTE and
  * dvlm_forward_text_only are unsupported on a paged engine.  max_pages * 64

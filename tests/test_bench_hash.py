@@ -36,11 +36,11 @@ def test_traffic_key_covers_only_the_kernels_sources(bench_copy):
 def test_source_hash_ignores_comments_but_not_code(bench_copy):
     bench, csrc = bench_copy
     h0 = bench.source_hash()
-    f = csrc / "attn.cu"
+    f = csrc / "attn_split.cu"
     text = f.read_text()
     f.write_text("// a note\n/* a block\n   comment */\n" + text.replace("\n", "\n\n", 3))
     assert bench.source_hash() == h0
-    f.write_text(text.replace("kChunk = 64", "kChunk = 32", 1))
+    f.write_text(text.replace("kSpKeys = 128", "kSpKeys = 64", 1))
     assert bench.source_hash() != h0
 
 
