@@ -111,7 +111,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   const int t_base = (blockIdx.z % n_groups) * 16;
   const int grp = blockIdx.z * a.Hkv + g;  // one merge group per (batch entry, row group, KV head)
 
-  griddep_wait();
+  // The cache length is final before this kernel's predecessor runs (only the
+  // end of a forward pass moves it), and so are the slots below it: both are
+  // read before waiting for the predecessor.  Slots L.. and the queries come
+  // from the QKV projection this kernel follows: the loader waits for it
+  // before those loads, and every other input of the kernel reaches it
+  // through the loader's copies.
   int L = (a.d_lens ? a.d_lens[bidx] : a.d_len ? *a.d_len : a.L_static) - a.len_sub;
   if (a.block_table && L + a.n_rows > a.max_pages * 64) {
     record_error(a.status, DVLM_ERR_BOUNDS);
@@ -160,9 +165,6 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   if (warp == 0) {
     if (lane == 0 && nc > 0) {
       const uint64_t pol = l2_policy_evict_first();
-      mbar_arrive_expect_tx(q_full, 2 * kSpAtom);
-      for (int d = 0; d < 2; ++d)
-        tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, bidx * a.n_rows + t_base, pol);
       // coordinates of 64-key half `hf` of this CTA's chunk c (one page each
       // in a paged cache)
       auto coords = [&](int c, int hf, int& krow, int& vrow, int& vx) {
@@ -203,12 +205,26 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &v_full[st], vx, vrow, pol);
         }
       };
+      // the first stages' chunks that lie wholly below the cache length load
+      // before the wait for the predecessor
+      bool early[kSpStages];
+      for (int c = 0; c < kSpStages; ++c) {
+        early[c] = c < nc && (sp + c * S + 1) * kSpKeys <= L;
+        if (early[c]) {
+          load_k(c);
+          load_v(c);
+        }
+      }
+      griddep_wait();
+      mbar_arrive_expect_tx(q_full, 2 * kSpAtom);
+      for (int d = 0; d < 2; ++d)
+        tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, bidx * a.n_rows + t_base, pol);
       int pf = kSpStages;
       for (int i = 0; i <= nc; ++i) {
         if (i < nc) {
           if (i >= kSpStages && !mbar_wait(&k_empty[i % kSpStages], ((i / kSpStages) - 1) & 1, a.status, sabort))
             break;
-          load_k(i);
+          if (i >= kSpStages || !early[i]) load_k(i);
           for (; pf < nc && pf <= i + kSpPrefetch; ++pf) {
             for (int hf = 0; hf < 2; ++hf) {
               int krow, vrow, vx;
@@ -222,7 +238,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           const int c = i - 1;
           if (c >= kSpStages && !mbar_wait(&v_empty[c % kSpStages], ((c / kSpStages) - 1) & 1, a.status, sabort))
             break;
-          load_v(c);
+          if (c >= kSpStages || !early[c]) load_v(c);
         }
       }
     }
