@@ -1213,10 +1213,15 @@ dvlm_status engine_set_option(dvlm_engine* e, const char* name, int v) {
   } else if (n == "down_stages") {
     if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
     if (!cluster_ok(EPI_RESID, e->s_down, v, h_tiles)) return DVLM_ERR_UNSUPPORTED;
+    // 5-stage down CTAs fit beside 5-stage gate/up CTAs: launched early, they
+    // could take the room of gate/up CTAs not yet resident, whose stream-K
+    // partials the resident ones wait for (the wait would run out)
+    if (v == 5 && e->gu_stages == 5) return DVLM_ERR_UNSUPPORTED;
     e->down_stages = v;
   } else if (n == "gateup_stages") {
     if (v != 5 && v != 10) return DVLM_ERR_SHAPE;
     if (v == 10 && e->gu_cps == 2) return DVLM_ERR_UNSUPPORTED;
+    if (v == 5 && e->down_stages == 5) return DVLM_ERR_UNSUPPORTED;  // see "down_stages"
     e->gu_stages = v;
   } else if (n == "gateup_ctas_per_sm") {
     if (v != 1 && v != 2) return DVLM_ERR_SHAPE;

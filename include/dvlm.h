@@ -459,7 +459,8 @@ DVLM_API dvlm_status dvlm_forward_quad(dvlm_engine* e, const int32_t* draft, int
  * creation from occupancy queries).  Names and values:
  *   "qkv_cluster", "o_cluster", "down_cluster": CTAs per cluster of the
  *       cluster split-K projections (2..16; 0 = stream-K kernel instead);
- *   "down_stages", "gateup_stages": TMA pipeline depth, 5 or 10;
+ *   "down_stages", "gateup_stages": TMA pipeline depth, 5 or 10 (not both 5:
+ *       UNSUPPORTED);
  *   "gateup_ctas_per_sm": 1, or 2 with 5 gate/up stages;
  *   "attn_cluster": CTAs per attention cluster, 8 or 16;
  *   "pdl": 1/0, programmatic dependent launch between kernels;
