@@ -145,6 +145,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
     e->pao = c.take<void>(C * HD * 2);
     e->pact = c.take<void>(C * I * 2);
     e->pssq = c.take<float>(static_cast<size_t>(H / 128 + 1) * C * 4);
+    e->rope_cs = c.take<float2>(C * 64 * 8);
     e->qtok = c.take<int32_t>(C * 4);
     e->d_k = c.take<int32_t>(4);
     e->kside = c.take<void>(static_cast<size_t>(m.n_kv_heads) * kQuadSideKeys * 128 * 2);
@@ -613,6 +614,8 @@ cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, c
   ta.L0 = 0;
   ta.log2_rope_base = std::log2(static_cast<double>(m.rope_base));
   ta.status = e->d_status;
+  ta.rope_cs = e->rope_cs;
+  DVLM_CK(launch_rope_table(e->rope_cs, ta, s));
   PrefillAttnArgs pa{};
   pa.n_tok = n;
   pa.L0 = 0;
@@ -716,6 +719,8 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
   ta.kside = static_cast<bf16*>(e->kside);
   ta.vside = static_cast<bf16*>(e->vside);
   ta.side_n = kQuadSideKeys;
+  ta.rope_cs = e->rope_cs;
+  DVLM_CK(launch_rope_table(e->rope_cs, ta, s));
   AttnArgs aa{};
   aa.n_rows = B;
   aa.n_clean = B;

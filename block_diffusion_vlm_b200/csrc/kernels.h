@@ -239,6 +239,9 @@ struct TmArgs {
   int splits;
   float* part;
   int* cnt;
+  // QKV: (cos, sin) of the RoPE angle of row tok and frequency j at
+  // rope_cs[tok * 64 + j] (launch_rope_table fills it for these arguments)
+  const float2* rope_cs;
   // QKV of the fused draft+verify forward (quad_B = B > 0): rows 0..B-1 are
   // the verify rows (slots L..L+B-1, K/V to the cache); row B + i*B + r is row
   // r of candidate block i at position L+i+1+r, its K/V to kside
@@ -251,6 +254,12 @@ struct TmArgs {
 };
 // y = x W^T over n_wtiles tiles of 256 weight rows (SWIGLU: 128 rows of W and
 // the same 128 rows of W2) starting at weight row w_row_base; kb = K / 64.
+// (cos, sin) of every row's RoPE angles for the token-major QKV epilogue:
+// row tok sits at position L0 + tok (L0 = *d_len when set), or for the
+// candidate rows of a fused draft+verify forward (quad_B > 0, tok >= B) at
+// L0 + i + 1 + r for row r of block i; frequency j of 64 is
+// base^(-2j/128).  Angles and sincos in fp64, rounded to fp32.
+cudaError_t launch_rope_table(float2* cs, const TmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, const CUtensorMap& mapW2, int kb,
                            int w_row_base, int n_wtiles, const TmArgs& a, cudaStream_t s);
 struct PrefillAttnArgs {

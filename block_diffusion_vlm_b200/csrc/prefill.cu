@@ -86,6 +86,21 @@ __device__ __forceinline__ void store_bf16x16(bf16* dst, const float (&v)[16]) {
 }
 }  // namespace
 
+// (cos, sin) of the RoPE angle of row tok, frequency j (see launch_rope_table).
+__global__ void rope_table_kernel(float2* __restrict__ cs, const TmArgs a) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= a.n_tok * 64) return;
+  const int tok = idx >> 6, j = idx & 63;
+  const int L0 = a.d_len ? *a.d_len : a.L0;
+  const int Bq = a.quad_B;
+  const bool cand = Bq > 0 && tok >= Bq;
+  const int pos = cand ? L0 + (tok - Bq) / Bq + 1 + (tok - Bq) % Bq : L0 + tok;
+  const double inv_freq = exp2(-(2.0 * j / 128.0) * a.log2_rope_base);
+  double sn, c;
+  sincos(static_cast<double>(pos) * inv_freq, &sn, &c);
+  cs[idx] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kTmThreads, 1)
     gemm_tm_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
@@ -183,14 +198,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
     const int tile = tt * gridDim.y + T;
     if (S > 1) {
       if (got) {
-        float* mine = a.part + (static_cast<size_t>(tile) * S + z) * 128 * 256 + static_cast<size_t>(row) * 256;
+        // partial tile as [column group of 4][row] float4: a warp's 32 rows
+        // of one group are 512 contiguous bytes (stores and the last CTA's
+        // loads coalesce)
+        float4* mine = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(tile) * S + z) * 128 * 256) + row;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 16) {
           float v[16];
           acc16(tmem, quarter, c, v);
 #pragma unroll
-          for (int q = 0; q < 16; q += 4)
-            __stcg(reinterpret_cast<float4*>(mine + c + q), make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]));
+          for (int q = 0; q < 16; q += 4) __stcg(mine + ((c + q) >> 2) * 128, make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]));
         }
       }
       __threadfence();
@@ -213,11 +230,11 @@ __global__ void __launch_bounds__(kTmThreads, 1)
 #pragma unroll
       for (int q = 0; q < 16; ++q) v[q] = 0.f;
       for (int zz = 0; zz < S; ++zz) {
-        const float4* src = reinterpret_cast<const float4*>(
-            a.part + (static_cast<size_t>(tile) * S + zz) * 128 * 256 + static_cast<size_t>(row) * 256 + c);
+        const float4* src =
+            reinterpret_cast<const float4*>(a.part + (static_cast<size_t>(tile) * S + zz) * 128 * 256) + row;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float4 f = __ldcg(src + q);
+          const float4 f = __ldcg(src + ((c >> 2) + q) * 128);
           v[4 * q] += f.x;
           v[4 * q + 1] += f.y;
           v[4 * q + 2] += f.z;
@@ -289,13 +306,17 @@ __global__ void __launch_bounds__(kTmThreads, 1)
               float x1[16], x2[16], y1[16], y2[16];
               cols(i * 128 + j0, x1);
               cols(i * 128 + 64 + j0, x2);
+              const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(valid ? tok : 0) * 64 + j0);
+              float2 csj[16];
+#pragma unroll
+              for (int k = 0; k < 16; k += 2) {
+                const float4 f = __ldg(cs4 + k / 2);
+                csj[k] = make_float2(f.x, f.y);
+                csj[k + 1] = make_float2(f.z, f.w);
+              }
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
-                const int j = j0 + k;
-                const double inv_freq = exp2(-(2.0 * j / 128.0) * a.log2_rope_base);
-                double sn, cs;
-                sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
-                const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+                const float c = csj[k].x, s = csj[k].y;
                 const float u1 = x1[k] * r, u2 = x2[k] * r;
                 y1[k] = u1 * c - u2 * s;
                 y2[k] = u2 * c + u1 * s;
@@ -642,9 +663,16 @@ static cudaError_t tm_launch(const CUtensorMap& mapX, const CUtensorMap& mapW, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_rope_table(float2* cs, const TmArgs& a, cudaStream_t s) {
+  if (!cs || a.n_tok < 1) return cudaErrorInvalidValue;
+  rope_table_kernel<<<(a.n_tok * 64 + 255) / 256, 256, 0, s>>>(cs, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, const CUtensorMap& mapW2, int kb,
                            int w_row_base, int n_wtiles, const TmArgs& a, cudaStream_t s) {
   if (a.n_tok < 1 || kb < 1 || n_wtiles < 1) return cudaErrorInvalidValue;
+  if (a.epi == EPI_QKV && !a.rope_cs) return cudaErrorInvalidValue;
   if (a.quad_B > 0 && (a.side_n < 64 * a.quad_B || !a.kside || !a.vside)) return cudaErrorInvalidValue;
   switch (a.epi) {
     case EPI_QKV: return tm_launch<EPI_QKV>(mapX, mapW, mapW2, kb, w_row_base, n_wtiles, a, s);
