@@ -144,7 +144,7 @@ static size_t carve(dvlm_engine* e, uint8_t* base, bool dry, int P) {
     e->pq = c.take<void>(C * HD * 2);
     e->pao = c.take<void>(C * HD * 2);
     e->pact = c.take<void>(C * I * 2);
-    e->pssq = c.take<float>(static_cast<size_t>(H / 128 + 1) * C * 4);
+    e->pssq = c.take<float>(static_cast<size_t>(std::max(H / 128 + 1, (H / 256) * 16)) * C * 4);
     e->rope_cs = c.take<float2>(C * 64 * 8);
     e->qtok = c.take<int32_t>(C * 4);
     e->d_k = c.take<int32_t>(4);
@@ -672,10 +672,12 @@ cudaError_t engine_prefill_gemm(dvlm_engine* e, const void* vision, int n_vis, c
 }
 
 // Split-K factor of a token-major GEMM with n_tiles output tiles and kb k
-// blocks: enough CTAs to cover the SMs, at least 4 k blocks each.
-static int tm_splits(const dvlm_engine* e, int n_tiles, int kb) {
+// blocks: enough CTAs to cover the SMs (all resident: the CTAs of a tile
+// wait for one another), at least 4 k blocks each, at most `cap` (the tile's
+// epilogue units: 16 for the residual epilogue, 8 otherwise).
+static int tm_splits(const dvlm_engine* e, int n_tiles, int kb, int cap) {
   if (n_tiles >= e->sm) return 1;
-  return std::max(1, std::min(kb / 4, e->sm / n_tiles));
+  return std::max(1, std::min(cap, std::min(kb / 4, e->sm / n_tiles)));
 }
 
 bool quad_supported(const dvlm_engine* e, int B) {
@@ -744,15 +746,21 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
   pa.quad_B = B;
   pa.d_len = e->d_len;
   pa.side_n = kQuadSideKeys;
+  // split-K factors (the residual epilogues leave (H / 256) * S sums of
+  // squares per row for the next RMSNorm)
+  const int s_qkv = tm_splits(e, n_tt * (qkv_rows / 256), H / 64, 8);
+  const int s_o = tm_splits(e, n_tt * (H / 256), Hq * D / 64, 16);
+  const int s_gu = tm_splits(e, n_tt * (I / 128), H / 64, 8);
+  const int s_down = tm_splits(e, n_tt * (H / 256), I / 64, 16);
   for (int l = 0; l < m.n_layers; ++l) {
     ta.epi = EPI_QKV;
     ta.ssq_in = e->pssq;
-    ta.n_ssq = l == 0 ? H / 128 : H / 256;
+    ta.n_ssq = l == 0 ? H / 128 : (H / 256) * s_down;
     ta.out = static_cast<bf16*>(e->pq);
     ta.out_ld = Hq * D;
     ta.kcache = static_cast<bf16*>(e->kc) + l * kv_layer;
     ta.vcache = static_cast<bf16*>(e->vc) + l * kv_layer;
-    ta.splits = tm_splits(e, n_tt * (qkv_rows / 256), H / 64);
+    ta.splits = s_qkv;
     DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wqkv_p, e->tm_wqkv_p, H / 64, l * qkv_rows, qkv_rows / 256, ta, s));
     aa.kv_base = l;
     DVLM_CK(launch_attn_split_cl(e->tm_q3, e->tm_k, e->tm_v, aa, e->attn_cs, false, s));
@@ -762,16 +770,16 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
     ta.resid = px;
     ta.resid_ld = H;
     ta.ssq_out = e->pssq;
-    ta.splits = tm_splits(e, n_tt * (H / 256), Hq * D / 64);
+    ta.splits = s_o;
     DVLM_CK(launch_gemm_tm(e->tm_pao, e->tm_wo_p, e->tm_wo_p, Hq * D / 64, l * H, H / 256, ta, s));
     ta.epi = EPI_SWIGLU;
-    ta.n_ssq = H / 256;
+    ta.n_ssq = (H / 256) * s_o;
     ta.out = static_cast<bf16*>(e->pact);
     ta.out_ld = I;
-    ta.splits = tm_splits(e, n_tt * (I / 128), H / 64);
+    ta.splits = s_gu;
     DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wg_p, e->tm_wu_p, H / 64, l * I, I / 128, ta, s));
     ta.epi = EPI_RESID;
-    ta.splits = tm_splits(e, n_tt * (H / 256), I / 64);
+    ta.splits = s_down;
     DVLM_CK(launch_gemm_tm(e->tm_pact, e->tm_wd_p, e->tm_wd_p, I / 64, l * H, H / 256, ta, s));
   }
   return cudaSuccess;

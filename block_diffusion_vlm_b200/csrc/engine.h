@@ -145,7 +145,7 @@ struct dvlm_engine {
   void* pq = nullptr;            // [max_ctx][Hq*D]
   void* pao = nullptr;           // [max_ctx][Hq*D] attention output
   void* pact = nullptr;          // [max_ctx][I] SwiGLU activation
-  float* pssq = nullptr;         // [H/128][max_ctx] sums of squares
+  float* pssq = nullptr;         // [max(H/128 + 1, 16 H/256)][max_ctx] sums of squares
   float2* rope_cs = nullptr;     // [max_ctx][64] (cos, sin) of each context row's RoPE angles
   float* amax_act = nullptr;     // fp8: [I/64][NT] largest |SwiGLU activation| per gate/up tile
   void* attn_scratch = nullptr;  // split attention partials (up to kMaxAttnSplit CTAs per KV head)

@@ -234,8 +234,10 @@ struct TmArgs {
   int* status;
   // split-K: grid z = splits CTAs per output tile, each over k blocks
   // [z*kb/splits, (z+1)*kb/splits); fp32 partial tiles part[(tile*splits+z)]
-  // [128][256] and per-tile arrival counters cnt (zero between launches): the
-  // last CTA of a tile adds the partials in z order and runs the epilogue.
+  // (128 x 256) and per-tile counters cnt[0..1024) (zero between launches):
+  // the whole grid is resident, the CTAs of a tile wait for one another and
+  // CTA z adds the partials in z order for its 1/splits of the epilogue
+  // (RESID: its sums of squares go to ssq_out entry T * splits + z).
   int splits;
   float* part;
   int* cnt;

@@ -42,6 +42,7 @@ namespace {
 // ---------------------------------------------------------------- GEMM
 constexpr int kTmThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTmStages = 4;
+constexpr int kTmCntStride = 512;      // split-K counters: [0, 512) arrivals per tile, [512, 1024) past the wait
 constexpr int kTmA = 128 * 128;        // 128 context rows x 64 k (bf16)
 constexpr int kTmB = 256 * 128;        // 256 weight rows x 64 k
 constexpr int kTmStage = kTmA + kTmB;
@@ -192,15 +193,19 @@ __global__ void __launch_bounds__(kTmThreads, 1)
     bool got = mbar_wait(accf, 0, a.status, sabort);
     __syncwarp();
     if (got) tc_fence_after();
-    // Split-K: every CTA stores its fp32 partial tile; the last to arrive on
-    // the tile's counter adds all partials in z order (deterministic) and runs
-    // the epilogue on the sums.
+    // Split-K: every CTA stores its fp32 partial tile and counts itself on
+    // the tile's counter; once all S have arrived (the S CTAs of a tile are
+    // resident together: the grid is at most one CTA per SM), CTA z adds the
+    // partials in z order (deterministic) for its 1/S of the tile's epilogue
+    // units and runs the epilogue on those sums.  A second counter, of CTAs
+    // past the wait, lets the last of them zero both for the next launch.
     const int tile = tt * gridDim.y + T;
+    constexpr int kUnits = EPI == EPI_RESID ? 16 : 8;  // 16-column groups (QKV: a head's quarter)
+    int u_lo = 0, u_hi = kUnits;
     if (S > 1) {
       if (got) {
         // partial tile as [column group of 4][row] float4: a warp's 32 rows
-        // of one group are 512 contiguous bytes (stores and the last CTA's
-        // loads coalesce)
+        // of one group are 512 contiguous bytes (stores and loads coalesce)
         float4* mine = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(tile) * S + z) * 128 * 256) + row;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 16) {
@@ -212,13 +217,19 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       }
       __threadfence();
       named_bar_sync(1, 128);
-      if (threadIdx.x == 64) *sflag = (atomicAdd(&a.cnt[tile], 1) == S - 1) ? 1 : 0;
+      if (threadIdx.x == 64) {
+        atomicAdd(&a.cnt[tile], 1);
+        *sflag = wait_counter(&a.cnt[tile], S, a.status, sabort) ? 1 : 0;
+        if (atomicAdd(&a.cnt[kTmCntStride + tile], 1) == S - 1) {  // every CTA of the tile is past the wait
+          a.cnt[tile] = 0;
+          a.cnt[kTmCntStride + tile] = 0;
+        }
+      }
       named_bar_sync(1, 128);
       got = got && *sflag;
-      if (got) {
-        __threadfence();
-        if (threadIdx.x == 64) a.cnt[tile] = 0;  // every partial arrived: zero for the next launch
-      }
+      __threadfence();
+      u_lo = z * kUnits / S;
+      u_hi = (z + 1) * kUnits / S;
     }
     // Columns [c, c+16) of this thread's row: the accumulator, or the sum of
     // the split partials.
@@ -247,7 +258,8 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         bf16* x = a.resid + static_cast<size_t>(tok) * a.resid_ld + T * 256;
         float sq = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 16) {
+        for (int u = u_lo; u < u_hi; ++u) {
+          const int c = u * 16;
           float v[16];
           cols(c, v);  // TMEM loads are warp-collective: every lane loads
           if (valid) {
@@ -269,11 +281,13 @@ __global__ void __launch_bounds__(kTmThreads, 1)
             store_bf16x16(x + c, o);
           }
         }
-        if (valid) a.ssq_out[static_cast<size_t>(T) * a.tok_stride + tok] = sq;
+        // sum of squares over this CTA's columns of the tile: entry T * S + z
+        if (valid) a.ssq_out[(static_cast<size_t>(T) * S + z) * a.tok_stride + tok] = sq;
       } else if (EPI == EPI_SWIGLU) {
         bf16* out = a.out + static_cast<size_t>(tok) * a.out_ld + T * 128;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 16) {
+        for (int uu = u_lo; uu < u_hi; ++uu) {
+          const int c = uu * 16;
           float g[16], u[16];
           cols(c, g);
           cols(128 + c, u);
@@ -295,14 +309,15 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         const int pos = cand ? L0 + ci + 1 + cr : L0 + tok;
         const int side_n = a.side_n;  // keys per KV head in the side buffers
 #pragma unroll 1
-        for (int i = 0; i < 2; ++i) {
+        for (int uu = u_lo; uu < u_hi; ++uu) {  // unit uu: quarter sub of head i of the tile
+          const int i = uu >> 2, sub = uu & 3;
           const int hh = 2 * T + i;
           if (hh < nq + nkv) {
             bf16* dst = hh < nq ? a.out + static_cast<size_t>(tok) * a.out_ld + hh * 128
                         : cand ? a.kside + (static_cast<size_t>(hh - nq) * side_n + ci * 64 + cr) * 128
                                : a.kcache + (static_cast<size_t>(hh - nq) * a.Lmax + pos) * 128;
 #pragma unroll 1
-            for (int j0 = 0; j0 < 64; j0 += 16) {
+            for (int j0 = sub * 16; j0 < sub * 16 + 16; j0 += 16) {
               float x1[16], x2[16], y1[16], y2[16];
               cols(i * 128 + j0, x1);
               cols(i * 128 + 64 + j0, x2);
@@ -329,7 +344,7 @@ __global__ void __launch_bounds__(kTmThreads, 1)
           } else {
             const int h = hh - nq - nkv;
 #pragma unroll 1
-            for (int c = 0; c < 128; c += 16) {
+            for (int c = sub * 32; c < sub * 32 + 32; c += 16) {
               float v[16];
               cols(i * 128 + c, v);
               if (valid) {
@@ -659,6 +674,11 @@ static cudaError_t tm_launch(const CUtensorMap& mapX, const CUtensorMap& mapW, c
   const int n_tt = (a.n_tok + 127) / 128;
   const int S = a.splits > 1 ? a.splits : 1;
   if (S > 1 && (!a.part || !a.cnt || S > kb)) return cudaErrorInvalidValue;
+  // split-K: the S CTAs of a tile wait for one another, so the whole grid
+  // must be resident (one CTA per SM); S <= the tile's epilogue units
+  if (S > 1 && (n_tt * n_wtiles > kTmCntStride || n_tt * n_wtiles * S > device_sm_count() ||
+                S > (EPI == EPI_RESID ? 16 : 8)))
+    return cudaErrorInvalidValue;
   kern<<<dim3(n_tt, n_wtiles, S), kTmThreads, kTmSmem, s>>>(mapX, mapW, mapW2, kb, w_row_base, a);
   return cudaGetLastError();
 }
