@@ -76,7 +76,8 @@ size_t attn_split_scratch_bytes(int n_groups_total, int S) {
 template <int kCL>
 __global__ void __launch_bounds__(kSpThreads, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                      const __grid_constant__ CUtensorMap mapV, const AttnArgs a, float* part, float2* ml,
+                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapKs,
+                      const __grid_constant__ CUtensorMap mapVs, const AttnArgs a, float* part, float2* ml,
                       int* cnt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -117,15 +118,22 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   // from the QKV projection this kernel follows: the loader waits for it
   // before those loads, and every other input of the kernel reaches it
   // through the loader's copies.
-  int L = (a.d_lens ? a.d_lens[bidx] : a.d_len ? *a.d_len : a.L_static) - a.len_sub;
+  // candidate block bidx (cand_B > 0): the cache prefix 0..*d_len + bidx,
+  // then one side chunk of its own cand_B keys
+  const bool cand = a.cand_B > 0;
+  const int L_old = a.d_len ? *a.d_len : a.L_static;  // slots below it predate the predecessor
+  int L = cand ? L_old + bidx + 1 : (a.d_lens ? a.d_lens[bidx] : L_old) - a.len_sub;
   if (a.block_table && L + a.n_rows > a.max_pages * 64) {
     record_error(a.status, DVLM_ERR_BOUNDS);
     L = a.max_pages * 64 - a.n_rows;
   }
-  const int Ltot = L + a.n_rows;
-  const int n_all = (Ltot + kSpKeys - 1) / kSpKeys;
+  const int Ltot = cand ? L : L + a.n_rows;  // cache slots this entry's rows may see
+  const int n_cache = (Ltot + kSpKeys - 1) / kSpKeys;
+  const int n_all = n_cache + (cand ? 1 : 0);
   const int nc = sp < n_all ? (n_all - sp + S - 1) / S : 0;  // this CTA's chunks sp, sp+S, ...
-  const int kv_row0 = (a.kv_base + bidx) * a.Hkv + g;
+  // (cache entry, KV head) row block: batch entry b reads cache entry kv_base + b; the candidate
+  // blocks all read entry kv_base
+  const int kv_row0 = (a.kv_base + (cand ? 0 : bidx)) * a.Hkv + g;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSpBars; ++i) {
@@ -167,8 +175,16 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       const uint64_t pol = l2_policy_evict_first();
       // coordinates of 64-key half `hf` of this CTA's chunk c (one page each
       // in a paged cache)
-      auto coords = [&](int c, int hf, int& krow, int& vrow, int& vx) {
+      // (the side chunk of a candidate block: rows of the side buffers; a
+      // half past its 64 keys reads the next block's rows or zero fill)
+      auto coords = [&](int c, int hf, int& krow, int& vrow, int& vx) -> bool {
         const int key = (sp + c * S) * kSpKeys + hf * 64;
+        if (cand && sp + c * S == n_cache) {
+          krow = g * a.side_n + bidx * 64 + hf * 64;
+          vrow = g * 128;
+          vx = bidx * 64 + hf * 64;
+          return true;
+        }
         if (a.block_table) {
           const int pe = page_entry(key);
           krow = pe * 64;
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           vrow = kv_row0 * 128;
           vx = key;
         }
+        return false;
       };
       // Keys and values have two stages each, released separately: a key
       // stage as soon as S of its chunk is done, a value stage once PV is.
@@ -191,9 +208,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         mbar_arrive_expect_tx(&k_full[st], 2 * kSpAtom);
         for (int hf = 0; hf < 2; ++hf) {
           int krow, vrow, vx;
-          coords(c, hf, krow, vrow, vx);
+          const CUtensorMap* mk = coords(c, hf, krow, vrow, vx) ? &mapKs : &mapK;
           for (int d = 0; d < 2; ++d)
-            tma_load_2d(sK + (2 * st + d) * kSpAtom + hf * (kSpAtom / 2), &mapK, &k_full[st], d * 64, krow, pol);
+            tma_load_2d(sK + (2 * st + d) * kSpAtom + hf * (kSpAtom / 2), mk, &k_full[st], d * 64, krow, pol);
         }
       };
       auto load_v = [&](int c) {
@@ -201,15 +218,15 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         mbar_arrive_expect_tx(&v_full[st], 2 * kSpAtom);
         for (int hf = 0; hf < 2; ++hf) {
           int krow, vrow, vx;
-          coords(c, hf, krow, vrow, vx);
-          tma_load_2d(sV + (2 * st + hf) * kSpAtom, &mapV, &v_full[st], vx, vrow, pol);
+          const CUtensorMap* mv = coords(c, hf, krow, vrow, vx) ? &mapVs : &mapV;
+          tma_load_2d(sV + (2 * st + hf) * kSpAtom, mv, &v_full[st], vx, vrow, pol);
         }
       };
       // the first stages' chunks that lie wholly below the cache length load
       // before the wait for the predecessor
       bool early[kSpStages];
       for (int c = 0; c < kSpStages; ++c) {
-        early[c] = c < nc && (sp + c * S + 1) * kSpKeys <= L;
+        early[c] = c < nc && (sp + c * S + 1) * kSpKeys <= (cand ? L_old : L);
         if (early[c]) {
           load_k(c);
           load_v(c);
@@ -218,7 +235,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       griddep_wait();
       mbar_arrive_expect_tx(q_full, 2 * kSpAtom);
       for (int d = 0; d < 2; ++d)
-        tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, bidx * a.n_rows + t_base, pol);
+        tma_load_3d(sQ + d * kSpAtom, &mapQ, q_full, d * 64, g * 8, a.q_row0 + bidx * a.n_rows + t_base, pol);
       int pf = kSpStages;
       for (int i = 0; i <= nc; ++i) {
         if (i < nc) {
@@ -228,9 +245,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           for (; pf < nc && pf <= i + kSpPrefetch; ++pf) {
             for (int hf = 0; hf < 2; ++hf) {
               int krow, vrow, vx;
-              coords(pf, hf, krow, vrow, vx);
-              for (int d = 0; d < 2; ++d) tma_prefetch_2d(&mapK, d * 64, krow);
-              tma_prefetch_2d(&mapV, vx, vrow);
+              const bool sd = coords(pf, hf, krow, vrow, vx);
+              for (int d = 0; d < 2; ++d) tma_prefetch_2d(sd ? &mapKs : &mapK, d * 64, krow);
+              tma_prefetch_2d(sd ? &mapVs : &mapV, vx, vrow);
             }
           }
         }
@@ -310,11 +327,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     for (int c = 0; c < nc; ++c) {
       const int vs = c % kSpStages;
       if (!mbar_wait(&v_full[vs], (c / kSpStages) & 1, a.status, sabort)) break;
-      const int key0 = (sp + c * S) * kSpKeys;
+      const bool side = cand && sp + c * S == n_cache;  // a candidate block's own keys
+      const int key0 = side ? 0 : (sp + c * S) * kSpKeys;
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         const int at = j & 1, d = 64 * cw + 32 * (j >> 1) + lane;
-        const int n_valid = Ltot - key0 - at * 64;
+        const int n_valid = (side ? a.cand_B : Ltot) - key0 - at * 64;
         uint8_t* vrow = sV + (2 * vs + at) * kSpAtom + d * 128;
         uint4 w[8];
 #pragma unroll
@@ -389,8 +407,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     }
     for (int c = 0; ok && c < nc; ++c) {
       const int st = c & 1;
-      const int key0 = (sp + c * S) * kSpKeys;
-      const bool full = key0 + kSpKeys <= limit;  // every key of the chunk visible to this row
+      // chunk keys key0 .. key0 + 127 against the visible bound lim (the side
+      // chunk of a candidate block: its own keys 0 .. cand_B - 1)
+      const bool side = cand && sp + c * S == n_cache;
+      const int key0 = side ? 0 : (sp + c * S) * kSpKeys;
+      const int lim = side ? a.cand_B : limit;
+      const bool full = key0 + kSpKeys <= lim;  // every key of the chunk visible to this row
       if (!mbar_wait(&s_full[st], (c >> 1) & 1, a.status, sabort)) {
         ok = false;
         break;
@@ -411,7 +433,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         const int kme = key0 + hf * 64;
 #pragma unroll
         for (int k = 0; k < 64; ++k)
-          if (kme + k < limit) mv[k & 7] = fmaxf(mv[k & 7], sc[k]);
+          if (kme + k < lim) mv[k & 7] = fmaxf(mv[k & 7], sc[k]);
       }
       const float mh = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
                              fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
@@ -446,9 +468,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         const int kme = key0 + hf * 64;
 #pragma unroll
         for (int k = 0; k < 64; k += 2) {
-          const float p0 = (kme + k < limit && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
+          const float p0 = (kme + k < lim && m_new != -INFINITY) ? ex2_approx(sc[k] * a.scale_log2 - m_new) : 0.f;
           const float p1 =
-              (kme + k + 1 < limit && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
+              (kme + k + 1 < lim && m_new != -INFINITY) ? ex2_approx(sc[k + 1] * a.scale_log2 - m_new) : 0.f;
           ps[(k >> 1) & 3] += p0 + p1;
           const __half2 ph = __floats2half2_rn(p0, p1);
           packed[k / 2] = *reinterpret_cast<const uint32_t*>(&ph);
@@ -571,7 +593,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
       const int tr = t_base + (r >> 3);
       if (tr < a.n_rows) {
         const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
-        bf16* dst_o = a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + f0;
+        bf16* dst_o =
+            a.out + ((static_cast<size_t>(a.q_row0) + bidx * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + f0;
 #pragma unroll
         for (int k = 0; k < FPT; k += 4) {
           const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
@@ -661,7 +684,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
           if (tr < a.n_rows) {
             const float inv = sinv[r];
             bf16* dst =
-                a.out + ((static_cast<size_t>(bidx) * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 + lane * 4;
+                a.out + ((static_cast<size_t>(a.q_row0) + bidx * a.n_rows + tr) * a.Hq + g * 8 + (r & 7)) * 128 +
+                lane * 4;
             const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[j].x * inv, acc[j].y * inv);
             const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[j].z * inv, acc[j].w * inv);
             *reinterpret_cast<uint2*>(dst) =
@@ -719,7 +743,7 @@ cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, 
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_split_kernel<0>, mapQ, mapK, mapV, a, p, m, c);
+  return cudaLaunchKernelEx(&cfg, attn_split_kernel<0>, mapQ, mapK, mapV, mapK, mapV, a, p, m, c);
 }
 
 template <int CL>
@@ -732,8 +756,9 @@ static cudaError_t split_cl_attr() {
 
 // One cluster of cs CTAs (8 or 16) per (batch entry, row group, KV head);
 // no scratch.
-cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                                 const AttnArgs& a, int cs, bool pdl, cudaStream_t s) {
+static cudaError_t split_cl_launch(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                   const CUtensorMap& mapKs, const CUtensorMap& mapVs, const AttnArgs& a, int cs,
+                                   bool pdl, cudaStream_t s) {
   if (cs != 8 && cs != 16) return cudaErrorInvalidValue;
   static bool attr_set[2][64] = {};
   int dev = 0;
@@ -760,10 +785,25 @@ cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& map
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   if (cs == 16)
-    return cudaLaunchKernelEx(&cfg, attn_split_kernel<16>, mapQ, mapK, mapV, a, static_cast<float*>(nullptr),
-                              static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
-  return cudaLaunchKernelEx(&cfg, attn_split_kernel<8>, mapQ, mapK, mapV, a, static_cast<float*>(nullptr),
-                            static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
+    return cudaLaunchKernelEx(&cfg, attn_split_kernel<16>, mapQ, mapK, mapV, mapKs, mapVs, a,
+                              static_cast<float*>(nullptr), static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
+  return cudaLaunchKernelEx(&cfg, attn_split_kernel<8>, mapQ, mapK, mapV, mapKs, mapVs, a,
+                            static_cast<float*>(nullptr), static_cast<float2*>(nullptr), static_cast<int*>(nullptr));
+}
+
+cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                 const AttnArgs& a, int cs, bool pdl, cudaStream_t s) {
+  if (a.cand_B > 0) return cudaErrorInvalidValue;
+  return split_cl_launch(mapQ, mapK, mapV, mapK, mapV, a, cs, pdl, s);
+}
+
+cudaError_t launch_attn_cand_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                const CUtensorMap& mapKs, const CUtensorMap& mapVs, const AttnArgs& a, int cs,
+                                cudaStream_t s) {
+  if (a.cand_B < 1 || a.cand_B > 16 || a.n_rows != a.cand_B || a.n_clean != 0 || a.n_batch != a.cand_B ||
+      !a.d_len || a.block_table || a.len_sub || a.side_n < 64 * a.cand_B)
+    return cudaErrorInvalidValue;
+  return split_cl_launch(mapQ, mapK, mapV, mapKs, mapVs, a, cs, false, s);
 }
 
 // Clusters of cs CTAs of the cluster-merge form that can be resident at once

@@ -204,6 +204,7 @@ static bool build_maps(dvlm_engine* e) {
     ok &= make_tmap_2d(&e->tm_kp, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 128);
     ok &= make_tmap_3d(&e->tm_q3, e->pq, D, Hq, C, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
     ok &= make_tmap_2d(&e->tm_ks, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 128);
+    ok &= make_tmap_2d(&e->tm_ks64, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 64);
     ok &= make_tmap_2d(&e->tm_vs, e->vside, kQuadSideKeys, static_cast<uint64_t>(Hkv) * D, kQuadSideKeys * 2, 64,
                        128);
   }
@@ -734,6 +735,13 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
   aa.scale_log2 = scale_log2;
   aa.out = static_cast<bf16*>(e->pao);
   aa.status = e->d_status;
+  // candidate blocks: B batch entries of B noisy rows from row B on
+  AttnArgs ac = aa;
+  ac.n_clean = 0;
+  ac.n_batch = B;
+  ac.q_row0 = B;
+  ac.cand_B = B;
+  ac.side_n = kQuadSideKeys;
   PrefillAttnArgs pa{};
   pa.n_tok = n;
   pa.Lmax = e->Lmax;
@@ -765,7 +773,8 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
     aa.kv_base = l;
     DVLM_CK(launch_attn_split_cl(e->tm_q3, e->tm_k, e->tm_v, aa, e->attn_cs, false, s));
     pa.kv_base = l;
-    DVLM_CK(launch_attn_cand(e->tm_q3, e->tm_kp, e->tm_v, e->tm_ks, e->tm_vs, pa, s));
+    ac.kv_base = l;
+    DVLM_CK(launch_attn_cand_cl(e->tm_q3, e->tm_k, e->tm_v, e->tm_ks64, e->tm_vs, ac, e->attn_cs, s));
     ta.epi = EPI_RESID;
     ta.resid = px;
     ta.resid_ld = H;

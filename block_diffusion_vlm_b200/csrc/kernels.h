@@ -194,6 +194,15 @@ struct AttnArgs {
   const int* block_table;
   int max_pages, n_pages;
   const int* d_lens;
+  // Queries and outputs start at row q_row0 of their buffers (batch entry b's
+  // rows at q_row0 + b * n_rows).
+  int q_row0;
+  // Candidate blocks of a fused draft+verify forward (cand_B = B > 0,
+  // launch_attn_cand_cl): batch entry b is candidate block b, B noisy rows
+  // that see the cache slots 0..*d_len + b (the context and the first b + 1
+  // draft tokens) and the block's own B keys, side_n-key rows of the side
+  // buffers (K [Hkv][side_n][128], V^T [Hkv][128][side_n]) from key b * 64.
+  int cand_B, side_n;
 };
 // Block attention (csrc/attn_split.cu), two forms of one kernel.  Split form:
 // S independent CTAs per (batch entry, 16-row group, KV head), merged by the
@@ -209,6 +218,11 @@ cudaError_t launch_attn_split(const CUtensorMap& mapQ, const CUtensorMap& mapK, 
 // shared memory; no scratch.
 cudaError_t launch_attn_split_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                  const AttnArgs& a, int cs, bool pdl, cudaStream_t s);
+// Cluster form over the candidate blocks (a.cand_B > 0); mapKs / mapVs: the
+// side buffers with the boxes of mapK / mapV.
+cudaError_t launch_attn_cand_cl(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                                const CUtensorMap& mapKs, const CUtensorMap& mapVs, const AttnArgs& a, int cs,
+                                cudaStream_t s);
 int attn_split_cl_max_clusters(int cs);
 
 // Prefill (compute-bound path over the whole context; csrc/prefill.cu).
