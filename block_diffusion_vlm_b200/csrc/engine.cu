@@ -203,8 +203,7 @@ static bool build_maps(dvlm_engine* e) {
     ok &= make_tmap_2d(&e->tm_wu_p, m.wup, H, static_cast<uint64_t>(L) * I, H * 2, 64, 128);
     ok &= make_tmap_2d(&e->tm_kp, e->kc, D, static_cast<uint64_t>(L) * Hkv * e->Lmax, D * 2, 64, 128);
     ok &= make_tmap_3d(&e->tm_q3, e->pq, D, Hq, C, D * 2, static_cast<uint64_t>(Hq) * D * 2, 64, 8, 16);
-    ok &= make_tmap_2d(&e->tm_ks, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 128);
-    ok &= make_tmap_2d(&e->tm_ks64, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 64);
+    ok &= make_tmap_2d(&e->tm_ks, e->kside, D, static_cast<uint64_t>(Hkv) * kQuadSideKeys, D * 2, 64, 64);
     ok &= make_tmap_2d(&e->tm_vs, e->vside, kQuadSideKeys, static_cast<uint64_t>(Hkv) * D, kQuadSideKeys * 2, 64,
                        128);
   }
@@ -742,18 +741,6 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
   ac.q_row0 = B;
   ac.cand_B = B;
   ac.side_n = kQuadSideKeys;
-  PrefillAttnArgs pa{};
-  pa.n_tok = n;
-  pa.Lmax = e->Lmax;
-  pa.Hq = Hq;
-  pa.Hkv = Hkv;
-  pa.scale_log2 = scale_log2;
-  pa.out = static_cast<bf16*>(e->pao);
-  pa.out_ld = Hq * D;
-  pa.status = e->d_status;
-  pa.quad_B = B;
-  pa.d_len = e->d_len;
-  pa.side_n = kQuadSideKeys;
   // split-K factors (the residual epilogues leave (H / 256) * S sums of
   // squares per row for the next RMSNorm)
   const int s_qkv = tm_splits(e, n_tt * (qkv_rows / 256), H / 64, 8);
@@ -772,9 +759,8 @@ static cudaError_t quad_forward(dvlm_engine* e, int B, cudaStream_t s) {
     DVLM_CK(launch_gemm_tm(e->tm_px, e->tm_wqkv_p, e->tm_wqkv_p, H / 64, l * qkv_rows, qkv_rows / 256, ta, s));
     aa.kv_base = l;
     DVLM_CK(launch_attn_split_cl(e->tm_q3, e->tm_k, e->tm_v, aa, e->attn_cs, false, s));
-    pa.kv_base = l;
     ac.kv_base = l;
-    DVLM_CK(launch_attn_cand_cl(e->tm_q3, e->tm_k, e->tm_v, e->tm_ks64, e->tm_vs, ac, e->attn_cs, s));
+    DVLM_CK(launch_attn_cand_cl(e->tm_q3, e->tm_k, e->tm_v, e->tm_ks, e->tm_vs, ac, e->attn_cs, s));
     ta.epi = EPI_RESID;
     ta.resid = px;
     ta.resid_ld = H;

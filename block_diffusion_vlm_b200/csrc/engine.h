@@ -167,11 +167,10 @@ struct dvlm_engine {
   int32_t* f_id = nullptr;       // [NT]
   // tensor maps
   CUtensorMap tm_wqkv, tm_wo, tm_wg, tm_wu, tm_wd, tm_lm, tm_x, tm_ao, tm_act, tm_q, tm_k, tm_v;
-  CUtensorMap tm_ks64;  // candidate blocks' side K with the decode K box (64 features x 64 keys)
   // prefill: activations (128-row boxes), weights (256-row boxes; gate/up 128), K (128-key boxes)
   CUtensorMap tm_px, tm_pq, tm_pao, tm_pact, tm_wqkv_p, tm_wo_p, tm_wd_p, tm_wg_p, tm_wu_p, tm_kp;
   // fused forward: q rows as 16-row x 8-head boxes, candidate side buffers
-  CUtensorMap tm_q3, tm_ks, tm_vs;
+  CUtensorMap tm_q3, tm_ks, tm_vs;  // quad: q rows (3-D), side K and V^T with the decode attention's boxes
   // captured graphs keyed by (kind, B, threshold bits, max_new)
   std::map<std::vector<long long>, cudaGraphExec_t> graphs;
 };

@@ -286,22 +286,9 @@ struct PrefillAttnArgs {
   bf16* out;                  // [n_tok][out_ld], head h at column h * 128
   int out_ld;
   int* status;
-  // candidate blocks of the fused draft+verify forward (launch_attn_cand):
-  // B = quad_B, cache length *d_len, side buffers with side_n keys per head
-  int quad_B;
-  const int* d_len;
-  int side_n;
 };
 cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                 const PrefillAttnArgs& a, cudaStream_t s);
-// Candidate block i (B noisy rows at positions L+i+1..) of the fused forward
-// sees cache slots 0..L+i and its own B keys from the side buffers
-// [Fast-dVLM technical overview (ocdem.com), section 2.3.1].  mapQ: 3-D map
-// of the q rows (box 64 x 8 heads x 16 rows); mapK/mapV: the cache maps
-// (128-key K boxes, 64-key V^T boxes); mapKs/mapVs: the side buffers.
-cudaError_t launch_attn_cand(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                             const CUtensorMap& mapKs, const CUtensorMap& mapVs, const PrefillAttnArgs& a,
-                             cudaStream_t s);
 
 // FP8 E4M3 row quantisation (csrc/fp8.cu): codes [rows][K], scales [rows].
 cudaError_t launch_quantize_rows_e4m3(const bf16* a, int rows, int K, uint8_t* codes, float* scales, cudaStream_t s);

@@ -372,16 +372,11 @@ __global__ void __launch_bounds__(kTmThreads, 1)
 }
 
 // Causal attention of n_tok prefill rows (slots L0..L0+n_tok-1, their K/V
-// already in the cache) over the cache slots 0..L0+n_tok-1 (CAND = false:
-// one CTA per 128 rows of one query head).  CAND = true: candidate block
-// blockIdx.x of the fused draft+verify forward, one CTA per (block, KV head),
-// its 16 rows x 8 query heads as the 128-row tile; it sees cache slots
-// 0..L+i (chunks of 128 keys) and then its own B keys (one side chunk).
-template <bool CAND>
+// already in the cache) over the cache slots 0..L0+n_tok-1: one CTA per 128
+// rows of one query head.
 __global__ void __launch_bounds__(kPaThreads, 1)
     attn_tile_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapKs,
-                     const __grid_constant__ CUtensorMap mapVs, const PrefillAttnArgs a) {
+                     const __grid_constant__ CUtensorMap mapV, const PrefillAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem + oPaQ;
@@ -400,14 +395,12 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   volatile int* sabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x;                              // query tile (CAND: candidate block)
-  const int h = CAND ? 0 : blockIdx.y;                    // query head (prefill)
-  const int g = CAND ? blockIdx.y : h / (a.Hq / a.Hkv);   // KV head
+  const int qt = blockIdx.x;                              // query tile
+  const int h = blockIdx.y;                               // query head
+  const int g = h / (a.Hq / a.Hkv);                       // KV head
   const int Ltot = a.L0 + a.n_tok;
-  const int Lc = CAND ? *a.d_len + qt + 1 : 0;            // cache slots a candidate block sees
   const int q_last = min(a.L0 + qt * 128 + 127, Ltot - 1);  // last query slot of a prefill tile
-  const int n_cache = CAND ? (Lc + kPaKeys - 1) / kPaKeys : q_last / kPaKeys + 1;
-  const int nc = n_cache + (CAND ? 1 : 0);                // + the candidate's own keys
+  const int nc = q_last / kPaKeys + 1;
   const int kv_row0 = a.kv_base * a.Hkv + g;  // (layer, KV head) entry of the cache
 
   if (threadIdx.x == 0) {
@@ -417,10 +410,6 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     tma_prefetch_map(&mapQ);
     tma_prefetch_map(&mapK);
     tma_prefetch_map(&mapV);
-    if (CAND) {
-      tma_prefetch_map(&mapKs);
-      tma_prefetch_map(&mapVs);
-    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kPaTmem);
@@ -435,28 +424,16 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_last();
       mbar_arrive_expect_tx(q_full, 2 * kPaAtom);
-      for (int d = 0; d < 2; ++d) {
-        if (CAND)  // 16 rows x 8 heads of the block: row r*8 + hl of the tile
-          tma_load_3d(sQ + d * kPaAtom, &mapQ, q_full, d * 64, g * 8, a.quad_B + qt * a.quad_B, pol);
-        else
-          tma_load_2d(sQ + d * kPaAtom, &mapQ, q_full, h * 128 + d * 64, qt * 128, pol);
-      }
+      for (int d = 0; d < 2; ++d) tma_load_2d(sQ + d * kPaAtom, &mapQ, q_full, h * 128 + d * 64, qt * 128, pol);
       for (int c = 0; c < nc; ++c) {
         const int st = c & 1;
         if (c >= 2 && !mbar_wait(&kv_empty[st], ((c >> 1) - 1) & 1, a.status, sabort)) break;
         mbar_arrive_expect_tx(&kv_full[st], 4 * kPaAtom);
-        if (CAND && c == n_cache) {  // the block's own keys: side entries qt*64 .. qt*64 + B - 1
-          for (int d = 0; d < 2; ++d)
-            tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapKs, &kv_full[st], d * 64, g * a.side_n + qt * 64, pol);
-          for (int k = 0; k < 2; ++k)
-            tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapVs, &kv_full[st], qt * 64 + k * 64, g * 128, pol);
-        } else {
-          const int key0 = c * kPaKeys;
-          for (int d = 0; d < 2; ++d)
-            tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapK, &kv_full[st], d * 64, kv_row0 * a.Lmax + key0, pol);
-          for (int k = 0; k < 2; ++k)
-            tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapV, &kv_full[st], key0 + k * 64, kv_row0 * 128, pol);
-        }
+        const int key0 = c * kPaKeys;
+        for (int d = 0; d < 2; ++d)
+          tma_load_2d(sK + (2 * st + d) * kPaAtom, &mapK, &kv_full[st], d * 64, kv_row0 * a.Lmax + key0, pol);
+        for (int k = 0; k < 2; ++k)
+          tma_load_2d(sV + (2 * st + k) * kPaAtom, &mapV, &kv_full[st], key0 + k * 64, kv_row0 * 128, pol);
       }
     }
   } else if (warp == 1) {
@@ -518,12 +495,10 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int tok = qt * 128 + row;
-    const int cr = row >> 3, hl = row & 7;      // CAND: block row and query head within the group
-    const bool valid = CAND ? cr < a.quad_B : tok < a.n_tok;
+    const bool valid = tok < a.n_tok;
     const int qslot = valid ? a.L0 + tok : Ltot - 1;  // prefill rows past the end: finite, never written
     // key j of chunk c is visible to this row
     auto visible = [&](int c, int j) -> bool {
-      if (CAND) return c == n_cache ? j < a.quad_B : c * kPaKeys + j < Lc;
       return c * kPaKeys + j <= qslot;
     };
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -604,7 +579,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       // (prefill) or are zeroed here (candidate blocks: stale or poisoned
       // slots past L+i, padding of the side chunk)
       {
-        const int n_valid = CAND ? (c == n_cache ? a.quad_B : Lc - c * kPaKeys) : kPaKeys;
+        const int n_valid = kPaKeys;
         if (!mbar_wait(&kv_full[st], (c >> 1) & 1, a.status, sabort)) {
           ok = false;
           break;
@@ -639,8 +614,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     if (ok && mbar_wait(pv_done, (nc - 1) & 1, a.status, sabort)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      bf16* dst = CAND ? a.out + static_cast<size_t>(a.quad_B + qt * a.quad_B + cr) * a.out_ld + (g * 8 + hl) * 128
-                       : a.out + static_cast<size_t>(tok) * a.out_ld + h * 128;
+      bf16* dst = a.out + static_cast<size_t>(tok) * a.out_ld + h * 128;
 #pragma unroll 1
       for (int cc = 0; cc < 128; cc += 64) {
         float o[64];
@@ -705,22 +679,11 @@ cudaError_t launch_gemm_tm(const CUtensorMap& mapX, const CUtensorMap& mapW, con
 cudaError_t launch_attn_prefill(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                                 const PrefillAttnArgs& a, cudaStream_t s) {
   if (a.n_tok < 1 || a.Hq % a.Hkv) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
+  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
   if (e != cudaSuccess) return e;
-  attn_tile_kernel<false><<<dim3((a.n_tok + 127) / 128, a.Hq), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, mapK,
-                                                                                         mapV, a);
+  attn_tile_kernel<<<dim3((a.n_tok + 127) / 128, a.Hq), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_cand(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                             const CUtensorMap& mapKs, const CUtensorMap& mapVs, const PrefillAttnArgs& a,
-                             cudaStream_t s) {
-  if (a.quad_B < 1 || a.quad_B > 16 || !a.d_len || a.Hq != 8 * a.Hkv || a.side_n < 64 * a.quad_B)
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmem);
-  if (e != cudaSuccess) return e;
-  attn_tile_kernel<true><<<dim3(a.quad_B, a.Hkv), kPaThreads, kPaSmem, s>>>(mapQ, mapK, mapV, mapKs, mapVs, a);
-  return cudaGetLastError();
-}
 
 }  // namespace dvlm
