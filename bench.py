@@ -574,10 +574,11 @@ def run_sweep(args, local, sink=None):
         del qd, kd, vt, out
 
     def auto_splits(B, L, nb):
-        # enough CTAs to fill the SMs (one CTA per 128-key chunk at most)
+        # as many CTAs as fit in one wave on the SMs (one CTA per SM; at most
+        # one CTA per 128-key chunk)
         n_chunks = (L + B + 127) // 128
         groups = nb * ((B + 15) // 16) * Hkv
-        return max(1, min(n_chunks, 32, (148 + groups - 1) // groups))
+        return max(1, min(n_chunks, 32, 148 // groups))
 
     if args.sweep == "compact":
         # the decode shape and the bandwidth case, one line each per kernel
