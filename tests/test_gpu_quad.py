@@ -5,8 +5,10 @@ O(B^2) cost] against the oracle's forward_quadratic / decode_spec_quadratic.
 * The fused forward alone (dvlm_forward_quad): all B + B*B final hidden rows
   (verify rows, then every candidate block) and the verify rows' K/V in the
   cache, against the oracle's fused forward within the bf16 bar (2e-2 plus
-  one storage ulp), for B = 4 and B = 16 over a 48-slot context, and after
-  stale NaN-poisoned slots past L + B (no candidate block may read them).
+  one storage ulp), for B = 4 and B = 16 over a 48-slot context, for B = 8
+  on a wider model (SwiGLU 4096: the token-major GEMMs split their k range up
+  to 16 ways, gate/up tiles included), and after stale NaN-poisoned slots
+  past L + B (no candidate block may read them).
 * Decoding through the engine's own graph path (mode DVLM_MODE_SPEC_QUAD):
   every forward replayed against the oracle, teacher-forced
   (tests/decode_replay.py): verify and candidate rows within the bf16 bar,
@@ -32,15 +34,22 @@ SMALL = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_d
                       lm_scale=25.0, dtype="bf16")
 
 
+# SwiGLU width 4096: the token-major down projection (64 k blocks) splits its
+# k range 16 ways over 4 output tiles at B = 8 (72 rows, one token tile), the
+# largest split the residual epilogue allows
+WIDE = gen.ModelDims(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=128, inter=4096, vocab=4096,
+                     lm_scale=25.0, dtype="bf16")
+
+
 class Quad:
-    def __init__(self, cuda, seed, Lmax=512, max_ctx=320):
-        self.cuda, self.seed = cuda, seed
-        self.dm = DeviceModel(SMALL, seed, device=cuda)
+    def __init__(self, cuda, seed, Lmax=512, max_ctx=320, dims=SMALL):
+        self.cuda, self.seed, self.dims = cuda, seed, dims
+        self.dm = DeviceModel(dims, seed, device=cuda)
         self.cm = self.dm.c_model()
-        self.kc, self.vc = kv_buffers(SMALL, Lmax, device=cuda)
+        self.kc, self.vc = kv_buffers(dims, Lmax, device=cuda)
         self.ws = ws_tensor(dv.engine_workspace_size(self.cm, Lmax, 16, max_ctx), cuda)
         self.eng = dv.Engine(self.cm, self.kc, self.vc, Lmax, 16, max_ctx, self.ws)
-        self.vis_t, self.vis, self.ids = gen.decode_context(SMALL, seed, 32, 16)
+        self.vis_t, self.vis, self.ids = gen.decode_context(dims, seed, 32, 16)
         self.Lmax = Lmax
 
     def prefill(self):
@@ -49,23 +58,23 @@ class Quad:
         return self.eng.position()
 
     def oracle(self):
-        m = O.OracleModel(O.dims_from(SMALL), weights=O.weights_from_generator(gen, SMALL, self.seed), bf16=True,
-                          Lmax=self.Lmax)
+        m = O.OracleModel(O.dims_from(self.dims), weights=O.weights_from_generator(gen, self.dims, self.seed),
+                          bf16=True, Lmax=self.Lmax)
         s = O.prefill(m, self.vis.astype(np.float64), self.ids)
         return m, s
 
 
-@pytest.mark.parametrize("B", [4, 16])
+@pytest.mark.parametrize("B,dims", [(4, SMALL), (16, SMALL), (8, WIDE)], ids=["B4", "B16", "B8-wide"])
 @pytest.mark.parametrize("poison", [False, True])
-def test_fused_forward_matches_oracle(cuda, B, poison):
-    q = Quad(cuda, 2)
+def test_fused_forward_matches_oracle(cuda, B, dims, poison):
+    q = Quad(cuda, 2, dims=dims)
     L, seed = q.prefill()
     if poison:   # stale slots past the context
         q.kc[:, :, :, L:] = float("nan")
         q.vc[:, :, :, :, L:] = float("nan")
     rng = np.random.default_rng(B)
-    draft = [seed] + [int(t) for t in rng.integers(0, SMALL.vocab - 1, size=B - 1)]
-    x = torch.zeros((B + B * B, SMALL.hidden), dtype=torch.bfloat16, device=cuda)
+    draft = [seed] + [int(t) for t in rng.integers(0, dims.vocab - 1, size=B - 1)]
+    x = torch.zeros((B + B * B, dims.hidden), dtype=torch.bfloat16, device=cuda)
     q.eng.forward_quad(torch.tensor(draft, dtype=torch.int32, device=cuda), B, x)
     q.eng.check()
     assert q.eng.position()[0] == L
@@ -74,7 +83,7 @@ def test_fused_forward_matches_oracle(cuda, B, poison):
     assert_bf16_close(f64(x[:B]), xo[:B], 2e-2, "verify rows")
     for i in range(B):
         assert_bf16_close(f64(x[B + i * B:B + (i + 1) * B]), xo[B + i * B:B + (i + 1) * B], 2e-2, f"candidate {i}")
-    for l in range(SMALL.n_layers):
+    for l in range(dims.n_layers):
         assert_bf16_close(f64(q.kc[l, 0, :, L:L + B]), m.K[l][:, L:L + B], 2e-2, f"K layer {l}")
         assert_bf16_close(f64(q.vc[l, 0, :, :, L:L + B]).transpose(0, 2, 1), m.V[l][:, L:L + B], 2e-2,
                           f"V layer {l}")
