@@ -310,3 +310,24 @@ def test_bf16_reduced_model_routing_engine_path(cuda, seed, k):
     assert st.n_text_passes == sum(r.kind == 9 for r in recs) > 0
     print(f"routing seed {seed} k {k}: {rp.t}, text passes {st.n_text_passes} of {st.nfe}")
     s.eng.close()
+
+
+def test_engine_refuses_option_pairs_that_can_stall(cuda):
+    """5-stage gate/up with 5-stage down: early-launched down CTAs fit beside
+    gate/up CTAs and could take the room of gate/up CTAs whose stream-K
+    partials the resident ones wait for, so the engine refuses the pair in
+    either order (DVLM_ERR_UNSUPPORTED = 3) and keeps its settings."""
+    s = Setup(SMALL_BF16, 0, cuda, 32, 16, 0)
+    eng = s.eng
+    eng.set_option("gateup_stages", 5)
+    with pytest.raises(dv.DvlmError) as e:
+        eng.set_option("down_stages", 5)
+    assert e.value.status == 3
+    assert eng.get_option("down_stages") == 10
+    eng.set_option("gateup_stages", 10)
+    eng.set_option("down_stages", 5)
+    with pytest.raises(dv.DvlmError) as e:
+        eng.set_option("gateup_stages", 5)
+    assert e.value.status == 3
+    assert eng.get_option("gateup_stages") == 10
+    eng.close()
