@@ -536,8 +536,9 @@ def run_sweep(args, local, sink=None):
     D, Hq, Hkv = dims.head_dim, dims.n_q_heads, dims.n_kv_heads
 
     def attn_case(B, L, nb, split_list):
-        """Times the cluster kernel and the split kernel (each S in split_list)
-        on one shape; prints one line per kernel configuration."""
+        """Times the attention kernel's cluster form (the decode path) and its
+        split form (each S in split_list) on one shape; prints one line per
+        configuration."""
         Lmax = (L + B + 7) // 8 * 8
         q, k, v = (t for t, _ in gen.attn_case(1, B, L, Lmax=Lmax, n_batch=nb))
         qd, kd = q.to(dev).contiguous(), k.to(dev).contiguous()
