@@ -23,10 +23,11 @@
 //   split form (kCL = 0, the bandwidth-bound form): fp32 partial rows to
 //   global scratch, a counter per group, the last CTA to arrive merges in
 //   split order; no CTA waits for another;
-//   cluster form (kCL = S = 8 or 16, the decode path): the S CTAs are one
-//   thread-block cluster; fp16 partial rows go by bulk copies straight into
-//   the shared memory of the CTA owning those rows, which merges them in
-//   source order; no scratch, no second kernel.
+//   cluster form (kCL = S = 8 or 16, the decode path and the candidate blocks
+//   of the quadratic forward): the S CTAs are one thread-block cluster; fp16
+//   partial rows go by bulk copies straight into the shared memory of the
+//   CTA owning those rows, which merges them in source order; no scratch, no
+//   second kernel.
 // Paged caches read each 64-key half chunk through the block table.
 #include <cuda_fp16.h>
 
@@ -69,10 +70,13 @@ size_t attn_split_scratch_bytes(int n_groups_total, int S) {
 
 // kCL = 0: S = gridDim.x independent CTAs, partials through global scratch,
 // merged by the last CTA of the group.  kCL = 8 or 16: the S = kCL CTAs of a
-// group form one thread-block cluster; each sends its fp16 partial rows
-// O / l and (m, l) straight into the shared memory of the CTA that owns
-// those rows (128 / kCL rows each), which merges them after one cluster
-// barrier: no global scratch, no counter.
+// group form one thread-block cluster; each CTA with keys bulk-copies its
+// fp16 partial rows O / l and (m, l) straight into the shared memory of the
+// CTA that owns those rows (128 / kCL rows each), counted on that CTA's
+// receive barrier, and the owner merges them: no global scratch, no counter.
+// Candidate blocks of a fused draft+verify forward (a.cand_B > 0, cluster
+// form) are batch entries whose key set is a cache prefix plus one side
+// chunk of the block's own keys (AttnArgs).
 template <int kCL>
 __global__ void __launch_bounds__(kSpThreads, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
