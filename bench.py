@@ -508,6 +508,15 @@ def _device_ms_per_call(fn, reps, dev):
     return e0.elapsed_time(e1) / reps, mode
 
 
+def attn_auto_splits(B: int, L: int, nb: int, Hkv: int, sms: int = 148) -> int:
+    """Split count of the split-form attention on nb caches of L slots with B
+    rows: as many CTAs as fit in one wave on the SMs (one CTA per SM), at most
+    one CTA per 128-key chunk and 32 per group, at least 1."""
+    n_chunks = (L + B + 127) // 128
+    groups = nb * ((B + 15) // 16) * Hkv
+    return max(1, min(n_chunks, 32, sms // groups))
+
+
 def run_sweep(args, local, sink=None):
     """Timings of the single-kernel configurations, one JSON line per case:
     block attention for B in {4, 8, 16, 32} x L in {256, 1024, 4096}, both one
@@ -575,11 +584,7 @@ def run_sweep(args, local, sink=None):
         del qd, kd, vt, out
 
     def auto_splits(B, L, nb):
-        # as many CTAs as fit in one wave on the SMs (one CTA per SM; at most
-        # one CTA per 128-key chunk)
-        n_chunks = (L + B + 127) // 128
-        groups = nb * ((B + 15) // 16) * Hkv
-        return max(1, min(n_chunks, 32, 148 // groups))
+        return attn_auto_splits(B, L, nb, Hkv)
 
     if args.sweep == "compact":
         # the decode shape and the bandwidth case, one line each per kernel

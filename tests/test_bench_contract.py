@@ -237,3 +237,23 @@ def test_full_line_carries_modes_and_compact_sweep(monkeypatch, capsys):
     for key in ("spec_linear", "spec_quadratic", "route"):
         assert d[key]["nfe"] == 71 and d[key]["tokens_per_s"] > 0
     assert d["route"]["route_k"] == bench.ROUTE_K and d["route"]["hidden_vision_slots"] == 1280
+
+
+def test_attention_auto_splits_fill_one_wave():
+    """The sweep's split count for the split-form attention: one wave of CTAs
+    (groups x S <= 148 whenever a split of 1 fits), no CTA without a 128-key
+    chunk, and the largest such S."""
+    import importlib
+    bench = importlib.import_module("bench")
+    for B in (4, 8, 16, 32):
+        for L in (256, 1024, 1344, 4096):
+            for nb in (1, 36):
+                S = bench.attn_auto_splits(B, L, nb, 2)
+                groups = nb * ((B + 15) // 16) * 2
+                n_chunks = (L + B + 127) // 128
+                assert 1 <= S <= min(32, n_chunks) or (S == 1 and n_chunks >= 1)
+                if groups <= 148:
+                    assert groups * S <= 148
+                    assert S == min(32, n_chunks) or groups * (S + 1) > 148
+    assert bench.attn_auto_splits(16, 4096, 36, 2) == 2   # the bandwidth case: 144 CTAs
+    assert bench.attn_auto_splits(16, 1344, 1, 2) == 11   # the decode shape: one CTA per chunk
