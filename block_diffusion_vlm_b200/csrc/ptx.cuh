@@ -97,8 +97,8 @@ __device__ __forceinline__ bool mbar_wait_budget(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------- TMA loads
-// No .multicast::cluster anywhere in this library: every CTA fetches its own
-// tiles from this GPU's memory.
+// No cluster-multicast form of these loads anywhere in this library: every
+// CTA fetches its own tiles from this GPU's memory.
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
